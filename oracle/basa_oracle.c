@@ -1,0 +1,210 @@
+/*
+ * CPU fp64 oracle for shifted local window attention with optional K/V-pooled
+ * global memory.  TEST INFRASTRUCTURE ONLY: the parity tests, the package's
+ * smoke check and the benchmark's CPU-baseline leg call it.  The product path
+ * (the CUDA library) never links, loads or calls this file, and this file uses
+ * nothing from it.
+ *
+ * What it computes (plain definitions, no blocking, fusion or reordering):
+ *
+ *  - Shifted local window attention replaces full visual self-attention: each
+ *    token attends only to the tokens of its own window, and the window
+ *    partition is offset by a per-block shift ("BASA: Backend-Agnostic Sparse
+ *    Attention for Fast High-Resolution Diffusion Transformers", zhichai.net
+ *    topic 178635722, sections "Summary" and "The BASA Method").
+ *    Reading used here (the pages give no formula): on every grid axis a with
+ *    size G, window size w and shift s, token coordinate x belongs to window
+ *        wid(x) = floor( ((x - s) mod G) / w ),
+ *    with a cyclic wrap at the border and no extra mask.  Shift 0 is the plain
+ *    partitioned window attention that the same pages contrast it with.
+ *
+ *  - K/V-pooled global memory: the forum review of the same paper (zhichai.net
+ *    topic 178635722, reply 178634520, the four-part method list) names
+ *    "K/V pooled global memory" as a second component.  Reading used here:
+ *    pooled tokens are the plain means of K and V over non-overlapping
+ *    pt x ph x pw cells aligned to the unshifted grid origin, and they are
+ *    appended to every query's key set under one joint softmax, with no
+ *    count correction.
+ *
+ *  - Full attention (the quadratic baseline in the same pages) is the case of
+ *    one window covering the whole grid.
+ *
+ * Arithmetic: every input value is read as a double; dot products, the
+ * max-subtracted softmax and the weighted sum are all in double precision.
+ *
+ * Layout: all token tensors are [B, T, Hg, Wg, H, d] row-major doubles.
+ * Pooled tensors are [B, T/pt, Hg/ph, Wg/pw, H, d].
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+typedef struct {
+  int64_t B, H, T, Hg, Wg, d;
+  int64_t wt, wh, ww;   /* window size per axis (t, rows, columns) */
+  int64_t st, sh, sw;   /* shift per axis */
+  int64_t pt, ph, pw;   /* pooled cell size; all zero = no global memory */
+  double scale;         /* softmax scale applied to q.k */
+} oracle_params;
+
+static int64_t floor_mod(int64_t a, int64_t n) {
+  int64_t r = a % n;
+  return r < 0 ? r + n : r;
+}
+
+static int64_t tok_index(const oracle_params* p, int64_t b, int64_t t, int64_t y,
+                         int64_t x, int64_t h) {
+  return ((((b * p->T + t) * p->Hg + y) * p->Wg + x) * p->H + h) * p->d;
+}
+
+/* Mean of x over each pooled cell. */
+void oracle_pool(const double* x, double* xp, const oracle_params* p) {
+  const int64_t Pt = p->T / p->pt, Ph = p->Hg / p->ph, Pw = p->Wg / p->pw;
+  const double inv = 1.0 / (double)(p->pt * p->ph * p->pw);
+  for (int64_t b = 0; b < p->B; ++b)
+    for (int64_t ct = 0; ct < Pt; ++ct)
+      for (int64_t cy = 0; cy < Ph; ++cy)
+        for (int64_t cx = 0; cx < Pw; ++cx)
+          for (int64_t h = 0; h < p->H; ++h)
+            for (int64_t c = 0; c < p->d; ++c) {
+              double acc = 0.0;
+              for (int64_t i = 0; i < p->pt; ++i)
+                for (int64_t j = 0; j < p->ph; ++j)
+                  for (int64_t l = 0; l < p->pw; ++l)
+                    acc += x[tok_index(p, b, ct * p->pt + i, cy * p->ph + j,
+                                       cx * p->pw + l, h) + c];
+              int64_t o = (((((b * Pt + ct) * Ph + cy) * Pw + cx) * p->H + h) * p->d) + c;
+              xp[o] = acc * inv;
+            }
+}
+
+/*
+ * Output (and optionally log-sum-exp) of one query token (b, t, y, x, h).
+ * kp/vp may be NULL (no global memory).  Scratch z must hold m + P doubles.
+ */
+static void one_query(const double* q, const double* k, const double* v,
+                      const double* kp, const double* vp, int64_t P,
+                      const oracle_params* p, int64_t b, int64_t t, int64_t y,
+                      int64_t x, int64_t h, double* z, double* out_row,
+                      double* lse_out) {
+  const int64_t d = p->d;
+  const double* qv = q + tok_index(p, b, t, y, x, h);
+  /* window id of the query on each axis */
+  const int64_t it = floor_mod(t - p->st, p->T) / p->wt;
+  const int64_t iy = floor_mod(y - p->sh, p->Hg) / p->wh;
+  const int64_t ix = floor_mod(x - p->sw, p->Wg) / p->ww;
+  const int64_t m = p->wt * p->wh * p->ww;
+
+  /* logits over the window members, enumerated from the window id */
+  int64_t j = 0;
+  for (int64_t lt = 0; lt < p->wt; ++lt)
+    for (int64_t ly = 0; ly < p->wh; ++ly)
+      for (int64_t lx = 0; lx < p->ww; ++lx) {
+        const int64_t tt = floor_mod(it * p->wt + p->st + lt, p->T);
+        const int64_t yy = floor_mod(iy * p->wh + p->sh + ly, p->Hg);
+        const int64_t xx = floor_mod(ix * p->ww + p->sw + lx, p->Wg);
+        const double* kv = k + tok_index(p, b, tt, yy, xx, h);
+        double s = 0.0;
+        for (int64_t c = 0; c < d; ++c) s += qv[c] * kv[c];
+        z[j++] = p->scale * s;
+      }
+  /* logits over the pooled tokens */
+  for (int64_t c2 = 0; c2 < P; ++c2) {
+    const double* kv = kp + ((b * P + c2) * p->H + h) * d;
+    double s = 0.0;
+    for (int64_t c = 0; c < d; ++c) s += qv[c] * kv[c];
+    z[j++] = p->scale * s;
+  }
+  const int64_t nk = m + P;
+  double mx = -INFINITY;
+  for (int64_t i = 0; i < nk; ++i) mx = z[i] > mx ? z[i] : mx;
+  double den = 0.0;
+  for (int64_t i = 0; i < nk; ++i) {
+    z[i] = exp(z[i] - mx);
+    den += z[i];
+  }
+  for (int64_t c = 0; c < d; ++c) out_row[c] = 0.0;
+  j = 0;
+  for (int64_t lt = 0; lt < p->wt; ++lt)
+    for (int64_t ly = 0; ly < p->wh; ++ly)
+      for (int64_t lx = 0; lx < p->ww; ++lx) {
+        const int64_t tt = floor_mod(it * p->wt + p->st + lt, p->T);
+        const int64_t yy = floor_mod(iy * p->wh + p->sh + ly, p->Hg);
+        const int64_t xx = floor_mod(ix * p->ww + p->sw + lx, p->Wg);
+        const double* vv = v + tok_index(p, b, tt, yy, xx, h);
+        const double a = z[j++] / den;
+        for (int64_t c = 0; c < d; ++c) out_row[c] += a * vv[c];
+      }
+  for (int64_t c2 = 0; c2 < P; ++c2) {
+    const double* vv = vp + ((b * P + c2) * p->H + h) * d;
+    const double a = z[j++] / den;
+    for (int64_t c = 0; c < d; ++c) out_row[c] += a * vv[c];
+  }
+  if (lse_out) *lse_out = mx + log(den);
+}
+
+/*
+ * Window attention over all queries, or over a selection.
+ *   kp, vp : pooled K/V ([B, P, H, d] flattened cells) or NULL for none
+ *   out    : [B, T, Hg, Wg, H, d] when sel == NULL, else [nsel, d]
+ *   lse    : [B, H, N] when sel == NULL, else [nsel]; may be NULL
+ *   sel    : nsel triples (b, n, h) with n the flattened token index
+ *            ((t * Hg + y) * Wg + x), or NULL for every query
+ * Returns 0, or -1 on an invalid size.
+ */
+int oracle_window_attn(const double* q, const double* k, const double* v,
+                       const double* kp, const double* vp, double* out,
+                       double* lse, const oracle_params* p, const int64_t* sel,
+                       int64_t nsel, int nthreads) {
+  if (p->T % p->wt || p->Hg % p->wh || p->Wg % p->ww) return -1;
+  int64_t P = 0;
+  if (kp) {
+    if (p->pt <= 0 || p->ph <= 0 || p->pw <= 0) return -1;
+    P = (p->T / p->pt) * (p->Hg / p->ph) * (p->Wg / p->pw);
+  }
+  const int64_t N = p->T * p->Hg * p->Wg;
+  const int64_t m = p->wt * p->wh * p->ww;
+  const int64_t total = sel ? nsel : p->B * N * p->H;
+#ifdef _OPENMP
+  if (nthreads > 0) omp_set_num_threads(nthreads);
+#else
+  (void)nthreads;
+#endif
+#pragma omp parallel
+  {
+    double* z = (double*)malloc(sizeof(double) * (size_t)(m + P));
+#pragma omp for schedule(dynamic, 64)
+    for (int64_t i = 0; i < total; ++i) {
+      int64_t b, n, h;
+      if (sel) {
+        b = sel[3 * i];
+        n = sel[3 * i + 1];
+        h = sel[3 * i + 2];
+      } else {
+        b = i / (N * p->H);
+        n = (i / p->H) % N;
+        h = i % p->H;
+      }
+      const int64_t x = n % p->Wg, y = (n / p->Wg) % p->Hg, t = n / (p->Wg * p->Hg);
+      double* orow = sel ? out + i * p->d : out + tok_index(p, b, t, y, x, h);
+      double* l = NULL;
+      if (lse) l = sel ? lse + i : lse + (b * p->H + h) * N + n;
+      one_query(q, k, v, kp, vp, P, p, b, t, y, x, h, z, orow, l);
+    }
+    free(z);
+  }
+  return 0;
+}
+
+/* Number of OpenMP threads the oracle would use (1 without OpenMP). */
+int oracle_max_threads(void) {
+#ifdef _OPENMP
+  return omp_get_max_threads();
+#else
+  return 1;
+#endif
+}

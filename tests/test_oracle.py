@@ -1,0 +1,345 @@
+"""Pins of the CPU fp64 oracle against facts fixed outside the oracle itself.
+
+Each test is chosen so that a plausible slip in the oracle (a wrong shift sign,
+a dropped scale, a transposed operand, pooled cells on the wrong origin, a bad
+log-sum-exp) fails at least one of them:
+
+* a hand-worked example (tests/golden/hand_1x6.json) with closed-form values;
+* shift 0 equals partitioned window attention written with numpy reshapes;
+* one window covering the grid equals torch's CPU scaled_dot_product_attention;
+* a dense-mask brute force on tiny grids, every shift;
+* rolling the input by the shift commutes with the output, and shifts are
+  periodic in the window size;
+* closed forms (q = 0, constant v, pool factor 1, constant cells);
+* the support of each output row is exactly its window (one-hot values and
+  perturbations), and two blocks with shifts (0, w/2) reach neighbouring windows;
+* large logits stay finite and pick the dominant key.
+"""
+import itertools
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _rng(seed):
+    return np.random.Generator(np.random.PCG64(seed))
+
+
+def _P(shape, window, shift=(0, 0, 0), pool=(0, 0, 0), scale=None):
+    import oracle
+    B, T, Hg, Wg, H, d = shape
+    return oracle.OracleParams(B, T, Hg, Wg, H, d, tuple(window), tuple(shift),
+                               tuple(pool), scale)
+
+
+def _expr(s):
+    s = s.strip()
+    if s == "0":
+        return 0.0
+    if s.startswith("ln "):
+        return math.log(float(s[3:]))
+    return float(eval(s, {"sqrt": math.sqrt}))
+
+
+# --------------------------------------------------------------------------
+# hand-worked example
+# --------------------------------------------------------------------------
+
+def test_hand_worked_example(oracle_mod):
+    g = json.load(open(os.path.join(GOLDEN, "hand_1x6.json")))
+    grid = g["grid"]
+    shape = (grid["B"], grid["T"], grid["Hg"], grid["Wg"], grid["H"], grid["d"])
+    q = np.array(g["q"], dtype=np.float64).reshape(shape)
+    k = np.array([_expr(s) for s in g["k_expr"]]).reshape(shape)
+    v = np.array(g["v"], dtype=np.float64).reshape(shape)
+    prm = _P(shape, g["window"], g["shift"], scale=g["scale"])
+    out, lse = oracle_mod.window_attn(q, k, v, prm, want_lse=True)
+    np.testing.assert_allclose(out.reshape(-1), g["out_no_pool"], rtol=0, atol=1e-13)
+    want_lse = [_expr(s) for s in g["lse_no_pool_expr"]]
+    np.testing.assert_allclose(lse.reshape(-1), want_lse, rtol=0, atol=1e-13)
+
+    prm = _P(shape, g["window"], g["shift"], g["pool"], scale=g["scale"])
+    out = oracle_mod.window_attn(q, k, v, prm).reshape(-1)
+    a = _expr(g["out_pool_expr"]["window_123"])
+    b = _expr(g["out_pool_expr"]["window_450"])
+    np.testing.assert_allclose(out, [b, a, a, a, b, b], rtol=0, atol=1e-13)
+
+
+# --------------------------------------------------------------------------
+# special cases reducing to other routines
+# --------------------------------------------------------------------------
+
+def _partitioned_reference(q, k, v, window, scale):
+    """Unshifted windows via reshape into [windows, m] blocks + dense softmax."""
+    B, T, Hg, Wg, H, d = q.shape
+    wt, wh, ww = window
+
+    def blocks(x):
+        r = x.reshape(B, T // wt, wt, Hg // wh, wh, Wg // ww, ww, H, d)
+        r = r.transpose(0, 1, 3, 5, 7, 2, 4, 6, 8)  # b, it, iy, ix, h, lt, ly, lx, d
+        return r.reshape(B, T // wt, Hg // wh, Wg // ww, H, wt * wh * ww, d)
+
+    qb, kb, vb = blocks(q), blocks(k), blocks(v)
+    z = scale * np.einsum("...ic,...jc->...ij", qb, kb)
+    z = z - z.max(axis=-1, keepdims=True)
+    a = np.exp(z)
+    a = a / a.sum(axis=-1, keepdims=True)
+    ob = np.einsum("...ij,...jc->...ic", a, vb)
+    ob = ob.reshape(B, T // wt, Hg // wh, Wg // ww, H, wt, wh, ww, d)
+    ob = ob.transpose(0, 1, 5, 2, 6, 3, 7, 4, 8)
+    return ob.reshape(B, T, Hg, Wg, H, d)
+
+
+@pytest.mark.parametrize("shape,window", [
+    ((1, 1, 8, 8, 2, 16), (1, 4, 4)),
+    ((2, 4, 6, 8, 1, 8), (2, 3, 4)),
+    ((1, 1, 16, 16, 2, 64), (1, 8, 8)),
+])
+def test_shift_zero_is_partitioned_attention(oracle_mod, shape, window):
+    r = _rng(11)
+    q, k, v = (r.standard_normal(shape) for _ in range(3))
+    sc = 1.0 / math.sqrt(shape[-1])
+    got = oracle_mod.window_attn(q, k, v, _P(shape, window))
+    want = _partitioned_reference(q, k, v, window, sc)
+    np.testing.assert_allclose(got, want, rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("shape", [(1, 1, 8, 8, 2, 16), (2, 3, 4, 5, 3, 8)])
+def test_window_covering_grid_is_full_attention(oracle_mod, shape):
+    r = _rng(12)
+    q, k, v = (r.standard_normal(shape) for _ in range(3))
+    B, T, Hg, Wg, H, d = shape
+    N = T * Hg * Wg
+    got, lse = oracle_mod.full_attn(q, k, v, _P(shape, (T, Hg, Wg)), want_lse=True)
+    # a shifted window that covers the grid is the same set of keys
+    got_s = oracle_mod.window_attn(q, k, v, _P(shape, (T, Hg, Wg), (1, 2, 3)))
+    tq = torch.from_numpy(q).reshape(B, N, H, d).transpose(1, 2)
+    tk = torch.from_numpy(k).reshape(B, N, H, d).transpose(1, 2)
+    tv = torch.from_numpy(v).reshape(B, N, H, d).transpose(1, 2)
+    want = torch.nn.functional.scaled_dot_product_attention(tq, tk, tv)
+    want = want.transpose(1, 2).reshape(shape).numpy()
+    np.testing.assert_allclose(got, want, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(got_s, want, rtol=0, atol=1e-12)
+    z = torch.einsum("bhic,bhjc->bhij", tq, tk) / math.sqrt(d)
+    want_lse = torch.logsumexp(z, dim=-1).numpy()
+    np.testing.assert_allclose(lse, want_lse, rtol=0, atol=1e-12)
+
+
+# --------------------------------------------------------------------------
+# dense-mask brute force on tiny grids, every shift
+# --------------------------------------------------------------------------
+
+TINY = [
+    ((1, 1, 4, 4, 2, 8), (1, 2, 2), (0, 0, 0)),
+    ((1, 1, 8, 8, 1, 16), (1, 4, 4), (1, 2, 2)),
+    ((1, 4, 6, 8, 1, 8), (2, 3, 4), (2, 3, 2)),
+    ((2, 1, 6, 6, 2, 4), (1, 3, 2), (1, 3, 2)),
+]
+
+
+@pytest.mark.parametrize("shape,window,pool", TINY)
+def test_oracle_matches_brute_force_all_shifts(oracle_mod, shape, window, pool):
+    r = _rng(13)
+    q, k, v = (r.standard_normal(shape) for _ in range(3))
+    ranges = [range(-w, w + 1) for w in window]
+    shifts = list(itertools.product(*ranges))
+    if len(shifts) > 40:
+        idx = _rng(5).choice(len(shifts), 40, replace=False)
+        shifts = [shifts[i] for i in idx]
+    for s in shifts:
+        prm = _P(shape, window, s, pool)
+        got, lse = oracle_mod.window_attn(q, k, v, prm, want_lse=True)
+        want, want_lse = oracle_mod.brute_window_attn(q, k, v, window, s, pool,
+                                                      want_lse=True)
+        np.testing.assert_allclose(got, want, rtol=0, atol=1e-12, err_msg=str(s))
+        np.testing.assert_allclose(lse, want_lse, rtol=0, atol=1e-12, err_msg=str(s))
+
+
+def test_brute_force_d64(oracle_mod):
+    shape, window = (1, 1, 8, 8, 1, 64), (1, 4, 4)
+    r = _rng(14)
+    q, k, v = (r.standard_normal(shape) for _ in range(3))
+    for s in [(0, 0, 0), (0, 1, 3), (0, 2, 2)]:
+        got = oracle_mod.window_attn(q, k, v, _P(shape, window, s, (1, 2, 2)))
+        want = oracle_mod.brute_window_attn(q, k, v, window, s, (1, 2, 2))
+        np.testing.assert_allclose(got, want, rtol=0, atol=1e-12)
+
+
+def test_selected_queries_match_full_output(oracle_mod):
+    shape, window, shift = (2, 2, 6, 8, 3, 8), (1, 3, 4), (1, 1, 2)
+    r = _rng(15)
+    q, k, v = (r.standard_normal(shape) for _ in range(3))
+    prm = _P(shape, window, shift, (1, 2, 2))
+    full, lse = oracle_mod.window_attn(q, k, v, prm, want_lse=True)
+    N = 2 * 6 * 8
+    sel = np.array([[b, n, h] for b in range(2) for n in (0, 5, 47, N - 1) for h in (0, 2)])
+    part, plse = oracle_mod.window_attn(q, k, v, prm, want_lse=True, select=sel)
+    B, T, Hg, Wg, H, d = shape
+    flat = full.reshape(B, N, H, d)
+    for i, (b, n, h) in enumerate(sel):
+        np.testing.assert_array_equal(part[i], flat[b, n, h])
+        assert plse[i] == lse[b, h, n]
+
+
+# --------------------------------------------------------------------------
+# roll commutation and periodicity
+# --------------------------------------------------------------------------
+
+@pytest.mark.parametrize("shape,window,shift", [
+    ((1, 1, 8, 8, 2, 8), (1, 4, 4), (0, 2, 2)),
+    ((1, 1, 12, 12, 1, 8), (1, 4, 6), (0, 1, 5)),
+    ((1, 6, 6, 8, 1, 4), (3, 3, 4), (1, 2, 3)),
+])
+def test_roll_commutes_with_shift(oracle_mod, shape, window, shift):
+    r = _rng(16)
+    q, k, v = (r.standard_normal(shape) for _ in range(3))
+    axes = (1, 2, 3)
+    neg = tuple(-s for s in shift)
+    got = oracle_mod.window_attn(q, k, v, _P(shape, window, shift))
+    rq, rk, rv = (np.roll(x, neg, axis=axes) for x in (q, k, v))
+    base = oracle_mod.window_attn(rq, rk, rv, _P(shape, window, (0, 0, 0)))
+    want = np.roll(base, shift, axis=axes)
+    np.testing.assert_allclose(got, want, rtol=0, atol=1e-12)
+    per = tuple(s + w for s, w in zip(shift, window))
+    got2 = oracle_mod.window_attn(q, k, v, _P(shape, window, per))
+    np.testing.assert_allclose(got2, got, rtol=0, atol=0)
+
+
+# --------------------------------------------------------------------------
+# closed forms
+# --------------------------------------------------------------------------
+
+def test_zero_queries_give_window_mean(oracle_mod):
+    shape, window, shift, pool = (1, 1, 8, 8, 2, 4), (1, 4, 4), (0, 1, 3), (1, 2, 4)
+    r = _rng(17)
+    k, v = r.standard_normal(shape), r.standard_normal(shape)
+    q = np.zeros(shape)
+    prm = _P(shape, window, shift, pool)
+    out, lse = oracle_mod.window_attn(q, k, v, prm, want_lse=True)
+    vp = v.reshape(1, 1, 4, 2, 2, 4, 2, 4).mean(axis=(3, 5))  # pooled cells of 2 x 4
+    P = 4 * 2
+    for y in range(8):
+        for x in range(8):
+            wy = ((y - 1) % 8) // 4
+            wx = ((x - 3) % 8) // 4
+            ys = [yy for yy in range(8) if ((yy - 1) % 8) // 4 == wy]
+            xs = [xx for xx in range(8) if ((xx - 3) % 8) // 4 == wx]
+            acc = sum(v[0, 0, yy, xx] for yy in ys for xx in xs) + vp.reshape(P, 2, 4).sum(0)
+            np.testing.assert_allclose(out[0, 0, y, x], acc / (16 + P), rtol=0, atol=1e-13)
+    np.testing.assert_allclose(lse, math.log(16 + P), rtol=0, atol=1e-13)
+
+
+def test_constant_values_give_constant_output(oracle_mod):
+    shape = (1, 2, 6, 6, 2, 8)
+    r = _rng(18)
+    q, k = r.standard_normal(shape) * 3, r.standard_normal(shape) * 3
+    c = r.standard_normal((2, 8))
+    v = np.broadcast_to(c, shape).copy()
+    out = oracle_mod.window_attn(q, k, v, _P(shape, (2, 3, 3), (1, 1, 2), (1, 2, 3)))
+    np.testing.assert_allclose(out, np.broadcast_to(c, shape), rtol=0, atol=1e-13)
+
+
+def test_pool_factor_one_and_constant_cells(oracle_mod):
+    shape = (2, 2, 4, 6, 3, 8)
+    r = _rng(19)
+    x = r.standard_normal(shape)
+    np.testing.assert_array_equal(oracle_mod.pool_kv(x, _P(shape, (1, 2, 2), pool=(1, 1, 1))), x)
+    cells = r.standard_normal((2, 1, 2, 2, 3, 8))
+    xc = np.repeat(np.repeat(np.repeat(cells, 2, axis=1), 2, axis=2), 3, axis=3)
+    np.testing.assert_allclose(oracle_mod.pool_kv(xc, _P(shape, (1, 2, 2), pool=(2, 2, 3))),
+                               cells, rtol=4e-16 * 12, atol=0)
+    # a pooled token equal to a window key behaves like a duplicate of that key
+    shape1 = (1, 1, 1, 4, 1, 1)
+    q = np.ones(shape1)
+    k = np.zeros(shape1)
+    v = np.array([1.0, 2.0, 3.0, 4.0]).reshape(shape1)
+    out = oracle_mod.window_attn(q, k, v, _P(shape1, (1, 1, 2), (0, 0, 0), (1, 1, 4)))
+    # keys: own window (2 tokens) + one pooled token of mean 2.5, all logits 0
+    want = np.array([(1 + 2 + 2.5) / 3, (1 + 2 + 2.5) / 3, (3 + 4 + 2.5) / 3, (3 + 4 + 2.5) / 3])
+    np.testing.assert_allclose(out.reshape(-1), want, rtol=0, atol=1e-14)
+
+
+# --------------------------------------------------------------------------
+# support and receptive field
+# --------------------------------------------------------------------------
+
+def test_support_is_exactly_the_window(oracle_mod):
+    T, Hg, Wg = 1, 6, 6
+    N = T * Hg * Wg
+    shape = (1, T, Hg, Wg, 1, N)
+    window, shift = (1, 3, 3), (0, 1, 2)
+    r = _rng(20)
+    q, k = r.standard_normal(shape), r.standard_normal(shape)
+    v = np.eye(N).reshape(shape)  # value of token j is the one-hot e_j
+    out = oracle_mod.window_attn(q, k, v, _P(shape, window, shift)).reshape(N, N)
+    iy = ((np.arange(Hg) - 1) % Hg) // 3
+    ix = ((np.arange(Wg) - 2) % Wg) // 3
+    wid = (iy[:, None] * 10 + ix[None, :]).reshape(N)
+    for p in range(N):
+        support = set(np.nonzero(out[p] > 0)[0].tolist())
+        assert support == set(np.nonzero(wid == wid[p])[0].tolist())
+        assert abs(out[p].sum() - 1.0) < 1e-13
+
+
+def test_perturbation_reaches_only_window_then_neighbours(oracle_mod):
+    shape = (1, 1, 8, 8, 1, 4)
+    window = (1, 4, 4)
+    r = _rng(21)
+    q, k, v = (r.standard_normal(shape) for _ in range(3))
+    src = (0, 0, 3, 3)  # (b, t, y, x) of the perturbed token
+
+    def run(vv, s):
+        return oracle_mod.window_attn(q, k, vv, _P(shape, window, s))
+
+    def changed(f):
+        v2 = v.copy()
+        v2[src + (0,)] += 1.0
+        a, b = f(v), f(v2)
+        return np.abs(a - b).max(axis=(0, 1, 4, 5)) > 1e-12  # [Hg, Wg]
+
+    one = changed(lambda vv: run(vv, (0, 0, 0)))
+    want = np.zeros((8, 8), dtype=bool)
+    want[0:4, 0:4] = True
+    np.testing.assert_array_equal(one, want)
+    # two blocks: unshifted then shifted by half a window; the output of the
+    # first block is the value input of the second
+    two = changed(lambda vv: run(run(vv, (0, 0, 0)), (0, 2, 2)))
+    # the first block spreads to window [0,4)x[0,4); the second block's windows
+    # (shift 2) that meet it are rows/cols {6,7,0,1} and {2,3,4,5}: all 64 tokens
+    assert two.sum() > one.sum()
+    assert two[5, 5] and two[7, 7] and not one[5, 5]
+
+
+# --------------------------------------------------------------------------
+# stability
+# --------------------------------------------------------------------------
+
+def test_large_logits_pick_dominant_key(oracle_mod):
+    shape = (1, 1, 4, 4, 1, 2)
+    q = np.zeros(shape)
+    k = np.zeros(shape)
+    v = np.arange(16 * 2, dtype=np.float64).reshape(shape)
+    q[..., 0] = 1.0
+    k[0, 0, 1, 1, 0, 0] = 1e4  # dominates its 2x2 window {0,1}x{0,1}
+    out = oracle_mod.window_attn(q, k, v, _P(shape, (1, 2, 2), scale=1.0))
+    assert np.isfinite(out).all()
+    for y in range(2):
+        for x in range(2):
+            np.testing.assert_allclose(out[0, 0, y, x, 0], v[0, 0, 1, 1, 0], rtol=0, atol=1e-12)
+
+
+def test_scaled_logits_match_brute_force(oracle_mod):
+    shape = (1, 1, 8, 8, 2, 16)
+    r = _rng(22)
+    q = r.standard_normal(shape) * 30.0
+    k, v = r.standard_normal(shape), r.standard_normal(shape)
+    got = oracle_mod.window_attn(q, k, v, _P(shape, (1, 4, 4), (0, 2, 2)))
+    want = oracle_mod.brute_window_attn(q, k, v, (1, 4, 4), (0, 2, 2))
+    assert np.isfinite(got).all()
+    np.testing.assert_allclose(got, want, rtol=0, atol=1e-12)
