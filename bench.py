@@ -1,0 +1,394 @@
+"""Benchmark of bf16 shifted local window attention on B200.
+
+Prints one JSON line.  A step is one call of the library's window attention on
+one batch of the workload (for workloads with global memory: pooling + window
+attention); inputs are seeded and synthetic.
+
+Kernel time: every step is bracketed by CUDA events on the launching stream.
+Before each step the L2 is flushed (a 256 MiB write) and a short device sleep
+is queued, so the event pair measures the kernel and not the host-side launch
+preparation; neither the flush nor the sleep is inside the events.  Reported:
+algorithmic TFLOP/s (4*B*H*N*(m+P)*d flops per step), latency, the dominant
+kernel's roofline fraction, and the realised full-attention / window-attention
+speedup against the theoretical N/m (N/(m+P) with global memory).
+
+e2e: the same metric through the public API with host buffers: pinned q, k, v
+copied to the device, the call, and the output copied back, all inside the
+events.
+
+cpu_baseline / --impl reference: the CPU fp64 oracle timed on the host cores on
+a bounded sample of the same workload (all queries of a few heads).
+
+Multi-GPU (torchrun): each rank runs an independent replica of the workload
+(the path has no exchange step); the time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+from basa_synth import WORKLOADS, workload_inputs  # noqa: E402
+
+METRIC = "window-attn latency (ms) & TFLOPS/% bf16 peak; realised/theoretical N/m speedup"
+DEFAULT_WORKLOAD = "flux2048"
+TC_SOURCE = os.path.join(ROOT, "sparse_attention_diffusion_basa_b200", "csrc", "basa_tc.cu")
+POOL_SOURCE = os.path.join(ROOT, "sparse_attention_diffusion_basa_b200", "csrc", "basa_pool.cu")
+
+
+def _peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        p = json.load(open(path))
+        return {"hbm_gbs": float(p["hbm_gbs"]), "bf16_tflops": float(p["bf16_tflops"]),
+                "bf16_tflops_sustained": float(p.get("bf16_tflops_sustained", p["bf16_tflops"])),
+                "source": "measured"}
+    except Exception:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                "source": "fallback"}
+
+
+def _source_hash(path):
+    return hashlib.sha256(open(path, "rb").read()).hexdigest()[:16]
+
+
+def _traffic(kernel_key, workload):
+    """Per-launch DRAM bytes from a committed ncu summary, if the kernel is unchanged."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        t = json.load(open(path))
+        e = t[kernel_key][workload]
+        src = TC_SOURCE if kernel_key == "tc_attn_kernel" else POOL_SOURCE
+        if e["source_sha"] != _source_hash(src):
+            return None
+        return float(e["dram_bytes_per_launch"])
+    except Exception:
+        return None
+
+
+def workload_numbers(w, shift):
+    B, T, Hg, Wg, H, d = w.shape()
+    N, m, P = w.N, w.m, w.P
+    flops = 4.0 * B * H * N * (m + P) * d
+    esize = 2 if w.dtype == "bf16" else 4
+    bytes_ = 4.0 * B * H * N * d * esize  # q, k, v read + out written once
+    return flops, bytes_, N, m, P
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle sampling during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.dev = device_index
+        self.proc = None
+        self.path = os.path.join("/tmp", f"basa_clocks_{os.getpid()}.csv")
+
+    def start(self):
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.dev), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.f.close()
+        rows = []
+        for line in open(self.path):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append(parts)
+            except Exception:
+                pass
+        os.unlink(self.path)
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        smax = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = set()
+        for r in rows:
+            for n, val in zip(names, r[5:9]):
+                if val.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": float(np.median(sm)) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(rows)}
+
+
+def _sleep_cycles(us):
+    # torch.cuda._sleep spins for a number of cycles; ~2 GHz upper bound on the clock
+    torch.cuda._sleep(int(us * 2000))
+
+
+def time_steps(fn, steps, flush, sleep_us=200.0):
+    """Per-step device time (ms) of fn() with an L2 flush and a sleep before each step."""
+    stream = torch.cuda.current_stream()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(steps)]
+    for i in range(steps):
+        flush.fill_(i & 0xFF)
+        if sleep_us > 0:
+            _sleep_cycles(sleep_us)
+        ev[i][0].record(stream)
+        fn()
+        ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    return [a.elapsed_time(b) for a, b in ev]
+
+
+def run_oracle_sample(w, shift, q, k, v, heads, threads=0):
+    """Oracle on all queries of `heads` heads (batch 0); returns (seconds, flops)."""
+    import oracle
+    B, T, Hg, Wg, H, d = w.shape()
+    N = w.N
+    sel = np.array([[0, n, h] for h in heads for n in range(N)], dtype=np.int64)
+    prm = oracle.OracleParams(B, T, Hg, Wg, H, d, w.window, shift, w.pool)
+    qf, kf, vf = oracle.as_f64(q), oracle.as_f64(k), oracle.as_f64(v)
+    kp = vp = None
+    if w.P:
+        kp = oracle.pool_kv(kf, prm)
+        vp = oracle.pool_kv(vf, prm)
+    t0 = time.perf_counter()
+    oracle.window_attn(qf, kf, vf, prm, kp=kp, vp=vp, select=sel, threads=threads)
+    dt = time.perf_counter() - t0
+    return dt, 4.0 * len(sel) * (w.m + w.P) * d
+
+
+def cpu_baseline(w, shift, q, k, v, budget_s=12.0):
+    import oracle
+    oracle.build_oracle()
+    cores = oracle.max_threads()
+    dt1, fl1 = run_oracle_sample(w, shift, q, k, v, [0])
+    nheads = max(1, min(w.H, int(budget_s / max(dt1, 1e-3))))
+    heads = list(range(nheads))
+    dt, fl = run_oracle_sample(w, shift, q, k, v, heads)
+    return {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+            "sample": f"all {w.N} queries of {nheads} of {w.H} heads, batch 0, shift {shift}; "
+                      f"{dt:.2f} s fp64 on {cores} host threads"}
+
+
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        backend = "nccl" if torch.cuda.is_available() and args.impl != "reference" else "gloo"
+        if torch.cuda.is_available():
+            torch.cuda.set_device(local)
+        torch.distributed.init_process_group(backend, timeout=datetime.timedelta(seconds=300))
+    return world, rank, local
+
+
+def max_over_ranks(x, world):
+    if world == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64,
+                     device="cuda" if torch.distributed.get_backend() == "nccl" else "cpu")
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+
+
+def main_reference(args, world, rank):
+    """The CPU oracle as the reference arm (rank 0 only)."""
+    if rank != 0:
+        return 0
+    import oracle
+    oracle.build_oracle()
+    w = WORKLOADS[args.workload]
+    shift = w.shifts[-1]
+    q, k, v = workload_inputs(w, len(w.shifts) - 1)
+    cores = oracle.max_threads()
+    flops_step = 0.0
+    for _ in range(args.warmup):
+        run_oracle_sample(w, shift, q, k, v, [0])
+    times = []
+    for _ in range(args.steps):
+        dt, fl = run_oracle_sample(w, shift, q, k, v, [0])
+        times.append(dt)
+        flops_step = fl
+    total = sum(times)
+    val = flops_step * args.steps / total / 1e12
+    line = {"impl": "reference", "metric": METRIC, "value": val, "unit": "TFLOP/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * total / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": f"{w.name}: oracle sample", "shift": list(shift)},
+            "cpu_baseline": {"value": val, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                             "sample": f"all {w.N} queries of head 0 of {w.H}, batch 0, per step"},
+            "e2e": {"value": val, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="basa", choices=["basa", "reference"])
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--full-steps", type=int, default=5)
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+    world, rank, local = dist_setup(args)
+    if args.impl == "reference":
+        rc = main_reference(args, world, rank)
+        if world > 1:
+            torch.distributed.destroy_process_group()
+        return rc
+
+    import sparse_attention_diffusion_basa_b200 as basa
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    w = WORKLOADS[args.workload]
+    blocks = list(range(len(w.shifts)))
+    # the timed step uses the workload's last shift (the wrapped case where shifts differ)
+    blk = blocks[-1]
+    shift = w.shifts[blk]
+    q, k, v = workload_inputs(w, blk)
+    qh, kh, vh = (x.pin_memory() for x in (q, k, v))
+    dq, dk, dv = (x.to(dev) for x in (q, k, v))
+    out = torch.empty_like(dq)
+    outh = torch.empty_like(qh).pin_memory()
+    ws_bytes = basa.workspace_size(w.shape(), dq.dtype, w.window, shift, w.pool)
+    ws = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    flops, bytes_, N, m, P = workload_numbers(w, shift)
+
+    def step():
+        basa.window_attn(dq, dk, dv, w.window, shift, w.pool, out=out,
+                         workspace=ws if ws_bytes else None)
+
+    def step_full():
+        basa.full_attn(dq, dk, dv, out=out)
+
+    def step_e2e():
+        dq.copy_(qh, non_blocking=True)
+        dk.copy_(kh, non_blocking=True)
+        dv.copy_(vh, non_blocking=True)
+        step()
+        outh.copy_(out, non_blocking=True)
+
+    for _ in range(args.warmup):
+        step()
+        step_e2e()
+    step_full()
+    torch.cuda.synchronize()
+    assert basa.get_status() == 0, "device wait timed out during warm-up"
+
+    clocks = ClockSampler(torch.cuda.current_device())
+    barrier(world)
+    torch.cuda.synchronize()
+    clocks.start()
+    t_steps = time_steps(step, args.steps, flush)
+    torch.cuda.synchronize()
+    barrier(world)
+    clk = clocks.stop()
+    ms = sum(t_steps) / len(t_steps)
+    ms_max = max_over_ranks(ms, world)
+
+    # full attention on the same inputs: the speedup denominator
+    t_full = time_steps(step_full, args.full_steps, flush)
+    ms_full = max_over_ranks(sum(t_full) / len(t_full), world)
+
+    # end to end through the public API with host buffers
+    stream = torch.cuda.current_stream()
+    e2e_ms = []
+    for i in range(args.steps):
+        flush.fill_(i & 0xFF)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        step_e2e()
+        b.record(stream)
+        b.synchronize()
+        e2e_ms.append(a.elapsed_time(b))
+    e2e = max_over_ranks(sum(e2e_ms) / len(e2e_ms), world)
+    assert basa.get_status() == 0, "device wait timed out during timing"
+
+    peaks = _peaks()
+    tflops = world * flops / (ms_max * 1e-3) / 1e12
+    per_gpu_tflops = flops / (ms_max * 1e-3) / 1e12
+    gbs = bytes_ / (ms_max * 1e-3) / 1e9
+    theo = N / (m + P)
+    if m + P >= 2 * 254:   # intensity (m+P)/2 flop per byte above the ridge
+        roof = {"bound": "tensor", "achieved": per_gpu_tflops, "peak": peaks["bf16_tflops"],
+                "unit": "TFLOP/s", "frac": per_gpu_tflops / peaks["bf16_tflops"]}
+    else:
+        roof = {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": gbs / peaks["hbm_gbs"]}
+    roof["peak_source"] = peaks["source"]
+    roof["traffic"] = _traffic("tc_attn_kernel", w.name)
+    roof["kernel"] = "tc_attn_kernel"
+
+    line = {
+        "metric": METRIC, "value": tflops, "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": f"{w.name}: B={w.B} grid {w.T}x{w.Hg}x{w.Wg} H={w.H} d={w.d} "
+                               f"window {'x'.join(map(str, w.window))} shift {shift} "
+                               f"pool {w.pool}",
+                   "N": N, "m": m, "P": P, "global_batch": w.B * world,
+                   "l2": "flushed before every step (256 MiB write, outside the events)",
+                   "parallelism": f"replicas x{world}"},
+        "latency_ms": ms_max,
+        "pct_bf16_peak": 100.0 * per_gpu_tflops / peaks["bf16_tflops"],
+        "speedup": {"full_attn_ms": ms_full, "window_attn_ms": ms_max,
+                    "realised": ms_full / ms_max, "theoretical": theo,
+                    "ratio": (ms_full / ms_max) / theo,
+                    "full_attn_tflops": 4.0 * w.B * w.H * N * N * w.d / (ms_full * 1e-3) / 1e12},
+        "roofline": roof,
+        "e2e": {"value": world * flops / (e2e * 1e-3) / 1e12, "unit": "TFLOP/s",
+                "ms_per_step": e2e,
+                "h2d_bytes_per_step": 3 * dq.numel() * dq.element_size(),
+                "d2h_bytes_per_step": out.numel() * out.element_size()},
+        "gpu_launches": args.steps * (2 if w.P else 1),
+        "clocks": clk,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w, shift, q, k, v)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        barrier(world)
+        torch.distributed.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

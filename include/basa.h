@@ -1,0 +1,189 @@
+/*
+ * basa.h — C ABI of the shifted local window attention library for NVIDIA B200
+ * (sm_100a).
+ *
+ * The operation.  Tokens of a Diffusion Transformer lie on a 2D image or 3D video
+ * latent grid.  Shifted local window attention replaces full visual
+ * self-attention: the grid is cut into fixed windows, the window partition is
+ * moved by a per-block shift, and each token attends only to the tokens of its
+ * own shifted window ("BASA: Backend-Agnostic Sparse Attention for Fast
+ * High-Resolution Diffusion Transformers", zhichai.net topic 178635722,
+ * sections "Summary" and "The BASA Method").  Optionally every query also
+ * attends to a small set of K/V mean-pooled "global memory" tokens (forum
+ * review of the same paper, zhichai.net topic 178635722 reply 178634520, the
+ * four-part method list).  Full attention, the quadratic baseline the same
+ * pages compare against, is the case of one window covering the whole grid.
+ *
+ * Readings taken where the pages give no formula:
+ *   - on each axis of size G with window w and shift s, coordinate x lies in
+ *     window floor(((x - s) mod G) / w): windows wrap cyclically at the border
+ *     and no extra mask is applied; s is reduced mod w;
+ *   - pooled cells are non-overlapping pt x ph x pw boxes aligned to the
+ *     unshifted origin; pooled K/V are plain means; window keys and pooled keys
+ *     share one softmax, with no count correction;
+ *   - softmax scale defaults to 1/sqrt(d).
+ *
+ * Layout.  q, k, v and out are dense row-major [B, T, Hg, Wg, H, d] arrays
+ * (batch, time, grid rows, grid columns, heads, head dim) in device memory,
+ * all of the same dtype.  A 2D grid has T = 1.  Pooled tensors are dense
+ * [B, T/pt, Hg/ph, Wg/pw, H, d] arrays of the same dtype.  The optional lse
+ * output is a dense fp32 [B, H, T*Hg*Wg] array holding the natural-log
+ * log-sum-exp of each query's scaled logits.
+ *
+ * Ownership.  The caller allocates and owns every buffer, including the
+ * workspace.  No entry point allocates device or host memory, keeps a pointer
+ * after it returns, or synchronises the stream (except basa_get_status).
+ *
+ * Ordering.  All device work is enqueued on the given stream, in order.
+ *
+ * Errors.  Arguments are validated synchronously before anything is launched;
+ * on an error nothing is enqueued and a status code is returned.  A launch
+ * failure returns BASA_ERR_CUDA.  Every wait inside the kernels is bounded in
+ * time; a wait that runs out makes the kernel stop early and sets a device
+ * status word that basa_get_status reports as BASA_ERR_TIMEOUT.  The library
+ * never aborts the process and never traps on the device.
+ *
+ * Supported sizes.
+ *   fp32 (BASA_F32): d in {32, 64, 128}; any window that divides the grid.
+ *     Exact fp32 arithmetic on CUDA cores (no reduced-precision tensor math).
+ *   bf16 (BASA_BF16): d in {64, 128}; window width ww <= 128; the window is
+ *     cut into tiles of whole rows of width ww, and every TMA box of a tile
+ *     (a piece of a tile that does not cross a wrapped border) must hold a
+ *     multiple of 8 tokens; at most 32 tiles (about 4096 tokens) per window;
+ *     at most 16 distinct box shapes per call.  Sizes outside these bounds
+ *     return BASA_ERR_UNSUPPORTED.  Tensor cores (tcgen05) with fp32
+ *     accumulation and an fp32 softmax; probabilities are rounded to bf16
+ *     before they multiply V; outputs are rounded to bf16.
+ *   All pointers 16-byte aligned.  B * H * T * Hg * Wg == 0 is a valid no-op.
+ */
+#ifndef BASA_H_
+#define BASA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#include <cuda_runtime_api.h>
+
+#if defined(__GNUC__)
+#define BASA_API __attribute__((visibility("default")))
+#else
+#define BASA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum basa_status {
+  BASA_OK = 0,
+  BASA_ERR_INVALID_ARG = 1, /* null pointer, negative size, bad dtype value */
+  BASA_ERR_SHAPE = 2,       /* window or pool cell does not divide the grid */
+  BASA_ERR_UNSUPPORTED = 3, /* head dim, window or box plan outside the bounds above */
+  BASA_ERR_ALIGN = 4,       /* a pointer is not 16-byte aligned */
+  BASA_ERR_WORKSPACE = 5,   /* workspace missing when global memory is requested */
+  BASA_ERR_CUDA = 6,        /* CUDA runtime or driver error at launch */
+  BASA_ERR_TIMEOUT = 7      /* a bounded wait inside a kernel ran out */
+} basa_status;
+
+typedef enum basa_dtype { BASA_F32 = 0, BASA_BF16 = 1 } basa_dtype;
+
+/* Test-only flag bits for basa_params.flags. */
+#define BASA_FLAG_TEST_WITHHOLD_LOADS 0x1u /* the bf16 kernel's loader issues nothing,
+                                              so its first wait runs out (tests the
+                                              timeout path); output is not written */
+
+typedef struct basa_params {
+  int32_t B, H;        /* batch, heads */
+  int32_t T, Hg, Wg;   /* grid: time (1 for images), rows, columns */
+  int32_t d;           /* head dim */
+  int32_t wt, wh, ww;  /* window size per axis (t, rows, columns) */
+  int32_t st, sh, sw;  /* window-partition shift per axis; any integer, reduced mod window */
+  int32_t pt, ph, pw;  /* pooled cell size per axis; all 0 = no global memory */
+  float scale;         /* softmax scale on q.k; 0 selects 1/sqrt(d) */
+  int32_t dtype;       /* basa_dtype of q, k, v, out and pooled tensors */
+  uint32_t flags;      /* 0, or BASA_FLAG_* test bits */
+  uint32_t wait_timeout_ms; /* bound on each device wait; 0 selects 2000 ms */
+} basa_params;
+
+/* Human-readable name of a status code (static string). */
+BASA_API const char* basa_status_string(basa_status s);
+
+/* Library ABI version (major * 100 + minor). */
+BASA_API int basa_version(void);
+
+/*
+ * Bytes of workspace basa_window_attn needs for params p: room for pooled K and
+ * pooled V (each [B, P, H, d] of p->dtype, 256-byte aligned), or 0 when p asks
+ * for no global memory.  Returns 0 for invalid params.
+ */
+BASA_API size_t basa_workspace_size(const basa_params* p);
+
+/*
+ * K/V mean pooling into global-memory tokens (forum review of the BASA paper,
+ * zhichai.net topic 178635722 reply 178634520, four-part method list: K/V
+ * pooled global memory).  kp[b, c, h, :] = mean of k over the tokens of cell c
+ * (cells of pt x ph x pw aligned to the grid origin); the same for v into vp.
+ * Accumulates in fp32, stores in p->dtype (round to nearest even for bf16).
+ * k, v: [B, T, Hg, Wg, H, d]; kp, vp: [B, T/pt, Hg/ph, Wg/pw, H, d].
+ */
+BASA_API basa_status basa_pool_kv(const void* k, const void* v, void* kp, void* vp,
+                         const basa_params* p, cudaStream_t stream);
+
+/*
+ * Shifted local window attention ("BASA: Backend-Agnostic Sparse Attention for
+ * Fast High-Resolution Diffusion Transformers", zhichai.net topic 178635722,
+ * "The BASA Method").  out[b, x, h, :] = softmax over the keys of x's shifted
+ * window (plus, when p asks for global memory, the pooled keys) of
+ * scale * q[b, x, h, :] . k[b, y, h, :], applied to v.
+ * If p asks for global memory, pooled K/V are first computed into
+ * `workspace` (basa_workspace_size(p) bytes) on the same stream; otherwise
+ * workspace may be NULL.  lse may be NULL.
+ */
+BASA_API basa_status basa_window_attn(const void* q, const void* k, const void* v, void* out,
+                             float* lse, void* workspace, const basa_params* p,
+                             cudaStream_t stream);
+
+/*
+ * Shifted local window attention with caller-supplied pooled global memory
+ * kp, vp ([B, T/pt, Hg/ph, Wg/pw, H, d], e.g. from basa_pool_kv).  The same
+ * operation as basa_window_attn without the pooling step; p must ask for global
+ * memory (pt, ph, pw >= 1).
+ */
+BASA_API basa_status basa_window_attn_gm(const void* q, const void* k, const void* v,
+                                const void* kp, const void* vp, void* out, float* lse,
+                                const basa_params* p, cudaStream_t stream);
+
+/*
+ * Full softmax attention over all T*Hg*Wg tokens: the same kernels with one
+ * window covering the whole grid (the quadratic baseline of the BASA pages).
+ * Window, shift and pool fields of p are ignored.
+ */
+BASA_API basa_status basa_full_attn(const void* q, const void* k, const void* v, void* out,
+                           float* lse, const basa_params* p, cudaStream_t stream);
+
+/*
+ * Test and diagnostics only: synchronises `stream`, then reports and clears the
+ * device status word of the current device.  BASA_ERR_TIMEOUT if a kernel
+ * wait ran out since the last call, BASA_ERR_CUDA on a pending CUDA error,
+ * else BASA_OK.
+ */
+BASA_API basa_status basa_get_status(cudaStream_t stream);
+
+/*
+ * Host-only description of the bf16 kernel's window tiling (no GPU needed).
+ * *n_windows = windows per (b, h) and *n_tiles = 128-row tiles per window.
+ * If rows != NULL it receives [n_windows][n_tiles][128] int32 entries: the
+ * flattened grid index (t * Hg + y) * Wg + x of the token that row r of the
+ * tile holds in shared memory, or -1 for a padding row.  Only the grid, window
+ * and shift fields and d/dtype of p are read; shapes outside the bf16 bounds
+ * return BASA_ERR_UNSUPPORTED.  rows_capacity is the number of int32 entries
+ * rows can hold.
+ */
+BASA_API basa_status basa_window_tiles(const basa_params* p, int32_t* n_windows, int32_t* n_tiles,
+                              int32_t* rows, int64_t rows_capacity);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BASA_H_ */

@@ -1,0 +1,168 @@
+"""Shifted local window attention for Diffusion Transformer tokens on B200.
+
+A thin Python binding over the C ABI of ``include/basa.h``: it checks tensor
+placement, allocates outputs with torch (device memory only) and passes raw
+pointers and the current CUDA stream to the library.  Every step of the
+computation runs in the library's CUDA kernels; there is no CPU or PyTorch
+fallback, and calls fail loudly when the library is missing.
+
+Tensors use the layout ``[B, T, Hg, Wg, H, d]``; ``window``, ``shift`` and
+``pool`` are (t, rows, columns) triples.
+"""
+from __future__ import annotations
+
+import ctypes
+from typing import Optional, Sequence, Tuple
+
+import torch
+
+from . import _lib
+from ._lib import BasaError, BasaParams, BASA_F32, BASA_BF16
+
+__all__ = ["window_attn", "window_attn_gm", "full_attn", "pool_kv", "workspace_size",
+           "get_status", "window_tiles", "make_params", "BasaError", "library_path"]
+
+library_path = _lib.LIB_PATH
+
+_DT = {torch.float32: BASA_F32, torch.bfloat16: BASA_BF16}
+
+
+def _triple(x, name) -> Tuple[int, int, int]:
+    t = tuple(int(v) for v in x)
+    if len(t) != 3:
+        raise ValueError(f"{name} must have 3 entries (t, rows, columns), got {x!r}")
+    return t
+
+
+def make_params(shape: Sequence[int], dtype, window=(1, 1, 1), shift=(0, 0, 0),
+                pool=(0, 0, 0), scale: Optional[float] = None, flags: int = 0,
+                wait_timeout_ms: int = 0) -> BasaParams:
+    B, T, Hg, Wg, H, d = (int(s) for s in shape)
+    if isinstance(dtype, torch.dtype):
+        dtype = _DT[dtype]
+    w, s, p = _triple(window, "window"), _triple(shift, "shift"), _triple(pool, "pool")
+    return BasaParams(B, H, T, Hg, Wg, d, *w, *s, *p, float(scale or 0.0), int(dtype),
+                      int(flags), int(wait_timeout_ms))
+
+
+def _check_inputs(*ts):
+    ref = ts[0]
+    for t in ts:
+        if not isinstance(t, torch.Tensor):
+            raise TypeError("expected torch tensors")
+        if not t.is_cuda:
+            raise ValueError("tensors must be on a CUDA device")
+        if t.dtype not in _DT:
+            raise TypeError(f"unsupported dtype {t.dtype}")
+        if t.dtype != ref.dtype or t.device != ref.device:
+            raise ValueError("q, k, v must share dtype and device")
+        if not t.is_contiguous():
+            raise ValueError("tensors must be contiguous [B, T, Hg, Wg, H, d]")
+        if t.dim() != 6:
+            raise ValueError("tensors must have 6 dims [B, T, Hg, Wg, H, d]")
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(t: torch.Tensor, stream=None):
+    s = stream if stream is not None else torch.cuda.current_stream(t.device)
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def workspace_size(shape, dtype, window, shift=(0, 0, 0), pool=(0, 0, 0)) -> int:
+    return int(_lib.load().basa_workspace_size(
+        ctypes.byref(make_params(shape, dtype, window, shift, pool))))
+
+
+def pool_kv(k: torch.Tensor, v: torch.Tensor, pool, stream=None):
+    """Mean-pool K and V over pt x ph x pw cells -> (kp, vp) [B, T/pt, Hg/ph, Wg/pw, H, d]."""
+    _check_inputs(k, v)
+    B, T, Hg, Wg, H, d = k.shape
+    pt, ph, pw = _triple(pool, "pool")
+    if min(pt, ph, pw) <= 0 or T % pt or Hg % ph or Wg % pw:
+        raise ValueError(f"pool {pool} must be positive and divide the grid {(T, Hg, Wg)}")
+    kp = torch.empty((B, T // pt, Hg // ph, Wg // pw, H, d), dtype=k.dtype, device=k.device)
+    vp = torch.empty_like(kp)
+    prm = make_params(k.shape, k.dtype, (1, 1, 1), (0, 0, 0), (pt, ph, pw))
+    lib = _lib.load()
+    with torch.cuda.device(k.device):
+        _lib.check(lib.basa_pool_kv(_ptr(k), _ptr(v), _ptr(kp), _ptr(vp), ctypes.byref(prm),
+                                    _stream(k, stream)), "basa_pool_kv")
+    return kp, vp
+
+
+def window_attn(q, k, v, window, shift=(0, 0, 0), pool=(0, 0, 0), scale=None,
+                return_lse=False, out=None, workspace=None, flags=0, wait_timeout_ms=0,
+                stream=None):
+    """Shifted local window attention (plus pooled global memory when pool != 0)."""
+    _check_inputs(q, k, v)
+    if q.shape != k.shape or q.shape != v.shape:
+        raise ValueError("q, k, v must have the same shape")
+    prm = make_params(q.shape, q.dtype, window, shift, pool, scale, flags, wait_timeout_ms)
+    lib = _lib.load()
+    out = torch.empty_like(q) if out is None else out
+    B, T, Hg, Wg, H, d = q.shape
+    lse = torch.empty((B, H, T * Hg * Wg), dtype=torch.float32, device=q.device) if return_lse else None
+    need = int(lib.basa_workspace_size(ctypes.byref(prm)))
+    if need and workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    with torch.cuda.device(q.device):
+        _lib.check(lib.basa_window_attn(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse),
+                                        _ptr(workspace) if need else None, ctypes.byref(prm),
+                                        _stream(q, stream)), "basa_window_attn")
+    return (out, lse) if return_lse else out
+
+
+def window_attn_gm(q, k, v, kp, vp, window, shift=(0, 0, 0), pool=(1, 1, 1), scale=None,
+                   return_lse=False, out=None, stream=None):
+    """Window attention with caller-supplied pooled global memory kp, vp."""
+    _check_inputs(q, k, v, kp, vp)
+    prm = make_params(q.shape, q.dtype, window, shift, pool, scale)
+    lib = _lib.load()
+    out = torch.empty_like(q) if out is None else out
+    B, T, Hg, Wg, H, d = q.shape
+    lse = torch.empty((B, H, T * Hg * Wg), dtype=torch.float32, device=q.device) if return_lse else None
+    with torch.cuda.device(q.device):
+        _lib.check(lib.basa_window_attn_gm(_ptr(q), _ptr(k), _ptr(v), _ptr(kp), _ptr(vp),
+                                           _ptr(out), _ptr(lse), ctypes.byref(prm),
+                                           _stream(q, stream)), "basa_window_attn_gm")
+    return (out, lse) if return_lse else out
+
+
+def full_attn(q, k, v, scale=None, return_lse=False, out=None, stream=None):
+    """Full softmax attention over all grid tokens (one window covering the grid)."""
+    _check_inputs(q, k, v)
+    prm = make_params(q.shape, q.dtype, (1, 1, 1), (0, 0, 0), (0, 0, 0), scale)
+    lib = _lib.load()
+    out = torch.empty_like(q) if out is None else out
+    B, T, Hg, Wg, H, d = q.shape
+    lse = torch.empty((B, H, T * Hg * Wg), dtype=torch.float32, device=q.device) if return_lse else None
+    with torch.cuda.device(q.device):
+        _lib.check(lib.basa_full_attn(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse),
+                                      ctypes.byref(prm), _stream(q, stream)), "basa_full_attn")
+    return (out, lse) if return_lse else out
+
+
+def get_status(stream=None) -> int:
+    """Synchronise and return (and clear) the device status code (test use)."""
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return int(_lib.load().basa_get_status(ctypes.c_void_p(s.cuda_stream)))
+
+
+def window_tiles(grid, window, shift=(0, 0, 0), d=128):
+    """Host-only tile plan of the bf16 kernel: int32 array [windows, tiles, 128] of
+    flattened token indices per shared-memory row (-1 = padding)."""
+    import numpy as np
+    T, Hg, Wg = grid
+    prm = make_params((1, T, Hg, Wg, 1, d), BASA_BF16, window, shift)
+    lib = _lib.load()
+    nw, nt = ctypes.c_int32(), ctypes.c_int32()
+    _lib.check(lib.basa_window_tiles(ctypes.byref(prm), ctypes.byref(nw), ctypes.byref(nt),
+                                     None, 0), "basa_window_tiles")
+    rows = np.empty((nw.value, nt.value, 128), dtype=np.int32)
+    _lib.check(lib.basa_window_tiles(ctypes.byref(prm), None, None,
+                                     rows.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)),
+                                     rows.size), "basa_window_tiles")
+    return rows

@@ -1,0 +1,104 @@
+// Internal declarations shared by the host API and the kernels of the library.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "basa.h"
+
+namespace basa {
+
+// ---------------------------------------------------------------------------
+// Normalised call description (after validation).
+// ---------------------------------------------------------------------------
+struct Dims {
+  int B, H, T, Hg, Wg, d;
+  int wt, wh, ww;     // window
+  int st, sh, sw;     // shift reduced to [0, w)
+  int pt, ph, pw;     // pool cell; 0 = none
+  int nwt, nwh, nww;  // windows per axis
+  long long N;        // tokens per (b, h)
+  long long P;        // pooled tokens per (b, h); 0 = none
+  float scale;
+  int dtype;
+};
+
+// Validates p and fills d.  `full` = one window covering the grid, no shift,
+// no pool (full attention).
+basa_status normalise(const basa_params* p, bool full, Dims* d);
+
+// ---------------------------------------------------------------------------
+// Tile plan of the bf16 tensor-core kernel (shifted-window index math).
+//
+// A window of wt x wh x ww tokens is cut into local boxes ("tiles") of whole
+// window rows: rows of width ww, grouped into chunks of at most 128/ww rows
+// along the window's row axis, and chunks of one row count stacked over t.
+// Each tile holds at most 128 tokens.  When a window wraps around the grid
+// border on an axis (only the last window on an axis with a non-zero shift
+// does), a tile is split along that axis into the part before the border and
+// the part after it; each part is one TMA box.  The wrap pattern of a window
+// is its "class": bit 0 = wraps in t, bit 1 = in rows, bit 2 = in columns.
+// ---------------------------------------------------------------------------
+constexpr int kMaxShapes = 16;  // distinct box shapes per call
+constexpr int kMaxTiles = 32;   // tiles per window
+constexpr int kMaxBoxes = 8;    // boxes per tile (2 per wrapped axis)
+constexpr int kClasses = 8;
+
+// One TMA box of a tile: local start of the box inside the window, its shape id
+// and its first shared-memory row / 8.  Packed in 32 bits:
+// [0,8) lt  [8,16) lh  [16,24) lw  [24,28) shape  [28,32) row8.
+__host__ __device__ inline uint32_t box_pack(int lt, int lh, int lw, int shape, int row8) {
+  return (uint32_t)lt | ((uint32_t)lh << 8) | ((uint32_t)lw << 16) | ((uint32_t)shape << 24) |
+         ((uint32_t)row8 << 28);
+}
+__host__ __device__ inline int box_lt(uint32_t e) { return (int)(e & 0xff); }
+__host__ __device__ inline int box_lh(uint32_t e) { return (int)((e >> 8) & 0xff); }
+__host__ __device__ inline int box_lw(uint32_t e) { return (int)((e >> 16) & 0xff); }
+__host__ __device__ inline int box_shape(uint32_t e) { return (int)((e >> 24) & 0xf); }
+__host__ __device__ inline int box_row8(uint32_t e) { return (int)(e >> 28); }
+
+struct TilePlan {
+  int n_tiles;
+  int n_shapes;
+  uint8_t shape_bt[kMaxShapes], shape_bh[kMaxShapes], shape_bw[kMaxShapes];
+  uint8_t tile_rows[kMaxTiles];                 // valid rows of each tile (same in every class)
+  uint8_t nbox[kClasses][kMaxTiles];
+  uint32_t box[kClasses][kMaxTiles][kMaxBoxes];
+};
+
+// Builds the plan for window (wt, wh, ww) with shifts already reduced to [0, w).
+// Returns BASA_ERR_UNSUPPORTED when the bounds of the bf16 kernel are exceeded.
+basa_status build_tile_plan(const Dims& d, TilePlan* plan);
+
+// Window class (wrap bits) of window (jt, jh, jw).
+__host__ __device__ inline int window_class(int jt, int jh, int jw, int nwt, int nwh, int nww,
+                                            int st, int sh, int sw) {
+  return ((st != 0 && jt == nwt - 1) ? 1 : 0) | ((sh != 0 && jh == nwh - 1) ? 2 : 0) |
+         ((sw != 0 && jw == nww - 1) ? 4 : 0);
+}
+
+// ---------------------------------------------------------------------------
+// Launchers (defined next to their kernels).
+// ---------------------------------------------------------------------------
+basa_status launch_pool(const Dims& d, const void* k, const void* v, void* kp, void* vp,
+                        cudaStream_t stream);
+
+// fp32 CUDA-core window attention (window mode; full attention = one window).
+basa_status launch_simt(const Dims& d, const void* q, const void* k, const void* v,
+                        const void* kp, const void* vp, void* out, float* lse,
+                        cudaStream_t stream);
+
+// bf16 tcgen05 window / full attention.  flat = full attention over the grid.
+basa_status launch_tc(const Dims& d, bool flat, const void* q, const void* k, const void* v,
+                      const void* kp, const void* vp, void* out, float* lse, uint32_t flags,
+                      uint32_t timeout_ms, cudaStream_t stream);
+
+// Device status word helpers (basa_tc.cu).
+basa_status read_and_clear_status(cudaStream_t stream);
+
+// Encodes a tiled TMA map through the driver entry point.
+basa_status encode_map(CUtensorMap* map, const void* base, int rank, const uint64_t* dims,
+                       const uint64_t* strides_bytes, const uint32_t* box);
+
+}  // namespace basa

@@ -1,0 +1,869 @@
+// bf16 shifted local window attention on the 5th-generation tensor cores
+// (tcgen05 + TMEM) of sm_100a.
+//
+// The operation ("BASA: Backend-Agnostic Sparse Attention for Fast
+// High-Resolution Diffusion Transformers", zhichai.net topic 178635722, "The
+// BASA Method"; forum review of the same paper, reply 178634520, four-part
+// method list): every query attends to the keys of its own cyclically shifted
+// window, plus the K/V-pooled global-memory tokens when they are given, under
+// one softmax.  Full attention is "flat" mode: 128-token tiles of the whole
+// grid, each query tile against every key tile.
+//
+// Work unit: (b, h, window, pair of 128-query tiles).  Persistent CTAs (one
+// per SM) walk the units.  Inside a CTA the warps specialise:
+//   warp 0        TMA loader: Q tiles, then K and V tiles of the unit through a
+//                 3-slot ring (boxes from the shifted-window tile plan; a tile
+//                 that crosses a wrapped border is fetched as up to 8 boxes,
+//                 so no rolled copy of the grid is ever made);
+//   warp 1        owns TMEM (512 columns) and issues the MMAs from one thread:
+//                 S_i = Q_i K_j^T into TMEM, then O_i += P_i V_j into TMEM;
+//   warps 4..7    softmax + epilogue for query tile 0 of the unit,
+//   warps 8..11   the same for query tile 1.
+// Each softmax thread owns one query row: it reads its 128 logits from TMEM,
+// keeps the running max and sum in fp32 (base-2 exponentials with the scale
+// folded in), writes the bf16 probabilities P to shared memory in the
+// 128-byte-swizzled K-major layout the MMA reads, and rescales its O row in
+// TMEM when the max grows.  The epilogue divides by the sum, rounds to bf16,
+// stages the tile in shared memory and stores it with TMA boxes that mirror
+// the load boxes.
+//
+// Every mbarrier wait is bounded (wall-clock limit from the call); on expiry the
+// kernel raises the device status word, lets every role leave its loop, waits
+// (bounded) for its own copies and MMAs in flight, frees TMEM and returns.
+#include <cuda_bf16.h>
+#include <math.h>
+#include <string.h>
+
+#include <new>
+
+#include "basa_internal.h"
+
+namespace basa {
+
+__device__ unsigned int g_basa_status;  // bit 0: a device wait timed out
+
+namespace {
+
+constexpr int kThreads = 384;
+constexpr int kHalf = 128 * 128;  // bytes of one 64-wide head-dim half of a 128-row tile
+
+struct __align__(64) TcParams {
+  CUtensorMap qm[kMaxShapes];  // window boxes, rank 5: [d, H, Wg, Hg, B*T]
+  CUtensorMap km[kMaxShapes];
+  CUtensorMap vm[kMaxShapes];
+  CUtensorMap om[kMaxShapes];
+  CUtensorMap qf, kf, vf, of;  // flat 128-row tiles, rank 4: [d, H, N, B]
+  CUtensorMap kpf, vpf;        // pooled 128-row tiles, rank 4: [d, H, P, B]
+  CUtensorMap fill;            // 8-row box over k's flat view, read out of bounds = zeros
+  uint32_t box[kClasses][kMaxTiles][kMaxBoxes];
+  uint8_t nbox[kClasses][kMaxTiles];
+  uint8_t tile_rows[kMaxTiles];
+  uint8_t shape_bt[kMaxShapes], shape_bh[kMaxShapes], shape_bw[kMaxShapes];
+  float* lse;
+  long long n_units;
+  long long N;
+  unsigned long long timeout_ns;
+  int B, H, T, Hg, Wg;
+  int wt, wh, ww, st, sh, sw, nwt, nwh, nww;
+  int n_windows;
+  int n_qt;   // query tiles per window (flat: per (b, h))
+  int n_pairs;
+  int n_wkt;  // key tiles from the window (flat: from the grid)
+  int n_pkt;  // pooled key tiles
+  int P;
+  int flat;
+  uint32_t flags;
+  float scale_log2;
+};
+
+// ---------------------------------------------------------------------------
+// PTX wrappers
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ uint64_t globaltimer() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+__device__ __forceinline__ void fence_barrier_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+__device__ __forceinline__ void fence_proxy_async() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+__device__ __forceinline__ void tma_load_5d(uint32_t dst, const CUtensorMap* map, uint32_t bar,
+                                            int c0, int c1, int c2, int c3, int c4) {
+  asm volatile(
+      "cp.async.bulk.tensor.5d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(c4)
+      : "memory");
+}
+__device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap* map, uint32_t bar,
+                                            int c0, int c1, int c2, int c3) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5, %6}], [%2];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+      : "memory");
+}
+__device__ __forceinline__ void tma_store_5d(const CUtensorMap* map, uint32_t src, int c0, int c1,
+                                             int c2, int c3, int c4) {
+  asm volatile(
+      "cp.async.bulk.tensor.5d.global.shared::cta.tile.bulk_group"
+      " [%0, {%2, %3, %4, %5, %6}], [%1];" ::"l"(reinterpret_cast<uint64_t>(map)),
+      "r"(src), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(c4)
+      : "memory");
+}
+__device__ __forceinline__ void tma_store_4d(const CUtensorMap* map, uint32_t src, int c0, int c1,
+                                             int c2, int c3) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.global.shared::cta.tile.bulk_group"
+      " [%0, {%2, %3, %4, %5}], [%1];" ::"l"(reinterpret_cast<uint64_t>(map)),
+      "r"(src), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+      : "memory");
+}
+__device__ __forceinline__ void bulk_commit() {
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+__device__ __forceinline__ void bulk_wait_read0() {
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+__device__ __forceinline__ void bulk_wait_all0() {
+  asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_alloc(uint32_t slot_smem, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(slot_smem),
+               "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+               : "memory");
+}
+
+// Shared-memory matrix descriptor, 128-byte swizzle (sm_100 layout: start
+// address >> 4 in bits 0-13, leading byte offset >> 4 in 16-29, stride byte
+// offset >> 4 in 32-45, descriptor version 1 in 46-47, swizzle mode 2 in 61-63).
+__device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
+         ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
+}
+// Instruction descriptor of kind::f16: bf16 A and B, fp32 accumulator, A K-major,
+// B K-major or MN-major, M = 128, N = n.
+__host__ __device__ constexpr uint32_t idesc_bf16(int n, bool b_mn) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((b_mn ? 1u : 0u) << 16) |
+         ((uint32_t)(n >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
+}
+__device__ __forceinline__ void mma_bf16(uint32_t tmem_d, uint64_t a, uint64_t b, uint32_t idesc,
+                                         uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
+      "l"(a), "l"(b), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+__device__ __forceinline__ void mma_commit(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                   bar)
+               : "memory");
+}
+
+#define TMEM_REGS32(r)                                                                         \
+  "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),         \
+      "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), \
+      "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),           \
+      "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),           \
+      "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+#define TMEM_INREGS32(r)                                                                          \
+  "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),         \
+      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),          \
+      "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]),        \
+      "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]),        \
+      "r"(r[29]), "r"(r[30]), "r"(r[31])
+#define TMEM_RWREGS32(r)                                                                         \
+  "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]),           \
+      "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]),   \
+      "+r"(r[14]), "+r"(r[15]), "+r"(r[16]), "+r"(r[17]), "+r"(r[18]), "+r"(r[19]),             \
+      "+r"(r[20]), "+r"(r[21]), "+r"(r[22]), "+r"(r[23]), "+r"(r[24]), "+r"(r[25]),             \
+      "+r"(r[26]), "+r"(r[27]), "+r"(r[28]), "+r"(r[29]), "+r"(r[30]), "+r"(r[31])
+
+// 32 consecutive fp32 columns of this thread's TMEM lane; the values are valid
+// only after tmem_wait_ld, which takes them as operands so that no use can be
+// scheduled before it.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+      "%11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, "
+      "%28, %29, %30, %31}, [%32];"
+      : TMEM_REGS32(r)
+      : "r"(taddr)
+      : "memory");
+}
+__device__ __forceinline__ void tmem_wait_ld(uint32_t (&r)[32]) {
+  asm volatile("tcgen05.wait::ld.sync.aligned;" : TMEM_RWREGS32(r)::"memory");
+}
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+      "%11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, "
+      "%28, %29, %30, %31, %32};" ::"r"(taddr),
+      TMEM_INREGS32(r)
+      : "memory");
+}
+__device__ __forceinline__ void tmem_wait_st() {
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
+                                             uint32_t d) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c),
+               "r"(d)
+               : "memory");
+}
+// Byte offset of 16-byte chunk `chunk` (0..7) of row `row` inside a 128-byte
+// swizzled, 1024-byte-aligned block of rows.
+__device__ __forceinline__ uint32_t swz(int row, int chunk) {
+  return (uint32_t)(row * 128 + ((chunk ^ (row & 7)) << 4));
+}
+
+// ---------------------------------------------------------------------------
+// Bounded waits.  `abort_flag` lives in shared memory; any role that gives up
+// raises it so that the others leave their loops promptly.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity,
+                                             volatile uint32_t* abort_flag, uint64_t limit_ns,
+                                             bool honour_abort = true) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer();
+  while (true) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (honour_abort && *abort_flag) return false;
+    if (globaltimer() - t0 > limit_ns) {
+      *abort_flag = 1u;
+      atomicOr(&g_basa_status, 1u);
+      return false;
+    }
+  }
+}
+// Warp-uniform variant: every lane waits, and the warp proceeds only if all did.
+__device__ __forceinline__ bool wait_warp(uint32_t bar, uint32_t parity,
+                                          volatile uint32_t* abort_flag, uint64_t limit_ns) {
+  const bool ok = wait_bounded(bar, parity, abort_flag, limit_ns);
+  return __all_sync(0xffffffffu, ok);
+}
+
+// ---------------------------------------------------------------------------
+// Work-unit decoding
+// ---------------------------------------------------------------------------
+struct Unit {
+  int b, h, pair, cls, ot, oh, ow, nq;
+};
+
+__device__ __forceinline__ Unit decode_unit(const TcParams& p, long long u) {
+  Unit U;
+  U.pair = (int)(u % p.n_pairs);
+  long long r = u / p.n_pairs;
+  if (p.flat) {
+    U.cls = 0;
+    U.ot = U.oh = U.ow = 0;
+  } else {
+    const int win = (int)(r % p.n_windows);
+    r /= p.n_windows;
+    const int jw = win % p.nww, jh = (win / p.nww) % p.nwh, jt = win / (p.nww * p.nwh);
+    U.cls = window_class(jt, jh, jw, p.nwt, p.nwh, p.nww, p.st, p.sh, p.sw);
+    U.ot = jt * p.wt + p.st;
+    U.oh = jh * p.wh + p.sh;
+    U.ow = jw * p.ww + p.sw;
+  }
+  U.h = (int)(r % p.H);
+  U.b = (int)(r / p.H);
+  const int left = p.n_qt - 2 * U.pair;
+  U.nq = left < 2 ? left : 2;
+  return U;
+}
+
+// Valid rows of key tile j (rows past them are zero-filled and masked).
+__device__ __forceinline__ int key_valid(const TcParams& p, int j) {
+  if (p.flat) {
+    const long long left = p.N - 128LL * j;
+    return left < 128 ? (int)left : 128;
+  }
+  if (j < p.n_wkt) return p.tile_rows[j];
+  const int left = p.P - 128 * (j - p.n_wkt);
+  return left < 128 ? left : 128;
+}
+__device__ __forceinline__ int query_valid(const TcParams& p, int qt) {
+  if (p.flat) {
+    const long long left = p.N - 128LL * qt;
+    return left < 128 ? (int)left : 128;
+  }
+  return p.tile_rows[qt];
+}
+
+// kind: 0 = q, 1 = k, 2 = v.  Loads one 128-row tile (all head-dim halves) into
+// shared memory at dst and signals bar with the transaction bytes.
+template <int D>
+__device__ __forceinline__ void load_tile(const TcParams& p, int kind, const Unit& U, int tile,
+                                          uint32_t dst, uint32_t bar) {
+  constexpr int NH = D / 64;
+  if (p.flat) {
+    const CUtensorMap* m = kind == 0 ? &p.qf : kind == 1 ? &p.kf : &p.vf;
+#pragma unroll
+    for (int hf = 0; hf < NH; ++hf) tma_load_4d(dst + hf * kHalf, m, bar, hf * 64, U.h, tile * 128, U.b);
+    return;
+  }
+  if (kind != 0 && tile >= p.n_wkt) {  // pooled global-memory keys
+    const CUtensorMap* m = kind == 1 ? &p.kpf : &p.vpf;
+#pragma unroll
+    for (int hf = 0; hf < NH; ++hf)
+      tma_load_4d(dst + hf * kHalf, m, bar, hf * 64, U.h, (tile - p.n_wkt) * 128, U.b);
+    return;
+  }
+  const int nb = p.nbox[U.cls][tile];
+  for (int bi = 0; bi < nb; ++bi) {
+    const uint32_t e = p.box[U.cls][tile][bi];
+    const int sid = box_shape(e);
+    const int gt = (U.ot + box_lt(e)) % p.T;
+    const int gh = (U.oh + box_lh(e)) % p.Hg;
+    const int gw = (U.ow + box_lw(e)) % p.Wg;
+    const CUtensorMap* m = kind == 0 ? &p.qm[sid] : kind == 1 ? &p.km[sid] : &p.vm[sid];
+    const uint32_t d0 = dst + box_row8(e) * 1024;
+#pragma unroll
+    for (int hf = 0; hf < NH; ++hf)
+      tma_load_5d(d0 + hf * kHalf, m, bar, hf * 64, U.h, gw, gh, U.b * p.T + gt);
+  }
+  for (int r = p.tile_rows[tile]; r < 128; r += 8) {  // zero rows past the window's tokens
+#pragma unroll
+    for (int hf = 0; hf < NH; ++hf)
+      tma_load_4d(dst + hf * kHalf + r * 128, &p.fill, bar, hf * 64, 0, (int)p.N, 0);
+  }
+}
+
+template <int D>
+__device__ __forceinline__ void store_tile(const TcParams& p, const Unit& U, int qt, uint32_t src) {
+  constexpr int NH = D / 64;
+  if (p.flat) {
+#pragma unroll
+    for (int hf = 0; hf < NH; ++hf) tma_store_4d(&p.of, src + hf * kHalf, hf * 64, U.h, qt * 128, U.b);
+    return;
+  }
+  const int nb = p.nbox[U.cls][qt];
+  for (int bi = 0; bi < nb; ++bi) {
+    const uint32_t e = p.box[U.cls][qt][bi];
+    const int sid = box_shape(e);
+    const int gt = (U.ot + box_lt(e)) % p.T;
+    const int gh = (U.oh + box_lh(e)) % p.Hg;
+    const int gw = (U.ow + box_lw(e)) % p.Wg;
+    const uint32_t s0 = src + box_row8(e) * 1024;
+#pragma unroll
+    for (int hf = 0; hf < NH; ++hf)
+      tma_store_5d(&p.om[sid], s0 + hf * kHalf, hf * 64, U.h, gw, gh, U.b * p.T + gt);
+  }
+}
+
+// Flattened grid index of the token held in row r of query tile qt.
+__device__ __forceinline__ long long row_token(const TcParams& p, const Unit& U, int qt, int r) {
+  if (p.flat) return 128LL * qt + r;
+  const int nb = p.nbox[U.cls][qt];
+  for (int bi = 0; bi < nb; ++bi) {
+    const uint32_t e = p.box[U.cls][qt][bi];
+    const int sid = box_shape(e);
+    const int bt = p.shape_bt[sid], bh = p.shape_bh[sid], bw = p.shape_bw[sid];
+    const int r0 = box_row8(e) * 8;
+    if (r >= r0 && r < r0 + bt * bh * bw) {
+      const int idx = r - r0;
+      const int it = idx / (bh * bw), ih = (idx / bw) % bh, iw = idx % bw;
+      const int gt = (U.ot + box_lt(e)) % p.T + it;
+      const int gh = (U.oh + box_lh(e)) % p.Hg + ih;
+      const int gw = (U.ow + box_lw(e)) % p.Wg + iw;
+      return ((long long)gt * p.Hg + gh) * p.Wg + gw;
+    }
+  }
+  return -1;
+}
+
+// Shared-memory plan.
+template <int D>
+struct Smem {
+  static constexpr int kTile = (D / 64) * kHalf;  // Q/K/V tile bytes
+  static constexpr int kPO = 2 * kHalf;           // P (128 x 128 bf16) or O staging
+  static constexpr int NS = D == 128 ? 3 : 6;     // K/V ring slots
+  static constexpr int q0 = 0;
+  static constexpr int po0 = 2 * kTile;
+  static constexpr int ring0 = po0 + 2 * kPO;
+  static constexpr int bars = ring0 + NS * kTile;
+  // barrier indices
+  static constexpr int QFULL = 0, QEMPTY = 2, SFULL = 4, SFREE = 6, PFULL = 8, PVDONE = 10,
+                       OSTAGED = 12, OFREE = 14, DRAIN = 16, KVFULL = 17, KVEMPTY = 17 + NS,
+                       NBARS = 17 + 2 * NS;
+  static constexpr int misc = bars + NBARS * 8;  // tmem slot, abort flag
+  static constexpr int bytes = misc + 64;
+  static constexpr int alloc = bytes + 1024;     // slack for 1024-byte alignment
+};
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1) tc_attn_kernel(const __grid_constant__ TcParams p) {
+  using S = Smem<D>;
+  constexpr int NS = S::NS;
+  constexpr int NH = D / 64;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t bar0 = sbase + S::bars;
+  auto BAR = [&](int i) -> uint32_t { return bar0 + 8u * (uint32_t)i; };
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + S::misc);
+  volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(smem + S::misc + 4);
+
+  const int warp = threadIdx.x / 32;
+  const int lane = threadIdx.x % 32;
+  const uint64_t limit = p.timeout_ns;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(BAR(S::QFULL + i), 1);
+      mbar_init(BAR(S::QEMPTY + i), 1);
+      mbar_init(BAR(S::SFULL + i), 1);
+      mbar_init(BAR(S::SFREE + i), 128);
+      mbar_init(BAR(S::PFULL + i), 128);
+      mbar_init(BAR(S::PVDONE + i), 1);
+      mbar_init(BAR(S::OSTAGED + i), 128);
+      mbar_init(BAR(S::OFREE + i), 1);
+    }
+    mbar_init(BAR(S::DRAIN), 1);
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(BAR(S::KVFULL + s), 1);
+      mbar_init(BAR(S::KVEMPTY + s), 1);
+    }
+    *abort_flag = 0u;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const int n_kt = p.n_wkt + p.n_pkt;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA loader
+    if (lane == 0 && !(p.flags & BASA_FLAG_TEST_WITHHOLD_LOADS)) {
+      uint32_t qn[2] = {0u, 0u};
+      uint32_t kv = 0;
+      uint32_t issued_mask = 0, last_par = 0, q_issued = 0, q_last = 0;
+      bool ok = true;
+      auto load_kv = [&](int kind, const Unit& U, int j) -> bool {
+        const uint32_t slot = kv % NS, par = (kv / NS) & 1u;
+        if (!wait_bounded(BAR(S::KVEMPTY + slot), par ^ 1u, abort_flag, limit)) return false;
+        mbar_expect_tx(BAR(S::KVFULL + slot), S::kTile);
+        load_tile<D>(p, kind, U, j, sbase + S::ring0 + slot * S::kTile, BAR(S::KVFULL + slot));
+        issued_mask |= 1u << slot;
+        last_par = (last_par & ~(1u << slot)) | (par << slot);
+        ++kv;
+        return true;
+      };
+      for (long long u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
+        const Unit U = decode_unit(p, u);
+        for (int i = 0; i < U.nq && ok; ++i) {
+          if (!wait_bounded(BAR(S::QEMPTY + i), (qn[i] & 1u) ^ 1u, abort_flag, limit)) {
+            ok = false;
+            break;
+          }
+          mbar_expect_tx(BAR(S::QFULL + i), S::kTile);
+          load_tile<D>(p, 0, U, 2 * U.pair + i, sbase + S::q0 + i * S::kTile, BAR(S::QFULL + i));
+          q_issued |= 1u << i;
+          q_last = (q_last & ~(1u << i)) | ((qn[i] & 1u) << i);
+          ++qn[i];
+        }
+        if (!ok) break;
+        ok = load_kv(1, U, 0);
+        for (int j = 0; j < n_kt && ok; ++j) {
+          if (j + 1 < n_kt) ok = load_kv(1, U, j + 1);
+          if (ok) ok = load_kv(2, U, j);
+        }
+      }
+      // Drain: wait (bounded, regardless of an abort) until every copy issued has landed.
+      for (int s = 0; s < NS; ++s)
+        if (issued_mask & (1u << s))
+          wait_bounded(BAR(S::KVFULL + s), (last_par >> s) & 1u, abort_flag, limit, false);
+      for (int i = 0; i < 2; ++i)
+        if (q_issued & (1u << i))
+          wait_bounded(BAR(S::QFULL + i), (q_last >> i) & 1u, abort_flag, limit, false);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t IDS = idesc_bf16(128, false);
+      constexpr uint32_t IDO = idesc_bf16(D, true);
+      uint32_t qf[2] = {0u, 0u}, sfree[2] = {0u, 0u}, pfull[2] = {0u, 0u};
+      uint32_t kv = 0;
+      bool ok = true;
+      auto take_slot = [&](uint32_t& slot) -> bool {
+        slot = kv % NS;
+        const uint32_t par = (kv / NS) & 1u;
+        ++kv;
+        if (!wait_bounded(BAR(S::KVFULL + slot), par, abort_flag, limit)) return false;
+        tc_fence_after();
+        return true;
+      };
+      auto issue_s = [&](int i, uint32_t kslot, bool last) -> bool {
+        if (!wait_bounded(BAR(S::SFREE + i), (sfree[i] & 1u) ^ 1u, abort_flag, limit)) return false;
+        ++sfree[i];
+        tc_fence_after();
+        const uint32_t qa = sbase + S::q0 + i * S::kTile;
+        const uint32_t ka = sbase + S::ring0 + kslot * S::kTile;
+#pragma unroll
+        for (int k = 0; k < D / 16; ++k) {
+          const uint32_t off = (k / 4) * kHalf + (k % 4) * 32;
+          mma_bf16(tmem + i * 128, sdesc(qa + off, 16, 1024), sdesc(ka + off, 16, 1024), IDS,
+                   k > 0 ? 1u : 0u);
+        }
+        mma_commit(BAR(S::SFULL + i));
+        if (last) mma_commit(BAR(S::QEMPTY + i));
+        return true;
+      };
+      for (long long u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
+        const Unit U = decode_unit(p, u);
+        for (int i = 0; i < U.nq && ok; ++i) {
+          ok = wait_bounded(BAR(S::QFULL + i), qf[i] & 1u, abort_flag, limit);
+          ++qf[i];
+        }
+        if (!ok) break;
+        tc_fence_after();
+        uint32_t kslot;
+        if (!(ok = take_slot(kslot))) break;
+        for (int i = 0; i < U.nq && ok; ++i) ok = issue_s(i, kslot, n_kt == 1);
+        if (!ok) break;
+        mma_commit(BAR(S::KVEMPTY + kslot));
+        for (int j = 0; j < n_kt && ok; ++j) {
+          if (j + 1 < n_kt) {
+            if (!(ok = take_slot(kslot))) break;
+            for (int i = 0; i < U.nq && ok; ++i) ok = issue_s(i, kslot, j + 1 == n_kt - 1);
+            if (!ok) break;
+            mma_commit(BAR(S::KVEMPTY + kslot));
+          }
+          uint32_t vslot;
+          if (!(ok = take_slot(vslot))) break;
+          const uint32_t va = sbase + S::ring0 + vslot * S::kTile;
+          for (int i = 0; i < U.nq && ok; ++i) {
+            if (!(ok = wait_bounded(BAR(S::PFULL + i), pfull[i] & 1u, abort_flag, limit))) break;
+            ++pfull[i];
+            tc_fence_after();
+            const uint32_t pa = sbase + S::po0 + i * S::kPO;
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+              const uint32_t aoff = (k / 4) * kHalf + (k % 4) * 32;
+              mma_bf16(tmem + 256 + i * 128, sdesc(pa + aoff, 16, 1024),
+                       sdesc(va + k * 2048, kHalf, 1024), IDO, (j > 0 || k > 0) ? 1u : 0u);
+            }
+            mma_commit(BAR(S::PVDONE + i));
+          }
+          if (!ok) break;
+          mma_commit(BAR(S::KVEMPTY + vslot));
+        }
+      }
+      // Drain: every MMA issued has completed before TMEM is released.
+      mma_commit(BAR(S::DRAIN));
+      wait_bounded(BAR(S::DRAIN), 0u, abort_flag, limit, false);
+    }
+  } else if (warp >= 4) {
+    // ------------------------------------------------------------ softmax + epilogue
+    const int i = (warp - 4) / 4;      // query tile slot of the unit
+    const int q4 = warp & 3;           // TMEM lane quadrant
+    const int r = q4 * 32 + lane;      // query row owned by this thread
+    const uint32_t tl = (uint32_t)(q4 * 32) << 16;
+    const uint32_t tS = tmem + tl + i * 128;
+    const uint32_t tO = tmem + tl + 256 + i * 128;
+    const uint32_t po = sbase + S::po0 + i * S::kPO;
+    const bool leader = (warp % 4 == 0) && lane == 0;
+    uint32_t sfull = 0, pvdone = 0, ostaged = 0, ofree = 0;
+    const float c = p.scale_log2;
+    bool ok = true;
+    for (long long u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
+      const Unit U = decode_unit(p, u);
+      if (i >= U.nq) continue;
+      const int qt = 2 * U.pair + i;
+      float m = -INFINITY, l = 0.f;
+      for (int j = 0; j < n_kt; ++j) {
+        if (!(ok = wait_warp(BAR(S::SFULL + i), sfull & 1u, abort_flag, limit))) break;
+        ++sfull;
+        tc_fence_after();
+        uint32_t s[4][32];
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc) tmem_ld32(tS + cc * 32, s[cc]);
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc) tmem_wait_ld(s[cc]);
+        tc_fence_before();
+        mbar_arrive(BAR(S::SFREE + i));
+        const int kvalid = key_valid(p, j);
+        float mx = -INFINITY;
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc)
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            const float x = (cc * 32 + e < kvalid) ? __uint_as_float(s[cc][e]) : -INFINITY;
+            s[cc][e] = __float_as_uint(x);
+            mx = fmaxf(mx, x);
+          }
+        const float mnew = fmaxf(m, mx * c);
+        const float alpha = ex2(m - mnew);  // 0 on the first key tile
+        float rs = 0.f;
+        uint32_t pk[4][16];
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc)
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const float p0 = ex2(fmaf(__uint_as_float(s[cc][2 * e]), c, -mnew));
+            const float p1 = ex2(fmaf(__uint_as_float(s[cc][2 * e + 1]), c, -mnew));
+            rs += p0 + p1;
+            pk[cc][e] = pack_bf16(p0, p1);
+          }
+        l = l * alpha + rs;
+        m = mnew;
+        if (j > 0) {  // PV of the previous key tile must be done: O is stable, P is free
+          if (!(ok = wait_warp(BAR(S::PVDONE + i), pvdone & 1u, abort_flag, limit))) break;
+          ++pvdone;
+          tc_fence_after();
+        }
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc)
+#pragma unroll
+          for (int v4 = 0; v4 < 4; ++v4) {
+            const int chunk = cc * 4 + v4;  // 8 keys per 16-byte chunk
+            st_shared_v4(po + (chunk / 8) * kHalf + swz(r, chunk % 8), pk[cc][4 * v4],
+                         pk[cc][4 * v4 + 1], pk[cc][4 * v4 + 2], pk[cc][4 * v4 + 3]);
+          }
+        if (j > 0 && alpha < 1.0f) {
+#pragma unroll
+          for (int cc = 0; cc < D / 32; ++cc) {
+            uint32_t o[32];
+            tmem_ld32(tO + cc * 32, o);
+            tmem_wait_ld(o);
+#pragma unroll
+            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+            tmem_st32(tO + cc * 32, o);
+          }
+          tmem_wait_st();
+        }
+        fence_proxy_async();
+        tc_fence_before();
+        mbar_arrive(BAR(S::PFULL + i));
+      }
+      if (!ok) break;
+      if (!(ok = wait_warp(BAR(S::PVDONE + i), pvdone & 1u, abort_flag, limit))) break;
+      ++pvdone;
+      tc_fence_after();
+      // epilogue: O / l -> bf16 -> staging (the P buffer, free now) -> TMA store
+      const float inv = 1.0f / l;
+#pragma unroll
+      for (int cc = 0; cc < D / 32; ++cc) {
+        uint32_t o[32];
+        tmem_ld32(tO + cc * 32, o);
+        tmem_wait_ld(o);
+#pragma unroll
+        for (int v4 = 0; v4 < 4; ++v4) {
+          const int col = cc * 32 + v4 * 8;
+          uint32_t w[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            w[e] = pack_bf16(__uint_as_float(o[v4 * 8 + 2 * e]) * inv,
+                             __uint_as_float(o[v4 * 8 + 2 * e + 1]) * inv);
+          st_shared_v4(po + (col / 64) * kHalf + swz(r, (col % 64) / 8), w[0], w[1], w[2], w[3]);
+        }
+      }
+      tc_fence_before();
+      if (p.lse && r < query_valid(p, qt)) {
+        const long long n = row_token(p, U, qt, r);
+        if (n >= 0)
+          p.lse[((long long)U.b * p.H + U.h) * p.N + n] = (m + __log2f(l)) * 0.69314718055994531f;
+      }
+      fence_proxy_async();
+      mbar_arrive(BAR(S::OSTAGED + i));
+      if (leader) {
+        const bool staged = wait_bounded(BAR(S::OSTAGED + i), ostaged & 1u, abort_flag, limit);
+        if (staged) {
+          store_tile<D>(p, U, qt, po);
+          bulk_commit();
+          bulk_wait_read0();
+        }
+        mbar_arrive(BAR(S::OFREE + i));
+      }
+      ++ostaged;
+      if (!(ok = wait_warp(BAR(S::OFREE + i), ofree & 1u, abort_flag, limit))) break;
+      ++ofree;
+    }
+    if (leader) bulk_wait_all0();
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem, 512);
+}
+
+int sm_count() {
+  int dev = 0, n = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n > 0 ? n : 1;
+}
+
+template <int D>
+basa_status launch_impl(TcParams* prm, cudaStream_t stream) {
+  const int smem = Smem<D>::alloc;
+  static_assert(Smem<D>::alloc <= 232448, "shared memory plan exceeds 227 KB");
+  if (cudaFuncSetAttribute(tc_attn_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+      cudaSuccess)
+    return BASA_ERR_CUDA;
+  long long grid = sm_count();
+  if (grid > prm->n_units) grid = prm->n_units;
+  tc_attn_kernel<D><<<(unsigned)grid, kThreads, smem, stream>>>(*prm);
+  return cudaGetLastError() == cudaSuccess ? BASA_OK : BASA_ERR_CUDA;
+}
+
+}  // namespace
+
+basa_status launch_tc(const Dims& d, bool flat, const void* q, const void* k, const void* v,
+                      const void* kp, const void* vp, void* out, float* lse, uint32_t flags,
+                      uint32_t timeout_ms, cudaStream_t stream) {
+  TcParams* prm = new (std::nothrow) TcParams;
+  if (!prm) return BASA_ERR_INVALID_ARG;
+  memset(prm, 0, sizeof(*prm));
+  basa_status st = BASA_OK;
+  const uint64_t D = (uint64_t)d.d;
+  const uint64_t H = (uint64_t)d.H;
+  prm->B = d.B; prm->H = d.H; prm->T = d.T; prm->Hg = d.Hg; prm->Wg = d.Wg;
+  prm->wt = d.wt; prm->wh = d.wh; prm->ww = d.ww;
+  prm->st = d.st; prm->sh = d.sh; prm->sw = d.sw;
+  prm->nwt = d.nwt; prm->nwh = d.nwh; prm->nww = d.nww;
+  prm->N = d.N;
+  prm->lse = lse;
+  prm->flags = flags;
+  prm->timeout_ns = (unsigned long long)(timeout_ms ? timeout_ms : 2000u) * 1000000ull;
+  prm->scale_log2 = d.scale * 1.4426950408889634f;
+  prm->flat = flat ? 1 : 0;
+  prm->P = kp ? (int)d.P : 0;
+  TilePlan plan;
+  if (!flat && (st = build_tile_plan(d, &plan)) != BASA_OK) goto done;  // before any driver call
+  // flat [d, H, N, B] views (full attention tiles; the fill source)
+  {
+    const uint64_t dims[4] = {D, H, (uint64_t)d.N, (uint64_t)d.B};
+    const uint64_t strides[3] = {D * 2, H * D * 2, (uint64_t)d.N * H * D * 2};
+    const uint32_t box128[4] = {64, 1, 128, 1};
+    const uint32_t box8[4] = {64, 1, 8, 1};
+    if (flat) {
+      if ((st = encode_map(&prm->qf, q, 4, dims, strides, box128)) != BASA_OK) goto done;
+      if ((st = encode_map(&prm->kf, k, 4, dims, strides, box128)) != BASA_OK) goto done;
+      if ((st = encode_map(&prm->vf, v, 4, dims, strides, box128)) != BASA_OK) goto done;
+      if ((st = encode_map(&prm->of, out, 4, dims, strides, box128)) != BASA_OK) goto done;
+    } else {
+      if ((st = encode_map(&prm->fill, k, 4, dims, strides, box8)) != BASA_OK) goto done;
+    }
+  }
+  if (flat) {
+    const long long nt = (d.N + 127) / 128;
+    if (nt > (1LL << 24)) { st = BASA_ERR_UNSUPPORTED; goto done; }
+    prm->n_qt = (int)nt;
+    prm->n_wkt = (int)nt;
+    prm->n_pkt = 0;
+    prm->n_windows = 1;
+    prm->n_pairs = (prm->n_qt + 1) / 2;
+    prm->n_units = (long long)d.B * d.H * prm->n_pairs;
+  } else {
+    memcpy(prm->box, plan.box, sizeof(plan.box));
+    memcpy(prm->nbox, plan.nbox, sizeof(plan.nbox));
+    memcpy(prm->tile_rows, plan.tile_rows, sizeof(plan.tile_rows));
+    memcpy(prm->shape_bt, plan.shape_bt, sizeof(plan.shape_bt));
+    memcpy(prm->shape_bh, plan.shape_bh, sizeof(plan.shape_bh));
+    memcpy(prm->shape_bw, plan.shape_bw, sizeof(plan.shape_bw));
+    const uint64_t dims[5] = {D, H, (uint64_t)d.Wg, (uint64_t)d.Hg, (uint64_t)d.B * d.T};
+    const uint64_t strides[4] = {D * 2, H * D * 2, (uint64_t)d.Wg * H * D * 2,
+                                 (uint64_t)d.Hg * d.Wg * H * D * 2};
+    for (int s = 0; s < plan.n_shapes; ++s) {
+      const uint32_t box[5] = {64, 1, plan.shape_bw[s], plan.shape_bh[s], plan.shape_bt[s]};
+      if ((st = encode_map(&prm->qm[s], q, 5, dims, strides, box)) != BASA_OK) goto done;
+      if ((st = encode_map(&prm->km[s], k, 5, dims, strides, box)) != BASA_OK) goto done;
+      if ((st = encode_map(&prm->vm[s], v, 5, dims, strides, box)) != BASA_OK) goto done;
+      if ((st = encode_map(&prm->om[s], out, 5, dims, strides, box)) != BASA_OK) goto done;
+    }
+    if (kp) {
+      const uint64_t pdims[4] = {D, H, (uint64_t)d.P, (uint64_t)d.B};
+      const uint64_t pstr[3] = {D * 2, H * D * 2, (uint64_t)d.P * H * D * 2};
+      const uint32_t box128[4] = {64, 1, 128, 1};
+      if ((st = encode_map(&prm->kpf, kp, 4, pdims, pstr, box128)) != BASA_OK) goto done;
+      if ((st = encode_map(&prm->vpf, vp, 4, pdims, pstr, box128)) != BASA_OK) goto done;
+    }
+    prm->n_qt = plan.n_tiles;
+    prm->n_wkt = plan.n_tiles;
+    prm->n_pkt = kp ? (int)((d.P + 127) / 128) : 0;
+    prm->n_windows = d.nwt * d.nwh * d.nww;
+    prm->n_pairs = (prm->n_qt + 1) / 2;
+    prm->n_units = (long long)d.B * d.H * prm->n_windows * prm->n_pairs;
+  }
+  st = d.d == 128 ? launch_impl<128>(prm, stream) : launch_impl<64>(prm, stream);
+done:
+  delete prm;
+  return st;
+}
+
+basa_status read_and_clear_status(cudaStream_t stream) {
+  if (cudaStreamSynchronize(stream) != cudaSuccess) return BASA_ERR_CUDA;
+  unsigned int v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_basa_status, sizeof(v)) != cudaSuccess) return BASA_ERR_CUDA;
+  if (v) {
+    const unsigned int zero = 0;
+    if (cudaMemcpyToSymbol(g_basa_status, &zero, sizeof(zero)) != cudaSuccess) return BASA_ERR_CUDA;
+    return BASA_ERR_TIMEOUT;
+  }
+  return cudaGetLastError() == cudaSuccess ? BASA_OK : BASA_ERR_CUDA;
+}
+
+}  // namespace basa

@@ -1,0 +1,155 @@
+"""Host-side tests of the C ABI: symbols, validation codes and the window tile
+plan.  None of these launch anything, so they run without a GPU."""
+import ctypes
+import itertools
+import os
+import re
+
+import numpy as np
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="session")
+def lib():
+    from sparse_attention_diffusion_basa_b200 import build
+    build.build()
+    from sparse_attention_diffusion_basa_b200 import _lib
+    return _lib.load()
+
+
+def _declared_symbols():
+    src = open(os.path.join(ROOT, "include", "basa.h")).read()
+    return sorted(set(re.findall(r"BASA_API\s+[\w\s\*]*?\b(basa_\w+)\s*\(", src)))
+
+
+def test_exports_every_declared_symbol(lib):
+    from sparse_attention_diffusion_basa_b200 import _lib
+    declared = _declared_symbols()
+    assert len(declared) >= 9
+    assert set(declared) == set(_lib.EXPORTS)
+    for name in declared:
+        assert hasattr(lib, name), name
+    assert lib.basa_version() >= 100
+    for code in range(8):
+        assert lib.basa_status_string(code)
+
+
+def _p(**kw):
+    from sparse_attention_diffusion_basa_b200 import make_params
+    shape = kw.pop("shape", (1, 1, 16, 16, 2, 64))
+    dtype = kw.pop("dtype", 1)
+    return make_params(shape, dtype, kw.pop("window", (1, 8, 8)), kw.pop("shift", (0, 4, 4)),
+                       kw.pop("pool", (0, 0, 0)), kw.pop("scale", None))
+
+
+def _fake(addr=0x10000):
+    return ctypes.c_void_p(addr)
+
+
+def test_validation_codes(lib):
+    from sparse_attention_diffusion_basa_b200 import _lib
+    call = lambda prm, q=_fake(), ws=None: lib.basa_window_attn(
+        q, _fake(), _fake(), _fake(), None, ws, ctypes.byref(prm), None)
+    assert call(_p(window=(1, 5, 8))) == 2                      # does not divide the grid
+    assert call(_p(window=(0, 8, 8))) == 1                      # zero window
+    assert call(_p(shape=(1, 1, 16, 16, 2, 48))) == 3           # head dim
+    assert call(_p(shape=(1, 1, 16, 16, 2, 32), dtype=1)) == 3  # bf16 needs d in {64, 128}
+    assert call(_p(), q=_fake(0x10008)) == 4                    # misaligned
+    assert call(_p(), q=None) == 1                              # null
+    assert call(_p(pool=(1, 2, 2))) == 5                        # workspace missing
+    assert call(_p(pool=(1, 3, 2))) == 2                        # pool does not divide
+    assert call(_p(pool=(0, 2, 2))) == 1                        # partial pool spec
+    prm = _p()
+    prm.dtype = 7
+    assert call(prm) == 1
+    # empty problems are valid no-ops and touch nothing
+    assert call(_p(shape=(0, 1, 16, 16, 2, 64)), q=None) == 0
+    assert lib.basa_full_attn(None, None, None, None, None,
+                              ctypes.byref(_p(shape=(1, 1, 16, 16, 0, 64))), None) == 0
+    # bf16 plans whose wrapped boxes are not a multiple of 8 tokens are refused
+    assert call(_p(shape=(1, 1, 16, 16, 2, 64), window=(1, 8, 8), shift=(0, 3, 3))) == 3
+    # gm variant needs pooled tensors and a pool spec
+    assert lib.basa_window_attn_gm(_fake(), _fake(), _fake(), None, None, _fake(), None,
+                                   ctypes.byref(_p(pool=(1, 2, 2))), None) == 1
+    assert lib.basa_window_attn_gm(_fake(), _fake(), _fake(), _fake(), _fake(), _fake(), None,
+                                   ctypes.byref(_p()), None) == 1
+    # pooling: needs a pool spec, aligned pointers
+    assert lib.basa_pool_kv(_fake(), _fake(), _fake(), _fake(), ctypes.byref(_p()), None) == 1
+    assert lib.basa_pool_kv(_fake(), _fake(), _fake(0x10004), _fake(),
+                            ctypes.byref(_p(pool=(1, 2, 2))), None) == 4
+    assert _lib.STATUS_NAMES[4] == "BASA_ERR_ALIGN"
+
+
+def test_workspace_size(lib):
+    from sparse_attention_diffusion_basa_b200 import workspace_size
+    import torch
+    assert workspace_size((1, 1, 16, 16, 2, 64), torch.bfloat16, (1, 8, 8)) == 0
+    # pooled K and V of [B, P, H, d] bf16, each rounded up to 256 bytes
+    n = 2 * 64 * 24 * 128 * 2
+    assert workspace_size((2, 1, 32, 32, 24, 128), torch.bfloat16, (1, 16, 16),
+                          pool=(1, 4, 4)) == 2 * ((n + 255) // 256 * 256)
+    assert workspace_size((1, 1, 4, 4, 1, 32), torch.float32, (1, 2, 2),
+                          pool=(1, 2, 2)) == 2 * 512  # 4 cells x 32 x fp32
+
+
+def _window_sets(grid, window, shift):
+    """Token sets of every shifted window, from the window-id formula."""
+    T, Hg, Wg = grid
+    ids = {}
+    for t, y, x in itertools.product(range(T), range(Hg), range(Wg)):
+        key = (((t - shift[0]) % T) // window[0], ((y - shift[1]) % Hg) // window[1],
+               ((x - shift[2]) % Wg) // window[2])
+        ids.setdefault(key, set()).add((t * Hg + y) * Wg + x)
+    return ids
+
+
+PLAN_CASES = [
+    ((1, 16, 16), (1, 8, 8), [(0, 0, 0), (0, 4, 0), (0, 0, 4), (0, 4, 4)]),
+    ((1, 64, 64), (1, 16, 16), [(0, 0, 0), (0, 8, 8), (0, 8, 0), (0, 0, 8), (0, -8, 24)]),
+    ((21, 45, 80), (7, 9, 16), [(3, 4, 8), (0, 0, 0), (1, 5, 8), (6, 8, 0)]),
+    ((4, 6, 32), (2, 3, 16), [(1, 1, 8), (1, 2, 0)]),
+    ((2, 8, 8), (2, 8, 8), [(0, 0, 0), (1, 0, 0)]),
+    ((1, 24, 8), (1, 24, 8), [(0, 5, 0), (0, 16, 0)]),
+]
+
+
+@pytest.mark.parametrize("grid,window,shifts", PLAN_CASES)
+def test_tile_plan_covers_each_shifted_window_once(lib, grid, window, shifts):
+    from sparse_attention_diffusion_basa_b200 import window_tiles
+    for shift in shifts:
+        rows = window_tiles(grid, window, shift)
+        sets = _window_sets(grid, window, shift)
+        assert rows.shape[0] == len(sets)
+        m = window[0] * window[1] * window[2]
+        seen = set()
+        for w in range(rows.shape[0]):
+            toks = rows[w][rows[w] >= 0]
+            assert len(toks) == m, (shift, w)
+            assert len(set(toks.tolist())) == m
+            assert set(toks.tolist()) in [s for s in sets.values()], (shift, w)
+            seen |= set(toks.tolist())
+            # every 128-row tile is a prefix of real rows followed by padding
+            for tile in rows[w]:
+                n = int((tile >= 0).sum())
+                assert (tile[:n] >= 0).all() and (tile[n:] < 0).all()
+                assert n % 8 == 0
+        assert seen == set(range(grid[0] * grid[1] * grid[2]))
+
+
+def test_tile_plan_counts(lib):
+    from sparse_attention_diffusion_basa_b200 import window_tiles
+    assert window_tiles((1, 128, 128), (1, 16, 16), (0, 8, 8)).shape == (64, 2, 128)
+    # the video window of 7 x 9 x 16 tokens: seven 8-row tiles and one of 7 x 1 rows
+    r = window_tiles((21, 45, 80), (7, 9, 16), (3, 4, 8))
+    assert r.shape == (75, 8, 128)
+    assert sorted(int((t >= 0).sum()) for t in r[0]) == [112] + [128] * 7
+
+
+def test_tile_plan_rejects_unsupported(lib):
+    from sparse_attention_diffusion_basa_b200 import window_tiles, BasaError
+    with pytest.raises(BasaError):
+        window_tiles((1, 16, 256), (1, 16, 256), (0, 0, 0))   # window row wider than 128
+    with pytest.raises(BasaError):
+        window_tiles((1, 16, 16), (1, 8, 8), (0, 3, 5))        # wrapped boxes of 3 x 5 tokens
