@@ -61,23 +61,45 @@ def build_oracle(force: bool = False) -> str:
     return _build.build(force=force)
 
 
+def _bind(path):
+    lib = ctypes.CDLL(path)
+    dp = ctypes.POINTER(ctypes.c_double)
+    lib.oracle_pool.argtypes = [dp, dp, ctypes.POINTER(_CParams)]
+    lib.oracle_pool.restype = None
+    lib.oracle_window_attn.argtypes = [dp, dp, dp, dp, dp, dp, dp,
+                                       ctypes.POINTER(_CParams),
+                                       ctypes.POINTER(ctypes.c_int64),
+                                       ctypes.c_int64, ctypes.c_int]
+    lib.oracle_window_attn.restype = ctypes.c_int
+    lib.oracle_max_threads.argtypes = []
+    lib.oracle_max_threads.restype = ctypes.c_int
+    return lib
+
+
 def _load():
     global _lib
     if _lib is None:
-        path = _build.build()
-        lib = ctypes.CDLL(path)
-        dp = ctypes.POINTER(ctypes.c_double)
-        lib.oracle_pool.argtypes = [dp, dp, ctypes.POINTER(_CParams)]
-        lib.oracle_pool.restype = None
-        lib.oracle_window_attn.argtypes = [dp, dp, dp, dp, dp, dp, dp,
-                                           ctypes.POINTER(_CParams),
-                                           ctypes.POINTER(ctypes.c_int64),
-                                           ctypes.c_int64, ctypes.c_int]
-        lib.oracle_window_attn.restype = ctypes.c_int
-        lib.oracle_max_threads.argtypes = []
-        lib.oracle_max_threads.restype = ctypes.c_int
-        _lib = lib
+        _lib = _bind(_build.build())
     return _lib
+
+
+class use_library:
+    """Context manager that routes oracle calls to another compiled copy of the
+    oracle (used by the tests that plant mistakes in a copy of the C source)."""
+
+    def __init__(self, path):
+        self.path = path
+
+    def __enter__(self):
+        global _lib
+        self.saved = _load()
+        _lib = _bind(self.path)
+        return self
+
+    def __exit__(self, *exc):
+        global _lib
+        _lib = self.saved
+        return False
 
 
 def _ptr(a: Optional[np.ndarray]):

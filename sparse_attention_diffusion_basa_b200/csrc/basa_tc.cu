@@ -32,6 +32,8 @@
 // (bounded) for its own copies and MMAs in flight, frees TMEM and returns.
 #include <cuda_bf16.h>
 #include <math.h>
+#include <stdio.h>
+#include <stdlib.h>
 #include <string.h>
 
 #include <new>
@@ -41,6 +43,7 @@
 namespace basa {
 
 __device__ unsigned int g_basa_status;  // bit 0: a device wait timed out
+__device__ unsigned int g_basa_where;   // site of the first wait that gave up
 
 namespace {
 
@@ -273,18 +276,29 @@ __device__ __forceinline__ uint32_t swz(int row, int chunk) {
 
 // ---------------------------------------------------------------------------
 // Bounded waits.  `abort_flag` lives in shared memory; any role that gives up
-// raises it so that the others leave their loops promptly.
+// raises it so that the others leave their loops promptly.  A wait is bounded
+// both by the global nanosecond timer and by SM cycles (at most 2 per ns), and
+// the first wait that gives up records its site in g_basa_where.
 // ---------------------------------------------------------------------------
+enum WaitSite : uint32_t {
+  kSiteLoadKvEmpty = 1, kSiteLoadQEmpty, kSiteLoadDrainKv, kSiteLoadDrainQ, kSiteMmaQFull,
+  kSiteMmaKvFull, kSiteMmaSFree, kSiteMmaPFull, kSiteMmaDrain, kSiteSmxSFull, kSiteSmxPvDone,
+  kSiteSmxPvLast, kSiteSmxOStaged, kSiteSmxOFree
+};
+
 __device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity,
                                              volatile uint32_t* abort_flag, uint64_t limit_ns,
-                                             bool honour_abort = true) {
+                                             uint32_t site, bool honour_abort = true) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer();
+  const long long c0 = clock64();
+  const long long climit = (long long)(limit_ns * 2ull);
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
     if (honour_abort && *abort_flag) return false;
-    if (globaltimer() - t0 > limit_ns) {
+    if (globaltimer() - t0 > limit_ns || clock64() - c0 > climit) {
       *abort_flag = 1u;
+      atomicCAS(&g_basa_where, 0u, site);
       atomicOr(&g_basa_status, 1u);
       return false;
     }
@@ -292,8 +306,9 @@ __device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity,
 }
 // Warp-uniform variant: every lane waits, and the warp proceeds only if all did.
 __device__ __forceinline__ bool wait_warp(uint32_t bar, uint32_t parity,
-                                          volatile uint32_t* abort_flag, uint64_t limit_ns) {
-  const bool ok = wait_bounded(bar, parity, abort_flag, limit_ns);
+                                          volatile uint32_t* abort_flag, uint64_t limit_ns,
+                                          uint32_t site, bool honour_abort = true) {
+  const bool ok = wait_bounded(bar, parity, abort_flag, limit_ns, site, honour_abort);
   return __all_sync(0xffffffffu, ok);
 }
 
@@ -495,16 +510,21 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attn_kernel(const __grid_const
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA loader
-    if (lane == 0 && !(p.flags & BASA_FLAG_TEST_WITHHOLD_LOADS)) {
+    // The whole warp walks the schedule and waits; lane 0 issues the copies.
+    if (!(p.flags & BASA_FLAG_TEST_WITHHOLD_LOADS)) {
       uint32_t qn[2] = {0u, 0u};
       uint32_t kv = 0;
       uint32_t issued_mask = 0, last_par = 0, q_issued = 0, q_last = 0;
       bool ok = true;
       auto load_kv = [&](int kind, const Unit& U, int j) -> bool {
         const uint32_t slot = kv % NS, par = (kv / NS) & 1u;
-        if (!wait_bounded(BAR(S::KVEMPTY + slot), par ^ 1u, abort_flag, limit)) return false;
-        mbar_expect_tx(BAR(S::KVFULL + slot), S::kTile);
-        load_tile<D>(p, kind, U, j, sbase + S::ring0 + slot * S::kTile, BAR(S::KVFULL + slot));
+        if (!wait_warp(BAR(S::KVEMPTY + slot), par ^ 1u, abort_flag, limit, kSiteLoadKvEmpty))
+          return false;
+        if (lane == 0) {
+          mbar_expect_tx(BAR(S::KVFULL + slot), S::kTile);
+          load_tile<D>(p, kind, U, j, sbase + S::ring0 + slot * S::kTile, BAR(S::KVFULL + slot));
+        }
+        __syncwarp();
         issued_mask |= 1u << slot;
         last_par = (last_par & ~(1u << slot)) | (par << slot);
         ++kv;
@@ -513,12 +533,15 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attn_kernel(const __grid_const
       for (long long u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
         const Unit U = decode_unit(p, u);
         for (int i = 0; i < U.nq && ok; ++i) {
-          if (!wait_bounded(BAR(S::QEMPTY + i), (qn[i] & 1u) ^ 1u, abort_flag, limit)) {
-            ok = false;
+          if (!(ok = wait_warp(BAR(S::QEMPTY + i), (qn[i] & 1u) ^ 1u, abort_flag, limit,
+                               kSiteLoadQEmpty)))
             break;
+          if (lane == 0) {
+            mbar_expect_tx(BAR(S::QFULL + i), S::kTile);
+            load_tile<D>(p, 0, U, 2 * U.pair + i, sbase + S::q0 + i * S::kTile,
+                         BAR(S::QFULL + i));
           }
-          mbar_expect_tx(BAR(S::QFULL + i), S::kTile);
-          load_tile<D>(p, 0, U, 2 * U.pair + i, sbase + S::q0 + i * S::kTile, BAR(S::QFULL + i));
+          __syncwarp();
           q_issued |= 1u << i;
           q_last = (q_last & ~(1u << i)) | ((qn[i] & 1u) << i);
           ++qn[i];
@@ -533,31 +556,35 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attn_kernel(const __grid_const
       // Drain: wait (bounded, regardless of an abort) until every copy issued has landed.
       for (int s = 0; s < NS; ++s)
         if (issued_mask & (1u << s))
-          wait_bounded(BAR(S::KVFULL + s), (last_par >> s) & 1u, abort_flag, limit, false);
+          wait_warp(BAR(S::KVFULL + s), (last_par >> s) & 1u, abort_flag, limit,
+                    kSiteLoadDrainKv, false);
       for (int i = 0; i < 2; ++i)
         if (q_issued & (1u << i))
-          wait_bounded(BAR(S::QFULL + i), (q_last >> i) & 1u, abort_flag, limit, false);
+          wait_warp(BAR(S::QFULL + i), (q_last >> i) & 1u, abort_flag, limit, kSiteLoadDrainQ,
+                    false);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t IDS = idesc_bf16(128, false);
-      constexpr uint32_t IDO = idesc_bf16(D, true);
-      uint32_t qf[2] = {0u, 0u}, sfree[2] = {0u, 0u}, pfull[2] = {0u, 0u};
-      uint32_t kv = 0;
-      bool ok = true;
-      auto take_slot = [&](uint32_t& slot) -> bool {
-        slot = kv % NS;
-        const uint32_t par = (kv / NS) & 1u;
-        ++kv;
-        if (!wait_bounded(BAR(S::KVFULL + slot), par, abort_flag, limit)) return false;
-        tc_fence_after();
-        return true;
-      };
-      auto issue_s = [&](int i, uint32_t kslot, bool last) -> bool {
-        if (!wait_bounded(BAR(S::SFREE + i), (sfree[i] & 1u) ^ 1u, abort_flag, limit)) return false;
-        ++sfree[i];
-        tc_fence_after();
+    // The whole warp walks the schedule and waits; lane 0 issues MMAs and commits.
+    constexpr uint32_t IDS = idesc_bf16(128, false);
+    constexpr uint32_t IDO = idesc_bf16(D, true);
+    uint32_t qf[2] = {0u, 0u}, sfree[2] = {0u, 0u}, pfull[2] = {0u, 0u};
+    uint32_t kv = 0;
+    bool ok = true;
+    auto take_slot = [&](uint32_t& slot) -> bool {
+      slot = kv % NS;
+      const uint32_t par = (kv / NS) & 1u;
+      ++kv;
+      if (!wait_warp(BAR(S::KVFULL + slot), par, abort_flag, limit, kSiteMmaKvFull)) return false;
+      tc_fence_after();
+      return true;
+    };
+    auto issue_s = [&](int i, uint32_t kslot, bool last) -> bool {
+      if (!wait_warp(BAR(S::SFREE + i), (sfree[i] & 1u) ^ 1u, abort_flag, limit, kSiteMmaSFree))
+        return false;
+      ++sfree[i];
+      tc_fence_after();
+      if (lane == 0) {
         const uint32_t qa = sbase + S::q0 + i * S::kTile;
         const uint32_t ka = sbase + S::ring0 + kslot * S::kTile;
 #pragma unroll
@@ -568,35 +595,44 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attn_kernel(const __grid_const
         }
         mma_commit(BAR(S::SFULL + i));
         if (last) mma_commit(BAR(S::QEMPTY + i));
-        return true;
-      };
-      for (long long u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
-        const Unit U = decode_unit(p, u);
-        for (int i = 0; i < U.nq && ok; ++i) {
-          ok = wait_bounded(BAR(S::QFULL + i), qf[i] & 1u, abort_flag, limit);
-          ++qf[i];
+      }
+      __syncwarp();
+      return true;
+    };
+    auto release = [&](uint32_t slot) {
+      if (lane == 0) mma_commit(BAR(S::KVEMPTY + slot));
+      __syncwarp();
+    };
+    for (long long u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
+      const Unit U = decode_unit(p, u);
+      for (int i = 0; i < U.nq && ok; ++i) {
+        ok = wait_warp(BAR(S::QFULL + i), qf[i] & 1u, abort_flag, limit, kSiteMmaQFull);
+        ++qf[i];
+      }
+      if (!ok) break;
+      tc_fence_after();
+      uint32_t kslot;
+      if (!(ok = take_slot(kslot))) break;
+      for (int i = 0; i < U.nq && ok; ++i) ok = issue_s(i, kslot, n_kt == 1);
+      if (!ok) break;
+      release(kslot);
+      for (int j = 0; j < n_kt && ok; ++j) {
+        if (j + 1 < n_kt) {
+          if (!(ok = take_slot(kslot))) break;
+          for (int i = 0; i < U.nq && ok; ++i) ok = issue_s(i, kslot, j + 1 == n_kt - 1);
+          if (!ok) break;
+          release(kslot);
         }
-        if (!ok) break;
-        tc_fence_after();
-        uint32_t kslot;
-        if (!(ok = take_slot(kslot))) break;
-        for (int i = 0; i < U.nq && ok; ++i) ok = issue_s(i, kslot, n_kt == 1);
-        if (!ok) break;
-        mma_commit(BAR(S::KVEMPTY + kslot));
-        for (int j = 0; j < n_kt && ok; ++j) {
-          if (j + 1 < n_kt) {
-            if (!(ok = take_slot(kslot))) break;
-            for (int i = 0; i < U.nq && ok; ++i) ok = issue_s(i, kslot, j + 1 == n_kt - 1);
-            if (!ok) break;
-            mma_commit(BAR(S::KVEMPTY + kslot));
-          }
-          uint32_t vslot;
-          if (!(ok = take_slot(vslot))) break;
-          const uint32_t va = sbase + S::ring0 + vslot * S::kTile;
-          for (int i = 0; i < U.nq && ok; ++i) {
-            if (!(ok = wait_bounded(BAR(S::PFULL + i), pfull[i] & 1u, abort_flag, limit))) break;
-            ++pfull[i];
-            tc_fence_after();
+        uint32_t vslot;
+        if (!(ok = take_slot(vslot))) break;
+        const uint32_t va = sbase + S::ring0 + vslot * S::kTile;
+        for (int i = 0; i < U.nq && ok; ++i) {
+          if (!(ok = wait_warp(BAR(S::PFULL + i), pfull[i] & 1u, abort_flag, limit,
+                               kSiteMmaPFull)))
+            break;
+          ++pfull[i];
+          tc_fence_after();
+          if (lane == 0) {
             const uint32_t pa = sbase + S::po0 + i * S::kPO;
 #pragma unroll
             for (int k = 0; k < 8; ++k) {
@@ -606,14 +642,16 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attn_kernel(const __grid_const
             }
             mma_commit(BAR(S::PVDONE + i));
           }
-          if (!ok) break;
-          mma_commit(BAR(S::KVEMPTY + vslot));
+          __syncwarp();
         }
+        if (!ok) break;
+        release(vslot);
       }
-      // Drain: every MMA issued has completed before TMEM is released.
-      mma_commit(BAR(S::DRAIN));
-      wait_bounded(BAR(S::DRAIN), 0u, abort_flag, limit, false);
     }
+    // Drain: every MMA issued has completed before TMEM is released.
+    if (lane == 0) mma_commit(BAR(S::DRAIN));
+    __syncwarp();
+    wait_warp(BAR(S::DRAIN), 0u, abort_flag, limit, kSiteMmaDrain, false);
   } else if (warp >= 4) {
     // ------------------------------------------------------------ softmax + epilogue
     const int i = (warp - 4) / 4;      // query tile slot of the unit
@@ -633,7 +671,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attn_kernel(const __grid_const
       const int qt = 2 * U.pair + i;
       float m = -INFINITY, l = 0.f;
       for (int j = 0; j < n_kt; ++j) {
-        if (!(ok = wait_warp(BAR(S::SFULL + i), sfull & 1u, abort_flag, limit))) break;
+        if (!(ok = wait_warp(BAR(S::SFULL + i), sfull & 1u, abort_flag, limit, kSiteSmxSFull)))
+          break;
         ++sfull;
         tc_fence_after();
         uint32_t s[4][32];
@@ -669,7 +708,9 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attn_kernel(const __grid_const
         l = l * alpha + rs;
         m = mnew;
         if (j > 0) {  // PV of the previous key tile must be done: O is stable, P is free
-          if (!(ok = wait_warp(BAR(S::PVDONE + i), pvdone & 1u, abort_flag, limit))) break;
+          if (!(ok = wait_warp(BAR(S::PVDONE + i), pvdone & 1u, abort_flag, limit,
+                               kSiteSmxPvDone)))
+            break;
           ++pvdone;
           tc_fence_after();
         }
@@ -681,7 +722,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attn_kernel(const __grid_const
             st_shared_v4(po + (chunk / 8) * kHalf + swz(r, chunk % 8), pk[cc][4 * v4],
                          pk[cc][4 * v4 + 1], pk[cc][4 * v4 + 2], pk[cc][4 * v4 + 3]);
           }
-        if (j > 0 && alpha < 1.0f) {
+        // tcgen05.ld/st are warp-collective: the whole warp rescales if any row needs it
+        if (j > 0 && __any_sync(0xffffffffu, alpha < 1.0f)) {
 #pragma unroll
           for (int cc = 0; cc < D / 32; ++cc) {
             uint32_t o[32];
@@ -698,7 +740,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attn_kernel(const __grid_const
         mbar_arrive(BAR(S::PFULL + i));
       }
       if (!ok) break;
-      if (!(ok = wait_warp(BAR(S::PVDONE + i), pvdone & 1u, abort_flag, limit))) break;
+      if (!(ok = wait_warp(BAR(S::PVDONE + i), pvdone & 1u, abort_flag, limit, kSiteSmxPvLast)))
+        break;
       ++pvdone;
       tc_fence_after();
       // epilogue: O / l -> bf16 -> staging (the P buffer, free now) -> TMA store
@@ -728,7 +771,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attn_kernel(const __grid_const
       fence_proxy_async();
       mbar_arrive(BAR(S::OSTAGED + i));
       if (leader) {
-        const bool staged = wait_bounded(BAR(S::OSTAGED + i), ostaged & 1u, abort_flag, limit);
+        const bool staged =
+            wait_bounded(BAR(S::OSTAGED + i), ostaged & 1u, abort_flag, limit, kSiteSmxOStaged);
         if (staged) {
           store_tile<D>(p, U, qt, po);
           bulk_commit();
@@ -737,7 +781,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attn_kernel(const __grid_const
         mbar_arrive(BAR(S::OFREE + i));
       }
       ++ostaged;
-      if (!(ok = wait_warp(BAR(S::OFREE + i), ofree & 1u, abort_flag, limit))) break;
+      if (!(ok = wait_warp(BAR(S::OFREE + i), ofree & 1u, abort_flag, limit, kSiteSmxOFree)))
+        break;
       ++ofree;
     }
     if (leader) bulk_wait_all0();
@@ -746,7 +791,10 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attn_kernel(const __grid_const
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 1) tmem_dealloc(tmem, 512);
+  if (warp == 1) {
+    __syncwarp();
+    tmem_dealloc(tmem, 512);
+  }
 }
 
 int sm_count() {
@@ -859,8 +907,13 @@ basa_status read_and_clear_status(cudaStream_t stream) {
   unsigned int v = 0;
   if (cudaMemcpyFromSymbol(&v, g_basa_status, sizeof(v)) != cudaSuccess) return BASA_ERR_CUDA;
   if (v) {
+    unsigned int where = 0;
+    cudaMemcpyFromSymbol(&where, g_basa_where, sizeof(where));
+    if (getenv("BASA_DEBUG")) fprintf(stderr, "basa: device wait gave up at site %u\n", where);
     const unsigned int zero = 0;
-    if (cudaMemcpyToSymbol(g_basa_status, &zero, sizeof(zero)) != cudaSuccess) return BASA_ERR_CUDA;
+    if (cudaMemcpyToSymbol(g_basa_status, &zero, sizeof(zero)) != cudaSuccess ||
+        cudaMemcpyToSymbol(g_basa_where, &zero, sizeof(zero)) != cudaSuccess)
+      return BASA_ERR_CUDA;
     return BASA_ERR_TIMEOUT;
   }
   return cudaGetLastError() == cudaSuccess ? BASA_OK : BASA_ERR_CUDA;

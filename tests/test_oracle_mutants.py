@@ -1,0 +1,79 @@
+"""The oracle's pins must catch plausible mistakes.
+
+Each case below plants one mistake in a copy of the C oracle (a textual edit of
+oracle/basa_oracle.c compiled into a temporary library), routes the oracle
+calls to that copy, and runs the pins of test_oracle.py: at least one pin must
+fail.  The real oracle is never modified.
+"""
+import os
+import subprocess
+
+import pytest
+
+import oracle
+from oracle import build as obuild
+from oracle.oracle import use_library
+
+import test_oracle as pins
+
+MUTANTS = {
+    "shift sign on the column axis": ("floor_mod(x - p->sw, p->Wg)", "floor_mod(x + p->sw, p->Wg)"),
+    "dropped softmax scale": ("z[j++] = p->scale * s;", "z[j++] = s;"),
+    "pooled sum not divided": ("xp[o] = acc * inv;", "xp[o] = acc;"),
+    "log-sum-exp without the max": ("*lse_out = mx + log(den);", "*lse_out = log(den);"),
+    "window members without the shift": (
+        "const int64_t xx = floor_mod(ix * p->ww + p->sw + lx, p->Wg);",
+        "const int64_t xx = floor_mod(ix * p->ww + lx, p->Wg);"),
+    "no max subtraction": ("z[i] = exp(z[i] - mx);", "z[i] = exp(z[i]);"),
+    "rows and columns swapped for keys": (
+        "const double* kv = k + tok_index(p, b, tt, yy, xx, h);",
+        "const double* kv = k + tok_index(p, b, tt, xx % p->Hg, yy % p->Wg, h);"),
+    "pooled cells on the shifted origin": (
+        "acc += x[tok_index(p, b, ct * p->pt + i, cy * p->ph + j,\n"
+        "                                       cx * p->pw + l, h) + c];",
+        "acc += x[tok_index(p, b, ct * p->pt + i, (cy * p->ph + j + 1) % p->Hg,\n"
+        "                                       (cx * p->pw + l + 1) % p->Wg, h) + c];"),
+}
+
+
+def _pins():
+    yield pins.test_hand_worked_example, {}
+    for shape, window in [((1, 1, 8, 8, 2, 16), (1, 4, 4)), ((2, 4, 6, 8, 1, 8), (2, 3, 4))]:
+        yield pins.test_shift_zero_is_partitioned_attention, {"shape": shape, "window": window}
+    yield pins.test_window_covering_grid_is_full_attention, {"shape": (2, 3, 4, 5, 3, 8)}
+    for shape, window, pool in pins.TINY:
+        yield pins.test_oracle_matches_brute_force_all_shifts, {"shape": shape, "window": window,
+                                                                "pool": pool}
+    yield pins.test_roll_commutes_with_shift, {"shape": (1, 1, 12, 12, 1, 8), "window": (1, 4, 6),
+                                               "shift": (0, 1, 5)}
+    yield pins.test_zero_queries_give_window_mean, {}
+    yield pins.test_constant_values_give_constant_output, {}
+    yield pins.test_pool_factor_one_and_constant_cells, {}
+    yield pins.test_support_is_exactly_the_window, {}
+    yield pins.test_large_logits_pick_dominant_key, {}
+
+
+def _build_mutant(tmp_path, old, new):
+    src = open(obuild.SRC).read()
+    assert src.count(old) >= 1, f"mutation anchor not found: {old!r}"
+    mutated = src.replace(old, new, 1)
+    c = tmp_path / "mutant.c"
+    c.write_text(mutated)
+    so = tmp_path / "libmutant.so"
+    subprocess.check_call(["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-std=c11",
+                           "-o", str(so), str(c), "-lm"])
+    return str(so)
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_pins_catch_mutant(tmp_path, oracle_mod, name):
+    old, new = MUTANTS[name]
+    so = _build_mutant(tmp_path, old, new)
+    failed = []
+    with use_library(so):
+        for fn, kw in _pins():
+            try:
+                fn(oracle_mod, **kw)
+            except (AssertionError, ValueError, FloatingPointError):
+                failed.append(fn.__name__)
+    assert failed, f"no pin caught the mutant: {name}"
