@@ -82,7 +82,8 @@ typedef enum basa_status {
   BASA_ERR_ALIGN = 4,       /* a pointer is not 16-byte aligned */
   BASA_ERR_WORKSPACE = 5,   /* workspace missing when global memory is requested */
   BASA_ERR_CUDA = 6,        /* CUDA runtime or driver error at launch */
-  BASA_ERR_TIMEOUT = 7      /* a bounded wait inside a kernel ran out */
+  BASA_ERR_TIMEOUT = 7,     /* a bounded wait inside a kernel ran out */
+  BASA_ERR_SCRATCH_LIMIT = 8 /* basa_window_attn_noalloc: pooled K/V exceed its fixed scratch */
 } basa_status;
 
 typedef enum basa_dtype { BASA_F32 = 0, BASA_BF16 = 1 } basa_dtype;
@@ -160,6 +161,35 @@ BASA_API basa_status basa_window_attn_gm(const void* q, const void* k, const voi
  */
 BASA_API basa_status basa_full_attn(const void* q, const void* k, const void* v, void* out,
                            float* lse, const basa_params* p, cudaStream_t stream);
+
+/*
+ * basa_window_attn without any device allocation.  There is no counterpart on
+ * the pages that describe the method; this exists for callers that cannot
+ * allocate device memory, such as an operator inside a host framework that owns
+ * all device memory and gives its operators no workspace, or a latency-critical
+ * serving path that reserves memory at start-up and forbids cudaMalloc/cudaFree
+ * (which can block the host and, for cudaFree, synchronise the device).
+ *
+ * Same operation, arguments and layouts as basa_window_attn, minus the
+ * workspace: the pooled K/V tokens go to a fixed 32 MiB scratch array inside
+ * the library's device code.
+ *  - Every GPU that loads the library's device code holds that array until the
+ *    process exits.
+ *  - If pooled K and V together need more than 32 MiB (each [B, P, H, d] of
+ *    p->dtype, rounded up to 256 bytes), the call returns
+ *    BASA_ERR_SCRATCH_LIMIT and enqueues nothing.
+ *  - The first call with a given device current looks up the array's device
+ *    address (cudaGetSymbolAddress) and caches it; that first call should be
+ *    made before any stream capture begins.
+ *  - All calls on a device share the array: calls whose work overlaps on the
+ *    GPU (e.g. on unordered streams) race on it and must be ordered by the
+ *    caller.  Nothing in it needs to start at zero: each call overwrites every
+ *    byte it reads.
+ *  - The call makes no device or host heap allocation.
+ */
+BASA_API basa_status basa_window_attn_noalloc(const void* q, const void* k, const void* v,
+                                              void* out, float* lse, const basa_params* p,
+                                              cudaStream_t stream);
 
 /*
  * Test and diagnostics only: synchronises `stream`, then reports and clears the

@@ -11,6 +11,7 @@ BASA_OK = 0
 STATUS_NAMES = {
     0: "BASA_OK", 1: "BASA_ERR_INVALID_ARG", 2: "BASA_ERR_SHAPE", 3: "BASA_ERR_UNSUPPORTED",
     4: "BASA_ERR_ALIGN", 5: "BASA_ERR_WORKSPACE", 6: "BASA_ERR_CUDA", 7: "BASA_ERR_TIMEOUT",
+    8: "BASA_ERR_SCRATCH_LIMIT",
 }
 BASA_F32, BASA_BF16 = 0, 1
 BASA_FLAG_TEST_WITHHOLD_LOADS = 0x1
@@ -18,7 +19,7 @@ BASA_FLAG_TEST_WITHHOLD_LOADS = 0x1
 # Every symbol include/basa.h declares.
 EXPORTS = ("basa_status_string", "basa_version", "basa_workspace_size", "basa_pool_kv",
            "basa_window_attn", "basa_window_attn_gm", "basa_full_attn", "basa_get_status",
-           "basa_window_tiles")
+           "basa_window_tiles", "basa_window_attn_noalloc")
 
 
 class BasaParams(ctypes.Structure):
@@ -70,6 +71,8 @@ def load():
                                       ctypes.POINTER(ctypes.c_int32),
                                       ctypes.POINTER(ctypes.c_int32), ctypes.c_int64]
     lib.basa_window_tiles.restype = ctypes.c_int
+    lib.basa_window_attn_noalloc.argtypes = [vp, vp, vp, vp, vp, P, vp]
+    lib.basa_window_attn_noalloc.restype = ctypes.c_int
     _lib = lib
     return lib
 

@@ -188,6 +188,7 @@ const char* basa_status_string(basa_status s) {
     case BASA_ERR_WORKSPACE: return "workspace missing";
     case BASA_ERR_CUDA: return "CUDA error";
     case BASA_ERR_TIMEOUT: return "device wait timed out";
+    case BASA_ERR_SCRATCH_LIMIT: return "pooled K/V exceed the fixed no-alloc scratch";
   }
   return "unknown status";
 }

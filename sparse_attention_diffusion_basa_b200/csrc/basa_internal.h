@@ -94,6 +94,13 @@ basa_status launch_tc(const Dims& d, bool flat, const void* q, const void* k, co
                       const void* kp, const void* vp, void* out, float* lse, uint32_t flags,
                       uint32_t timeout_ms, cudaStream_t stream);
 
+// The same launch with its parameter block in static storage (no host heap use);
+// calls are serialised by a lock held until the launch has copied the block.
+basa_status launch_tc_static_params(const Dims& d, bool flat, const void* q, const void* k,
+                                    const void* v, const void* kp, const void* vp, void* out,
+                                    float* lse, uint32_t flags, uint32_t timeout_ms,
+                                    cudaStream_t stream);
+
 // Device status word helpers (basa_tc.cu).
 basa_status read_and_clear_status(cudaStream_t stream);
 

@@ -36,6 +36,7 @@
 #include <stdlib.h>
 #include <string.h>
 
+#include <mutex>
 #include <new>
 
 #include "basa_internal.h"
@@ -819,12 +820,13 @@ basa_status launch_impl(TcParams* prm, cudaStream_t stream) {
 
 }  // namespace
 
-basa_status launch_tc(const Dims& d, bool flat, const void* q, const void* k, const void* v,
-                      const void* kp, const void* vp, void* out, float* lse, uint32_t flags,
-                      uint32_t timeout_ms, cudaStream_t stream) {
-  TcParams* prm = new (std::nothrow) TcParams;
-  if (!prm) return BASA_ERR_INVALID_ARG;
-  memset(prm, 0, sizeof(*prm));
+namespace {
+
+// Fills *prm (zeroed by the caller) for one call and launches the kernel.
+basa_status build_and_launch(TcParams* prm, const Dims& d, bool flat, const void* q,
+                             const void* k, const void* v, const void* kp, const void* vp,
+                             void* out, float* lse, uint32_t flags, uint32_t timeout_ms,
+                             cudaStream_t stream) {
   basa_status st = BASA_OK;
   const uint64_t D = (uint64_t)d.d;
   const uint64_t H = (uint64_t)d.H;
@@ -898,8 +900,36 @@ basa_status launch_tc(const Dims& d, bool flat, const void* q, const void* k, co
   }
   st = d.d == 128 ? launch_impl<128>(prm, stream) : launch_impl<64>(prm, stream);
 done:
+  return st;
+}
+
+// Parameter block of the entry points that allocate nothing: one static block,
+// used under a lock (the launch copies it, so it is free again on return).
+TcParams g_static_params;
+std::mutex g_static_params_mu;
+
+}  // namespace
+
+basa_status launch_tc(const Dims& d, bool flat, const void* q, const void* k, const void* v,
+                      const void* kp, const void* vp, void* out, float* lse, uint32_t flags,
+                      uint32_t timeout_ms, cudaStream_t stream) {
+  TcParams* prm = new (std::nothrow) TcParams;
+  if (!prm) return BASA_ERR_INVALID_ARG;
+  memset(prm, 0, sizeof(*prm));
+  const basa_status st =
+      build_and_launch(prm, d, flat, q, k, v, kp, vp, out, lse, flags, timeout_ms, stream);
   delete prm;
   return st;
+}
+
+basa_status launch_tc_static_params(const Dims& d, bool flat, const void* q, const void* k,
+                                    const void* v, const void* kp, const void* vp, void* out,
+                                    float* lse, uint32_t flags, uint32_t timeout_ms,
+                                    cudaStream_t stream) {
+  std::lock_guard<std::mutex> lock(g_static_params_mu);
+  memset(&g_static_params, 0, sizeof(g_static_params));
+  return build_and_launch(&g_static_params, d, flat, q, k, v, kp, vp, out, lse, flags,
+                          timeout_ms, stream);
 }
 
 basa_status read_and_clear_status(cudaStream_t stream) {

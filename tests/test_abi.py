@@ -32,7 +32,7 @@ def test_exports_every_declared_symbol(lib):
     for name in declared:
         assert hasattr(lib, name), name
     assert lib.basa_version() >= 100
-    for code in range(8):
+    for code in range(9):
         assert lib.basa_status_string(code)
 
 
@@ -80,6 +80,18 @@ def test_validation_codes(lib):
     assert lib.basa_pool_kv(_fake(), _fake(), _fake(0x10004), _fake(),
                             ctypes.byref(_p(pool=(1, 2, 2))), None) == 4
     assert _lib.STATUS_NAMES[4] == "BASA_ERR_ALIGN"
+
+
+def test_noalloc_refuses_problems_beyond_its_scratch(lib):
+    # pooled K + V of 2 x [B, P, H, d] bf16 = 2 x 4 x 1024 x 24 x 128 x 2 bytes > 32 MiB
+    prm = _p(shape=(4, 1, 128, 128, 24, 128), window=(1, 16, 16), shift=(0, 8, 8),
+             pool=(1, 4, 4))
+    assert lib.basa_window_attn_noalloc(_fake(), _fake(), _fake(), _fake(), None,
+                                        ctypes.byref(prm), None) == 8
+    assert lib.basa_status_string(8)
+    # validation runs first, exactly as for basa_window_attn
+    assert lib.basa_window_attn_noalloc(_fake(0x10008), _fake(), _fake(), _fake(), None,
+                                        ctypes.byref(_p(pool=(1, 2, 2))), None) == 4
 
 
 def test_workspace_size(lib):
