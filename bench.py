@@ -29,7 +29,6 @@ import hashlib
 import json
 import math
 import os
-import subprocess
 import sys
 import time
 
@@ -87,59 +86,59 @@ def workload_numbers(w, shift):
 
 
 class ClockSampler:
-    """nvidia-smi clock / throttle sampling during the timed region."""
+    """SM clock and throttle-reason sampling (NVML, every ~2 ms) during the timed region."""
 
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = {  # NVML clocks-event-reason bits
+        0x8: "hw_slowdown", 0x40: "hw_thermal_slowdown", 0x20: "sw_thermal_slowdown",
+        0x4: "sw_power_cap",
+    }
 
     def __init__(self, device_index):
         self.dev = device_index
-        self.proc = None
-        self.path = os.path.join("/tmp", f"basa_clocks_{os.getpid()}.csv")
+        self.samples = []
+        self._stop = None
+        self._thread = None
 
     def start(self):
+        import threading
         try:
-            self.f = open(self.path, "w")
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", str(self.dev), f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "100"],
-                stdout=self.f, stderr=subprocess.DEVNULL)
+            import pynvml
+            pynvml.nvmlInit()
+            # NVML numbers devices as the driver does; honour CUDA_VISIBLE_DEVICES
+            vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+            idx = int(vis.split(",")[self.dev]) if vis else self.dev
+            h = pynvml.nvmlDeviceGetHandleByIndex(idx)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
         except Exception:
-            self.proc = None
+            return
+        self._stop = threading.Event()
+
+        def run():
+            while not self._stop.is_set():
+                try:
+                    mhz = pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM)
+                    rs = pynvml.nvmlDeviceGetCurrentClocksEventReasons(h)
+                    self.samples.append((mhz, rs))
+                except Exception:
+                    pass
+                self._stop.wait(0.002)
+
+        self._thread = threading.Thread(target=run, daemon=True)
+        self._thread.start()
 
     def stop(self):
-        if self.proc is None:
+        if self._thread is None:
             return None
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except Exception:
-            self.proc.kill()
-        self.f.close()
-        rows = []
-        for line in open(self.path):
-            parts = [x.strip() for x in line.split(",")]
-            if len(parts) < 9:
-                continue
-            try:
-                rows.append(parts)
-            except Exception:
-                pass
-        os.unlink(self.path)
-        if not rows:
+        self._stop.set()
+        self._thread.join(timeout=5)
+        if not self.samples:
             return None
-        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
-        smax = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = set()
-        for r in rows:
-            for n, val in zip(names, r[5:9]):
-                if val.lower() == "active":
-                    reasons.add(n)
-        return {"sm_mhz": float(np.median(sm)) if sm else None,
-                "sm_max_mhz": max(smax) if smax else None,
-                "reasons": sorted(reasons), "samples": len(rows)}
+        mhz = [m for m, _ in self.samples]
+        reasons = sorted({name for _, rs in self.samples for bit, name in self.REASONS.items()
+                          if rs & bit})
+        return {"sm_mhz": float(np.median(mhz)), "sm_min_mhz": float(min(mhz)),
+                "sm_max_mhz": float(self.max_mhz), "reasons": reasons,
+                "samples": len(self.samples), "source": "nvml"}
 
 
 def _sleep_cycles(us):
@@ -322,6 +321,18 @@ def main():
     ms = sum(t_steps) / len(t_steps)
     ms_max = max_over_ranks(ms, world)
 
+    # the step's kernels on their own: pooling into the workspace, then the
+    # attention kernel on the pooled tokens (only for workloads with global memory)
+    ms_attn, ms_pool = ms_max, 0.0
+    if w.P:
+        kpt, vpt = basa.pool_kv(dk, dv, w.pool)
+        t_pool = time_steps(lambda: basa.pool_kv(dk, dv, w.pool, out=(kpt, vpt)), args.steps,
+                            flush)
+        t_attn = time_steps(lambda: basa.window_attn_gm(dq, dk, dv, kpt, vpt, w.window, shift,
+                                                        w.pool, out=out), args.steps, flush)
+        ms_pool = max_over_ranks(sum(t_pool) / len(t_pool), world)
+        ms_attn = max_over_ranks(sum(t_attn) / len(t_attn), world)
+
     # full attention on the same inputs: the speedup denominator
     t_full = time_steps(step_full, args.full_steps, flush)
     ms_full = max_over_ranks(sum(t_full) / len(t_full), world)
@@ -343,17 +354,19 @@ def main():
     peaks = _peaks()
     tflops = world * flops / (ms_max * 1e-3) / 1e12
     per_gpu_tflops = flops / (ms_max * 1e-3) / 1e12
-    gbs = bytes_ / (ms_max * 1e-3) / 1e9
+    attn_tflops = flops / (ms_attn * 1e-3) / 1e12   # the attention kernel alone
+    gbs = bytes_ / (ms_attn * 1e-3) / 1e9
     theo = N / (m + P)
     if m + P >= 2 * 254:   # intensity (m+P)/2 flop per byte above the ridge
-        roof = {"bound": "tensor", "achieved": per_gpu_tflops, "peak": peaks["bf16_tflops"],
-                "unit": "TFLOP/s", "frac": per_gpu_tflops / peaks["bf16_tflops"]}
+        roof = {"bound": "tensor", "achieved": attn_tflops, "peak": peaks["bf16_tflops"],
+                "unit": "TFLOP/s", "frac": attn_tflops / peaks["bf16_tflops"]}
     else:
         roof = {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "frac": gbs / peaks["hbm_gbs"]}
     roof["peak_source"] = peaks["source"]
     roof["traffic"] = _traffic("tc_attn_kernel", w.name)
     roof["kernel"] = "tc_attn_kernel"
+    roof["kernel_ms"] = ms_attn
 
     line = {
         "metric": METRIC, "value": tflops, "unit": "TFLOP/s", "n_gpus": world,
@@ -377,6 +390,7 @@ def main():
                 "ms_per_step": e2e,
                 "h2d_bytes_per_step": 3 * dq.numel() * dq.element_size(),
                 "d2h_bytes_per_step": out.numel() * out.element_size()},
+        "kernels_ms": {"tc_attn_kernel": ms_attn, "pool_kernel": ms_pool},
         "gpu_launches": args.steps * (2 if w.P else 1),
         "clocks": clk,
     }

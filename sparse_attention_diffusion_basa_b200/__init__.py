@@ -76,15 +76,24 @@ def workspace_size(shape, dtype, window, shift=(0, 0, 0), pool=(0, 0, 0)) -> int
         ctypes.byref(make_params(shape, dtype, window, shift, pool))))
 
 
-def pool_kv(k: torch.Tensor, v: torch.Tensor, pool, stream=None):
-    """Mean-pool K and V over pt x ph x pw cells -> (kp, vp) [B, T/pt, Hg/ph, Wg/pw, H, d]."""
+def pool_kv(k: torch.Tensor, v: torch.Tensor, pool, out=None, stream=None):
+    """Mean-pool K and V over pt x ph x pw cells -> (kp, vp) [B, T/pt, Hg/ph, Wg/pw, H, d].
+
+    ``out`` may give the (kp, vp) tensors to write into."""
     _check_inputs(k, v)
     B, T, Hg, Wg, H, d = k.shape
     pt, ph, pw = _triple(pool, "pool")
     if min(pt, ph, pw) <= 0 or T % pt or Hg % ph or Wg % pw:
         raise ValueError(f"pool {pool} must be positive and divide the grid {(T, Hg, Wg)}")
-    kp = torch.empty((B, T // pt, Hg // ph, Wg // pw, H, d), dtype=k.dtype, device=k.device)
-    vp = torch.empty_like(kp)
+    shape = (B, T // pt, Hg // ph, Wg // pw, H, d)
+    if out is None:
+        kp = torch.empty(shape, dtype=k.dtype, device=k.device)
+        vp = torch.empty_like(kp)
+    else:
+        kp, vp = out
+        _check_inputs(k, kp, vp)
+        if tuple(kp.shape) != shape or tuple(vp.shape) != shape:
+            raise ValueError(f"pooled outputs must have shape {shape}")
     prm = make_params(k.shape, k.dtype, (1, 1, 1), (0, 0, 0), (pt, ph, pw))
     lib = _lib.load()
     with torch.cuda.device(k.device):

@@ -280,6 +280,12 @@ basa_status basa_full_attn(const void* q, const void* k, const void* v, void* ou
   return attn_common(d, q, k, v, nullptr, nullptr, out, lse, p, stream, true);
 }
 
+basa_status basa_test_exp2(const float* x, float* y, int64_t n, cudaStream_t stream) {
+  if (n < 0 || (n > 0 && (!x || !y))) return BASA_ERR_INVALID_ARG;
+  if (n > (1LL << 40)) return BASA_ERR_UNSUPPORTED;
+  return launch_ex2_poly_test(x, y, (long long)n, stream);
+}
+
 basa_status basa_get_status(cudaStream_t stream) {
   return read_and_clear_status(stream);
 }

@@ -101,6 +101,9 @@ basa_status launch_tc_static_params(const Dims& d, bool flat, const void* q, con
                                     float* lse, uint32_t flags, uint32_t timeout_ms,
                                     cudaStream_t stream);
 
+// Test hook: y = the kernels' polynomial 2^x (device pointers, n floats).
+basa_status launch_ex2_poly_test(const float* x, float* y, long long n, cudaStream_t stream);
+
 // Device status word helpers (basa_tc.cu).
 basa_status read_and_clear_status(cudaStream_t stream);
 

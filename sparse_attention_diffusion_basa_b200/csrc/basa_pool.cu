@@ -4,10 +4,12 @@
 // origin; each pooled token is the plain mean of its cell's tokens.
 //
 // HBM-bound: every input byte is read once, every output byte written once.
-// One CTA per (pooled cell, batch); each thread owns one 16-byte vector of the
-// cell's H*d values and walks the cell's pt*ph*pw tokens with 16-byte loads
-// (consecutive threads read consecutive 16-byte pieces of a token's H*d row, so
-// every warp load is fully coalesced), accumulating in fp32.
+// A CTA of 128 threads owns 128 consecutive 16-byte vectors of one pooled
+// cell's H*d row (a cell's row splits over ceil(H*d*esize/2048) CTAs).  Each
+// thread walks the cell's pt*ph*pw tokens eight at a time, issuing all sixteen
+// 16-byte K and V loads of a batch before accumulating them in fp32, so that
+// enough loads are in flight to cover HBM latency.  Consecutive threads read
+// consecutive 16-byte pieces of a token row, so every warp load is coalesced.
 #include <cuda_bf16.h>
 
 #include "basa_internal.h"
@@ -23,6 +25,8 @@ struct PoolArgs {
   int T, Hg, Wg, pt, ph, pw;
   int Pt, Ph, Pw;
   int vec_per_token;  // 16-byte vectors per token row of H*d values
+  int vec_blocks;     // CTAs per pooled cell
+  int P;              // pooled cells per batch
   float inv_count;
 };
 
@@ -44,55 +48,68 @@ __device__ __forceinline__ uint4 pack_bf16(const float* a, float s) {
   return r;
 }
 
+constexpr int kPoolThreads = 128;
+constexpr int kPoolBatch = 8;  // tokens whose loads are issued together
+
 template <bool kBf16>
-__global__ void __launch_bounds__(512) pool_kernel(PoolArgs a) {
-  const int cell = blockIdx.x;  // flattened (ct, cy, cx)
+__global__ void __launch_bounds__(kPoolThreads) pool_kernel(PoolArgs a) {
+  const int cell = blockIdx.x / a.vec_blocks;  // flattened (ct, cy, cx)
+  const int vi = (blockIdx.x % a.vec_blocks) * kPoolThreads + threadIdx.x;
   const int b = blockIdx.y;
+  if (vi >= a.vec_per_token) return;
   const int cx = cell % a.Pw, cy = (cell / a.Pw) % a.Ph, ct = cell / (a.Pw * a.Ph);
   constexpr int E = kBf16 ? 8 : 4;  // elements per 16-byte vector
-  for (int vi = threadIdx.x; vi < a.vec_per_token; vi += blockDim.x) {
-    float ak[E], av[E];
+  const int ncell = a.pt * a.ph * a.pw;
+  float ak[E], av[E];
 #pragma unroll
-    for (int i = 0; i < E; ++i) ak[i] = av[i] = 0.f;
-    for (int i = 0; i < a.pt; ++i)
-      for (int j = 0; j < a.ph; ++j) {
+  for (int i = 0; i < E; ++i) ak[i] = av[i] = 0.f;
+  for (int i0 = 0; i0 < ncell; i0 += kPoolBatch) {
+    uint4 xk[kPoolBatch], xv[kPoolBatch];
+#pragma unroll
+    for (int u = 0; u < kPoolBatch; ++u) {
+      const int i = i0 + u;
+      if (i < ncell) {
+        const int it = i / (a.ph * a.pw), ih = (i / a.pw) % a.ph, iw = i % a.pw;
         const long long row =
-            (((long long)b * a.T + ct * a.pt + i) * a.Hg + cy * a.ph + j) * a.Wg + cx * a.pw;
-#pragma unroll 4
-        for (int l = 0; l < a.pw; ++l) {
-          const long long off = (row + l) * a.vec_per_token + vi;
-          const uint4 xk = __ldcs(a.k + off);
-          const uint4 xv = __ldcs(a.v + off);
-          if (kBf16) {
-            acc_bf16(ak, xk);
-            acc_bf16(av, xv);
-          } else {
-            const float* fk = reinterpret_cast<const float*>(&xk);
-            const float* fv = reinterpret_cast<const float*>(&xv);
+            (((long long)b * a.T + ct * a.pt + it) * a.Hg + cy * a.ph + ih) * a.Wg + cx * a.pw + iw;
+        const long long off = row * a.vec_per_token + vi;
+        xk[u] = __ldcs(a.k + off);
+        xv[u] = __ldcs(a.v + off);
+      }
+    }
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              ak[e] += fk[e];
-              av[e] += fv[e];
-            }
+    for (int u = 0; u < kPoolBatch; ++u) {
+      if (i0 + u < ncell) {
+        if (kBf16) {
+          acc_bf16(ak, xk[u]);
+          acc_bf16(av, xv[u]);
+        } else {
+          const float* fk = reinterpret_cast<const float*>(&xk[u]);
+          const float* fv = reinterpret_cast<const float*>(&xv[u]);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            ak[e] += fk[e];
+            av[e] += fv[e];
           }
         }
       }
-    const long long o = ((long long)b * gridDim.x + cell) * a.vec_per_token + vi;
-    if (kBf16) {
-      a.kp[o] = pack_bf16(ak, a.inv_count);
-      a.vp[o] = pack_bf16(av, a.inv_count);
-    } else {
-      uint4 rk, rv;
-      float* fk = reinterpret_cast<float*>(&rk);
-      float* fv = reinterpret_cast<float*>(&rv);
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        fk[e] = ak[e] * a.inv_count;
-        fv[e] = av[e] * a.inv_count;
-      }
-      a.kp[o] = rk;
-      a.vp[o] = rv;
     }
+  }
+  const long long o = ((long long)b * a.P + cell) * a.vec_per_token + vi;
+  if (kBf16) {
+    a.kp[o] = pack_bf16(ak, a.inv_count);
+    a.vp[o] = pack_bf16(av, a.inv_count);
+  } else {
+    uint4 rk, rv;
+    float* fk = reinterpret_cast<float*>(&rk);
+    float* fv = reinterpret_cast<float*>(&rv);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      fk[e] = ak[e] * a.inv_count;
+      fv[e] = av[e] * a.inv_count;
+    }
+    a.kp[o] = rk;
+    a.vp[o] = rv;
   }
 }
 
@@ -111,13 +128,14 @@ basa_status launch_pool(const Dims& d, const void* k, const void* v, void* kp, v
   const int es = d.dtype == BASA_BF16 ? 2 : 4;
   a.vec_per_token = d.H * d.d * es / 16;
   a.inv_count = 1.0f / (float)(d.pt * d.ph * d.pw);
-  if (d.P > 0x7fffffffLL || d.B > 65535) return BASA_ERR_UNSUPPORTED;
-  dim3 grid((unsigned)d.P, (unsigned)d.B);
-  int threads = a.vec_per_token < 512 ? ((a.vec_per_token + 31) / 32) * 32 : 512;
+  a.vec_blocks = (a.vec_per_token + kPoolThreads - 1) / kPoolThreads;
+  a.P = (int)d.P;
+  if (d.P * a.vec_blocks > 0x7fffffffLL || d.B > 65535) return BASA_ERR_UNSUPPORTED;
+  dim3 grid((unsigned)(d.P * a.vec_blocks), (unsigned)d.B);
   if (d.dtype == BASA_BF16)
-    pool_kernel<true><<<grid, threads, 0, stream>>>(a);
+    pool_kernel<true><<<grid, kPoolThreads, 0, stream>>>(a);
   else
-    pool_kernel<false><<<grid, threads, 0, stream>>>(a);
+    pool_kernel<false><<<grid, kPoolThreads, 0, stream>>>(a);
   return cudaGetLastError() == cudaSuccess ? BASA_OK : BASA_ERR_CUDA;
 }
 

@@ -10,22 +10,23 @@
 // grid, each query tile against every key tile.
 //
 // Work unit: (b, h, window, pair of 128-query tiles).  Persistent CTAs (one
-// per SM) walk the units.  Inside a CTA the warps specialise:
-//   warp 0        TMA loader: Q tiles, then K and V tiles of the unit through a
-//                 3-slot ring (boxes from the shifted-window tile plan; a tile
-//                 that crosses a wrapped border is fetched as up to 8 boxes,
-//                 so no rolled copy of the grid is ever made);
+// per SM) walk the units, heads fastest.  Inside a CTA the warps specialise:
+//   warp 0        TMA loader: the two query tiles of each unit, then its K and V
+//                 tiles through a 3-slot ring (boxes from the shifted-window
+//                 tile plan; a tile that crosses a wrapped border is fetched as
+//                 up to 8 boxes, so no rolled copy of the grid is ever made);
 //   warp 1        owns TMEM (512 columns) and issues the MMAs from one thread:
-//                 S_i = Q_i K_j^T into TMEM, then O_i += P_i V_j into TMEM;
+//                 S_i = Q_i K_j^T into TMEM (the next key tile's logits while the
+//                 softmax works on the current ones), then O_i += P_i V_j;
 //   warps 4..7    softmax + epilogue for query tile 0 of the unit,
 //   warps 8..11   the same for query tile 1.
 // Each softmax thread owns one query row: it reads its 128 logits from TMEM,
 // keeps the running max and sum in fp32 (base-2 exponentials with the scale
 // folded in), writes the bf16 probabilities P to shared memory in the
 // 128-byte-swizzled K-major layout the MMA reads, and rescales its O row in
-// TMEM when the max grows.  The epilogue divides by the sum, rounds to bf16,
-// stages the tile in shared memory and stores it with TMA boxes that mirror
-// the load boxes.
+// TMEM when the max grows by more than 2^8.  The epilogue divides by the sum,
+// rounds to bf16, stages the tile in the P buffer and stores it with TMA boxes
+// that mirror the load boxes.
 //
 // Every mbarrier wait is bounded (wall-clock limit from the call); on expiry the
 // kernel raises the device status word, lets every role leave its loop, waits
@@ -50,6 +51,8 @@ namespace {
 
 constexpr int kThreads = 384;
 constexpr int kHalf = 128 * 128;  // bytes of one 64-wide head-dim half of a 128-row tile
+constexpr int kPlanBytes = 1536;  // shared-memory room for the compact tile plan
+constexpr int kPlanWords = kPlanBytes / 4;
 
 struct __align__(64) TcParams {
   CUtensorMap qm[kMaxShapes];  // window boxes, rank 5: [d, H, Wg, Hg, B*T]
@@ -59,17 +62,18 @@ struct __align__(64) TcParams {
   CUtensorMap qf, kf, vf, of;  // flat 128-row tiles, rank 4: [d, H, N, B]
   CUtensorMap kpf, vpf;        // pooled 128-row tiles, rank 4: [d, H, P, B]
   CUtensorMap fill;            // 8-row box over k's flat view, read out of bounds = zeros
-  uint32_t box[kClasses][kMaxTiles][kMaxBoxes];
-  uint8_t nbox[kClasses][kMaxTiles];
-  uint8_t tile_rows[kMaxTiles];
-  uint8_t shape_bt[kMaxShapes], shape_bh[kMaxShapes], shape_bw[kMaxShapes];
+  uint32_t plan[kPlanWords];  // compact tile plan image, copied to shared memory at start
+  int plan_words;
+  int plan_off_rows, plan_off_bt, plan_off_bh, plan_off_bw, plan_off_entries;  // bytes
   float* lse;
-  long long n_units;
+  __nv_bfloat16* out;  // [B, T, Hg, Wg, H, d]
+  uint32_t n_units;
   long long N;
   unsigned long long timeout_ns;
   int B, H, T, Hg, Wg;
   int wt, wh, ww, st, sh, sw, nwt, nwh, nww;
   int n_windows;
+  int n_shapes;
   int n_qt;   // query tiles per window (flat: per (b, h))
   int n_pairs;
   int n_wkt;  // key tiles from the window (flat: from the grid)
@@ -85,11 +89,6 @@ struct __align__(64) TcParams {
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-__device__ __forceinline__ uint64_t globaltimer() {
-  uint64_t t;
-  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-  return t;
 }
 __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
@@ -157,6 +156,9 @@ __device__ __forceinline__ void tma_store_4d(const CUtensorMap* map, uint32_t sr
       "r"(src), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
       : "memory");
 }
+__device__ __forceinline__ void prefetch_tmap(const CUtensorMap* map) {
+  asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
 __device__ __forceinline__ void bulk_commit() {
   asm volatile("cp.async.bulk.commit_group;" ::: "memory");
 }
@@ -200,6 +202,17 @@ __device__ __forceinline__ void mma_bf16(uint32_t tmem_d, uint64_t a, uint64_t b
       "setp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
       "l"(a), "l"(b), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// The same with the A operand (M x K, K-major) read from TMEM: two 16-bit
+// elements per 32-bit column, lower half first.
+__device__ __forceinline__ void mma_bf16_ts(uint32_t tmem_d, uint32_t tmem_a, uint64_t b,
+                                            uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(tmem_d),
+      "r"(tmem_a), "l"(b), "r"(idesc), "r"(accumulate)
       : "memory");
 }
 __device__ __forceinline__ void mma_commit(uint32_t bar) {
@@ -263,6 +276,81 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&h);
 }
+// Packed pairs of fp32 (f32x2 arithmetic of sm_100).
+__device__ __forceinline__ uint64_t f2pack(float lo, float hi) {
+  uint64_t d;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(d) : "f"(lo), "f"(hi));
+  return d;
+}
+__device__ __forceinline__ void f2unpack(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t f2add(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ uint64_t f2mul(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// 2^x for a pair of x <= 0, computed on the FMA and integer pipes so that part
+// of the softmax's exponentials bypass the MUFU unit (its throughput limit).
+// Method: round-to-nearest argument reduction x = j + f, |f| <= 1/2, through the
+// float constant 1.5 * 2^23 (after the addition its low mantissa bits hold j;
+// the additive reduction of Cody and Waite), a cubic fit of 2^f on [-1/2, 1/2]
+// minimising the maximum relative error (Remez exchange, fitted for this
+// library: 7.5e-5 worst case in fp32 Horner evaluation), then the scale by 2^j
+// applied by adding j to the exponent field (Schraudolph, "A fast, compact
+// approximation of the exponential function", 1999).  x is clamped at -125 so
+// the exponent field cannot underflow; results there are below 2^-124.
+constexpr float kEx2C0 = 0x1.fff692p-1f;
+constexpr float kEx2C1 = 0x1.62f31ap-1f;
+constexpr float kEx2C2 = 0x1.f0de1ap-3f;
+constexpr float kEx2C3 = 0x1.c3f76p-5f;
+__device__ __forceinline__ uint64_t ex2_poly_x2(uint64_t x2) {
+  float x0, x1;
+  f2unpack(x2, x0, x1);
+  x0 = fmaxf(x0, -125.0f);
+  x1 = fmaxf(x1, -125.0f);
+  const uint64_t t = f2add(f2pack(x0, x1), f2pack(12582912.0f, 12582912.0f));
+  const uint64_t j = f2add(t, f2pack(-12582912.0f, -12582912.0f));
+  const uint64_t f = f2fma(j, f2pack(-1.0f, -1.0f), f2pack(x0, x1));
+  uint64_t q = f2fma(f, f2pack(kEx2C3, kEx2C3), f2pack(kEx2C2, kEx2C2));
+  q = f2fma(q, f, f2pack(kEx2C1, kEx2C1));
+  q = f2fma(q, f, f2pack(kEx2C0, kEx2C0));
+  float q0, q1, t0, t1;
+  f2unpack(q, q0, q1);
+  f2unpack(t, t0, t1);
+  return f2pack(__int_as_float(__float_as_int(q0) + (__float_as_int(t0) << 23)),
+                __int_as_float(__float_as_int(q1) + (__float_as_int(t1) << 23)));
+}
+
+// Which exponential pairs go to the polynomial: pair e of every 16 when
+// e % kEx2Period == kEx2Period - 1 (period 3: 5 of 16 pairs); 0 = none.
+#ifndef BASA_DIRECT_STORE
+#define BASA_DIRECT_STORE 0
+#endif
+#ifndef BASA_EX2_PERIOD
+#define BASA_EX2_PERIOD 0
+#endif
+constexpr int kEx2Period = BASA_EX2_PERIOD;
+// Rescale O only when a tile's row max exceeds the reference max by more than
+// 2^kLazyRescale; until then the stale reference is kept (P stays <= 2^8).
+constexpr float kLazyRescale = 8.0f;
+
 __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
                                              uint32_t d) {
   asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c),
@@ -277,9 +365,11 @@ __device__ __forceinline__ uint32_t swz(int row, int chunk) {
 
 // ---------------------------------------------------------------------------
 // Bounded waits.  `abort_flag` lives in shared memory; any role that gives up
-// raises it so that the others leave their loops promptly.  A wait is bounded
-// both by the global nanosecond timer and by SM cycles (at most 2 per ns), and
-// the first wait that gives up records its site in g_basa_where.
+// raises it so that the others leave their loops promptly.  The poll loop is
+// tight (try_wait itself sleeps until the phase completes or a short hardware
+// limit passes); the abort flag and the bound, in SM cycles (2 per ns of the
+// limit, so at least the limit at clocks up to 2 GHz), are checked every 64
+// polls.  The first wait that gives up records its site in g_basa_where.
 // ---------------------------------------------------------------------------
 enum WaitSite : uint32_t {
   kSiteLoadKvEmpty = 1, kSiteLoadQEmpty, kSiteLoadDrainKv, kSiteLoadDrainQ, kSiteMmaQFull,
@@ -291,17 +381,18 @@ __device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity,
                                              volatile uint32_t* abort_flag, uint64_t limit_ns,
                                              uint32_t site, bool honour_abort = true) {
   if (mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = globaltimer();
   const long long c0 = clock64();
   const long long climit = (long long)(limit_ns * 2ull);
-  while (true) {
+  for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
-    if (honour_abort && *abort_flag) return false;
-    if (globaltimer() - t0 > limit_ns || clock64() - c0 > climit) {
-      *abort_flag = 1u;
-      atomicCAS(&g_basa_where, 0u, site);
-      atomicOr(&g_basa_status, 1u);
-      return false;
+    if ((it & 63u) == 0u) {
+      if (honour_abort && *abort_flag) return false;
+      if (clock64() - c0 > climit) {
+        *abort_flag = 1u;
+        atomicCAS(&g_basa_where, 0u, site);
+        atomicOr(&g_basa_status, 1u);
+        return false;
+      }
     }
   }
 }
@@ -320,52 +411,75 @@ struct Unit {
   int b, h, pair, cls, ot, oh, ow, nq;
 };
 
-__device__ __forceinline__ Unit decode_unit(const TcParams& p, long long u) {
+// Window mode walks the heads fastest: concurrently running CTAs then read the
+// same tokens for all heads, so each token's H*d row (a few DRAM pages) is
+// fetched as a whole.  Full-attention mode walks the query-tile pairs fastest,
+// so the CTAs in flight share one (b, h)'s K and V through L2.
+__device__ __forceinline__ Unit decode_unit(const TcParams& p, uint32_t u) {
   Unit U;
-  U.pair = (int)(u % p.n_pairs);
-  long long r = u / p.n_pairs;
   if (p.flat) {
+    U.pair = (int)(u % (uint32_t)p.n_pairs);
+    const uint32_t r = u / (uint32_t)p.n_pairs;
+    U.h = (int)(r % (uint32_t)p.H);
+    U.b = (int)(r / (uint32_t)p.H);
     U.cls = 0;
     U.ot = U.oh = U.ow = 0;
   } else {
-    const int win = (int)(r % p.n_windows);
-    r /= p.n_windows;
+    U.h = (int)(u % (uint32_t)p.H);
+    uint32_t r = u / (uint32_t)p.H;
+    U.pair = (int)(r % (uint32_t)p.n_pairs);
+    r /= (uint32_t)p.n_pairs;
+    const int win = (int)(r % (uint32_t)p.n_windows);
+    U.b = (int)(r / (uint32_t)p.n_windows);
     const int jw = win % p.nww, jh = (win / p.nww) % p.nwh, jt = win / (p.nww * p.nwh);
     U.cls = window_class(jt, jh, jw, p.nwt, p.nwh, p.nww, p.st, p.sh, p.sw);
     U.ot = jt * p.wt + p.st;
     U.oh = jh * p.wh + p.sh;
     U.ow = jw * p.ww + p.sw;
   }
-  U.h = (int)(r % p.H);
-  U.b = (int)(r / p.H);
   const int left = p.n_qt - 2 * U.pair;
   U.nq = left < 2 ? left : 2;
   return U;
 }
 
+// The tile plan as seen from shared memory.  Image layout (bytes): per (class,
+// tile) a 16-bit word (first box << 4 | box count); per tile its valid rows;
+// per box shape its t, row and column extents; then the packed box entries.
+struct PlanView {
+  const uint16_t* idx;
+  const uint8_t* rows;
+  const uint8_t* bt;
+  const uint8_t* bh;
+  const uint8_t* bw;
+  const uint32_t* entries;
+  int n_tiles;
+  __device__ __forceinline__ int first(int cls, int tile) const { return idx[cls * n_tiles + tile] >> 4; }
+  __device__ __forceinline__ int count(int cls, int tile) const { return idx[cls * n_tiles + tile] & 15; }
+};
+
 // Valid rows of key tile j (rows past them are zero-filled and masked).
-__device__ __forceinline__ int key_valid(const TcParams& p, int j) {
+__device__ __forceinline__ int key_valid(const TcParams& p, const PlanView& pv, int j) {
   if (p.flat) {
     const long long left = p.N - 128LL * j;
     return left < 128 ? (int)left : 128;
   }
-  if (j < p.n_wkt) return p.tile_rows[j];
+  if (j < p.n_wkt) return pv.rows[j];
   const int left = p.P - 128 * (j - p.n_wkt);
   return left < 128 ? left : 128;
 }
-__device__ __forceinline__ int query_valid(const TcParams& p, int qt) {
+__device__ __forceinline__ int query_valid(const TcParams& p, const PlanView& pv, int qt) {
   if (p.flat) {
     const long long left = p.N - 128LL * qt;
     return left < 128 ? (int)left : 128;
   }
-  return p.tile_rows[qt];
+  return pv.rows[qt];
 }
 
 // kind: 0 = q, 1 = k, 2 = v.  Loads one 128-row tile (all head-dim halves) into
 // shared memory at dst and signals bar with the transaction bytes.
 template <int D>
-__device__ __forceinline__ void load_tile(const TcParams& p, int kind, const Unit& U, int tile,
-                                          uint32_t dst, uint32_t bar) {
+__device__ __forceinline__ void load_tile(const TcParams& p, const PlanView& pv, int kind,
+                                          const Unit& U, int tile, uint32_t dst, uint32_t bar) {
   constexpr int NH = D / 64;
   if (p.flat) {
     const CUtensorMap* m = kind == 0 ? &p.qf : kind == 1 ? &p.kf : &p.vf;
@@ -380,9 +494,9 @@ __device__ __forceinline__ void load_tile(const TcParams& p, int kind, const Uni
       tma_load_4d(dst + hf * kHalf, m, bar, hf * 64, U.h, (tile - p.n_wkt) * 128, U.b);
     return;
   }
-  const int nb = p.nbox[U.cls][tile];
+  const int b0 = pv.first(U.cls, tile), nb = pv.count(U.cls, tile);
   for (int bi = 0; bi < nb; ++bi) {
-    const uint32_t e = p.box[U.cls][tile][bi];
+    const uint32_t e = pv.entries[b0 + bi];
     const int sid = box_shape(e);
     const int gt = (U.ot + box_lt(e)) % p.T;
     const int gh = (U.oh + box_lh(e)) % p.Hg;
@@ -393,7 +507,7 @@ __device__ __forceinline__ void load_tile(const TcParams& p, int kind, const Uni
     for (int hf = 0; hf < NH; ++hf)
       tma_load_5d(d0 + hf * kHalf, m, bar, hf * 64, U.h, gw, gh, U.b * p.T + gt);
   }
-  for (int r = p.tile_rows[tile]; r < 128; r += 8) {  // zero rows past the window's tokens
+  for (int r = pv.rows[tile]; r < 128; r += 8) {  // zero rows past the window's tokens
 #pragma unroll
     for (int hf = 0; hf < NH; ++hf)
       tma_load_4d(dst + hf * kHalf + r * 128, &p.fill, bar, hf * 64, 0, (int)p.N, 0);
@@ -401,16 +515,17 @@ __device__ __forceinline__ void load_tile(const TcParams& p, int kind, const Uni
 }
 
 template <int D>
-__device__ __forceinline__ void store_tile(const TcParams& p, const Unit& U, int qt, uint32_t src) {
+__device__ __forceinline__ void store_tile(const TcParams& p, const PlanView& pv, const Unit& U,
+                                           int qt, uint32_t src) {
   constexpr int NH = D / 64;
   if (p.flat) {
 #pragma unroll
     for (int hf = 0; hf < NH; ++hf) tma_store_4d(&p.of, src + hf * kHalf, hf * 64, U.h, qt * 128, U.b);
     return;
   }
-  const int nb = p.nbox[U.cls][qt];
+  const int b0 = pv.first(U.cls, qt), nb = pv.count(U.cls, qt);
   for (int bi = 0; bi < nb; ++bi) {
-    const uint32_t e = p.box[U.cls][qt][bi];
+    const uint32_t e = pv.entries[b0 + bi];
     const int sid = box_shape(e);
     const int gt = (U.ot + box_lt(e)) % p.T;
     const int gh = (U.oh + box_lh(e)) % p.Hg;
@@ -423,13 +538,14 @@ __device__ __forceinline__ void store_tile(const TcParams& p, const Unit& U, int
 }
 
 // Flattened grid index of the token held in row r of query tile qt.
-__device__ __forceinline__ long long row_token(const TcParams& p, const Unit& U, int qt, int r) {
+__device__ __forceinline__ long long row_token(const TcParams& p, const PlanView& pv,
+                                               const Unit& U, int qt, int r) {
   if (p.flat) return 128LL * qt + r;
-  const int nb = p.nbox[U.cls][qt];
+  const int b0 = pv.first(U.cls, qt), nb = pv.count(U.cls, qt);
   for (int bi = 0; bi < nb; ++bi) {
-    const uint32_t e = p.box[U.cls][qt][bi];
+    const uint32_t e = pv.entries[b0 + bi];
     const int sid = box_shape(e);
-    const int bt = p.shape_bt[sid], bh = p.shape_bh[sid], bw = p.shape_bw[sid];
+    const int bt = pv.bt[sid], bh = pv.bh[sid], bw = pv.bw[sid];
     const int r0 = box_row8(e) * 8;
     if (r >= r0 && r < r0 + bt * bh * bw) {
       const int idx = r - r0;
@@ -443,30 +559,38 @@ __device__ __forceinline__ long long row_token(const TcParams& p, const Unit& U,
   return -1;
 }
 
-// Shared-memory plan.
+// Shared-memory plan: two 128-row query tiles, the two tiles' bf16
+// probability blocks P (128 x 128, the A operand of P.V) and a ring of K/V tiles.
 template <int D>
 struct Smem {
   static constexpr int kTile = (D / 64) * kHalf;  // Q/K/V tile bytes
-  static constexpr int kPO = 2 * kHalf;           // P (128 x 128 bf16) or O staging
+  static constexpr int kP = 2 * kHalf;            // P block bytes (128 rows x 128 keys)
   static constexpr int NS = D == 128 ? 3 : 6;     // K/V ring slots
   static constexpr int q0 = 0;
-  static constexpr int po0 = 2 * kTile;
-  static constexpr int ring0 = po0 + 2 * kPO;
+  static constexpr int p0 = 2 * kTile;
+  static constexpr int ring0 = p0 + 2 * kP;
   static constexpr int bars = ring0 + NS * kTile;
   // barrier indices
   static constexpr int QFULL = 0, QEMPTY = 2, SFULL = 4, SFREE = 6, PFULL = 8, PVDONE = 10,
                        OSTAGED = 12, OFREE = 14, DRAIN = 16, KVFULL = 17, KVEMPTY = 17 + NS,
                        NBARS = 17 + 2 * NS;
   static constexpr int misc = bars + NBARS * 8;  // tmem slot, abort flag
-  static constexpr int bytes = misc + 64;
+  static constexpr int plan = misc + 64;         // compact tile plan (kPlanBytes)
+  static constexpr int bytes = plan + kPlanBytes;
   static constexpr int alloc = bytes + 1024;     // slack for 1024-byte alignment
 };
 
+// Schedule of one unit (two query tiles i = 0, 1 against key tiles j = 0..n-1).
+// TMEM columns: S_0 | S_1 | O_0 | O_1 (128 each).  The MMA warp issues, per key
+// tile j, S_i(j+1) = Q_i K_{j+1}^T for both tiles as soon as each softmax has
+// read S_i(j) out of TMEM, and then O_i += P_i(j) V_j once each softmax has
+// written P_i(j) to shared memory.  So the tensor core computes the next logits
+// while the softmax warpgroups work on the current ones, and both query tiles
+// share every K/V tile the loader brings in.
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1) tc_attn_kernel(const __grid_constant__ TcParams p) {
   using S = Smem<D>;
   constexpr int NS = S::NS;
-  constexpr int NH = D / 64;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -480,6 +604,19 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attn_kernel(const __grid_const
   const int lane = threadIdx.x % 32;
   const uint64_t limit = p.timeout_ns;
 
+  {  // the compact tile plan, from the parameter block into shared memory
+    uint32_t* dst = reinterpret_cast<uint32_t*>(smem + S::plan);
+    for (int w = threadIdx.x; w < p.plan_words; w += kThreads) dst[w] = p.plan[w];
+  }
+  const uint8_t* pimg = smem + S::plan;
+  PlanView pv;
+  pv.idx = reinterpret_cast<const uint16_t*>(pimg);
+  pv.rows = pimg + p.plan_off_rows;
+  pv.bt = pimg + p.plan_off_bt;
+  pv.bh = pimg + p.plan_off_bh;
+  pv.bw = pimg + p.plan_off_bw;
+  pv.entries = reinterpret_cast<const uint32_t*>(pimg + p.plan_off_entries);
+  pv.n_tiles = p.n_qt;
   if (threadIdx.x == 0) {
     for (int i = 0; i < 2; ++i) {
       mbar_init(BAR(S::QFULL + i), 1);
@@ -508,14 +645,32 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attn_kernel(const __grid_const
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const int n_kt = p.n_wkt + p.n_pkt;
+  // Pull every tensor map this launch uses into the TMA descriptor cache.
+  if (threadIdx.x == 0) {
+    if (p.flat) {
+      prefetch_tmap(&p.qf); prefetch_tmap(&p.kf); prefetch_tmap(&p.vf); prefetch_tmap(&p.of);
+    } else {
+      for (int sid = 0; sid < p.n_shapes; ++sid) {
+        prefetch_tmap(&p.qm[sid]); prefetch_tmap(&p.km[sid]);
+        prefetch_tmap(&p.vm[sid]); prefetch_tmap(&p.om[sid]);
+      }
+      prefetch_tmap(&p.fill);
+      if (p.n_pkt) { prefetch_tmap(&p.kpf); prefetch_tmap(&p.vpf); }
+    }
+  }
 
+  const bool withhold = (p.flags & BASA_FLAG_TEST_WITHHOLD_LOADS) != 0;
   if (warp == 0) {
     // ------------------------------------------------------------ TMA loader
     // The whole warp walks the schedule and waits; lane 0 issues the copies.
-    if (!(p.flags & BASA_FLAG_TEST_WITHHOLD_LOADS)) {
+    // Per unit: the two query tiles (each slot refilled as soon as the last S
+    // MMA of its previous unit has read it), then the key/value tiles through
+    // the ring in the order the MMA warp consumes them: K_0, then K_{j+1}, V_j.
+    if (!withhold) {
       uint32_t qn[2] = {0u, 0u};
+      uint32_t q_issued = 0, q_last = 0;
       uint32_t kv = 0;
-      uint32_t issued_mask = 0, last_par = 0, q_issued = 0, q_last = 0;
+      uint32_t issued_mask = 0, last_par = 0;
       bool ok = true;
       auto load_kv = [&](int kind, const Unit& U, int j) -> bool {
         const uint32_t slot = kv % NS, par = (kv / NS) & 1u;
@@ -523,7 +678,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attn_kernel(const __grid_const
           return false;
         if (lane == 0) {
           mbar_expect_tx(BAR(S::KVFULL + slot), S::kTile);
-          load_tile<D>(p, kind, U, j, sbase + S::ring0 + slot * S::kTile, BAR(S::KVFULL + slot));
+          load_tile<D>(p, pv, kind, U, j, sbase + S::ring0 + slot * S::kTile,
+                       BAR(S::KVFULL + slot));
         }
         __syncwarp();
         issued_mask |= 1u << slot;
@@ -531,7 +687,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attn_kernel(const __grid_const
         ++kv;
         return true;
       };
-      for (long long u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
+      for (uint32_t u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
         const Unit U = decode_unit(p, u);
         for (int i = 0; i < U.nq && ok; ++i) {
           if (!(ok = wait_warp(BAR(S::QEMPTY + i), (qn[i] & 1u) ^ 1u, abort_flag, limit,
@@ -539,7 +695,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attn_kernel(const __grid_const
             break;
           if (lane == 0) {
             mbar_expect_tx(BAR(S::QFULL + i), S::kTile);
-            load_tile<D>(p, 0, U, 2 * U.pair + i, sbase + S::q0 + i * S::kTile,
+            load_tile<D>(p, pv, 0, U, 2 * U.pair + i, sbase + S::q0 + i * S::kTile,
                          BAR(S::QFULL + i));
           }
           __syncwarp();
@@ -580,6 +736,11 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attn_kernel(const __grid_const
       tc_fence_after();
       return true;
     };
+    auto release = [&](uint32_t slot) {
+      if (lane == 0) mma_commit(BAR(S::KVEMPTY + slot));
+      __syncwarp();
+    };
+    // S_i = Q_i K^T once softmax i has read the previous S_i out of TMEM
     auto issue_s = [&](int i, uint32_t kslot, bool last) -> bool {
       if (!wait_warp(BAR(S::SFREE + i), (sfree[i] & 1u) ^ 1u, abort_flag, limit, kSiteMmaSFree))
         return false;
@@ -595,16 +756,12 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attn_kernel(const __grid_const
                    k > 0 ? 1u : 0u);
         }
         mma_commit(BAR(S::SFULL + i));
-        if (last) mma_commit(BAR(S::QEMPTY + i));
+        if (last) mma_commit(BAR(S::QEMPTY + i));  // Q_i read for the last time
       }
       __syncwarp();
       return true;
     };
-    auto release = [&](uint32_t slot) {
-      if (lane == 0) mma_commit(BAR(S::KVEMPTY + slot));
-      __syncwarp();
-    };
-    for (long long u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
+    for (uint32_t u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
       const Unit U = decode_unit(p, u);
       for (int i = 0; i < U.nq && ok; ++i) {
         ok = wait_warp(BAR(S::QFULL + i), qf[i] & 1u, abort_flag, limit, kSiteMmaQFull);
@@ -620,7 +777,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attn_kernel(const __grid_const
       for (int j = 0; j < n_kt && ok; ++j) {
         if (j + 1 < n_kt) {
           if (!(ok = take_slot(kslot))) break;
-          for (int i = 0; i < U.nq && ok; ++i) ok = issue_s(i, kslot, j + 1 == n_kt - 1);
+          for (int i = 0; i < U.nq && ok; ++i) ok = issue_s(i, kslot, j + 2 == n_kt);
           if (!ok) break;
           release(kslot);
         }
@@ -634,9 +791,9 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attn_kernel(const __grid_const
           ++pfull[i];
           tc_fence_after();
           if (lane == 0) {
-            const uint32_t pa = sbase + S::po0 + i * S::kPO;
+            const uint32_t pa = sbase + S::p0 + i * S::kP;
 #pragma unroll
-            for (int k = 0; k < 8; ++k) {
+            for (int k = 0; k < 8; ++k) {  // O_i += P_i V_j, 16 keys per MMA
               const uint32_t aoff = (k / 4) * kHalf + (k % 4) * 32;
               mma_bf16(tmem + 256 + i * 128, sdesc(pa + aoff, 16, 1024),
                        sdesc(va + k * 2048, kHalf, 1024), IDO, (j > 0 || k > 0) ? 1u : 0u);
@@ -661,12 +818,13 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attn_kernel(const __grid_const
     const uint32_t tl = (uint32_t)(q4 * 32) << 16;
     const uint32_t tS = tmem + tl + i * 128;
     const uint32_t tO = tmem + tl + 256 + i * 128;
-    const uint32_t po = sbase + S::po0 + i * S::kPO;
-    const bool leader = (warp % 4 == 0) && lane == 0;
+    const uint32_t pbuf = sbase + S::p0 + i * S::kP;  // P_i, 128-byte swizzled K-major
     uint32_t sfull = 0, pvdone = 0, ostaged = 0, ofree = 0;
+    const bool leader = (warp % 4 == 0) && lane == 0;
+    bool store_pending = false;  // the previous unit's output store may still read P_i
     const float c = p.scale_log2;
     bool ok = true;
-    for (long long u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
+    for (uint32_t u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
       const Unit U = decode_unit(p, u);
       if (i >= U.nq) continue;
       const int qt = 2 * U.pair + i;
@@ -682,47 +840,80 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attn_kernel(const __grid_const
 #pragma unroll
         for (int cc = 0; cc < 4; ++cc) tmem_wait_ld(s[cc]);
         tc_fence_before();
-        mbar_arrive(BAR(S::SFREE + i));
-        const int kvalid = key_valid(p, j);
-        float mx = -INFINITY;
+        mbar_arrive(BAR(S::SFREE + i));  // the next S_i may overwrite these columns
+        const int kvalid = key_valid(p, pv, j);
+        if (kvalid < 128) {  // padding keys of a partial tile
+#pragma unroll
+          for (int cc = 0; cc < 4; ++cc)
+#pragma unroll
+            for (int e = 0; e < 32; ++e)
+              if (cc * 32 + e >= kvalid) s[cc][e] = __float_as_uint(-INFINITY);
+        }
+        float mx0 = -INFINITY, mx1 = -INFINITY;
 #pragma unroll
         for (int cc = 0; cc < 4; ++cc)
 #pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            const float x = (cc * 32 + e < kvalid) ? __uint_as_float(s[cc][e]) : -INFINITY;
-            s[cc][e] = __float_as_uint(x);
-            mx = fmaxf(mx, x);
+          for (int e = 0; e < 32; e += 4) {
+            mx0 = max3(mx0, __uint_as_float(s[cc][e]), __uint_as_float(s[cc][e + 1]));
+            mx1 = max3(mx1, __uint_as_float(s[cc][e + 2]), __uint_as_float(s[cc][e + 3]));
           }
-        const float mnew = fmaxf(m, mx * c);
-        const float alpha = ex2(m - mnew);  // 0 on the first key tile
-        float rs = 0.f;
-        uint32_t pk[4][16];
+        const float mtile = fmaxf(mx0, mx1) * c;
+        float alpha = 1.0f;
+        if (mtile > m + kLazyRescale) {  // first tile (m = -inf) or a large jump
+          alpha = ex2(m - mtile);
+          m = mtile;
+        }
+        const uint64_t c2 = f2pack(c, c);
+        const uint64_t nm2 = f2pack(-m, -m);
+        uint64_t rsa = f2pack(0.f, 0.f), rsb = rsa;
+        uint32_t pk[2][32];  // P as bf16 pairs of keys (2c, 2c + 1) in pk[c / 32][c % 32]
 #pragma unroll
         for (int cc = 0; cc < 4; ++cc)
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
-            const float p0 = ex2(fmaf(__uint_as_float(s[cc][2 * e]), c, -mnew));
-            const float p1 = ex2(fmaf(__uint_as_float(s[cc][2 * e + 1]), c, -mnew));
-            rs += p0 + p1;
-            pk[cc][e] = pack_bf16(p0, p1);
+            const uint64_t x2 = f2fma(f2pack(__uint_as_float(s[cc][2 * e]),
+                                             __uint_as_float(s[cc][2 * e + 1])), c2, nm2);
+            uint64_t p2;
+            if (kEx2Period > 0 && e % (kEx2Period > 0 ? kEx2Period : 1) == kEx2Period - 1) {
+              p2 = ex2_poly_x2(x2);
+            } else {
+              float a0, a1;
+              f2unpack(x2, a0, a1);
+              p2 = f2pack(ex2(a0), ex2(a1));
+            }
+            if (e & 1) rsb = f2add(rsb, p2); else rsa = f2add(rsa, p2);
+            float p0, p1;
+            f2unpack(p2, p0, p1);
+            pk[cc / 2][(cc % 2) * 16 + e] = pack_bf16(p0, p1);
           }
-        l = l * alpha + rs;
-        m = mnew;
-        if (j > 0) {  // PV of the previous key tile must be done: O is stable, P is free
+        float ra0, ra1, rb0, rb1;
+        f2unpack(rsa, ra0, ra1);
+        f2unpack(rsb, rb0, rb1);
+        l = l * alpha + ((ra0 + ra1) + (rb0 + rb1));
+        if (j > 0) {  // P.V of the previous key tile must be done: O is stable, P is free
           if (!(ok = wait_warp(BAR(S::PVDONE + i), pvdone & 1u, abort_flag, limit,
                                kSiteSmxPvDone)))
             break;
           ++pvdone;
           tc_fence_after();
         }
-#pragma unroll
-        for (int cc = 0; cc < 4; ++cc)
-#pragma unroll
-          for (int v4 = 0; v4 < 4; ++v4) {
-            const int chunk = cc * 4 + v4;  // 8 keys per 16-byte chunk
-            st_shared_v4(po + (chunk / 8) * kHalf + swz(r, chunk % 8), pk[cc][4 * v4],
-                         pk[cc][4 * v4 + 1], pk[cc][4 * v4 + 2], pk[cc][4 * v4 + 3]);
+#if !BASA_DIRECT_STORE
+        if (store_pending) {  // P_i doubled as the last unit's output staging
+          if (leader) {
+            bulk_wait_read0();
+            mbar_arrive(BAR(S::OFREE + i));
           }
+          if (!(ok = wait_warp(BAR(S::OFREE + i), ofree & 1u, abort_flag, limit, kSiteSmxOFree)))
+            break;
+          ++ofree;
+          store_pending = false;
+        }
+#endif
+#pragma unroll
+        for (int ch = 0; ch < 16; ++ch)  // 8 keys per 16-byte chunk
+          st_shared_v4(pbuf + (ch / 8) * kHalf + swz(r, ch % 8), pk[ch / 8][(ch % 8) * 4],
+                       pk[ch / 8][(ch % 8) * 4 + 1], pk[ch / 8][(ch % 8) * 4 + 2],
+                       pk[ch / 8][(ch % 8) * 4 + 3]);
         // tcgen05.ld/st are warp-collective: the whole warp rescales if any row needs it
         if (j > 0 && __any_sync(0xffffffffu, alpha < 1.0f)) {
 #pragma unroll
@@ -730,13 +921,19 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attn_kernel(const __grid_const
             uint32_t o[32];
             tmem_ld32(tO + cc * 32, o);
             tmem_wait_ld(o);
+            const uint64_t a2 = f2pack(alpha, alpha);
 #pragma unroll
-            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+            for (int e = 0; e < 32; e += 2) {
+              float o0, o1;
+              f2unpack(f2mul(f2pack(__uint_as_float(o[e]), __uint_as_float(o[e + 1])), a2), o0, o1);
+              o[e] = __float_as_uint(o0);
+              o[e + 1] = __float_as_uint(o1);
+            }
             tmem_st32(tO + cc * 32, o);
           }
-          tmem_wait_st();
         }
-        fence_proxy_async();
+        fence_proxy_async();  // P's generic-proxy stores, visible to the MMA
+        tmem_wait_st();
         tc_fence_before();
         mbar_arrive(BAR(S::PFULL + i));
       }
@@ -745,8 +942,16 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attn_kernel(const __grid_const
         break;
       ++pvdone;
       tc_fence_after();
-      // epilogue: O / l -> bf16 -> staging (the P buffer, free now) -> TMA store
+#if BASA_DIRECT_STORE
+      // epilogue: O / l -> bf16 -> this thread's token row, written straight from
+      // registers with streaming 16-byte stores
+      const long long n = r < query_valid(p, pv, qt) ? row_token(p, pv, U, qt, r) : -1;
+      uint4* orow = n >= 0 ? reinterpret_cast<uint4*>(p.out + ((((long long)U.b * p.N + n) *
+                                                                p.H + U.h) * D))
+                           : nullptr;
+#endif
       const float inv = 1.0f / l;
+      const uint64_t inv2 = f2pack(inv, inv);
 #pragma unroll
       for (int cc = 0; cc < D / 32; ++cc) {
         uint32_t o[32];
@@ -754,18 +959,31 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attn_kernel(const __grid_const
         tmem_wait_ld(o);
 #pragma unroll
         for (int v4 = 0; v4 < 4; ++v4) {
-          const int col = cc * 32 + v4 * 8;
           uint32_t w[4];
 #pragma unroll
-          for (int e = 0; e < 4; ++e)
-            w[e] = pack_bf16(__uint_as_float(o[v4 * 8 + 2 * e]) * inv,
-                             __uint_as_float(o[v4 * 8 + 2 * e + 1]) * inv);
-          st_shared_v4(po + (col / 64) * kHalf + swz(r, (col % 64) / 8), w[0], w[1], w[2], w[3]);
+          for (int e = 0; e < 4; ++e) {
+            float o0, o1;
+            f2unpack(f2mul(f2pack(__uint_as_float(o[v4 * 8 + 2 * e]),
+                                  __uint_as_float(o[v4 * 8 + 2 * e + 1])), inv2), o0, o1);
+            w[e] = pack_bf16(o0, o1);
+          }
+#if BASA_DIRECT_STORE
+          if (orow) __stcs(orow + cc * 4 + v4, make_uint4(w[0], w[1], w[2], w[3]));
+#else
+          // epilogue: O / l -> bf16 -> staging in P_i (free now) -> TMA store
+          const int col = cc * 32 + v4 * 8;
+          st_shared_v4(pbuf + (col / 64) * kHalf + swz(r, (col % 64) / 8), w[0], w[1], w[2],
+                       w[3]);
+#endif
         }
       }
       tc_fence_before();
-      if (p.lse && r < query_valid(p, qt)) {
-        const long long n = row_token(p, U, qt, r);
+#if BASA_DIRECT_STORE
+      if (p.lse && n >= 0)
+        p.lse[((long long)U.b * p.H + U.h) * p.N + n] = (m + __log2f(l)) * 0.69314718055994531f;
+#else
+      if (p.lse && r < query_valid(p, pv, qt)) {
+        const long long n = row_token(p, pv, U, qt, r);
         if (n >= 0)
           p.lse[((long long)U.b * p.H + U.h) * p.N + n] = (m + __log2f(l)) * 0.69314718055994531f;
       }
@@ -775,20 +993,17 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attn_kernel(const __grid_const
         const bool staged =
             wait_bounded(BAR(S::OSTAGED + i), ostaged & 1u, abort_flag, limit, kSiteSmxOStaged);
         if (staged) {
-          store_tile<D>(p, U, qt, po);
+          store_tile<D>(p, pv, U, qt, pbuf);
           bulk_commit();
-          bulk_wait_read0();
         }
-        mbar_arrive(BAR(S::OFREE + i));
       }
       ++ostaged;
-      if (!(ok = wait_warp(BAR(S::OFREE + i), ofree & 1u, abort_flag, limit, kSiteSmxOFree)))
-        break;
-      ++ofree;
+      store_pending = true;  // waited for before the next unit's first P write
+#endif
     }
-    if (leader) bulk_wait_all0();
   }
 
+  if (warp >= 4 && (warp % 4 == 0) && lane == 0) bulk_wait_all0();  // stores issued
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -822,6 +1037,41 @@ basa_status launch_impl(TcParams* prm, cudaStream_t stream) {
 
 namespace {
 
+// Packs the tile plan into the compact image the kernel copies to shared memory.
+basa_status pack_plan(const TilePlan& plan, TcParams* prm) {
+  const int T = plan.n_tiles, NSh = plan.n_shapes;
+  uint8_t* img = reinterpret_cast<uint8_t*>(prm->plan);
+  const int off_rows = 2 * kClasses * T;
+  const int off_bt = off_rows + T, off_bh = off_bt + NSh, off_bw = off_bh + NSh;
+  const int off_entries = (off_bw + NSh + 3) & ~3;
+  int n = 0;
+  for (int c = 0; c < kClasses; ++c)
+    for (int t = 0; t < T; ++t) n += plan.nbox[c][t];
+  const int total = off_entries + 4 * n;
+  if (total > kPlanBytes || n >= 4096) return BASA_ERR_UNSUPPORTED;
+  uint16_t* idx = reinterpret_cast<uint16_t*>(img);
+  uint32_t* entries = reinterpret_cast<uint32_t*>(img + off_entries);
+  int e = 0;
+  for (int c = 0; c < kClasses; ++c)
+    for (int t = 0; t < T; ++t) {
+      idx[c * T + t] = (uint16_t)((e << 4) | plan.nbox[c][t]);
+      for (int b = 0; b < plan.nbox[c][t]; ++b) entries[e++] = plan.box[c][t][b];
+    }
+  for (int t = 0; t < T; ++t) img[off_rows + t] = plan.tile_rows[t];
+  for (int s2 = 0; s2 < NSh; ++s2) {
+    img[off_bt + s2] = plan.shape_bt[s2];
+    img[off_bh + s2] = plan.shape_bh[s2];
+    img[off_bw + s2] = plan.shape_bw[s2];
+  }
+  prm->plan_words = (total + 3) / 4;
+  prm->plan_off_rows = off_rows;
+  prm->plan_off_bt = off_bt;
+  prm->plan_off_bh = off_bh;
+  prm->plan_off_bw = off_bw;
+  prm->plan_off_entries = off_entries;
+  return BASA_OK;
+}
+
 // Fills *prm (zeroed by the caller) for one call and launches the kernel.
 basa_status build_and_launch(TcParams* prm, const Dims& d, bool flat, const void* q,
                              const void* k, const void* v, const void* kp, const void* vp,
@@ -836,6 +1086,7 @@ basa_status build_and_launch(TcParams* prm, const Dims& d, bool flat, const void
   prm->nwt = d.nwt; prm->nwh = d.nwh; prm->nww = d.nww;
   prm->N = d.N;
   prm->lse = lse;
+  prm->out = static_cast<__nv_bfloat16*>(out);
   prm->flags = flags;
   prm->timeout_ns = (unsigned long long)(timeout_ms ? timeout_ms : 2000u) * 1000000ull;
   prm->scale_log2 = d.scale * 1.4426950408889634f;
@@ -866,14 +1117,11 @@ basa_status build_and_launch(TcParams* prm, const Dims& d, bool flat, const void
     prm->n_pkt = 0;
     prm->n_windows = 1;
     prm->n_pairs = (prm->n_qt + 1) / 2;
-    prm->n_units = (long long)d.B * d.H * prm->n_pairs;
+    const long long units = (long long)d.B * d.H * prm->n_pairs;
+    if (units > 0x7fffffffLL) { st = BASA_ERR_UNSUPPORTED; goto done; }
+    prm->n_units = (uint32_t)units;
   } else {
-    memcpy(prm->box, plan.box, sizeof(plan.box));
-    memcpy(prm->nbox, plan.nbox, sizeof(plan.nbox));
-    memcpy(prm->tile_rows, plan.tile_rows, sizeof(plan.tile_rows));
-    memcpy(prm->shape_bt, plan.shape_bt, sizeof(plan.shape_bt));
-    memcpy(prm->shape_bh, plan.shape_bh, sizeof(plan.shape_bh));
-    memcpy(prm->shape_bw, plan.shape_bw, sizeof(plan.shape_bw));
+    if ((st = pack_plan(plan, prm)) != BASA_OK) goto done;
     const uint64_t dims[5] = {D, H, (uint64_t)d.Wg, (uint64_t)d.Hg, (uint64_t)d.B * d.T};
     const uint64_t strides[4] = {D * 2, H * D * 2, (uint64_t)d.Wg * H * D * 2,
                                  (uint64_t)d.Hg * d.Wg * H * D * 2};
@@ -891,12 +1139,15 @@ basa_status build_and_launch(TcParams* prm, const Dims& d, bool flat, const void
       if ((st = encode_map(&prm->kpf, kp, 4, pdims, pstr, box128)) != BASA_OK) goto done;
       if ((st = encode_map(&prm->vpf, vp, 4, pdims, pstr, box128)) != BASA_OK) goto done;
     }
+    prm->n_shapes = plan.n_shapes;
     prm->n_qt = plan.n_tiles;
     prm->n_wkt = plan.n_tiles;
     prm->n_pkt = kp ? (int)((d.P + 127) / 128) : 0;
     prm->n_windows = d.nwt * d.nwh * d.nww;
     prm->n_pairs = (prm->n_qt + 1) / 2;
-    prm->n_units = (long long)d.B * d.H * prm->n_windows * prm->n_pairs;
+    const long long units = (long long)d.B * d.H * prm->n_windows * prm->n_pairs;
+    if (units > 0x7fffffffLL) { st = BASA_ERR_UNSUPPORTED; goto done; }
+    prm->n_units = (uint32_t)units;
   }
   st = d.d == 128 ? launch_impl<128>(prm, stream) : launch_impl<64>(prm, stream);
 done:
@@ -930,6 +1181,25 @@ basa_status launch_tc_static_params(const Dims& d, bool flat, const void* q, con
   memset(&g_static_params, 0, sizeof(g_static_params));
   return build_and_launch(&g_static_params, d, flat, q, k, v, kp, vp, out, lse, flags,
                           timeout_ms, stream);
+}
+
+namespace {
+__global__ void ex2_poly_test_kernel(const float* x, float* y, long long n) {
+  const long long i = 2 * ((long long)blockIdx.x * blockDim.x + threadIdx.x);
+  if (i >= n) return;
+  const float x1 = i + 1 < n ? x[i + 1] : 0.0f;
+  float y0, y1;
+  f2unpack(ex2_poly_x2(f2pack(x[i], x1)), y0, y1);
+  y[i] = y0;
+  if (i + 1 < n) y[i + 1] = y1;
+}
+}  // namespace
+
+basa_status launch_ex2_poly_test(const float* x, float* y, long long n, cudaStream_t stream) {
+  if (n <= 0) return BASA_OK;
+  const long long pairs = (n + 1) / 2;
+  ex2_poly_test_kernel<<<(unsigned)((pairs + 255) / 256), 256, 0, stream>>>(x, y, n);
+  return cudaGetLastError() == cudaSuccess ? BASA_OK : BASA_ERR_CUDA;
 }
 
 basa_status read_and_clear_status(cudaStream_t stream) {
