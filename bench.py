@@ -5,7 +5,9 @@ one batch of the workload (for workloads with global memory: pooling + window
 attention); inputs are seeded and synthetic.
 
 Kernel time: every step is bracketed by CUDA events on the launching stream.
-Before each step the L2 is flushed (a 256 MiB write) and a short device sleep
+Before each step the L2 is evicted (a 256 MiB write, then a 256 MiB read of
+another buffer, so no dirty lines are left to be written back during the
+timed kernel) and a short device sleep
 is queued, so the event pair measures the kernel and not the host-side launch
 preparation; neither the flush nor the sleep is inside the events.  Reported:
 algorithmic TFLOP/s (4*B*H*N*(m+P)*d flops per step), latency, the dominant
@@ -146,13 +148,33 @@ def _sleep_cycles(us):
     torch.cuda._sleep(int(us * 2000))
 
 
+class L2Flush:
+    """Evicts the L2 (126 MB on B200) between timed steps.
+
+    A 256 MiB write replaces every line, then a 256 MiB read of another buffer
+    replaces the dirty lines the write left, so the timed kernel starts with an
+    L2 that holds none of its data and owes no write-backs of someone else's.
+    Both run outside the timing events.
+    """
+
+    def __init__(self, device, nbytes=256 << 20):
+        self.w = torch.empty(nbytes, dtype=torch.uint8, device=device)
+        self.r = torch.zeros(nbytes // 4, dtype=torch.int32, device=device)
+        self.i = 0
+
+    def __call__(self):
+        self.i += 1
+        self.w.fill_(self.i & 0xFF)
+        self.sink = torch.amax(self.r)
+
+
 def time_steps(fn, steps, flush, sleep_us=200.0):
     """Per-step device time (ms) of fn() with an L2 flush and a sleep before each step."""
     stream = torch.cuda.current_stream()
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
           for _ in range(steps)]
     for i in range(steps):
-        flush.fill_(i & 0xFF)
+        flush()
         if sleep_us > 0:
             _sleep_cycles(sleep_us)
         ev[i][0].record(stream)
@@ -188,9 +210,14 @@ def cpu_baseline(w, shift, q, k, v, budget_s=12.0):
     nheads = max(1, min(w.H, int(budget_s / max(dt1, 1e-3))))
     heads = list(range(nheads))
     dt, fl = run_oracle_sample(w, shift, q, k, v, heads)
+    reps = 1
+    # a whole batch finishing well inside the budget: repeat it for a steadier number
+    while nheads == w.H and dt < budget_s * 0.75 and reps < 16:
+        dti, fli = run_oracle_sample(w, shift, q, k, v, heads)
+        dt, fl, reps = dt + dti, fl + fli, reps + 1
     return {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
-            "sample": f"all {w.N} queries of {nheads} of {w.H} heads, batch 0, shift {shift}; "
-                      f"{dt:.2f} s fp64 on {cores} host threads"}
+            "sample": f"all {w.N} queries of {nheads} of {w.H} heads, batch 0, shift {shift}, "
+                      f"{reps} run(s); {dt:.2f} s fp64 on {cores} host threads"}
 
 
 def dist_setup(args):
@@ -286,7 +313,7 @@ def main():
     outh = torch.empty_like(qh).pin_memory()
     ws_bytes = basa.workspace_size(w.shape(), dq.dtype, w.window, shift, w.pool)
     ws = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=dev)
-    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    flush = L2Flush(dev)
     flops, bytes_, N, m, P = workload_numbers(w, shift)
 
     def step():
@@ -341,7 +368,7 @@ def main():
     stream = torch.cuda.current_stream()
     e2e_ms = []
     for i in range(args.steps):
-        flush.fill_(i & 0xFF)
+        flush()
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record(stream)
         step_e2e()
@@ -377,7 +404,7 @@ def main():
                                f"window {'x'.join(map(str, w.window))} shift {shift} "
                                f"pool {w.pool}",
                    "N": N, "m": m, "P": P, "global_batch": w.B * world,
-                   "l2": "flushed before every step (256 MiB write, outside the events)",
+                   "l2": "evicted before every step (256 MiB write, then 256 MiB read; outside the events)",
                    "parallelism": f"replicas x{world}"},
         "latency_ms": ms_max,
         "pct_bf16_peak": 100.0 * per_gpu_tflops / peaks["bf16_tflops"],

@@ -17,7 +17,7 @@ from typing import Optional, Sequence, Tuple
 import torch
 
 from . import _lib
-from ._lib import BasaError, BasaParams, BASA_F32, BASA_BF16
+from ._lib import BasaError, BasaParams, BASA_F32, BASA_BF16  # noqa: F401
 
 __all__ = ["window_attn", "window_attn_gm", "full_attn", "pool_kv", "workspace_size",
            "get_status", "window_tiles", "make_params", "BasaError", "library_path"]
@@ -125,10 +125,10 @@ def window_attn(q, k, v, window, shift=(0, 0, 0), pool=(0, 0, 0), scale=None,
 
 
 def window_attn_gm(q, k, v, kp, vp, window, shift=(0, 0, 0), pool=(1, 1, 1), scale=None,
-                   return_lse=False, out=None, stream=None):
+                   return_lse=False, out=None, flags=0, stream=None):
     """Window attention with caller-supplied pooled global memory kp, vp."""
     _check_inputs(q, k, v, kp, vp)
-    prm = make_params(q.shape, q.dtype, window, shift, pool, scale)
+    prm = make_params(q.shape, q.dtype, window, shift, pool, scale, flags)
     lib = _lib.load()
     out = torch.empty_like(q) if out is None else out
     B, T, Hg, Wg, H, d = q.shape
@@ -140,10 +140,10 @@ def window_attn_gm(q, k, v, kp, vp, window, shift=(0, 0, 0), pool=(1, 1, 1), sca
     return (out, lse) if return_lse else out
 
 
-def full_attn(q, k, v, scale=None, return_lse=False, out=None, stream=None):
+def full_attn(q, k, v, scale=None, return_lse=False, out=None, flags=0, stream=None):
     """Full softmax attention over all grid tokens (one window covering the grid)."""
     _check_inputs(q, k, v)
-    prm = make_params(q.shape, q.dtype, (1, 1, 1), (0, 0, 0), (0, 0, 0), scale)
+    prm = make_params(q.shape, q.dtype, (1, 1, 1), (0, 0, 0), (0, 0, 0), scale, flags)
     lib = _lib.load()
     out = torch.empty_like(q) if out is None else out
     B, T, Hg, Wg, H, d = q.shape

@@ -11,22 +11,26 @@
 //
 // Work unit: (b, h, window, pair of 128-query tiles).  Persistent CTAs (one
 // per SM) walk the units, heads fastest.  Inside a CTA the warps specialise:
-//   warp 0        TMA loader: the two query tiles of each unit, then its K and V
-//                 tiles through a 3-slot ring (boxes from the shifted-window
-//                 tile plan; a tile that crosses a wrapped border is fetched as
-//                 up to 8 boxes, so no rolled copy of the grid is ever made);
+//   warp 0        TMA loader of the K and V tiles, through a 4-slot ring (boxes
+//                 from the shifted-window tile plan; a tile that crosses a
+//                 wrapped border is fetched as up to 8 boxes, so no rolled copy
+//                 of the grid is ever made);
+//   warp 2        TMA loader of the two query tiles of each unit;
 //   warp 1        owns TMEM (512 columns) and issues the MMAs from one thread:
-//                 S_i = Q_i K_j^T into TMEM (the next key tile's logits while the
-//                 softmax works on the current ones), then O_i += P_i V_j;
+//                 S_i = Q_i K_j^T into TMEM, and O_i += P_i V_j with P_i read
+//                 from TMEM; the two query tiles alternate so that one tile's
+//                 exponentials overlap the other tile's MMAs;
 //   warps 4..7    softmax + epilogue for query tile 0 of the unit,
 //   warps 8..11   the same for query tile 1.
 // Each softmax thread owns one query row: it reads its 128 logits from TMEM,
 // keeps the running max and sum in fp32 (base-2 exponentials with the scale
-// folded in), writes the bf16 probabilities P to shared memory in the
-// 128-byte-swizzled K-major layout the MMA reads, and rescales its O row in
-// TMEM when the max grows by more than 2^8.  The epilogue divides by the sum,
-// rounds to bf16, stages the tile in the P buffer and stores it with TMA boxes
-// that mirror the load boxes.
+// folded in), writes the bf16 probabilities P back into TMEM over its logits,
+// and rescales its O row in TMEM when the max grows by more than 2^8.  The
+// epilogue divides by the sum and rounds to bf16; each warp then either stages
+// its 32 rows in shared memory and writes them back with 16-byte stores that
+// cover whole 128-byte row segments, or (windows of more than two key tiles)
+// the warpgroup stages the tile and stores it with TMA boxes that mirror the
+// load boxes.
 //
 // Every mbarrier wait is bounded (wall-clock limit from the call); on expiry the
 // kernel raises the device status word, lets every role leave its loop, waits
@@ -67,6 +71,7 @@ struct __align__(64) TcParams {
   int plan_off_rows, plan_off_bt, plan_off_bh, plan_off_bw, plan_off_entries;  // bytes
   float* lse;
   __nv_bfloat16* out;  // [B, T, Hg, Wg, H, d]
+  int warp_stores;  // output by warp-staged 16-byte stores (1) or by TMA boxes (0)
   uint32_t n_units;
   long long N;
   unsigned long long timeout_ns;
@@ -263,6 +268,15 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
       TMEM_INREGS32(r)
       : "memory");
 }
+// 16 consecutive 32-bit columns of this thread's lane.
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+      "%11, %12, %13, %14, %15, %16};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+      : "memory");
+}
 __device__ __forceinline__ void tmem_wait_st() {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
@@ -340,17 +354,23 @@ __device__ __forceinline__ uint64_t ex2_poly_x2(uint64_t x2) {
 
 // Which exponential pairs go to the polynomial: pair e of every 16 when
 // e % kEx2Period == kEx2Period - 1 (period 3: 5 of 16 pairs); 0 = none.
-#ifndef BASA_DIRECT_STORE
-#define BASA_DIRECT_STORE 0
-#endif
 #ifndef BASA_EX2_PERIOD
 #define BASA_EX2_PERIOD 0
 #endif
 constexpr int kEx2Period = BASA_EX2_PERIOD;
+
 // Rescale O only when a tile's row max exceeds the reference max by more than
 // 2^kLazyRescale; until then the stale reference is kept (P stays <= 2^8).
 constexpr float kLazyRescale = 8.0f;
 
+__device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "r"(addr)
+               : "memory");
+  return v;
+}
 __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
                                              uint32_t d) {
   asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c),
@@ -514,13 +534,15 @@ __device__ __forceinline__ void load_tile(const TcParams& p, const PlanView& pv,
   }
 }
 
+// Stores d-half hf of query tile qt from a 128-row x 64-column staging block
+// (128-byte swizzled) with TMA boxes that mirror the load boxes.
+// Stores d-half hf of query tile qt from a 128-row x 64-column staging block
+// (128-byte swizzled) with TMA boxes that mirror the load boxes.
 template <int D>
-__device__ __forceinline__ void store_tile(const TcParams& p, const PlanView& pv, const Unit& U,
-                                           int qt, uint32_t src) {
-  constexpr int NH = D / 64;
+__device__ __forceinline__ void store_half(const TcParams& p, const PlanView& pv, const Unit& U,
+                                           int qt, int hf, uint32_t src) {
   if (p.flat) {
-#pragma unroll
-    for (int hf = 0; hf < NH; ++hf) tma_store_4d(&p.of, src + hf * kHalf, hf * 64, U.h, qt * 128, U.b);
+    tma_store_4d(&p.of, src, hf * 64, U.h, qt * 128, U.b);
     return;
   }
   const int b0 = pv.first(U.cls, qt), nb = pv.count(U.cls, qt);
@@ -530,10 +552,7 @@ __device__ __forceinline__ void store_tile(const TcParams& p, const PlanView& pv
     const int gt = (U.ot + box_lt(e)) % p.T;
     const int gh = (U.oh + box_lh(e)) % p.Hg;
     const int gw = (U.ow + box_lw(e)) % p.Wg;
-    const uint32_t s0 = src + box_row8(e) * 1024;
-#pragma unroll
-    for (int hf = 0; hf < NH; ++hf)
-      tma_store_5d(&p.om[sid], s0 + hf * kHalf, hf * 64, U.h, gw, gh, U.b * p.T + gt);
+    tma_store_5d(&p.om[sid], src + box_row8(e) * 1024, hf * 64, U.h, gw, gh, U.b * p.T + gt);
   }
 }
 
@@ -559,34 +578,37 @@ __device__ __forceinline__ long long row_token(const TcParams& p, const PlanView
   return -1;
 }
 
-// Shared-memory plan: two 128-row query tiles, the two tiles' bf16
-// probability blocks P (128 x 128, the A operand of P.V) and a ring of K/V tiles.
+// Shared-memory plan: the unit's two 128-row query tiles, one 64-column output
+// staging block per query tile, and a ring of K/V tiles.  The probabilities P
+// never touch shared memory: they are written into TMEM over their logits and
+// read from there by the P.V MMA.
 template <int D>
 struct Smem {
   static constexpr int kTile = (D / 64) * kHalf;  // Q/K/V tile bytes
-  static constexpr int kP = 2 * kHalf;            // P block bytes (128 rows x 128 keys)
-  static constexpr int NS = D == 128 ? 3 : 6;     // K/V ring slots
+  static constexpr int NS = D == 128 ? 4 : 8;     // K/V ring slots
   static constexpr int q0 = 0;
-  static constexpr int p0 = 2 * kTile;
-  static constexpr int ring0 = p0 + 2 * kP;
+  static constexpr int stg0 = 2 * kTile;
+  static constexpr int ring0 = stg0 + 2 * kHalf;
   static constexpr int bars = ring0 + NS * kTile;
   // barrier indices
-  static constexpr int QFULL = 0, QEMPTY = 2, SFULL = 4, SFREE = 6, PFULL = 8, PVDONE = 10,
-                       OSTAGED = 12, OFREE = 14, DRAIN = 16, KVFULL = 17, KVEMPTY = 17 + NS,
-                       NBARS = 17 + 2 * NS;
+  static constexpr int QFULL = 0, QEMPTY = 2, SFULL = 4, PFULL = 6, OFULL = 8, STAGED = 10,
+                       STGFREE = 12, DRAIN = 14, KVFULL = 15, KVEMPTY = 15 + NS,
+                       NBARS = 15 + 2 * NS;
   static constexpr int misc = bars + NBARS * 8;  // tmem slot, abort flag
   static constexpr int plan = misc + 64;         // compact tile plan (kPlanBytes)
   static constexpr int bytes = plan + kPlanBytes;
   static constexpr int alloc = bytes + 1024;     // slack for 1024-byte alignment
 };
 
-// Schedule of one unit (two query tiles i = 0, 1 against key tiles j = 0..n-1).
-// TMEM columns: S_0 | S_1 | O_0 | O_1 (128 each).  The MMA warp issues, per key
-// tile j, S_i(j+1) = Q_i K_{j+1}^T for both tiles as soon as each softmax has
-// read S_i(j) out of TMEM, and then O_i += P_i(j) V_j once each softmax has
-// written P_i(j) to shared memory.  So the tensor core computes the next logits
-// while the softmax warpgroups work on the current ones, and both query tiles
-// share every K/V tile the loader brings in.
+// Schedule of one unit (query tiles i = 0, 1 against key tiles j = 0..n-1).
+// TMEM columns: S_0 | S_1 | O_0 | O_1 (128 each); P_i is written as bf16 pairs
+// over the first 64 columns of S_i.  The MMA warp issues S_0(0), S_1(0), then
+// per key tile j: O_0 += P_0(j) V_j, S_0(j+1), O_1 += P_1(j) V_j, S_1(j+1).
+// The tensor core executes one thread's MMAs in issue order, so S_i(j+1) only
+// overwrites P_i(j) after the P.V MMA that reads it.  The two query tiles
+// alternate: while softmax 0 exponentiates S_0(j+1), the tensor core runs
+// P_1(j) V_j and S_1(j+1), and the other way round, so the exponentials of one
+// tile overlap the MMAs of the other.
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1) tc_attn_kernel(const __grid_constant__ TcParams p) {
   using S = Smem<D>;
@@ -622,11 +644,10 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attn_kernel(const __grid_const
       mbar_init(BAR(S::QFULL + i), 1);
       mbar_init(BAR(S::QEMPTY + i), 1);
       mbar_init(BAR(S::SFULL + i), 1);
-      mbar_init(BAR(S::SFREE + i), 128);
       mbar_init(BAR(S::PFULL + i), 128);
-      mbar_init(BAR(S::PVDONE + i), 1);
-      mbar_init(BAR(S::OSTAGED + i), 128);
-      mbar_init(BAR(S::OFREE + i), 1);
+      mbar_init(BAR(S::OFULL + i), 1);
+      mbar_init(BAR(S::STAGED + i), 128);
+      mbar_init(BAR(S::STGFREE + i), 1);
     }
     mbar_init(BAR(S::DRAIN), 1);
     for (int s = 0; s < NS; ++s) {
@@ -661,32 +682,47 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attn_kernel(const __grid_const
 
   const bool withhold = (p.flags & BASA_FLAG_TEST_WITHHOLD_LOADS) != 0;
   if (warp == 0) {
-    // ------------------------------------------------------------ TMA loader
+    // ------------------------------------------------------------ K/V loader
     // The whole warp walks the schedule and waits; lane 0 issues the copies.
-    // Per unit: the two query tiles (each slot refilled as soon as the last S
-    // MMA of its previous unit has read it), then the key/value tiles through
-    // the ring in the order the MMA warp consumes them: K_0, then K_{j+1}, V_j.
+    // Ring order per unit: K_0, V_0, K_1, V_1, ... (the MMA warp's order).
     if (!withhold) {
-      uint32_t qn[2] = {0u, 0u};
-      uint32_t q_issued = 0, q_last = 0;
       uint32_t kv = 0;
       uint32_t issued_mask = 0, last_par = 0;
       bool ok = true;
-      auto load_kv = [&](int kind, const Unit& U, int j) -> bool {
-        const uint32_t slot = kv % NS, par = (kv / NS) & 1u;
-        if (!wait_warp(BAR(S::KVEMPTY + slot), par ^ 1u, abort_flag, limit, kSiteLoadKvEmpty))
-          return false;
-        if (lane == 0) {
-          mbar_expect_tx(BAR(S::KVFULL + slot), S::kTile);
-          load_tile<D>(p, pv, kind, U, j, sbase + S::ring0 + slot * S::kTile,
-                       BAR(S::KVFULL + slot));
+      for (uint32_t u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
+        const Unit U = decode_unit(p, u);
+        for (int j = 0; j < n_kt && ok; ++j) {
+          for (int kind = 1; kind <= 2 && ok; ++kind) {
+            const uint32_t slot = kv % NS, par = (kv / NS) & 1u;
+            if (!(ok = wait_warp(BAR(S::KVEMPTY + slot), par ^ 1u, abort_flag, limit,
+                                 kSiteLoadKvEmpty)))
+              break;
+            if (lane == 0) {
+              mbar_expect_tx(BAR(S::KVFULL + slot), S::kTile);
+              load_tile<D>(p, pv, kind, U, j, sbase + S::ring0 + slot * S::kTile,
+                           BAR(S::KVFULL + slot));
+            }
+            __syncwarp();
+            issued_mask |= 1u << slot;
+            last_par = (last_par & ~(1u << slot)) | (par << slot);
+            ++kv;
+          }
         }
-        __syncwarp();
-        issued_mask |= 1u << slot;
-        last_par = (last_par & ~(1u << slot)) | (par << slot);
-        ++kv;
-        return true;
-      };
+      }
+      // Drain: wait (bounded, regardless of an abort) until every copy issued has landed.
+      for (int s = 0; s < NS; ++s)
+        if (issued_mask & (1u << s))
+          wait_warp(BAR(S::KVFULL + s), (last_par >> s) & 1u, abort_flag, limit,
+                    kSiteLoadDrainKv, false);
+    }
+  } else if (warp == 2) {
+    // ------------------------------------------------------------ query loader
+    // Q_i of the next unit is fetched as soon as the last S MMA of the current
+    // unit has read Q_i.
+    if (!withhold) {
+      uint32_t qn[2] = {0u, 0u};
+      uint32_t q_issued = 0, q_last = 0;
+      bool ok = true;
       for (uint32_t u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
         const Unit U = decode_unit(p, u);
         for (int i = 0; i < U.nq && ok; ++i) {
@@ -703,18 +739,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attn_kernel(const __grid_const
           q_last = (q_last & ~(1u << i)) | ((qn[i] & 1u) << i);
           ++qn[i];
         }
-        if (!ok) break;
-        ok = load_kv(1, U, 0);
-        for (int j = 0; j < n_kt && ok; ++j) {
-          if (j + 1 < n_kt) ok = load_kv(1, U, j + 1);
-          if (ok) ok = load_kv(2, U, j);
-        }
+        __syncwarp();
       }
-      // Drain: wait (bounded, regardless of an abort) until every copy issued has landed.
-      for (int s = 0; s < NS; ++s)
-        if (issued_mask & (1u << s))
-          wait_warp(BAR(S::KVFULL + s), (last_par >> s) & 1u, abort_flag, limit,
-                    kSiteLoadDrainKv, false);
       for (int i = 0; i < 2; ++i)
         if (q_issued & (1u << i))
           wait_warp(BAR(S::QFULL + i), (q_last >> i) & 1u, abort_flag, limit, kSiteLoadDrainQ,
@@ -725,7 +751,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attn_kernel(const __grid_const
     // The whole warp walks the schedule and waits; lane 0 issues MMAs and commits.
     constexpr uint32_t IDS = idesc_bf16(128, false);
     constexpr uint32_t IDO = idesc_bf16(D, true);
-    uint32_t qf[2] = {0u, 0u}, sfree[2] = {0u, 0u}, pfull[2] = {0u, 0u};
+    uint32_t qf[2] = {0u, 0u}, pfull[2] = {0u, 0u};
     uint32_t kv = 0;
     bool ok = true;
     auto take_slot = [&](uint32_t& slot) -> bool {
@@ -740,70 +766,71 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attn_kernel(const __grid_const
       if (lane == 0) mma_commit(BAR(S::KVEMPTY + slot));
       __syncwarp();
     };
-    // S_i = Q_i K^T once softmax i has read the previous S_i out of TMEM
-    auto issue_s = [&](int i, uint32_t kslot, bool last) -> bool {
-      if (!wait_warp(BAR(S::SFREE + i), (sfree[i] & 1u) ^ 1u, abort_flag, limit, kSiteMmaSFree))
-        return false;
-      ++sfree[i];
-      tc_fence_after();
-      if (lane == 0) {
-        const uint32_t qa = sbase + S::q0 + i * S::kTile;
-        const uint32_t ka = sbase + S::ring0 + kslot * S::kTile;
+    // S_i = Q_i K^T (lane 0 only)
+    auto mma_s = [&](int i, uint32_t kslot) {
+      const uint32_t qa = sbase + S::q0 + i * S::kTile;
+      const uint32_t ka = sbase + S::ring0 + kslot * S::kTile;
 #pragma unroll
-        for (int k = 0; k < D / 16; ++k) {
-          const uint32_t off = (k / 4) * kHalf + (k % 4) * 32;
-          mma_bf16(tmem + i * 128, sdesc(qa + off, 16, 1024), sdesc(ka + off, 16, 1024), IDS,
-                   k > 0 ? 1u : 0u);
-        }
-        mma_commit(BAR(S::SFULL + i));
-        if (last) mma_commit(BAR(S::QEMPTY + i));  // Q_i read for the last time
+      for (int k = 0; k < D / 16; ++k) {
+        const uint32_t off = (k / 4) * kHalf + (k % 4) * 32;
+        mma_bf16(tmem + i * 128, sdesc(qa + off, 16, 1024), sdesc(ka + off, 16, 1024), IDS,
+                 k > 0 ? 1u : 0u);
       }
-      __syncwarp();
-      return true;
+    };
+    // O_i (+)= P_i V, P_i from TMEM (8 columns per 16 keys) (lane 0 only)
+    auto mma_pv = [&](int i, uint32_t vslot, bool accumulate) {
+      const uint32_t va = sbase + S::ring0 + vslot * S::kTile;
+#pragma unroll
+      for (int k = 0; k < 8; ++k)
+        mma_bf16_ts(tmem + 256 + i * 128, tmem + i * 128 + k * 8,
+                    sdesc(va + k * 2048, kHalf, 1024), IDO, (accumulate || k > 0) ? 1u : 0u);
     };
     for (uint32_t u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
       const Unit U = decode_unit(p, u);
-      for (int i = 0; i < U.nq && ok; ++i) {
-        ok = wait_warp(BAR(S::QFULL + i), qf[i] & 1u, abort_flag, limit, kSiteMmaQFull);
-        ++qf[i];
-      }
-      if (!ok) break;
-      tc_fence_after();
       uint32_t kslot;
       if (!(ok = take_slot(kslot))) break;
-      for (int i = 0; i < U.nq && ok; ++i) ok = issue_s(i, kslot, n_kt == 1);
+      for (int i = 0; i < U.nq && ok; ++i) {
+        if (!(ok = wait_warp(BAR(S::QFULL + i), qf[i] & 1u, abort_flag, limit, kSiteMmaQFull)))
+          break;
+        ++qf[i];
+        tc_fence_after();
+        if (lane == 0) {
+          mma_s(i, kslot);
+          mma_commit(BAR(S::SFULL + i));
+          if (n_kt == 1) mma_commit(BAR(S::QEMPTY + i));  // Q_i read for the last time
+        }
+        __syncwarp();
+      }
       if (!ok) break;
       release(kslot);
       for (int j = 0; j < n_kt && ok; ++j) {
-        if (j + 1 < n_kt) {
-          if (!(ok = take_slot(kslot))) break;
-          for (int i = 0; i < U.nq && ok; ++i) ok = issue_s(i, kslot, j + 2 == n_kt);
-          if (!ok) break;
-          release(kslot);
-        }
+        const bool next = j + 1 < n_kt;
         uint32_t vslot;
         if (!(ok = take_slot(vslot))) break;
-        const uint32_t va = sbase + S::ring0 + vslot * S::kTile;
+        if (next && !(ok = take_slot(kslot))) break;
         for (int i = 0; i < U.nq && ok; ++i) {
+          // P_i(j) in TMEM and O_i rescaled; for j = 0 this also orders the
+          // previous unit's epilogue reads of O_i before the overwrite below.
           if (!(ok = wait_warp(BAR(S::PFULL + i), pfull[i] & 1u, abort_flag, limit,
                                kSiteMmaPFull)))
             break;
           ++pfull[i];
           tc_fence_after();
           if (lane == 0) {
-            const uint32_t pa = sbase + S::p0 + i * S::kP;
-#pragma unroll
-            for (int k = 0; k < 8; ++k) {  // O_i += P_i V_j, 16 keys per MMA
-              const uint32_t aoff = (k / 4) * kHalf + (k % 4) * 32;
-              mma_bf16(tmem + 256 + i * 128, sdesc(pa + aoff, 16, 1024),
-                       sdesc(va + k * 2048, kHalf, 1024), IDO, (j > 0 || k > 0) ? 1u : 0u);
+            mma_pv(i, vslot, j > 0);
+            if (next) {
+              mma_s(i, kslot);
+              mma_commit(BAR(S::SFULL + i));
+              if (j + 2 == n_kt) mma_commit(BAR(S::QEMPTY + i));  // Q_i read for the last time
+            } else {
+              mma_commit(BAR(S::OFULL + i));
             }
-            mma_commit(BAR(S::PVDONE + i));
           }
           __syncwarp();
         }
         if (!ok) break;
         release(vslot);
+        if (next) release(kslot);
       }
     }
     // Drain: every MMA issued has completed before TMEM is released.
@@ -818,10 +845,10 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attn_kernel(const __grid_const
     const uint32_t tl = (uint32_t)(q4 * 32) << 16;
     const uint32_t tS = tmem + tl + i * 128;
     const uint32_t tO = tmem + tl + 256 + i * 128;
-    const uint32_t pbuf = sbase + S::p0 + i * S::kP;  // P_i, 128-byte swizzled K-major
-    uint32_t sfull = 0, pvdone = 0, ostaged = 0, ofree = 0;
+    const uint32_t stg = sbase + S::stg0 + i * kHalf;  // output staging, 128 x 64, swizzled
+    uint32_t sfull = 0, ofull = 0, staged = 0, stgfree = 0;
     const bool leader = (warp % 4 == 0) && lane == 0;
-    bool store_pending = false;  // the previous unit's output store may still read P_i
+    bool stg_busy = false;  // a TMA store may still be reading the staging block
     const float c = p.scale_log2;
     bool ok = true;
     for (uint32_t u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
@@ -839,8 +866,6 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attn_kernel(const __grid_const
         for (int cc = 0; cc < 4; ++cc) tmem_ld32(tS + cc * 32, s[cc]);
 #pragma unroll
         for (int cc = 0; cc < 4; ++cc) tmem_wait_ld(s[cc]);
-        tc_fence_before();
-        mbar_arrive(BAR(S::SFREE + i));  // the next S_i may overwrite these columns
         const int kvalid = key_valid(p, pv, j);
         if (kvalid < 128) {  // padding keys of a partial tile
 #pragma unroll
@@ -866,9 +891,9 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attn_kernel(const __grid_const
         const uint64_t c2 = f2pack(c, c);
         const uint64_t nm2 = f2pack(-m, -m);
         uint64_t rsa = f2pack(0.f, 0.f), rsb = rsa;
-        uint32_t pk[2][32];  // P as bf16 pairs of keys (2c, 2c + 1) in pk[c / 32][c % 32]
 #pragma unroll
-        for (int cc = 0; cc < 4; ++cc)
+        for (int cc = 0; cc < 4; ++cc) {
+          uint32_t pk[16];  // P as bf16 pairs of keys (2e, 2e + 1) of this 32-key chunk
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
             const uint64_t x2 = f2fma(f2pack(__uint_as_float(s[cc][2 * e]),
@@ -884,37 +909,17 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attn_kernel(const __grid_const
             if (e & 1) rsb = f2add(rsb, p2); else rsa = f2add(rsa, p2);
             float p0, p1;
             f2unpack(p2, p0, p1);
-            pk[cc / 2][(cc % 2) * 16 + e] = pack_bf16(p0, p1);
+            pk[e] = pack_bf16(p0, p1);
           }
+          tmem_st16(tS + cc * 16, pk);  // over logits already read
+        }
         float ra0, ra1, rb0, rb1;
         f2unpack(rsa, ra0, ra1);
         f2unpack(rsb, rb0, rb1);
         l = l * alpha + ((ra0 + ra1) + (rb0 + rb1));
-        if (j > 0) {  // P.V of the previous key tile must be done: O is stable, P is free
-          if (!(ok = wait_warp(BAR(S::PVDONE + i), pvdone & 1u, abort_flag, limit,
-                               kSiteSmxPvDone)))
-            break;
-          ++pvdone;
-          tc_fence_after();
-        }
-#if !BASA_DIRECT_STORE
-        if (store_pending) {  // P_i doubled as the last unit's output staging
-          if (leader) {
-            bulk_wait_read0();
-            mbar_arrive(BAR(S::OFREE + i));
-          }
-          if (!(ok = wait_warp(BAR(S::OFREE + i), ofree & 1u, abort_flag, limit, kSiteSmxOFree)))
-            break;
-          ++ofree;
-          store_pending = false;
-        }
-#endif
-#pragma unroll
-        for (int ch = 0; ch < 16; ++ch)  // 8 keys per 16-byte chunk
-          st_shared_v4(pbuf + (ch / 8) * kHalf + swz(r, ch % 8), pk[ch / 8][(ch % 8) * 4],
-                       pk[ch / 8][(ch % 8) * 4 + 1], pk[ch / 8][(ch % 8) * 4 + 2],
-                       pk[ch / 8][(ch % 8) * 4 + 3]);
-        // tcgen05.ld/st are warp-collective: the whole warp rescales if any row needs it
+        // O_i is stable here: S_i(j) was issued after P_i(j-1) V_{j-1}, so its
+        // completion covers that MMA.  tcgen05.ld/st are warp-collective: the
+        // whole warp rescales if any of its rows needs it.
         if (j > 0 && __any_sync(0xffffffffu, alpha < 1.0f)) {
 #pragma unroll
           for (int cc = 0; cc < D / 32; ++cc) {
@@ -932,74 +937,101 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attn_kernel(const __grid_const
             tmem_st32(tO + cc * 32, o);
           }
         }
-        fence_proxy_async();  // P's generic-proxy stores, visible to the MMA
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(BAR(S::PFULL + i));
       }
       if (!ok) break;
-      if (!(ok = wait_warp(BAR(S::PVDONE + i), pvdone & 1u, abort_flag, limit, kSiteSmxPvLast)))
+      // epilogue: O / l -> bf16 -> staging, one 64-column half at a time -> TMA store
+      if (!(ok = wait_warp(BAR(S::OFULL + i), ofull & 1u, abort_flag, limit, kSiteSmxPvLast)))
         break;
-      ++pvdone;
+      ++ofull;
       tc_fence_after();
-#if BASA_DIRECT_STORE
-      // epilogue: O / l -> bf16 -> this thread's token row, written straight from
-      // registers with streaming 16-byte stores
-      const long long n = r < query_valid(p, pv, qt) ? row_token(p, pv, U, qt, r) : -1;
-      uint4* orow = n >= 0 ? reinterpret_cast<uint4*>(p.out + ((((long long)U.b * p.N + n) *
-                                                                p.H + U.h) * D))
-                           : nullptr;
-#endif
       const float inv = 1.0f / l;
       const uint64_t inv2 = f2pack(inv, inv);
+      if (p.warp_stores) {
+        // Warp-staged stores: each warp converts its 32 rows one 64-column half
+        // at a time into its own 4 KB of shared memory (128-byte rows, 16-byte
+        // chunks XOR-swizzled by row), then reads them back so that each 16-byte
+        // store instruction writes four whole 128-byte row segments.
+        const uint32_t wst = sbase + S::stg0 + (uint32_t)(warp - 4) * 4096u;
+        const long long tok = r < query_valid(p, pv, qt) ? row_token(p, pv, U, qt, r) : -1;
 #pragma unroll
-      for (int cc = 0; cc < D / 32; ++cc) {
-        uint32_t o[32];
-        tmem_ld32(tO + cc * 32, o);
-        tmem_wait_ld(o);
+        for (int hf = 0; hf < D / 64; ++hf) {
+          uint32_t o[2][32];
+          tmem_ld32(tO + hf * 64, o[0]);
+          tmem_ld32(tO + hf * 64 + 32, o[1]);
+          tmem_wait_ld(o[0]);
+          tmem_wait_ld(o[1]);
+          uint32_t w[32];
 #pragma unroll
-        for (int v4 = 0; v4 < 4; ++v4) {
-          uint32_t w[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
+          for (int e = 0; e < 32; ++e) {
             float o0, o1;
-            f2unpack(f2mul(f2pack(__uint_as_float(o[v4 * 8 + 2 * e]),
-                                  __uint_as_float(o[v4 * 8 + 2 * e + 1])), inv2), o0, o1);
+            f2unpack(f2mul(f2pack(__uint_as_float(o[e / 16][(2 * e) % 32]),
+                                  __uint_as_float(o[e / 16][(2 * e) % 32 + 1])), inv2), o0, o1);
             w[e] = pack_bf16(o0, o1);
           }
-#if BASA_DIRECT_STORE
-          if (orow) __stcs(orow + cc * 4 + v4, make_uint4(w[0], w[1], w[2], w[3]));
-#else
-          // epilogue: O / l -> bf16 -> staging in P_i (free now) -> TMA store
-          const int col = cc * 32 + v4 * 8;
-          st_shared_v4(pbuf + (col / 64) * kHalf + swz(r, (col % 64) / 8), w[0], w[1], w[2],
-                       w[3]);
-#endif
+#pragma unroll
+          for (int ch = 0; ch < 8; ++ch)
+            st_shared_v4(wst + lane * 128 + ((ch ^ (lane & 7)) << 4), w[4 * ch], w[4 * ch + 1],
+                         w[4 * ch + 2], w[4 * ch + 3]);
+          __syncwarp();
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            const int rr = k * 4 + lane / 8, c = lane % 8;
+            const uint4 val = ld_shared_v4(wst + rr * 128 + ((c ^ (rr & 7)) << 4));
+            const long long t = __shfl_sync(0xffffffffu, tok, rr);
+            if (t >= 0)
+              *reinterpret_cast<uint4*>(p.out + (((long long)U.b * p.N + t) * p.H + U.h) * D +
+                                        hf * 64 + c * 8) = val;
+          }
+          __syncwarp();
         }
       }
-      tc_fence_before();
-#if BASA_DIRECT_STORE
-      if (p.lse && n >= 0)
-        p.lse[((long long)U.b * p.H + U.h) * p.N + n] = (m + __log2f(l)) * 0.69314718055994531f;
-#else
+#pragma unroll
+      for (int hf = 0; hf < (p.warp_stores ? 0 : D / 64); ++hf) {
+        uint32_t o[2][32];
+        tmem_ld32(tO + hf * 64, o[0]);
+        tmem_ld32(tO + hf * 64 + 32, o[1]);
+        tmem_wait_ld(o[0]);
+        tmem_wait_ld(o[1]);
+        uint32_t w[32];
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          float o0, o1;
+          f2unpack(f2mul(f2pack(__uint_as_float(o[e / 16][(2 * e) % 32]),
+                                __uint_as_float(o[e / 16][(2 * e) % 32 + 1])), inv2), o0, o1);
+          w[e] = pack_bf16(o0, o1);
+        }
+        if (stg_busy) {  // the previous store out of this block has read it
+          if (!(ok = wait_warp(BAR(S::STGFREE + i), stgfree & 1u, abort_flag, limit,
+                               kSiteSmxOFree)))
+            break;
+          ++stgfree;
+        }
+#pragma unroll
+        for (int ch = 0; ch < 8; ++ch)  // 8 output columns per 16-byte chunk
+          st_shared_v4(stg + swz(r, ch), w[4 * ch], w[4 * ch + 1], w[4 * ch + 2], w[4 * ch + 3]);
+        fence_proxy_async();
+        mbar_arrive(BAR(S::STAGED + i));
+        if (leader) {
+          if (wait_bounded(BAR(S::STAGED + i), staged & 1u, abort_flag, limit, kSiteSmxOStaged)) {
+            store_half<D>(p, pv, U, qt, hf, stg);
+            bulk_commit();
+            bulk_wait_read0();
+          }
+          mbar_arrive(BAR(S::STGFREE + i));
+        }
+        ++staged;
+        stg_busy = true;
+      }
+      if (!ok) break;
+      tc_fence_before();  // the reads of O_i precede the next unit's first P.V MMA
       if (p.lse && r < query_valid(p, pv, qt)) {
         const long long n = row_token(p, pv, U, qt, r);
         if (n >= 0)
           p.lse[((long long)U.b * p.H + U.h) * p.N + n] = (m + __log2f(l)) * 0.69314718055994531f;
       }
-      fence_proxy_async();
-      mbar_arrive(BAR(S::OSTAGED + i));
-      if (leader) {
-        const bool staged =
-            wait_bounded(BAR(S::OSTAGED + i), ostaged & 1u, abort_flag, limit, kSiteSmxOStaged);
-        if (staged) {
-          store_tile<D>(p, pv, U, qt, pbuf);
-          bulk_commit();
-        }
-      }
-      ++ostaged;
-      store_pending = true;  // waited for before the next unit's first P write
-#endif
     }
   }
 
@@ -1087,6 +1119,8 @@ basa_status build_and_launch(TcParams* prm, const Dims& d, bool flat, const void
   prm->N = d.N;
   prm->lse = lse;
   prm->out = static_cast<__nv_bfloat16*>(out);
+
+
   prm->flags = flags;
   prm->timeout_ns = (unsigned long long)(timeout_ms ? timeout_ms : 2000u) * 1000000ull;
   prm->scale_log2 = d.scale * 1.4426950408889634f;
@@ -1149,6 +1183,9 @@ basa_status build_and_launch(TcParams* prm, const Dims& d, bool flat, const void
     if (units > 0x7fffffffLL) { st = BASA_ERR_UNSUPPORTED; goto done; }
     prm->n_units = (uint32_t)units;
   }
+  // Output path: warp-staged stores, except for windows of more than two key
+  // tiles, where the TMA store boxes measured faster.
+  prm->warp_stores = (flat || prm->n_wkt <= 2) ? 1 : 0;
   st = d.d == 128 ? launch_impl<128>(prm, stream) : launch_impl<64>(prm, stream);
 done:
   return st;

@@ -30,9 +30,9 @@ def _inputs(shape, dtype, seed, q_mult=1.0):
     return q, k, v
 
 
-def _run_window(basa, q, k, v, window, shift, pool=(0, 0, 0), lse=True):
+def _run_window(basa, q, k, v, window, shift, pool=(0, 0, 0), lse=True, flags=0):
     dq, dk, dv = (x.cuda() for x in (q, k, v))
-    out = basa.window_attn(dq, dk, dv, window, shift, pool, return_lse=lse)
+    out = basa.window_attn(dq, dk, dv, window, shift, pool, return_lse=lse, flags=flags)
     if lse:
         o, l = out
         torch.cuda.synchronize()
@@ -42,9 +42,9 @@ def _run_window(basa, q, k, v, window, shift, pool=(0, 0, 0), lse=True):
 
 
 def _check_window(basa, shape, dtype, window, shift, pool=(0, 0, 0), seed=1, q_mult=1.0,
-                  what=""):
+                  what="", flags=0):
     q, k, v = _inputs(shape, dtype, seed, q_mult)
-    out, lse = _run_window(basa, q, k, v, window, shift, pool)
+    out, lse = _run_window(basa, q, k, v, window, shift, pool, flags=flags)
     prm = oracle_params(shape, window, shift, pool)
     ref, ref_lse = oracle.window_attn(oracle.as_f64(q), oracle.as_f64(k), oracle.as_f64(v),
                                       prm, want_lse=True)
