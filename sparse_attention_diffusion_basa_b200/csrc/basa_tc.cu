@@ -397,10 +397,9 @@ enum WaitSite : uint32_t {
   kSiteSmxPvLast, kSiteSmxOStaged, kSiteSmxOFree
 };
 
-__device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity,
-                                             volatile uint32_t* abort_flag, uint64_t limit_ns,
-                                             uint32_t site, bool honour_abort = true) {
-  if (mbar_try_wait(bar, parity)) return true;
+__device__ __noinline__ bool wait_slow(uint32_t bar, uint32_t parity,
+                                       volatile uint32_t* abort_flag, uint64_t limit_ns,
+                                       uint32_t site, bool honour_abort) {
   const long long c0 = clock64();
   const long long climit = (long long)(limit_ns * 2ull);
   for (uint32_t it = 1;; ++it) {
@@ -415,6 +414,12 @@ __device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity,
       }
     }
   }
+}
+__device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity,
+                                             volatile uint32_t* abort_flag, uint64_t limit_ns,
+                                             uint32_t site, bool honour_abort = true) {
+  if (mbar_try_wait(bar, parity)) return true;
+  return wait_slow(bar, parity, abort_flag, limit_ns, site, honour_abort);
 }
 // Warp-uniform variant: every lane waits, and the warp proceeds only if all did.
 __device__ __forceinline__ bool wait_warp(uint32_t bar, uint32_t parity,
@@ -495,6 +500,10 @@ __device__ __forceinline__ int query_valid(const TcParams& p, const PlanView& pv
   return pv.rows[qt];
 }
 
+// x mod G for 0 <= x < 2G: a window origin (below G) plus an offset inside the
+// window (below w <= G).
+__device__ __forceinline__ int wrap(int x, int G) { return x >= G ? x - G : x; }
+
 // kind: 0 = q, 1 = k, 2 = v.  Loads one 128-row tile (all head-dim halves) into
 // shared memory at dst and signals bar with the transaction bytes.
 template <int D>
@@ -515,18 +524,20 @@ __device__ __forceinline__ void load_tile(const TcParams& p, const PlanView& pv,
     return;
   }
   const int b0 = pv.first(U.cls, tile), nb = pv.count(U.cls, tile);
+#pragma unroll 1
   for (int bi = 0; bi < nb; ++bi) {
     const uint32_t e = pv.entries[b0 + bi];
     const int sid = box_shape(e);
-    const int gt = (U.ot + box_lt(e)) % p.T;
-    const int gh = (U.oh + box_lh(e)) % p.Hg;
-    const int gw = (U.ow + box_lw(e)) % p.Wg;
+    const int gt = wrap(U.ot + box_lt(e), p.T);
+    const int gh = wrap(U.oh + box_lh(e), p.Hg);
+    const int gw = wrap(U.ow + box_lw(e), p.Wg);
     const CUtensorMap* m = kind == 0 ? &p.qm[sid] : kind == 1 ? &p.km[sid] : &p.vm[sid];
     const uint32_t d0 = dst + box_row8(e) * 1024;
 #pragma unroll
     for (int hf = 0; hf < NH; ++hf)
       tma_load_5d(d0 + hf * kHalf, m, bar, hf * 64, U.h, gw, gh, U.b * p.T + gt);
   }
+#pragma unroll 1
   for (int r = pv.rows[tile]; r < 128; r += 8) {  // zero rows past the window's tokens
 #pragma unroll
     for (int hf = 0; hf < NH; ++hf)
@@ -546,12 +557,13 @@ __device__ __forceinline__ void store_half(const TcParams& p, const PlanView& pv
     return;
   }
   const int b0 = pv.first(U.cls, qt), nb = pv.count(U.cls, qt);
+#pragma unroll 1
   for (int bi = 0; bi < nb; ++bi) {
     const uint32_t e = pv.entries[b0 + bi];
     const int sid = box_shape(e);
-    const int gt = (U.ot + box_lt(e)) % p.T;
-    const int gh = (U.oh + box_lh(e)) % p.Hg;
-    const int gw = (U.ow + box_lw(e)) % p.Wg;
+    const int gt = wrap(U.ot + box_lt(e), p.T);
+    const int gh = wrap(U.oh + box_lh(e), p.Hg);
+    const int gw = wrap(U.ow + box_lw(e), p.Wg);
     tma_store_5d(&p.om[sid], src + box_row8(e) * 1024, hf * 64, U.h, gw, gh, U.b * p.T + gt);
   }
 }
@@ -561,6 +573,7 @@ __device__ __forceinline__ long long row_token(const TcParams& p, const PlanView
                                                const Unit& U, int qt, int r) {
   if (p.flat) return 128LL * qt + r;
   const int b0 = pv.first(U.cls, qt), nb = pv.count(U.cls, qt);
+#pragma unroll 1
   for (int bi = 0; bi < nb; ++bi) {
     const uint32_t e = pv.entries[b0 + bi];
     const int sid = box_shape(e);
@@ -569,9 +582,9 @@ __device__ __forceinline__ long long row_token(const TcParams& p, const PlanView
     if (r >= r0 && r < r0 + bt * bh * bw) {
       const int idx = r - r0;
       const int it = idx / (bh * bw), ih = (idx / bw) % bh, iw = idx % bw;
-      const int gt = (U.ot + box_lt(e)) % p.T + it;
-      const int gh = (U.oh + box_lh(e)) % p.Hg + ih;
-      const int gw = (U.ow + box_lw(e)) % p.Wg + iw;
+      const int gt = wrap(U.ot + box_lt(e), p.T) + it;
+      const int gh = wrap(U.oh + box_lh(e), p.Hg) + ih;
+      const int gw = wrap(U.ow + box_lw(e), p.Wg) + iw;
       return ((long long)gt * p.Hg + gh) * p.Wg + gw;
     }
   }
