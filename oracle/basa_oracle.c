@@ -29,6 +29,12 @@
  *  - Full attention (the quadratic baseline in the same pages) is the case of
  *    one window covering the whole grid.
  *
+ *  - Joint text + image attention (MM-DiT blocks such as FLUX's): the method
+ *    replaces the *visual* self-attention (same pages, "The BASA Method"), so
+ *    reading used here: image queries attend to their window plus every text
+ *    token, text queries attend to every image and text token, each under one
+ *    softmax.
+ *
  * Arithmetic: every input value is read as a double; dot products, the
  * max-subtracted softmax and the weighted sum are all in double precision.
  *
@@ -156,6 +162,11 @@ static void one_query(const double* q, const double* k, const double* v,
  *            ((t * Hg + y) * Wg + x), or NULL for every query
  * Returns 0, or -1 on an invalid size.
  */
+static int window_attn_keys(const double* q, const double* k, const double* v,
+                            const double* kp, const double* vp, int64_t P, double* out,
+                            double* lse, const oracle_params* p, const int64_t* sel,
+                            int64_t nsel, int nthreads);
+
 int oracle_window_attn(const double* q, const double* k, const double* v,
                        const double* kp, const double* vp, double* out,
                        double* lse, const oracle_params* p, const int64_t* sel,
@@ -166,6 +177,28 @@ int oracle_window_attn(const double* q, const double* k, const double* v,
     if (p->pt <= 0 || p->ph <= 0 || p->pw <= 0) return -1;
     P = (p->T / p->pt) * (p->Hg / p->ph) * (p->Wg / p->pw);
   }
+  return window_attn_keys(q, k, v, kp, vp, P, out, lse, p, sel, nsel, nthreads);
+}
+
+/*
+ * Window attention whose extra keys are nx given tokens kx, vx ([B, nx, H, d])
+ * instead of pooled cells: the visual queries of joint text + image attention
+ * (every image token sees its own window plus every text token, one softmax).
+ */
+int oracle_window_attn_extra(const double* q, const double* k, const double* v,
+                             const double* kx, const double* vx, int64_t nx, double* out,
+                             double* lse, const oracle_params* p, const int64_t* sel,
+                             int64_t nsel, int nthreads) {
+  if (p->T % p->wt || p->Hg % p->wh || p->Wg % p->ww) return -1;
+  if (nx < 0 || (nx > 0 && (!kx || !vx))) return -1;
+  return window_attn_keys(q, k, v, nx ? kx : NULL, nx ? vx : NULL, nx, out, lse, p, sel, nsel,
+                          nthreads);
+}
+
+static int window_attn_keys(const double* q, const double* k, const double* v,
+                            const double* kp, const double* vp, int64_t P, double* out,
+                            double* lse, const oracle_params* p, const int64_t* sel,
+                            int64_t nsel, int nthreads) {
   const int64_t N = p->T * p->Hg * p->Wg;
   const int64_t m = p->wt * p->wh * p->ww;
   const int64_t total = sel ? nsel : p->B * N * p->H;
@@ -194,6 +227,61 @@ int oracle_window_attn(const double* q, const double* k, const double* v,
       double* l = NULL;
       if (lse) l = sel ? lse + i : lse + (b * p->H + h) * N + n;
       one_query(q, k, v, kp, vp, P, p, b, t, y, x, h, z, orow, l);
+    }
+    free(z);
+  }
+  return 0;
+}
+
+/*
+ * The text queries of joint text + image attention: every text query attends
+ * to all N image tokens and all L text tokens under one softmax (plain dense
+ * attention over the concatenated key set; the window restriction applies to
+ * image queries only).
+ *   qt, kt, vt : [B, L, H, d]      k, v : [B, T, Hg, Wg, H, d]
+ *   out_t      : [B, L, H, d]      lse_t: [B, H, L] or NULL
+ */
+int oracle_joint_text_attn(const double* qt, const double* kt, const double* vt,
+                           const double* k, const double* v, int64_t L, double* out_t,
+                           double* lse_t, const oracle_params* p, int nthreads) {
+  if (L < 0) return -1;
+  const int64_t N = p->T * p->Hg * p->Wg, d = p->d, H = p->H;
+  const int64_t total = p->B * L * H;
+#ifdef _OPENMP
+  if (nthreads > 0) omp_set_num_threads(nthreads);
+#else
+  (void)nthreads;
+#endif
+#pragma omp parallel
+  {
+    double* z = (double*)malloc(sizeof(double) * (size_t)(N + L + 1));
+#pragma omp for schedule(dynamic, 16)
+    for (int64_t i = 0; i < total; ++i) {
+      const int64_t b = i / (L * H), lq = (i / H) % L, h = i % H;
+      const double* qv = qt + ((b * L + lq) * H + h) * d;
+      for (int64_t j = 0; j < N + L; ++j) {
+        const double* kv = j < N ? k + ((b * N + j) * H + h) * d
+                                 : kt + ((b * L + (j - N)) * H + h) * d;
+        double s = 0.0;
+        for (int64_t c = 0; c < d; ++c) s += qv[c] * kv[c];
+        z[j] = p->scale * s;
+      }
+      double mx = -INFINITY;
+      for (int64_t j = 0; j < N + L; ++j) mx = z[j] > mx ? z[j] : mx;
+      double den = 0.0;
+      for (int64_t j = 0; j < N + L; ++j) {
+        z[j] = exp(z[j] - mx);
+        den += z[j];
+      }
+      double* orow = out_t + ((b * L + lq) * H + h) * d;
+      for (int64_t c = 0; c < d; ++c) orow[c] = 0.0;
+      for (int64_t j = 0; j < N + L; ++j) {
+        const double* vv = j < N ? v + ((b * N + j) * H + h) * d
+                                 : vt + ((b * L + (j - N)) * H + h) * d;
+        const double a = z[j] / den;
+        for (int64_t c = 0; c < d; ++c) orow[c] += a * vv[c];
+      }
+      if (lse_t) lse_t[(b * H + h) * L + lq] = mx + log(den);
     }
     free(z);
   }

@@ -66,3 +66,34 @@ def brute_window_attn(q, k, v, window, shift=(0, 0, 0), pool=(0, 0, 0), scale=No
         lse = (mx + np.log(den))[..., 0]  # [B, H, N]
         return out, lse
     return out
+
+
+def brute_joint_attn(q, k, v, qt, kt, vt, window, shift=(0, 0, 0), scale=None, want_lse=False):
+    """Joint text + image attention as one dense masked softmax over the
+    concatenated sequence [N image tokens, L text tokens]: image-image pairs keep
+    the same-window mask, every pair that involves a text token is allowed."""
+    q, k, v, qt, kt, vt = (np.asarray(x, dtype=np.float64) for x in (q, k, v, qt, kt, vt))
+    B, T, Hg, Wg, H, d = q.shape
+    N, L = T * Hg * Wg, qt.shape[1]
+    sc = 1.0 / math.sqrt(d) if scale is None else scale
+    it = window_ids(T, window[0], shift[0])
+    iy = window_ids(Hg, window[1], shift[1])
+    ix = window_ids(Wg, window[2], shift[2])
+    wid = np.stack(np.meshgrid(it, iy, ix, indexing="ij"), axis=-1).reshape(N, 3)
+    mask = np.ones((N + L, N + L), dtype=bool)
+    mask[:N, :N] = np.all(wid[:, None, :] == wid[None, :, :], axis=-1)
+    qa = np.concatenate([q.reshape(B, N, H, d), qt], axis=1).transpose(0, 2, 1, 3)
+    ka = np.concatenate([k.reshape(B, N, H, d), kt], axis=1).transpose(0, 2, 1, 3)
+    va = np.concatenate([v.reshape(B, N, H, d), vt], axis=1).transpose(0, 2, 1, 3)
+    z = sc * np.einsum("bhnc,bhjc->bhnj", qa, ka)
+    z = np.where(mask[None, None], z, -np.inf)
+    mx = z.max(axis=-1, keepdims=True)
+    e = np.exp(z - mx)
+    den = e.sum(axis=-1, keepdims=True)
+    o = np.einsum("bhnj,bhjc->bhnc", e / den, va).transpose(0, 2, 1, 3)  # [B, N+L, H, d]
+    out = o[:, :N].reshape(B, T, Hg, Wg, H, d)
+    out_t = o[:, N:]
+    if want_lse:
+        lse = (mx + np.log(den))[..., 0]  # [B, H, N+L]
+        return out, out_t, lse[:, :, :N], lse[:, :, N:]
+    return out, out_t

@@ -71,6 +71,14 @@ def _bind(path):
                                        ctypes.POINTER(ctypes.c_int64),
                                        ctypes.c_int64, ctypes.c_int]
     lib.oracle_window_attn.restype = ctypes.c_int
+    lib.oracle_window_attn_extra.argtypes = [dp, dp, dp, dp, dp, ctypes.c_int64, dp, dp,
+                                             ctypes.POINTER(_CParams),
+                                             ctypes.POINTER(ctypes.c_int64),
+                                             ctypes.c_int64, ctypes.c_int]
+    lib.oracle_window_attn_extra.restype = ctypes.c_int
+    lib.oracle_joint_text_attn.argtypes = [dp, dp, dp, dp, dp, ctypes.c_int64, dp, dp,
+                                           ctypes.POINTER(_CParams), ctypes.c_int]
+    lib.oracle_joint_text_attn.restype = ctypes.c_int
     lib.oracle_max_threads.argtypes = []
     lib.oracle_max_threads.restype = ctypes.c_int
     return lib
@@ -179,3 +187,47 @@ def full_attn(q, k, v, prm: OracleParams, want_lse=False,
     full = OracleParams(prm.B, prm.T, prm.Hg, prm.Wg, prm.H, prm.d,
                         (prm.T, prm.Hg, prm.Wg), (0, 0, 0), (0, 0, 0), prm.scale)
     return window_attn(q, k, v, full, want_lse=want_lse, select=select, threads=threads)
+
+
+def joint_attn(q, k, v, qt, kt, vt, prm: OracleParams, want_lse=False,
+               select: Optional[np.ndarray] = None, threads: int = 0):
+    """Joint text + image attention with shifted windows for the image queries.
+
+    Image queries (``q``, ``[B, T, Hg, Wg, H, d]``) attend to their own shifted
+    window plus every text token; text queries (``qt``, ``[B, L, H, d]``) attend to
+    every image token and every text token; one softmax per query.  ``prm.pool``
+    must be (0, 0, 0): the text tokens take the place of the global memory.
+    ``select`` (rows (b, n, h)) restricts the image outputs as in window_attn;
+    the text outputs are always complete.
+    Returns ``(out, out_t)`` or ``(out, out_t, lse, lse_t)``.
+    """
+    if tuple(prm.pool) != (0, 0, 0):
+        raise ValueError("joint attention takes no pooled memory")
+    q, k, v, qt, kt, vt = (np.ascontiguousarray(x, dtype=np.float64)
+                           for x in (q, k, v, qt, kt, vt))
+    L = qt.shape[1]
+    assert qt.shape == (prm.B, L, prm.H, prm.d) and kt.shape == qt.shape and vt.shape == qt.shape
+    sel_ptr, nsel = None, 0
+    if select is not None:
+        select = np.ascontiguousarray(select, dtype=np.int64).reshape(-1, 3)
+        sel_ptr = select.ctypes.data_as(ctypes.POINTER(ctypes.c_int64))
+        nsel = select.shape[0]
+        out = np.empty((nsel, prm.d))
+        lse = np.empty((nsel,)) if want_lse else None
+    else:
+        out = np.empty(q.shape)
+        lse = np.empty((prm.B, prm.H, prm.N)) if want_lse else None
+    c = prm.c()
+    lib = _load()
+    rc = lib.oracle_window_attn_extra(_ptr(q), _ptr(k), _ptr(v), _ptr(kt) if L else None,
+                                      _ptr(vt) if L else None, L, _ptr(out), _ptr(lse),
+                                      ctypes.byref(c), sel_ptr, nsel, int(threads))
+    if rc != 0:
+        raise ValueError("oracle: window size does not divide the grid")
+    out_t = np.empty(qt.shape)
+    lse_t = np.empty((prm.B, prm.H, L)) if want_lse else None
+    rc = lib.oracle_joint_text_attn(_ptr(qt), _ptr(kt), _ptr(vt), _ptr(k), _ptr(v), L,
+                                    _ptr(out_t), _ptr(lse_t), ctypes.byref(c), int(threads))
+    if rc != 0:
+        raise ValueError("oracle: bad text length")
+    return (out, out_t, lse, lse_t) if want_lse else (out, out_t)

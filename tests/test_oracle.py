@@ -343,3 +343,70 @@ def test_scaled_logits_match_brute_force(oracle_mod):
     want = oracle_mod.brute_window_attn(q, k, v, (1, 4, 4), (0, 2, 2))
     assert np.isfinite(got).all()
     np.testing.assert_allclose(got, want, rtol=0, atol=1e-12)
+
+
+# --------------------------------------------------------------------------
+# joint text + image attention (image queries: window + every text token;
+# text queries: every token)
+# --------------------------------------------------------------------------
+
+JOINT = [
+    ((1, 1, 4, 4, 2, 8), (1, 2, 2), (0, 1, 1), 3),
+    ((2, 2, 4, 6, 1, 8), (1, 2, 3), (1, 1, 2), 5),
+    ((1, 4, 6, 8, 1, 4), (2, 3, 4), (3, 2, 1), 1),
+    ((1, 1, 4, 4, 1, 8), (1, 2, 2), (0, 0, 0), 0),
+]
+
+
+@pytest.mark.parametrize("shape,window,shift,L", JOINT)
+def test_joint_matches_dense_mask_brute_force(oracle_mod, shape, window, shift, L):
+    r = _rng(71)
+    B, T, Hg, Wg, H, d = shape
+    q, k, v = (r.standard_normal(shape) for _ in range(3))
+    qt, kt, vt = (r.standard_normal((B, L, H, d)) for _ in range(3))
+    got = oracle_mod.joint_attn(q, k, v, qt, kt, vt, _P(shape, window, shift), want_lse=True)
+    want = oracle_mod.brute_joint_attn(q, k, v, qt, kt, vt, window, shift, want_lse=True)
+    for g, w in zip(got, want):
+        np.testing.assert_allclose(g, w, rtol=0, atol=1e-12)
+
+
+def test_joint_without_text_is_window_attention(oracle_mod):
+    r = _rng(72)
+    shape = (1, 2, 4, 6, 2, 8)
+    q, k, v = (r.standard_normal(shape) for _ in range(3))
+    empty = np.zeros((1, 0, 2, 8))
+    out, out_t = oracle_mod.joint_attn(q, k, v, empty, empty, empty,
+                                       _P(shape, (1, 2, 3), (1, 1, 1)))
+    want = oracle_mod.window_attn(q, k, v, _P(shape, (1, 2, 3), (1, 1, 1)))
+    np.testing.assert_allclose(out, want, rtol=0, atol=1e-12)
+    assert out_t.shape == (1, 0, 2, 8)
+
+
+def test_joint_with_grid_window_is_full_attention_over_all_tokens(oracle_mod):
+    """One window covering the grid: image and text queries both see every token,
+    so both equal torch's SDPA over the concatenated sequence."""
+    r = _rng(73)
+    shape = (2, 1, 4, 4, 2, 8)
+    B, T, Hg, Wg, H, d = shape
+    N, L = T * Hg * Wg, 6
+    q, k, v = (r.standard_normal(shape) for _ in range(3))
+    qt, kt, vt = (r.standard_normal((B, L, H, d)) for _ in range(3))
+    out, out_t = oracle_mod.joint_attn(q, k, v, qt, kt, vt, _P(shape, (T, Hg, Wg), (0, 1, 2)))
+    cat = lambda a, b: torch.from_numpy(np.concatenate([a.reshape(B, N, H, d), b], axis=1))
+    tq, tk, tv = (cat(a, b).transpose(1, 2) for a, b in ((q, qt), (k, kt), (v, vt)))
+    want = torch.nn.functional.scaled_dot_product_attention(tq, tk, tv).transpose(1, 2).numpy()
+    np.testing.assert_allclose(out, want[:, :N].reshape(shape), rtol=0, atol=1e-12)
+    np.testing.assert_allclose(out_t, want[:, N:], rtol=0, atol=1e-12)
+
+
+def test_joint_zero_text_queries_average_every_value(oracle_mod):
+    r = _rng(74)
+    shape = (1, 1, 4, 4, 1, 8)
+    q, k, v = (r.standard_normal(shape) for _ in range(3))
+    kt, vt = (r.standard_normal((1, 3, 1, 8)) for _ in range(2))
+    qt = np.zeros((1, 3, 1, 8))
+    _, out_t, _, lse_t = oracle_mod.joint_attn(q, k, v, qt, kt, vt, _P(shape, (1, 2, 2)),
+                                               want_lse=True)
+    mean = (v.reshape(16, 8).sum(axis=0) + vt.reshape(3, 8).sum(axis=0)) / 19.0
+    np.testing.assert_allclose(out_t[0, :, 0], np.tile(mean, (3, 1)), rtol=0, atol=1e-12)
+    np.testing.assert_allclose(lse_t, np.log(19.0), rtol=0, atol=1e-12)
