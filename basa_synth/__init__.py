@@ -25,7 +25,8 @@ from typing import Optional, Sequence, Tuple
 import numpy as np
 import torch
 
-__all__ = ["Workload", "WORKLOADS", "make_qkv", "to_storage", "seed_for"]
+__all__ = ["Workload", "WORKLOADS", "make_qkv", "make_text_qkv", "to_storage", "seed_for",
+           "workload_inputs", "text_inputs"]
 
 
 @dataclass(frozen=True)
@@ -44,6 +45,7 @@ class Workload:
     shifts: Tuple[Tuple[int, int, int], ...]  # one (st, sh, sw) per DiT block
     pool: Tuple[int, int, int] = (0, 0, 0)     # (pt, ph, pw); zeros = no global memory
     head_scale: Optional[Tuple[float, float]] = None  # U(lo, hi) per-head |q| factor
+    text: int = 0                   # text tokens of a joint text + image block (0 = none)
 
     @property
     def N(self) -> int:
@@ -86,10 +88,14 @@ WORKLOADS = {
                              (1, 16, 16),
                              ((0, 0, 0), (0, 8, 0), (0, 0, 8), (0, 8, 8)),
                              pool=(1, 4, 4)),
+    # a FLUX-like joint (double-stream) block: 1024^2 image tokens plus 512 text
+    # tokens (the T5 prompt length FLUX uses); q, k, v ~ N(0, 1) for both streams
+    "flux1024_text512": Workload("flux1024_text512", 1, 1, 64, 64, 24, 128, "bf16",
+                                 (1, 16, 16), ((0, 8, 8),), text=512),
 }
 
 WORKLOAD_INDEX = {"grid16_f32": 0, "flux1024": 1, "flux2048": 2, "wan_video": 3,
-                  "flux2048_gm4": 4}
+                  "flux2048_gm4": 4, "flux1024_text512": 5}
 
 
 def seed_for(workload_index: int, block: int, which: str) -> int:
@@ -134,3 +140,21 @@ def workload_inputs(w: Workload, block: int = 0, q_mult: float = 1.0):
     return make_qkv(w.shape(), w.dtype, seed_for(i, block, "q"), seed_for(i, block, "k"),
                     seed_for(i, block, "v"), head_scale=w.head_scale,
                     seed_hs=seed_for(i, block, "head_scale"), q_mult=q_mult)
+
+
+def make_text_qkv(B: int, L: int, H: int, d: int, dtype: str, seed_q: int, seed_k: int,
+                  seed_v: int):
+    """Return CPU text-token tensors (qt, kt, vt) of shape [B, L, H, d]."""
+    def draw(seed):
+        g = np.random.Generator(np.random.PCG64(seed))
+        return g.standard_normal(size=(B, L, H, d), dtype=np.float64)
+
+    return to_storage(draw(seed_q), dtype), to_storage(draw(seed_k), dtype), \
+        to_storage(draw(seed_v), dtype)
+
+
+def text_inputs(w: Workload, block: int = 0):
+    """Seeded text tokens (qt, kt, vt) of a joint workload; seeds offset by 5."""
+    i = WORKLOAD_INDEX.get(w.name, 9)
+    return make_text_qkv(w.B, w.text, w.H, w.d, w.dtype, seed_for(i, block, "q") + 5,
+                         seed_for(i, block, "k") + 5, seed_for(i, block, "v") + 5)

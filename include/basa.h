@@ -155,6 +155,28 @@ BASA_API basa_status basa_window_attn_gm(const void* q, const void* k, const voi
                                 const basa_params* p, cudaStream_t stream);
 
 /*
+ * Joint text + image attention of an MM-DiT block (FLUX-style double-stream
+ * attention) with the visual self-attention replaced by shifted windows.  The
+ * pages ("BASA: Backend-Agnostic Sparse Attention for Fast High-Resolution
+ * Diffusion Transformers", zhichai.net topic 178635722, "The BASA Method") say
+ * the method replaces the *visual* self-attention; the reading taken here for
+ * the text tokens of a joint block:
+ *   - image query p attends to Win(p) plus all L text tokens, one softmax;
+ *   - text query attends to all N image tokens plus all L text tokens.
+ * q, k, v, out: image tokens [B, T, Hg, Wg, H, d]; qt, kt, vt, out_t: text
+ * tokens [B, L, H, d]; lse / lse_t: fp32 [B, H, N] / [B, H, L], or NULL.  Same
+ * dtype for all, 16-byte aligned.  p gives the window and shift; its pool cell
+ * must be (0, 0, 0) (text tokens take the place of the global memory), else
+ * BASA_ERR_UNSUPPORTED.  L = 0 is plain window attention (text pointers
+ * unused).  Two launches on `stream`: the image queries, then the text queries.
+ * Validation happens before the first launch.  The caller owns every buffer.
+ */
+BASA_API basa_status basa_joint_attn(const void* q, const void* k, const void* v,
+                                     const void* qt, const void* kt, const void* vt, int64_t L,
+                                     void* out, void* out_t, float* lse, float* lse_t,
+                                     const basa_params* p, cudaStream_t stream);
+
+/*
  * Full softmax attention over all T*Hg*Wg tokens: the same kernels with one
  * window covering the whole grid (the quadratic baseline of the BASA pages).
  * Window, shift and pool fields of p are ignored.

@@ -154,6 +154,40 @@ def full_attn(q, k, v, scale=None, return_lse=False, out=None, flags=0, stream=N
     return (out, lse) if return_lse else out
 
 
+def joint_attn(q, k, v, qt, kt, vt, window, shift=(0, 0, 0), scale=None, return_lse=False,
+               out=None, out_t=None, flags=0, stream=None):
+    """Joint text + image attention with shifted windows for the image queries.
+
+    q, k, v: image tokens [B, T, Hg, Wg, H, d]; qt, kt, vt: text tokens [B, L, H, d].
+    Image queries attend to their window plus every text token; text queries
+    attend to every token.  Returns (out, out_t) or (out, out_t, lse, lse_t)."""
+    _check_inputs(q, k, v)
+    for t in (qt, kt, vt):
+        if not isinstance(t, torch.Tensor) or t.dtype != q.dtype or t.device != q.device:
+            raise ValueError("text tensors must be torch tensors with q's dtype and device")
+        if not t.is_contiguous():
+            raise ValueError("text tensors must be contiguous [B, L, H, d]")
+    B, T, Hg, Wg, H, d = q.shape
+    if qt.dim() != 4 or qt.shape[0] != B or qt.shape[2:] != (H, d):
+        raise ValueError(f"text tokens must be [B, L, H, d] = [{B}, L, {H}, {d}], got {tuple(qt.shape)}")
+    if kt.shape != qt.shape or vt.shape != qt.shape:
+        raise ValueError("qt, kt and vt must have the same shape")
+    L = qt.shape[1]
+    prm = make_params(q.shape, q.dtype, window, shift, (0, 0, 0), scale, flags)
+    lib = _lib.load()
+    out = torch.empty_like(q) if out is None else out
+    out_t = torch.empty_like(qt) if out_t is None else out_t
+    lse = lse_t = None
+    if return_lse:
+        lse = torch.empty((B, H, T * Hg * Wg), dtype=torch.float32, device=q.device)
+        lse_t = torch.empty((B, H, L), dtype=torch.float32, device=q.device)
+    with torch.cuda.device(q.device):
+        _lib.check(lib.basa_joint_attn(_ptr(q), _ptr(k), _ptr(v), _ptr(qt), _ptr(kt), _ptr(vt),
+                                       int(L), _ptr(out), _ptr(out_t), _ptr(lse), _ptr(lse_t),
+                                       ctypes.byref(prm), _stream(q, stream)), "basa_joint_attn")
+    return (out, out_t, lse, lse_t) if return_lse else (out, out_t)
+
+
 def get_status(stream=None) -> int:
     """Synchronise and return (and clear) the device status code (test use)."""
     s = stream if stream is not None else torch.cuda.current_stream()

@@ -24,6 +24,7 @@ basa_status normalise(const basa_params* p, bool full, Dims* d) {
   d->B = p->B; d->H = p->H; d->T = p->T; d->Hg = p->Hg; d->Wg = p->Wg; d->d = p->d;
   d->dtype = p->dtype;
   d->N = (long long)p->T * p->Hg * p->Wg;
+  d->Nq = d->N;
   d->scale = p->scale > 0.0f ? p->scale : 1.0f / sqrtf((float)p->d);
   if (p->dtype == BASA_F32) {
     if (p->d != 32 && p->d != 64 && p->d != 128) return BASA_ERR_UNSUPPORTED;
@@ -268,6 +269,36 @@ basa_status basa_window_attn_gm(const void* q, const void* k, const void* v, con
   if (!kp || !vp) return BASA_ERR_INVALID_ARG;
   if (misaligned(kp) || misaligned(vp)) return BASA_ERR_ALIGN;
   return attn_common(d, q, k, v, kp, vp, out, lse, p, stream, false);
+}
+
+basa_status basa_joint_attn(const void* q, const void* k, const void* v, const void* qt,
+                            const void* kt, const void* vt, int64_t L, void* out, void* out_t,
+                            float* lse, float* lse_t, const basa_params* p, cudaStream_t stream) {
+  Dims d;
+  basa_status s = normalise(p, false, &d);
+  if (s != BASA_OK) return s;
+  if (d.pt || d.ph || d.pw) return BASA_ERR_UNSUPPORTED;  // text takes the global-memory slot
+  if (L < 0) return BASA_ERR_INVALID_ARG;
+  if (L > (1LL << 24)) return BASA_ERR_UNSUPPORTED;
+  if ((long long)d.B * d.H * d.N == 0) return BASA_OK;
+  if ((s = check_qkvo(q, k, v, out, lse)) != BASA_OK) return s;
+  if (L == 0) return attn_common(d, q, k, v, nullptr, nullptr, out, lse, p, stream, false);
+  if ((s = check_qkvo(qt, kt, vt, out_t, lse_t)) != BASA_OK) return s;
+  // the text-query pass is validated before the image pass is launched
+  Dims dt;
+  if ((s = normalise(p, true, &dt)) != BASA_OK) return s;
+  dt.P = L;
+  dt.Nq = L;
+  dt.qsep = 1;
+  if (d.dtype == BASA_BF16) {
+    TilePlan plan;
+    if ((s = build_tile_plan(d, &plan)) != BASA_OK) return s;
+  }
+  // image queries: their window plus every text token
+  d.P = L;
+  if ((s = attn_common(d, q, k, v, kt, vt, out, lse, p, stream, false)) != BASA_OK) return s;
+  // text queries: every image token plus every text token
+  return attn_common(dt, qt, k, v, kt, vt, out_t, lse_t, p, stream, true);
 }
 
 basa_status basa_full_attn(const void* q, const void* k, const void* v, void* out, float* lse,

@@ -19,7 +19,9 @@ struct Dims {
   int pt, ph, pw;     // pool cell; 0 = none
   int nwt, nwh, nww;  // windows per axis
   long long N;        // tokens per (b, h)
-  long long P;        // pooled tokens per (b, h); 0 = none
+  long long P;        // extra (pooled or text) key tokens per (b, h); 0 = none
+  long long Nq;       // query tokens per (b, h): N, or the text length for text queries
+  int qsep;           // 1: queries are separate rows [B, Nq, H, d] (text queries)
   float scale;
   int dtype;
 };

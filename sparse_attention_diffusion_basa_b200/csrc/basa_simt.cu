@@ -36,6 +36,8 @@ struct SimtArgs {
   int P;            // pooled tokens (0 = none)
   int n_qchunks;    // query chunks per window
   long long N;
+  long long Nq;     // query rows per (b, h) when qsep (text queries)
+  int qsep;         // 1: queries are rows [B, Nq, H, d] against the whole grid
   float scale;
 };
 
@@ -65,11 +67,17 @@ __global__ void __launch_bounds__(kThreads) simt_window_kernel(SimtArgs a) {
 
   const int part = threadIdx.x % TPQ;
   const int lq = qc * QPC + threadIdx.x / TPQ;
-  const bool valid = lq < a.m;
+  const bool valid = a.qsep ? lq < a.Nq : lq < a.m;
   long long qrow = 0;
   long long qn = 0;
   float qr[DPT];
-  if (valid) {
+  if (valid && a.qsep) {  // a text query: its own row, the grid is one window
+    qn = lq;
+    qrow = (long long)b * a.Nq + lq;
+    const float* qp = a.q + (qrow * a.H + h) * D + part * DPT;
+#pragma unroll
+    for (int c = 0; c < DPT; ++c) qr[c] = qp[c];
+  } else if (valid) {
     const int lt = lq / (a.wh * a.ww), lh = (lq / a.ww) % a.wh, lw = lq % a.ww;
     const int t = (ot + lt) % a.T, y = (oh + lh) % a.Hg, x = (ow + lw) % a.Wg;
     qn = ((long long)t * a.Hg + y) * a.Wg + x;
@@ -148,7 +156,8 @@ __global__ void __launch_bounds__(kThreads) simt_window_kernel(SimtArgs a) {
     for (int c = 0; c < DPT; c += 4)
       *reinterpret_cast<float4*>(op + c) =
           make_float4(acc[c] * inv, acc[c + 1] * inv, acc[c + 2] * inv, acc[c + 3] * inv);
-    if (a.lse && part == 0) a.lse[((long long)b * a.H + h) * a.N + qn] = mrun + logf(l);
+    if (a.lse && part == 0) a.lse[((long long)b * a.H + h) * (a.qsep ? a.Nq : a.N) + qn] =
+        mrun + logf(l);
   }
 }
 
@@ -174,11 +183,16 @@ basa_status launch_simt(const Dims& d, const void* q, const void* k, const void*
   a.m = (int)m;
   a.P = kp ? (int)d.P : 0;
   a.N = d.N;
+  a.Nq = d.Nq;
+  a.qsep = d.qsep;
   a.scale = d.scale;
   const int qpc = d.d > 64 ? kThreads / 2 : kThreads;
-  a.n_qchunks = (int)((m + qpc - 1) / qpc);
+  const long long nq = d.qsep ? d.Nq : m;
+  if (nq > (1LL << 30)) return BASA_ERR_UNSUPPORTED;
+  a.n_qchunks = (int)((nq + qpc - 1) / qpc);
   const long long units = (long long)d.B * d.H * d.nwt * d.nwh * d.nww * a.n_qchunks;
   if (units > 0x7fffffffLL) return BASA_ERR_UNSUPPORTED;
+  if (units == 0) return BASA_OK;
   switch (d.d) {
     case 32: simt_window_kernel<32><<<(unsigned)units, kThreads, 0, stream>>>(a); break;
     case 64: simt_window_kernel<64><<<(unsigned)units, kThreads, 0, stream>>>(a); break;

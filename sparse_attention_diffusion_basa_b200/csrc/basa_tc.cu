@@ -73,7 +73,8 @@ struct __align__(64) TcParams {
   __nv_bfloat16* out;  // [B, T, Hg, Wg, H, d]
   int warp_stores;  // output by warp-staged 16-byte stores (1) or by TMA boxes (0)
   uint32_t n_units;
-  long long N;
+  long long N;   // key tokens of the grid per (b, h)
+  long long Nq;  // query (and output) tokens per (b, h): N, or the text length
   unsigned long long timeout_ns;
   int B, H, T, Hg, Wg;
   int wt, wh, ww, st, sh, sw, nwt, nwh, nww;
@@ -484,17 +485,19 @@ struct PlanView {
 
 // Valid rows of key tile j (rows past them are zero-filled and masked).
 __device__ __forceinline__ int key_valid(const TcParams& p, const PlanView& pv, int j) {
+  if (j >= p.n_wkt) {  // extra keys: pooled cells or text tokens
+    const int left = p.P - 128 * (j - p.n_wkt);
+    return left < 128 ? left : 128;
+  }
   if (p.flat) {
     const long long left = p.N - 128LL * j;
     return left < 128 ? (int)left : 128;
   }
-  if (j < p.n_wkt) return pv.rows[j];
-  const int left = p.P - 128 * (j - p.n_wkt);
-  return left < 128 ? left : 128;
+  return pv.rows[j];
 }
 __device__ __forceinline__ int query_valid(const TcParams& p, const PlanView& pv, int qt) {
   if (p.flat) {
-    const long long left = p.N - 128LL * qt;
+    const long long left = p.Nq - 128LL * qt;
     return left < 128 ? (int)left : 128;
   }
   return pv.rows[qt];
@@ -510,17 +513,17 @@ template <int D>
 __device__ __forceinline__ void load_tile(const TcParams& p, const PlanView& pv, int kind,
                                           const Unit& U, int tile, uint32_t dst, uint32_t bar) {
   constexpr int NH = D / 64;
-  if (p.flat) {
-    const CUtensorMap* m = kind == 0 ? &p.qf : kind == 1 ? &p.kf : &p.vf;
-#pragma unroll
-    for (int hf = 0; hf < NH; ++hf) tma_load_4d(dst + hf * kHalf, m, bar, hf * 64, U.h, tile * 128, U.b);
-    return;
-  }
-  if (kind != 0 && tile >= p.n_wkt) {  // pooled global-memory keys
+  if (kind != 0 && tile >= p.n_wkt) {  // extra keys: pooled global memory or text tokens
     const CUtensorMap* m = kind == 1 ? &p.kpf : &p.vpf;
 #pragma unroll
     for (int hf = 0; hf < NH; ++hf)
       tma_load_4d(dst + hf * kHalf, m, bar, hf * 64, U.h, (tile - p.n_wkt) * 128, U.b);
+    return;
+  }
+  if (p.flat) {
+    const CUtensorMap* m = kind == 0 ? &p.qf : kind == 1 ? &p.kf : &p.vf;
+#pragma unroll
+    for (int hf = 0; hf < NH; ++hf) tma_load_4d(dst + hf * kHalf, m, bar, hf * 64, U.h, tile * 128, U.b);
     return;
   }
   const int b0 = pv.first(U.cls, tile), nb = pv.count(U.cls, tile);
@@ -689,8 +692,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attn_kernel(const __grid_const
         prefetch_tmap(&p.vm[sid]); prefetch_tmap(&p.om[sid]);
       }
       prefetch_tmap(&p.fill);
-      if (p.n_pkt) { prefetch_tmap(&p.kpf); prefetch_tmap(&p.vpf); }
     }
+    if (p.n_pkt) { prefetch_tmap(&p.kpf); prefetch_tmap(&p.vpf); }
   }
 
   const bool withhold = (p.flags & BASA_FLAG_TEST_WITHHOLD_LOADS) != 0;
@@ -995,7 +998,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attn_kernel(const __grid_const
             const uint4 val = ld_shared_v4(wst + rr * 128 + ((c ^ (rr & 7)) << 4));
             const long long t = __shfl_sync(0xffffffffu, tok, rr);
             if (t >= 0)
-              *reinterpret_cast<uint4*>(p.out + (((long long)U.b * p.N + t) * p.H + U.h) * D +
+              *reinterpret_cast<uint4*>(p.out + (((long long)U.b * p.Nq + t) * p.H + U.h) * D +
                                         hf * 64 + c * 8) = val;
           }
           __syncwarp();
@@ -1043,7 +1046,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attn_kernel(const __grid_const
       if (p.lse && r < query_valid(p, pv, qt)) {
         const long long n = row_token(p, pv, U, qt, r);
         if (n >= 0)
-          p.lse[((long long)U.b * p.H + U.h) * p.N + n] = (m + __log2f(l)) * 0.69314718055994531f;
+          p.lse[((long long)U.b * p.H + U.h) * p.Nq + n] = (m + __log2f(l)) * 0.69314718055994531f;
       }
     }
   }
@@ -1130,6 +1133,7 @@ basa_status build_and_launch(TcParams* prm, const Dims& d, bool flat, const void
   prm->st = d.st; prm->sh = d.sh; prm->sw = d.sw;
   prm->nwt = d.nwt; prm->nwh = d.nwh; prm->nww = d.nww;
   prm->N = d.N;
+  prm->Nq = d.Nq;
   prm->lse = lse;
   prm->out = static_cast<__nv_bfloat16*>(out);
 
@@ -1141,27 +1145,38 @@ basa_status build_and_launch(TcParams* prm, const Dims& d, bool flat, const void
   prm->P = kp ? (int)d.P : 0;
   TilePlan plan;
   if (!flat && (st = build_tile_plan(d, &plan)) != BASA_OK) goto done;  // before any driver call
-  // flat [d, H, N, B] views (full attention tiles; the fill source)
+  // flat [d, H, N, B] views (full attention tiles; the fill source); the query
+  // and output views hold Nq tokens (the text length for text queries)
   {
     const uint64_t dims[4] = {D, H, (uint64_t)d.N, (uint64_t)d.B};
     const uint64_t strides[3] = {D * 2, H * D * 2, (uint64_t)d.N * H * D * 2};
+    const uint64_t qdims[4] = {D, H, (uint64_t)d.Nq, (uint64_t)d.B};
+    const uint64_t qstrides[3] = {D * 2, H * D * 2, (uint64_t)d.Nq * H * D * 2};
     const uint32_t box128[4] = {64, 1, 128, 1};
     const uint32_t box8[4] = {64, 1, 8, 1};
     if (flat) {
-      if ((st = encode_map(&prm->qf, q, 4, dims, strides, box128)) != BASA_OK) goto done;
+      if ((st = encode_map(&prm->qf, q, 4, qdims, qstrides, box128)) != BASA_OK) goto done;
       if ((st = encode_map(&prm->kf, k, 4, dims, strides, box128)) != BASA_OK) goto done;
       if ((st = encode_map(&prm->vf, v, 4, dims, strides, box128)) != BASA_OK) goto done;
-      if ((st = encode_map(&prm->of, out, 4, dims, strides, box128)) != BASA_OK) goto done;
+      if ((st = encode_map(&prm->of, out, 4, qdims, qstrides, box128)) != BASA_OK) goto done;
     } else {
       if ((st = encode_map(&prm->fill, k, 4, dims, strides, box8)) != BASA_OK) goto done;
     }
   }
+  if (kp) {  // extra keys (pooled cells or text tokens) [d, H, P, B]
+    const uint64_t pdims[4] = {D, H, (uint64_t)d.P, (uint64_t)d.B};
+    const uint64_t pstr[3] = {D * 2, H * D * 2, (uint64_t)d.P * H * D * 2};
+    const uint32_t box128[4] = {64, 1, 128, 1};
+    if ((st = encode_map(&prm->kpf, kp, 4, pdims, pstr, box128)) != BASA_OK) goto done;
+    if ((st = encode_map(&prm->vpf, vp, 4, pdims, pstr, box128)) != BASA_OK) goto done;
+  }
   if (flat) {
     const long long nt = (d.N + 127) / 128;
-    if (nt > (1LL << 24)) { st = BASA_ERR_UNSUPPORTED; goto done; }
-    prm->n_qt = (int)nt;
+    const long long nqt = (d.Nq + 127) / 128;
+    if (nt > (1LL << 24) || nqt > (1LL << 24)) { st = BASA_ERR_UNSUPPORTED; goto done; }
+    prm->n_qt = (int)nqt;
     prm->n_wkt = (int)nt;
-    prm->n_pkt = 0;
+    prm->n_pkt = kp ? (int)((d.P + 127) / 128) : 0;
     prm->n_windows = 1;
     prm->n_pairs = (prm->n_qt + 1) / 2;
     const long long units = (long long)d.B * d.H * prm->n_pairs;
@@ -1178,13 +1193,6 @@ basa_status build_and_launch(TcParams* prm, const Dims& d, bool flat, const void
       if ((st = encode_map(&prm->km[s], k, 5, dims, strides, box)) != BASA_OK) goto done;
       if ((st = encode_map(&prm->vm[s], v, 5, dims, strides, box)) != BASA_OK) goto done;
       if ((st = encode_map(&prm->om[s], out, 5, dims, strides, box)) != BASA_OK) goto done;
-    }
-    if (kp) {
-      const uint64_t pdims[4] = {D, H, (uint64_t)d.P, (uint64_t)d.B};
-      const uint64_t pstr[3] = {D * 2, H * D * 2, (uint64_t)d.P * H * D * 2};
-      const uint32_t box128[4] = {64, 1, 128, 1};
-      if ((st = encode_map(&prm->kpf, kp, 4, pdims, pstr, box128)) != BASA_OK) goto done;
-      if ((st = encode_map(&prm->vpf, vp, 4, pdims, pstr, box128)) != BASA_OK) goto done;
     }
     prm->n_shapes = plan.n_shapes;
     prm->n_qt = plan.n_tiles;
