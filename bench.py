@@ -40,7 +40,7 @@ sys.path.insert(0, ROOT)
 import numpy as np  # noqa: E402
 import torch  # noqa: E402
 
-from basa_synth import WORKLOADS, workload_inputs  # noqa: E402
+from basa_synth import WORKLOADS, text_inputs, workload_inputs  # noqa: E402
 
 METRIC = "window-attn latency (ms) & TFLOPS/% bf16 peak; realised/theoretical N/m speedup"
 DEFAULT_WORKLOAD = "flux2048"
@@ -79,12 +79,18 @@ def _traffic(kernel_key, workload):
 
 
 def workload_numbers(w, shift):
+    """Algorithmic flops and bytes of one step, and the full-attention cost ratio.
+
+    Image queries see m window keys + P pooled + L text keys; text queries see all
+    N + L tokens.  Bytes: q, k, v read and out written once, image and text."""
     B, T, Hg, Wg, H, d = w.shape()
-    N, m, P = w.N, w.m, w.P
-    flops = 4.0 * B * H * N * (m + P) * d
+    N, m, P, L = w.N, w.m, w.P, w.text
+    pairs = N * (m + P + L) + L * (N + L)
+    flops = 4.0 * B * H * d * pairs
     esize = 2 if w.dtype == "bf16" else 4
-    bytes_ = 4.0 * B * H * N * d * esize  # q, k, v read + out written once
-    return flops, bytes_, N, m, P
+    bytes_ = 4.0 * B * H * (N + L) * d * esize
+    theo = (N + L) ** 2 / pairs  # full attention over all tokens / this step
+    return flops, bytes_, N, m, P, theo
 
 
 class ClockSampler:
@@ -314,7 +320,8 @@ def main():
     ws_bytes = basa.workspace_size(w.shape(), dq.dtype, w.window, shift, w.pool)
     ws = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=dev)
     flush = L2Flush(dev)
-    flops, bytes_, N, m, P = workload_numbers(w, shift)
+    flops, bytes_, N, m, P, theo = workload_numbers(w, shift)
+    L = w.text
 
     def step():
         basa.window_attn(dq, dk, dv, w.window, shift, w.pool, out=out,
@@ -323,12 +330,30 @@ def main():
     def step_full():
         basa.full_attn(dq, dk, dv, out=out)
 
+    host_in, host_out = [(qh, dq), (kh, dk), (vh, dv)], [(outh, out)]
+    if L:  # joint text + image block
+        qt, kt, vt = text_inputs(w, blk)
+        dqt, dkt, dvt = (x.to(dev) for x in (qt, kt, vt))
+        out_t = torch.empty_like(dqt)
+        host_in += [(x.pin_memory(), y) for x, y in ((qt, dqt), (kt, dkt), (vt, dvt))]
+        host_out.append((torch.empty_like(qt).pin_memory(), out_t))
+        # full attention over every image and text token, as one flat grid
+        cat = [torch.cat([a.reshape(w.B, N, w.H, w.d), b], 1).reshape(w.B, 1, 1, N + L, w.H, w.d)
+               for a, b in ((dq, dqt), (dk, dkt), (dv, dvt))]
+        out_cat = torch.empty_like(cat[0])
+
+        def step():
+            basa.joint_attn(dq, dk, dv, dqt, dkt, dvt, w.window, shift, out=out, out_t=out_t)
+
+        def step_full():
+            basa.full_attn(*cat, out=out_cat)
+
     def step_e2e():
-        dq.copy_(qh, non_blocking=True)
-        dk.copy_(kh, non_blocking=True)
-        dv.copy_(vh, non_blocking=True)
+        for h, d_ in host_in:
+            d_.copy_(h, non_blocking=True)
         step()
-        outh.copy_(out, non_blocking=True)
+        for h, d_ in host_out:
+            h.copy_(d_, non_blocking=True)
 
     for _ in range(args.warmup):
         step()
@@ -383,8 +408,8 @@ def main():
     per_gpu_tflops = flops / (ms_max * 1e-3) / 1e12
     attn_tflops = flops / (ms_attn * 1e-3) / 1e12   # the attention kernel alone
     gbs = bytes_ / (ms_attn * 1e-3) / 1e9
-    theo = N / (m + P)
-    if m + P >= 2 * 254:   # intensity (m+P)/2 flop per byte above the ridge
+    ridge = peaks["bf16_tflops"] * 1e12 / (peaks["hbm_gbs"] * 1e9)
+    if flops / bytes_ >= ridge:   # arithmetic intensity above the ridge point
         roof = {"bound": "tensor", "achieved": attn_tflops, "peak": peaks["bf16_tflops"],
                 "unit": "TFLOP/s", "frac": attn_tflops / peaks["bf16_tflops"]}
     else:
@@ -402,7 +427,7 @@ def main():
         "data": "synthetic",
         "config": {"workload": f"{w.name}: B={w.B} grid {w.T}x{w.Hg}x{w.Wg} H={w.H} d={w.d} "
                                f"window {'x'.join(map(str, w.window))} shift {shift} "
-                               f"pool {w.pool}",
+                               f"pool {w.pool}" + (f" text {L}" if L else ""),
                    "N": N, "m": m, "P": P, "global_batch": w.B * world,
                    "l2": "evicted before every step (256 MiB write, then 256 MiB read; outside the events)",
                    "parallelism": f"replicas x{world}"},
@@ -411,17 +436,17 @@ def main():
         "speedup": {"full_attn_ms": ms_full, "window_attn_ms": ms_max,
                     "realised": ms_full / ms_max, "theoretical": theo,
                     "ratio": (ms_full / ms_max) / theo,
-                    "full_attn_tflops": 4.0 * w.B * w.H * N * N * w.d / (ms_full * 1e-3) / 1e12},
+                    "full_attn_tflops": 4.0 * w.B * w.H * (N + L) ** 2 * w.d / (ms_full * 1e-3) / 1e12},
         "roofline": roof,
         "e2e": {"value": world * flops / (e2e * 1e-3) / 1e12, "unit": "TFLOP/s",
                 "ms_per_step": e2e,
-                "h2d_bytes_per_step": 3 * dq.numel() * dq.element_size(),
-                "d2h_bytes_per_step": out.numel() * out.element_size()},
+                "h2d_bytes_per_step": sum(h.numel() * h.element_size() for h, _ in host_in),
+                "d2h_bytes_per_step": sum(h.numel() * h.element_size() for h, _ in host_out)},
         "kernels_ms": {"tc_attn_kernel": ms_attn, "pool_kernel": ms_pool},
-        "gpu_launches": args.steps * (2 if w.P else 1),
+        "gpu_launches": args.steps * (2 if (w.P or L) else 1),
         "clocks": clk,
     }
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and not L:
         line["cpu_baseline"] = cpu_baseline(w, shift, q, k, v)
     if rank == 0:
         print(json.dumps(line), flush=True)
