@@ -55,6 +55,7 @@ typedef struct {
   int64_t st, sh, sw;   /* shift per axis */
   int64_t pt, ph, pw;   /* pooled cell size; all zero = no global memory */
   double scale;         /* softmax scale applied to q.k */
+  int64_t Hkv;          /* K/V heads (grouped-query attention); 0 = H */
 } oracle_params;
 
 static int64_t floor_mod(int64_t a, int64_t n) {
@@ -67,6 +68,14 @@ static int64_t tok_index(const oracle_params* p, int64_t b, int64_t t, int64_t y
   return ((((b * p->T + t) * p->Hg + y) * p->Wg + x) * p->H + h) * p->d;
 }
 
+/* K/V tensors have Hkv heads; query head h reads K/V head h / (H / Hkv). */
+static int64_t kv_heads(const oracle_params* p) { return p->Hkv > 0 ? p->Hkv : p->H; }
+static int64_t kv_head(const oracle_params* p, int64_t h) { return h / (p->H / kv_heads(p)); }
+static int64_t kv_index(const oracle_params* p, int64_t b, int64_t t, int64_t y, int64_t x,
+                        int64_t hk) {
+  return ((((b * p->T + t) * p->Hg + y) * p->Wg + x) * kv_heads(p) + hk) * p->d;
+}
+
 /* Mean of x over each pooled cell. */
 void oracle_pool(const double* x, double* xp, const oracle_params* p) {
   const int64_t Pt = p->T / p->pt, Ph = p->Hg / p->ph, Pw = p->Wg / p->pw;
@@ -75,15 +84,15 @@ void oracle_pool(const double* x, double* xp, const oracle_params* p) {
     for (int64_t ct = 0; ct < Pt; ++ct)
       for (int64_t cy = 0; cy < Ph; ++cy)
         for (int64_t cx = 0; cx < Pw; ++cx)
-          for (int64_t h = 0; h < p->H; ++h)
+          for (int64_t h = 0; h < kv_heads(p); ++h)
             for (int64_t c = 0; c < p->d; ++c) {
               double acc = 0.0;
               for (int64_t i = 0; i < p->pt; ++i)
                 for (int64_t j = 0; j < p->ph; ++j)
                   for (int64_t l = 0; l < p->pw; ++l)
-                    acc += x[tok_index(p, b, ct * p->pt + i, cy * p->ph + j,
+                    acc += x[kv_index(p, b, ct * p->pt + i, cy * p->ph + j,
                                        cx * p->pw + l, h) + c];
-              int64_t o = (((((b * Pt + ct) * Ph + cy) * Pw + cx) * p->H + h) * p->d) + c;
+              int64_t o = (((((b * Pt + ct) * Ph + cy) * Pw + cx) * kv_heads(p) + h) * p->d) + c;
               xp[o] = acc * inv;
             }
 }
@@ -113,14 +122,14 @@ static void one_query(const double* q, const double* k, const double* v,
         const int64_t tt = floor_mod(it * p->wt + p->st + lt, p->T);
         const int64_t yy = floor_mod(iy * p->wh + p->sh + ly, p->Hg);
         const int64_t xx = floor_mod(ix * p->ww + p->sw + lx, p->Wg);
-        const double* kv = k + tok_index(p, b, tt, yy, xx, h);
+        const double* kv = k + kv_index(p, b, tt, yy, xx, kv_head(p, h));
         double s = 0.0;
         for (int64_t c = 0; c < d; ++c) s += qv[c] * kv[c];
         z[j++] = p->scale * s;
       }
   /* logits over the pooled tokens */
   for (int64_t c2 = 0; c2 < P; ++c2) {
-    const double* kv = kp + ((b * P + c2) * p->H + h) * d;
+    const double* kv = kp + ((b * P + c2) * kv_heads(p) + kv_head(p, h)) * d;
     double s = 0.0;
     for (int64_t c = 0; c < d; ++c) s += qv[c] * kv[c];
     z[j++] = p->scale * s;
@@ -141,12 +150,12 @@ static void one_query(const double* q, const double* k, const double* v,
         const int64_t tt = floor_mod(it * p->wt + p->st + lt, p->T);
         const int64_t yy = floor_mod(iy * p->wh + p->sh + ly, p->Hg);
         const int64_t xx = floor_mod(ix * p->ww + p->sw + lx, p->Wg);
-        const double* vv = v + tok_index(p, b, tt, yy, xx, h);
+        const double* vv = v + kv_index(p, b, tt, yy, xx, kv_head(p, h));
         const double a = z[j++] / den;
         for (int64_t c = 0; c < d; ++c) out_row[c] += a * vv[c];
       }
   for (int64_t c2 = 0; c2 < P; ++c2) {
-    const double* vv = vp + ((b * P + c2) * p->H + h) * d;
+    const double* vv = vp + ((b * P + c2) * kv_heads(p) + kv_head(p, h)) * d;
     const double a = z[j++] / den;
     for (int64_t c = 0; c < d; ++c) out_row[c] += a * vv[c];
   }
@@ -245,7 +254,7 @@ int oracle_joint_text_attn(const double* qt, const double* kt, const double* vt,
                            const double* k, const double* v, int64_t L, double* out_t,
                            double* lse_t, const oracle_params* p, int nthreads) {
   if (L < 0) return -1;
-  const int64_t N = p->T * p->Hg * p->Wg, d = p->d, H = p->H;
+  const int64_t N = p->T * p->Hg * p->Wg, d = p->d, H = p->H, Hk = kv_heads(p);
   const int64_t total = p->B * L * H;
 #ifdef _OPENMP
   if (nthreads > 0) omp_set_num_threads(nthreads);
@@ -260,8 +269,9 @@ int oracle_joint_text_attn(const double* qt, const double* kt, const double* vt,
       const int64_t b = i / (L * H), lq = (i / H) % L, h = i % H;
       const double* qv = qt + ((b * L + lq) * H + h) * d;
       for (int64_t j = 0; j < N + L; ++j) {
-        const double* kv = j < N ? k + ((b * N + j) * H + h) * d
-                                 : kt + ((b * L + (j - N)) * H + h) * d;
+        const int64_t hk = kv_head(p, h);
+        const double* kv = j < N ? k + ((b * N + j) * Hk + hk) * d
+                                 : kt + ((b * L + (j - N)) * Hk + hk) * d;
         double s = 0.0;
         for (int64_t c = 0; c < d; ++c) s += qv[c] * kv[c];
         z[j] = p->scale * s;
@@ -276,8 +286,9 @@ int oracle_joint_text_attn(const double* qt, const double* kt, const double* vt,
       double* orow = out_t + ((b * L + lq) * H + h) * d;
       for (int64_t c = 0; c < d; ++c) orow[c] = 0.0;
       for (int64_t j = 0; j < N + L; ++j) {
-        const double* vv = j < N ? v + ((b * N + j) * H + h) * d
-                                 : vt + ((b * L + (j - N)) * H + h) * d;
+        const int64_t hk = kv_head(p, h);
+        const double* vv = j < N ? v + ((b * N + j) * Hk + hk) * d
+                                 : vt + ((b * L + (j - N)) * Hk + hk) * d;
         const double a = z[j] / den;
         for (int64_t c = 0; c < d; ++c) orow[c] += a * vv[c];
       }

@@ -20,7 +20,7 @@ from . import build as _build
 class _CParams(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int64) for n in
                 ("B", "H", "T", "Hg", "Wg", "d", "wt", "wh", "ww", "st", "sh", "sw",
-                 "pt", "ph", "pw")] + [("scale", ctypes.c_double)]
+                 "pt", "ph", "pw")] + [("scale", ctypes.c_double), ("Hkv", ctypes.c_int64)]
 
 
 @dataclass
@@ -37,11 +37,16 @@ class OracleParams:
     shift: Tuple[int, int, int] = (0, 0, 0)
     pool: Tuple[int, int, int] = (0, 0, 0)
     scale: Optional[float] = None
+    Hkv: int = 0  # K/V heads (grouped-query attention); 0 = H
 
     def c(self) -> _CParams:
         sc = self.scale if self.scale is not None else 1.0 / math.sqrt(self.d)
         return _CParams(self.B, self.H, self.T, self.Hg, self.Wg, self.d,
-                        *self.window, *self.shift, *self.pool, sc)
+                        *self.window, *self.shift, *self.pool, sc, self.Hkv)
+
+    @property
+    def kv_heads(self) -> int:
+        return self.Hkv if self.Hkv > 0 else self.H
 
     @property
     def N(self) -> int:
@@ -136,7 +141,7 @@ def pool_kv(x: np.ndarray, prm: OracleParams) -> np.ndarray:
     """Mean of x over pooled cells -> [B, T/pt, Hg/ph, Wg/pw, H, d]."""
     x = np.ascontiguousarray(x, dtype=np.float64)
     pt, ph, pw = prm.pool
-    out = np.empty((prm.B, prm.T // pt, prm.Hg // ph, prm.Wg // pw, prm.H, prm.d))
+    out = np.empty((prm.B, prm.T // pt, prm.Hg // ph, prm.Wg // pw, prm.kv_heads, prm.d))
     c = prm.c()
     _load().oracle_pool(_ptr(x), _ptr(out), ctypes.byref(c))
     return out
@@ -185,7 +190,7 @@ def full_attn(q, k, v, prm: OracleParams, want_lse=False,
               select: Optional[np.ndarray] = None, threads: int = 0):
     """Full softmax attention: one window covering the whole grid, no shift."""
     full = OracleParams(prm.B, prm.T, prm.Hg, prm.Wg, prm.H, prm.d,
-                        (prm.T, prm.Hg, prm.Wg), (0, 0, 0), (0, 0, 0), prm.scale)
+                        (prm.T, prm.Hg, prm.Wg), (0, 0, 0), (0, 0, 0), prm.scale, prm.Hkv)
     return window_attn(q, k, v, full, want_lse=want_lse, select=select, threads=threads)
 
 
@@ -206,7 +211,8 @@ def joint_attn(q, k, v, qt, kt, vt, prm: OracleParams, want_lse=False,
     q, k, v, qt, kt, vt = (np.ascontiguousarray(x, dtype=np.float64)
                            for x in (q, k, v, qt, kt, vt))
     L = qt.shape[1]
-    assert qt.shape == (prm.B, L, prm.H, prm.d) and kt.shape == qt.shape and vt.shape == qt.shape
+    assert qt.shape == (prm.B, L, prm.H, prm.d)
+    assert kt.shape == (prm.B, L, prm.kv_heads, prm.d) and vt.shape == kt.shape
     sel_ptr, nsel = None, 0
     if select is not None:
         select = np.ascontiguousarray(select, dtype=np.int64).reshape(-1, 3)

@@ -410,3 +410,47 @@ def test_joint_zero_text_queries_average_every_value(oracle_mod):
     mean = (v.reshape(16, 8).sum(axis=0) + vt.reshape(3, 8).sum(axis=0)) / 19.0
     np.testing.assert_allclose(out_t[0, :, 0], np.tile(mean, (3, 1)), rtol=0, atol=1e-12)
     np.testing.assert_allclose(lse_t, np.log(19.0), rtol=0, atol=1e-12)
+
+
+# --------------------------------------------------------------------------
+# grouped-query attention: K/V heads shared by groups of query heads
+# --------------------------------------------------------------------------
+
+@pytest.mark.parametrize("shape,window,shift,pool,Hkv", [
+    ((1, 1, 4, 8, 4, 8), (1, 2, 4), (0, 1, 2), (0, 0, 0), 2),
+    ((2, 2, 4, 4, 6, 4), (1, 2, 2), (1, 1, 1), (1, 2, 2), 3),
+    ((1, 1, 4, 4, 4, 8), (1, 2, 2), (0, 1, 1), (1, 2, 2), 1),
+])
+def test_grouped_query_equals_repeated_kv_heads(oracle_mod, shape, window, shift, pool, Hkv):
+    """Query head h reading K/V head h / (H / Hkv) is multi-head attention on K/V
+    whose heads are each repeated H / Hkv times."""
+    r = _rng(81)
+    B, T, Hg, Wg, H, d = shape
+    q = r.standard_normal(shape)
+    k, v = (r.standard_normal((B, T, Hg, Wg, Hkv, d)) for _ in range(2))
+    prm = _P(shape, window, shift, pool)
+    prm.Hkv = Hkv
+    got, lse = oracle_mod.window_attn(q, k, v, prm, want_lse=True)
+    rep = lambda x: np.repeat(x, H // Hkv, axis=4)
+    want, want_lse = oracle_mod.window_attn(q, rep(k), rep(v), _P(shape, window, shift, pool),
+                                            want_lse=True)
+    np.testing.assert_allclose(got, want, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(lse, want_lse, rtol=0, atol=1e-12)
+
+
+def test_grouped_query_joint_equals_repeated_kv_heads(oracle_mod):
+    r = _rng(82)
+    shape, Hkv, L = (1, 1, 4, 4, 4, 8), 2, 5
+    B, T, Hg, Wg, H, d = shape
+    q = r.standard_normal(shape)
+    k, v = (r.standard_normal((B, T, Hg, Wg, Hkv, d)) for _ in range(2))
+    qt = r.standard_normal((B, L, H, d))
+    kt, vt = (r.standard_normal((B, L, Hkv, d)) for _ in range(2))
+    prm = _P(shape, (1, 2, 2), (0, 1, 1))
+    prm.Hkv = Hkv
+    got = oracle_mod.joint_attn(q, k, v, qt, kt, vt, prm)
+    rep = lambda x, ax: np.repeat(x, H // Hkv, axis=ax)
+    want = oracle_mod.joint_attn(q, rep(k, 4), rep(v, 4), qt, rep(kt, 2), rep(vt, 2),
+                                 _P(shape, (1, 2, 2), (0, 1, 1)))
+    for g, w in zip(got, want):
+        np.testing.assert_allclose(g, w, rtol=0, atol=1e-12)

@@ -26,13 +26,16 @@ MUTANTS = {
         "const int64_t xx = floor_mod(ix * p->ww + lx, p->Wg);"),
     "no max subtraction": ("z[i] = exp(z[i] - mx);", "z[i] = exp(z[i]);"),
     "rows and columns swapped for keys": (
-        "const double* kv = k + tok_index(p, b, tt, yy, xx, h);",
-        "const double* kv = k + tok_index(p, b, tt, xx % p->Hg, yy % p->Wg, h);"),
+        "const double* kv = k + kv_index(p, b, tt, yy, xx, kv_head(p, h));",
+        "const double* kv = k + kv_index(p, b, tt, xx % p->Hg, yy % p->Wg, kv_head(p, h));"),
     "pooled cells on the shifted origin": (
-        "acc += x[tok_index(p, b, ct * p->pt + i, cy * p->ph + j,\n"
+        "acc += x[kv_index(p, b, ct * p->pt + i, cy * p->ph + j,\n"
         "                                       cx * p->pw + l, h) + c];",
-        "acc += x[tok_index(p, b, ct * p->pt + i, (cy * p->ph + j + 1) % p->Hg,\n"
+        "acc += x[kv_index(p, b, ct * p->pt + i, (cy * p->ph + j + 1) % p->Hg,\n"
         "                                       (cx * p->pw + l + 1) % p->Wg, h) + c];"),
+    "K/V head by modulo instead of by group": (
+        "static int64_t kv_head(const oracle_params* p, int64_t h) { return h / (p->H / kv_heads(p)); }",
+        "static int64_t kv_head(const oracle_params* p, int64_t h) { return h % kv_heads(p); }"),
 }
 
 
@@ -51,6 +54,12 @@ def _pins():
     yield pins.test_pool_factor_one_and_constant_cells, {}
     yield pins.test_support_is_exactly_the_window, {}
     yield pins.test_large_logits_pick_dominant_key, {}
+    yield pins.test_grouped_query_equals_repeated_kv_heads, {
+        "shape": (1, 1, 4, 8, 4, 8), "window": (1, 2, 4), "shift": (0, 1, 2), "pool": (0, 0, 0),
+        "Hkv": 2}
+    for shape, window, shift, L in pins.JOINT:
+        yield pins.test_joint_matches_dense_mask_brute_force, {"shape": shape, "window": window,
+                                                              "shift": shift, "L": L}
 
 
 def _build_mutant(tmp_path, old, new):
