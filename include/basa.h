@@ -104,6 +104,9 @@ typedef struct basa_params {
   int32_t dtype;       /* basa_dtype of q, k, v, out and pooled tensors */
   uint32_t flags;      /* 0, or BASA_FLAG_* test bits */
   uint32_t wait_timeout_ms; /* bound on each device wait; 0 selects 2000 ms */
+  int32_t Hkv;         /* K/V heads (grouped-query attention); 0 selects H.  H must be a
+                          multiple of Hkv; query head h reads K/V head h / (H / Hkv).
+                          k, v and pooled / text K/V then have Hkv heads, q and out H. */
 } basa_params;
 
 /* Human-readable name of a status code (static string). */

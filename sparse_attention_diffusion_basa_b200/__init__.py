@@ -36,13 +36,25 @@ def _triple(x, name) -> Tuple[int, int, int]:
 
 def make_params(shape: Sequence[int], dtype, window=(1, 1, 1), shift=(0, 0, 0),
                 pool=(0, 0, 0), scale: Optional[float] = None, flags: int = 0,
-                wait_timeout_ms: int = 0) -> BasaParams:
+                wait_timeout_ms: int = 0, hkv: int = 0) -> BasaParams:
     B, T, Hg, Wg, H, d = (int(s) for s in shape)
     if isinstance(dtype, torch.dtype):
         dtype = _DT[dtype]
     w, s, p = _triple(window, "window"), _triple(shift, "shift"), _triple(pool, "pool")
     return BasaParams(B, H, T, Hg, Wg, d, *w, *s, *p, float(scale or 0.0), int(dtype),
-                      int(flags), int(wait_timeout_ms))
+                      int(flags), int(wait_timeout_ms), int(hkv))
+
+
+def _kv_heads(q, k, v) -> int:
+    """K/V head count for grouped-query attention (0 when it equals q's)."""
+    if k.shape != v.shape:
+        raise ValueError("k and v must have the same shape")
+    if k.shape[:-2] != q.shape[:-2] or k.shape[-1] != q.shape[-1]:
+        raise ValueError(f"k {tuple(k.shape)} must match q {tuple(q.shape)} except in heads")
+    H, Hkv = q.shape[-2], k.shape[-2]
+    if Hkv == 0 or H % Hkv:
+        raise ValueError(f"q heads {H} must be a multiple of k/v heads {Hkv}")
+    return 0 if Hkv == H else Hkv
 
 
 def _check_inputs(*ts):
@@ -71,9 +83,9 @@ def _stream(t: torch.Tensor, stream=None):
     return ctypes.c_void_p(s.cuda_stream)
 
 
-def workspace_size(shape, dtype, window, shift=(0, 0, 0), pool=(0, 0, 0)) -> int:
+def workspace_size(shape, dtype, window, shift=(0, 0, 0), pool=(0, 0, 0), hkv=0) -> int:
     return int(_lib.load().basa_workspace_size(
-        ctypes.byref(make_params(shape, dtype, window, shift, pool))))
+        ctypes.byref(make_params(shape, dtype, window, shift, pool, hkv=hkv))))
 
 
 def pool_kv(k: torch.Tensor, v: torch.Tensor, pool, out=None, stream=None):
@@ -107,9 +119,8 @@ def window_attn(q, k, v, window, shift=(0, 0, 0), pool=(0, 0, 0), scale=None,
                 stream=None):
     """Shifted local window attention (plus pooled global memory when pool != 0)."""
     _check_inputs(q, k, v)
-    if q.shape != k.shape or q.shape != v.shape:
-        raise ValueError("q, k, v must have the same shape")
-    prm = make_params(q.shape, q.dtype, window, shift, pool, scale, flags, wait_timeout_ms)
+    hkv = _kv_heads(q, k, v)
+    prm = make_params(q.shape, q.dtype, window, shift, pool, scale, flags, wait_timeout_ms, hkv)
     lib = _lib.load()
     out = torch.empty_like(q) if out is None else out
     B, T, Hg, Wg, H, d = q.shape
@@ -128,7 +139,8 @@ def window_attn_gm(q, k, v, kp, vp, window, shift=(0, 0, 0), pool=(1, 1, 1), sca
                    return_lse=False, out=None, flags=0, stream=None):
     """Window attention with caller-supplied pooled global memory kp, vp."""
     _check_inputs(q, k, v, kp, vp)
-    prm = make_params(q.shape, q.dtype, window, shift, pool, scale, flags)
+    hkv = _kv_heads(q, k, v)
+    prm = make_params(q.shape, q.dtype, window, shift, pool, scale, flags, hkv=hkv)
     lib = _lib.load()
     out = torch.empty_like(q) if out is None else out
     B, T, Hg, Wg, H, d = q.shape
@@ -143,7 +155,8 @@ def window_attn_gm(q, k, v, kp, vp, window, shift=(0, 0, 0), pool=(1, 1, 1), sca
 def full_attn(q, k, v, scale=None, return_lse=False, out=None, flags=0, stream=None):
     """Full softmax attention over all grid tokens (one window covering the grid)."""
     _check_inputs(q, k, v)
-    prm = make_params(q.shape, q.dtype, (1, 1, 1), (0, 0, 0), (0, 0, 0), scale, flags)
+    hkv = _kv_heads(q, k, v)
+    prm = make_params(q.shape, q.dtype, (1, 1, 1), (0, 0, 0), (0, 0, 0), scale, flags, hkv=hkv)
     lib = _lib.load()
     out = torch.empty_like(q) if out is None else out
     B, T, Hg, Wg, H, d = q.shape
@@ -162,6 +175,7 @@ def joint_attn(q, k, v, qt, kt, vt, window, shift=(0, 0, 0), scale=None, return_
     Image queries attend to their window plus every text token; text queries
     attend to every token.  Returns (out, out_t) or (out, out_t, lse, lse_t)."""
     _check_inputs(q, k, v)
+    hkv = _kv_heads(q, k, v)
     for t in (qt, kt, vt):
         if not isinstance(t, torch.Tensor) or t.dtype != q.dtype or t.device != q.device:
             raise ValueError("text tensors must be torch tensors with q's dtype and device")
@@ -170,10 +184,10 @@ def joint_attn(q, k, v, qt, kt, vt, window, shift=(0, 0, 0), scale=None, return_
     B, T, Hg, Wg, H, d = q.shape
     if qt.dim() != 4 or qt.shape[0] != B or qt.shape[2:] != (H, d):
         raise ValueError(f"text tokens must be [B, L, H, d] = [{B}, L, {H}, {d}], got {tuple(qt.shape)}")
-    if kt.shape != qt.shape or vt.shape != qt.shape:
-        raise ValueError("qt, kt and vt must have the same shape")
+    if kt.shape != vt.shape or kt.shape != (qt.shape[0], qt.shape[1], k.shape[4], qt.shape[3]):
+        raise ValueError("kt and vt must be [B, L, Hkv, d] with qt's B, L, d and k's heads")
     L = qt.shape[1]
-    prm = make_params(q.shape, q.dtype, window, shift, (0, 0, 0), scale, flags)
+    prm = make_params(q.shape, q.dtype, window, shift, (0, 0, 0), scale, flags, hkv=hkv)
     lib = _lib.load()
     out = torch.empty_like(q) if out is None else out
     out_t = torch.empty_like(qt) if out_t is None else out_t

@@ -28,7 +28,7 @@ class BasaParams(ctypes.Structure):
                 ("B", "H", "T", "Hg", "Wg", "d", "wt", "wh", "ww", "st", "sh", "sw",
                  "pt", "ph", "pw")] + [
         ("scale", ctypes.c_float), ("dtype", ctypes.c_int32), ("flags", ctypes.c_uint32),
-        ("wait_timeout_ms", ctypes.c_uint32)]
+        ("wait_timeout_ms", ctypes.c_uint32), ("Hkv", ctypes.c_int32)]
 
 
 class BasaError(RuntimeError):

@@ -22,6 +22,8 @@ basa_status normalise(const basa_params* p, bool full, Dims* d) {
   if (!(p->scale >= 0.0f) || isinf(p->scale)) return BASA_ERR_INVALID_ARG;
   memset(d, 0, sizeof(*d));
   d->B = p->B; d->H = p->H; d->T = p->T; d->Hg = p->Hg; d->Wg = p->Wg; d->d = p->d;
+  if (p->Hkv < 0 || (p->Hkv > 0 && p->H % p->Hkv != 0)) return BASA_ERR_INVALID_ARG;
+  d->Hkv = p->Hkv > 0 ? p->Hkv : p->H;
   d->dtype = p->dtype;
   d->N = (long long)p->T * p->Hg * p->Wg;
   d->Nq = d->N;
@@ -174,7 +176,7 @@ static size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
 static size_t pooled_bytes(const Dims& d) {
   const size_t es = d.dtype == BASA_BF16 ? 2 : 4;
-  return align256((size_t)d.B * (size_t)d.P * (size_t)d.H * (size_t)d.d * es);
+  return align256((size_t)d.B * (size_t)d.P * (size_t)d.Hkv * (size_t)d.d * es);
 }
 
 extern "C" {

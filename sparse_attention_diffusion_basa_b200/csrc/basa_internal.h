@@ -14,6 +14,7 @@ namespace basa {
 // ---------------------------------------------------------------------------
 struct Dims {
   int B, H, T, Hg, Wg, d;
+  int Hkv;            // K/V heads (H for plain multi-head attention)
   int wt, wh, ww;     // window
   int st, sh, sw;     // shift reduced to [0, w)
   int pt, ph, pw;     // pool cell; 0 = none

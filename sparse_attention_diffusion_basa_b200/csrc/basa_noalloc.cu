@@ -80,7 +80,7 @@ extern "C" basa_status basa_window_attn_noalloc(const void* q, const void* k, co
   const void* vp = nullptr;
   if (d.P > 0) {
     const size_t es = d.dtype == BASA_BF16 ? 2 : 4;
-    const size_t one = (((size_t)d.B * (size_t)d.P * (size_t)d.H * (size_t)d.d * es) + 255) &
+    const size_t one = (((size_t)d.B * (size_t)d.P * (size_t)d.Hkv * (size_t)d.d * es) + 255) &
                        ~(size_t)255;
     if (2 * one > kNoAllocScratchBytes) return BASA_ERR_SCRATCH_LIMIT;
     void* base = nullptr;

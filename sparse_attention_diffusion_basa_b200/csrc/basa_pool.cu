@@ -126,7 +126,7 @@ basa_status launch_pool(const Dims& d, const void* k, const void* v, void* kp, v
   a.pt = d.pt; a.ph = d.ph; a.pw = d.pw;
   a.Pt = d.T / d.pt; a.Ph = d.Hg / d.ph; a.Pw = d.Wg / d.pw;
   const int es = d.dtype == BASA_BF16 ? 2 : 4;
-  a.vec_per_token = d.H * d.d * es / 16;
+  a.vec_per_token = d.Hkv * d.d * es / 16;
   a.inv_count = 1.0f / (float)(d.pt * d.ph * d.pw);
   a.vec_blocks = (a.vec_per_token + kPoolThreads - 1) / kPoolThreads;
   a.P = (int)d.P;

@@ -30,6 +30,7 @@ struct SimtArgs {
   float* out;
   float* lse;       // [B, H, N] or null
   int B, H, T, Hg, Wg;
+  int Hkv;          // K/V heads; query head h reads K/V head h / (H / Hkv)
   int wt, wh, ww, st, sh, sw;
   int nwt, nwh, nww;
   int m;            // tokens per window
@@ -62,6 +63,7 @@ __global__ void __launch_bounds__(kThreads) simt_window_kernel(SimtArgs a) {
   u /= nwin;
   const int h = (int)(u % a.H);
   const int b = (int)(u / a.H);
+  const int hk = h / (a.H / a.Hkv);
   const int jw = win % a.nww, jh = (win / a.nww) % a.nwh, jt = win / (a.nww * a.nwh);
   const int ot = jt * a.wt + a.st, oh = jh * a.wh + a.sh, ow = jw * a.ww + a.sw;
 
@@ -108,12 +110,12 @@ __global__ void __launch_bounds__(kThreads) simt_window_kernel(SimtArgs a) {
         const int lt = j / (a.wh * a.ww), lh = (j / a.ww) % a.wh, lw = j % a.ww;
         const long long row =
             token_row(a, b, (ot + lt) % a.T, (oh + lh) % a.Hg, (ow + lw) % a.Wg);
-        kr = reinterpret_cast<const float4*>(a.k + (row * a.H + h) * D);
-        vr = reinterpret_cast<const float4*>(a.v + (row * a.H + h) * D);
+        kr = reinterpret_cast<const float4*>(a.k + (row * a.Hkv + hk) * D);
+        vr = reinterpret_cast<const float4*>(a.v + (row * a.Hkv + hk) * D);
       } else {
         const long long prow = (long long)b * a.P + (j - a.m);
-        kr = reinterpret_cast<const float4*>(a.kp + (prow * a.H + h) * D);
-        vr = reinterpret_cast<const float4*>(a.vp + (prow * a.H + h) * D);
+        kr = reinterpret_cast<const float4*>(a.kp + (prow * a.Hkv + hk) * D);
+        vr = reinterpret_cast<const float4*>(a.vp + (prow * a.Hkv + hk) * D);
       }
       ks[jj][c4] = kr[c4];
       vs[jj][c4] = vr[c4];
@@ -175,6 +177,7 @@ basa_status launch_simt(const Dims& d, const void* q, const void* k, const void*
   a.out = static_cast<float*>(out);
   a.lse = lse;
   a.B = d.B; a.H = d.H; a.T = d.T; a.Hg = d.Hg; a.Wg = d.Wg;
+  a.Hkv = d.Hkv;
   a.wt = d.wt; a.wh = d.wh; a.ww = d.ww;
   a.st = d.st; a.sh = d.sh; a.sw = d.sw;
   a.nwt = d.nwt; a.nwh = d.nwh; a.nww = d.nww;

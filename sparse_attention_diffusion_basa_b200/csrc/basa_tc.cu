@@ -77,6 +77,7 @@ struct __align__(64) TcParams {
   long long Nq;  // query (and output) tokens per (b, h): N, or the text length
   unsigned long long timeout_ns;
   int B, H, T, Hg, Wg;
+  int group;  // query heads per K/V head
   int wt, wh, ww, st, sh, sw, nwt, nwh, nww;
   int n_windows;
   int n_shapes;
@@ -434,7 +435,7 @@ __device__ __forceinline__ bool wait_warp(uint32_t bar, uint32_t parity,
 // Work-unit decoding
 // ---------------------------------------------------------------------------
 struct Unit {
-  int b, h, pair, cls, ot, oh, ow, nq;
+  int b, h, hk, pair, cls, ot, oh, ow, nq;  // hk: the K/V head of query head h
 };
 
 // Window mode walks the heads fastest: concurrently running CTAs then read the
@@ -465,6 +466,7 @@ __device__ __forceinline__ Unit decode_unit(const TcParams& p, uint32_t u) {
   }
   const int left = p.n_qt - 2 * U.pair;
   U.nq = left < 2 ? left : 2;
+  U.hk = p.group == 1 ? U.h : U.h / p.group;
   return U;
 }
 
@@ -517,13 +519,14 @@ __device__ __forceinline__ void load_tile(const TcParams& p, const PlanView& pv,
     const CUtensorMap* m = kind == 1 ? &p.kpf : &p.vpf;
 #pragma unroll
     for (int hf = 0; hf < NH; ++hf)
-      tma_load_4d(dst + hf * kHalf, m, bar, hf * 64, U.h, (tile - p.n_wkt) * 128, U.b);
+      tma_load_4d(dst + hf * kHalf, m, bar, hf * 64, U.hk, (tile - p.n_wkt) * 128, U.b);
     return;
   }
+  const int head = kind == 0 ? U.h : U.hk;
   if (p.flat) {
     const CUtensorMap* m = kind == 0 ? &p.qf : kind == 1 ? &p.kf : &p.vf;
 #pragma unroll
-    for (int hf = 0; hf < NH; ++hf) tma_load_4d(dst + hf * kHalf, m, bar, hf * 64, U.h, tile * 128, U.b);
+    for (int hf = 0; hf < NH; ++hf) tma_load_4d(dst + hf * kHalf, m, bar, hf * 64, head, tile * 128, U.b);
     return;
   }
   const int b0 = pv.first(U.cls, tile), nb = pv.count(U.cls, tile);
@@ -538,7 +541,7 @@ __device__ __forceinline__ void load_tile(const TcParams& p, const PlanView& pv,
     const uint32_t d0 = dst + box_row8(e) * 1024;
 #pragma unroll
     for (int hf = 0; hf < NH; ++hf)
-      tma_load_5d(d0 + hf * kHalf, m, bar, hf * 64, U.h, gw, gh, U.b * p.T + gt);
+      tma_load_5d(d0 + hf * kHalf, m, bar, hf * 64, head, gw, gh, U.b * p.T + gt);
   }
 #pragma unroll 1
   for (int r = pv.rows[tile]; r < 128; r += 8) {  // zero rows past the window's tokens
@@ -1128,7 +1131,9 @@ basa_status build_and_launch(TcParams* prm, const Dims& d, bool flat, const void
   basa_status st = BASA_OK;
   const uint64_t D = (uint64_t)d.d;
   const uint64_t H = (uint64_t)d.H;
+  const uint64_t Hk = (uint64_t)d.Hkv;
   prm->B = d.B; prm->H = d.H; prm->T = d.T; prm->Hg = d.Hg; prm->Wg = d.Wg;
+  prm->group = d.H / d.Hkv;
   prm->wt = d.wt; prm->wh = d.wh; prm->ww = d.ww;
   prm->st = d.st; prm->sh = d.sh; prm->sw = d.sw;
   prm->nwt = d.nwt; prm->nwh = d.nwh; prm->nww = d.nww;
@@ -1148,8 +1153,8 @@ basa_status build_and_launch(TcParams* prm, const Dims& d, bool flat, const void
   // flat [d, H, N, B] views (full attention tiles; the fill source); the query
   // and output views hold Nq tokens (the text length for text queries)
   {
-    const uint64_t dims[4] = {D, H, (uint64_t)d.N, (uint64_t)d.B};
-    const uint64_t strides[3] = {D * 2, H * D * 2, (uint64_t)d.N * H * D * 2};
+    const uint64_t dims[4] = {D, Hk, (uint64_t)d.N, (uint64_t)d.B};  // k, v (and the fill)
+    const uint64_t strides[3] = {D * 2, Hk * D * 2, (uint64_t)d.N * Hk * D * 2};
     const uint64_t qdims[4] = {D, H, (uint64_t)d.Nq, (uint64_t)d.B};
     const uint64_t qstrides[3] = {D * 2, H * D * 2, (uint64_t)d.Nq * H * D * 2};
     const uint32_t box128[4] = {64, 1, 128, 1};
@@ -1163,9 +1168,9 @@ basa_status build_and_launch(TcParams* prm, const Dims& d, bool flat, const void
       if ((st = encode_map(&prm->fill, k, 4, dims, strides, box8)) != BASA_OK) goto done;
     }
   }
-  if (kp) {  // extra keys (pooled cells or text tokens) [d, H, P, B]
-    const uint64_t pdims[4] = {D, H, (uint64_t)d.P, (uint64_t)d.B};
-    const uint64_t pstr[3] = {D * 2, H * D * 2, (uint64_t)d.P * H * D * 2};
+  if (kp) {  // extra keys (pooled cells or text tokens) [d, Hkv, P, B]
+    const uint64_t pdims[4] = {D, Hk, (uint64_t)d.P, (uint64_t)d.B};
+    const uint64_t pstr[3] = {D * 2, Hk * D * 2, (uint64_t)d.P * Hk * D * 2};
     const uint32_t box128[4] = {64, 1, 128, 1};
     if ((st = encode_map(&prm->kpf, kp, 4, pdims, pstr, box128)) != BASA_OK) goto done;
     if ((st = encode_map(&prm->vpf, vp, 4, pdims, pstr, box128)) != BASA_OK) goto done;
@@ -1187,11 +1192,14 @@ basa_status build_and_launch(TcParams* prm, const Dims& d, bool flat, const void
     const uint64_t dims[5] = {D, H, (uint64_t)d.Wg, (uint64_t)d.Hg, (uint64_t)d.B * d.T};
     const uint64_t strides[4] = {D * 2, H * D * 2, (uint64_t)d.Wg * H * D * 2,
                                  (uint64_t)d.Hg * d.Wg * H * D * 2};
+    const uint64_t kdims[5] = {D, Hk, (uint64_t)d.Wg, (uint64_t)d.Hg, (uint64_t)d.B * d.T};
+    const uint64_t kstrides[4] = {D * 2, Hk * D * 2, (uint64_t)d.Wg * Hk * D * 2,
+                                  (uint64_t)d.Hg * d.Wg * Hk * D * 2};
     for (int s = 0; s < plan.n_shapes; ++s) {
       const uint32_t box[5] = {64, 1, plan.shape_bw[s], plan.shape_bh[s], plan.shape_bt[s]};
       if ((st = encode_map(&prm->qm[s], q, 5, dims, strides, box)) != BASA_OK) goto done;
-      if ((st = encode_map(&prm->km[s], k, 5, dims, strides, box)) != BASA_OK) goto done;
-      if ((st = encode_map(&prm->vm[s], v, 5, dims, strides, box)) != BASA_OK) goto done;
+      if ((st = encode_map(&prm->km[s], k, 5, kdims, kstrides, box)) != BASA_OK) goto done;
+      if ((st = encode_map(&prm->vm[s], v, 5, kdims, kstrides, box)) != BASA_OK) goto done;
       if ((st = encode_map(&prm->om[s], out, 5, dims, strides, box)) != BASA_OK) goto done;
     }
     prm->n_shapes = plan.n_shapes;
