@@ -601,10 +601,10 @@ __device__ __forceinline__ long long row_token(const TcParams& p, const PlanView
 // staging block per query tile, and a ring of K/V tiles.  The probabilities P
 // never touch shared memory: they are written into TMEM over their logits and
 // read from there by the P.V MMA.
-template <int D>
+template <int D, int kRing>
 struct Smem {
   static constexpr int kTile = (D / 64) * kHalf;  // Q/K/V tile bytes
-  static constexpr int NS = D == 128 ? 4 : 8;     // K/V ring slots
+  static constexpr int NS = kRing;                // K/V ring slots
   static constexpr int q0 = 0;
   static constexpr int stg0 = 2 * kTile;
   static constexpr int ring0 = stg0 + 2 * kHalf;
@@ -628,9 +628,9 @@ struct Smem {
 // alternate: while softmax 0 exponentiates S_0(j+1), the tensor core runs
 // P_1(j) V_j and S_1(j+1), and the other way round, so the exponentials of one
 // tile overlap the MMAs of the other.
-template <int D>
+template <int D, int kRing>
 __global__ void __launch_bounds__(kThreads, 1) tc_attn_kernel(const __grid_constant__ TcParams p) {
-  using S = Smem<D>;
+  using S = Smem<D, kRing>;
   constexpr int NS = S::NS;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -1071,16 +1071,16 @@ int sm_count() {
   return n > 0 ? n : 1;
 }
 
-template <int D>
+template <int D, int kRing>
 basa_status launch_impl(TcParams* prm, cudaStream_t stream) {
-  const int smem = Smem<D>::alloc;
-  static_assert(Smem<D>::alloc <= 232448, "shared memory plan exceeds 227 KB");
-  if (cudaFuncSetAttribute(tc_attn_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
-      cudaSuccess)
+  const int smem = Smem<D, kRing>::alloc;
+  static_assert(Smem<D, kRing>::alloc <= 232448, "shared memory plan exceeds 227 KB");
+  if (cudaFuncSetAttribute(tc_attn_kernel<D, kRing>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           smem) != cudaSuccess)
     return BASA_ERR_CUDA;
   long long grid = sm_count();
   if (grid > prm->n_units) grid = prm->n_units;
-  tc_attn_kernel<D><<<(unsigned)grid, kThreads, smem, stream>>>(*prm);
+  tc_attn_kernel<D, kRing><<<(unsigned)grid, kThreads, smem, stream>>>(*prm);
   return cudaGetLastError() == cudaSuccess ? BASA_OK : BASA_ERR_CUDA;
 }
 
@@ -1215,7 +1215,15 @@ basa_status build_and_launch(TcParams* prm, const Dims& d, bool flat, const void
   // Output path: warp-staged stores, except for windows of more than two key
   // tiles, where the TMA store boxes measured faster.
   prm->warp_stores = (flat || prm->n_wkt <= 2) ? 1 : 0;
-  st = d.d == 128 ? launch_impl<128>(prm, stream) : launch_impl<64>(prm, stream);
+  // K/V ring depth: windows of at most two key tiles and no extra keys stream
+  // each K/V tile once per unit and ran faster with 3 slots in flight than with
+  // 4; everything else reuses K/V tiles from L2 and runs faster with 4.
+  if (d.d == 64)
+    st = launch_impl<64, 8>(prm, stream);
+  else if (!flat && prm->n_wkt + prm->n_pkt <= 2)
+    st = launch_impl<128, 3>(prm, stream);
+  else
+    st = launch_impl<128, 4>(prm, stream);
 done:
   return st;
 }
