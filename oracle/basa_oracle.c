@@ -307,3 +307,90 @@ int oracle_max_threads(void) {
   return 1;
 #endif
 }
+
+/*
+ * Gradients of window attention (no global memory) for one output gradient dO:
+ * with P_ij the softmax weights of query i over the keys j of its window,
+ *   dV_j = sum_i P_ij dO_i
+ *   dP_ij = dO_i . V_j,   D_i = dO_i . O_i = sum_j P_ij dP_ij
+ *   dS_ij = P_ij (dP_ij - D_i)
+ *   dQ_i = scale sum_j dS_ij K_j,   dK_j = scale sum_i dS_ij Q_i
+ * (the chain rule through softmax(scale * Q K^T) V restricted to each window).
+ * The forward quantities are recomputed here from q, k, v; nothing is taken
+ * from a forward pass.  All tensors [B, T, Hg, Wg, H, d] (k, v, dk, dv with Hkv
+ * heads; with Hkv < H the query heads of one group add into the same dK, dV).
+ */
+int oracle_window_attn_bwd(const double* q, const double* k, const double* v,
+                           const double* dout, double* dq, double* dk, double* dv,
+                           const oracle_params* p) {
+  if (p->T % p->wt || p->Hg % p->wh || p->Wg % p->ww) return -1;
+  const int64_t d = p->d, N = p->T * p->Hg * p->Wg, m = p->wt * p->wh * p->ww;
+  const int64_t nwt = p->T / p->wt, nwh = p->Hg / p->wh, nww = p->Wg / p->ww;
+  memset(dq, 0, sizeof(double) * (size_t)(p->B * N * p->H * d));
+  memset(dk, 0, sizeof(double) * (size_t)(p->B * N * kv_heads(p) * d));
+  memset(dv, 0, sizeof(double) * (size_t)(p->B * N * kv_heads(p) * d));
+  int64_t* tok = (int64_t*)malloc(sizeof(int64_t) * (size_t)m * 3);
+  double* P = (double*)malloc(sizeof(double) * (size_t)(m * m));
+  double* dS = (double*)malloc(sizeof(double) * (size_t)(m * m));
+  for (int64_t b = 0; b < p->B; ++b)
+    for (int64_t h = 0; h < p->H; ++h) {
+      const int64_t hk = kv_head(p, h);
+      for (int64_t wi = 0; wi < nwt * nwh * nww; ++wi) {
+        const int64_t it = wi / (nwh * nww), iy = (wi / nww) % nwh, ix = wi % nww;
+        int64_t j = 0;  /* members of window (it, iy, ix), enumerated from its id */
+        for (int64_t lt = 0; lt < p->wt; ++lt)
+          for (int64_t ly = 0; ly < p->wh; ++ly)
+            for (int64_t lx = 0; lx < p->ww; ++lx) {
+              tok[3 * j] = floor_mod(it * p->wt + p->st + lt, p->T);
+              tok[3 * j + 1] = floor_mod(iy * p->wh + p->sh + ly, p->Hg);
+              tok[3 * j + 2] = floor_mod(ix * p->ww + p->sw + lx, p->Wg);
+              ++j;
+            }
+        for (int64_t a = 0; a < m; ++a) {  /* query a: softmax row, then dS row */
+          const double* qa = q + tok_index(p, b, tok[3 * a], tok[3 * a + 1], tok[3 * a + 2], h);
+          const double* ga = dout + tok_index(p, b, tok[3 * a], tok[3 * a + 1], tok[3 * a + 2], h);
+          double mx = -INFINITY;
+          for (int64_t c2 = 0; c2 < m; ++c2) {
+            const double* kc = k + kv_index(p, b, tok[3 * c2], tok[3 * c2 + 1], tok[3 * c2 + 2], hk);
+            double s = 0.0;
+            for (int64_t c = 0; c < d; ++c) s += qa[c] * kc[c];
+            P[a * m + c2] = p->scale * s;
+            if (P[a * m + c2] > mx) mx = P[a * m + c2];
+          }
+          double den = 0.0;
+          for (int64_t c2 = 0; c2 < m; ++c2) {
+            P[a * m + c2] = exp(P[a * m + c2] - mx);
+            den += P[a * m + c2];
+          }
+          double Da = 0.0;
+          for (int64_t c2 = 0; c2 < m; ++c2) {
+            P[a * m + c2] /= den;
+            const double* vc = v + kv_index(p, b, tok[3 * c2], tok[3 * c2 + 1], tok[3 * c2 + 2], hk);
+            double dp = 0.0;
+            for (int64_t c = 0; c < d; ++c) dp += ga[c] * vc[c];
+            dS[a * m + c2] = dp;
+            Da += P[a * m + c2] * dp;
+          }
+          for (int64_t c2 = 0; c2 < m; ++c2) dS[a * m + c2] = P[a * m + c2] * (dS[a * m + c2] - Da);
+        }
+        for (int64_t a = 0; a < m; ++a) {
+          double* dqa = dq + tok_index(p, b, tok[3 * a], tok[3 * a + 1], tok[3 * a + 2], h);
+          const double* qa = q + tok_index(p, b, tok[3 * a], tok[3 * a + 1], tok[3 * a + 2], h);
+          const double* ga = dout + tok_index(p, b, tok[3 * a], tok[3 * a + 1], tok[3 * a + 2], h);
+          for (int64_t c2 = 0; c2 < m; ++c2) {
+            const int64_t kvo = kv_index(p, b, tok[3 * c2], tok[3 * c2 + 1], tok[3 * c2 + 2], hk);
+            const double ds = dS[a * m + c2], pw = P[a * m + c2];
+            for (int64_t c = 0; c < d; ++c) {
+              dqa[c] += p->scale * ds * k[kvo + c];
+              dk[kvo + c] += p->scale * ds * qa[c];
+              dv[kvo + c] += pw * ga[c];
+            }
+          }
+        }
+      }
+    }
+  free(tok);
+  free(P);
+  free(dS);
+  return 0;
+}

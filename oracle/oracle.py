@@ -84,6 +84,8 @@ def _bind(path):
     lib.oracle_joint_text_attn.argtypes = [dp, dp, dp, dp, dp, ctypes.c_int64, dp, dp,
                                            ctypes.POINTER(_CParams), ctypes.c_int]
     lib.oracle_joint_text_attn.restype = ctypes.c_int
+    lib.oracle_window_attn_bwd.argtypes = [dp, dp, dp, dp, dp, dp, dp, ctypes.POINTER(_CParams)]
+    lib.oracle_window_attn_bwd.restype = ctypes.c_int
     lib.oracle_max_threads.argtypes = []
     lib.oracle_max_threads.restype = ctypes.c_int
     return lib
@@ -237,3 +239,18 @@ def joint_attn(q, k, v, qt, kt, vt, prm: OracleParams, want_lse=False,
     if rc != 0:
         raise ValueError("oracle: bad text length")
     return (out, out_t, lse, lse_t) if want_lse else (out, out_t)
+
+
+def window_attn_bwd(q, k, v, dout, prm: OracleParams):
+    """Gradients (dq, dk, dv) of window attention (no global memory) for the
+    output gradient ``dout``; the forward is recomputed from q, k, v."""
+    if tuple(prm.pool) != (0, 0, 0):
+        raise ValueError("the backward oracle takes no pooled memory")
+    q, k, v, dout = (np.ascontiguousarray(x, dtype=np.float64) for x in (q, k, v, dout))
+    dq, dk, dv = np.empty(q.shape), np.empty(k.shape), np.empty(v.shape)
+    c = prm.c()
+    rc = _load().oracle_window_attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(dout), _ptr(dq),
+                                        _ptr(dk), _ptr(dv), ctypes.byref(c))
+    if rc != 0:
+        raise ValueError("oracle: window size does not divide the grid")
+    return dq, dk, dv

@@ -454,3 +454,62 @@ def test_grouped_query_joint_equals_repeated_kv_heads(oracle_mod):
                                  _P(shape, (1, 2, 2), (0, 1, 1)))
     for g, w in zip(got, want):
         np.testing.assert_allclose(g, w, rtol=0, atol=1e-12)
+
+
+# --------------------------------------------------------------------------
+# backward: gradients of window attention
+# --------------------------------------------------------------------------
+
+def _dense_mask(T, Hg, Wg, window, shift):
+    from oracle import window_ids
+    it, iy, ix = (window_ids(G, w, s) for G, w, s in zip((T, Hg, Wg), window, shift))
+    wid = np.stack(np.meshgrid(it, iy, ix, indexing="ij"), axis=-1).reshape(-1, 3)
+    return np.all(wid[:, None, :] == wid[None, :, :], axis=-1)
+
+
+@pytest.mark.parametrize("shape,window,shift,Hkv", [
+    ((1, 1, 4, 6, 2, 8), (1, 2, 3), (0, 1, 2), 0),
+    ((2, 4, 6, 4, 2, 4), (2, 3, 2), (1, 2, 1), 0),
+    ((1, 1, 4, 4, 4, 8), (1, 2, 2), (0, 1, 1), 2),
+])
+def test_backward_matches_autograd_of_masked_attention(oracle_mod, shape, window, shift, Hkv):
+    """The oracle's gradients equal torch autograd through masked SDPA (fp64),
+    with the same-window mask, for plain and grouped-query heads."""
+    r = _rng(91)
+    B, T, Hg, Wg, H, d = shape
+    hk = Hkv or H
+    q, g = r.standard_normal(shape), r.standard_normal(shape)
+    k, v = (r.standard_normal((B, T, Hg, Wg, hk, d)) for _ in range(2))
+    prm = _P(shape, window, shift)
+    prm.Hkv = Hkv
+    dq, dk, dv = oracle_mod.window_attn_bwd(q, k, v, g, prm)
+    N = T * Hg * Wg
+    mask = torch.from_numpy(_dense_mask(T, Hg, Wg, window, shift))
+    tq = torch.from_numpy(q).reshape(B, N, H, d).transpose(1, 2).requires_grad_()
+    tk = torch.from_numpy(k).reshape(B, N, hk, d).transpose(1, 2).requires_grad_()
+    tv = torch.from_numpy(v).reshape(B, N, hk, d).transpose(1, 2).requires_grad_()
+    rep = lambda x: x.repeat_interleave(H // hk, dim=1)
+    o = torch.nn.functional.scaled_dot_product_attention(tq, rep(tk), rep(tv), attn_mask=mask)
+    o.backward(torch.from_numpy(g).reshape(B, N, H, d).transpose(1, 2))
+    for got, t in ((dq, tq), (dk, tk), (dv, tv)):
+        want = t.grad.transpose(1, 2).reshape(got.shape).numpy()
+        np.testing.assert_allclose(got, want, rtol=0, atol=1e-12)
+
+
+def test_backward_matches_central_differences(oracle_mod):
+    """d/dx of sum(dO * out) by central differences, at a few coordinates of q, k, v."""
+    r = _rng(92)
+    shape, window, shift = (1, 1, 4, 4, 1, 4), (1, 2, 2), (0, 1, 1)
+    q, k, v, g = (r.standard_normal(shape) for _ in range(4))
+    prm = _P(shape, window, shift)
+    dq, dk, dv = oracle_mod.window_attn_bwd(q, k, v, g, prm)
+    f = lambda q_, k_, v_: float((oracle_mod.window_attn(q_, k_, v_, prm) * g).sum())
+    h = 1e-6
+    for which, grad in ((0, dq), (1, dk), (2, dv)):
+        for idx in [(0, 0, 0, 0, 0, 1), (0, 0, 2, 3, 0, 2), (0, 0, 3, 0, 0, 3)]:
+            args = [q.copy(), k.copy(), v.copy()]
+            args[which][idx] += h
+            up = f(*args)
+            args[which][idx] -= 2 * h
+            dn = f(*args)
+            assert abs((up - dn) / (2 * h) - grad[idx]) < 1e-7

@@ -33,6 +33,9 @@ MUTANTS = {
         "                                       cx * p->pw + l, h) + c];",
         "acc += x[kv_index(p, b, ct * p->pt + i, (cy * p->ph + j + 1) % p->Hg,\n"
         "                                       (cx * p->pw + l + 1) % p->Wg, h) + c];"),
+    "softmax backward without the row term": (
+        "for (int64_t c2 = 0; c2 < m; ++c2) dS[a * m + c2] = P[a * m + c2] * (dS[a * m + c2] - Da);",
+        "for (int64_t c2 = 0; c2 < m; ++c2) dS[a * m + c2] = P[a * m + c2] * dS[a * m + c2];"),
     "K/V head by modulo instead of by group": (
         "static int64_t kv_head(const oracle_params* p, int64_t h) { return h / (p->H / kv_heads(p)); }",
         "static int64_t kv_head(const oracle_params* p, int64_t h) { return h % kv_heads(p); }"),
@@ -57,6 +60,8 @@ def _pins():
     yield pins.test_grouped_query_equals_repeated_kv_heads, {
         "shape": (1, 1, 4, 8, 4, 8), "window": (1, 2, 4), "shift": (0, 1, 2), "pool": (0, 0, 0),
         "Hkv": 2}
+    yield pins.test_backward_matches_autograd_of_masked_attention, {
+        "shape": (1, 1, 4, 6, 2, 8), "window": (1, 2, 3), "shift": (0, 1, 2), "Hkv": 0}
     for shape, window, shift, L in pins.JOINT:
         yield pins.test_joint_matches_dense_mask_brute_force, {"shape": shape, "window": window,
                                                               "shift": shift, "L": L}
