@@ -180,6 +180,29 @@ BASA_API basa_status basa_joint_attn(const void* q, const void* k, const void* v
                                      const basa_params* p, cudaStream_t stream);
 
 /*
+ * Backward of shifted window attention (no global memory): the gradients dq,
+ * dk, dv of basa_window_attn's output for the output gradient dout.  The
+ * dense-teacher adaptation on the pages ("BASA: Backend-Agnostic Sparse
+ * Attention for Fast High-Resolution Diffusion Transformers", zhichai.net topic
+ * 178635722, forum review reply 178634520) trains through this attention.
+ * With P the softmax weights of each query over its window (recomputed from q,
+ * k and the forward's lse) and D_i = dout_i . out_i:
+ *   dS_ij = P_ij (dout_i . v_j - D_i),  dq_i = scale sum_j dS_ij k_j,
+ *   dk_j = scale sum_i dS_ij q_i,  dv_j = sum_i P_ij dout_i.
+ * q, out, dout, dq: [B, T, Hg, Wg, H, d]; k, v, dk, dv: [B, T, Hg, Wg, Hkv, d]
+ * (query heads of one group add into the shared dk, dv); lse: fp32 [B, H, N]
+ * from the forward call; workspace: basa_bwd_workspace_size(p) bytes, 16-byte
+ * aligned.  fp32 arithmetic on CUDA cores for both dtypes; bf16 gradients are
+ * rounded once.  A pool cell in p gives BASA_ERR_UNSUPPORTED.  Three launches
+ * on `stream`; nothing is allocated.
+ */
+BASA_API size_t basa_bwd_workspace_size(const basa_params* p);
+BASA_API basa_status basa_window_attn_bwd(const void* q, const void* k, const void* v,
+                                          const void* out, const void* dout, const float* lse,
+                                          void* dq, void* dk, void* dv, void* workspace,
+                                          const basa_params* p, cudaStream_t stream);
+
+/*
  * Full softmax attention over all T*Hg*Wg tokens: the same kernels with one
  * window covering the whole grid (the quadratic baseline of the BASA pages).
  * Window, shift and pool fields of p are ignored.

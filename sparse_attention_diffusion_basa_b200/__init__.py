@@ -19,8 +19,9 @@ import torch
 from . import _lib
 from ._lib import BasaError, BasaParams, BASA_F32, BASA_BF16  # noqa: F401
 
-__all__ = ["window_attn", "window_attn_gm", "full_attn", "pool_kv", "workspace_size",
-           "get_status", "window_tiles", "make_params", "BasaError", "library_path"]
+__all__ = ["window_attn", "window_attn_gm", "full_attn", "joint_attn", "window_attn_bwd",
+           "pool_kv", "workspace_size", "get_status", "window_tiles", "make_params", "BasaError",
+           "library_path"]
 
 library_path = _lib.LIB_PATH
 
@@ -200,6 +201,29 @@ def joint_attn(q, k, v, qt, kt, vt, window, shift=(0, 0, 0), scale=None, return_
                                        int(L), _ptr(out), _ptr(out_t), _ptr(lse), _ptr(lse_t),
                                        ctypes.byref(prm), _stream(q, stream)), "basa_joint_attn")
     return (out, out_t, lse, lse_t) if return_lse else (out, out_t)
+
+
+def window_attn_bwd(q, k, v, out, dout, lse, window, shift=(0, 0, 0), scale=None,
+                    workspace=None, flags=0, stream=None):
+    """Gradients (dq, dk, dv) of window attention for the output gradient ``dout``.
+
+    ``out`` and ``lse`` are the forward call's output and log-sum-exp."""
+    _check_inputs(q, k, v, out, dout)
+    hkv = _kv_heads(q, k, v)
+    if lse is None or lse.dtype != torch.float32 or not lse.is_contiguous():
+        raise ValueError("lse must be the forward's contiguous fp32 log-sum-exp")
+    prm = make_params(q.shape, q.dtype, window, shift, (0, 0, 0), scale, flags, hkv=hkv)
+    lib = _lib.load()
+    need = int(lib.basa_bwd_workspace_size(ctypes.byref(prm)))
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    with torch.cuda.device(q.device):
+        _lib.check(lib.basa_window_attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(dout),
+                                            _ptr(lse), _ptr(dq), _ptr(dk), _ptr(dv),
+                                            _ptr(workspace), ctypes.byref(prm),
+                                            _stream(q, stream)), "basa_window_attn_bwd")
+    return dq, dk, dv
 
 
 def get_status(stream=None) -> int:

@@ -303,6 +303,30 @@ basa_status basa_joint_attn(const void* q, const void* k, const void* v, const v
   return attn_common(dt, qt, k, v, kt, vt, out_t, lse_t, p, stream, true);
 }
 
+size_t basa_bwd_workspace_size(const basa_params* p) {
+  Dims d;
+  if (normalise(p, false, &d) != BASA_OK) return 0;
+  return align256((size_t)d.B * (size_t)d.H * (size_t)d.N * sizeof(float));
+}
+
+basa_status basa_window_attn_bwd(const void* q, const void* k, const void* v, const void* out,
+                                 const void* dout, const float* lse, void* dq, void* dk,
+                                 void* dv, void* workspace, const basa_params* p,
+                                 cudaStream_t stream) {
+  Dims d;
+  basa_status s = normalise(p, false, &d);
+  if (s != BASA_OK) return s;
+  if (d.pt || d.ph || d.pw) return BASA_ERR_UNSUPPORTED;  // pooled keys: no backward yet
+  if ((long long)d.B * d.H * d.N == 0) return BASA_OK;
+  if ((s = check_qkvo(q, k, v, out, lse)) != BASA_OK) return s;
+  if ((s = check_qkvo(dout, dq, dk, dv, nullptr)) != BASA_OK) return s;
+  if (!lse) return BASA_ERR_INVALID_ARG;
+  if (!workspace) return BASA_ERR_WORKSPACE;
+  if (misaligned(workspace)) return BASA_ERR_ALIGN;
+  return launch_bwd(d, q, k, v, out, dout, lse, static_cast<float*>(workspace), dq, dk, dv,
+                    stream);
+}
+
 basa_status basa_full_attn(const void* q, const void* k, const void* v, void* out, float* lse,
                            const basa_params* p, cudaStream_t stream) {
   Dims d;

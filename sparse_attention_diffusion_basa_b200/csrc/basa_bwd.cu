@@ -1,0 +1,277 @@
+// Backward of shifted local window attention on CUDA cores: dQ, dK, dV for an
+// output gradient dO ("BASA: Backend-Agnostic Sparse Attention for Fast
+// High-Resolution Diffusion Transformers", zhichai.net topic 178635722, "The
+// BASA Method": each query attends to the keys of its own cyclically shifted
+// window; the same pages' review names the dense-teacher adaptation that
+// trains through this attention).
+//
+// With P_ij = exp(scale * q_i . k_j - lse_i) over the keys j of query i's
+// window (lse from the forward pass), and D_i = dO_i . O_i:
+//   dS_ij = P_ij (dO_i . v_j - D_i)
+//   dQ_i  = scale * sum_j dS_ij k_j
+//   dK_j  = scale * sum_i dS_ij q_i      (over the query heads sharing k_j)
+//   dV_j  = sum_i P_ij dO_i
+// Every key of a window is attended only by that window's queries, so each
+// (b, K/V head, window) owns its dK, dV rows: no atomics.  Three launches:
+// D = rowsum(dO * O) into the caller's workspace, then dQ (a group of threads
+// per query, keys staged in shared memory), then dK and dV (a group of threads
+// per key, queries staged; D / 32 threads per row).  Arithmetic is fp32; bf16
+// inputs are widened on load and the gradients rounded once on store.
+#include <cuda_bf16.h>
+#include <math.h>
+
+#include "basa_internal.h"
+
+namespace basa {
+namespace {
+
+constexpr int kBwdThreads = 128;
+constexpr int kChunk = 32;  // keys (or queries) staged per step
+
+struct BwdArgs {
+  const void* q;
+  const void* k;
+  const void* v;
+  const void* o;
+  const void* dout;
+  const float* lse;  // [B, H, N]
+  float* dD;         // [B, H, N] workspace: dO . O
+  void* dq;
+  void* dk;
+  void* dv;
+  int B, H, Hkv, T, Hg, Wg;
+  int wt, wh, ww, st, sh, sw, nwt, nwh, nww;
+  int m;            // tokens per window
+  int n_chunks;     // query (or key) chunks per window
+  long long N;
+  float scale;
+};
+
+template <bool BF16>
+__device__ __forceinline__ float ld1(const void* base, long long i) {
+  if (BF16) return __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(base)[i]);
+  return reinterpret_cast<const float*>(base)[i];
+}
+template <bool BF16>
+__device__ __forceinline__ void st1(void* base, long long i, float x) {
+  if (BF16)
+    reinterpret_cast<__nv_bfloat16*>(base)[i] = __float2bfloat16_rn(x);
+  else
+    reinterpret_cast<float*>(base)[i] = x;
+}
+
+// Flattened grid token of member j of window (jt, jh, jw).
+__device__ __forceinline__ long long member(const BwdArgs& a, int jt, int jh, int jw, int j) {
+  const int lt = j / (a.wh * a.ww), lh = (j / a.ww) % a.wh, lw = j % a.ww;
+  int t = jt * a.wt + a.st + lt, y = jh * a.wh + a.sh + lh, x = jw * a.ww + a.sw + lw;
+  t = t >= a.T ? t - a.T : t;
+  y = y >= a.Hg ? y - a.Hg : y;
+  x = x >= a.Wg ? x - a.Wg : x;
+  return ((long long)t * a.Hg + y) * a.Wg + x;
+}
+
+// D = rowsum(dO * O) for every (b, n, h).
+template <bool BF16, int D>
+__global__ void __launch_bounds__(kBwdThreads) bwd_prep_kernel(BwdArgs a) {
+  const long long rows = (long long)a.B * a.N * a.H;
+  const long long r = (long long)blockIdx.x * kBwdThreads + threadIdx.x;
+  if (r >= rows) return;
+  float acc = 0.f;
+  for (int c = 0; c < D; ++c) acc = fmaf(ld1<BF16>(a.dout, r * D + c), ld1<BF16>(a.o, r * D + c), acc);
+  const long long h = r % a.H, n = (r / a.H) % a.N, b = r / (a.H * a.N);
+  a.dD[(b * a.H + h) * a.N + n] = acc;
+}
+
+// Sum of x over the TPQ consecutive lanes that share one query (or key).
+template <int TPQ>
+__device__ __forceinline__ float lane_sum(float x) {
+#pragma unroll
+  for (int o = 1; o < TPQ; o <<= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+  return x;
+}
+
+// dQ: one CTA per (b, h, window, query chunk); D / 32 threads per query.
+template <bool BF16, int D>
+__global__ void __launch_bounds__(kBwdThreads) bwd_dq_kernel(BwdArgs a) {
+  constexpr int TPQ = D / 32;
+  constexpr int DPT = D / TPQ;
+  constexpr int QPC = kBwdThreads / TPQ;
+  __shared__ float ks[kChunk][D];
+  __shared__ float vs[kChunk][D];
+  long long u = blockIdx.x;
+  const int qc = (int)(u % a.n_chunks);
+  u /= a.n_chunks;
+  const int nwin = a.nwt * a.nwh * a.nww;
+  const int win = (int)(u % nwin);
+  u /= nwin;
+  const int h = (int)(u % a.H);
+  const int b = (int)(u / a.H);
+  const int hk = h / (a.H / a.Hkv);
+  const int jw = win % a.nww, jh = (win / a.nww) % a.nwh, jt = win / (a.nww * a.nwh);
+  const int part = threadIdx.x % TPQ;
+  const int lq = qc * QPC + threadIdx.x / TPQ;
+  const bool valid = lq < a.m;
+  float qr[DPT], gr[DPT], acc[DPT];
+  float lse = 0.f, dd = 0.f;
+  long long qrow = 0;
+  if (valid) {
+    const long long n = member(a, jt, jh, jw, lq);
+    qrow = (((long long)b * a.N + n) * a.H + h) * D + part * DPT;
+    for (int c = 0; c < DPT; ++c) {
+      qr[c] = ld1<BF16>(a.q, qrow + c);
+      gr[c] = ld1<BF16>(a.dout, qrow + c);
+    }
+    lse = a.lse[((long long)b * a.H + h) * a.N + n];
+    dd = a.dD[((long long)b * a.H + h) * a.N + n];
+  } else {
+    for (int c = 0; c < DPT; ++c) qr[c] = gr[c] = 0.f;
+  }
+  for (int c = 0; c < DPT; ++c) acc[c] = 0.f;
+  for (int k0 = 0; k0 < a.m; k0 += kChunk) {
+    const int nk = a.m - k0 < kChunk ? a.m - k0 : kChunk;
+    __syncthreads();
+    for (int idx = threadIdx.x; idx < nk * D; idx += kBwdThreads) {
+      const int jj = idx / D, c = idx % D;
+      const long long n = member(a, jt, jh, jw, k0 + jj);
+      const long long off = (((long long)b * a.N + n) * a.Hkv + hk) * D + c;
+      ks[jj][c] = ld1<BF16>(a.k, off);
+      vs[jj][c] = ld1<BF16>(a.v, off);
+    }
+    __syncthreads();
+    for (int jj = 0; jj < nk; ++jj) {
+      float s = 0.f, dp = 0.f;
+      for (int c = 0; c < DPT; ++c) {
+        s = fmaf(qr[c], ks[jj][part * DPT + c], s);
+        dp = fmaf(gr[c], vs[jj][part * DPT + c], dp);
+      }
+      s = lane_sum<TPQ>(s);
+      dp = lane_sum<TPQ>(dp);
+      const float pw = expf(s * a.scale - lse);
+      const float ds = pw * (dp - dd);
+      for (int c = 0; c < DPT; ++c) acc[c] = fmaf(ds, ks[jj][part * DPT + c], acc[c]);
+    }
+  }
+  if (valid)
+    for (int c = 0; c < DPT; ++c) st1<BF16>(a.dq, qrow + c, acc[c] * a.scale);
+}
+
+// dK, dV: one CTA per (b, K/V head, window, key chunk); the queries of every
+// head of the group are staged in turn.
+template <bool BF16, int D>
+__global__ void __launch_bounds__(kBwdThreads) bwd_dkv_kernel(BwdArgs a) {
+  constexpr int TPQ = D / 32;
+  constexpr int DPT = D / TPQ;
+  constexpr int KPC = kBwdThreads / TPQ;
+  __shared__ float qs[kChunk][D];
+  __shared__ float gs[kChunk][D];
+  __shared__ float ls[kChunk], ds_[kChunk];
+  long long u = blockIdx.x;
+  const int kc = (int)(u % a.n_chunks);
+  u /= a.n_chunks;
+  const int nwin = a.nwt * a.nwh * a.nww;
+  const int win = (int)(u % nwin);
+  u /= nwin;
+  const int hk = (int)(u % a.Hkv);
+  const int b = (int)(u / a.Hkv);
+  const int group = a.H / a.Hkv;
+  const int jw = win % a.nww, jh = (win / a.nww) % a.nwh, jt = win / (a.nww * a.nwh);
+  const int part = threadIdx.x % TPQ;
+  const int lk = kc * KPC + threadIdx.x / TPQ;
+  const bool valid = lk < a.m;
+  float kr[DPT], vr[DPT], dk[DPT], dv[DPT];
+  long long krow = 0;
+  if (valid) {
+    const long long n = member(a, jt, jh, jw, lk);
+    krow = (((long long)b * a.N + n) * a.Hkv + hk) * D + part * DPT;
+    for (int c = 0; c < DPT; ++c) {
+      kr[c] = ld1<BF16>(a.k, krow + c);
+      vr[c] = ld1<BF16>(a.v, krow + c);
+    }
+  } else {
+    for (int c = 0; c < DPT; ++c) kr[c] = vr[c] = 0.f;
+  }
+  for (int c = 0; c < DPT; ++c) dk[c] = dv[c] = 0.f;
+  for (int h = hk * group; h < (hk + 1) * group; ++h) {
+    for (int q0 = 0; q0 < a.m; q0 += kChunk) {
+      const int nq = a.m - q0 < kChunk ? a.m - q0 : kChunk;
+      __syncthreads();
+      for (int idx = threadIdx.x; idx < nq * D; idx += kBwdThreads) {
+        const int ii = idx / D, c = idx % D;
+        const long long n = member(a, jt, jh, jw, q0 + ii);
+        const long long off = (((long long)b * a.N + n) * a.H + h) * D + c;
+        qs[ii][c] = ld1<BF16>(a.q, off);
+        gs[ii][c] = ld1<BF16>(a.dout, off);
+        if (c == 0) {
+          ls[ii] = a.lse[((long long)b * a.H + h) * a.N + n];
+          ds_[ii] = a.dD[((long long)b * a.H + h) * a.N + n];
+        }
+      }
+      __syncthreads();
+      for (int ii = 0; ii < nq; ++ii) {
+        float s = 0.f, dp = 0.f;
+        for (int c = 0; c < DPT; ++c) {
+          s = fmaf(qs[ii][part * DPT + c], kr[c], s);
+          dp = fmaf(gs[ii][part * DPT + c], vr[c], dp);
+        }
+        s = lane_sum<TPQ>(s);
+        dp = lane_sum<TPQ>(dp);
+        const float pw = expf(s * a.scale - ls[ii]);
+        const float dsv = pw * (dp - ds_[ii]);
+        for (int c = 0; c < DPT; ++c) {
+          dk[c] = fmaf(dsv, qs[ii][part * DPT + c], dk[c]);
+          dv[c] = fmaf(pw, gs[ii][part * DPT + c], dv[c]);
+        }
+      }
+    }
+  }
+  if (valid)
+    for (int c = 0; c < DPT; ++c) {
+      st1<BF16>(a.dk, krow + c, dk[c] * a.scale);
+      st1<BF16>(a.dv, krow + c, dv[c]);
+    }
+}
+
+template <bool BF16, int D>
+basa_status launch_bwd_typed(BwdArgs& a, const Dims& d, cudaStream_t stream) {
+  const long long rows = (long long)d.B * d.N * d.H;
+  const long long nwin = (long long)d.nwt * d.nwh * d.nww;
+  constexpr int per = kBwdThreads / (D / 32);  // queries (keys) per CTA
+  a.n_chunks = (a.m + per - 1) / per;
+  const long long dq_blocks = (long long)d.B * d.H * nwin * a.n_chunks;
+  const long long dkv_blocks = (long long)d.B * d.Hkv * nwin * a.n_chunks;
+  if ((rows + kBwdThreads - 1) / kBwdThreads > 0x7fffffffLL || dq_blocks > 0x7fffffffLL)
+    return BASA_ERR_UNSUPPORTED;
+  bwd_prep_kernel<BF16, D><<<(unsigned)((rows + kBwdThreads - 1) / kBwdThreads), kBwdThreads, 0,
+                             stream>>>(a);
+  bwd_dq_kernel<BF16, D><<<(unsigned)dq_blocks, kBwdThreads, 0, stream>>>(a);
+  bwd_dkv_kernel<BF16, D><<<(unsigned)dkv_blocks, kBwdThreads, 0, stream>>>(a);
+  return cudaGetLastError() == cudaSuccess ? BASA_OK : BASA_ERR_CUDA;
+}
+
+}  // namespace
+
+basa_status launch_bwd(const Dims& d, const void* q, const void* k, const void* v,
+                       const void* o, const void* dout, const float* lse, float* dD, void* dq,
+                       void* dk, void* dv, cudaStream_t stream) {
+  BwdArgs a;
+  a.q = q; a.k = k; a.v = v; a.o = o; a.dout = dout; a.lse = lse; a.dD = dD;
+  a.dq = dq; a.dk = dk; a.dv = dv;
+  a.B = d.B; a.H = d.H; a.Hkv = d.Hkv; a.T = d.T; a.Hg = d.Hg; a.Wg = d.Wg;
+  a.wt = d.wt; a.wh = d.wh; a.ww = d.ww;
+  a.st = d.st; a.sh = d.sh; a.sw = d.sw;
+  a.nwt = d.nwt; a.nwh = d.nwh; a.nww = d.nww;
+  const long long m = (long long)d.wt * d.wh * d.ww;
+  if (m > (1LL << 30)) return BASA_ERR_UNSUPPORTED;
+  a.m = (int)m;
+  a.N = d.N;
+  a.scale = d.scale;
+  const bool bf = d.dtype == BASA_BF16;
+  switch (d.d) {
+    case 32: return bf ? launch_bwd_typed<true, 32>(a, d, stream) : launch_bwd_typed<false, 32>(a, d, stream);
+    case 64: return bf ? launch_bwd_typed<true, 64>(a, d, stream) : launch_bwd_typed<false, 64>(a, d, stream);
+    case 128: return bf ? launch_bwd_typed<true, 128>(a, d, stream) : launch_bwd_typed<false, 128>(a, d, stream);
+    default: return BASA_ERR_UNSUPPORTED;
+  }
+}
+
+}  // namespace basa

@@ -97,6 +97,12 @@ basa_status launch_tc(const Dims& d, bool flat, const void* q, const void* k, co
                       const void* kp, const void* vp, void* out, float* lse, uint32_t flags,
                       uint32_t timeout_ms, cudaStream_t stream);
 
+// Backward of window attention (no global memory): D = rowsum(dO * O) into dD,
+// then dQ, then dK and dV.
+basa_status launch_bwd(const Dims& d, const void* q, const void* k, const void* v,
+                       const void* o, const void* dout, const float* lse, float* dD, void* dq,
+                       void* dk, void* dv, cudaStream_t stream);
+
 // The same launch with its parameter block in static storage (no host heap use);
 // calls are serialised by a lock held until the launch has copied the block.
 basa_status launch_tc_static_params(const Dims& d, bool flat, const void* q, const void* k,

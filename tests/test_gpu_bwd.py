@@ -1,0 +1,67 @@
+"""GPU parity of the window-attention backward (basa_window_attn_bwd) against
+the CPU fp64 oracle's gradients.  fp32: max-abs <= 1e-5 on gradients of unit
+scale.  bf16 (bf16 inputs, the bf16 forward's output and lse, fp32 arithmetic,
+gradients rounded once): max-abs <= 2e-2 and relative RMS <= 5e-3."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from basa_synth import make_qkv
+from gpu_util import assert_close, oracle_params
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def basa():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from sparse_attention_diffusion_basa_b200 import build
+    build.build()
+    import sparse_attention_diffusion_basa_b200 as m
+    oracle.build_oracle()
+    return m
+
+
+CASES = [
+    # shape, Hkv (0 = H), window, shift, dtype
+    ((1, 1, 16, 16, 2, 64), 0, (1, 8, 8), (0, 4, 4), "f32"),
+    ((2, 2, 8, 8, 2, 32), 0, (1, 4, 4), (1, 2, 2), "f32"),
+    ((1, 1, 16, 16, 4, 128), 2, (1, 8, 8), (0, 4, 4), "f32"),
+    ((1, 1, 32, 32, 2, 128), 0, (1, 16, 16), (0, 8, 8), "bf16"),
+    ((1, 14, 18, 32, 1, 64), 0, (7, 9, 16), (3, 4, 8), "bf16"),
+    ((1, 1, 32, 32, 4, 128), 2, (1, 16, 16), (0, 8, 8), "bf16"),
+]
+
+
+@pytest.mark.parametrize("shape,Hkv,window,shift,dtype", CASES)
+def test_window_attention_backward(basa, shape, Hkv, window, shift, dtype):
+    B, T, Hg, Wg, H, d = shape
+    hk = Hkv or H
+    q, _, _ = make_qkv(shape, dtype, 151, 152, 153)
+    _, k, v = make_qkv((B, T, Hg, Wg, hk, d), dtype, 151, 152, 153)
+    g, _, _ = make_qkv(shape, dtype, 154, 155, 156)
+    dq_, dk_, dv_, dg = (x.cuda() for x in (q, k, v, g))
+    out, lse = basa.window_attn(dq_, dk_, dv_, window, shift, return_lse=True)
+    gq, gk, gv = basa.window_attn_bwd(dq_, dk_, dv_, out, dg, lse, window, shift)
+    torch.cuda.synchronize()
+    prm = oracle_params(shape, window, shift)
+    prm.Hkv = Hkv
+    f = oracle.as_f64
+    rq, rk, rv = oracle.window_attn_bwd(f(q), f(k), f(v), f(g), prm)
+    for got, ref, name in ((gq, rq, "dq"), (gk, rk, "dk"), (gv, rv, "dv")):
+        assert_close(got, ref, dtype, f"{name} {shape} Hkv={Hkv}")
+
+
+def test_backward_refuses_pooled_memory(basa):
+    from sparse_attention_diffusion_basa_b200 import BasaError
+    x = torch.zeros((1, 1, 16, 16, 2, 64), device="cuda")
+    lse = torch.zeros((1, 2, 256), device="cuda")
+    import ctypes
+    from sparse_attention_diffusion_basa_b200 import _lib
+    prm = basa.make_params(x.shape, x.dtype, (1, 8, 8), (0, 4, 4), (1, 2, 2))
+    p = lambda t: ctypes.c_void_p(t.data_ptr())
+    code = _lib.load().basa_window_attn_bwd(p(x), p(x), p(x), p(x), p(x), p(lse), p(x), p(x),
+                                            p(x), p(lse), ctypes.byref(prm), None)
+    assert code == 3  # BASA_ERR_UNSUPPORTED
