@@ -226,6 +226,63 @@ def cpu_baseline(w, shift, q, k, v, budget_s=12.0):
                       f"{reps} run(s); {dt:.2f} s fp64 on {cores} host threads"}
 
 
+# fp32 CUDA-core peak from the unit counts and the clock: 148 SMs x 128 fp32
+# lanes x 2 flops (FMA) x 1.965 GHz
+FP32_ALU_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
+
+
+def main_backward(args, world, rank, local):
+    """Backward of the workload's window attention: dq, dk, dv for a random dout."""
+    import sparse_attention_diffusion_basa_b200 as basa
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    w = WORKLOADS[args.workload]
+    if w.P or w.text:
+        raise SystemExit("the backward takes no pooled memory or text tokens")
+    shift = w.shifts[-1]
+    q, k, v = workload_inputs(w, len(w.shifts) - 1)
+    dq, dk, dv = (x.to(dev) for x in (q, k, v))
+    g = torch.randn(dq.shape, generator=torch.Generator().manual_seed(7)).to(dq.dtype).to(dev)
+    out, lse = basa.window_attn(dq, dk, dv, w.window, shift, return_lse=True)
+    ws = torch.empty(max(basa.bwd_workspace_size(w.shape(), dq.dtype, w.window, shift), 1),
+                     dtype=torch.uint8, device=dev)
+    flush = L2Flush(dev)
+    step = lambda: basa.window_attn_bwd(dq, dk, dv, out, g, lse, w.window, shift, workspace=ws)
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(torch.cuda.current_device())
+    barrier(world)
+    clocks.start()
+    t = time_steps(step, args.steps, flush)
+    torch.cuda.synchronize()
+    barrier(world)
+    clk = clocks.stop()
+    assert basa.get_status() == 0
+    ms = max_over_ranks(sum(t) / len(t), world)
+    B, T, Hg, Wg, H, d = w.shape()
+    # five contractions per window: S, dP, dV, dQ, dK (the forward has two)
+    flops = 10.0 * B * H * w.N * w.m * d
+    tflops = flops / (ms * 1e-3) / 1e12
+    line = {"metric": "window-attn backward latency (ms) & TFLOP/s", "value": world * tflops,
+            "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "f32 (math) on " + w.dtype + " tensors", "data": "synthetic",
+            "config": {"workload": f"{w.name} backward", "N": w.N, "m": w.m,
+                       "l2": "evicted before every step (256 MiB write, then 256 MiB read; outside the events)"},
+            "roofline": {"bound": "alu", "achieved": tflops, "peak": FP32_ALU_TFLOPS,
+                         "unit": "TFLOP/s", "frac": tflops / FP32_ALU_TFLOPS,
+                         "peak_source": "derived: 148 SMs x 128 fp32 lanes x 2 x 1.965 GHz",
+                         "kernel": "bwd_prep + bwd_dq + bwd_dkv (CUDA cores)"},
+            "gpu_launches": 3 * args.steps, "clocks": clk}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        barrier(world)
+        torch.distributed.destroy_process_group()
+    return 0
+
+
 def dist_setup(args):
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -295,6 +352,8 @@ def main():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--full-steps", type=int, default=5)
+    ap.add_argument("--backward", action="store_true",
+                    help="time the backward (dq, dk, dv) of the workload's window attention")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     world, rank, local = dist_setup(args)
@@ -303,6 +362,9 @@ def main():
         if world > 1:
             torch.distributed.destroy_process_group()
         return rc
+
+    if args.backward:
+        return main_backward(args, world, rank, local)
 
     import sparse_attention_diffusion_basa_b200 as basa
     dev = torch.device("cuda", local)

@@ -20,7 +20,7 @@ from . import _lib
 from ._lib import BasaError, BasaParams, BASA_F32, BASA_BF16  # noqa: F401
 
 __all__ = ["window_attn", "window_attn_gm", "full_attn", "joint_attn", "window_attn_bwd",
-           "pool_kv", "workspace_size", "get_status", "window_tiles", "make_params", "BasaError",
+           "pool_kv", "workspace_size", "bwd_workspace_size", "get_status", "window_tiles", "make_params", "BasaError",
            "library_path"]
 
 library_path = _lib.LIB_PATH
@@ -87,6 +87,12 @@ def _stream(t: torch.Tensor, stream=None):
 def workspace_size(shape, dtype, window, shift=(0, 0, 0), pool=(0, 0, 0), hkv=0) -> int:
     return int(_lib.load().basa_workspace_size(
         ctypes.byref(make_params(shape, dtype, window, shift, pool, hkv=hkv))))
+
+
+def bwd_workspace_size(shape, dtype, window, shift=(0, 0, 0), hkv=0) -> int:
+    """Bytes of device workspace that window_attn_bwd needs for this problem."""
+    return int(_lib.load().basa_bwd_workspace_size(
+        ctypes.byref(make_params(shape, dtype, window, shift, (0, 0, 0), hkv=hkv))))
 
 
 def pool_kv(k: torch.Tensor, v: torch.Tensor, pool, out=None, stream=None):
