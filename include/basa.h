@@ -92,6 +92,8 @@ typedef enum basa_dtype { BASA_F32 = 0, BASA_BF16 = 1 } basa_dtype;
 #define BASA_FLAG_TEST_WITHHOLD_LOADS 0x1u /* the bf16 kernel's loader issues nothing,
                                               so its first wait runs out (tests the
                                               timeout path); output is not written */
+#define BASA_FLAG_BWD_CUDA_CORES 0x2u      /* basa_window_attn_bwd: take the fp32 CUDA-core
+                                              kernels for bf16 too (comparison and tests) */
 
 typedef struct basa_params {
   int32_t B, H;        /* batch, heads */
@@ -192,9 +194,12 @@ BASA_API basa_status basa_joint_attn(const void* q, const void* k, const void* v
  * q, out, dout, dq: [B, T, Hg, Wg, H, d]; k, v, dk, dv: [B, T, Hg, Wg, Hkv, d]
  * (query heads of one group add into the shared dk, dv); lse: fp32 [B, H, N]
  * from the forward call; workspace: basa_bwd_workspace_size(p) bytes, 16-byte
- * aligned.  fp32 arithmetic on CUDA cores for both dtypes; bf16 gradients are
- * rounded once.  A pool cell in p gives BASA_ERR_UNSUPPORTED.  Three launches
- * on `stream`; nothing is allocated.
+ * aligned.  bf16 with d = 64 or 128 runs on the tensor cores: fp32 logits,
+ * exponentials and accumulators, with P and dS rounded to bf16 as the operands
+ * of their MMAs, and the gradients rounded once.  fp32 (and bf16 windows beyond
+ * the tensor-core tile plan's bounds, or with BASA_FLAG_BWD_CUDA_CORES) runs in
+ * fp32 on CUDA cores.  A pool cell in p gives BASA_ERR_UNSUPPORTED.  Three
+ * launches on `stream`; nothing is allocated.
  */
 BASA_API size_t basa_bwd_workspace_size(const basa_params* p);
 BASA_API basa_status basa_window_attn_bwd(const void* q, const void* k, const void* v,

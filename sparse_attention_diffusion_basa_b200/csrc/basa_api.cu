@@ -323,8 +323,12 @@ basa_status basa_window_attn_bwd(const void* q, const void* k, const void* v, co
   if (!lse) return BASA_ERR_INVALID_ARG;
   if (!workspace) return BASA_ERR_WORKSPACE;
   if (misaligned(workspace)) return BASA_ERR_ALIGN;
-  return launch_bwd(d, q, k, v, out, dout, lse, static_cast<float*>(workspace), dq, dk, dv,
-                    stream);
+  float* dD = static_cast<float*>(workspace);
+  if (!(p->flags & BASA_FLAG_BWD_CUDA_CORES) && d.dtype == BASA_BF16 && (d.d == 64 || d.d == 128)) {
+    s = launch_bwd_tc(d, q, k, v, out, dout, lse, dD, dq, dk, dv, p->wait_timeout_ms, stream);
+    if (s != BASA_ERR_UNSUPPORTED) return s;  // outside the tile plan's bounds: CUDA cores
+  }
+  return launch_bwd(d, q, k, v, out, dout, lse, dD, dq, dk, dv, stream);
 }
 
 basa_status basa_full_attn(const void* q, const void* k, const void* v, void* out, float* lse,

@@ -232,7 +232,7 @@ __global__ void __launch_bounds__(kBwdThreads) bwd_dkv_kernel(BwdArgs a) {
 }
 
 template <bool BF16, int D>
-basa_status launch_bwd_typed(BwdArgs& a, const Dims& d, cudaStream_t stream) {
+basa_status launch_bwd_typed(BwdArgs& a, const Dims& d, bool prep_only, cudaStream_t stream) {
   const long long rows = (long long)d.B * d.N * d.H;
   const long long nwin = (long long)d.nwt * d.nwh * d.nww;
   constexpr int per = kBwdThreads / (D / 32);  // queries (keys) per CTA
@@ -243,16 +243,15 @@ basa_status launch_bwd_typed(BwdArgs& a, const Dims& d, cudaStream_t stream) {
     return BASA_ERR_UNSUPPORTED;
   bwd_prep_kernel<BF16, D><<<(unsigned)((rows + kBwdThreads - 1) / kBwdThreads), kBwdThreads, 0,
                              stream>>>(a);
+  if (prep_only) return cudaGetLastError() == cudaSuccess ? BASA_OK : BASA_ERR_CUDA;
   bwd_dq_kernel<BF16, D><<<(unsigned)dq_blocks, kBwdThreads, 0, stream>>>(a);
   bwd_dkv_kernel<BF16, D><<<(unsigned)dkv_blocks, kBwdThreads, 0, stream>>>(a);
   return cudaGetLastError() == cudaSuccess ? BASA_OK : BASA_ERR_CUDA;
 }
 
-}  // namespace
-
-basa_status launch_bwd(const Dims& d, const void* q, const void* k, const void* v,
-                       const void* o, const void* dout, const float* lse, float* dD, void* dq,
-                       void* dk, void* dv, cudaStream_t stream) {
+basa_status launch_bwd_common(const Dims& d, const void* q, const void* k, const void* v,
+                              const void* o, const void* dout, const float* lse, float* dD,
+                              void* dq, void* dk, void* dv, bool prep_only, cudaStream_t stream) {
   BwdArgs a;
   a.q = q; a.k = k; a.v = v; a.o = o; a.dout = dout; a.lse = lse; a.dD = dD;
   a.dq = dq; a.dk = dk; a.dv = dv;
@@ -267,11 +266,25 @@ basa_status launch_bwd(const Dims& d, const void* q, const void* k, const void* 
   a.scale = d.scale;
   const bool bf = d.dtype == BASA_BF16;
   switch (d.d) {
-    case 32: return bf ? launch_bwd_typed<true, 32>(a, d, stream) : launch_bwd_typed<false, 32>(a, d, stream);
-    case 64: return bf ? launch_bwd_typed<true, 64>(a, d, stream) : launch_bwd_typed<false, 64>(a, d, stream);
-    case 128: return bf ? launch_bwd_typed<true, 128>(a, d, stream) : launch_bwd_typed<false, 128>(a, d, stream);
+    case 32: return bf ? launch_bwd_typed<true, 32>(a, d, prep_only, stream) : launch_bwd_typed<false, 32>(a, d, prep_only, stream);
+    case 64: return bf ? launch_bwd_typed<true, 64>(a, d, prep_only, stream) : launch_bwd_typed<false, 64>(a, d, prep_only, stream);
+    case 128: return bf ? launch_bwd_typed<true, 128>(a, d, prep_only, stream) : launch_bwd_typed<false, 128>(a, d, prep_only, stream);
     default: return BASA_ERR_UNSUPPORTED;
   }
+}
+
+}  // namespace
+
+basa_status launch_bwd(const Dims& d, const void* q, const void* k, const void* v,
+                       const void* o, const void* dout, const float* lse, float* dD, void* dq,
+                       void* dk, void* dv, cudaStream_t stream) {
+  return launch_bwd_common(d, q, k, v, o, dout, lse, dD, dq, dk, dv, false, stream);
+}
+
+basa_status launch_bwd_prep(const Dims& d, const void* o, const void* dout, float* dD,
+                            cudaStream_t stream) {
+  return launch_bwd_common(d, nullptr, nullptr, nullptr, o, dout, nullptr, dD, nullptr, nullptr,
+                           nullptr, true, stream);
 }
 
 }  // namespace basa

@@ -103,6 +103,17 @@ basa_status launch_bwd(const Dims& d, const void* q, const void* k, const void* 
                        const void* o, const void* dout, const float* lse, float* dD, void* dq,
                        void* dk, void* dv, cudaStream_t stream);
 
+// D = rowsum(dO * O) alone (fp32 [B, H, N] into dD).
+basa_status launch_bwd_prep(const Dims& d, const void* o, const void* dout, float* dD,
+                            cudaStream_t stream);
+
+// bf16 backward on the tensor cores (d = 64 or 128, window mode): D into dD,
+// then dQ, then dK and dV.  BASA_ERR_UNSUPPORTED, before any launch, when the
+// shape is outside the tile plan's bounds.
+basa_status launch_bwd_tc(const Dims& d, const void* q, const void* k, const void* v,
+                          const void* out, const void* dout, const float* lse, float* dD,
+                          void* dq, void* dk, void* dv, uint32_t timeout_ms, cudaStream_t stream);
+
 // The same launch with its parameter block in static storage (no host heap use);
 // calls are serialised by a lock held until the launch has copied the block.
 basa_status launch_tc_static_params(const Dims& d, bool flat, const void* q, const void* k,
@@ -113,8 +124,11 @@ basa_status launch_tc_static_params(const Dims& d, bool flat, const void* q, con
 // Test hook: y = the kernels' polynomial 2^x (device pointers, n floats).
 basa_status launch_ex2_poly_test(const float* x, float* y, long long n, cudaStream_t stream);
 
-// Device status word helpers (basa_tc.cu).
+// Device status word helpers.  read_and_clear_status (basa_tc.cu) synchronises
+// the stream and reads and clears the status words of every kernel file;
+// take_bwd_status does that for the tensor-core backward's own word.
 basa_status read_and_clear_status(cudaStream_t stream);
+cudaError_t take_bwd_status(cudaStream_t stream, unsigned int* status, unsigned int* where);
 
 // Encodes a tiled TMA map through the driver entry point.
 basa_status encode_map(CUtensorMap* map, const void* base, int rank, const uint64_t* dims,

@@ -45,18 +45,13 @@
 #include <new>
 
 #include "basa_internal.h"
+#include "tc_device.cuh"
 
 namespace basa {
-
-__device__ unsigned int g_basa_status;  // bit 0: a device wait timed out
-__device__ unsigned int g_basa_where;   // site of the first wait that gave up
 
 namespace {
 
 constexpr int kThreads = 384;
-constexpr int kHalf = 128 * 128;  // bytes of one 64-wide head-dim half of a 128-row tile
-constexpr int kPlanBytes = 1536;  // shared-memory room for the compact tile plan
-constexpr int kPlanWords = kPlanBytes / 4;
 
 struct __align__(64) TcParams {
   CUtensorMap qm[kMaxShapes];  // window boxes, rank 5: [d, H, Wg, Hg, B*T]
@@ -66,9 +61,7 @@ struct __align__(64) TcParams {
   CUtensorMap qf, kf, vf, of;  // flat 128-row tiles, rank 4: [d, H, N, B]
   CUtensorMap kpf, vpf;        // pooled 128-row tiles, rank 4: [d, H, P, B]
   CUtensorMap fill;            // 8-row box over k's flat view, read out of bounds = zeros
-  uint32_t plan[kPlanWords];  // compact tile plan image, copied to shared memory at start
-  int plan_words;
-  int plan_off_rows, plan_off_bt, plan_off_bh, plan_off_bw, plan_off_entries;  // bytes
+  PlanImage plan;             // compact tile plan, copied to shared memory at start
   float* lse;
   __nv_bfloat16* out;  // [B, T, Hg, Wg, H, d]
   int warp_stores;  // output by warp-staged 16-byte stores (1) or by TMA boxes (0)
@@ -91,345 +84,14 @@ struct __align__(64) TcParams {
   float scale_log2;
 };
 
-// ---------------------------------------------------------------------------
-// PTX wrappers
-// ---------------------------------------------------------------------------
-__device__ __forceinline__ uint32_t smem_u32(const void* p) {
-  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
-}
-__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
-}
-__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
-               : "memory");
-}
-__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(bar), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-__device__ __forceinline__ void fence_barrier_init() {
-  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-}
-__device__ __forceinline__ void fence_proxy_async() {
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-__device__ __forceinline__ void tc_fence_before() {
-  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
-}
-__device__ __forceinline__ void tc_fence_after() {
-  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-}
 
-__device__ __forceinline__ void tma_load_5d(uint32_t dst, const CUtensorMap* map, uint32_t bar,
-                                            int c0, int c1, int c2, int c3, int c4) {
-  asm volatile(
-      "cp.async.bulk.tensor.5d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(c4)
-      : "memory");
-}
-__device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap* map, uint32_t bar,
-                                            int c0, int c1, int c2, int c3) {
-  asm volatile(
-      "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%3, %4, %5, %6}], [%2];" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
-      : "memory");
-}
-__device__ __forceinline__ void tma_store_5d(const CUtensorMap* map, uint32_t src, int c0, int c1,
-                                             int c2, int c3, int c4) {
-  asm volatile(
-      "cp.async.bulk.tensor.5d.global.shared::cta.tile.bulk_group"
-      " [%0, {%2, %3, %4, %5, %6}], [%1];" ::"l"(reinterpret_cast<uint64_t>(map)),
-      "r"(src), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(c4)
-      : "memory");
-}
-__device__ __forceinline__ void tma_store_4d(const CUtensorMap* map, uint32_t src, int c0, int c1,
-                                             int c2, int c3) {
-  asm volatile(
-      "cp.async.bulk.tensor.4d.global.shared::cta.tile.bulk_group"
-      " [%0, {%2, %3, %4, %5}], [%1];" ::"l"(reinterpret_cast<uint64_t>(map)),
-      "r"(src), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
-      : "memory");
-}
-__device__ __forceinline__ void prefetch_tmap(const CUtensorMap* map) {
-  asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
-}
-__device__ __forceinline__ void bulk_commit() {
-  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
-}
-__device__ __forceinline__ void bulk_wait_read0() {
-  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
-}
-__device__ __forceinline__ void bulk_wait_all0() {
-  asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
-}
-
-__device__ __forceinline__ void tmem_alloc(uint32_t slot_smem, uint32_t ncols) {
-  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(slot_smem),
-               "r"(ncols)
-               : "memory");
-}
-__device__ __forceinline__ void tmem_relinquish() {
-  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
-}
-__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
-  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
-               : "memory");
-}
-
-// Shared-memory matrix descriptor, 128-byte swizzle (sm_100 layout: start
-// address >> 4 in bits 0-13, leading byte offset >> 4 in 16-29, stride byte
-// offset >> 4 in 32-45, descriptor version 1 in 46-47, swizzle mode 2 in 61-63).
-__device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
-  return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
-         ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
-}
-// Instruction descriptor of kind::f16: bf16 A and B, fp32 accumulator, A K-major,
-// B K-major or MN-major, M = 128, N = n.
-__host__ __device__ constexpr uint32_t idesc_bf16(int n, bool b_mn) {
-  return (1u << 4) | (1u << 7) | (1u << 10) | ((b_mn ? 1u : 0u) << 16) |
-         ((uint32_t)(n >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
-}
-__device__ __forceinline__ void mma_bf16(uint32_t tmem_d, uint64_t a, uint64_t b, uint32_t idesc,
-                                         uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
-      "l"(a), "l"(b), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-// The same with the A operand (M x K, K-major) read from TMEM: two 16-bit
-// elements per 32-bit column, lower half first.
-__device__ __forceinline__ void mma_bf16_ts(uint32_t tmem_d, uint32_t tmem_a, uint64_t b,
-                                            uint32_t idesc, uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(tmem_d),
-      "r"(tmem_a), "l"(b), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-__device__ __forceinline__ void mma_commit(uint32_t bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-                   bar)
-               : "memory");
-}
-
-#define TMEM_REGS32(r)                                                                         \
-  "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),         \
-      "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), \
-      "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),           \
-      "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),           \
-      "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
-#define TMEM_INREGS32(r)                                                                          \
-  "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),         \
-      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),          \
-      "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]),        \
-      "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]),        \
-      "r"(r[29]), "r"(r[30]), "r"(r[31])
-#define TMEM_RWREGS32(r)                                                                         \
-  "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]),           \
-      "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]),   \
-      "+r"(r[14]), "+r"(r[15]), "+r"(r[16]), "+r"(r[17]), "+r"(r[18]), "+r"(r[19]),             \
-      "+r"(r[20]), "+r"(r[21]), "+r"(r[22]), "+r"(r[23]), "+r"(r[24]), "+r"(r[25]),             \
-      "+r"(r[26]), "+r"(r[27]), "+r"(r[28]), "+r"(r[29]), "+r"(r[30]), "+r"(r[31])
-
-// 32 consecutive fp32 columns of this thread's TMEM lane; the values are valid
-// only after tmem_wait_ld, which takes them as operands so that no use can be
-// scheduled before it.
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
-      "%11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, "
-      "%28, %29, %30, %31}, [%32];"
-      : TMEM_REGS32(r)
-      : "r"(taddr)
-      : "memory");
-}
-__device__ __forceinline__ void tmem_wait_ld(uint32_t (&r)[32]) {
-  asm volatile("tcgen05.wait::ld.sync.aligned;" : TMEM_RWREGS32(r)::"memory");
-}
-__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
-      "%11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, "
-      "%28, %29, %30, %31, %32};" ::"r"(taddr),
-      TMEM_INREGS32(r)
-      : "memory");
-}
-// 16 consecutive 32-bit columns of this thread's lane.
-__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
-      "%11, %12, %13, %14, %15, %16};" ::"r"(taddr),
-      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
-      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
-      : "memory");
-}
-__device__ __forceinline__ void tmem_wait_st() {
-  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
-}
-
-__device__ __forceinline__ float ex2(float x) {
-  float y;
-  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
-}
-__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
-  __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
-  return *reinterpret_cast<uint32_t*>(&h);
-}
-// Packed pairs of fp32 (f32x2 arithmetic of sm_100).
-__device__ __forceinline__ uint64_t f2pack(float lo, float hi) {
-  uint64_t d;
-  asm("mov.b64 %0, {%1, %2};" : "=l"(d) : "f"(lo), "f"(hi));
-  return d;
-}
-__device__ __forceinline__ void f2unpack(uint64_t v, float& lo, float& hi) {
-  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
-}
-__device__ __forceinline__ uint64_t f2fma(uint64_t a, uint64_t b, uint64_t c) {
-  uint64_t d;
-  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
-  return d;
-}
-__device__ __forceinline__ uint64_t f2add(uint64_t a, uint64_t b) {
-  uint64_t d;
-  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-  return d;
-}
-__device__ __forceinline__ uint64_t f2mul(uint64_t a, uint64_t b) {
-  uint64_t d;
-  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-  return d;
-}
-__device__ __forceinline__ float max3(float a, float b, float c) {
-  float d;
-  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
-  return d;
-}
-
-// 2^x for a pair of x <= 0, computed on the FMA and integer pipes so that part
-// of the softmax's exponentials bypass the MUFU unit (its throughput limit).
-// Method: round-to-nearest argument reduction x = j + f, |f| <= 1/2, through the
-// float constant 1.5 * 2^23 (after the addition its low mantissa bits hold j;
-// the additive reduction of Cody and Waite), a cubic fit of 2^f on [-1/2, 1/2]
-// minimising the maximum relative error (Remez exchange, fitted for this
-// library: 7.5e-5 worst case in fp32 Horner evaluation), then the scale by 2^j
-// applied by adding j to the exponent field (Schraudolph, "A fast, compact
-// approximation of the exponential function", 1999).  x is clamped at -125 so
-// the exponent field cannot underflow; results there are below 2^-124.
-constexpr float kEx2C0 = 0x1.fff692p-1f;
-constexpr float kEx2C1 = 0x1.62f31ap-1f;
-constexpr float kEx2C2 = 0x1.f0de1ap-3f;
-constexpr float kEx2C3 = 0x1.c3f76p-5f;
-__device__ __forceinline__ uint64_t ex2_poly_x2(uint64_t x2) {
-  float x0, x1;
-  f2unpack(x2, x0, x1);
-  x0 = fmaxf(x0, -125.0f);
-  x1 = fmaxf(x1, -125.0f);
-  const uint64_t t = f2add(f2pack(x0, x1), f2pack(12582912.0f, 12582912.0f));
-  const uint64_t j = f2add(t, f2pack(-12582912.0f, -12582912.0f));
-  const uint64_t f = f2fma(j, f2pack(-1.0f, -1.0f), f2pack(x0, x1));
-  uint64_t q = f2fma(f, f2pack(kEx2C3, kEx2C3), f2pack(kEx2C2, kEx2C2));
-  q = f2fma(q, f, f2pack(kEx2C1, kEx2C1));
-  q = f2fma(q, f, f2pack(kEx2C0, kEx2C0));
-  float q0, q1, t0, t1;
-  f2unpack(q, q0, q1);
-  f2unpack(t, t0, t1);
-  return f2pack(__int_as_float(__float_as_int(q0) + (__float_as_int(t0) << 23)),
-                __int_as_float(__float_as_int(q1) + (__float_as_int(t1) << 23)));
-}
-
-// Which exponential pairs go to the polynomial: pair e of every 16 when
-// e % kEx2Period == kEx2Period - 1 (period 3: 5 of 16 pairs); 0 = none.
-#ifndef BASA_EX2_PERIOD
-#define BASA_EX2_PERIOD 0
-#endif
-constexpr int kEx2Period = BASA_EX2_PERIOD;
-
-// Rescale O only when a tile's row max exceeds the reference max by more than
-// 2^kLazyRescale; until then the stale reference is kept (P stays <= 2^8).
-constexpr float kLazyRescale = 8.0f;
-
-__device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr) {
-  uint4 v;
-  asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
-               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-               : "r"(addr)
-               : "memory");
-  return v;
-}
-__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
-                                             uint32_t d) {
-  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c),
-               "r"(d)
-               : "memory");
-}
-// Byte offset of 16-byte chunk `chunk` (0..7) of row `row` inside a 128-byte
-// swizzled, 1024-byte-aligned block of rows.
-__device__ __forceinline__ uint32_t swz(int row, int chunk) {
-  return (uint32_t)(row * 128 + ((chunk ^ (row & 7)) << 4));
-}
-
-// ---------------------------------------------------------------------------
-// Bounded waits.  `abort_flag` lives in shared memory; any role that gives up
-// raises it so that the others leave their loops promptly.  The poll loop is
-// tight (try_wait itself sleeps until the phase completes or a short hardware
-// limit passes); the abort flag and the bound, in SM cycles (2 per ns of the
-// limit, so at least the limit at clocks up to 2 GHz), are checked every 64
-// polls.  The first wait that gives up records its site in g_basa_where.
-// ---------------------------------------------------------------------------
+// Sites recorded by the first wait that gives up (host debug output only).
 enum WaitSite : uint32_t {
   kSiteLoadKvEmpty = 1, kSiteLoadQEmpty, kSiteLoadDrainKv, kSiteLoadDrainQ, kSiteMmaQFull,
   kSiteMmaKvFull, kSiteMmaSFree, kSiteMmaPFull, kSiteMmaDrain, kSiteSmxSFull, kSiteSmxPvDone,
   kSiteSmxPvLast, kSiteSmxOStaged, kSiteSmxOFree
 };
 
-__device__ __noinline__ bool wait_slow(uint32_t bar, uint32_t parity,
-                                       volatile uint32_t* abort_flag, uint64_t limit_ns,
-                                       uint32_t site, bool honour_abort) {
-  const long long c0 = clock64();
-  const long long climit = (long long)(limit_ns * 2ull);
-  for (uint32_t it = 1;; ++it) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 63u) == 0u) {
-      if (honour_abort && *abort_flag) return false;
-      if (clock64() - c0 > climit) {
-        *abort_flag = 1u;
-        atomicCAS(&g_basa_where, 0u, site);
-        atomicOr(&g_basa_status, 1u);
-        return false;
-      }
-    }
-  }
-}
-__device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity,
-                                             volatile uint32_t* abort_flag, uint64_t limit_ns,
-                                             uint32_t site, bool honour_abort = true) {
-  if (mbar_try_wait(bar, parity)) return true;
-  return wait_slow(bar, parity, abort_flag, limit_ns, site, honour_abort);
-}
-// Warp-uniform variant: every lane waits, and the warp proceeds only if all did.
-__device__ __forceinline__ bool wait_warp(uint32_t bar, uint32_t parity,
-                                          volatile uint32_t* abort_flag, uint64_t limit_ns,
-                                          uint32_t site, bool honour_abort = true) {
-  const bool ok = wait_bounded(bar, parity, abort_flag, limit_ns, site, honour_abort);
-  return __all_sync(0xffffffffu, ok);
-}
 
 // ---------------------------------------------------------------------------
 // Work-unit decoding
@@ -470,20 +132,6 @@ __device__ __forceinline__ Unit decode_unit(const TcParams& p, uint32_t u) {
   return U;
 }
 
-// The tile plan as seen from shared memory.  Image layout (bytes): per (class,
-// tile) a 16-bit word (first box << 4 | box count); per tile its valid rows;
-// per box shape its t, row and column extents; then the packed box entries.
-struct PlanView {
-  const uint16_t* idx;
-  const uint8_t* rows;
-  const uint8_t* bt;
-  const uint8_t* bh;
-  const uint8_t* bw;
-  const uint32_t* entries;
-  int n_tiles;
-  __device__ __forceinline__ int first(int cls, int tile) const { return idx[cls * n_tiles + tile] >> 4; }
-  __device__ __forceinline__ int count(int cls, int tile) const { return idx[cls * n_tiles + tile] & 15; }
-};
 
 // Valid rows of key tile j (rows past them are zero-filled and masked).
 __device__ __forceinline__ int key_valid(const TcParams& p, const PlanView& pv, int j) {
@@ -505,9 +153,6 @@ __device__ __forceinline__ int query_valid(const TcParams& p, const PlanView& pv
   return pv.rows[qt];
 }
 
-// x mod G for 0 <= x < 2G: a window origin (below G) plus an offset inside the
-// window (below w <= G).
-__device__ __forceinline__ int wrap(int x, int G) { return x >= G ? x - G : x; }
 
 // kind: 0 = q, 1 = k, 2 = v.  Loads one 128-row tile (all head-dim halves) into
 // shared memory at dst and signals bar with the transaction bytes.
@@ -529,30 +174,11 @@ __device__ __forceinline__ void load_tile(const TcParams& p, const PlanView& pv,
     for (int hf = 0; hf < NH; ++hf) tma_load_4d(dst + hf * kHalf, m, bar, hf * 64, head, tile * 128, U.b);
     return;
   }
-  const int b0 = pv.first(U.cls, tile), nb = pv.count(U.cls, tile);
-#pragma unroll 1
-  for (int bi = 0; bi < nb; ++bi) {
-    const uint32_t e = pv.entries[b0 + bi];
-    const int sid = box_shape(e);
-    const int gt = wrap(U.ot + box_lt(e), p.T);
-    const int gh = wrap(U.oh + box_lh(e), p.Hg);
-    const int gw = wrap(U.ow + box_lw(e), p.Wg);
-    const CUtensorMap* m = kind == 0 ? &p.qm[sid] : kind == 1 ? &p.km[sid] : &p.vm[sid];
-    const uint32_t d0 = dst + box_row8(e) * 1024;
-#pragma unroll
-    for (int hf = 0; hf < NH; ++hf)
-      tma_load_5d(d0 + hf * kHalf, m, bar, hf * 64, head, gw, gh, U.b * p.T + gt);
-  }
-#pragma unroll 1
-  for (int r = pv.rows[tile]; r < 128; r += 8) {  // zero rows past the window's tokens
-#pragma unroll
-    for (int hf = 0; hf < NH; ++hf)
-      tma_load_4d(dst + hf * kHalf + r * 128, &p.fill, bar, hf * 64, 0, (int)p.N, 0);
-  }
+  const CUtensorMap* maps = kind == 0 ? p.qm : kind == 1 ? p.km : p.vm;
+  load_window_tile<NH>(pv, maps, &p.fill, WinAt{U.cls, U.ot, U.oh, U.ow, U.b}, tile, head, p.T,
+                       p.Hg, p.Wg, p.N, dst, bar);
 }
 
-// Stores d-half hf of query tile qt from a 128-row x 64-column staging block
-// (128-byte swizzled) with TMA boxes that mirror the load boxes.
 // Stores d-half hf of query tile qt from a 128-row x 64-column staging block
 // (128-byte swizzled) with TMA boxes that mirror the load boxes.
 template <int D>
@@ -578,23 +204,7 @@ __device__ __forceinline__ void store_half(const TcParams& p, const PlanView& pv
 __device__ __forceinline__ long long row_token(const TcParams& p, const PlanView& pv,
                                                const Unit& U, int qt, int r) {
   if (p.flat) return 128LL * qt + r;
-  const int b0 = pv.first(U.cls, qt), nb = pv.count(U.cls, qt);
-#pragma unroll 1
-  for (int bi = 0; bi < nb; ++bi) {
-    const uint32_t e = pv.entries[b0 + bi];
-    const int sid = box_shape(e);
-    const int bt = pv.bt[sid], bh = pv.bh[sid], bw = pv.bw[sid];
-    const int r0 = box_row8(e) * 8;
-    if (r >= r0 && r < r0 + bt * bh * bw) {
-      const int idx = r - r0;
-      const int it = idx / (bh * bw), ih = (idx / bw) % bh, iw = idx % bw;
-      const int gt = wrap(U.ot + box_lt(e), p.T) + it;
-      const int gh = wrap(U.oh + box_lh(e), p.Hg) + ih;
-      const int gw = wrap(U.ow + box_lw(e), p.Wg) + iw;
-      return ((long long)gt * p.Hg + gh) * p.Wg + gw;
-    }
-  }
-  return -1;
+  return window_row_token(pv, WinAt{U.cls, U.ot, U.oh, U.ow, U.b}, qt, r, p.T, p.Hg, p.Wg);
 }
 
 // Shared-memory plan: the unit's two 128-row query tiles, one 64-column output
@@ -645,19 +255,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attn_kernel(const __grid_const
   const int lane = threadIdx.x % 32;
   const uint64_t limit = p.timeout_ns;
 
-  {  // the compact tile plan, from the parameter block into shared memory
-    uint32_t* dst = reinterpret_cast<uint32_t*>(smem + S::plan);
-    for (int w = threadIdx.x; w < p.plan_words; w += kThreads) dst[w] = p.plan[w];
-  }
-  const uint8_t* pimg = smem + S::plan;
-  PlanView pv;
-  pv.idx = reinterpret_cast<const uint16_t*>(pimg);
-  pv.rows = pimg + p.plan_off_rows;
-  pv.bt = pimg + p.plan_off_bt;
-  pv.bh = pimg + p.plan_off_bh;
-  pv.bw = pimg + p.plan_off_bw;
-  pv.entries = reinterpret_cast<const uint32_t*>(pimg + p.plan_off_entries);
-  pv.n_tiles = p.n_qt;
+  // the compact tile plan, from the parameter block into shared memory
+  const PlanView pv = plan_to_smem(p.plan, smem + S::plan, p.n_qt, threadIdx.x, kThreads);
   if (threadIdx.x == 0) {
     for (int i = 0; i < 2; ++i) {
       mbar_init(BAR(S::QFULL + i), 1);
@@ -1064,13 +663,6 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attn_kernel(const __grid_const
   }
 }
 
-int sm_count() {
-  int dev = 0, n = 0;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-  return n > 0 ? n : 1;
-}
-
 template <int D, int kRing>
 basa_status launch_impl(TcParams* prm, cudaStream_t stream) {
   const int smem = Smem<D, kRing>::alloc;
@@ -1078,7 +670,7 @@ basa_status launch_impl(TcParams* prm, cudaStream_t stream) {
   if (cudaFuncSetAttribute(tc_attn_kernel<D, kRing>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            smem) != cudaSuccess)
     return BASA_ERR_CUDA;
-  long long grid = sm_count();
+  long long grid = tc_sm_count();
   if (grid > prm->n_units) grid = prm->n_units;
   tc_attn_kernel<D, kRing><<<(unsigned)grid, kThreads, smem, stream>>>(*prm);
   return cudaGetLastError() == cudaSuccess ? BASA_OK : BASA_ERR_CUDA;
@@ -1087,41 +679,6 @@ basa_status launch_impl(TcParams* prm, cudaStream_t stream) {
 }  // namespace
 
 namespace {
-
-// Packs the tile plan into the compact image the kernel copies to shared memory.
-basa_status pack_plan(const TilePlan& plan, TcParams* prm) {
-  const int T = plan.n_tiles, NSh = plan.n_shapes;
-  uint8_t* img = reinterpret_cast<uint8_t*>(prm->plan);
-  const int off_rows = 2 * kClasses * T;
-  const int off_bt = off_rows + T, off_bh = off_bt + NSh, off_bw = off_bh + NSh;
-  const int off_entries = (off_bw + NSh + 3) & ~3;
-  int n = 0;
-  for (int c = 0; c < kClasses; ++c)
-    for (int t = 0; t < T; ++t) n += plan.nbox[c][t];
-  const int total = off_entries + 4 * n;
-  if (total > kPlanBytes || n >= 4096) return BASA_ERR_UNSUPPORTED;
-  uint16_t* idx = reinterpret_cast<uint16_t*>(img);
-  uint32_t* entries = reinterpret_cast<uint32_t*>(img + off_entries);
-  int e = 0;
-  for (int c = 0; c < kClasses; ++c)
-    for (int t = 0; t < T; ++t) {
-      idx[c * T + t] = (uint16_t)((e << 4) | plan.nbox[c][t]);
-      for (int b = 0; b < plan.nbox[c][t]; ++b) entries[e++] = plan.box[c][t][b];
-    }
-  for (int t = 0; t < T; ++t) img[off_rows + t] = plan.tile_rows[t];
-  for (int s2 = 0; s2 < NSh; ++s2) {
-    img[off_bt + s2] = plan.shape_bt[s2];
-    img[off_bh + s2] = plan.shape_bh[s2];
-    img[off_bw + s2] = plan.shape_bw[s2];
-  }
-  prm->plan_words = (total + 3) / 4;
-  prm->plan_off_rows = off_rows;
-  prm->plan_off_bt = off_bt;
-  prm->plan_off_bh = off_bh;
-  prm->plan_off_bw = off_bw;
-  prm->plan_off_entries = off_entries;
-  return BASA_OK;
-}
 
 // Fills *prm (zeroed by the caller) for one call and launches the kernel.
 basa_status build_and_launch(TcParams* prm, const Dims& d, bool flat, const void* q,
@@ -1188,7 +745,7 @@ basa_status build_and_launch(TcParams* prm, const Dims& d, bool flat, const void
     if (units > 0x7fffffffLL) { st = BASA_ERR_UNSUPPORTED; goto done; }
     prm->n_units = (uint32_t)units;
   } else {
-    if ((st = pack_plan(plan, prm)) != BASA_OK) goto done;
+    if ((st = pack_plan_image(plan, &prm->plan)) != BASA_OK) goto done;
     const uint64_t dims[5] = {D, H, (uint64_t)d.Wg, (uint64_t)d.Hg, (uint64_t)d.B * d.T};
     const uint64_t strides[4] = {D * 2, H * D * 2, (uint64_t)d.Wg * H * D * 2,
                                  (uint64_t)d.Hg * d.Wg * H * D * 2};
@@ -1277,17 +834,12 @@ basa_status launch_ex2_poly_test(const float* x, float* y, long long n, cudaStre
 }
 
 basa_status read_and_clear_status(cudaStream_t stream) {
-  if (cudaStreamSynchronize(stream) != cudaSuccess) return BASA_ERR_CUDA;
-  unsigned int v = 0;
-  if (cudaMemcpyFromSymbol(&v, g_basa_status, sizeof(v)) != cudaSuccess) return BASA_ERR_CUDA;
-  if (v) {
-    unsigned int where = 0;
-    cudaMemcpyFromSymbol(&where, g_basa_where, sizeof(where));
-    if (getenv("BASA_DEBUG")) fprintf(stderr, "basa: device wait gave up at site %u\n", where);
-    const unsigned int zero = 0;
-    if (cudaMemcpyToSymbol(g_basa_status, &zero, sizeof(zero)) != cudaSuccess ||
-        cudaMemcpyToSymbol(g_basa_where, &zero, sizeof(zero)) != cudaSuccess)
-      return BASA_ERR_CUDA;
+  unsigned int v = 0, where = 0, vb = 0, whereb = 0;
+  if (tc_take_status(stream, &v, &where) != cudaSuccess) return BASA_ERR_CUDA;
+  if (take_bwd_status(stream, &vb, &whereb) != cudaSuccess) return BASA_ERR_CUDA;
+  if (v | vb) {
+    if (getenv("BASA_DEBUG"))
+      fprintf(stderr, "basa: device wait gave up at site %u (backward: %u)\n", where, whereb);
     return BASA_ERR_TIMEOUT;
   }
   return cudaGetLastError() == cudaSuccess ? BASA_OK : BASA_ERR_CUDA;

@@ -1,0 +1,628 @@
+// Backward of bf16 shifted local window attention on the 5th-generation tensor
+// cores (tcgen05 + TMEM + TMA) of sm_100a.
+//
+// The operation ("BASA: Backend-Agnostic Sparse Attention for Fast
+// High-Resolution Diffusion Transformers", zhichai.net topic 178635722, "The
+// BASA Method": every query attends to the keys of its own cyclically shifted
+// window; the forum review of the same paper, reply 178634520, names the
+// dense-teacher adaptation that trains through this attention).  With
+// P = exp(scale * Q K^T - lse) over each query's window (lse from the forward
+// pass) and D = rowsum(dO * O):
+//   dP = dO V^T,  dS = P * (dP - D),
+//   dQ = scale * dS K,  dK = scale * dS^T Q,  dV = P^T dO.
+// A key is seen only by the queries of its own window, so every gradient row
+// depends on one window alone: two kernels, no atomics.
+//
+// One kernel template serves both, because they have the same shape:
+//   dQ  (KV = false): unit (b, h, window, query tile).  Fixed per unit: A0 = Q,
+//       A1 = dO of the tile (and lse, D of its rows).  Step j over the key
+//       tiles of the window: B0 = K_j, B1 = V_j.
+//   dKV (KV = true):  unit (b, K/V head, window, key tile).  Fixed per unit:
+//       A0 = K, A1 = V of the tile.  Step over (query head of the group, query
+//       tile): B0 = Q_i, B1 = dO_i (and lse, D of its rows).
+// Per step the tensor core computes X = A0 B0^T and Y = A1 B1^T into TMEM
+// (dQ: S and dP; dKV: S^T and dP^T).  The elementwise warps form P and dS in
+// fp32 and write them back into TMEM as bf16 pairs over X (and Y), and the
+// tensor core accumulates, with the bf16 operand read from TMEM,
+//   dQ:  dQ += dS K_j                  (B0 read MN-major)
+//   dKV: dV += P^T dO_i, dK += dS^T Q_i (B1, B0 read MN-major).
+// TMEM columns: X [0, 128), Y [128, 256), accumulators from 256.
+//
+// Persistent CTAs (one per SM, 384 threads):
+//   warp 0       TMA loader of the step pairs through a two-slot ring (dKV:
+//                with the lse and D of the step's queries);
+//   warp 1       owns TMEM (512 columns) and issues the MMAs from one thread;
+//   warp 2       TMA loader of the unit pair (dQ: with its rows' lse and D);
+//   warps 4..11  two warpgroups, one per 64-column half of X and Y: the
+//                elementwise stage, then the epilogue (scale, round to bf16,
+//                warp-staged 16-byte stores to the window's token rows).
+// Tiles, TMA boxes and the zero rows of partial tiles come from the forward's
+// shifted-window tile plan.  Every mbarrier wait is bounded: on expiry the
+// kernel raises its device status word, lets every role leave its loop, waits
+// (bounded) for its own copies and MMAs in flight, frees TMEM and returns.
+#include <cuda_bf16.h>
+#include <math.h>
+#include <string.h>
+
+#include <new>
+
+#include "basa_internal.h"
+#include "tc_device.cuh"
+
+namespace basa {
+namespace {
+
+constexpr int kBwdTcThreads = 384;
+constexpr float kLog2e = 1.4426950408889634f;
+
+struct __align__(64) BwdTcParams {
+  CUtensorMap qm[kMaxShapes];  // window boxes over q, rank 5: [d, H, Wg, Hg, B*T]
+  CUtensorMap gm[kMaxShapes];  // the same over dout
+  CUtensorMap km[kMaxShapes];  // over k: [d, Hkv, Wg, Hg, B*T]
+  CUtensorMap vm[kMaxShapes];  // over v
+  CUtensorMap fill;            // 8-row box over k's flat view, read out of bounds = zeros
+  PlanImage plan;
+  const float* lse;  // [B, H, N] natural-log log-sum-exp of the forward pass
+  const float* dD;   // [B, H, N] rowsum(dout * out)
+  __nv_bfloat16* dq;  // [B, N, H, d]
+  __nv_bfloat16* dk;  // [B, N, Hkv, d]
+  __nv_bfloat16* dv;
+  unsigned long long timeout_ns;
+  long long N;
+  uint32_t n_units;
+  int H, Hkv, group, T, Hg, Wg;
+  int wt, wh, ww, st, sh, sw, nwt, nwh, nww;
+  int n_windows, n_tiles, n_shapes;
+  float scale, scale_log2;
+};
+
+// Shared memory: the unit pair, a two-slot ring of step pairs, 2 KB of output
+// staging per epilogue warp, the per-row lse/D values of each ring slot (the dQ
+// kernel keeps its unit's values in slot 0), barriers, the tile plan.
+template <int D>
+struct BwdSmem {
+  static constexpr int kTile = (D / 64) * kHalf;
+  static constexpr int a0 = 0;               // A0 | A1
+  static constexpr int ring = 2 * kTile;     // slot s: B0 | B1 at ring + 2 s kTile
+  static constexpr int stg = ring + 4 * kTile;
+  static constexpr int rowv = stg + 8 * 2048;  // slot s: lse * log2(e) [128], D [128]
+  static constexpr int bars = rowv + 2 * 1024;
+  static constexpr int AFULL = 0, AEMPTY = 1, BFULL = 2, BEMPTY = 4, SFULL = 6, PFULL = 7,
+                       OFULL = 8, DRAIN = 9, NBARS = 10;
+  static constexpr int misc = bars + NBARS * 8;  // tmem slot, abort flag
+  static constexpr int plan = misc + 64;
+  static constexpr int bytes = plan + kPlanBytes;
+  static constexpr int alloc = bytes + 1024;  // slack for 1024-byte alignment
+};
+
+enum BwdWaitSite : uint32_t {
+  kBSiteLoadAEmpty = 101, kBSiteLoadBEmpty, kBSiteLoadDrainA, kBSiteLoadDrainB, kBSiteMmaAFull,
+  kBSiteMmaBFull, kBSiteMmaPFull, kBSiteMmaDrain, kBSiteEwAFull, kBSiteEwBFull, kBSiteEwSFull,
+  kBSiteEwOFull
+};
+
+struct BwdUnit {
+  WinAt w;
+  int h;     // dQ: the query head; dKV: the first query head of the group
+  int hk;    // the K/V head
+  int tile;  // dQ: the query tile; dKV: the key tile
+};
+
+// Heads fastest, then the tile, the window and the batch.
+template <bool KV>
+__device__ __forceinline__ BwdUnit decode_bwd_unit(const BwdTcParams& p, uint32_t u) {
+  BwdUnit U;
+  const uint32_t nh = (uint32_t)(KV ? p.Hkv : p.H);
+  const int head = (int)(u % nh);
+  uint32_t r = u / nh;
+  U.tile = (int)(r % (uint32_t)p.n_tiles);
+  r /= (uint32_t)p.n_tiles;
+  const int win = (int)(r % (uint32_t)p.n_windows);
+  const int b = (int)(r / (uint32_t)p.n_windows);
+  const int jw = win % p.nww, jh = (win / p.nww) % p.nwh, jt = win / (p.nww * p.nwh);
+  U.w.cls = window_class(jt, jh, jw, p.nwt, p.nwh, p.nww, p.st, p.sh, p.sw);
+  U.w.ot = jt * p.wt + p.st;
+  U.w.oh = jh * p.wh + p.sh;
+  U.w.ow = jw * p.ww + p.sw;
+  U.w.b = b;
+  if (KV) {
+    U.hk = head;
+    U.h = head * p.group;
+  } else {
+    U.h = head;
+    U.hk = head / p.group;
+  }
+  return U;
+}
+
+template <bool KV>
+__device__ __forceinline__ int bwd_steps(const BwdTcParams& p) {
+  return KV ? p.group * p.n_tiles : p.n_tiles;
+}
+
+// lse * log2(e) and D of the 128 rows of query tile `tile` of head h into
+// shared memory (dst[0..127], dst[128..255]); padding rows get +inf and 0, so
+// that their probabilities and dS vanish.  Lane l handles rows l + 32 k.
+__device__ __forceinline__ void write_row_values(const BwdTcParams& p, const PlanView& pv,
+                                                 const WinAt& w, int tile, int h, float* dst,
+                                                 int lane) {
+#pragma unroll 1
+  for (int k = 0; k < 4; ++k) {
+    const int r = lane + 32 * k;
+    const long long t = r < pv.rows[tile] ? window_row_token(pv, w, tile, r, p.T, p.Hg, p.Wg) : -1;
+    float l2 = INFINITY, dd = 0.f;
+    if (t >= 0) {
+      const long long i = ((long long)w.b * p.H + h) * p.N + t;
+      l2 = p.lse[i] * kLog2e;
+      dd = p.dD[i];
+    }
+    dst[r] = l2;
+    dst[128 + r] = dd;
+  }
+}
+
+// Writes 64 bf16 columns (w: 32 packed pairs) of this lane's row to
+// base[roff + col0 ...] (roff < 0: padding row, nothing written), through the
+// warp's 2 KB staging block: each half of 32 columns is staged as 64-byte rows
+// (16-byte chunks XOR-swizzled by row pair) and read back so that each store
+// instruction writes 64 contiguous bytes of eight rows.
+__device__ __forceinline__ void warp_store_row64(uint32_t stg, const uint32_t (&w)[32],
+                                                 long long roff, __nv_bfloat16* base, int col0,
+                                                 int lane) {
+#pragma unroll
+  for (int ps = 0; ps < 2; ++ps) {
+#pragma unroll
+    for (int ch = 0; ch < 4; ++ch)
+      st_shared_v4(stg + lane * 64 + ((ch ^ ((lane >> 1) & 3)) << 4), w[16 * ps + 4 * ch],
+                   w[16 * ps + 4 * ch + 1], w[16 * ps + 4 * ch + 2], w[16 * ps + 4 * ch + 3]);
+    __syncwarp();
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int rr = k * 8 + lane / 4, c = lane % 4;
+      const uint4 val = ld_shared_v4(stg + rr * 64 + ((c ^ ((rr >> 1) & 3)) << 4));
+      const long long t = __shfl_sync(0xffffffffu, roff, rr);
+      if (t >= 0) *reinterpret_cast<uint4*>(base + t + col0 + ps * 32 + c * 8) = val;
+    }
+    __syncwarp();
+  }
+}
+
+template <int D, bool KV>
+__global__ void __launch_bounds__(kBwdTcThreads, 1)
+    tc_bwd_kernel(const __grid_constant__ BwdTcParams p) {
+  using S = BwdSmem<D>;
+  constexpr int NH = D / 64;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t bar0 = sbase + S::bars;
+  auto BAR = [&](int i) -> uint32_t { return bar0 + 8u * (uint32_t)i; };
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + S::misc);
+  volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(smem + S::misc + 4);
+  float* rowv = reinterpret_cast<float*>(smem + S::rowv);
+
+  const int warp = threadIdx.x / 32;
+  const int lane = threadIdx.x % 32;
+  const uint64_t limit = p.timeout_ns;
+  const PlanView pv = plan_to_smem(p.plan, smem + S::plan, p.n_tiles, threadIdx.x, kBwdTcThreads);
+  if (threadIdx.x == 0) {
+    mbar_init(BAR(S::AFULL), 33);  // lane 0's expect_tx + every lane after its row values
+    mbar_init(BAR(S::AEMPTY), 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(BAR(S::BFULL + s), 33);
+      mbar_init(BAR(S::BEMPTY + s), 1);
+    }
+    mbar_init(BAR(S::SFULL), 1);
+    mbar_init(BAR(S::PFULL), 256);
+    mbar_init(BAR(S::OFULL), 1);
+    mbar_init(BAR(S::DRAIN), 1);
+    *abort_flag = 0u;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  if (threadIdx.x == 0) {
+    for (int sid = 0; sid < p.n_shapes; ++sid) {
+      prefetch_tmap(&p.qm[sid]); prefetch_tmap(&p.gm[sid]);
+      prefetch_tmap(&p.km[sid]); prefetch_tmap(&p.vm[sid]);
+    }
+    prefetch_tmap(&p.fill);
+  }
+  const int n_steps = bwd_steps<KV>(p);
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ step-pair loader
+    uint32_t nb = 0, issued = 0, last_par = 0;
+    bool ok = true;
+    for (uint32_t u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
+      const BwdUnit U = decode_bwd_unit<KV>(p, u);
+      for (int s = 0; s < n_steps && ok; ++s) {
+        const uint32_t slot = nb & 1u, par = (nb >> 1) & 1u;
+        if (!(ok = wait_warp(BAR(S::BEMPTY + slot), par ^ 1u, abort_flag, limit, kBSiteLoadBEmpty)))
+          break;
+        const uint32_t dst = sbase + S::ring + slot * 2 * S::kTile;
+        const int h = KV ? U.h + s / p.n_tiles : U.h;  // dKV: the step's query head
+        const int tile = KV ? s % p.n_tiles : s;
+        if (lane == 0) {
+          mbar_expect_tx(BAR(S::BFULL + slot), 2 * S::kTile);
+          load_window_tile<NH>(pv, KV ? p.qm : p.km, &p.fill, U.w, tile, KV ? h : U.hk, p.T, p.Hg,
+                               p.Wg, p.N, dst, BAR(S::BFULL + slot));
+          load_window_tile<NH>(pv, KV ? p.gm : p.vm, &p.fill, U.w, tile, KV ? h : U.hk, p.T, p.Hg,
+                               p.Wg, p.N, dst + S::kTile, BAR(S::BFULL + slot));
+        }
+        if (KV) write_row_values(p, pv, U.w, tile, h, rowv + slot * 256, lane);
+        mbar_arrive(BAR(S::BFULL + slot));
+        issued |= 1u << slot;
+        last_par = (last_par & ~(1u << slot)) | (par << slot);
+        ++nb;
+      }
+    }
+    for (int s = 0; s < 2; ++s)  // every copy issued has landed before the CTA exits
+      if (issued & (1u << s))
+        wait_warp(BAR(S::BFULL + s), (last_par >> s) & 1u, abort_flag, limit, kBSiteLoadDrainB,
+                  false);
+  } else if (warp == 2) {
+    // ------------------------------------------------------------ unit-pair loader
+    uint32_t na = 0;
+    bool ok = true;
+    for (uint32_t u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
+      const BwdUnit U = decode_bwd_unit<KV>(p, u);
+      if (!(ok = wait_warp(BAR(S::AEMPTY), (na & 1u) ^ 1u, abort_flag, limit, kBSiteLoadAEmpty)))
+        break;
+      const uint32_t dst = sbase + S::a0;
+      if (lane == 0) {
+        mbar_expect_tx(BAR(S::AFULL), 2 * S::kTile);
+        load_window_tile<NH>(pv, KV ? p.km : p.qm, &p.fill, U.w, U.tile, KV ? U.hk : U.h, p.T,
+                             p.Hg, p.Wg, p.N, dst, BAR(S::AFULL));
+        load_window_tile<NH>(pv, KV ? p.vm : p.gm, &p.fill, U.w, U.tile, KV ? U.hk : U.h, p.T,
+                             p.Hg, p.Wg, p.N, dst + S::kTile, BAR(S::AFULL));
+      }
+      if (!KV) write_row_values(p, pv, U.w, U.tile, U.h, rowv, lane);
+      mbar_arrive(BAR(S::AFULL));
+      ++na;
+    }
+    if (na) wait_warp(BAR(S::AFULL), (na - 1) & 1u, abort_flag, limit, kBSiteLoadDrainA, false);
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    constexpr uint32_t IDX = idesc_bf16(128, false);  // X, Y: N = 128 rows of B, K-major
+    constexpr uint32_t IDG = idesc_bf16(D, true);     // gradients: N = d, B MN-major
+    uint32_t na = 0, nb = 0, pf = 0;
+    bool ok = true;
+    auto take_b = [&](uint32_t& slot) -> bool {
+      slot = nb & 1u;
+      const uint32_t par = (nb >> 1) & 1u;
+      ++nb;
+      if (!wait_warp(BAR(S::BFULL + slot), par, abort_flag, limit, kBSiteMmaBFull)) return false;
+      tc_fence_after();
+      return true;
+    };
+    // X = A0 B0^T into columns [0, 128), Y = A1 B1^T into [128, 256) (lane 0 only)
+    auto mma_xy = [&](uint32_t slot) {
+      const uint32_t a = sbase + S::a0;
+      const uint32_t b = sbase + S::ring + slot * 2 * S::kTile;
+#pragma unroll
+      for (int t = 0; t < 2; ++t)
+#pragma unroll
+        for (int k = 0; k < D / 16; ++k) {
+          const uint32_t off = t * S::kTile + (k / 4) * kHalf + (k % 4) * 32;
+          mma_bf16(tmem + t * 128, sdesc(a + off, 16, 1024), sdesc(b + off, 16, 1024), IDX,
+                   k > 0 ? 1u : 0u);
+        }
+    };
+    // TMEM column of the bf16 operand for keys (or queries) 16 kk .. 16 kk + 15:
+    // each elementwise warpgroup packs its 64 columns into the first 32 of them.
+    auto opcol = [](int kk) -> uint32_t { return (uint32_t)(kk < 4 ? kk * 8 : 64 + (kk - 4) * 8); };
+    // the gradient MMAs of one step (lane 0 only)
+    auto mma_grad = [&](uint32_t slot, bool acc) {
+      const uint32_t b = sbase + S::ring + slot * 2 * S::kTile;
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk) {
+        const uint32_t a1 = acc || kk > 0 ? 1u : 0u;
+        if (KV) {
+          // dV += P^T dO_i (P^T over X), dK += dS^T Q_i (dS^T over Y)
+          mma_bf16_ts(tmem + 256, tmem + opcol(kk), sdesc(b + S::kTile + kk * 2048, kHalf, 1024),
+                      IDG, a1);
+          mma_bf16_ts(tmem + 256 + D, tmem + 128 + opcol(kk), sdesc(b + kk * 2048, kHalf, 1024),
+                      IDG, a1);
+        } else {
+          // dQ += dS K_j (dS over X)
+          mma_bf16_ts(tmem + 256, tmem + opcol(kk), sdesc(b + kk * 2048, kHalf, 1024), IDG, a1);
+        }
+      }
+    };
+    for (uint32_t u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
+      if (!(ok = wait_warp(BAR(S::AFULL), na & 1u, abort_flag, limit, kBSiteMmaAFull))) break;
+      ++na;
+      tc_fence_after();
+      uint32_t slot;
+      if (!(ok = take_b(slot))) break;
+      if (lane == 0) {
+        mma_xy(slot);
+        mma_commit(BAR(S::SFULL));
+      }
+      __syncwarp();
+      for (int s = 0; s < n_steps && ok; ++s) {
+        // P and dS of step s in TMEM; for s = 0 this also orders the previous
+        // unit's epilogue reads of the accumulators before the overwrite below.
+        if (!(ok = wait_warp(BAR(S::PFULL), pf & 1u, abort_flag, limit, kBSiteMmaPFull))) break;
+        ++pf;
+        tc_fence_after();
+        if (lane == 0) {
+          mma_grad(slot, s > 0);
+          mma_commit(BAR(S::BEMPTY + slot));
+          // The unit pair is read for the last time by the X, Y MMAs of the
+          // last step, and (dQ) its row values by the elementwise warps in
+          // step 0, which PFULL of step 0 covers.
+          if (n_steps == 1) mma_commit(BAR(S::AEMPTY));
+        }
+        __syncwarp();
+        if (s + 1 < n_steps) {
+          if (!(ok = take_b(slot))) break;
+          if (lane == 0) {
+            mma_xy(slot);
+            if (s + 2 == n_steps) mma_commit(BAR(S::AEMPTY));
+            mma_commit(BAR(S::SFULL));
+          }
+          __syncwarp();
+        } else {
+          if (lane == 0) mma_commit(BAR(S::OFULL));
+          __syncwarp();
+        }
+      }
+    }
+    if (lane == 0) mma_commit(BAR(S::DRAIN));  // every MMA issued completes before TMEM is freed
+    __syncwarp();
+    wait_warp(BAR(S::DRAIN), 0u, abort_flag, limit, kBSiteMmaDrain, false);
+  } else if (warp >= 4) {
+    // ------------------------------------------------------------ elementwise + epilogue
+    const int hc = (warp - 4) >> 2;  // 64-column half of X and Y
+    const int q4 = warp & 3;         // TMEM lane quadrant
+    const int r = q4 * 32 + lane;    // row of X, Y and the accumulators
+    const uint32_t tl = (uint32_t)(q4 * 32) << 16;
+    const uint32_t tX = tmem + tl + 64 * hc;
+    const uint32_t tY = tmem + tl + 128 + 64 * hc;
+    const uint32_t stg = sbase + S::stg + (uint32_t)(warp - 4) * 2048u;
+    const float c = p.scale_log2;
+    const uint64_t c2 = f2pack(c, c);
+    uint32_t sf = 0, af = 0, nb = 0, of = 0;
+    bool ok = true;
+    for (uint32_t u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
+      const BwdUnit U = decode_bwd_unit<KV>(p, u);
+      uint64_t nl2 = 0, nd2 = 0;  // dQ: -lse*log2(e) and -D of this thread's query row
+      for (int s = 0; s < n_steps; ++s) {
+        const float* rv = rowv;
+        if (!KV && s == 0) {
+          if (!(ok = wait_warp(BAR(S::AFULL), af & 1u, abort_flag, limit, kBSiteEwAFull))) break;
+          ++af;
+          nl2 = f2pack(-rowv[r], -rowv[r]);
+          nd2 = f2pack(-rowv[128 + r], -rowv[128 + r]);
+        }
+        if (KV) {
+          const uint32_t slot = nb & 1u;
+          if (!(ok = wait_warp(BAR(S::BFULL + slot), (nb >> 1) & 1u, abort_flag, limit,
+                               kBSiteEwBFull)))
+            break;
+          ++nb;
+          rv = rowv + slot * 256;
+        }
+        if (!(ok = wait_warp(BAR(S::SFULL), sf & 1u, abort_flag, limit, kBSiteEwSFull))) break;
+        ++sf;
+        tc_fence_after();
+        // Two chunks of 32 columns; each chunk's bf16 pairs go over the 16
+        // columns of X (and Y) that the chunk itself came from.
+#pragma unroll
+        for (int cc = 0; cc < 2; ++cc) {
+          uint32_t x[32], y[32];
+          tmem_ld32(tX + 32 * cc, x);
+          tmem_ld32(tY + 32 * cc, y);
+          tmem_wait_ld(x);
+          tmem_wait_ld(y);
+          uint32_t wp[16], wd[16];  // bf16 pairs of P and dS for columns 2e, 2e + 1
+          float lz = 0.f, lw = 0.f, gz = 0.f, gw = 0.f;  // dKV: the second pair of four columns
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            uint64_t l2 = nl2, d2 = nd2;
+            if (KV) {  // lse*log2(e) and D of query columns 2e, 2e + 1 (loaded four at a time)
+              if ((e % 2) == 0) {
+                const int col = 64 * hc + 32 * cc + 2 * e;
+                const uint4 L = ld_shared_v4(smem_u32(rv + col));
+                const uint4 G = ld_shared_v4(smem_u32(rv + 128 + col));
+                l2 = f2pack(-__uint_as_float(L.x), -__uint_as_float(L.y));
+                d2 = f2pack(-__uint_as_float(G.x), -__uint_as_float(G.y));
+                lz = __uint_as_float(L.z);
+                lw = __uint_as_float(L.w);
+                gz = __uint_as_float(G.z);
+                gw = __uint_as_float(G.w);
+              } else {
+                l2 = f2pack(-lz, -lw);
+                d2 = f2pack(-gz, -gw);
+              }
+            }
+            const uint64_t t2 =
+                f2fma(f2pack(__uint_as_float(x[2 * e]), __uint_as_float(x[2 * e + 1])), c2, l2);
+            float t0, t1;
+            f2unpack(t2, t0, t1);
+            const uint64_t p2 = f2pack(ex2(t0), ex2(t1));
+            const uint64_t g2 =
+                f2add(f2pack(__uint_as_float(y[2 * e]), __uint_as_float(y[2 * e + 1])), d2);
+            float p0, p1, g0, g1;
+            f2unpack(p2, p0, p1);
+            f2unpack(f2mul(g2, p2), g0, g1);
+            wp[e] = pack_bf16(p0, p1);
+            wd[e] = pack_bf16(g0, g1);
+          }
+          if (KV) {
+            tmem_st16(tX + 16 * cc, wp);  // P^T
+            tmem_st16(tY + 16 * cc, wd);  // dS^T
+          } else {
+            tmem_st16(tX + 16 * cc, wd);  // dS
+          }
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(BAR(S::PFULL));
+      }
+      if (!ok) break;
+      // epilogue: the accumulators of this unit -> bf16 -> token rows
+      if (!(ok = wait_warp(BAR(S::OFULL), of & 1u, abort_flag, limit, kBSiteEwOFull))) break;
+      ++of;
+      tc_fence_after();
+      const long long tok =
+          r < pv.rows[U.tile] ? window_row_token(pv, U.w, U.tile, r, p.T, p.Hg, p.Wg) : -1;
+      if (KV) {
+        // warpgroup 0 writes dV, warpgroup 1 writes dK (times the scale)
+        const long long roff = tok >= 0 ? (((long long)U.w.b * p.N + tok) * p.Hkv + U.hk) * D : -1;
+        __nv_bfloat16* base = hc == 0 ? p.dv : p.dk;
+        const float mul = hc == 0 ? 1.0f : p.scale;
+        const uint64_t m2 = f2pack(mul, mul);
+#pragma unroll
+        for (int hf = 0; hf < NH; ++hf) {
+          uint32_t o[2][32];
+          tmem_ld32(tmem + tl + 256 + hc * D + hf * 64, o[0]);
+          tmem_ld32(tmem + tl + 256 + hc * D + hf * 64 + 32, o[1]);
+          tmem_wait_ld(o[0]);
+          tmem_wait_ld(o[1]);
+          uint32_t w[32];
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            float o0, o1;
+            f2unpack(f2mul(f2pack(__uint_as_float(o[e / 16][(2 * e) % 32]),
+                                  __uint_as_float(o[e / 16][(2 * e) % 32 + 1])), m2), o0, o1);
+            w[e] = pack_bf16(o0, o1);
+          }
+          warp_store_row64(stg, w, roff, base, hf * 64, lane);
+        }
+      } else if (hc < NH) {
+        // warpgroup hc writes columns [64 hc, 64 hc + 64) of dQ (times the scale)
+        const long long roff = tok >= 0 ? (((long long)U.w.b * p.N + tok) * p.H + U.h) * D : -1;
+        const uint64_t m2 = f2pack(p.scale, p.scale);
+        uint32_t o[2][32];
+        tmem_ld32(tmem + tl + 256 + hc * 64, o[0]);
+        tmem_ld32(tmem + tl + 256 + hc * 64 + 32, o[1]);
+        tmem_wait_ld(o[0]);
+        tmem_wait_ld(o[1]);
+        uint32_t w[32];
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          float o0, o1;
+          f2unpack(f2mul(f2pack(__uint_as_float(o[e / 16][(2 * e) % 32]),
+                                __uint_as_float(o[e / 16][(2 * e) % 32 + 1])), m2), o0, o1);
+          w[e] = pack_bf16(o0, o1);
+        }
+        warp_store_row64(stg, w, roff, p.dq, hc * 64, lane);
+      }
+      tc_fence_before();  // the reads of the accumulators precede the next unit's MMAs
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) {
+    __syncwarp();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+template <int D, bool KV>
+basa_status launch_bwd_kernel(BwdTcParams* prm, long long units, cudaStream_t stream) {
+  static_assert(BwdSmem<D>::alloc <= 232448, "shared memory plan exceeds 227 KB");
+  const int smem = BwdSmem<D>::alloc;
+  if (units > 0x7fffffffLL) return BASA_ERR_UNSUPPORTED;
+  if (cudaFuncSetAttribute(tc_bwd_kernel<D, KV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           smem) != cudaSuccess)
+    return BASA_ERR_CUDA;
+  prm->n_units = (uint32_t)units;
+  long long grid = tc_sm_count();
+  if (grid > units) grid = units;
+  tc_bwd_kernel<D, KV><<<(unsigned)grid, kBwdTcThreads, smem, stream>>>(*prm);
+  return cudaGetLastError() == cudaSuccess ? BASA_OK : BASA_ERR_CUDA;
+}
+
+basa_status build_and_launch_bwd(BwdTcParams* prm, const Dims& d, const TilePlan& plan,
+                                 const void* q, const void* k, const void* v, const void* out,
+                                 const void* dout, const float* lse, float* dD, void* dq,
+                                 void* dk, void* dv, uint32_t timeout_ms, cudaStream_t stream) {
+  basa_status st;
+  const uint64_t D = (uint64_t)d.d, H = (uint64_t)d.H, Hk = (uint64_t)d.Hkv;
+  if ((st = pack_plan_image(plan, &prm->plan)) != BASA_OK) return st;
+  const uint64_t qdims[5] = {D, H, (uint64_t)d.Wg, (uint64_t)d.Hg, (uint64_t)d.B * d.T};
+  const uint64_t qstr[4] = {D * 2, H * D * 2, (uint64_t)d.Wg * H * D * 2,
+                            (uint64_t)d.Hg * d.Wg * H * D * 2};
+  const uint64_t kdims[5] = {D, Hk, (uint64_t)d.Wg, (uint64_t)d.Hg, (uint64_t)d.B * d.T};
+  const uint64_t kstr[4] = {D * 2, Hk * D * 2, (uint64_t)d.Wg * Hk * D * 2,
+                            (uint64_t)d.Hg * d.Wg * Hk * D * 2};
+  for (int s = 0; s < plan.n_shapes; ++s) {
+    const uint32_t box[5] = {64, 1, plan.shape_bw[s], plan.shape_bh[s], plan.shape_bt[s]};
+    if ((st = encode_map(&prm->qm[s], q, 5, qdims, qstr, box)) != BASA_OK) return st;
+    if ((st = encode_map(&prm->gm[s], dout, 5, qdims, qstr, box)) != BASA_OK) return st;
+    if ((st = encode_map(&prm->km[s], k, 5, kdims, kstr, box)) != BASA_OK) return st;
+    if ((st = encode_map(&prm->vm[s], v, 5, kdims, kstr, box)) != BASA_OK) return st;
+  }
+  {
+    const uint64_t fdims[4] = {D, Hk, (uint64_t)d.N, (uint64_t)d.B};
+    const uint64_t fstr[3] = {D * 2, Hk * D * 2, (uint64_t)d.N * Hk * D * 2};
+    const uint32_t box8[4] = {64, 1, 8, 1};
+    if ((st = encode_map(&prm->fill, k, 4, fdims, fstr, box8)) != BASA_OK) return st;
+  }
+  prm->lse = lse;
+  prm->dD = dD;
+  prm->dq = static_cast<__nv_bfloat16*>(dq);
+  prm->dk = static_cast<__nv_bfloat16*>(dk);
+  prm->dv = static_cast<__nv_bfloat16*>(dv);
+  prm->timeout_ns = (unsigned long long)(timeout_ms ? timeout_ms : 2000u) * 1000000ull;
+  prm->N = d.N;
+  prm->H = d.H; prm->Hkv = d.Hkv; prm->group = d.H / d.Hkv;
+  prm->T = d.T; prm->Hg = d.Hg; prm->Wg = d.Wg;
+  prm->wt = d.wt; prm->wh = d.wh; prm->ww = d.ww;
+  prm->st = d.st; prm->sh = d.sh; prm->sw = d.sw;
+  prm->nwt = d.nwt; prm->nwh = d.nwh; prm->nww = d.nww;
+  prm->n_windows = d.nwt * d.nwh * d.nww;
+  prm->n_tiles = plan.n_tiles;
+  prm->n_shapes = plan.n_shapes;
+  prm->scale = d.scale;
+  prm->scale_log2 = d.scale * kLog2e;
+  const long long per = (long long)prm->n_windows * plan.n_tiles;
+  // D = rowsum(dout * out), then dQ, then dK and dV
+  if ((st = launch_bwd_prep(d, out, dout, dD, stream)) != BASA_OK) return st;
+  if (d.d == 64) {
+    if ((st = launch_bwd_kernel<64, false>(prm, (long long)d.B * d.H * per, stream)) != BASA_OK)
+      return st;
+    return launch_bwd_kernel<64, true>(prm, (long long)d.B * d.Hkv * per, stream);
+  }
+  if ((st = launch_bwd_kernel<128, false>(prm, (long long)d.B * d.H * per, stream)) != BASA_OK)
+    return st;
+  return launch_bwd_kernel<128, true>(prm, (long long)d.B * d.Hkv * per, stream);
+}
+
+}  // namespace
+
+basa_status launch_bwd_tc(const Dims& d, const void* q, const void* k, const void* v,
+                          const void* out, const void* dout, const float* lse, float* dD,
+                          void* dq, void* dk, void* dv, uint32_t timeout_ms, cudaStream_t stream) {
+  if (d.dtype != BASA_BF16 || (d.d != 64 && d.d != 128) || d.P || d.qsep)
+    return BASA_ERR_UNSUPPORTED;
+  TilePlan plan;
+  basa_status st = build_tile_plan(d, &plan);  // before any launch
+  if (st != BASA_OK) return st;
+  BwdTcParams* prm = new (std::nothrow) BwdTcParams;
+  if (!prm) return BASA_ERR_INVALID_ARG;
+  memset(prm, 0, sizeof(*prm));
+  st = build_and_launch_bwd(prm, d, plan, q, k, v, out, dout, lse, dD, dq, dk, dv, timeout_ms,
+                            stream);
+  delete prm;
+  return st;
+}
+
+cudaError_t take_bwd_status(cudaStream_t stream, unsigned int* status, unsigned int* where) {
+  return tc_take_status(stream, status, where);
+}
+
+}  // namespace basa
