@@ -70,24 +70,52 @@ __device__ __forceinline__ long long member(const BwdArgs& a, int jt, int jh, in
   return ((long long)t * a.Hg + y) * a.Wg + x;
 }
 
-// D = rowsum(dO * O) for every (b, n, h).
-template <bool BF16, int D>
-__global__ void __launch_bounds__(kBwdThreads) bwd_prep_kernel(BwdArgs a) {
-  const long long rows = (long long)a.B * a.N * a.H;
-  const long long r = (long long)blockIdx.x * kBwdThreads + threadIdx.x;
-  if (r >= rows) return;
-  float acc = 0.f;
-  for (int c = 0; c < D; ++c) acc = fmaf(ld1<BF16>(a.dout, r * D + c), ld1<BF16>(a.o, r * D + c), acc);
-  const long long h = r % a.H, n = (r / a.H) % a.N, b = r / (a.H * a.N);
-  a.dD[(b * a.H + h) * a.N + n] = acc;
-}
-
 // Sum of x over the TPQ consecutive lanes that share one query (or key).
 template <int TPQ>
 __device__ __forceinline__ float lane_sum(float x) {
 #pragma unroll
   for (int o = 1; o < TPQ; o <<= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
   return x;
+}
+
+// D = rowsum(dO * O) for every (b, n, h).  HBM-bound: LPR = d * esize / 16
+// consecutive lanes read one row with 16-byte loads (a warp covers 32 / LPR
+// whole rows, so every load instruction reads contiguous bytes), multiply in
+// fp32 and add across their lanes.
+template <bool BF16, int D>
+__global__ void __launch_bounds__(kBwdThreads) bwd_prep_kernel(BwdArgs a) {
+  constexpr int LPR = D * (BF16 ? 2 : 4) / 16;  // lanes per row
+  constexpr int RPW = 32 / LPR;                 // rows per warp
+  const long long rows = (long long)a.B * a.N * a.H;
+  const long long warp = ((long long)blockIdx.x * kBwdThreads + threadIdx.x) / 32;
+  const int lane = threadIdx.x % 32;
+  const long long r = warp * RPW + lane / LPR;
+  const int sub = lane % LPR;
+  float acc = 0.f;
+  if (r < rows) {
+    const uint4 x = __ldcs(reinterpret_cast<const uint4*>(a.dout) + r * LPR + sub);
+    const uint4 y = __ldcs(reinterpret_cast<const uint4*>(a.o) + r * LPR + sub);
+    if (BF16) {
+      const __nv_bfloat162* hx = reinterpret_cast<const __nv_bfloat162*>(&x);
+      const __nv_bfloat162* hy = reinterpret_cast<const __nv_bfloat162*>(&y);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float2 fx = __bfloat1622float2(hx[i]), fy = __bfloat1622float2(hy[i]);
+        acc = fmaf(fx.x, fy.x, acc);
+        acc = fmaf(fx.y, fy.y, acc);
+      }
+    } else {
+      acc = fmaf(__uint_as_float(x.x), __uint_as_float(y.x), acc);
+      acc = fmaf(__uint_as_float(x.y), __uint_as_float(y.y), acc);
+      acc = fmaf(__uint_as_float(x.z), __uint_as_float(y.z), acc);
+      acc = fmaf(__uint_as_float(x.w), __uint_as_float(y.w), acc);
+    }
+  }
+  acc = lane_sum<LPR>(acc);
+  if (r < rows && sub == 0) {
+    const long long h = r % a.H, n = (r / a.H) % a.N, b = r / ((long long)a.H * a.N);
+    a.dD[(b * a.H + h) * a.N + n] = acc;
+  }
 }
 
 // dQ: one CTA per (b, h, window, query chunk); D / 32 threads per query.
@@ -239,10 +267,10 @@ basa_status launch_bwd_typed(BwdArgs& a, const Dims& d, bool prep_only, cudaStre
   a.n_chunks = (a.m + per - 1) / per;
   const long long dq_blocks = (long long)d.B * d.H * nwin * a.n_chunks;
   const long long dkv_blocks = (long long)d.B * d.Hkv * nwin * a.n_chunks;
-  if ((rows + kBwdThreads - 1) / kBwdThreads > 0x7fffffffLL || dq_blocks > 0x7fffffffLL)
-    return BASA_ERR_UNSUPPORTED;
-  bwd_prep_kernel<BF16, D><<<(unsigned)((rows + kBwdThreads - 1) / kBwdThreads), kBwdThreads, 0,
-                             stream>>>(a);
+  constexpr int rows_per_block = (kBwdThreads / 32) * (32 / (D * (BF16 ? 2 : 4) / 16));
+  const long long prep_blocks = (rows + rows_per_block - 1) / rows_per_block;
+  if (prep_blocks > 0x7fffffffLL || dq_blocks > 0x7fffffffLL) return BASA_ERR_UNSUPPORTED;
+  bwd_prep_kernel<BF16, D><<<(unsigned)prep_blocks, kBwdThreads, 0, stream>>>(a);
   if (prep_only) return cudaGetLastError() == cudaSuccess ? BASA_OK : BASA_ERR_CUDA;
   bwd_dq_kernel<BF16, D><<<(unsigned)dq_blocks, kBwdThreads, 0, stream>>>(a);
   bwd_dkv_kernel<BF16, D><<<(unsigned)dkv_blocks, kBwdThreads, 0, stream>>>(a);
