@@ -54,6 +54,7 @@ namespace {
 
 constexpr int kBwdTcThreads = 384;
 constexpr float kLog2e = 1.4426950408889634f;
+constexpr uint32_t kTmemA = 384;  // dQ: TMEM columns of Q (64) and dO (64) as bf16 pairs
 
 struct __align__(64) BwdTcParams {
   CUtensorMap qm[kMaxShapes];  // window boxes over q, rank 5: [d, H, Wg, Hg, B*T]
@@ -88,7 +89,7 @@ struct BwdSmem {
   static constexpr int rowv = stg + 8 * 2048;  // slot s: lse * log2(e) [128], D [128]
   static constexpr int bars = rowv + 2 * 1024;
   static constexpr int AFULL = 0, AEMPTY = 1, BFULL = 2, BEMPTY = 4, SFULL = 6, PFULL = 7,
-                       OFULL = 8, DRAIN = 9, NBARS = 10;
+                       OFULL = 8, DRAIN = 9, ATFULL = 10, ATFREE = 11, NBARS = 12;
   static constexpr int misc = bars + NBARS * 8;  // tmem slot, abort flag
   static constexpr int plan = misc + 64;
   static constexpr int bytes = plan + kPlanBytes;
@@ -98,7 +99,7 @@ struct BwdSmem {
 enum BwdWaitSite : uint32_t {
   kBSiteLoadAEmpty = 101, kBSiteLoadBEmpty, kBSiteLoadDrainA, kBSiteLoadDrainB, kBSiteMmaAFull,
   kBSiteMmaBFull, kBSiteMmaPFull, kBSiteMmaDrain, kBSiteEwAFull, kBSiteEwBFull, kBSiteEwSFull,
-  kBSiteEwOFull
+  kBSiteEwOFull, kBSiteEwATFree
 };
 
 struct BwdUnit {
@@ -208,7 +209,11 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
   const PlanView pv = plan_to_smem(p.plan, smem + S::plan, p.n_tiles, threadIdx.x, kBwdTcThreads);
   if (threadIdx.x == 0) {
     mbar_init(BAR(S::AFULL), 33);  // lane 0's expect_tx + every lane after its row values
-    mbar_init(BAR(S::AEMPTY), 1);
+    // dKV: the MMA warp frees the unit pair; dQ: the elementwise threads, once
+    // they have copied it into TMEM
+    mbar_init(BAR(S::AEMPTY), KV ? 1 : 256);
+    mbar_init(BAR(S::ATFULL), 256);  // dQ: the pair is in TMEM
+    mbar_init(BAR(S::ATFREE), 1);    // dQ: the last X, Y MMAs of the unit have read it
     for (int s = 0; s < 2; ++s) {
       mbar_init(BAR(S::BFULL + s), 33);
       mbar_init(BAR(S::BEMPTY + s), 1);
@@ -303,7 +308,9 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
       tc_fence_after();
       return true;
     };
-    // X = A0 B0^T into columns [0, 128), Y = A1 B1^T into [128, 256) (lane 0 only)
+    // X = A0 B0^T into columns [0, 128), Y = A1 B1^T into [128, 256) (lane 0
+    // only).  dKV reads A0, A1 from shared memory; dQ from TMEM columns
+    // [384, 448) and [448, 512), where the elementwise threads copied them.
     auto mma_xy = [&](uint32_t slot) {
       const uint32_t a = sbase + S::a0;
       const uint32_t b = sbase + S::ring + slot * 2 * S::kTile;
@@ -312,8 +319,12 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
 #pragma unroll
         for (int k = 0; k < D / 16; ++k) {
           const uint32_t off = t * S::kTile + (k / 4) * kHalf + (k % 4) * 32;
-          mma_bf16(tmem + t * 128, sdesc(a + off, 16, 1024), sdesc(b + off, 16, 1024), IDX,
-                   k > 0 ? 1u : 0u);
+          if (KV)
+            mma_bf16(tmem + t * 128, sdesc(a + off, 16, 1024), sdesc(b + off, 16, 1024), IDX,
+                     k > 0 ? 1u : 0u);
+          else
+            mma_bf16_ts(tmem + t * 128, tmem + kTmemA + t * 64 + k * 8, sdesc(b + off, 16, 1024),
+                        IDX, k > 0 ? 1u : 0u);
         }
     };
     // TMEM column of the bf16 operand for keys (or queries) 16 kk .. 16 kk + 15:
@@ -337,14 +348,20 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
         }
       }
     };
+    // The unit pair is read for the last time by the X, Y MMAs of the last
+    // step: dKV then frees its shared-memory slot, dQ its TMEM copy.
+    const int a_free = KV ? S::AEMPTY : S::ATFREE;
     for (uint32_t u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
-      if (!(ok = wait_warp(BAR(S::AFULL), na & 1u, abort_flag, limit, kBSiteMmaAFull))) break;
+      if (!(ok = wait_warp(BAR(KV ? S::AFULL : S::ATFULL), na & 1u, abort_flag, limit,
+                           kBSiteMmaAFull)))
+        break;
       ++na;
       tc_fence_after();
       uint32_t slot;
       if (!(ok = take_b(slot))) break;
       if (lane == 0) {
         mma_xy(slot);
+        if (n_steps == 1) mma_commit(BAR(a_free));
         mma_commit(BAR(S::SFULL));
       }
       __syncwarp();
@@ -357,17 +374,13 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
         if (lane == 0) {
           mma_grad(slot, s > 0);
           mma_commit(BAR(S::BEMPTY + slot));
-          // The unit pair is read for the last time by the X, Y MMAs of the
-          // last step, and (dQ) its row values by the elementwise warps in
-          // step 0, which PFULL of step 0 covers.
-          if (n_steps == 1) mma_commit(BAR(S::AEMPTY));
         }
         __syncwarp();
         if (s + 1 < n_steps) {
           if (!(ok = take_b(slot))) break;
           if (lane == 0) {
             mma_xy(slot);
-            if (s + 2 == n_steps) mma_commit(BAR(S::AEMPTY));
+            if (s + 2 == n_steps) mma_commit(BAR(a_free));
             mma_commit(BAR(S::SFULL));
           }
           __syncwarp();
@@ -391,19 +404,47 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
     const uint32_t stg = sbase + S::stg + (uint32_t)(warp - 4) * 2048u;
     const float c = p.scale_log2;
     const uint64_t c2 = f2pack(c, c);
-    uint32_t sf = 0, af = 0, nb = 0, of = 0;
+    uint32_t sf = 0, af = 0, atf = 0, nb = 0, of = 0;
     bool ok = true;
+    // dQ: copies the unit pair from shared memory into TMEM (warpgroup hc
+    // copies tile hc, Q or dO, both head-dim halves of its rows) and reads the
+    // row's -lse*log2(e) and -D; then frees the shared-memory slot, so that
+    // the next unit's pair is loaded a whole unit ahead.
+    auto copy_a = [&](uint64_t& l2, uint64_t& d2) -> bool {
+      if (!wait_warp(BAR(S::AFULL), af & 1u, abort_flag, limit, kBSiteEwAFull)) return false;
+      ++af;
+      if (!wait_warp(BAR(S::ATFREE), (atf & 1u) ^ 1u, abort_flag, limit, kBSiteEwATFree))
+        return false;
+      ++atf;
+      tc_fence_after();
+      const uint32_t src = sbase + S::a0 + hc * S::kTile;
+#pragma unroll
+      for (int hf = 0; hf < NH; ++hf) {
+        uint32_t w[32];
+#pragma unroll
+        for (int ch = 0; ch < 8; ++ch) {
+          const uint4 v4 = ld_shared_v4(src + hf * kHalf + swz(r, ch));
+          w[4 * ch] = v4.x;
+          w[4 * ch + 1] = v4.y;
+          w[4 * ch + 2] = v4.z;
+          w[4 * ch + 3] = v4.w;
+        }
+        tmem_st32(tmem + tl + kTmemA + 64 * hc + 32 * hf, w);
+      }
+      l2 = f2pack(-rowv[r], -rowv[r]);
+      d2 = f2pack(-rowv[128 + r], -rowv[128 + r]);
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(BAR(S::AEMPTY));
+      mbar_arrive(BAR(S::ATFULL));
+      return true;
+    };
+    uint64_t nl2 = 0, nd2 = 0;  // dQ: -lse*log2(e) and -D of this thread's query row
+    if (!KV && blockIdx.x < p.n_units) ok = copy_a(nl2, nd2);
     for (uint32_t u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
       const BwdUnit U = decode_bwd_unit<KV>(p, u);
-      uint64_t nl2 = 0, nd2 = 0;  // dQ: -lse*log2(e) and -D of this thread's query row
       for (int s = 0; s < n_steps; ++s) {
         const float* rv = rowv;
-        if (!KV && s == 0) {
-          if (!(ok = wait_warp(BAR(S::AFULL), af & 1u, abort_flag, limit, kBSiteEwAFull))) break;
-          ++af;
-          nl2 = f2pack(-rowv[r], -rowv[r]);
-          nd2 = f2pack(-rowv[128 + r], -rowv[128 + r]);
-        }
         if (KV) {
           const uint32_t slot = nb & 1u;
           if (!(ok = wait_warp(BAR(S::BFULL + slot), (nb >> 1) & 1u, abort_flag, limit,
@@ -470,6 +511,8 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
         mbar_arrive(BAR(S::PFULL));
       }
       if (!ok) break;
+      uint64_t nl2n = 0, nd2n = 0;
+      if (!KV && u + gridDim.x < p.n_units && !(ok = copy_a(nl2n, nd2n))) break;
       // epilogue: the accumulators of this unit -> bf16 -> token rows
       if (!(ok = wait_warp(BAR(S::OFULL), of & 1u, abort_flag, limit, kBSiteEwOFull))) break;
       ++of;
@@ -519,6 +562,8 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
         warp_store_row64(stg, w, roff, p.dq, hc * 64, lane);
       }
       tc_fence_before();  // the reads of the accumulators precede the next unit's MMAs
+      nl2 = nl2n;
+      nd2 = nd2n;
     }
   }
 
