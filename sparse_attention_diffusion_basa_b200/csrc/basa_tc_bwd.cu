@@ -443,6 +443,10 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
     if (!KV && blockIdx.x < p.n_units) ok = copy_a(nl2, nd2);
     for (uint32_t u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
       const BwdUnit U = decode_bwd_unit<KV>(p, u);
+      // the grid token of this thread's gradient row, found while the unit's
+      // first MMAs run
+      const long long tok =
+          r < pv.rows[U.tile] ? window_row_token(pv, U.w, U.tile, r, p.T, p.Hg, p.Wg) : -1;
       for (int s = 0; s < n_steps; ++s) {
         const float* rv = rowv;
         if (KV) {
@@ -517,8 +521,6 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
       if (!(ok = wait_warp(BAR(S::OFULL), of & 1u, abort_flag, limit, kBSiteEwOFull))) break;
       ++of;
       tc_fence_after();
-      const long long tok =
-          r < pv.rows[U.tile] ? window_row_token(pv, U.w, U.tile, r, p.T, p.Hg, p.Wg) : -1;
       if (KV) {
         // warpgroup 0 writes dV, warpgroup 1 writes dK (times the scale)
         const long long roff = tok >= 0 ? (((long long)U.w.b * p.N + tok) * p.Hkv + U.hk) * D : -1;
