@@ -44,8 +44,13 @@ from basa_synth import WORKLOADS, text_inputs, workload_inputs  # noqa: E402
 
 METRIC = "window-attn latency (ms) & TFLOPS/% bf16 peak; realised/theoretical N/m speedup"
 DEFAULT_WORKLOAD = "flux2048"
-TC_SOURCE = os.path.join(ROOT, "sparse_attention_diffusion_basa_b200", "csrc", "basa_tc.cu")
-POOL_SOURCE = os.path.join(ROOT, "sparse_attention_diffusion_basa_b200", "csrc", "basa_pool.cu")
+_CSRC = os.path.join(ROOT, "sparse_attention_diffusion_basa_b200", "csrc")
+# the source files whose device code each profiled kernel is built from
+KERNEL_SOURCES = {
+    "tc_attn_kernel": [os.path.join(_CSRC, "basa_tc.cu"), os.path.join(_CSRC, "tc_device.cuh")],
+    "pool_kernel": [os.path.join(_CSRC, "basa_pool.cu")],
+    "tc_bwd_kernel": [os.path.join(_CSRC, "basa_tc_bwd.cu"), os.path.join(_CSRC, "tc_device.cuh")],
+}
 
 
 def _peaks():
@@ -60,8 +65,11 @@ def _peaks():
                 "source": "fallback"}
 
 
-def _source_hash(path):
-    return hashlib.sha256(open(path, "rb").read()).hexdigest()[:16]
+def _source_hash(paths):
+    h = hashlib.sha256()
+    for path in paths:
+        h.update(open(path, "rb").read())
+    return h.hexdigest()[:16]
 
 
 def _traffic(kernel_key, workload):
@@ -70,8 +78,7 @@ def _traffic(kernel_key, workload):
     try:
         t = json.load(open(path))
         e = t[kernel_key][workload]
-        src = TC_SOURCE if kernel_key == "tc_attn_kernel" else POOL_SOURCE
-        if e["source_sha"] != _source_hash(src):
+        if e["source_sha"] != _source_hash(KERNEL_SOURCES[kernel_key]):
             return None
         return float(e["dram_bytes_per_launch"])
     except Exception:
