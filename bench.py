@@ -420,9 +420,13 @@ def main():
         cat = [torch.cat([a.reshape(w.B, N, w.H, w.d), b], 1).reshape(w.B, 1, 1, N + L, w.H, w.d)
                for a, b in ((dq, dqt), (dk, dkt), (dv, dvt))]
         out_cat = torch.empty_like(cat[0])
+        # the text pass's split workspace, allocated once outside the timed steps
+        jws = torch.empty(max(basa.joint_workspace_size(w.shape(), dq.dtype, w.window, shift, L), 1),
+                          dtype=torch.uint8, device=dev)
 
         def step():
-            basa.joint_attn(dq, dk, dv, dqt, dkt, dvt, w.window, shift, out=out, out_t=out_t)
+            basa.joint_attn(dq, dk, dv, dqt, dkt, dvt, w.window, shift, out=out, out_t=out_t,
+                            workspace=jws)
 
         def step_full():
             basa.full_attn(*cat, out=out_cat)

@@ -173,13 +173,27 @@ BASA_API basa_status basa_window_attn_gm(const void* q, const void* k, const voi
  * dtype for all, 16-byte aligned.  p gives the window and shift; its pool cell
  * must be (0, 0, 0) (text tokens take the place of the global memory), else
  * BASA_ERR_UNSUPPORTED.  L = 0 is plain window attention (text pointers
- * unused).  Two launches on `stream`: the image queries, then the text queries.
- * Validation happens before the first launch.  The caller owns every buffer.
+ * unused).  Two launches on `stream`: the image queries, then the text queries
+ * (plus a combine launch when the text pass is split, see
+ * basa_joint_workspace_size; workspace may be NULL).  Validation happens before
+ * the first launch.  The caller owns every buffer.
  */
 BASA_API basa_status basa_joint_attn(const void* q, const void* k, const void* v,
                                      const void* qt, const void* kt, const void* vt, int64_t L,
                                      void* out, void* out_t, float* lse, float* lse_t,
-                                     const basa_params* p, cudaStream_t stream);
+                                     void* workspace, const basa_params* p,
+                                     cudaStream_t stream);
+
+/*
+ * Bytes of workspace basa_joint_attn can use for L text tokens, or 0.  The
+ * text-query pass has few work units (B * H * ceil(L / 256)); when they would
+ * leave most SMs idle and a workspace of this size (16-byte aligned) is given,
+ * the pass splits its key range over the SMs, writes fp32 partial outputs and
+ * per-row (max, sum) there, and merges them in one more launch.  With a NULL
+ * workspace the pass runs unsplit.  0 for fp32, for invalid params, and when
+ * no split is chosen on the current device.
+ */
+BASA_API size_t basa_joint_workspace_size(const basa_params* p, int64_t L);
 
 /*
  * Backward of shifted window attention (no global memory): the gradients dq,

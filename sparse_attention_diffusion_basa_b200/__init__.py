@@ -20,7 +20,7 @@ from . import _lib
 from ._lib import BasaError, BasaParams, BASA_F32, BASA_BF16  # noqa: F401
 
 __all__ = ["window_attn", "window_attn_gm", "full_attn", "joint_attn", "window_attn_bwd",
-           "pool_kv", "workspace_size", "bwd_workspace_size", "get_status", "window_tiles", "make_params", "BasaError",
+           "pool_kv", "workspace_size", "bwd_workspace_size", "joint_workspace_size", "get_status", "window_tiles", "make_params", "BasaError",
            "library_path"]
 
 library_path = _lib.LIB_PATH
@@ -93,6 +93,12 @@ def bwd_workspace_size(shape, dtype, window, shift=(0, 0, 0), hkv=0) -> int:
     """Bytes of device workspace that window_attn_bwd needs for this problem."""
     return int(_lib.load().basa_bwd_workspace_size(
         ctypes.byref(make_params(shape, dtype, window, shift, (0, 0, 0), hkv=hkv))))
+
+
+def joint_workspace_size(shape, dtype, window, shift, L, hkv=0) -> int:
+    """Bytes of device workspace joint_attn uses to split its text-query pass (0: none)."""
+    return int(_lib.load().basa_joint_workspace_size(
+        ctypes.byref(make_params(shape, dtype, window, shift, (0, 0, 0), hkv=hkv)), int(L)))
 
 
 def pool_kv(k: torch.Tensor, v: torch.Tensor, pool, out=None, stream=None):
@@ -175,12 +181,14 @@ def full_attn(q, k, v, scale=None, return_lse=False, out=None, flags=0, stream=N
 
 
 def joint_attn(q, k, v, qt, kt, vt, window, shift=(0, 0, 0), scale=None, return_lse=False,
-               out=None, out_t=None, flags=0, stream=None):
+               out=None, out_t=None, workspace=None, flags=0, stream=None):
     """Joint text + image attention with shifted windows for the image queries.
 
     q, k, v: image tokens [B, T, Hg, Wg, H, d]; qt, kt, vt: text tokens [B, L, H, d].
     Image queries attend to their window plus every text token; text queries
-    attend to every token.  Returns (out, out_t) or (out, out_t, lse, lse_t)."""
+    attend to every token.  Returns (out, out_t) or (out, out_t, lse, lse_t).
+    ``workspace`` (uint8 device tensor) is allocated here when the text pass
+    splits its key range and none is given."""
     _check_inputs(q, k, v)
     hkv = _kv_heads(q, k, v)
     for t in (qt, kt, vt):
@@ -203,9 +211,15 @@ def joint_attn(q, k, v, qt, kt, vt, window, shift=(0, 0, 0), scale=None, return_
         lse = torch.empty((B, H, T * Hg * Wg), dtype=torch.float32, device=q.device)
         lse_t = torch.empty((B, H, L), dtype=torch.float32, device=q.device)
     with torch.cuda.device(q.device):
+        need = int(lib.basa_joint_workspace_size(ctypes.byref(prm), int(L)))
+        if need and workspace is None:
+            workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+        if need and (workspace.device != q.device or workspace.numel() * workspace.element_size() < need):
+            raise ValueError(f"workspace must hold {need} bytes on {q.device}")
         _lib.check(lib.basa_joint_attn(_ptr(q), _ptr(k), _ptr(v), _ptr(qt), _ptr(kt), _ptr(vt),
                                        int(L), _ptr(out), _ptr(out_t), _ptr(lse), _ptr(lse_t),
-                                       ctypes.byref(prm), _stream(q, stream)), "basa_joint_attn")
+                                       _ptr(workspace) if need else None, ctypes.byref(prm),
+                                       _stream(q, stream)), "basa_joint_attn")
     return (out, out_t, lse, lse_t) if return_lse else (out, out_t)
 
 

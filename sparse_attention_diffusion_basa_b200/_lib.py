@@ -20,7 +20,8 @@ BASA_FLAG_TEST_WITHHOLD_LOADS = 0x1
 EXPORTS = ("basa_status_string", "basa_version", "basa_workspace_size", "basa_pool_kv",
            "basa_window_attn", "basa_window_attn_gm", "basa_full_attn", "basa_get_status",
            "basa_window_tiles", "basa_window_attn_noalloc", "basa_test_exp2",
-           "basa_joint_attn", "basa_window_attn_bwd", "basa_bwd_workspace_size")
+           "basa_joint_attn", "basa_window_attn_bwd", "basa_bwd_workspace_size",
+           "basa_joint_workspace_size")
 
 
 class BasaParams(ctypes.Structure):
@@ -66,12 +67,15 @@ def load():
     lib.basa_window_attn_gm.restype = ctypes.c_int
     lib.basa_full_attn.argtypes = [vp, vp, vp, vp, vp, P, vp]
     lib.basa_full_attn.restype = ctypes.c_int
-    lib.basa_joint_attn.argtypes = [vp, vp, vp, vp, vp, vp, ctypes.c_int64, vp, vp, vp, vp, P, vp]
+    lib.basa_joint_attn.argtypes = [vp, vp, vp, vp, vp, vp, ctypes.c_int64, vp, vp, vp, vp, vp, P,
+                                    vp]
     lib.basa_joint_attn.restype = ctypes.c_int
     lib.basa_window_attn_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, P, vp]
     lib.basa_window_attn_bwd.restype = ctypes.c_int
     lib.basa_bwd_workspace_size.argtypes = [P]
     lib.basa_bwd_workspace_size.restype = ctypes.c_size_t
+    lib.basa_joint_workspace_size.argtypes = [P, ctypes.c_int64]
+    lib.basa_joint_workspace_size.restype = ctypes.c_size_t
     lib.basa_get_status.argtypes = [vp]
     lib.basa_get_status.restype = ctypes.c_int
     lib.basa_window_tiles.argtypes = [P, ctypes.POINTER(ctypes.c_int32),

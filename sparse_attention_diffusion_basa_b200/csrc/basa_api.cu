@@ -196,7 +196,7 @@ const char* basa_status_string(basa_status s) {
   return "unknown status";
 }
 
-int basa_version(void) { return 100; }
+int basa_version(void) { return 200; }
 
 size_t basa_workspace_size(const basa_params* p) {
   Dims d;
@@ -273,9 +273,28 @@ basa_status basa_window_attn_gm(const void* q, const void* k, const void* v, con
   return attn_common(d, q, k, v, kp, vp, out, lse, p, stream, false);
 }
 
+// The text-query pass of a joint call: full attention of the L text queries
+// over the N image and L text keys.
+static basa_status joint_text_dims(const basa_params* p, int64_t L, Dims* dt) {
+  basa_status s = normalise(p, true, dt);
+  if (s != BASA_OK) return s;
+  dt->P = L;
+  dt->Nq = L;
+  dt->qsep = 1;
+  return BASA_OK;
+}
+
+size_t basa_joint_workspace_size(const basa_params* p, int64_t L) {
+  Dims dt;
+  if (L <= 0 || L > (1LL << 24) || joint_text_dims(p, L, &dt) != BASA_OK) return 0;
+  if (dt.dtype != BASA_BF16 || (long long)dt.B * dt.H * dt.N == 0) return 0;
+  return flat_split_bytes(dt, flat_split_count(dt, true));
+}
+
 basa_status basa_joint_attn(const void* q, const void* k, const void* v, const void* qt,
                             const void* kt, const void* vt, int64_t L, void* out, void* out_t,
-                            float* lse, float* lse_t, const basa_params* p, cudaStream_t stream) {
+                            float* lse, float* lse_t, void* workspace, const basa_params* p,
+                            cudaStream_t stream) {
   Dims d;
   basa_status s = normalise(p, false, &d);
   if (s != BASA_OK) return s;
@@ -288,18 +307,27 @@ basa_status basa_joint_attn(const void* q, const void* k, const void* v, const v
   if ((s = check_qkvo(qt, kt, vt, out_t, lse_t)) != BASA_OK) return s;
   // the text-query pass is validated before the image pass is launched
   Dims dt;
-  if ((s = normalise(p, true, &dt)) != BASA_OK) return s;
-  dt.P = L;
-  dt.Nq = L;
-  dt.qsep = 1;
+  if ((s = joint_text_dims(p, L, &dt)) != BASA_OK) return s;
+  SplitK sk{1, nullptr, nullptr};
   if (d.dtype == BASA_BF16) {
     TilePlan plan;
     if ((s = build_tile_plan(d, &plan)) != BASA_OK) return s;
+    const int n = workspace ? flat_split_count(dt, true) : 1;
+    if (n > 1) {
+      if (misaligned(workspace)) return BASA_ERR_ALIGN;
+      const size_t o = align256((size_t)n * dt.B * dt.H * dt.Nq * dt.d * sizeof(float));
+      sk.n = n;
+      sk.part_o = static_cast<float*>(workspace);
+      sk.part_ml = reinterpret_cast<float*>(static_cast<char*>(workspace) + o);
+    }
   }
   // image queries: their window plus every text token
   d.P = L;
   if ((s = attn_common(d, q, k, v, kt, vt, out, lse, p, stream, false)) != BASA_OK) return s;
   // text queries: every image token plus every text token
+  if (d.dtype == BASA_BF16)
+    return launch_tc(dt, true, qt, k, v, kt, vt, out_t, lse_t, p->flags, p->wait_timeout_ms,
+                     stream, &sk);
   return attn_common(dt, qt, k, v, kt, vt, out_t, lse_t, p, stream, true);
 }
 

@@ -92,10 +92,27 @@ basa_status launch_simt(const Dims& d, const void* q, const void* k, const void*
                         const void* kp, const void* vp, void* out, float* lse,
                         cudaStream_t stream);
 
+// Split key range of a flat launch: n splits; the partial outputs (fp32
+// [n, B, H, Nq, d]) and per-row (max, sum) ([n, B, H, Nq, 2]) in caller memory.
+struct SplitK {
+  int n;
+  float* part_o;
+  float* part_ml;
+};
+
 // bf16 tcgen05 window / full attention.  flat = full attention over the grid.
+// sk (flat only, nullable): split the key range and combine the partials.
 basa_status launch_tc(const Dims& d, bool flat, const void* q, const void* k, const void* v,
                       const void* kp, const void* vp, void* out, float* lse, uint32_t flags,
-                      uint32_t timeout_ms, cudaStream_t stream);
+                      uint32_t timeout_ms, cudaStream_t stream, const SplitK* sk = nullptr);
+
+// Splits that keep a flat launch's grid full when it has fewer than half as
+// many units as SMs (1 = no split); the workspace bytes they need; the
+// combine kernel (bf16 out [B, Nq, H, d], lse [B, H, Nq] nullable).
+int flat_split_count(const Dims& d, bool extra_keys);
+size_t flat_split_bytes(const Dims& d, int n_splits);
+basa_status launch_split_combine(const Dims& d, const SplitK& sk, void* out, float* lse,
+                                 cudaStream_t stream);
 
 // Backward of window attention (no global memory): D = rowsum(dO * O) into dD,
 // then dQ, then dK and dV.

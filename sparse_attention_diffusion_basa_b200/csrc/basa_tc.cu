@@ -82,6 +82,15 @@ struct __align__(64) TcParams {
   int flat;
   uint32_t flags;
   float scale_log2;
+  // Split key range (flat mode): units_per_split units per split; split s
+  // covers key tiles [s * kt_per_split, ...).  With part_o set, each unit
+  // writes its unnormalised fp32 output and its (max, sum) per row there
+  // instead of the output, for a separate combine.
+  int n_splits;
+  int kt_per_split;
+  uint32_t units_per_split;
+  float* part_o;   // [n_splits, B, H, Nq, d]
+  float* part_ml;  // [n_splits, B, H, Nq, 2]: base-2 running max, sum
 };
 
 
@@ -98,14 +107,24 @@ enum WaitSite : uint32_t {
 // ---------------------------------------------------------------------------
 struct Unit {
   int b, h, hk, pair, cls, ot, oh, ow, nq;  // hk: the K/V head of query head h
+  int split, j0, nk;                        // key tiles [j0, j0 + nk)
 };
 
 // Window mode walks the heads fastest: concurrently running CTAs then read the
 // same tokens for all heads, so each token's H*d row (a few DRAM pages) is
 // fetched as a whole.  Full-attention mode walks the query-tile pairs fastest,
 // so the CTAs in flight share one (b, h)'s K and V through L2.
+template <bool kSplit>
 __device__ __forceinline__ Unit decode_unit(const TcParams& p, uint32_t u) {
   Unit U;
+  if constexpr (kSplit) {
+    const int n_kt = p.n_wkt + p.n_pkt;
+    U.split = (int)(u / p.units_per_split);
+    u %= p.units_per_split;
+    U.j0 = U.split * p.kt_per_split;
+    const int left = n_kt - U.j0;
+    U.nk = left < p.kt_per_split ? left : p.kt_per_split;
+  }
   if (p.flat) {
     U.pair = (int)(u % (uint32_t)p.n_pairs);
     const uint32_t r = u / (uint32_t)p.n_pairs;
@@ -238,7 +257,7 @@ struct Smem {
 // alternate: while softmax 0 exponentiates S_0(j+1), the tensor core runs
 // P_1(j) V_j and S_1(j+1), and the other way round, so the exponentials of one
 // tile overlap the MMAs of the other.
-template <int D, int kRing>
+template <int D, int kRing, bool kSplit>
 __global__ void __launch_bounds__(kThreads, 1) tc_attn_kernel(const __grid_constant__ TcParams p) {
   using S = Smem<D, kRing>;
   constexpr int NS = S::NS;
@@ -284,6 +303,13 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attn_kernel(const __grid_const
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const int n_kt = p.n_wkt + p.n_pkt;
+  // Key tiles of unit U: [kbeg, kend); without a split, every key tile.
+  auto kbeg = [&](const Unit& U) -> int {
+    if constexpr (kSplit) return U.j0; else return 0;
+  };
+  auto kcount = [&](const Unit& U) -> int {
+    if constexpr (kSplit) return U.nk; else return n_kt;
+  };
   // Pull every tensor map this launch uses into the TMA descriptor cache.
   if (threadIdx.x == 0) {
     if (p.flat) {
@@ -308,8 +334,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attn_kernel(const __grid_const
       uint32_t issued_mask = 0, last_par = 0;
       bool ok = true;
       for (uint32_t u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
-        const Unit U = decode_unit(p, u);
-        for (int j = 0; j < n_kt && ok; ++j) {
+        const Unit U = decode_unit<kSplit>(p, u);
+        for (int j = kbeg(U); j < kbeg(U) + kcount(U) && ok; ++j) {
           for (int kind = 1; kind <= 2 && ok; ++kind) {
             const uint32_t slot = kv % NS, par = (kv / NS) & 1u;
             if (!(ok = wait_warp(BAR(S::KVEMPTY + slot), par ^ 1u, abort_flag, limit,
@@ -342,7 +368,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attn_kernel(const __grid_const
       uint32_t q_issued = 0, q_last = 0;
       bool ok = true;
       for (uint32_t u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
-        const Unit U = decode_unit(p, u);
+        const Unit U = decode_unit<kSplit>(p, u);
         for (int i = 0; i < U.nq && ok; ++i) {
           if (!(ok = wait_warp(BAR(S::QEMPTY + i), (qn[i] & 1u) ^ 1u, abort_flag, limit,
                                kSiteLoadQEmpty)))
@@ -404,7 +430,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attn_kernel(const __grid_const
                     sdesc(va + k * 2048, kHalf, 1024), IDO, (accumulate || k > 0) ? 1u : 0u);
     };
     for (uint32_t u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
-      const Unit U = decode_unit(p, u);
+      const Unit U = decode_unit<kSplit>(p, u);
       uint32_t kslot;
       if (!(ok = take_slot(kslot))) break;
       for (int i = 0; i < U.nq && ok; ++i) {
@@ -415,14 +441,14 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attn_kernel(const __grid_const
         if (lane == 0) {
           mma_s(i, kslot);
           mma_commit(BAR(S::SFULL + i));
-          if (n_kt == 1) mma_commit(BAR(S::QEMPTY + i));  // Q_i read for the last time
+          if (kcount(U) == 1) mma_commit(BAR(S::QEMPTY + i));  // Q_i read for the last time
         }
         __syncwarp();
       }
       if (!ok) break;
       release(kslot);
-      for (int j = 0; j < n_kt && ok; ++j) {
-        const bool next = j + 1 < n_kt;
+      for (int j = 0; j < kcount(U) && ok; ++j) {
+        const bool next = j + 1 < kcount(U);
         uint32_t vslot;
         if (!(ok = take_slot(vslot))) break;
         if (next && !(ok = take_slot(kslot))) break;
@@ -439,7 +465,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attn_kernel(const __grid_const
             if (next) {
               mma_s(i, kslot);
               mma_commit(BAR(S::SFULL + i));
-              if (j + 2 == n_kt) mma_commit(BAR(S::QEMPTY + i));  // Q_i read for the last time
+              if (j + 2 == kcount(U)) mma_commit(BAR(S::QEMPTY + i));  // Q_i read for the last time
             } else {
               mma_commit(BAR(S::OFULL + i));
             }
@@ -470,11 +496,11 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attn_kernel(const __grid_const
     const float c = p.scale_log2;
     bool ok = true;
     for (uint32_t u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
-      const Unit U = decode_unit(p, u);
+      const Unit U = decode_unit<kSplit>(p, u);
       if (i >= U.nq) continue;
       const int qt = 2 * U.pair + i;
       float m = -INFINITY, l = 0.f;
-      for (int j = 0; j < n_kt; ++j) {
+      for (int j = kbeg(U); j < kbeg(U) + kcount(U); ++j) {
         if (!(ok = wait_warp(BAR(S::SFULL + i), sfull & 1u, abort_flag, limit, kSiteSmxSFull)))
           break;
         ++sfull;
@@ -538,7 +564,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attn_kernel(const __grid_const
         // O_i is stable here: S_i(j) was issued after P_i(j-1) V_{j-1}, so its
         // completion covers that MMA.  tcgen05.ld/st are warp-collective: the
         // whole warp rescales if any of its rows needs it.
-        if (j > 0 && __any_sync(0xffffffffu, alpha < 1.0f)) {
+        if (j > kbeg(U) && __any_sync(0xffffffffu, alpha < 1.0f)) {
 #pragma unroll
           for (int cc = 0; cc < D / 32; ++cc) {
             uint32_t o[32];
@@ -565,6 +591,29 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attn_kernel(const __grid_const
         break;
       ++ofull;
       tc_fence_after();
+      if constexpr (kSplit) {
+        // Split key range: this split's unnormalised fp32 output and its
+        // (max, sum) in base 2, for the combine kernel.
+        const bool valid = r < query_valid(p, pv, qt);
+        const long long row =
+            (((long long)U.split * p.B + U.b) * p.H + U.h) * p.Nq + 128LL * qt + r;
+#pragma unroll
+        for (int cc = 0; cc < D / 32; ++cc) {
+          uint32_t o[32];
+          tmem_ld32(tO + cc * 32, o);
+          tmem_wait_ld(o);
+          if (valid) {
+            float4* dst = reinterpret_cast<float4*>(p.part_o + row * D + cc * 32);
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+              dst[e] = make_float4(__uint_as_float(o[4 * e]), __uint_as_float(o[4 * e + 1]),
+                                   __uint_as_float(o[4 * e + 2]), __uint_as_float(o[4 * e + 3]));
+          }
+        }
+        if (valid) *reinterpret_cast<float2*>(p.part_ml + 2 * row) = make_float2(m, l);
+        tc_fence_before();  // the reads of O_i precede the next unit's first P.V MMA
+        continue;
+      }
       const float inv = 1.0f / l;
       const uint64_t inv2 = f2pack(inv, inv);
       if (p.warp_stores) {
@@ -663,16 +712,16 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attn_kernel(const __grid_const
   }
 }
 
-template <int D, int kRing>
+template <int D, int kRing, bool kSplit = false>
 basa_status launch_impl(TcParams* prm, cudaStream_t stream) {
   const int smem = Smem<D, kRing>::alloc;
   static_assert(Smem<D, kRing>::alloc <= 232448, "shared memory plan exceeds 227 KB");
-  if (cudaFuncSetAttribute(tc_attn_kernel<D, kRing>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           smem) != cudaSuccess)
+  if (cudaFuncSetAttribute(tc_attn_kernel<D, kRing, kSplit>,
+                           cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
     return BASA_ERR_CUDA;
   long long grid = tc_sm_count();
   if (grid > prm->n_units) grid = prm->n_units;
-  tc_attn_kernel<D, kRing><<<(unsigned)grid, kThreads, smem, stream>>>(*prm);
+  tc_attn_kernel<D, kRing, kSplit><<<(unsigned)grid, kThreads, smem, stream>>>(*prm);
   return cudaGetLastError() == cudaSuccess ? BASA_OK : BASA_ERR_CUDA;
 }
 
@@ -684,7 +733,7 @@ namespace {
 basa_status build_and_launch(TcParams* prm, const Dims& d, bool flat, const void* q,
                              const void* k, const void* v, const void* kp, const void* vp,
                              void* out, float* lse, uint32_t flags, uint32_t timeout_ms,
-                             cudaStream_t stream) {
+                             cudaStream_t stream, const SplitK* sk) {
   basa_status st = BASA_OK;
   const uint64_t D = (uint64_t)d.d;
   const uint64_t H = (uint64_t)d.H;
@@ -744,6 +793,19 @@ basa_status build_and_launch(TcParams* prm, const Dims& d, bool flat, const void
     const long long units = (long long)d.B * d.H * prm->n_pairs;
     if (units > 0x7fffffffLL) { st = BASA_ERR_UNSUPPORTED; goto done; }
     prm->n_units = (uint32_t)units;
+    if (sk && sk->n > 1) {  // split key range, partials to the caller's workspace
+      const int n_kt = prm->n_wkt + prm->n_pkt;
+      prm->n_splits = sk->n;
+      prm->kt_per_split = (n_kt + sk->n - 1) / sk->n;
+      if ((long long)(sk->n - 1) * prm->kt_per_split >= n_kt || units * sk->n > 0x7fffffffLL) {
+        st = BASA_ERR_INVALID_ARG;
+        goto done;
+      }
+      prm->units_per_split = (uint32_t)units;
+      prm->n_units = (uint32_t)(units * sk->n);
+      prm->part_o = sk->part_o;
+      prm->part_ml = sk->part_ml;
+    }
   } else {
     if ((st = pack_plan_image(plan, &prm->plan)) != BASA_OK) goto done;
     const uint64_t dims[5] = {D, H, (uint64_t)d.Wg, (uint64_t)d.Hg, (uint64_t)d.B * d.T};
@@ -775,12 +837,17 @@ basa_status build_and_launch(TcParams* prm, const Dims& d, bool flat, const void
   // K/V ring depth: windows of at most two key tiles and no extra keys stream
   // each K/V tile once per unit and ran faster with 3 slots in flight than with
   // 4; everything else reuses K/V tiles from L2 and runs faster with 4.
-  if (d.d == 64)
+  // Split key range: its own instantiation, so that the window kernels carry
+  // none of its code.
+  if (prm->n_splits > 1)
+    st = d.d == 64 ? launch_impl<64, 8, true>(prm, stream) : launch_impl<128, 4, true>(prm, stream);
+  else if (d.d == 64)
     st = launch_impl<64, 8>(prm, stream);
   else if (!flat && prm->n_wkt + prm->n_pkt <= 2)
     st = launch_impl<128, 3>(prm, stream);
   else
     st = launch_impl<128, 4>(prm, stream);
+  if (st == BASA_OK && prm->n_splits > 1) st = launch_split_combine(d, *sk, out, lse, stream);
 done:
   return st;
 }
@@ -794,12 +861,12 @@ std::mutex g_static_params_mu;
 
 basa_status launch_tc(const Dims& d, bool flat, const void* q, const void* k, const void* v,
                       const void* kp, const void* vp, void* out, float* lse, uint32_t flags,
-                      uint32_t timeout_ms, cudaStream_t stream) {
+                      uint32_t timeout_ms, cudaStream_t stream, const SplitK* sk) {
   TcParams* prm = new (std::nothrow) TcParams;
   if (!prm) return BASA_ERR_INVALID_ARG;
   memset(prm, 0, sizeof(*prm));
   const basa_status st =
-      build_and_launch(prm, d, flat, q, k, v, kp, vp, out, lse, flags, timeout_ms, stream);
+      build_and_launch(prm, d, flat, q, k, v, kp, vp, out, lse, flags, timeout_ms, stream, sk);
   delete prm;
   return st;
 }
@@ -811,7 +878,78 @@ basa_status launch_tc_static_params(const Dims& d, bool flat, const void* q, con
   std::lock_guard<std::mutex> lock(g_static_params_mu);
   memset(&g_static_params, 0, sizeof(g_static_params));
   return build_and_launch(&g_static_params, d, flat, q, k, v, kp, vp, out, lse, flags,
-                          timeout_ms, stream);
+                          timeout_ms, stream, nullptr);
+}
+
+namespace {
+
+// Merges the split partials of every (b, h, query row): with M = max_s m_s and
+// w_s = 2^(m_s - M), out = sum_s w_s O_s / sum_s w_s l_s (rounded to bf16) and
+// lse = (M + log2 sum_s w_s l_s) ln 2.  One warp per row, D / 32 columns per lane.
+template <int D>
+__global__ void __launch_bounds__(256) split_combine_kernel(const float* po, const float* pml,
+                                                            __nv_bfloat16* out, float* lse,
+                                                            int n_splits, int H, long long Nq,
+                                                            long long rows) {
+  constexpr int C = D / 32;
+  const long long w = ((long long)blockIdx.x * blockDim.x + threadIdx.x) / 32;
+  const int lane = threadIdx.x % 32;
+  if (w >= rows) return;
+  float M = -INFINITY;
+  for (int sp = 0; sp < n_splits; ++sp) M = fmaxf(M, pml[2 * (sp * rows + w)]);
+  float den = 0.f, acc[C];
+#pragma unroll
+  for (int e = 0; e < C; ++e) acc[e] = 0.f;
+  for (int sp = 0; sp < n_splits; ++sp) {
+    const long long row = sp * rows + w;
+    const float ws = ex2(pml[2 * row] - M);
+    den = fmaf(ws, pml[2 * row + 1], den);
+    const float* src = po + row * D + lane * C;
+#pragma unroll
+    for (int e = 0; e < C; ++e) acc[e] = fmaf(ws, src[e], acc[e]);
+  }
+  const float inv = 1.0f / den;
+  const long long n = w % Nq, bh = w / Nq, h = bh % H, b = bh / H;
+  __nv_bfloat16* dst = out + ((b * Nq + n) * H + h) * D + lane * C;
+#pragma unroll
+  for (int e = 0; e < C; ++e) dst[e] = __float2bfloat16_rn(acc[e] * inv);
+  if (lse && lane == 0) lse[w] = (M + __log2f(den)) * 0.69314718055994531f;
+}
+
+}  // namespace
+
+int flat_split_count(const Dims& d, bool extra_keys) {
+  const long long nqt = (d.Nq + 127) / 128;
+  const long long units = (long long)d.B * d.H * ((nqt + 1) / 2);
+  const long long n_kt = (d.N + 127) / 128 + (extra_keys ? (d.P + 127) / 128 : 0);
+  const int sm = tc_sm_count();
+  if (units <= 0 || 2 * units > sm) return 1;
+  long long n = sm / units;
+  if (n > n_kt / 4) n = n_kt / 4;  // at least four key tiles per split
+  if (n < 2) return 1;
+  const long long per = (n_kt + n - 1) / n;
+  return (int)((n_kt + per - 1) / per);
+}
+
+size_t flat_split_bytes(const Dims& d, int n_splits) {
+  if (n_splits <= 1) return 0;
+  const size_t rows = (size_t)n_splits * d.B * d.H * d.Nq;
+  const size_t o = (rows * d.d * sizeof(float) + 255) & ~(size_t)255;
+  return o + ((rows * 2 * sizeof(float) + 255) & ~(size_t)255);
+}
+
+basa_status launch_split_combine(const Dims& d, const SplitK& sk, void* out, float* lse,
+                                 cudaStream_t stream) {
+  const long long rows = (long long)d.B * d.H * d.Nq;
+  const long long blocks = (rows * 32 + 255) / 256;
+  if (blocks > 0x7fffffffLL) return BASA_ERR_UNSUPPORTED;
+  if (d.d == 64)
+    split_combine_kernel<64><<<(unsigned)blocks, 256, 0, stream>>>(
+        sk.part_o, sk.part_ml, static_cast<__nv_bfloat16*>(out), lse, sk.n, d.H, d.Nq, rows);
+  else
+    split_combine_kernel<128><<<(unsigned)blocks, 256, 0, stream>>>(
+        sk.part_o, sk.part_ml, static_cast<__nv_bfloat16*>(out), lse, sk.n, d.H, d.Nq, rows);
+  return cudaGetLastError() == cudaSuccess ? BASA_OK : BASA_ERR_CUDA;
 }
 
 namespace {

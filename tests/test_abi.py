@@ -171,14 +171,14 @@ def test_joint_and_grouped_query_validation(lib):
     """Joint attention and grouped-query K/V are validated before anything runs."""
     f = _fake
     joint = lambda prm, L=4: lib.basa_joint_attn(f(), f(), f(), f(), f(), f(), L, f(), f(), None,
-                                                 None, ctypes.byref(prm), None)
+                                                 None, None, ctypes.byref(prm), None)
     assert joint(_p(pool=(1, 2, 2))) == 3          # text tokens take the global-memory slot
     assert joint(_p(), L=-1) == 1                   # negative text length
     assert joint(_p(shape=(0, 1, 16, 16, 2, 64))) == 0  # empty image stream: no-op
-    assert lib.basa_joint_attn(f(), f(), f(), None, f(), f(), 4, f(), f(), None, None,
+    assert lib.basa_joint_attn(f(), f(), f(), None, f(), f(), 4, f(), f(), None, None, None,
                                ctypes.byref(_p()), None) == 1  # null text q
     assert lib.basa_joint_attn(f(), f(), f(), f(0x10008), f(), f(), 4, f(), f(), None, None,
-                               ctypes.byref(_p()), None) == 4  # misaligned text q
+                               None, ctypes.byref(_p()), None) == 4  # misaligned text q
     win = lambda prm: lib.basa_window_attn(f(), f(), f(), f(), None, None, ctypes.byref(prm), None)
     prm = _p(shape=(1, 1, 16, 16, 4, 64))
     prm.Hkv = 3                                     # 4 query heads are not a multiple of 3

@@ -55,6 +55,46 @@ def test_joint_attention(basa, shape, window, shift, L, dtype):
     assert basa.get_status() == 0
 
 
+@pytest.mark.parametrize("shape,L", [((1, 1, 64, 64, 2, 128), 64),    # 33 key tiles in 7 splits
+                                     ((2, 1, 32, 64, 1, 64), 200),    # head dim 64, ragged text
+                                     ((1, 1, 64, 80, 3, 128), 300)])
+def test_joint_text_pass_split_key_range(basa, shape, L):
+    """Few text units: the text pass splits its key range over the SMs and
+    merges the partials; both the split and the unsplit call match the oracle."""
+    from sparse_attention_diffusion_basa_b200 import _lib
+    import ctypes
+    B, T, Hg, Wg, H, d = shape
+    window, shift = (1, 16, 16), (0, 8, 8)
+    prm = basa.make_params(shape, torch.bfloat16, window, shift)
+    assert _lib.load().basa_joint_workspace_size(ctypes.byref(prm), L) > 0  # the pass splits
+    q, k, v = make_qkv(shape, "bf16", 87, 88, 89)
+    qt, kt, vt = make_text_qkv(B, L, H, d, "bf16", 94, 95, 96)
+    args = [x.cuda() for x in (q, k, v, qt, kt, vt)]
+    out, out_t, lse, lse_t = basa.joint_attn(*args, window, shift, return_lse=True)
+    no_ws = torch.empty(0, dtype=torch.uint8, device="cuda")
+    torch.cuda.synchronize()
+    f = oracle.as_f64
+    ref, ref_t, rl, rl_t = oracle.joint_attn(f(q), f(k), f(v), f(qt), f(kt), f(vt),
+                                             oracle_params(shape, window, shift), want_lse=True)
+    assert_close(out, ref, "bf16", f"image {shape} L={L}")
+    assert_close(out_t, ref_t, "bf16", f"text {shape} L={L} (split)")
+    assert float(np.abs(lse_t.double().cpu().numpy() - rl_t).max()) <= 2e-2
+    # the same call without a workspace runs the text pass unsplit
+    raw = _lib.load()
+    out_t2 = torch.empty_like(args[3])
+    lse_t2 = torch.empty_like(lse_t)
+    p = lambda x: ctypes.c_void_p(x.data_ptr())
+    out2 = torch.empty_like(args[0])
+    code = raw.basa_joint_attn(*(p(x) for x in args), L, p(out2), p(out_t2), None, p(lse_t2),
+                               None, ctypes.byref(prm),
+                               ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+    assert code == 0
+    torch.cuda.synchronize()
+    assert_close(out_t2, ref_t, "bf16", f"text {shape} L={L} (unsplit)")
+    assert float(np.abs(lse_t2.double().cpu().numpy() - rl_t).max()) <= 2e-2
+    assert basa.get_status() == 0
+
+
 def test_joint_without_text_is_window_attention(basa):
     shape, window, shift = (1, 1, 32, 32, 2, 128), (1, 16, 16), (0, 8, 8)
     q, k, v = (x.cuda() for x in make_qkv(shape, "bf16", 91, 92, 93))
@@ -74,7 +114,7 @@ def test_joint_rejects_pooled_memory(basa):
     prm = basa.make_params(shape, torch.bfloat16, (1, 16, 16), (0, 8, 8), (1, 4, 4))
     p = lambda x: ctypes.c_void_p(x.data_ptr())
     code = _lib.load().basa_joint_attn(p(q), p(q), p(q), p(t), p(t), p(t), 4, p(q), p(t), None,
-                                       None, ctypes.byref(prm), None)
+                                       None, None, ctypes.byref(prm), None)
     assert code == 3  # BASA_ERR_UNSUPPORTED
 
 
