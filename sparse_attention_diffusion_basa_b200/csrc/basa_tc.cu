@@ -32,9 +32,16 @@
 // the warpgroup stages the tile and stores it with TMA boxes that mirror the
 // load boxes.
 //
+// A flat pass with few units (the text queries of a joint call) can split its
+// key tiles into ranges (template parameter kSplit): each split-unit writes its
+// unnormalised fp32 output and per-row (max, sum) to the caller's workspace and
+// split_combine_kernel merges them.
+//
 // Every mbarrier wait is bounded (wall-clock limit from the call); on expiry the
 // kernel raises the device status word, lets every role leave its loop, waits
-// (bounded) for its own copies and MMAs in flight, frees TMEM and returns.
+// (bounded) for its own copies and MMAs in flight, frees TMEM and returns.  The
+// PTX wrappers, the bounded waits and the tile-plan helpers shared with the
+// backward kernels are in tc_device.cuh.
 #include <cuda_bf16.h>
 #include <math.h>
 #include <stdio.h>
@@ -93,6 +100,17 @@ struct __align__(64) TcParams {
   float* part_ml;  // [n_splits, B, H, Nq, 2]: base-2 running max, sum
 };
 
+
+// Which exponential pairs go to the polynomial: pair e of every 16 when
+// e % kEx2Period == kEx2Period - 1 (period 3: 5 of 16 pairs); 0 = none.
+#ifndef BASA_EX2_PERIOD
+#define BASA_EX2_PERIOD 0
+#endif
+constexpr int kEx2Period = BASA_EX2_PERIOD;
+
+// Rescale O only when a tile's row max exceeds the reference max by more than
+// 2^kLazyRescale; until then the stale reference is kept (P stays <= 2^8).
+constexpr float kLazyRescale = 8.0f;
 
 // Sites recorded by the first wait that gives up (host debug output only).
 enum WaitSite : uint32_t {

@@ -284,17 +284,6 @@ __device__ __forceinline__ uint64_t ex2_poly_x2(uint64_t x2) {
                 __int_as_float(__float_as_int(q1) + (__float_as_int(t1) << 23)));
 }
 
-// Which exponential pairs go to the polynomial: pair e of every 16 when
-// e % kEx2Period == kEx2Period - 1 (period 3: 5 of 16 pairs); 0 = none.
-#ifndef BASA_EX2_PERIOD
-#define BASA_EX2_PERIOD 0
-#endif
-constexpr int kEx2Period = BASA_EX2_PERIOD;
-
-// Rescale O only when a tile's row max exceeds the reference max by more than
-// 2^kLazyRescale; until then the stale reference is kept (P stays <= 2^8).
-constexpr float kLazyRescale = 8.0f;
-
 __device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr) {
   uint4 v;
   asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
