@@ -309,29 +309,49 @@ int oracle_max_threads(void) {
 }
 
 /*
- * Gradients of window attention (no global memory) for one output gradient dO:
- * with P_ij the softmax weights of query i over the keys j of its window,
+ * Gradients of window attention for one output gradient dO: with P_ij the
+ * softmax weights of query i over its keys j (the keys of its window, plus the
+ * pooled tokens when a pool cell is set),
  *   dV_j = sum_i P_ij dO_i
  *   dP_ij = dO_i . V_j,   D_i = dO_i . O_i = sum_j P_ij dP_ij
  *   dS_ij = P_ij (dP_ij - D_i)
  *   dQ_i = scale sum_j dS_ij K_j,   dK_j = scale sum_i dS_ij Q_i
- * (the chain rule through softmax(scale * Q K^T) V restricted to each window).
- * The forward quantities are recomputed here from q, k, v; nothing is taken
- * from a forward pass.  All tensors [B, T, Hg, Wg, H, d] (k, v, dk, dv with Hkv
- * heads; with Hkv < H the query heads of one group add into the same dK, dV).
+ * (the chain rule through softmax(scale * Q K^T) V restricted to each query's
+ * keys).  A pooled token is the mean of its cell's keys (values), so its
+ * gradient, summed over every query of the batch that sees it, flows back to
+ * each token of the cell divided by the cell size.  The forward quantities are
+ * recomputed here from q, k, v; nothing is taken from a forward pass.  All
+ * tensors [B, T, Hg, Wg, H, d] (k, v, dk, dv with Hkv heads; with Hkv < H the
+ * query heads of one group add into the same dK, dV).
  */
 int oracle_window_attn_bwd(const double* q, const double* k, const double* v,
                            const double* dout, double* dq, double* dk, double* dv,
                            const oracle_params* p) {
   if (p->T % p->wt || p->Hg % p->wh || p->Wg % p->ww) return -1;
+  const int pooled = p->pt > 0 && p->ph > 0 && p->pw > 0;
+  if (pooled && (p->T % p->pt || p->Hg % p->ph || p->Wg % p->pw)) return -1;
   const int64_t d = p->d, N = p->T * p->Hg * p->Wg, m = p->wt * p->wh * p->ww;
   const int64_t nwt = p->T / p->wt, nwh = p->Hg / p->wh, nww = p->Wg / p->ww;
+  const int64_t Ph = pooled ? p->Hg / p->ph : 0, Pw = pooled ? p->Wg / p->pw : 0;
+  const int64_t Pn = pooled ? (p->T / p->pt) * Ph * Pw : 0; /* pooled tokens per batch */
+  const int64_t nk = m + Pn;                                /* keys of every query */
+  const int64_t Hk = kv_heads(p);
   memset(dq, 0, sizeof(double) * (size_t)(p->B * N * p->H * d));
-  memset(dk, 0, sizeof(double) * (size_t)(p->B * N * kv_heads(p) * d));
-  memset(dv, 0, sizeof(double) * (size_t)(p->B * N * kv_heads(p) * d));
+  memset(dk, 0, sizeof(double) * (size_t)(p->B * N * Hk * d));
+  memset(dv, 0, sizeof(double) * (size_t)(p->B * N * Hk * d));
+  double *kp = NULL, *vp = NULL, *dkp = NULL, *dvp = NULL;
+  if (pooled) {
+    const size_t np = (size_t)(p->B * Pn * Hk * d);
+    kp = (double*)malloc(sizeof(double) * np);
+    vp = (double*)malloc(sizeof(double) * np);
+    dkp = (double*)calloc(np, sizeof(double));
+    dvp = (double*)calloc(np, sizeof(double));
+    oracle_pool(k, kp, p);
+    oracle_pool(v, vp, p);
+  }
   int64_t* tok = (int64_t*)malloc(sizeof(int64_t) * (size_t)m * 3);
-  double* P = (double*)malloc(sizeof(double) * (size_t)(m * m));
-  double* dS = (double*)malloc(sizeof(double) * (size_t)(m * m));
+  double* P = (double*)malloc(sizeof(double) * (size_t)(m * nk));
+  double* dS = (double*)malloc(sizeof(double) * (size_t)(m * nk));
   for (int64_t b = 0; b < p->B; ++b)
     for (int64_t h = 0; h < p->H; ++h) {
       const int64_t hk = kv_head(p, h);
@@ -346,49 +366,79 @@ int oracle_window_attn_bwd(const double* q, const double* k, const double* v,
               tok[3 * j + 2] = floor_mod(ix * p->ww + p->sw + lx, p->Wg);
               ++j;
             }
+        /* key c2 < m: window member c2; key m + c: pooled token c of batch b */
+#define KEY(c2) ((c2) < m ? k + kv_index(p, b, tok[3 * (c2)], tok[3 * (c2) + 1], tok[3 * (c2) + 2], hk) \
+                          : kp + ((b * Pn + ((c2) - m)) * Hk + hk) * d)
+#define VAL(c2) ((c2) < m ? v + kv_index(p, b, tok[3 * (c2)], tok[3 * (c2) + 1], tok[3 * (c2) + 2], hk) \
+                          : vp + ((b * Pn + ((c2) - m)) * Hk + hk) * d)
         for (int64_t a = 0; a < m; ++a) {  /* query a: softmax row, then dS row */
           const double* qa = q + tok_index(p, b, tok[3 * a], tok[3 * a + 1], tok[3 * a + 2], h);
           const double* ga = dout + tok_index(p, b, tok[3 * a], tok[3 * a + 1], tok[3 * a + 2], h);
           double mx = -INFINITY;
-          for (int64_t c2 = 0; c2 < m; ++c2) {
-            const double* kc = k + kv_index(p, b, tok[3 * c2], tok[3 * c2 + 1], tok[3 * c2 + 2], hk);
+          for (int64_t c2 = 0; c2 < nk; ++c2) {
+            const double* kc = KEY(c2);
             double s = 0.0;
             for (int64_t c = 0; c < d; ++c) s += qa[c] * kc[c];
-            P[a * m + c2] = p->scale * s;
-            if (P[a * m + c2] > mx) mx = P[a * m + c2];
+            P[a * nk + c2] = p->scale * s;
+            if (P[a * nk + c2] > mx) mx = P[a * nk + c2];
           }
           double den = 0.0;
-          for (int64_t c2 = 0; c2 < m; ++c2) {
-            P[a * m + c2] = exp(P[a * m + c2] - mx);
-            den += P[a * m + c2];
+          for (int64_t c2 = 0; c2 < nk; ++c2) {
+            P[a * nk + c2] = exp(P[a * nk + c2] - mx);
+            den += P[a * nk + c2];
           }
           double Da = 0.0;
-          for (int64_t c2 = 0; c2 < m; ++c2) {
-            P[a * m + c2] /= den;
-            const double* vc = v + kv_index(p, b, tok[3 * c2], tok[3 * c2 + 1], tok[3 * c2 + 2], hk);
+          for (int64_t c2 = 0; c2 < nk; ++c2) {
+            P[a * nk + c2] /= den;
+            const double* vc = VAL(c2);
             double dp = 0.0;
             for (int64_t c = 0; c < d; ++c) dp += ga[c] * vc[c];
-            dS[a * m + c2] = dp;
-            Da += P[a * m + c2] * dp;
+            dS[a * nk + c2] = dp;
+            Da += P[a * nk + c2] * dp;
           }
-          for (int64_t c2 = 0; c2 < m; ++c2) dS[a * m + c2] = P[a * m + c2] * (dS[a * m + c2] - Da);
+          for (int64_t c2 = 0; c2 < nk; ++c2)
+            dS[a * nk + c2] = P[a * nk + c2] * (dS[a * nk + c2] - Da);
         }
         for (int64_t a = 0; a < m; ++a) {
           double* dqa = dq + tok_index(p, b, tok[3 * a], tok[3 * a + 1], tok[3 * a + 2], h);
           const double* qa = q + tok_index(p, b, tok[3 * a], tok[3 * a + 1], tok[3 * a + 2], h);
           const double* ga = dout + tok_index(p, b, tok[3 * a], tok[3 * a + 1], tok[3 * a + 2], h);
-          for (int64_t c2 = 0; c2 < m; ++c2) {
-            const int64_t kvo = kv_index(p, b, tok[3 * c2], tok[3 * c2 + 1], tok[3 * c2 + 2], hk);
-            const double ds = dS[a * m + c2], pw = P[a * m + c2];
+          for (int64_t c2 = 0; c2 < nk; ++c2) {
+            const double* kc = KEY(c2);
+            double* dkc = c2 < m ? dk + (kc - k) : dkp + (kc - kp);
+            double* dvc = c2 < m ? dv + (kc - k) : dvp + (kc - kp);
+            const double ds = dS[a * nk + c2], pw = P[a * nk + c2];
             for (int64_t c = 0; c < d; ++c) {
-              dqa[c] += p->scale * ds * k[kvo + c];
-              dk[kvo + c] += p->scale * ds * qa[c];
-              dv[kvo + c] += pw * ga[c];
+              dqa[c] += p->scale * ds * kc[c];
+              dkc[c] += p->scale * ds * qa[c];
+              dvc[c] += pw * ga[c];
             }
           }
         }
+#undef KEY
+#undef VAL
       }
     }
+  if (pooled) {  /* through the mean pooling: each cell token gets 1 / count of its cell's */
+    const double inv = 1.0 / (double)(p->pt * p->ph * p->pw);
+    for (int64_t b = 0; b < p->B; ++b)
+      for (int64_t t = 0; t < p->T; ++t)
+        for (int64_t y = 0; y < p->Hg; ++y)
+          for (int64_t x = 0; x < p->Wg; ++x) {
+            const int64_t cell = ((t / p->pt) * Ph + y / p->ph) * Pw + x / p->pw;
+            for (int64_t hk = 0; hk < Hk; ++hk) {
+              const int64_t o = kv_index(p, b, t, y, x, hk), po = ((b * Pn + cell) * Hk + hk) * d;
+              for (int64_t c = 0; c < d; ++c) {
+                dk[o + c] += inv * dkp[po + c];
+                dv[o + c] += inv * dvp[po + c];
+              }
+            }
+          }
+    free(kp);
+    free(vp);
+    free(dkp);
+    free(dvp);
+  }
   free(tok);
   free(P);
   free(dS);

@@ -242,15 +242,14 @@ def joint_attn(q, k, v, qt, kt, vt, prm: OracleParams, want_lse=False,
 
 
 def window_attn_bwd(q, k, v, dout, prm: OracleParams):
-    """Gradients (dq, dk, dv) of window attention (no global memory) for the
-    output gradient ``dout``; the forward is recomputed from q, k, v."""
-    if tuple(prm.pool) != (0, 0, 0):
-        raise ValueError("the backward oracle takes no pooled memory")
+    """Gradients (dq, dk, dv) of window attention for the output gradient
+    ``dout``, with the pooled global memory of ``prm.pool`` when it is set; the
+    forward is recomputed from q, k, v."""
     q, k, v, dout = (np.ascontiguousarray(x, dtype=np.float64) for x in (q, k, v, dout))
     dq, dk, dv = np.empty(q.shape), np.empty(k.shape), np.empty(v.shape)
     c = prm.c()
     rc = _load().oracle_window_attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(dout), _ptr(dq),
                                         _ptr(dk), _ptr(dv), ctypes.byref(c))
     if rc != 0:
-        raise ValueError("oracle: window size does not divide the grid")
+        raise ValueError("oracle: window or pool cell does not divide the grid")
     return dq, dk, dv

@@ -496,6 +496,63 @@ def test_backward_matches_autograd_of_masked_attention(oracle_mod, shape, window
         np.testing.assert_allclose(got, want, rtol=0, atol=1e-12)
 
 
+@pytest.mark.parametrize("shape,window,shift,pool,Hkv", [
+    ((1, 1, 4, 6, 2, 8), (1, 2, 3), (0, 1, 2), (1, 2, 3), 0),
+    ((2, 2, 4, 4, 2, 4), (2, 2, 2), (1, 1, 1), (1, 2, 2), 0),
+    ((1, 1, 4, 4, 4, 8), (1, 2, 2), (0, 1, 1), (1, 2, 2), 2),
+])
+def test_pooled_backward_matches_autograd(oracle_mod, shape, window, shift, pool, Hkv):
+    """With pooled global memory: torch autograd (fp64) through the cell means
+    (a reshape-mean), the keys and values [grid tokens, pooled tokens] and SDPA
+    with the mask [same window | every pooled token]; the pooled tokens' gradient
+    reaches k and v through the means."""
+    r = _rng(93)
+    B, T, Hg, Wg, H, d = shape
+    hk = Hkv or H
+    pt, ph, pw = pool
+    q, g = r.standard_normal(shape), r.standard_normal(shape)
+    k, v = (r.standard_normal((B, T, Hg, Wg, hk, d)) for _ in range(2))
+    prm = _P(shape, window, shift, pool)
+    prm.Hkv = Hkv
+    dq, dk, dv = oracle_mod.window_attn_bwd(q, k, v, g, prm)
+    N = T * Hg * Wg
+    Pn = (T // pt) * (Hg // ph) * (Wg // pw)
+    tq = torch.from_numpy(q).requires_grad_()
+    tk = torch.from_numpy(k).requires_grad_()
+    tv = torch.from_numpy(v).requires_grad_()
+    cells = lambda x: x.reshape(B, T // pt, pt, Hg // ph, ph, Wg // pw, pw, hk, d).mean(
+        dim=(2, 4, 6)).reshape(B, Pn, hk, d)
+    keys = lambda x: torch.cat([x.reshape(B, N, hk, d), cells(x)], 1).transpose(1, 2)
+    rep = lambda x: x.repeat_interleave(H // hk, dim=1)
+    mask = torch.cat([torch.from_numpy(_dense_mask(T, Hg, Wg, window, shift)),
+                      torch.ones(N, Pn, dtype=torch.bool)], 1)
+    o = torch.nn.functional.scaled_dot_product_attention(
+        tq.reshape(B, N, H, d).transpose(1, 2), rep(keys(tk)), rep(keys(tv)), attn_mask=mask)
+    o.backward(torch.from_numpy(g).reshape(B, N, H, d).transpose(1, 2))
+    for got, t in ((dq, tq), (dk, tk), (dv, tv)):
+        np.testing.assert_allclose(got, t.grad.numpy(), rtol=0, atol=1e-12)
+
+
+def test_pooled_backward_matches_central_differences(oracle_mod):
+    """d/dx of sum(dO * out) by central differences with pooled memory, at a few
+    coordinates of q, k, v (k and v also move the pooled tokens)."""
+    r = _rng(94)
+    shape, window, shift, pool = (1, 1, 4, 4, 1, 4), (1, 2, 2), (0, 1, 1), (1, 2, 2)
+    q, k, v, g = (r.standard_normal(shape) for _ in range(4))
+    prm = _P(shape, window, shift, pool)
+    dq, dk, dv = oracle_mod.window_attn_bwd(q, k, v, g, prm)
+    f = lambda q_, k_, v_: float((oracle_mod.window_attn(q_, k_, v_, prm) * g).sum())
+    h = 1e-6
+    for which, grad in ((0, dq), (1, dk), (2, dv)):
+        for idx in [(0, 0, 0, 0, 0, 1), (0, 0, 2, 3, 0, 2), (0, 0, 3, 0, 0, 3)]:
+            args = [q.copy(), k.copy(), v.copy()]
+            args[which][idx] += h
+            up = f(*args)
+            args[which][idx] -= 2 * h
+            dn = f(*args)
+            assert abs((up - dn) / (2 * h) - grad[idx]) < 1e-7
+
+
 def test_backward_matches_central_differences(oracle_mod):
     """d/dx of sum(dO * out) by central differences, at a few coordinates of q, k, v."""
     r = _rng(92)

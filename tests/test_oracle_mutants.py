@@ -34,8 +34,10 @@ MUTANTS = {
         "acc += x[kv_index(p, b, ct * p->pt + i, (cy * p->ph + j + 1) % p->Hg,\n"
         "                                       (cx * p->pw + l + 1) % p->Wg, h) + c];"),
     "softmax backward without the row term": (
-        "for (int64_t c2 = 0; c2 < m; ++c2) dS[a * m + c2] = P[a * m + c2] * (dS[a * m + c2] - Da);",
-        "for (int64_t c2 = 0; c2 < m; ++c2) dS[a * m + c2] = P[a * m + c2] * dS[a * m + c2];"),
+        "dS[a * nk + c2] = P[a * nk + c2] * (dS[a * nk + c2] - Da);",
+        "dS[a * nk + c2] = P[a * nk + c2] * dS[a * nk + c2];"),
+    "pooled key gradient not divided by the cell size": (
+        "dk[o + c] += inv * dkp[po + c];", "dk[o + c] += dkp[po + c];"),
     "K/V head by modulo instead of by group": (
         "static int64_t kv_head(const oracle_params* p, int64_t h) { return h / (p->H / kv_heads(p)); }",
         "static int64_t kv_head(const oracle_params* p, int64_t h) { return h % kv_heads(p); }"),
@@ -62,6 +64,9 @@ def _pins():
         "Hkv": 2}
     yield pins.test_backward_matches_autograd_of_masked_attention, {
         "shape": (1, 1, 4, 6, 2, 8), "window": (1, 2, 3), "shift": (0, 1, 2), "Hkv": 0}
+    yield pins.test_pooled_backward_matches_autograd, {
+        "shape": (1, 1, 4, 6, 2, 8), "window": (1, 2, 3), "shift": (0, 1, 2), "pool": (1, 2, 3),
+        "Hkv": 0}
     for shape, window, shift, L in pins.JOINT:
         yield pins.test_joint_matches_dense_mask_brute_force, {"shape": shape, "window": window,
                                                               "shift": shift, "L": L}
