@@ -208,12 +208,15 @@ BASA_API size_t basa_joint_workspace_size(const basa_params* p, int64_t L);
  * q, out, dout, dq: [B, T, Hg, Wg, H, d]; k, v, dk, dv: [B, T, Hg, Wg, Hkv, d]
  * (query heads of one group add into the shared dk, dv); lse: fp32 [B, H, N]
  * from the forward call; workspace: basa_bwd_workspace_size(p) bytes, 16-byte
- * aligned.  bf16 with d = 64 or 128 runs on the tensor cores: fp32 logits,
- * exponentials and accumulators, with P and dS rounded to bf16 as the operands
- * of their MMAs, and the gradients rounded once.  fp32 (and bf16 windows beyond
- * the tensor-core tile plan's bounds, or with BASA_FLAG_BWD_CUDA_CORES) runs in
- * fp32 on CUDA cores.  A pool cell in p gives BASA_ERR_UNSUPPORTED.  Three
- * launches on `stream`; nothing is allocated.
+ * aligned.  With a pool cell in p the pooled tokens join every query's keys as
+ * in the forward: their K, V are recomputed into the workspace, their gradients
+ * (summed over every query of the batch) reach dq and flow back to each cell
+ * token's dk, dv divided by the cell size.  bf16 with d = 64 or 128 runs on the
+ * tensor cores: fp32 logits, exponentials and accumulators, with P and dS
+ * rounded to bf16 as the operands of their MMAs, and the gradients rounded
+ * once.  fp32 (and bf16 windows beyond the tensor-core tile plan's bounds, or
+ * with BASA_FLAG_BWD_CUDA_CORES) runs in fp32 on CUDA cores.  Launches on
+ * `stream` only; nothing is allocated.
  */
 BASA_API size_t basa_bwd_workspace_size(const basa_params* p);
 BASA_API basa_status basa_window_attn_bwd(const void* q, const void* k, const void* v,

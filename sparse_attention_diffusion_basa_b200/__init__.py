@@ -89,10 +89,10 @@ def workspace_size(shape, dtype, window, shift=(0, 0, 0), pool=(0, 0, 0), hkv=0)
         ctypes.byref(make_params(shape, dtype, window, shift, pool, hkv=hkv))))
 
 
-def bwd_workspace_size(shape, dtype, window, shift=(0, 0, 0), hkv=0) -> int:
+def bwd_workspace_size(shape, dtype, window, shift=(0, 0, 0), pool=(0, 0, 0), hkv=0) -> int:
     """Bytes of device workspace that window_attn_bwd needs for this problem."""
     return int(_lib.load().basa_bwd_workspace_size(
-        ctypes.byref(make_params(shape, dtype, window, shift, (0, 0, 0), hkv=hkv))))
+        ctypes.byref(make_params(shape, dtype, window, shift, pool, hkv=hkv))))
 
 
 def joint_workspace_size(shape, dtype, window, shift, L, hkv=0) -> int:
@@ -223,16 +223,17 @@ def joint_attn(q, k, v, qt, kt, vt, window, shift=(0, 0, 0), scale=None, return_
     return (out, out_t, lse, lse_t) if return_lse else (out, out_t)
 
 
-def window_attn_bwd(q, k, v, out, dout, lse, window, shift=(0, 0, 0), scale=None,
-                    workspace=None, flags=0, stream=None):
+def window_attn_bwd(q, k, v, out, dout, lse, window, shift=(0, 0, 0), pool=(0, 0, 0),
+                    scale=None, workspace=None, flags=0, stream=None):
     """Gradients (dq, dk, dv) of window attention for the output gradient ``dout``.
 
-    ``out`` and ``lse`` are the forward call's output and log-sum-exp."""
+    ``out`` and ``lse`` are the forward call's output and log-sum-exp; ``pool``
+    the forward's pooled cell (its pooled K, V are recomputed in the workspace)."""
     _check_inputs(q, k, v, out, dout)
     hkv = _kv_heads(q, k, v)
     if lse is None or lse.dtype != torch.float32 or not lse.is_contiguous():
         raise ValueError("lse must be the forward's contiguous fp32 log-sum-exp")
-    prm = make_params(q.shape, q.dtype, window, shift, (0, 0, 0), scale, flags, hkv=hkv)
+    prm = make_params(q.shape, q.dtype, window, shift, pool, scale, flags, hkv=hkv)
     lib = _lib.load()
     need = int(lib.basa_bwd_workspace_size(ctypes.byref(prm)))
     if workspace is None:

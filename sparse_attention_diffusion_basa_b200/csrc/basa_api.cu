@@ -331,10 +331,18 @@ basa_status basa_joint_attn(const void* q, const void* k, const void* v, const v
   return attn_common(dt, qt, k, v, kt, vt, out_t, lse_t, p, stream, true);
 }
 
+// Backward workspace: D = rowsum(dO * O) (fp32 [B, H, N]); with pooled memory
+// also the pooled K, V (input dtype) and their gradients (fp32), [B, P, Hkv, d].
+static size_t bwd_pooled_bytes(const Dims& d, size_t esize) {
+  return align256((size_t)d.B * (size_t)d.P * (size_t)d.Hkv * (size_t)d.d * esize);
+}
+
 size_t basa_bwd_workspace_size(const basa_params* p) {
   Dims d;
   if (normalise(p, false, &d) != BASA_OK) return 0;
-  return align256((size_t)d.B * (size_t)d.H * (size_t)d.N * sizeof(float));
+  size_t n = align256((size_t)d.B * (size_t)d.H * (size_t)d.N * sizeof(float));
+  if (d.P) n += 2 * bwd_pooled_bytes(d, d.dtype == BASA_BF16 ? 2 : 4) + 2 * bwd_pooled_bytes(d, 4);
+  return n;
 }
 
 basa_status basa_window_attn_bwd(const void* q, const void* k, const void* v, const void* out,
@@ -344,7 +352,6 @@ basa_status basa_window_attn_bwd(const void* q, const void* k, const void* v, co
   Dims d;
   basa_status s = normalise(p, false, &d);
   if (s != BASA_OK) return s;
-  if (d.pt || d.ph || d.pw) return BASA_ERR_UNSUPPORTED;  // pooled keys: no backward yet
   if ((long long)d.B * d.H * d.N == 0) return BASA_OK;
   if ((s = check_qkvo(q, k, v, out, lse)) != BASA_OK) return s;
   if ((s = check_qkvo(dout, dq, dk, dv, nullptr)) != BASA_OK) return s;
@@ -352,11 +359,22 @@ basa_status basa_window_attn_bwd(const void* q, const void* k, const void* v, co
   if (!workspace) return BASA_ERR_WORKSPACE;
   if (misaligned(workspace)) return BASA_ERR_ALIGN;
   float* dD = static_cast<float*>(workspace);
-  if (!(p->flags & BASA_FLAG_BWD_CUDA_CORES) && d.dtype == BASA_BF16 && (d.d == 64 || d.d == 128)) {
-    s = launch_bwd_tc(d, q, k, v, out, dout, lse, dD, dq, dk, dv, p->wait_timeout_ms, stream);
-    if (s != BASA_ERR_UNSUPPORTED) return s;  // outside the tile plan's bounds: CUDA cores
+  PoolGrads pg{nullptr, nullptr, nullptr, nullptr};
+  if (d.P) {  // the pooled K, V the forward used, recomputed into the workspace
+    char* w = static_cast<char*>(workspace) + align256((size_t)d.B * d.H * d.N * sizeof(float));
+    const size_t pb = bwd_pooled_bytes(d, d.dtype == BASA_BF16 ? 2 : 4), pf = bwd_pooled_bytes(d, 4);
+    void* kp = w;
+    void* vp = w + pb;
+    pg = PoolGrads{kp, vp, reinterpret_cast<float*>(w + 2 * pb),
+                   reinterpret_cast<float*>(w + 2 * pb + pf)};
+    if ((s = launch_pool(d, k, v, kp, vp, stream)) != BASA_OK) return s;
   }
-  return launch_bwd(d, q, k, v, out, dout, lse, dD, dq, dk, dv, stream);
+  const PoolGrads* pgp = d.P ? &pg : nullptr;
+  if (!(p->flags & BASA_FLAG_BWD_CUDA_CORES) && d.dtype == BASA_BF16 && (d.d == 64 || d.d == 128)) {
+    s = launch_bwd_tc(d, q, k, v, out, dout, lse, dD, dq, dk, dv, pgp, p->wait_timeout_ms, stream);
+    if (s != BASA_ERR_UNSUPPORTED) return s;  // outside the tensor-core path: CUDA cores
+  }
+  return launch_bwd(d, q, k, v, out, dout, lse, dD, dq, dk, dv, pgp, stream);
 }
 
 basa_status basa_full_attn(const void* q, const void* k, const void* v, void* out, float* lse,

@@ -45,6 +45,15 @@ struct BwdArgs {
   int n_chunks;     // query (or key) chunks per window
   long long N;
   float scale;
+  // pooled global memory (P = 0: none)
+  const void* kp;   // pooled K, V [B, P, Hkv, d] in the input dtype
+  const void* vp;
+  float* dkp;       // [B, P, Hkv, d] fp32: sum over the batch's queries of dS^T Q (no scale)
+  float* dvp;       // [B, P, Hkv, d] fp32: sum of P^T dO
+  long long P;
+  int pt, ph, pw;
+  int p_chunks;     // pooled key chunks
+  float inv_count;  // 1 / (pt * ph * pw)
 };
 
 template <bool BF16>
@@ -155,15 +164,23 @@ __global__ void __launch_bounds__(kBwdThreads) bwd_dq_kernel(BwdArgs a) {
     for (int c = 0; c < DPT; ++c) qr[c] = gr[c] = 0.f;
   }
   for (int c = 0; c < DPT; ++c) acc[c] = 0.f;
-  for (int k0 = 0; k0 < a.m; k0 += kChunk) {
-    const int nk = a.m - k0 < kChunk ? a.m - k0 : kChunk;
+  const long long nkeys = a.m + a.P;  // the window's keys, then every pooled token
+  for (long long k0 = 0; k0 < nkeys; k0 += kChunk) {
+    const int nk = nkeys - k0 < kChunk ? (int)(nkeys - k0) : kChunk;
     __syncthreads();
     for (int idx = threadIdx.x; idx < nk * D; idx += kBwdThreads) {
       const int jj = idx / D, c = idx % D;
-      const long long n = member(a, jt, jh, jw, k0 + jj);
-      const long long off = (((long long)b * a.N + n) * a.Hkv + hk) * D + c;
-      ks[jj][c] = ld1<BF16>(a.k, off);
-      vs[jj][c] = ld1<BF16>(a.v, off);
+      const long long j = k0 + jj;
+      if (j < a.m) {
+        const long long n = member(a, jt, jh, jw, (int)j);
+        const long long off = (((long long)b * a.N + n) * a.Hkv + hk) * D + c;
+        ks[jj][c] = ld1<BF16>(a.k, off);
+        vs[jj][c] = ld1<BF16>(a.v, off);
+      } else {
+        const long long off = (((long long)b * a.P + (j - a.m)) * a.Hkv + hk) * D + c;
+        ks[jj][c] = ld1<BF16>(a.kp, off);
+        vs[jj][c] = ld1<BF16>(a.vp, off);
+      }
     }
     __syncthreads();
     for (int jj = 0; jj < nk; ++jj) {
@@ -184,8 +201,11 @@ __global__ void __launch_bounds__(kBwdThreads) bwd_dq_kernel(BwdArgs a) {
 }
 
 // dK, dV: one CTA per (b, K/V head, window, key chunk); the queries of every
-// head of the group are staged in turn.
-template <bool BF16, int D>
+// head of the group are staged in turn.  With pooled memory the row's share of
+// its cell's pooled gradient (dkp, dvp / count) is added before the scale.
+// POOL: the pooled tokens' gradients instead: one CTA per (b, K/V head, pooled
+// key chunk), the queries being every token of the batch; fp32 sums to dkp, dvp.
+template <bool BF16, int D, bool POOL>
 __global__ void __launch_bounds__(kBwdThreads) bwd_dkv_kernel(BwdArgs a) {
   constexpr int TPQ = D / 32;
   constexpr int DPT = D / TPQ;
@@ -194,9 +214,9 @@ __global__ void __launch_bounds__(kBwdThreads) bwd_dkv_kernel(BwdArgs a) {
   __shared__ float gs[kChunk][D];
   __shared__ float ls[kChunk], ds_[kChunk];
   long long u = blockIdx.x;
-  const int kc = (int)(u % a.n_chunks);
-  u /= a.n_chunks;
-  const int nwin = a.nwt * a.nwh * a.nww;
+  const int kc = (int)(u % (POOL ? a.p_chunks : a.n_chunks));
+  u /= (POOL ? a.p_chunks : a.n_chunks);
+  const int nwin = POOL ? 1 : a.nwt * a.nwh * a.nww;
   const int win = (int)(u % nwin);
   u /= nwin;
   const int hk = (int)(u % a.Hkv);
@@ -204,28 +224,33 @@ __global__ void __launch_bounds__(kBwdThreads) bwd_dkv_kernel(BwdArgs a) {
   const int group = a.H / a.Hkv;
   const int jw = win % a.nww, jh = (win / a.nww) % a.nwh, jt = win / (a.nww * a.nwh);
   const int part = threadIdx.x % TPQ;
-  const int lk = kc * KPC + threadIdx.x / TPQ;
-  const bool valid = lk < a.m;
+  const long long lk = (long long)kc * KPC + threadIdx.x / TPQ;
+  const bool valid = lk < (POOL ? a.P : a.m);
   float kr[DPT], vr[DPT], dk[DPT], dv[DPT];
-  long long krow = 0;
+  long long krow = 0, n_row = 0;
   if (valid) {
-    const long long n = member(a, jt, jh, jw, lk);
-    krow = (((long long)b * a.N + n) * a.Hkv + hk) * D + part * DPT;
+    if (POOL) {
+      krow = (((long long)b * a.P + lk) * a.Hkv + hk) * D + part * DPT;
+    } else {
+      n_row = member(a, jt, jh, jw, (int)lk);
+      krow = (((long long)b * a.N + n_row) * a.Hkv + hk) * D + part * DPT;
+    }
     for (int c = 0; c < DPT; ++c) {
-      kr[c] = ld1<BF16>(a.k, krow + c);
-      vr[c] = ld1<BF16>(a.v, krow + c);
+      kr[c] = ld1<BF16>(POOL ? a.kp : a.k, krow + c);
+      vr[c] = ld1<BF16>(POOL ? a.vp : a.v, krow + c);
     }
   } else {
     for (int c = 0; c < DPT; ++c) kr[c] = vr[c] = 0.f;
   }
   for (int c = 0; c < DPT; ++c) dk[c] = dv[c] = 0.f;
+  const long long nqry = POOL ? a.N : a.m;  // the queries that see these keys
   for (int h = hk * group; h < (hk + 1) * group; ++h) {
-    for (int q0 = 0; q0 < a.m; q0 += kChunk) {
-      const int nq = a.m - q0 < kChunk ? a.m - q0 : kChunk;
+    for (long long q0 = 0; q0 < nqry; q0 += kChunk) {
+      const int nq = nqry - q0 < kChunk ? (int)(nqry - q0) : kChunk;
       __syncthreads();
       for (int idx = threadIdx.x; idx < nq * D; idx += kBwdThreads) {
         const int ii = idx / D, c = idx % D;
-        const long long n = member(a, jt, jh, jw, q0 + ii);
+        const long long n = POOL ? q0 + ii : member(a, jt, jh, jw, (int)(q0 + ii));
         const long long off = (((long long)b * a.N + n) * a.H + h) * D + c;
         qs[ii][c] = ld1<BF16>(a.q, off);
         gs[ii][c] = ld1<BF16>(a.dout, off);
@@ -252,11 +277,28 @@ __global__ void __launch_bounds__(kBwdThreads) bwd_dkv_kernel(BwdArgs a) {
       }
     }
   }
-  if (valid)
+  if (!valid) return;
+  if (POOL) {
     for (int c = 0; c < DPT; ++c) {
-      st1<BF16>(a.dk, krow + c, dk[c] * a.scale);
-      st1<BF16>(a.dv, krow + c, dv[c]);
+      a.dkp[krow + c] = dk[c];
+      a.dvp[krow + c] = dv[c];
     }
+    return;
+  }
+  if (a.P) {  // this token's share of its cell's pooled gradient
+    const long long hw = (long long)a.Hg * a.Wg;
+    const long long t = n_row / hw, y = (n_row / a.Wg) % a.Hg, x = n_row % a.Wg;
+    const long long cell = ((t / a.pt) * (a.Hg / a.ph) + y / a.ph) * (a.Wg / a.pw) + x / a.pw;
+    const long long po = (((long long)b * a.P + cell) * a.Hkv + hk) * D + part * DPT;
+    for (int c = 0; c < DPT; ++c) {
+      dk[c] = fmaf(a.inv_count, a.dkp[po + c], dk[c]);
+      dv[c] = fmaf(a.inv_count, a.dvp[po + c], dv[c]);
+    }
+  }
+  for (int c = 0; c < DPT; ++c) {
+    st1<BF16>(a.dk, krow + c, dk[c] * a.scale);
+    st1<BF16>(a.dv, krow + c, dv[c]);
+  }
 }
 
 template <bool BF16, int D>
@@ -272,15 +314,34 @@ basa_status launch_bwd_typed(BwdArgs& a, const Dims& d, bool prep_only, cudaStre
   if (prep_blocks > 0x7fffffffLL || dq_blocks > 0x7fffffffLL) return BASA_ERR_UNSUPPORTED;
   bwd_prep_kernel<BF16, D><<<(unsigned)prep_blocks, kBwdThreads, 0, stream>>>(a);
   if (prep_only) return cudaGetLastError() == cudaSuccess ? BASA_OK : BASA_ERR_CUDA;
+  if (a.P) {  // the pooled tokens' gradients first: the window dK, dV add their share
+    a.p_chunks = (int)((a.P + per - 1) / per);
+    const long long pool_blocks = (long long)d.B * d.Hkv * a.p_chunks;
+    if (pool_blocks > 0x7fffffffLL) return BASA_ERR_UNSUPPORTED;
+    bwd_dkv_kernel<BF16, D, true><<<(unsigned)pool_blocks, kBwdThreads, 0, stream>>>(a);
+  }
   bwd_dq_kernel<BF16, D><<<(unsigned)dq_blocks, kBwdThreads, 0, stream>>>(a);
-  bwd_dkv_kernel<BF16, D><<<(unsigned)dkv_blocks, kBwdThreads, 0, stream>>>(a);
+  bwd_dkv_kernel<BF16, D, false><<<(unsigned)dkv_blocks, kBwdThreads, 0, stream>>>(a);
   return cudaGetLastError() == cudaSuccess ? BASA_OK : BASA_ERR_CUDA;
 }
 
 basa_status launch_bwd_common(const Dims& d, const void* q, const void* k, const void* v,
                               const void* o, const void* dout, const float* lse, float* dD,
-                              void* dq, void* dk, void* dv, bool prep_only, cudaStream_t stream) {
+                              void* dq, void* dk, void* dv, const PoolGrads* pg, bool prep_only,
+                              cudaStream_t stream) {
   BwdArgs a;
+  a.kp = a.vp = nullptr;
+  a.dkp = a.dvp = nullptr;
+  a.P = 0;
+  a.pt = a.ph = a.pw = 1;
+  a.p_chunks = 0;
+  a.inv_count = 1.0f;
+  if (pg && d.P > 0) {
+    a.kp = pg->kp; a.vp = pg->vp; a.dkp = pg->dkp; a.dvp = pg->dvp;
+    a.P = d.P;
+    a.pt = d.pt; a.ph = d.ph; a.pw = d.pw;
+    a.inv_count = 1.0f / (float)(d.pt * d.ph * d.pw);
+  }
   a.q = q; a.k = k; a.v = v; a.o = o; a.dout = dout; a.lse = lse; a.dD = dD;
   a.dq = dq; a.dk = dk; a.dv = dv;
   a.B = d.B; a.H = d.H; a.Hkv = d.Hkv; a.T = d.T; a.Hg = d.Hg; a.Wg = d.Wg;
@@ -305,14 +366,14 @@ basa_status launch_bwd_common(const Dims& d, const void* q, const void* k, const
 
 basa_status launch_bwd(const Dims& d, const void* q, const void* k, const void* v,
                        const void* o, const void* dout, const float* lse, float* dD, void* dq,
-                       void* dk, void* dv, cudaStream_t stream) {
-  return launch_bwd_common(d, q, k, v, o, dout, lse, dD, dq, dk, dv, false, stream);
+                       void* dk, void* dv, const PoolGrads* pg, cudaStream_t stream) {
+  return launch_bwd_common(d, q, k, v, o, dout, lse, dD, dq, dk, dv, pg, false, stream);
 }
 
 basa_status launch_bwd_prep(const Dims& d, const void* o, const void* dout, float* dD,
                             cudaStream_t stream) {
   return launch_bwd_common(d, nullptr, nullptr, nullptr, o, dout, nullptr, dD, nullptr, nullptr,
-                           nullptr, true, stream);
+                           nullptr, nullptr, true, stream);
 }
 
 }  // namespace basa

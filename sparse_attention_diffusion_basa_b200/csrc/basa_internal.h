@@ -114,11 +114,21 @@ size_t flat_split_bytes(const Dims& d, int n_splits);
 basa_status launch_split_combine(const Dims& d, const SplitK& sk, void* out, float* lse,
                                  cudaStream_t stream);
 
-// Backward of window attention (no global memory): D = rowsum(dO * O) into dD,
-// then dQ, then dK and dV.
+// Pooled global memory in the backward: the pooled K, V (as the forward used
+// them, in the input dtype) and fp32 buffers for the pooled tokens' gradients,
+// all [B, P, Hkv, d].
+struct PoolGrads {
+  const void* kp;
+  const void* vp;
+  float* dkp;
+  float* dvp;
+};
+
+// Backward of window attention on CUDA cores: D = rowsum(dO * O) into dD, the
+// pooled tokens' gradients (pg, nullable), then dQ, then dK and dV.
 basa_status launch_bwd(const Dims& d, const void* q, const void* k, const void* v,
                        const void* o, const void* dout, const float* lse, float* dD, void* dq,
-                       void* dk, void* dv, cudaStream_t stream);
+                       void* dk, void* dv, const PoolGrads* pg, cudaStream_t stream);
 
 // D = rowsum(dO * O) alone (fp32 [B, H, N] into dD).
 basa_status launch_bwd_prep(const Dims& d, const void* o, const void* dout, float* dD,
@@ -129,7 +139,8 @@ basa_status launch_bwd_prep(const Dims& d, const void* o, const void* dout, floa
 // shape is outside the tile plan's bounds.
 basa_status launch_bwd_tc(const Dims& d, const void* q, const void* k, const void* v,
                           const void* out, const void* dout, const float* lse, float* dD,
-                          void* dq, void* dk, void* dv, uint32_t timeout_ms, cudaStream_t stream);
+                          void* dq, void* dk, void* dv, const PoolGrads* pg, uint32_t timeout_ms,
+                          cudaStream_t stream);
 
 // The same launch with its parameter block in static storage (no host heap use);
 // calls are serialised by a lock held until the launch has copied the block.

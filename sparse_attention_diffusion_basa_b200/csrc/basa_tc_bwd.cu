@@ -653,9 +653,11 @@ basa_status build_and_launch_bwd(BwdTcParams* prm, const Dims& d, const TilePlan
 
 basa_status launch_bwd_tc(const Dims& d, const void* q, const void* k, const void* v,
                           const void* out, const void* dout, const float* lse, float* dD,
-                          void* dq, void* dk, void* dv, uint32_t timeout_ms, cudaStream_t stream) {
-  if (d.dtype != BASA_BF16 || (d.d != 64 && d.d != 128) || d.P || d.qsep)
+                          void* dq, void* dk, void* dv, const PoolGrads* pg, uint32_t timeout_ms,
+                          cudaStream_t stream) {
+  if (d.dtype != BASA_BF16 || (d.d != 64 && d.d != 128) || d.qsep || (d.P && !pg))
     return BASA_ERR_UNSUPPORTED;
+  if (d.P) return BASA_ERR_UNSUPPORTED;  // pooled memory: the CUDA-core kernels
   TilePlan plan;
   basa_status st = build_tile_plan(d, &plan);  // before any launch
   if (st != BASA_OK) return st;

@@ -95,14 +95,33 @@ def test_backward_flux1024_size(basa):
         assert_close(got, r, "bf16", f"{name} flux1024")
 
 
-def test_backward_refuses_pooled_memory(basa):
-    from sparse_attention_diffusion_basa_b200 import BasaError
-    x = torch.zeros((1, 1, 16, 16, 2, 64), device="cuda")
-    lse = torch.zeros((1, 2, 256), device="cuda")
-    import ctypes
-    from sparse_attention_diffusion_basa_b200 import _lib
-    prm = basa.make_params(x.shape, x.dtype, (1, 8, 8), (0, 4, 4), (1, 2, 2))
-    p = lambda t: ctypes.c_void_p(t.data_ptr())
-    code = _lib.load().basa_window_attn_bwd(p(x), p(x), p(x), p(x), p(x), p(lse), p(x), p(x),
-                                            p(x), p(lse), ctypes.byref(prm), None)
-    assert code == 3  # BASA_ERR_UNSUPPORTED
+POOLED = [
+    # shape, Hkv (0 = H), window, shift, pool, dtype
+    ((1, 1, 16, 16, 2, 64), 0, (1, 8, 8), (0, 4, 4), (1, 4, 4), "f32"),
+    ((1, 2, 8, 8, 2, 32), 0, (1, 4, 4), (1, 2, 2), (2, 2, 2), "f32"),
+    ((1, 1, 32, 32, 2, 128), 0, (1, 16, 16), (0, 8, 8), (1, 4, 4), "bf16"),
+    ((1, 1, 32, 32, 4, 128), 2, (1, 16, 16), (0, 8, 8), (1, 4, 4), "bf16"),
+    ((2, 1, 32, 32, 2, 64), 0, (1, 16, 16), (0, 8, 8), (1, 8, 8), "bf16"),
+]
+
+
+@pytest.mark.parametrize("shape,Hkv,window,shift,pool,dtype", POOLED)
+def test_pooled_memory_backward(basa, shape, Hkv, window, shift, pool, dtype):
+    """With K/V-pooled global memory: the pooled tokens' gradients reach every
+    query's dq and flow back to k and v through the cell means."""
+    B, T, Hg, Wg, H, d = shape
+    hk = Hkv or H
+    q, _, _ = make_qkv(shape, dtype, 181, 182, 183)
+    _, k, v = make_qkv((B, T, Hg, Wg, hk, d), dtype, 181, 182, 183)
+    g, _, _ = make_qkv(shape, dtype, 184, 185, 186)
+    dq_, dk_, dv_, dg = (x.cuda() for x in (q, k, v, g))
+    out, lse = basa.window_attn(dq_, dk_, dv_, window, shift, pool, return_lse=True)
+    gq, gk, gv = basa.window_attn_bwd(dq_, dk_, dv_, out, dg, lse, window, shift, pool)
+    torch.cuda.synchronize()
+    assert basa.get_status() == 0
+    prm = oracle_params(shape, window, shift, pool)
+    prm.Hkv = Hkv
+    f = oracle.as_f64
+    rq, rk, rv = oracle.window_attn_bwd(f(q), f(k), f(v), f(g), prm)
+    for got, ref, name in ((gq, rq, "dq"), (gk, rk, "dk"), (gv, rv, "dv")):
+        assert_close(got, ref, dtype, f"{name} {shape} pool {pool} Hkv={Hkv}")
