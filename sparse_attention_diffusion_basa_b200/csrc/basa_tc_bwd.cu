@@ -62,6 +62,8 @@ struct __align__(64) BwdTcParams {
   CUtensorMap km[kMaxShapes];  // over k: [d, Hkv, Wg, Hg, B*T]
   CUtensorMap vm[kMaxShapes];  // over v
   CUtensorMap fill;            // 8-row box over k's flat view, read out of bounds = zeros
+  CUtensorMap kpf, vpf;        // pooled K, V: [d, Hkv, P, B], 128-row boxes
+  CUtensorMap qf, gf;          // q and dout as flat rows: [d, H, N, B], 128-row boxes
   PlanImage plan;
   const float* lse;  // [B, H, N] natural-log log-sum-exp of the forward pass
   const float* dD;   // [B, H, N] rowsum(dout * out)
@@ -75,7 +77,21 @@ struct __align__(64) BwdTcParams {
   int wt, wh, ww, st, sh, sw, nwt, nwh, nww;
   int n_windows, n_tiles, n_shapes;
   float scale, scale_log2;
+  // pooled global memory (P = 0: none)
+  float* dkp;  // [B, P, Hkv, d] fp32: sum over the batch's queries of dS^T Q (no scale)
+  float* dvp;  // [B, P, Hkv, d] fp32: sum of P^T dO
+  long long P;
+  int n_pt;                      // pooled key tiles
+  int n_fqt;                     // query tiles of the whole grid (flat rows)
+  int fqt_per_split, n_fsplits;  // the pooled kernel's split of those query tiles
+  int pt, ph, pw;
+  float inv_count;               // 1 / (pt * ph * pw)
 };
+
+// Kernel modes: the dQ kernel (window key tiles, then the pooled tiles), the
+// window dK, dV kernel, and the pooled dK, dV kernel (a pooled key tile against
+// a range of the grid's query tiles, summed into dkp, dvp).
+constexpr int kModeDq = 0, kModeDkv = 1, kModePooled = 2;
 
 // Shared memory: the unit pair, a two-slot ring of step pairs, 2 KB of output
 // staging per epilogue warp, the per-row lse/D values of each ring slot (the dQ
@@ -106,13 +122,31 @@ struct BwdUnit {
   WinAt w;
   int h;     // dQ: the query head; dKV: the first query head of the group
   int hk;    // the K/V head
-  int tile;  // dQ: the query tile; dKV: the key tile
+  int tile;  // dQ: the query tile; dKV: the key tile; pooled: the pooled key tile
+  int q0, nq;  // pooled: the unit's query tiles [q0, q0 + nq) of the grid
 };
 
-// Heads fastest, then the tile, the window and the batch.
-template <bool KV>
+// Heads fastest, then the tile, the window and the batch (pooled: the K/V
+// head, the pooled tile, the query-tile split, the batch).
+template <int MODE>
 __device__ __forceinline__ BwdUnit decode_bwd_unit(const BwdTcParams& p, uint32_t u) {
+  constexpr bool KV = MODE != kModeDq;
   BwdUnit U;
+  if constexpr (MODE == kModePooled) {
+    U.hk = (int)(u % (uint32_t)p.Hkv);
+    U.h = U.hk * p.group;
+    uint32_t r = u / (uint32_t)p.Hkv;
+    U.tile = (int)(r % (uint32_t)p.n_pt);
+    r /= (uint32_t)p.n_pt;
+    const int sp = (int)(r % (uint32_t)p.n_fsplits);
+    U.w.b = (int)(r / (uint32_t)p.n_fsplits);
+    U.w.cls = U.w.ot = U.w.oh = U.w.ow = 0;
+    U.q0 = sp * p.fqt_per_split;
+    const int left = p.n_fqt - U.q0;
+    U.nq = left < p.fqt_per_split ? left : p.fqt_per_split;
+    return U;
+  }
+  U.q0 = U.nq = 0;
   const uint32_t nh = (uint32_t)(KV ? p.Hkv : p.H);
   const int head = (int)(u % nh);
   uint32_t r = u / nh;
@@ -136,9 +170,14 @@ __device__ __forceinline__ BwdUnit decode_bwd_unit(const BwdTcParams& p, uint32_
   return U;
 }
 
-template <bool KV>
-__device__ __forceinline__ int bwd_steps(const BwdTcParams& p) {
-  return KV ? p.group * p.n_tiles : p.n_tiles;
+// Steps of unit U: dQ, the window's key tiles then the pooled tiles; dKV, the
+// group's query heads times the window's query tiles; pooled, the group's query
+// heads times the unit's query tiles.
+template <int MODE>
+__device__ __forceinline__ int bwd_steps(const BwdTcParams& p, const BwdUnit& U) {
+  if constexpr (MODE == kModeDq) return p.n_tiles + p.n_pt;
+  if constexpr (MODE == kModeDkv) return p.group * p.n_tiles;
+  return p.group * U.nq;
 }
 
 // lse * log2(e) and D of the 128 rows of query tile `tile` of head h into
@@ -156,6 +195,24 @@ __device__ __forceinline__ void write_row_values(const BwdTcParams& p, const Pla
       const long long i = ((long long)w.b * p.H + h) * p.N + t;
       l2 = p.lse[i] * kLog2e;
       dd = p.dD[i];
+    }
+    dst[r] = l2;
+    dst[128 + r] = dd;
+  }
+}
+
+// The same for flat query tile i of the grid (rows 128 i .. 128 i + 127).
+__device__ __forceinline__ void write_row_values_flat(const BwdTcParams& p, int b, int i, int h,
+                                                      float* dst, int lane) {
+#pragma unroll 1
+  for (int k = 0; k < 4; ++k) {
+    const int r = lane + 32 * k;
+    const long long n = 128LL * i + r;
+    float l2 = INFINITY, dd = 0.f;
+    if (n < p.N) {
+      const long long x = ((long long)b * p.H + h) * p.N + n;
+      l2 = p.lse[x] * kLog2e;
+      dd = p.dD[x];
     }
     dst[r] = l2;
     dst[128 + r] = dd;
@@ -188,11 +245,12 @@ __device__ __forceinline__ void warp_store_row64(uint32_t stg, const uint32_t (&
   }
 }
 
-template <int D, bool KV>
+template <int D, int MODE>
 __global__ void __launch_bounds__(kBwdTcThreads, 1)
     tc_bwd_kernel(const __grid_constant__ BwdTcParams p) {
   using S = BwdSmem<D>;
   constexpr int NH = D / 64;
+  constexpr bool KV = MODE != kModeDq;  // dK, dV accumulators (window or pooled keys)
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -239,30 +297,54 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
       prefetch_tmap(&p.km[sid]); prefetch_tmap(&p.vm[sid]);
     }
     prefetch_tmap(&p.fill);
+    if (p.P) { prefetch_tmap(&p.kpf); prefetch_tmap(&p.vpf); }
+    if (MODE == kModePooled) { prefetch_tmap(&p.qf); prefetch_tmap(&p.gf); }
   }
-  const int n_steps = bwd_steps<KV>(p);
 
   if (warp == 0) {
     // ------------------------------------------------------------ step-pair loader
     uint32_t nb = 0, issued = 0, last_par = 0;
     bool ok = true;
     for (uint32_t u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
-      const BwdUnit U = decode_bwd_unit<KV>(p, u);
+      const BwdUnit U = decode_bwd_unit<MODE>(p, u);
+      const int n_steps = bwd_steps<MODE>(p, U);
+      const int per_head = MODE == kModePooled ? U.nq : p.n_tiles;
       for (int s = 0; s < n_steps && ok; ++s) {
         const uint32_t slot = nb & 1u, par = (nb >> 1) & 1u;
         if (!(ok = wait_warp(BAR(S::BEMPTY + slot), par ^ 1u, abort_flag, limit, kBSiteLoadBEmpty)))
           break;
         const uint32_t dst = sbase + S::ring + slot * 2 * S::kTile;
-        const int h = KV ? U.h + s / p.n_tiles : U.h;  // dKV: the step's query head
-        const int tile = KV ? s % p.n_tiles : s;
+        const uint32_t bar = BAR(S::BFULL + slot);
+        const int h = KV ? U.h + s / per_head : U.h;  // dKV: the step's query head
+        const int tile = KV ? s % per_head : s;
         if (lane == 0) {
-          mbar_expect_tx(BAR(S::BFULL + slot), 2 * S::kTile);
-          load_window_tile<NH>(pv, KV ? p.qm : p.km, &p.fill, U.w, tile, KV ? h : U.hk, p.T, p.Hg,
-                               p.Wg, p.N, dst, BAR(S::BFULL + slot));
-          load_window_tile<NH>(pv, KV ? p.gm : p.vm, &p.fill, U.w, tile, KV ? h : U.hk, p.T, p.Hg,
-                               p.Wg, p.N, dst + S::kTile, BAR(S::BFULL + slot));
+          mbar_expect_tx(bar, 2 * S::kTile);
+          if (MODE == kModePooled) {  // flat query tile U.q0 + tile of the grid
+#pragma unroll
+            for (int hf = 0; hf < NH; ++hf) {
+              tma_load_4d(dst + hf * kHalf, &p.qf, bar, hf * 64, h, (U.q0 + tile) * 128, U.w.b);
+              tma_load_4d(dst + S::kTile + hf * kHalf, &p.gf, bar, hf * 64, h,
+                          (U.q0 + tile) * 128, U.w.b);
+            }
+          } else if (!KV && tile >= p.n_tiles) {  // dQ: pooled key tile
+#pragma unroll
+            for (int hf = 0; hf < NH; ++hf) {
+              tma_load_4d(dst + hf * kHalf, &p.kpf, bar, hf * 64, U.hk, (tile - p.n_tiles) * 128,
+                          U.w.b);
+              tma_load_4d(dst + S::kTile + hf * kHalf, &p.vpf, bar, hf * 64, U.hk,
+                          (tile - p.n_tiles) * 128, U.w.b);
+            }
+          } else {
+            load_window_tile<NH>(pv, KV ? p.qm : p.km, &p.fill, U.w, tile, KV ? h : U.hk, p.T,
+                                 p.Hg, p.Wg, p.N, dst, bar);
+            load_window_tile<NH>(pv, KV ? p.gm : p.vm, &p.fill, U.w, tile, KV ? h : U.hk, p.T,
+                                 p.Hg, p.Wg, p.N, dst + S::kTile, bar);
+          }
         }
-        if (KV) write_row_values(p, pv, U.w, tile, h, rowv + slot * 256, lane);
+        if (MODE == kModePooled)
+          write_row_values_flat(p, U.w.b, U.q0 + tile, h, rowv + slot * 256, lane);
+        else if (KV)
+          write_row_values(p, pv, U.w, tile, h, rowv + slot * 256, lane);
         mbar_arrive(BAR(S::BFULL + slot));
         issued |= 1u << slot;
         last_par = (last_par & ~(1u << slot)) | (par << slot);
@@ -278,16 +360,26 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
     uint32_t na = 0;
     bool ok = true;
     for (uint32_t u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
-      const BwdUnit U = decode_bwd_unit<KV>(p, u);
+      const BwdUnit U = decode_bwd_unit<MODE>(p, u);
       if (!(ok = wait_warp(BAR(S::AEMPTY), (na & 1u) ^ 1u, abort_flag, limit, kBSiteLoadAEmpty)))
         break;
       const uint32_t dst = sbase + S::a0;
       if (lane == 0) {
         mbar_expect_tx(BAR(S::AFULL), 2 * S::kTile);
-        load_window_tile<NH>(pv, KV ? p.km : p.qm, &p.fill, U.w, U.tile, KV ? U.hk : U.h, p.T,
-                             p.Hg, p.Wg, p.N, dst, BAR(S::AFULL));
-        load_window_tile<NH>(pv, KV ? p.vm : p.gm, &p.fill, U.w, U.tile, KV ? U.hk : U.h, p.T,
-                             p.Hg, p.Wg, p.N, dst + S::kTile, BAR(S::AFULL));
+        if (MODE == kModePooled) {  // pooled key tile: Kp, Vp
+#pragma unroll
+          for (int hf = 0; hf < NH; ++hf) {
+            tma_load_4d(dst + hf * kHalf, &p.kpf, BAR(S::AFULL), hf * 64, U.hk, U.tile * 128,
+                        U.w.b);
+            tma_load_4d(dst + S::kTile + hf * kHalf, &p.vpf, BAR(S::AFULL), hf * 64, U.hk,
+                        U.tile * 128, U.w.b);
+          }
+        } else {
+          load_window_tile<NH>(pv, KV ? p.km : p.qm, &p.fill, U.w, U.tile, KV ? U.hk : U.h, p.T,
+                               p.Hg, p.Wg, p.N, dst, BAR(S::AFULL));
+          load_window_tile<NH>(pv, KV ? p.vm : p.gm, &p.fill, U.w, U.tile, KV ? U.hk : U.h, p.T,
+                               p.Hg, p.Wg, p.N, dst + S::kTile, BAR(S::AFULL));
+        }
       }
       if (!KV) write_row_values(p, pv, U.w, U.tile, U.h, rowv, lane);
       mbar_arrive(BAR(S::AFULL));
@@ -352,6 +444,8 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
     // step: dKV then frees its shared-memory slot, dQ its TMEM copy.
     const int a_free = KV ? S::AEMPTY : S::ATFREE;
     for (uint32_t u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
+      const BwdUnit U = decode_bwd_unit<MODE>(p, u);
+      const int n_steps = bwd_steps<MODE>(p, U);
       if (!(ok = wait_warp(BAR(KV ? S::AFULL : S::ATFULL), na & 1u, abort_flag, limit,
                            kBSiteMmaAFull)))
         break;
@@ -442,11 +536,15 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
     uint64_t nl2 = 0, nd2 = 0;  // dQ: -lse*log2(e) and -D of this thread's query row
     if (!KV && blockIdx.x < p.n_units) ok = copy_a(nl2, nd2);
     for (uint32_t u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
-      const BwdUnit U = decode_bwd_unit<KV>(p, u);
-      // the grid token of this thread's gradient row, found while the unit's
-      // first MMAs run
-      const long long tok =
-          r < pv.rows[U.tile] ? window_row_token(pv, U.w, U.tile, r, p.T, p.Hg, p.Wg) : -1;
+      const BwdUnit U = decode_bwd_unit<MODE>(p, u);
+      const int n_steps = bwd_steps<MODE>(p, U);
+      // the grid token (pooled: the pooled token) of this thread's gradient
+      // row, found while the unit's first MMAs run
+      long long tok;
+      if (MODE == kModePooled)
+        tok = 128LL * U.tile + r < p.P ? 128LL * U.tile + r : -1;
+      else
+        tok = r < pv.rows[U.tile] ? window_row_token(pv, U.w, U.tile, r, p.T, p.Hg, p.Wg) : -1;
       for (int s = 0; s < n_steps; ++s) {
         const float* rv = rowv;
         if (KV) {
@@ -521,12 +619,12 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
       if (!(ok = wait_warp(BAR(S::OFULL), of & 1u, abort_flag, limit, kBSiteEwOFull))) break;
       ++of;
       tc_fence_after();
-      if (KV) {
-        // warpgroup 0 writes dV, warpgroup 1 writes dK (times the scale)
-        const long long roff = tok >= 0 ? (((long long)U.w.b * p.N + tok) * p.Hkv + U.hk) * D : -1;
-        __nv_bfloat16* base = hc == 0 ? p.dv : p.dk;
-        const float mul = hc == 0 ? 1.0f : p.scale;
-        const uint64_t m2 = f2pack(mul, mul);
+      if (MODE == kModePooled) {
+        // warpgroup 0 adds its dV rows into dvp, warpgroup 1 its dK rows into
+        // dkp: fp32 sums over the query-tile splits of the batch (no scale yet)
+        float* dst = tok >= 0 ? (hc == 0 ? p.dvp : p.dkp) +
+                                    (((long long)U.w.b * p.P + tok) * p.Hkv + U.hk) * D
+                              : nullptr;
 #pragma unroll
         for (int hf = 0; hf < NH; ++hf) {
           uint32_t o[2][32];
@@ -534,6 +632,51 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
           tmem_ld32(tmem + tl + 256 + hc * D + hf * 64 + 32, o[1]);
           tmem_wait_ld(o[0]);
           tmem_wait_ld(o[1]);
+          if (dst) {
+#pragma unroll
+            for (int e = 0; e < 16; ++e)
+              atomicAdd(reinterpret_cast<float4*>(dst + hf * 64 + 4 * e),
+                        make_float4(__uint_as_float(o[e / 8][(4 * e) % 32]),
+                                    __uint_as_float(o[e / 8][(4 * e) % 32 + 1]),
+                                    __uint_as_float(o[e / 8][(4 * e) % 32 + 2]),
+                                    __uint_as_float(o[e / 8][(4 * e) % 32 + 3])));
+          }
+        }
+      } else if (KV) {
+        // warpgroup 0 writes dV, warpgroup 1 writes dK (times the scale); with
+        // pooled memory each row first adds its cell's pooled gradient / count
+        const long long roff = tok >= 0 ? (((long long)U.w.b * p.N + tok) * p.Hkv + U.hk) * D : -1;
+        __nv_bfloat16* base = hc == 0 ? p.dv : p.dk;
+        const float mul = hc == 0 ? 1.0f : p.scale;
+        const uint64_t m2 = f2pack(mul, mul);
+        const float* share = nullptr;
+        if (p.P && tok >= 0) {
+          const long long hw = (long long)p.Hg * p.Wg;
+          const long long t = tok / hw, y = (tok / p.Wg) % p.Hg, x = tok % p.Wg;
+          const long long cell =
+              ((t / p.pt) * (p.Hg / p.ph) + y / p.ph) * (p.Wg / p.pw) + x / p.pw;
+          share = (hc == 0 ? p.dvp : p.dkp) + (((long long)U.w.b * p.P + cell) * p.Hkv + U.hk) * D;
+        }
+        const uint64_t ic2 = f2pack(p.inv_count, p.inv_count);
+#pragma unroll
+        for (int hf = 0; hf < NH; ++hf) {
+          uint32_t o[2][32];
+          tmem_ld32(tmem + tl + 256 + hc * D + hf * 64, o[0]);
+          tmem_ld32(tmem + tl + 256 + hc * D + hf * 64 + 32, o[1]);
+          tmem_wait_ld(o[0]);
+          tmem_wait_ld(o[1]);
+          if (share) {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+              const float2 sv = *reinterpret_cast<const float2*>(share + hf * 64 + 2 * e);
+              float o0, o1;
+              f2unpack(f2fma(f2pack(sv.x, sv.y), ic2,
+                             f2pack(__uint_as_float(o[e / 16][(2 * e) % 32]),
+                                    __uint_as_float(o[e / 16][(2 * e) % 32 + 1]))), o0, o1);
+              o[e / 16][(2 * e) % 32] = __float_as_uint(o0);
+              o[e / 16][(2 * e) % 32 + 1] = __float_as_uint(o1);
+            }
+          }
           uint32_t w[32];
 #pragma unroll
           for (int e = 0; e < 32; ++e) {
@@ -578,25 +721,44 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
   }
 }
 
-template <int D, bool KV>
+template <int D, int MODE>
 basa_status launch_bwd_kernel(BwdTcParams* prm, long long units, cudaStream_t stream) {
   static_assert(BwdSmem<D>::alloc <= 232448, "shared memory plan exceeds 227 KB");
   const int smem = BwdSmem<D>::alloc;
   if (units > 0x7fffffffLL) return BASA_ERR_UNSUPPORTED;
-  if (cudaFuncSetAttribute(tc_bwd_kernel<D, KV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  if (cudaFuncSetAttribute(tc_bwd_kernel<D, MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            smem) != cudaSuccess)
     return BASA_ERR_CUDA;
   prm->n_units = (uint32_t)units;
   long long grid = tc_sm_count();
   if (grid > units) grid = units;
-  tc_bwd_kernel<D, KV><<<(unsigned)grid, kBwdTcThreads, smem, stream>>>(*prm);
+  tc_bwd_kernel<D, MODE><<<(unsigned)grid, kBwdTcThreads, smem, stream>>>(*prm);
   return cudaGetLastError() == cudaSuccess ? BASA_OK : BASA_ERR_CUDA;
+}
+
+// The three kernels in order: the pooled tokens' gradients (when P), dQ, then
+// the window dK, dV (which add each row's share of the pooled gradients).
+template <int D>
+basa_status launch_bwd_all(BwdTcParams* prm, const Dims& d, long long per, cudaStream_t stream) {
+  basa_status st;
+  if (d.P) {
+    const size_t bytes = (size_t)d.B * d.P * d.Hkv * d.d * sizeof(float);
+    if (cudaMemsetAsync(prm->dkp, 0, bytes, stream) != cudaSuccess ||
+        cudaMemsetAsync(prm->dvp, 0, bytes, stream) != cudaSuccess)
+      return BASA_ERR_CUDA;
+    const long long pooled_units = (long long)d.B * d.Hkv * prm->n_pt * prm->n_fsplits;
+    if ((st = launch_bwd_kernel<D, kModePooled>(prm, pooled_units, stream)) != BASA_OK) return st;
+  }
+  if ((st = launch_bwd_kernel<D, kModeDq>(prm, (long long)d.B * d.H * per, stream)) != BASA_OK)
+    return st;
+  return launch_bwd_kernel<D, kModeDkv>(prm, (long long)d.B * d.Hkv * per, stream);
 }
 
 basa_status build_and_launch_bwd(BwdTcParams* prm, const Dims& d, const TilePlan& plan,
                                  const void* q, const void* k, const void* v, const void* out,
                                  const void* dout, const float* lse, float* dD, void* dq,
-                                 void* dk, void* dv, uint32_t timeout_ms, cudaStream_t stream) {
+                                 void* dk, void* dv, const PoolGrads* pg, uint32_t timeout_ms,
+                                 cudaStream_t stream) {
   basa_status st;
   const uint64_t D = (uint64_t)d.d, H = (uint64_t)d.H, Hk = (uint64_t)d.Hkv;
   if ((st = pack_plan_image(plan, &prm->plan)) != BASA_OK) return st;
@@ -619,6 +781,32 @@ basa_status build_and_launch_bwd(BwdTcParams* prm, const Dims& d, const TilePlan
     const uint32_t box8[4] = {64, 1, 8, 1};
     if ((st = encode_map(&prm->fill, k, 4, fdims, fstr, box8)) != BASA_OK) return st;
   }
+  if (d.P) {  // pooled K, V tiles; q and dout as flat 128-row tiles for the pooled kernel
+    const uint64_t pdims[4] = {D, Hk, (uint64_t)d.P, (uint64_t)d.B};
+    const uint64_t pstr[3] = {D * 2, Hk * D * 2, (uint64_t)d.P * Hk * D * 2};
+    const uint64_t fqdims[4] = {D, H, (uint64_t)d.N, (uint64_t)d.B};
+    const uint64_t fqstr[3] = {D * 2, H * D * 2, (uint64_t)d.N * H * D * 2};
+    const uint32_t box128[4] = {64, 1, 128, 1};
+    if ((st = encode_map(&prm->kpf, pg->kp, 4, pdims, pstr, box128)) != BASA_OK) return st;
+    if ((st = encode_map(&prm->vpf, pg->vp, 4, pdims, pstr, box128)) != BASA_OK) return st;
+    if ((st = encode_map(&prm->qf, q, 4, fqdims, fqstr, box128)) != BASA_OK) return st;
+    if ((st = encode_map(&prm->gf, dout, 4, fqdims, fqstr, box128)) != BASA_OK) return st;
+    prm->dkp = pg->dkp;
+    prm->dvp = pg->dvp;
+    prm->P = d.P;
+    prm->n_pt = (int)((d.P + 127) / 128);
+    prm->n_fqt = (int)((d.N + 127) / 128);
+    // split the grid's query tiles so that the pooled kernel has about four
+    // units per SM
+    const long long base = (long long)d.B * d.Hkv * prm->n_pt;
+    long long n = (4LL * tc_sm_count() + base - 1) / base;
+    if (n > prm->n_fqt) n = prm->n_fqt;
+    if (n < 1) n = 1;
+    prm->fqt_per_split = (int)((prm->n_fqt + n - 1) / n);
+    prm->n_fsplits = (prm->n_fqt + prm->fqt_per_split - 1) / prm->fqt_per_split;
+    prm->pt = d.pt; prm->ph = d.ph; prm->pw = d.pw;
+    prm->inv_count = 1.0f / (float)(d.pt * d.ph * d.pw);
+  }
   prm->lse = lse;
   prm->dD = dD;
   prm->dq = static_cast<__nv_bfloat16*>(dq);
@@ -637,16 +825,10 @@ basa_status build_and_launch_bwd(BwdTcParams* prm, const Dims& d, const TilePlan
   prm->scale = d.scale;
   prm->scale_log2 = d.scale * kLog2e;
   const long long per = (long long)prm->n_windows * plan.n_tiles;
-  // D = rowsum(dout * out), then dQ, then dK and dV
+  // D = rowsum(dout * out), then the gradient kernels
   if ((st = launch_bwd_prep(d, out, dout, dD, stream)) != BASA_OK) return st;
-  if (d.d == 64) {
-    if ((st = launch_bwd_kernel<64, false>(prm, (long long)d.B * d.H * per, stream)) != BASA_OK)
-      return st;
-    return launch_bwd_kernel<64, true>(prm, (long long)d.B * d.Hkv * per, stream);
-  }
-  if ((st = launch_bwd_kernel<128, false>(prm, (long long)d.B * d.H * per, stream)) != BASA_OK)
-    return st;
-  return launch_bwd_kernel<128, true>(prm, (long long)d.B * d.Hkv * per, stream);
+  return d.d == 64 ? launch_bwd_all<64>(prm, d, per, stream)
+                   : launch_bwd_all<128>(prm, d, per, stream);
 }
 
 }  // namespace
@@ -657,14 +839,13 @@ basa_status launch_bwd_tc(const Dims& d, const void* q, const void* k, const voi
                           cudaStream_t stream) {
   if (d.dtype != BASA_BF16 || (d.d != 64 && d.d != 128) || d.qsep || (d.P && !pg))
     return BASA_ERR_UNSUPPORTED;
-  if (d.P) return BASA_ERR_UNSUPPORTED;  // pooled memory: the CUDA-core kernels
   TilePlan plan;
   basa_status st = build_tile_plan(d, &plan);  // before any launch
   if (st != BASA_OK) return st;
   BwdTcParams* prm = new (std::nothrow) BwdTcParams;
   if (!prm) return BASA_ERR_INVALID_ARG;
   memset(prm, 0, sizeof(*prm));
-  st = build_and_launch_bwd(prm, d, plan, q, k, v, out, dout, lse, dD, dq, dk, dv, timeout_ms,
+  st = build_and_launch_bwd(prm, d, plan, q, k, v, out, dout, lse, dD, dq, dk, dv, pg, timeout_ms,
                             stream);
   delete prm;
   return st;
