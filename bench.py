@@ -521,6 +521,10 @@ def main():
                    "l2": "evicted before every step (256 MiB write, then 256 MiB read; outside the events)",
                    "parallelism": f"replicas x{world}"},
         "latency_ms": ms_max,
+        # this rank's spread over the timed steps (the mean is latency_ms)
+        "latency_pct_ms": {"p10": float(np.percentile(t_steps, 10)),
+                           "p50": float(np.percentile(t_steps, 50)),
+                           "p90": float(np.percentile(t_steps, 90))},
         "pct_bf16_peak": 100.0 * per_gpu_tflops / peaks["bf16_tflops"],
         "speedup": {"full_attn_ms": ms_full, "window_attn_ms": ms_max,
                     "realised": ms_full / ms_max, "theoretical": theo,

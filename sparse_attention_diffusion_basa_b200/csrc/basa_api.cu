@@ -5,9 +5,18 @@
 
 #include <mutex>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "basa_internal.h"
 
 namespace basa {
+
+// An NVTX range over one library call, so that profilers show each call's
+// launches under its name (a pointer check when no tool is attached).
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+};
 
 static int floor_mod(long long a, int n) {
   long long r = a % n;
@@ -206,6 +215,7 @@ size_t basa_workspace_size(const basa_params* p) {
 
 basa_status basa_pool_kv(const void* k, const void* v, void* kp, void* vp, const basa_params* p,
                          cudaStream_t stream) {
+  NvtxRange nvtx("basa_pool_kv");
   Dims d;
   basa_status s = normalise(p, false, &d);
   if (s != BASA_OK) return s;
@@ -235,6 +245,7 @@ static basa_status check_qkvo(const void* q, const void* k, const void* v, const
 
 basa_status basa_window_attn(const void* q, const void* k, const void* v, void* out, float* lse,
                              void* workspace, const basa_params* p, cudaStream_t stream) {
+  NvtxRange nvtx("basa_window_attn");
   Dims d;
   basa_status s = normalise(p, false, &d);
   if (s != BASA_OK) return s;
@@ -262,6 +273,7 @@ basa_status basa_window_attn(const void* q, const void* k, const void* v, void* 
 basa_status basa_window_attn_gm(const void* q, const void* k, const void* v, const void* kp,
                                 const void* vp, void* out, float* lse, const basa_params* p,
                                 cudaStream_t stream) {
+  NvtxRange nvtx("basa_window_attn_gm");
   Dims d;
   basa_status s = normalise(p, false, &d);
   if (s != BASA_OK) return s;
@@ -295,6 +307,7 @@ basa_status basa_joint_attn(const void* q, const void* k, const void* v, const v
                             const void* kt, const void* vt, int64_t L, void* out, void* out_t,
                             float* lse, float* lse_t, void* workspace, const basa_params* p,
                             cudaStream_t stream) {
+  NvtxRange nvtx("basa_joint_attn");
   Dims d;
   basa_status s = normalise(p, false, &d);
   if (s != BASA_OK) return s;
@@ -349,6 +362,7 @@ basa_status basa_window_attn_bwd(const void* q, const void* k, const void* v, co
                                  const void* dout, const float* lse, void* dq, void* dk,
                                  void* dv, void* workspace, const basa_params* p,
                                  cudaStream_t stream) {
+  NvtxRange nvtx("basa_window_attn_bwd");
   Dims d;
   basa_status s = normalise(p, false, &d);
   if (s != BASA_OK) return s;
@@ -379,6 +393,7 @@ basa_status basa_window_attn_bwd(const void* q, const void* k, const void* v, co
 
 basa_status basa_full_attn(const void* q, const void* k, const void* v, void* out, float* lse,
                            const basa_params* p, cudaStream_t stream) {
+  NvtxRange nvtx("basa_full_attn");
   Dims d;
   basa_status s = normalise(p, true, &d);
   if (s != BASA_OK) return s;
