@@ -12,11 +12,14 @@
 //   dK_j  = scale * sum_i dS_ij q_i      (over the query heads sharing k_j)
 //   dV_j  = sum_i P_ij dO_i
 // Every key of a window is attended only by that window's queries, so each
-// (b, K/V head, window) owns its dK, dV rows: no atomics.  Three launches:
-// D = rowsum(dO * O) into the caller's workspace, then dQ (a group of threads
-// per query, keys staged in shared memory), then dK and dV (a group of threads
-// per key, queries staged; D / 32 threads per row).  Arithmetic is fp32; bf16
-// inputs are widened on load and the gradients rounded once on store.
+// (b, K/V head, window) owns its dK, dV rows: no atomics.  Launches: D =
+// rowsum(dO * O) into the caller's workspace (also used by the tensor-core
+// backward); with pooled memory the pooled tokens' gradients, each summed over
+// every query of its batch into fp32 buffers; dQ (a group of threads per query,
+// the window's keys and then the pooled keys staged in shared memory); dK and
+// dV (a group of threads per key, queries staged; d / 32 threads per row), each
+// row adding its cell's pooled gradient divided by the cell size.  Arithmetic
+// is fp32; bf16 inputs are widened on load and the gradients rounded once.
 #include <cuda_bf16.h>
 #include <math.h>
 

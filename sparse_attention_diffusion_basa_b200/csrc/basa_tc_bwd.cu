@@ -10,23 +10,33 @@
 // pass) and D = rowsum(dO * O):
 //   dP = dO V^T,  dS = P * (dP - D),
 //   dQ = scale * dS K,  dK = scale * dS^T Q,  dV = P^T dO.
-// A key is seen only by the queries of its own window, so every gradient row
-// depends on one window alone: two kernels, no atomics.
+// A window key is seen only by the queries of its own window, so its gradient
+// rows depend on one window alone and need no atomics.  Pooled global memory
+// (the review's K/V-pooled tokens, the means of fixed cells) adds keys that
+// every query of the batch sees: their gradients are summed over all queries
+// (fp32 atomics) and reach each cell token divided by the cell size.
 //
-// One kernel template serves both, because they have the same shape:
-//   dQ  (KV = false): unit (b, h, window, query tile).  Fixed per unit: A0 = Q,
-//       A1 = dO of the tile (and lse, D of its rows).  Step j over the key
-//       tiles of the window: B0 = K_j, B1 = V_j.
-//   dKV (KV = true):  unit (b, K/V head, window, key tile).  Fixed per unit:
-//       A0 = K, A1 = V of the tile.  Step over (query head of the group, query
-//       tile): B0 = Q_i, B1 = dO_i (and lse, D of its rows).
+// One kernel template serves three modes of the same shape:
+//   dQ (kModeDq): unit (b, h, window, query tile).  Fixed per unit: A0 = Q,
+//       A1 = dO of the tile (and lse, D of its rows), copied from shared memory
+//       into TMEM columns [384, 512) at unit start so that the slot refills a
+//       whole unit ahead.  Step j over the window's key tiles, then the pooled
+//       key tiles: B0 = K_j, B1 = V_j.
+//   window dK, dV (kModeDkv): unit (b, K/V head, window, key tile).  Fixed per
+//       unit: A0 = K, A1 = V of the tile.  Step over (query head of the group,
+//       query tile): B0 = Q_i, B1 = dO_i (and lse, D of its rows).  With pooled
+//       memory the epilogue adds the row's share of its cell's pooled gradient.
+//   pooled dK, dV (kModePooled): unit (b, K/V head, pooled key tile, split of
+//       the grid's query tiles); A0, A1 = pooled K, V; steps over flat query
+//       tiles; the epilogue adds its sums into fp32 dkp, dvp with atomics.
 // Per step the tensor core computes X = A0 B0^T and Y = A1 B1^T into TMEM
-// (dQ: S and dP; dKV: S^T and dP^T).  The elementwise warps form P and dS in
+// (dQ: S and dP; dK, dV: S^T and dP^T).  The elementwise warps form P and dS in
 // fp32 and write them back into TMEM as bf16 pairs over X (and Y), and the
 // tensor core accumulates, with the bf16 operand read from TMEM,
 //   dQ:  dQ += dS K_j                  (B0 read MN-major)
 //   dKV: dV += P^T dO_i, dK += dS^T Q_i (B1, B0 read MN-major).
-// TMEM columns: X [0, 128), Y [128, 256), accumulators from 256.
+// TMEM columns: X [0, 128), Y [128, 256), accumulators from 256 (dQ: dQ, then
+// Q and dO; dK, dV: dV, then dK).
 //
 // Persistent CTAs (one per SM, 384 threads):
 //   warp 0       TMA loader of the step pairs through a two-slot ring (dKV:
