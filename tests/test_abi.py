@@ -190,3 +190,30 @@ def test_joint_and_grouped_query_validation(lib):
     full = lib.basa_workspace_size(ctypes.byref(prm))
     prm.Hkv = 2
     assert lib.basa_workspace_size(ctypes.byref(prm)) * 2 == full
+
+
+def test_backward_workspace_sizes(lib):
+    """The backward workspace holds D = rowsum(dO * O) (fp32 [B, H, N]); with
+    pooled memory also the pooled K, V (input dtype) and their fp32 gradients
+    ([B, P, Hkv, d] each), every piece rounded up to 256 bytes."""
+    up = lambda x: (x + 255) // 256 * 256
+    B, T, Hg, Wg, H, d = 1, 1, 16, 16, 2, 64
+    N = T * Hg * Wg
+    plain = lib.basa_bwd_workspace_size(ctypes.byref(_p()))
+    assert plain == up(B * H * N * 4)
+    P = (Hg // 4) * (Wg // 4)
+    for dtype, es in ((1, 2), (0, 4)):
+        pooled = lib.basa_bwd_workspace_size(ctypes.byref(_p(pool=(1, 4, 4), dtype=dtype)))
+        assert pooled == up(B * H * N * 4) + 2 * up(B * P * H * d * es) + 2 * up(B * P * H * d * 4)
+    assert lib.basa_bwd_workspace_size(ctypes.byref(_p(pool=(1, 3, 3)))) == 0  # cell does not divide
+
+
+def test_joint_workspace_needs_bf16_and_text(lib):
+    """No split workspace for fp32, for L <= 0, or for invalid params; the bf16
+    size depends on the device's SM count, so only its form is checked here."""
+    assert lib.basa_joint_workspace_size(ctypes.byref(_p(dtype=0)), 512) == 0
+    assert lib.basa_joint_workspace_size(ctypes.byref(_p()), 0) == 0
+    assert lib.basa_joint_workspace_size(ctypes.byref(_p()), -3) == 0
+    assert lib.basa_joint_workspace_size(ctypes.byref(_p(window=(1, 5, 5))), 64) == 0
+    n = lib.basa_joint_workspace_size(ctypes.byref(_p()), 64)
+    assert n % 256 == 0
