@@ -26,6 +26,9 @@ a bounded sample of the same workload (all queries of a few heads).
 
 Multi-GPU (torchrun): each rank runs an independent replica of the workload
 (the path has no exchange step); the time is the max over ranks.
+
+--backward: the same timing for the gradients (dq, dk, dv) of the workload's
+window attention (with its pooled memory, if any) for a random output gradient.
 """
 from __future__ import annotations
 
