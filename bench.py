@@ -339,6 +339,18 @@ def barrier(world):
         torch.distributed.barrier()
 
 
+def arm_config(w, shift, world):
+    """The workload description both arms print in their JSON line."""
+    _, _, N, m, P, _ = workload_numbers(w, shift)
+    L = w.text
+    return {"workload": f"{w.name}: B={w.B} grid {w.T}x{w.Hg}x{w.Wg} H={w.H} d={w.d} "
+                        f"window {'x'.join(map(str, w.window))} shift {shift} "
+                        f"pool {w.pool}" + (f" text {L}" if L else ""),
+            "N": N, "m": m, "P": P, "global_batch": w.B * world,
+            "l2": "evicted before every step (256 MiB write, then 256 MiB read; outside the events)",
+            "parallelism": f"replicas x{world}"}
+
+
 def main_reference(args, world, rank):
     """The CPU oracle as the reference arm (rank 0 only)."""
     if rank != 0:
@@ -363,7 +375,7 @@ def main_reference(args, world, rank):
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": 1e3 * total / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": f"{w.name}: oracle sample", "shift": list(shift)},
+            "config": arm_config(w, shift, world),
             "cpu_baseline": {"value": val, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
                              "sample": f"all {w.N} queries of head 0 of {w.H}, batch 0, per step"},
             "e2e": {"value": val, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
@@ -547,12 +559,7 @@ def main():
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic",
-        "config": {"workload": f"{w.name}: B={w.B} grid {w.T}x{w.Hg}x{w.Wg} H={w.H} d={w.d} "
-                               f"window {'x'.join(map(str, w.window))} shift {shift} "
-                               f"pool {w.pool}" + (f" text {L}" if L else ""),
-                   "N": N, "m": m, "P": P, "global_batch": w.B * world,
-                   "l2": "evicted before every step (256 MiB write, then 256 MiB read; outside the events)",
-                   "parallelism": f"replicas x{world}"},
+        "config": arm_config(w, shift, world),
         "latency_ms": ms_max,
         # this rank's spread over the timed steps (the mean is latency_ms)
         "latency_pct_ms": {"p10": float(np.percentile(t_steps, 10)),
