@@ -83,7 +83,9 @@ typedef enum basa_status {
   BASA_ERR_WORKSPACE = 5,   /* workspace missing when global memory is requested */
   BASA_ERR_CUDA = 6,        /* CUDA runtime or driver error at launch */
   BASA_ERR_TIMEOUT = 7,     /* a bounded wait inside a kernel ran out */
-  BASA_ERR_SCRATCH_LIMIT = 8 /* basa_window_attn_noalloc: pooled K/V exceed its fixed scratch */
+  BASA_ERR_SCRATCH_LIMIT = 8, /* basa_window_attn_noalloc: pooled K/V exceed its fixed scratch */
+  BASA_ERR_CHECK = 9          /* checked build (BASA_CHECKED) only: a kernel found a TMA box or
+                                 an output index outside its tensor and skipped the access */
 } basa_status;
 
 typedef enum basa_dtype { BASA_F32 = 0, BASA_BF16 = 1 } basa_dtype;

@@ -5,13 +5,16 @@ import ctypes
 import os
 
 HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(HERE, "_lib", "libbasa.so")
+# BASA_LIBRARY=checked selects the build whose kernels check every box and
+# output index (python -m sparse_attention_diffusion_basa_b200.build --checked).
+LIB_PATH = os.path.join(HERE, "_lib", "libbasa_checked.so" if os.environ.get("BASA_LIBRARY") == "checked"
+                        else "libbasa.so")
 
 BASA_OK = 0
 STATUS_NAMES = {
     0: "BASA_OK", 1: "BASA_ERR_INVALID_ARG", 2: "BASA_ERR_SHAPE", 3: "BASA_ERR_UNSUPPORTED",
     4: "BASA_ERR_ALIGN", 5: "BASA_ERR_WORKSPACE", 6: "BASA_ERR_CUDA", 7: "BASA_ERR_TIMEOUT",
-    8: "BASA_ERR_SCRATCH_LIMIT",
+    8: "BASA_ERR_SCRATCH_LIMIT", 9: "BASA_ERR_CHECK",
 }
 BASA_F32, BASA_BF16 = 0, 1
 BASA_FLAG_TEST_WITHHOLD_LOADS = 0x1

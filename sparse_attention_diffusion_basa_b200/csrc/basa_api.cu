@@ -201,6 +201,7 @@ const char* basa_status_string(basa_status s) {
     case BASA_ERR_CUDA: return "CUDA error";
     case BASA_ERR_TIMEOUT: return "device wait timed out";
     case BASA_ERR_SCRATCH_LIMIT: return "pooled K/V exceed the fixed no-alloc scratch";
+    case BASA_ERR_CHECK: return "a checked kernel found an access outside its tensor";
   }
   return "unknown status";
 }

@@ -233,6 +233,14 @@ __device__ __forceinline__ void store_half(const TcParams& p, const PlanView& pv
     const int gt = wrap(U.ot + box_lt(e), p.T);
     const int gh = wrap(U.oh + box_lh(e), p.Hg);
     const int gw = wrap(U.ow + box_lw(e), p.Wg);
+    if constexpr (kChecked) {
+      const int bt = pv.bt[sid], bh = pv.bh[sid], bw = pv.bw[sid];
+      if (sid >= kMaxShapes || gt + bt > p.T || gh + bh > p.Hg || gw + bw > p.Wg ||
+          box_row8(e) * 8 + bt * bh * bw > 128) {
+        check_failed(kCheckStoreBox);
+        continue;
+      }
+    }
     tma_store_5d(&p.om[sid], src + box_row8(e) * 1024, hf * 64, U.h, gw, gh, U.b * p.T + gt);
   }
 }
@@ -666,9 +674,13 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attn_kernel(const __grid_const
             const int rr = k * 4 + lane / 8, c = lane % 8;
             const uint4 val = ld_shared_v4(wst + rr * 128 + ((c ^ (rr & 7)) << 4));
             const long long t = __shfl_sync(0xffffffffu, tok, rr);
-            if (t >= 0)
-              *reinterpret_cast<uint4*>(p.out + (((long long)U.b * p.Nq + t) * p.H + U.h) * D +
-                                        hf * 64 + c * 8) = val;
+            if (t >= 0) {
+              if (kChecked && t >= p.Nq)
+                check_failed(kCheckOutRow);
+              else
+                *reinterpret_cast<uint4*>(p.out + (((long long)U.b * p.Nq + t) * p.H + U.h) * D +
+                                          hf * 64 + c * 8) = val;
+            }
           }
           __syncwarp();
         }
@@ -714,7 +726,9 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attn_kernel(const __grid_const
       tc_fence_before();  // the reads of O_i precede the next unit's first P.V MMA
       if (p.lse && r < query_valid(p, pv, qt)) {
         const long long n = row_token(p, pv, U, qt, r);
-        if (n >= 0)
+        if (kChecked && n >= p.Nq)
+          check_failed(kCheckLseRow);
+        else if (n >= 0)
           p.lse[((long long)U.b * p.H + U.h) * p.Nq + n] = (m + __log2f(l)) * 0.69314718055994531f;
       }
     }
@@ -995,8 +1009,9 @@ basa_status read_and_clear_status(cudaStream_t stream) {
   if (take_bwd_status(stream, &vb, &whereb) != cudaSuccess) return BASA_ERR_CUDA;
   if (v | vb) {
     if (getenv("BASA_DEBUG"))
-      fprintf(stderr, "basa: device wait gave up at site %u (backward: %u)\n", where, whereb);
-    return BASA_ERR_TIMEOUT;
+      fprintf(stderr, "basa: device status %u at site %u (backward: %u at %u)\n", v, where, vb,
+              whereb);
+    return ((v | vb) & 2u) ? BASA_ERR_CHECK : BASA_ERR_TIMEOUT;
   }
   return cudaGetLastError() == cudaSuccess ? BASA_OK : BASA_ERR_CUDA;
 }

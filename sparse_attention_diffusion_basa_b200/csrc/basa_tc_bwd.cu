@@ -96,6 +96,7 @@ struct __align__(64) BwdTcParams {
   int fqt_per_split, n_fsplits;  // the pooled kernel's split of those query tiles
   int pt, ph, pw;
   float inv_count;               // 1 / (pt * ph * pw)
+  long long q_elems, kv_elems;   // elements of dq and of dk, dv (checked build)
 };
 
 // Kernel modes: the dQ kernel (window key tiles, then the pooled tiles), the
@@ -236,7 +237,7 @@ __device__ __forceinline__ void write_row_values_flat(const BwdTcParams& p, int 
 // instruction writes 64 contiguous bytes of eight rows.
 __device__ __forceinline__ void warp_store_row64(uint32_t stg, const uint32_t (&w)[32],
                                                  long long roff, __nv_bfloat16* base, int col0,
-                                                 int lane) {
+                                                 int lane, long long limit) {
 #pragma unroll
   for (int ps = 0; ps < 2; ++ps) {
 #pragma unroll
@@ -249,7 +250,12 @@ __device__ __forceinline__ void warp_store_row64(uint32_t stg, const uint32_t (&
       const int rr = k * 8 + lane / 4, c = lane % 4;
       const uint4 val = ld_shared_v4(stg + rr * 64 + ((c ^ ((rr >> 1) & 3)) << 4));
       const long long t = __shfl_sync(0xffffffffu, roff, rr);
-      if (t >= 0) *reinterpret_cast<uint4*>(base + t + col0 + ps * 32 + c * 8) = val;
+      if (t >= 0) {
+        if (kChecked && t + col0 + ps * 32 + c * 8 + 8 > limit)
+          check_failed(kCheckGradRow);
+        else
+          *reinterpret_cast<uint4*>(base + t + col0 + ps * 32 + c * 8) = val;
+      }
     }
     __syncwarp();
   }
@@ -665,7 +671,10 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
           const long long t = tok / hw, y = (tok / p.Wg) % p.Hg, x = tok % p.Wg;
           const long long cell =
               ((t / p.pt) * (p.Hg / p.ph) + y / p.ph) * (p.Wg / p.pw) + x / p.pw;
-          share = (hc == 0 ? p.dvp : p.dkp) + (((long long)U.w.b * p.P + cell) * p.Hkv + U.hk) * D;
+          if (kChecked && cell >= p.P)
+            check_failed(kCheckPooledRow);
+          else
+            share = (hc == 0 ? p.dvp : p.dkp) + (((long long)U.w.b * p.P + cell) * p.Hkv + U.hk) * D;
         }
         const uint64_t ic2 = f2pack(p.inv_count, p.inv_count);
 #pragma unroll
@@ -695,7 +704,7 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
                                   __uint_as_float(o[e / 16][(2 * e) % 32 + 1])), m2), o0, o1);
             w[e] = pack_bf16(o0, o1);
           }
-          warp_store_row64(stg, w, roff, base, hf * 64, lane);
+          warp_store_row64(stg, w, roff, base, hf * 64, lane, p.kv_elems);
         }
       } else if (hc < NH) {
         // warpgroup hc writes columns [64 hc, 64 hc + 64) of dQ (times the scale)
@@ -714,7 +723,7 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
                                 __uint_as_float(o[e / 16][(2 * e) % 32 + 1])), m2), o0, o1);
           w[e] = pack_bf16(o0, o1);
         }
-        warp_store_row64(stg, w, roff, p.dq, hc * 64, lane);
+        warp_store_row64(stg, w, roff, p.dq, hc * 64, lane, p.q_elems);
       }
       tc_fence_before();  // the reads of the accumulators precede the next unit's MMAs
       nl2 = nl2n;
@@ -819,6 +828,8 @@ basa_status build_and_launch_bwd(BwdTcParams* prm, const Dims& d, const TilePlan
   }
   prm->lse = lse;
   prm->dD = dD;
+  prm->q_elems = (long long)d.B * d.N * d.H * d.d;
+  prm->kv_elems = (long long)d.B * d.N * d.Hkv * d.d;
   prm->dq = static_cast<__nv_bfloat16*>(dq);
   prm->dk = static_cast<__nv_bfloat16*>(dk);
   prm->dv = static_cast<__nv_bfloat16*>(dv);

@@ -21,6 +21,24 @@ __device__ unsigned int g_basa_where;   // site of the first wait that gave up
 
 constexpr int kHalf = 128 * 128;  // bytes of one 64-wide head-dim half of a 128-row tile
 
+// Checked build (compiled with BASA_CHECKED): the kernels verify every TMA box
+// and every output index against their tensors before the access; a failed
+// check skips the access, sets bit 1 of the device status word and records its
+// site (codes from 200).  A skipped load leaves its barrier short, so the
+// consumer's bounded wait then ends the kernel cleanly as well.
+#ifdef BASA_CHECKED
+constexpr bool kChecked = true;
+#else
+constexpr bool kChecked = false;
+#endif
+enum CheckSite : uint32_t {
+  kCheckLoadBox = 200, kCheckStoreBox, kCheckOutRow, kCheckLseRow, kCheckGradRow, kCheckPooledRow
+};
+__device__ __noinline__ void check_failed(uint32_t site) {
+  atomicCAS(&g_basa_where, 0u, site);
+  atomicOr(&g_basa_status, 2u);
+}
+
 // ---------------------------------------------------------------------------
 // PTX wrappers
 // ---------------------------------------------------------------------------
@@ -454,6 +472,14 @@ __device__ __forceinline__ void load_window_tile(const PlanView& pv, const CUten
     const int gt = wrap(w.ot + box_lt(e), T);
     const int gh = wrap(w.oh + box_lh(e), Hg);
     const int gw = wrap(w.ow + box_lw(e), Wg);
+    if constexpr (kChecked) {  // the box lies inside the grid and inside the 128-row tile
+      const int bt = pv.bt[sid], bh = pv.bh[sid], bw = pv.bw[sid];
+      if (sid >= kMaxShapes || gt < 0 || gh < 0 || gw < 0 || gt + bt > T || gh + bh > Hg ||
+          gw + bw > Wg || box_row8(e) * 8 + bt * bh * bw > 128) {
+        check_failed(kCheckLoadBox);
+        continue;
+      }
+    }
     const uint32_t d0 = dst + box_row8(e) * 1024;
 #pragma unroll
     for (int hf = 0; hf < NH; ++hf)
