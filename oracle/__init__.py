@@ -6,9 +6,9 @@ import this package.  It shares no code with the CUDA library: the C oracle in
 ctypes, and ``brute.py`` is an independent dense-mask restatement for tiny grids.
 """
 from .oracle import (OracleParams, build_oracle, window_attn, full_attn, pool_kv,
-                     joint_attn, window_attn_bwd, max_threads, as_f64)
+                     joint_attn, joint_attn_bwd, window_attn_bwd, max_threads, as_f64)
 from .brute import brute_window_attn, brute_joint_attn, window_ids
 
 __all__ = ["OracleParams", "build_oracle", "window_attn", "full_attn", "pool_kv",
-           "joint_attn", "window_attn_bwd", "max_threads", "as_f64", "brute_window_attn", "brute_joint_attn",
+           "joint_attn", "joint_attn_bwd", "window_attn_bwd", "max_threads", "as_f64", "brute_window_attn", "brute_joint_attn",
            "window_ids"]

@@ -444,3 +444,118 @@ int oracle_window_attn_bwd(const double* q, const double* k, const double* v,
   free(dS);
   return 0;
 }
+
+/*
+ * Gradients of joint text + image attention for the output gradients dout
+ * (image queries) and dout_t (text queries).  The keys of image query i are
+ * the members of its shifted window and the L text tokens; the keys of text
+ * query t are the N image tokens and the L text tokens; one softmax per query.
+ * Per query row the chain rule of oracle_window_attn_bwd: P over the row's
+ * keys, dP_j = dO . V_j, D = sum_j P_j dP_j, dS_j = P_j (dP_j - D); dQ = scale
+ * sum_j dS_j K_j; every key's dK (scale dS Q) and dV (P dO) sum over all the
+ * queries that see it.  Image tensors [B, T, Hg, Wg, H or Hkv, d], text tensors
+ * [B, L, H or Hkv, d].
+ */
+static void joint_row_bwd(const double* qa, const double* ga, const double** kp,
+                          const double** vp, double** dkp, double** dvp, int64_t nk, int64_t d,
+                          double scale, double* z, double* dp, double* dqa) {
+  double mx = -INFINITY;
+  for (int64_t j = 0; j < nk; ++j) {
+    double s = 0.0;
+    for (int64_t c = 0; c < d; ++c) s += qa[c] * kp[j][c];
+    z[j] = scale * s;
+    if (z[j] > mx) mx = z[j];
+  }
+  double den = 0.0;
+  for (int64_t j = 0; j < nk; ++j) {
+    z[j] = exp(z[j] - mx);
+    den += z[j];
+  }
+  double D = 0.0;
+  for (int64_t j = 0; j < nk; ++j) {
+    z[j] /= den;
+    double g = 0.0;
+    for (int64_t c = 0; c < d; ++c) g += ga[c] * vp[j][c];
+    dp[j] = g;
+    D += z[j] * g;
+  }
+  for (int64_t j = 0; j < nk; ++j) {
+    const double ds = z[j] * (dp[j] - D);
+    for (int64_t c = 0; c < d; ++c) {
+      dqa[c] += scale * ds * kp[j][c];
+      dkp[j][c] += scale * ds * qa[c];
+      dvp[j][c] += z[j] * ga[c];
+    }
+  }
+}
+
+int oracle_joint_attn_bwd(const double* q, const double* k, const double* v, const double* qt,
+                          const double* kt, const double* vt, int64_t L, const double* dout,
+                          const double* dout_t, double* dq, double* dk, double* dv, double* dqt,
+                          double* dkt, double* dvt, const oracle_params* p) {
+  if (L < 0) return -1;
+  if (p->T % p->wt || p->Hg % p->wh || p->Wg % p->ww) return -1;
+  const int64_t d = p->d, N = p->T * p->Hg * p->Wg, m = p->wt * p->wh * p->ww;
+  const int64_t nwt = p->T / p->wt, nwh = p->Hg / p->wh, nww = p->Wg / p->ww;
+  const int64_t H = p->H, Hk = kv_heads(p);
+  memset(dq, 0, sizeof(double) * (size_t)(p->B * N * H * d));
+  memset(dk, 0, sizeof(double) * (size_t)(p->B * N * Hk * d));
+  memset(dv, 0, sizeof(double) * (size_t)(p->B * N * Hk * d));
+  if (L) {
+    memset(dqt, 0, sizeof(double) * (size_t)(p->B * L * H * d));
+    memset(dkt, 0, sizeof(double) * (size_t)(p->B * L * Hk * d));
+    memset(dvt, 0, sizeof(double) * (size_t)(p->B * L * Hk * d));
+  }
+  const int64_t nmax = N + L;
+  const double** kp = (const double**)malloc(sizeof(double*) * (size_t)nmax);
+  const double** vp = (const double**)malloc(sizeof(double*) * (size_t)nmax);
+  double** dkp = (double**)malloc(sizeof(double*) * (size_t)nmax);
+  double** dvp = (double**)malloc(sizeof(double*) * (size_t)nmax);
+  double* z = (double*)malloc(sizeof(double) * (size_t)nmax);
+  double* dpv = (double*)malloc(sizeof(double) * (size_t)nmax);
+  int64_t* tok = (int64_t*)malloc(sizeof(int64_t) * (size_t)m * 3);
+  for (int64_t b = 0; b < p->B; ++b)
+    for (int64_t h = 0; h < H; ++h) {
+      const int64_t hk = kv_head(p, h);
+      for (int64_t l = 0; l < L; ++l) {  /* the text keys, seen by every query */
+        const int64_t o = ((b * L + l) * Hk + hk) * d;
+        kp[N + l] = kt + o; vp[N + l] = vt + o; dkp[N + l] = dkt + o; dvp[N + l] = dvt + o;
+      }
+      /* image queries: their window, then the text keys */
+      for (int64_t wi = 0; wi < nwt * nwh * nww; ++wi) {
+        const int64_t it = wi / (nwh * nww), iy = (wi / nww) % nwh, ix = wi % nww;
+        int64_t j = 0;
+        for (int64_t lt = 0; lt < p->wt; ++lt)
+          for (int64_t ly = 0; ly < p->wh; ++ly)
+            for (int64_t lx = 0; lx < p->ww; ++lx) {
+              tok[3 * j] = floor_mod(it * p->wt + p->st + lt, p->T);
+              tok[3 * j + 1] = floor_mod(iy * p->wh + p->sh + ly, p->Hg);
+              tok[3 * j + 2] = floor_mod(ix * p->ww + p->sw + lx, p->Wg);
+              ++j;
+            }
+        /* window members in key slots N - m .. N - 1, so the text keys follow */
+        for (int64_t c2 = 0; c2 < m; ++c2) {
+          const int64_t o = kv_index(p, b, tok[3 * c2], tok[3 * c2 + 1], tok[3 * c2 + 2], hk);
+          kp[N - m + c2] = k + o; vp[N - m + c2] = v + o; dkp[N - m + c2] = dk + o;
+          dvp[N - m + c2] = dv + o;
+        }
+        for (int64_t a = 0; a < m; ++a) {
+          const int64_t qo = tok_index(p, b, tok[3 * a], tok[3 * a + 1], tok[3 * a + 2], h);
+          joint_row_bwd(q + qo, dout + qo, kp + (N - m), vp + (N - m), dkp + (N - m),
+                        dvp + (N - m), m + L, d, p->scale, z, dpv, dq + qo);
+        }
+      }
+      /* text queries: every image token, then the text keys */
+      for (int64_t j = 0; j < N; ++j) {
+        const int64_t o = ((b * N + j) * Hk + hk) * d;
+        kp[j] = k + o; vp[j] = v + o; dkp[j] = dk + o; dvp[j] = dv + o;
+      }
+      for (int64_t t = 0; t < L; ++t) {
+        const int64_t qo = ((b * L + t) * H + h) * d;
+        joint_row_bwd(qt + qo, dout_t + qo, kp, vp, dkp, dvp, N + L, d, p->scale, z, dpv,
+                      dqt + qo);
+      }
+    }
+  free(kp); free(vp); free(dkp); free(dvp); free(z); free(dpv); free(tok);
+  return 0;
+}

@@ -85,6 +85,9 @@ def _bind(path):
                                            ctypes.POINTER(_CParams), ctypes.c_int]
     lib.oracle_joint_text_attn.restype = ctypes.c_int
     lib.oracle_window_attn_bwd.argtypes = [dp, dp, dp, dp, dp, dp, dp, ctypes.POINTER(_CParams)]
+    lib.oracle_joint_attn_bwd.argtypes = [dp, dp, dp, dp, dp, dp, ctypes.c_int64, dp, dp,
+                                          dp, dp, dp, dp, dp, dp, ctypes.POINTER(_CParams)]
+    lib.oracle_joint_attn_bwd.restype = ctypes.c_int
     lib.oracle_window_attn_bwd.restype = ctypes.c_int
     lib.oracle_max_threads.argtypes = []
     lib.oracle_max_threads.restype = ctypes.c_int
@@ -239,6 +242,25 @@ def joint_attn(q, k, v, qt, kt, vt, prm: OracleParams, want_lse=False,
     if rc != 0:
         raise ValueError("oracle: bad text length")
     return (out, out_t, lse, lse_t) if want_lse else (out, out_t)
+
+
+def joint_attn_bwd(q, k, v, qt, kt, vt, dout, dout_t, prm: OracleParams):
+    """Gradients (dq, dk, dv, dqt, dkt, dvt) of joint text + image attention for
+    the output gradients ``dout`` (image queries) and ``dout_t`` (text queries);
+    the forward is recomputed from the inputs."""
+    if tuple(prm.pool) != (0, 0, 0):
+        raise ValueError("joint attention takes no pooled memory")
+    q, k, v, qt, kt, vt, dout, dout_t = (np.ascontiguousarray(x, dtype=np.float64)
+                                         for x in (q, k, v, qt, kt, vt, dout, dout_t))
+    L = qt.shape[1]
+    grads = [np.empty(x.shape) for x in (q, k, v, qt, kt, vt)]
+    c = prm.c()
+    rc = _load().oracle_joint_attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(qt), _ptr(kt), _ptr(vt),
+                                       ctypes.c_int64(L), _ptr(dout), _ptr(dout_t),
+                                       *(_ptr(g) for g in grads), ctypes.byref(c))
+    if rc != 0:
+        raise ValueError("oracle: window size does not divide the grid")
+    return tuple(grads)
 
 
 def window_attn_bwd(q, k, v, dout, prm: OracleParams):

@@ -553,6 +553,40 @@ def test_pooled_backward_matches_central_differences(oracle_mod):
             assert abs((up - dn) / (2 * h) - grad[idx]) < 1e-7
 
 
+@pytest.mark.parametrize("shape,window,shift,L,Hkv", [
+    ((1, 1, 4, 6, 2, 8), (1, 2, 3), (0, 1, 2), 3, 0),
+    ((2, 2, 4, 4, 2, 4), (2, 2, 2), (1, 1, 1), 5, 0),
+    ((1, 1, 4, 4, 4, 8), (1, 2, 2), (0, 1, 1), 2, 2),
+    ((1, 1, 4, 4, 2, 4), (1, 2, 2), (0, 1, 1), 0, 0),
+])
+def test_joint_backward_matches_autograd(oracle_mod, shape, window, shift, L, Hkv):
+    """Joint text + image gradients == torch autograd (fp64) through SDPA over the
+    concatenated sequence [image, text] with the joint mask (image-image pairs
+    windowed, every pair with a text token allowed)."""
+    r = _rng(95)
+    B, T, Hg, Wg, H, d = shape
+    hk = Hkv or H
+    N = T * Hg * Wg
+    q, g = r.standard_normal(shape), r.standard_normal(shape)
+    k, v = (r.standard_normal((B, T, Hg, Wg, hk, d)) for _ in range(2))
+    qt, gt = r.standard_normal((B, L, H, d)), r.standard_normal((B, L, H, d))
+    kt, vt = (r.standard_normal((B, L, hk, d)) for _ in range(2))
+    prm = _P(shape, window, shift)
+    prm.Hkv = Hkv
+    got = oracle_mod.joint_attn_bwd(q, k, v, qt, kt, vt, g, gt, prm)
+    ts = [torch.from_numpy(x).requires_grad_() for x in (q, k, v, qt, kt, vt)]
+    cat = lambda a, b, h: torch.cat([a.reshape(B, N, h, d), b], 1).transpose(1, 2)
+    rep = lambda x: x.repeat_interleave(H // hk, dim=1)
+    mask = torch.ones(N + L, N + L, dtype=torch.bool)
+    mask[:N, :N] = torch.from_numpy(_dense_mask(T, Hg, Wg, window, shift))
+    o = torch.nn.functional.scaled_dot_product_attention(
+        cat(ts[0], ts[3], H), rep(cat(ts[1], ts[4], hk)), rep(cat(ts[2], ts[5], hk)),
+        attn_mask=mask)
+    o.backward(cat(torch.from_numpy(g), torch.from_numpy(gt), H))
+    for gg, t in zip(got, ts):
+        np.testing.assert_allclose(gg, t.grad.numpy(), rtol=0, atol=1e-12)
+
+
 def test_backward_matches_central_differences(oracle_mod):
     """d/dx of sum(dO * out) by central differences, at a few coordinates of q, k, v."""
     r = _rng(92)

@@ -38,6 +38,9 @@ MUTANTS = {
         "dS[a * nk + c2] = P[a * nk + c2] * dS[a * nk + c2];"),
     "pooled key gradient not divided by the cell size": (
         "dk[o + c] += inv * dkp[po + c];", "dk[o + c] += dkp[po + c];"),
+    "joint backward: text query rows without the softmax scale": (
+        "joint_row_bwd(qt + qo, dout_t + qo, kp, vp, dkp, dvp, N + L, d, p->scale, z, dpv,",
+        "joint_row_bwd(qt + qo, dout_t + qo, kp, vp, dkp, dvp, N + L, d, 1.0, z, dpv,"),
     "K/V head by modulo instead of by group": (
         "static int64_t kv_head(const oracle_params* p, int64_t h) { return h / (p->H / kv_heads(p)); }",
         "static int64_t kv_head(const oracle_params* p, int64_t h) { return h % kv_heads(p); }"),
@@ -64,6 +67,8 @@ def _pins():
         "Hkv": 2}
     yield pins.test_backward_matches_autograd_of_masked_attention, {
         "shape": (1, 1, 4, 6, 2, 8), "window": (1, 2, 3), "shift": (0, 1, 2), "Hkv": 0}
+    yield pins.test_joint_backward_matches_autograd, {
+        "shape": (1, 1, 4, 6, 2, 8), "window": (1, 2, 3), "shift": (0, 1, 2), "L": 3, "Hkv": 0}
     yield pins.test_pooled_backward_matches_autograd, {
         "shape": (1, 1, 4, 6, 2, 8), "window": (1, 2, 3), "shift": (0, 1, 2), "pool": (1, 2, 3),
         "Hkv": 0}
