@@ -221,6 +221,28 @@ BASA_API size_t basa_joint_workspace_size(const basa_params* p, int64_t L);
  * `stream` only; nothing is allocated.
  */
 BASA_API size_t basa_bwd_workspace_size(const basa_params* p);
+
+/*
+ * Backward of joint text + image attention (basa_joint_attn): the gradients of
+ * both outputs for the output gradients dout (image) and dout_t (text).  Image
+ * query i's keys are its shifted window and the L text tokens, text query t's
+ * keys are every image and text token; per query row dS = P (dP - D) with
+ * D = dout . out, and every key's dk, dv sum over all the queries that see it
+ * (the text keys over every image and text query).  Image tensors
+ * [B, T, Hg, Wg, H or Hkv, d], text tensors [B, L, H or Hkv, d]; lse, lse_t from
+ * the forward call; workspace: basa_joint_bwd_workspace_size(p, L) bytes,
+ * 16-byte aligned.  fp32 arithmetic on CUDA cores for both dtypes, gradients
+ * rounded once.  L = 0 is basa_window_attn_bwd.  A pool cell in p gives
+ * BASA_ERR_UNSUPPORTED.  Launches on `stream` only; nothing is allocated.
+ */
+BASA_API size_t basa_joint_bwd_workspace_size(const basa_params* p, int64_t L);
+BASA_API basa_status basa_joint_attn_bwd(const void* q, const void* k, const void* v,
+                                         const void* qt, const void* kt, const void* vt,
+                                         int64_t L, const void* out, const void* out_t,
+                                         const void* dout, const void* dout_t, const float* lse,
+                                         const float* lse_t, void* dq, void* dk, void* dv,
+                                         void* dqt, void* dkt, void* dvt, void* workspace,
+                                         const basa_params* p, cudaStream_t stream);
 BASA_API basa_status basa_window_attn_bwd(const void* q, const void* k, const void* v,
                                           const void* out, const void* dout, const float* lse,
                                           void* dq, void* dk, void* dv, void* workspace,

@@ -20,6 +20,7 @@ from . import _lib
 from ._lib import BasaError, BasaParams, BASA_F32, BASA_BF16  # noqa: F401
 
 __all__ = ["window_attn", "window_attn_gm", "full_attn", "joint_attn", "window_attn_bwd",
+           "joint_attn_bwd",
            "pool_kv", "workspace_size", "bwd_workspace_size", "joint_workspace_size", "get_status", "window_tiles", "make_params", "BasaError",
            "library_path"]
 
@@ -245,6 +246,37 @@ def window_attn_bwd(q, k, v, out, dout, lse, window, shift=(0, 0, 0), pool=(0, 0
                                             _ptr(workspace), ctypes.byref(prm),
                                             _stream(q, stream)), "basa_window_attn_bwd")
     return dq, dk, dv
+
+
+def joint_attn_bwd(q, k, v, qt, kt, vt, out, out_t, dout, dout_t, lse, lse_t, window,
+                   shift=(0, 0, 0), scale=None, workspace=None, flags=0, stream=None):
+    """Gradients (dq, dk, dv, dqt, dkt, dvt) of joint_attn for the output gradients
+    ``dout`` (image) and ``dout_t`` (text); ``out``, ``out_t``, ``lse``, ``lse_t``
+    are the forward call's outputs."""
+    _check_inputs(q, k, v, out, dout)
+    hkv = _kv_heads(q, k, v)
+    for t in (qt, kt, vt, out_t, dout_t):
+        if not isinstance(t, torch.Tensor) or t.dtype != q.dtype or t.device != q.device:
+            raise ValueError("text tensors must be torch tensors with q's dtype and device")
+        if not t.is_contiguous():
+            raise ValueError("text tensors must be contiguous [B, L, H, d]")
+    for l_ in (lse, lse_t):
+        if l_ is None or l_.dtype != torch.float32 or not l_.is_contiguous():
+            raise ValueError("lse and lse_t must be the forward's contiguous fp32 log-sum-exp")
+    L = qt.shape[1]
+    prm = make_params(q.shape, q.dtype, window, shift, (0, 0, 0), scale, flags, hkv=hkv)
+    lib = _lib.load()
+    need = int(lib.basa_joint_bwd_workspace_size(ctypes.byref(prm), int(L)))
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+    grads = [torch.empty_like(x) for x in (q, k, v, qt, kt, vt)]
+    with torch.cuda.device(q.device):
+        _lib.check(lib.basa_joint_attn_bwd(
+            _ptr(q), _ptr(k), _ptr(v), _ptr(qt), _ptr(kt), _ptr(vt), int(L), _ptr(out),
+            _ptr(out_t), _ptr(dout), _ptr(dout_t), _ptr(lse), _ptr(lse_t),
+            *(_ptr(g_) for g_ in grads), _ptr(workspace), ctypes.byref(prm),
+            _stream(q, stream)), "basa_joint_attn_bwd")
+    return tuple(grads)
 
 
 def get_status(stream=None) -> int:

@@ -24,7 +24,7 @@ EXPORTS = ("basa_status_string", "basa_version", "basa_workspace_size", "basa_po
            "basa_window_attn", "basa_window_attn_gm", "basa_full_attn", "basa_get_status",
            "basa_window_tiles", "basa_window_attn_noalloc", "basa_test_exp2",
            "basa_joint_attn", "basa_window_attn_bwd", "basa_bwd_workspace_size",
-           "basa_joint_workspace_size")
+           "basa_joint_workspace_size", "basa_joint_attn_bwd", "basa_joint_bwd_workspace_size")
 
 
 class BasaParams(ctypes.Structure):
@@ -79,6 +79,10 @@ def load():
     lib.basa_bwd_workspace_size.restype = ctypes.c_size_t
     lib.basa_joint_workspace_size.argtypes = [P, ctypes.c_int64]
     lib.basa_joint_workspace_size.restype = ctypes.c_size_t
+    lib.basa_joint_bwd_workspace_size.argtypes = [P, ctypes.c_int64]
+    lib.basa_joint_bwd_workspace_size.restype = ctypes.c_size_t
+    lib.basa_joint_attn_bwd.argtypes = [vp, vp, vp, vp, vp, vp, ctypes.c_int64] + [vp] * 13 + [P, vp]
+    lib.basa_joint_attn_bwd.restype = ctypes.c_int
     lib.basa_get_status.argtypes = [vp]
     lib.basa_get_status.restype = ctypes.c_int
     lib.basa_window_tiles.argtypes = [P, ctypes.POINTER(ctypes.c_int32),

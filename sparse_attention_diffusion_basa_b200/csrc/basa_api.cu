@@ -392,6 +392,43 @@ basa_status basa_window_attn_bwd(const void* q, const void* k, const void* v, co
   return launch_bwd(d, q, k, v, out, dout, lse, dD, dq, dk, dv, pgp, stream);
 }
 
+size_t basa_joint_bwd_workspace_size(const basa_params* p, int64_t L) {
+  Dims d;
+  if (L < 0 || L > (1LL << 24) || normalise(p, false, &d) != BASA_OK) return 0;
+  return align256((size_t)d.B * d.H * d.N * sizeof(float)) +
+         align256((size_t)d.B * d.H * (size_t)L * sizeof(float));
+}
+
+basa_status basa_joint_attn_bwd(const void* q, const void* k, const void* v, const void* qt,
+                                const void* kt, const void* vt, int64_t L, const void* out,
+                                const void* out_t, const void* dout, const void* dout_t,
+                                const float* lse, const float* lse_t, void* dq, void* dk, void* dv,
+                                void* dqt, void* dkt, void* dvt, void* workspace,
+                                const basa_params* p, cudaStream_t stream) {
+  NvtxRange nvtx("basa_joint_attn_bwd");
+  Dims d;
+  basa_status s = normalise(p, false, &d);
+  if (s != BASA_OK) return s;
+  if (d.pt || d.ph || d.pw) return BASA_ERR_UNSUPPORTED;  // text takes the global-memory slot
+  if (L < 0) return BASA_ERR_INVALID_ARG;
+  if (L > (1LL << 24)) return BASA_ERR_UNSUPPORTED;
+  if ((long long)d.B * d.H * d.N == 0) return BASA_OK;
+  if (L == 0)
+    return basa_window_attn_bwd(q, k, v, out, dout, lse, dq, dk, dv, workspace, p, stream);
+  if ((s = check_qkvo(q, k, v, out, lse)) != BASA_OK) return s;
+  if ((s = check_qkvo(dout, dq, dk, dv, nullptr)) != BASA_OK) return s;
+  if ((s = check_qkvo(qt, kt, vt, out_t, lse_t)) != BASA_OK) return s;
+  if ((s = check_qkvo(dout_t, dqt, dkt, dvt, nullptr)) != BASA_OK) return s;
+  if (!lse || !lse_t) return BASA_ERR_INVALID_ARG;
+  if (!workspace) return BASA_ERR_WORKSPACE;
+  if (misaligned(workspace)) return BASA_ERR_ALIGN;
+  float* dD = static_cast<float*>(workspace);
+  float* dD_t = reinterpret_cast<float*>(static_cast<char*>(workspace) +
+                                         align256((size_t)d.B * d.H * d.N * sizeof(float)));
+  const JointGrads jg{qt, kt, vt, out_t, dout_t, lse_t, dD_t, dqt, dkt, dvt, (long long)L};
+  return launch_bwd_joint(d, q, k, v, out, dout, lse, dD, dq, dk, dv, jg, stream);
+}
+
 basa_status basa_full_attn(const void* q, const void* k, const void* v, void* out, float* lse,
                            const basa_params* p, cudaStream_t stream) {
   NvtxRange nvtx("basa_full_attn");

@@ -57,6 +57,18 @@ struct BwdArgs {
   int pt, ph, pw;
   int p_chunks;     // pooled key chunks
   float inv_count;  // 1 / (pt * ph * pw)
+  // joint text tokens: the extra keys (kp, vp, P) are then the L text tokens,
+  // not pooled cells, and the L text queries see every image and text token
+  int joint;
+  const void* qt;       // [B, L, H, d]
+  const void* dout_t;
+  const float* lse_t;   // [B, H, L]
+  const float* dD_t;    // [B, H, L]: dout_t . out_t
+  void* dqt;            // [B, L, H, d]
+  void* dkt;            // [B, L, Hkv, d]
+  void* dvt;
+  int t_chunks;         // text query chunks
+  const void* joint_out;  // out_t [B, L, H, d] (for D of the text rows)
 };
 
 template <bool BF16>
@@ -131,7 +143,9 @@ __global__ void __launch_bounds__(kBwdThreads) bwd_prep_kernel(BwdArgs a) {
 }
 
 // dQ: one CTA per (b, h, window, query chunk); D / 32 threads per query.
-template <bool BF16, int D>
+// TEXTQ (joint): one CTA per (b, h, text query chunk); the keys are every
+// image token and then every text token.
+template <bool BF16, int D, bool TEXTQ>
 __global__ void __launch_bounds__(kBwdThreads) bwd_dq_kernel(BwdArgs a) {
   constexpr int TPQ = D / 32;
   constexpr int DPT = D / TPQ;
@@ -139,9 +153,9 @@ __global__ void __launch_bounds__(kBwdThreads) bwd_dq_kernel(BwdArgs a) {
   __shared__ float ks[kChunk][D];
   __shared__ float vs[kChunk][D];
   long long u = blockIdx.x;
-  const int qc = (int)(u % a.n_chunks);
-  u /= a.n_chunks;
-  const int nwin = a.nwt * a.nwh * a.nww;
+  const int qc = (int)(u % (TEXTQ ? a.t_chunks : a.n_chunks));
+  u /= (TEXTQ ? a.t_chunks : a.n_chunks);
+  const int nwin = TEXTQ ? 1 : a.nwt * a.nwh * a.nww;
   const int win = (int)(u % nwin);
   u /= nwin;
   const int h = (int)(u % a.H);
@@ -149,38 +163,41 @@ __global__ void __launch_bounds__(kBwdThreads) bwd_dq_kernel(BwdArgs a) {
   const int hk = h / (a.H / a.Hkv);
   const int jw = win % a.nww, jh = (win / a.nww) % a.nwh, jt = win / (a.nww * a.nwh);
   const int part = threadIdx.x % TPQ;
-  const int lq = qc * QPC + threadIdx.x / TPQ;
-  const bool valid = lq < a.m;
+  const long long lq = (long long)qc * QPC + threadIdx.x / TPQ;
+  const bool valid = lq < (TEXTQ ? (long long)a.P : (long long)a.m);
   float qr[DPT], gr[DPT], acc[DPT];
   float lse = 0.f, dd = 0.f;
   long long qrow = 0;
   if (valid) {
-    const long long n = member(a, jt, jh, jw, lq);
-    qrow = (((long long)b * a.N + n) * a.H + h) * D + part * DPT;
+    const long long n = TEXTQ ? lq : member(a, jt, jh, jw, (int)lq);
+    const long long nrows = TEXTQ ? (long long)a.P : a.N;
+    qrow = (((long long)b * nrows + n) * a.H + h) * D + part * DPT;
     for (int c = 0; c < DPT; ++c) {
-      qr[c] = ld1<BF16>(a.q, qrow + c);
-      gr[c] = ld1<BF16>(a.dout, qrow + c);
+      qr[c] = ld1<BF16>(TEXTQ ? a.qt : a.q, qrow + c);
+      gr[c] = ld1<BF16>(TEXTQ ? a.dout_t : a.dout, qrow + c);
     }
-    lse = a.lse[((long long)b * a.H + h) * a.N + n];
-    dd = a.dD[((long long)b * a.H + h) * a.N + n];
+    lse = (TEXTQ ? a.lse_t : a.lse)[((long long)b * a.H + h) * nrows + n];
+    dd = (TEXTQ ? a.dD_t : a.dD)[((long long)b * a.H + h) * nrows + n];
   } else {
     for (int c = 0; c < DPT; ++c) qr[c] = gr[c] = 0.f;
   }
   for (int c = 0; c < DPT; ++c) acc[c] = 0.f;
-  const long long nkeys = a.m + a.P;  // the window's keys, then every pooled token
+  // the window's keys (text queries: every image token), then the extra keys
+  const long long nbase = TEXTQ ? a.N : (long long)a.m;
+  const long long nkeys = nbase + a.P;
   for (long long k0 = 0; k0 < nkeys; k0 += kChunk) {
     const int nk = nkeys - k0 < kChunk ? (int)(nkeys - k0) : kChunk;
     __syncthreads();
     for (int idx = threadIdx.x; idx < nk * D; idx += kBwdThreads) {
       const int jj = idx / D, c = idx % D;
       const long long j = k0 + jj;
-      if (j < a.m) {
-        const long long n = member(a, jt, jh, jw, (int)j);
+      if (j < nbase) {
+        const long long n = TEXTQ ? j : member(a, jt, jh, jw, (int)j);
         const long long off = (((long long)b * a.N + n) * a.Hkv + hk) * D + c;
         ks[jj][c] = ld1<BF16>(a.k, off);
         vs[jj][c] = ld1<BF16>(a.v, off);
       } else {
-        const long long off = (((long long)b * a.P + (j - a.m)) * a.Hkv + hk) * D + c;
+        const long long off = (((long long)b * a.P + (j - nbase)) * a.Hkv + hk) * D + c;
         ks[jj][c] = ld1<BF16>(a.kp, off);
         vs[jj][c] = ld1<BF16>(a.vp, off);
       }
@@ -200,7 +217,7 @@ __global__ void __launch_bounds__(kBwdThreads) bwd_dq_kernel(BwdArgs a) {
     }
   }
   if (valid)
-    for (int c = 0; c < DPT; ++c) st1<BF16>(a.dq, qrow + c, acc[c] * a.scale);
+    for (int c = 0; c < DPT; ++c) st1<BF16>(TEXTQ ? a.dqt : a.dq, qrow + c, acc[c] * a.scale);
 }
 
 // dK, dV: one CTA per (b, K/V head, window, key chunk); the queries of every
@@ -246,13 +263,27 @@ __global__ void __launch_bounds__(kBwdThreads) bwd_dkv_kernel(BwdArgs a) {
     for (int c = 0; c < DPT; ++c) kr[c] = vr[c] = 0.f;
   }
   for (int c = 0; c < DPT; ++c) dk[c] = dv[c] = 0.f;
-  const long long nqry = POOL ? a.N : a.m;  // the queries that see these keys
+  // Query sets: 0, the image queries that see these keys (the window's, or
+  // every one for pooled / text keys); 1 (joint), the L text queries.
+  for (int set = 0; set < (a.joint ? 2 : 1); ++set)
   for (int h = hk * group; h < (hk + 1) * group; ++h) {
+    const long long nqry = set ? (long long)a.P : (POOL ? a.N : a.m);
     for (long long q0 = 0; q0 < nqry; q0 += kChunk) {
       const int nq = nqry - q0 < kChunk ? (int)(nqry - q0) : kChunk;
       __syncthreads();
       for (int idx = threadIdx.x; idx < nq * D; idx += kBwdThreads) {
         const int ii = idx / D, c = idx % D;
+        if (set) {  // text query q0 + ii
+          const long long n = q0 + ii;
+          const long long off = (((long long)b * a.P + n) * a.H + h) * D + c;
+          qs[ii][c] = ld1<BF16>(a.qt, off);
+          gs[ii][c] = ld1<BF16>(a.dout_t, off);
+          if (c == 0) {
+            ls[ii] = a.lse_t[((long long)b * a.H + h) * a.P + n];
+            ds_[ii] = a.dD_t[((long long)b * a.H + h) * a.P + n];
+          }
+          continue;
+        }
         const long long n = POOL ? q0 + ii : member(a, jt, jh, jw, (int)(q0 + ii));
         const long long off = (((long long)b * a.N + n) * a.H + h) * D + c;
         qs[ii][c] = ld1<BF16>(a.q, off);
@@ -281,6 +312,13 @@ __global__ void __launch_bounds__(kBwdThreads) bwd_dkv_kernel(BwdArgs a) {
     }
   }
   if (!valid) return;
+  if (POOL && a.joint) {  // text keys: their final gradients
+    for (int c = 0; c < DPT; ++c) {
+      st1<BF16>(a.dkt, krow + c, dk[c] * a.scale);
+      st1<BF16>(a.dvt, krow + c, dv[c]);
+    }
+    return;
+  }
   if (POOL) {
     for (int c = 0; c < DPT; ++c) {
       a.dkp[krow + c] = dk[c];
@@ -288,7 +326,7 @@ __global__ void __launch_bounds__(kBwdThreads) bwd_dkv_kernel(BwdArgs a) {
     }
     return;
   }
-  if (a.P) {  // this token's share of its cell's pooled gradient
+  if (a.P && !a.joint) {  // this token's share of its cell's pooled gradient
     const long long hw = (long long)a.Hg * a.Wg;
     const long long t = n_row / hw, y = (n_row / a.Wg) % a.Hg, x = n_row % a.Wg;
     const long long cell = ((t / a.pt) * (a.Hg / a.ph) + y / a.ph) * (a.Wg / a.pw) + x / a.pw;
@@ -317,13 +355,29 @@ basa_status launch_bwd_typed(BwdArgs& a, const Dims& d, bool prep_only, cudaStre
   if (prep_blocks > 0x7fffffffLL || dq_blocks > 0x7fffffffLL) return BASA_ERR_UNSUPPORTED;
   bwd_prep_kernel<BF16, D><<<(unsigned)prep_blocks, kBwdThreads, 0, stream>>>(a);
   if (prep_only) return cudaGetLastError() == cudaSuccess ? BASA_OK : BASA_ERR_CUDA;
-  if (a.P) {  // the pooled tokens' gradients first: the window dK, dV add their share
+  if (a.joint) {  // D of the text rows: the prep kernel over [B, L, H] rows
+    BwdArgs t = a;
+    t.o = t.joint_out;
+    t.dout = a.dout_t;
+    t.dD = const_cast<float*>(a.dD_t);
+    t.N = a.P;
+    const long long trows = (long long)d.B * a.P * d.H;
+    bwd_prep_kernel<BF16, D><<<(unsigned)((trows + rows_per_block - 1) / rows_per_block),
+                               kBwdThreads, 0, stream>>>(t);
+  }
+  if (a.P) {  // the extra keys' gradients first: the window dK, dV add a pooled share
     a.p_chunks = (int)((a.P + per - 1) / per);
     const long long pool_blocks = (long long)d.B * d.Hkv * a.p_chunks;
     if (pool_blocks > 0x7fffffffLL) return BASA_ERR_UNSUPPORTED;
     bwd_dkv_kernel<BF16, D, true><<<(unsigned)pool_blocks, kBwdThreads, 0, stream>>>(a);
   }
-  bwd_dq_kernel<BF16, D><<<(unsigned)dq_blocks, kBwdThreads, 0, stream>>>(a);
+  bwd_dq_kernel<BF16, D, false><<<(unsigned)dq_blocks, kBwdThreads, 0, stream>>>(a);
+  if (a.joint) {  // the text queries' dq
+    a.t_chunks = (int)((a.P + per - 1) / per);
+    const long long tq_blocks = (long long)d.B * d.H * a.t_chunks;
+    if (tq_blocks > 0x7fffffffLL) return BASA_ERR_UNSUPPORTED;
+    bwd_dq_kernel<BF16, D, true><<<(unsigned)tq_blocks, kBwdThreads, 0, stream>>>(a);
+  }
   bwd_dkv_kernel<BF16, D, false><<<(unsigned)dkv_blocks, kBwdThreads, 0, stream>>>(a);
   return cudaGetLastError() == cudaSuccess ? BASA_OK : BASA_ERR_CUDA;
 }
@@ -331,8 +385,13 @@ basa_status launch_bwd_typed(BwdArgs& a, const Dims& d, bool prep_only, cudaStre
 basa_status launch_bwd_common(const Dims& d, const void* q, const void* k, const void* v,
                               const void* o, const void* dout, const float* lse, float* dD,
                               void* dq, void* dk, void* dv, const PoolGrads* pg, bool prep_only,
-                              cudaStream_t stream) {
+                              cudaStream_t stream, const JointGrads* jg = nullptr) {
   BwdArgs a;
+  a.joint = 0;
+  a.qt = a.dout_t = a.joint_out = nullptr;
+  a.lse_t = a.dD_t = nullptr;
+  a.dqt = a.dkt = a.dvt = nullptr;
+  a.t_chunks = 0;
   a.kp = a.vp = nullptr;
   a.dkp = a.dvp = nullptr;
   a.P = 0;
@@ -344,6 +403,14 @@ basa_status launch_bwd_common(const Dims& d, const void* q, const void* k, const
     a.P = d.P;
     a.pt = d.pt; a.ph = d.ph; a.pw = d.pw;
     a.inv_count = 1.0f / (float)(d.pt * d.ph * d.pw);
+  }
+  if (jg && jg->L > 0) {  // the text tokens are the extra keys; text queries see every token
+    a.joint = 1;
+    a.kp = jg->kt; a.vp = jg->vt;
+    a.P = jg->L;
+    a.qt = jg->qt; a.dout_t = jg->dout_t; a.joint_out = jg->out_t;
+    a.lse_t = jg->lse_t; a.dD_t = jg->dD_t;
+    a.dqt = jg->dqt; a.dkt = jg->dkt; a.dvt = jg->dvt;
   }
   a.q = q; a.k = k; a.v = v; a.o = o; a.dout = dout; a.lse = lse; a.dD = dD;
   a.dq = dq; a.dk = dk; a.dv = dv;
@@ -371,6 +438,13 @@ basa_status launch_bwd(const Dims& d, const void* q, const void* k, const void* 
                        const void* o, const void* dout, const float* lse, float* dD, void* dq,
                        void* dk, void* dv, const PoolGrads* pg, cudaStream_t stream) {
   return launch_bwd_common(d, q, k, v, o, dout, lse, dD, dq, dk, dv, pg, false, stream);
+}
+
+basa_status launch_bwd_joint(const Dims& d, const void* q, const void* k, const void* v,
+                             const void* o, const void* dout, const float* lse, float* dD,
+                             void* dq, void* dk, void* dv, const JointGrads& jg,
+                             cudaStream_t stream) {
+  return launch_bwd_common(d, q, k, v, o, dout, lse, dD, dq, dk, dv, nullptr, false, stream, &jg);
 }
 
 basa_status launch_bwd_prep(const Dims& d, const void* o, const void* dout, float* dD,

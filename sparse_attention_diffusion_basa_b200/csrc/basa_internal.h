@@ -124,6 +124,31 @@ struct PoolGrads {
   float* dvp;
 };
 
+// Joint text + image backward: the text tokens' tensors ([B, L, H or Hkv, d];
+// lse_t [B, H, L]) and the workspace for their D = rowsum(dout_t * out_t).
+struct JointGrads {
+  const void* qt;
+  const void* kt;
+  const void* vt;
+  const void* out_t;
+  const void* dout_t;
+  const float* lse_t;
+  float* dD_t;
+  void* dqt;
+  void* dkt;
+  void* dvt;
+  long long L;
+};
+
+// Joint backward on CUDA cores (fp32 arithmetic): D of the image and text rows,
+// the text keys' gradients over every query, dQ of the image queries (window
+// and text keys) and of the text queries (every key), then the image keys' dK,
+// dV over their window's queries and every text query.
+basa_status launch_bwd_joint(const Dims& d, const void* q, const void* k, const void* v,
+                             const void* o, const void* dout, const float* lse, float* dD,
+                             void* dq, void* dk, void* dv, const JointGrads& jg,
+                             cudaStream_t stream);
+
 // Backward of window attention on CUDA cores: D = rowsum(dO * O) into dD, the
 // pooled tokens' gradients (pg, nullable), then dQ, then dK and dV.
 basa_status launch_bwd(const Dims& d, const void* q, const void* k, const void* v,
