@@ -35,6 +35,14 @@
  *    token, text queries attend to every image and text token, each under one
  *    softmax.
  *
+ *  - Grids that a window size does not divide (only with `pad` set; the pages
+ *    are silent here).  Reading used here, the one shifted-window attention
+ *    commonly takes: each axis is padded at its far end to the next multiple
+ *    of the window, Gp = ceil(G / w) * w; the shift rolls the padded axis
+ *    (wid(x) = floor(((x - s) mod Gp) / w)); padded positions hold no token,
+ *    so they are neither queries nor keys, and a window holds only its real
+ *    members.  With w dividing G this is the definition above.
+ *
  * Arithmetic: every input value is read as a double; dot products, the
  * max-subtracted softmax and the weighted sum are all in double precision.
  *
@@ -56,11 +64,49 @@ typedef struct {
   int64_t pt, ph, pw;   /* pooled cell size; all zero = no global memory */
   double scale;         /* softmax scale applied to q.k */
   int64_t Hkv;          /* K/V heads (grouped-query attention); 0 = H */
+  int64_t pad;          /* 1: pad axes the window does not divide (see above) */
 } oracle_params;
 
 static int64_t floor_mod(int64_t a, int64_t n) {
   int64_t r = a % n;
   return r < 0 ? r + n : r;
+}
+
+/* Padded extent of an axis: G itself, or with `pad` the next multiple of w. */
+static int64_t padded(int64_t G, int64_t w, int64_t pad) {
+  return pad ? (G + w - 1) / w * w : G;
+}
+
+/* 0 when the window fits the grid: w divides G on every axis, or `pad` is set. */
+static int grid_ok(const oracle_params* p) {
+  if (p->wt <= 0 || p->wh <= 0 || p->ww <= 0) return -1;
+  if (p->pad) return 0;
+  return (p->T % p->wt || p->Hg % p->wh || p->Wg % p->ww) ? -1 : 0;
+}
+
+/*
+ * Members of window (it, iy, ix) in (t, row, column) order: coordinate l of
+ * the window on an axis is (i * w + s + l) mod Gp; positions past the real
+ * grid are padding and skipped.  Writes (t, y, x) triples, returns the count.
+ */
+static int64_t window_members(const oracle_params* p, int64_t it, int64_t iy, int64_t ix,
+                              int64_t* tok) {
+  const int64_t Tp = padded(p->T, p->wt, p->pad), Hp = padded(p->Hg, p->wh, p->pad),
+                Wp = padded(p->Wg, p->ww, p->pad);
+  int64_t j = 0;
+  for (int64_t lt = 0; lt < p->wt; ++lt)
+    for (int64_t ly = 0; ly < p->wh; ++ly)
+      for (int64_t lx = 0; lx < p->ww; ++lx) {
+        const int64_t tt = floor_mod(it * p->wt + p->st + lt, Tp);
+        const int64_t yy = floor_mod(iy * p->wh + p->sh + ly, Hp);
+        const int64_t xx = floor_mod(ix * p->ww + p->sw + lx, Wp);
+        if (tt >= p->T || yy >= p->Hg || xx >= p->Wg) continue;
+        tok[3 * j] = tt;
+        tok[3 * j + 1] = yy;
+        tok[3 * j + 2] = xx;
+        ++j;
+      }
+  return j;
 }
 
 static int64_t tok_index(const oracle_params* p, int64_t b, int64_t t, int64_t y,
@@ -104,29 +150,24 @@ void oracle_pool(const double* x, double* xp, const oracle_params* p) {
 static void one_query(const double* q, const double* k, const double* v,
                       const double* kp, const double* vp, int64_t P,
                       const oracle_params* p, int64_t b, int64_t t, int64_t y,
-                      int64_t x, int64_t h, double* z, double* out_row,
+                      int64_t x, int64_t h, double* z, int64_t* tok, double* out_row,
                       double* lse_out) {
   const int64_t d = p->d;
   const double* qv = q + tok_index(p, b, t, y, x, h);
-  /* window id of the query on each axis */
-  const int64_t it = floor_mod(t - p->st, p->T) / p->wt;
-  const int64_t iy = floor_mod(y - p->sh, p->Hg) / p->wh;
-  const int64_t ix = floor_mod(x - p->sw, p->Wg) / p->ww;
-  const int64_t m = p->wt * p->wh * p->ww;
+  /* window id of the query on each (padded) axis */
+  const int64_t it = floor_mod(t - p->st, padded(p->T, p->wt, p->pad)) / p->wt;
+  const int64_t iy = floor_mod(y - p->sh, padded(p->Hg, p->wh, p->pad)) / p->wh;
+  const int64_t ix = floor_mod(x - p->sw, padded(p->Wg, p->ww, p->pad)) / p->ww;
+  const int64_t m = window_members(p, it, iy, ix, tok);
 
-  /* logits over the window members, enumerated from the window id */
+  /* logits over the window members */
   int64_t j = 0;
-  for (int64_t lt = 0; lt < p->wt; ++lt)
-    for (int64_t ly = 0; ly < p->wh; ++ly)
-      for (int64_t lx = 0; lx < p->ww; ++lx) {
-        const int64_t tt = floor_mod(it * p->wt + p->st + lt, p->T);
-        const int64_t yy = floor_mod(iy * p->wh + p->sh + ly, p->Hg);
-        const int64_t xx = floor_mod(ix * p->ww + p->sw + lx, p->Wg);
-        const double* kv = k + kv_index(p, b, tt, yy, xx, kv_head(p, h));
-        double s = 0.0;
-        for (int64_t c = 0; c < d; ++c) s += qv[c] * kv[c];
-        z[j++] = p->scale * s;
-      }
+  for (int64_t a = 0; a < m; ++a) {
+    const double* kv = k + kv_index(p, b, tok[3 * a], tok[3 * a + 1], tok[3 * a + 2], kv_head(p, h));
+    double s = 0.0;
+    for (int64_t c = 0; c < d; ++c) s += qv[c] * kv[c];
+    z[j++] = p->scale * s;
+  }
   /* logits over the pooled tokens */
   for (int64_t c2 = 0; c2 < P; ++c2) {
     const double* kv = kp + ((b * P + c2) * kv_heads(p) + kv_head(p, h)) * d;
@@ -144,16 +185,11 @@ static void one_query(const double* q, const double* k, const double* v,
   }
   for (int64_t c = 0; c < d; ++c) out_row[c] = 0.0;
   j = 0;
-  for (int64_t lt = 0; lt < p->wt; ++lt)
-    for (int64_t ly = 0; ly < p->wh; ++ly)
-      for (int64_t lx = 0; lx < p->ww; ++lx) {
-        const int64_t tt = floor_mod(it * p->wt + p->st + lt, p->T);
-        const int64_t yy = floor_mod(iy * p->wh + p->sh + ly, p->Hg);
-        const int64_t xx = floor_mod(ix * p->ww + p->sw + lx, p->Wg);
-        const double* vv = v + kv_index(p, b, tt, yy, xx, kv_head(p, h));
-        const double a = z[j++] / den;
-        for (int64_t c = 0; c < d; ++c) out_row[c] += a * vv[c];
-      }
+  for (int64_t a = 0; a < m; ++a) {
+    const double* vv = v + kv_index(p, b, tok[3 * a], tok[3 * a + 1], tok[3 * a + 2], kv_head(p, h));
+    const double w = z[j++] / den;
+    for (int64_t c = 0; c < d; ++c) out_row[c] += w * vv[c];
+  }
   for (int64_t c2 = 0; c2 < P; ++c2) {
     const double* vv = vp + ((b * P + c2) * kv_heads(p) + kv_head(p, h)) * d;
     const double a = z[j++] / den;
@@ -180,7 +216,7 @@ int oracle_window_attn(const double* q, const double* k, const double* v,
                        const double* kp, const double* vp, double* out,
                        double* lse, const oracle_params* p, const int64_t* sel,
                        int64_t nsel, int nthreads) {
-  if (p->T % p->wt || p->Hg % p->wh || p->Wg % p->ww) return -1;
+  if (grid_ok(p)) return -1;
   int64_t P = 0;
   if (kp) {
     if (p->pt <= 0 || p->ph <= 0 || p->pw <= 0) return -1;
@@ -198,7 +234,7 @@ int oracle_window_attn_extra(const double* q, const double* k, const double* v,
                              const double* kx, const double* vx, int64_t nx, double* out,
                              double* lse, const oracle_params* p, const int64_t* sel,
                              int64_t nsel, int nthreads) {
-  if (p->T % p->wt || p->Hg % p->wh || p->Wg % p->ww) return -1;
+  if (grid_ok(p)) return -1;
   if (nx < 0 || (nx > 0 && (!kx || !vx))) return -1;
   return window_attn_keys(q, k, v, nx ? kx : NULL, nx ? vx : NULL, nx, out, lse, p, sel, nsel,
                           nthreads);
@@ -219,6 +255,7 @@ static int window_attn_keys(const double* q, const double* k, const double* v,
 #pragma omp parallel
   {
     double* z = (double*)malloc(sizeof(double) * (size_t)(m + P));
+    int64_t* tok = (int64_t*)malloc(sizeof(int64_t) * (size_t)m * 3);
 #pragma omp for schedule(dynamic, 64)
     for (int64_t i = 0; i < total; ++i) {
       int64_t b, n, h;
@@ -235,9 +272,10 @@ static int window_attn_keys(const double* q, const double* k, const double* v,
       double* orow = sel ? out + i * p->d : out + tok_index(p, b, t, y, x, h);
       double* l = NULL;
       if (lse) l = sel ? lse + i : lse + (b * p->H + h) * N + n;
-      one_query(q, k, v, kp, vp, P, p, b, t, y, x, h, z, orow, l);
+      one_query(q, k, v, kp, vp, P, p, b, t, y, x, h, z, tok, orow, l);
     }
     free(z);
+    free(tok);
   }
   return 0;
 }
@@ -327,14 +365,15 @@ int oracle_max_threads(void) {
 int oracle_window_attn_bwd(const double* q, const double* k, const double* v,
                            const double* dout, double* dq, double* dk, double* dv,
                            const oracle_params* p) {
-  if (p->T % p->wt || p->Hg % p->wh || p->Wg % p->ww) return -1;
+  if (grid_ok(p)) return -1;
   const int pooled = p->pt > 0 && p->ph > 0 && p->pw > 0;
   if (pooled && (p->T % p->pt || p->Hg % p->ph || p->Wg % p->pw)) return -1;
-  const int64_t d = p->d, N = p->T * p->Hg * p->Wg, m = p->wt * p->wh * p->ww;
-  const int64_t nwt = p->T / p->wt, nwh = p->Hg / p->wh, nww = p->Wg / p->ww;
+  const int64_t d = p->d, N = p->T * p->Hg * p->Wg, mmax = p->wt * p->wh * p->ww;
+  const int64_t nwt = padded(p->T, p->wt, p->pad) / p->wt, nwh = padded(p->Hg, p->wh, p->pad) / p->wh,
+                nww = padded(p->Wg, p->ww, p->pad) / p->ww;
   const int64_t Ph = pooled ? p->Hg / p->ph : 0, Pw = pooled ? p->Wg / p->pw : 0;
   const int64_t Pn = pooled ? (p->T / p->pt) * Ph * Pw : 0; /* pooled tokens per batch */
-  const int64_t nk = m + Pn;                                /* keys of every query */
+  const int64_t nkmax = mmax + Pn;                          /* keys of a query, at most */
   const int64_t Hk = kv_heads(p);
   memset(dq, 0, sizeof(double) * (size_t)(p->B * N * p->H * d));
   memset(dk, 0, sizeof(double) * (size_t)(p->B * N * Hk * d));
@@ -349,23 +388,17 @@ int oracle_window_attn_bwd(const double* q, const double* k, const double* v,
     oracle_pool(k, kp, p);
     oracle_pool(v, vp, p);
   }
-  int64_t* tok = (int64_t*)malloc(sizeof(int64_t) * (size_t)m * 3);
-  double* P = (double*)malloc(sizeof(double) * (size_t)(m * nk));
-  double* dS = (double*)malloc(sizeof(double) * (size_t)(m * nk));
+  int64_t* tok = (int64_t*)malloc(sizeof(int64_t) * (size_t)mmax * 3);
+  double* P = (double*)malloc(sizeof(double) * (size_t)(mmax * nkmax));
+  double* dS = (double*)malloc(sizeof(double) * (size_t)(mmax * nkmax));
   for (int64_t b = 0; b < p->B; ++b)
     for (int64_t h = 0; h < p->H; ++h) {
       const int64_t hk = kv_head(p, h);
       for (int64_t wi = 0; wi < nwt * nwh * nww; ++wi) {
         const int64_t it = wi / (nwh * nww), iy = (wi / nww) % nwh, ix = wi % nww;
-        int64_t j = 0;  /* members of window (it, iy, ix), enumerated from its id */
-        for (int64_t lt = 0; lt < p->wt; ++lt)
-          for (int64_t ly = 0; ly < p->wh; ++ly)
-            for (int64_t lx = 0; lx < p->ww; ++lx) {
-              tok[3 * j] = floor_mod(it * p->wt + p->st + lt, p->T);
-              tok[3 * j + 1] = floor_mod(iy * p->wh + p->sh + ly, p->Hg);
-              tok[3 * j + 2] = floor_mod(ix * p->ww + p->sw + lx, p->Wg);
-              ++j;
-            }
+        /* members of window (it, iy, ix), enumerated from its id */
+        const int64_t m = window_members(p, it, iy, ix, tok);
+        const int64_t nk = m + Pn;  /* keys of every query of this window */
         /* key c2 < m: window member c2; key m + c: pooled token c of batch b */
 #define KEY(c2) ((c2) < m ? k + kv_index(p, b, tok[3 * (c2)], tok[3 * (c2) + 1], tok[3 * (c2) + 2], hk) \
                           : kp + ((b * Pn + ((c2) - m)) * Hk + hk) * d)
@@ -494,9 +527,10 @@ int oracle_joint_attn_bwd(const double* q, const double* k, const double* v, con
                           const double* dout_t, double* dq, double* dk, double* dv, double* dqt,
                           double* dkt, double* dvt, const oracle_params* p) {
   if (L < 0) return -1;
-  if (p->T % p->wt || p->Hg % p->wh || p->Wg % p->ww) return -1;
-  const int64_t d = p->d, N = p->T * p->Hg * p->Wg, m = p->wt * p->wh * p->ww;
-  const int64_t nwt = p->T / p->wt, nwh = p->Hg / p->wh, nww = p->Wg / p->ww;
+  if (grid_ok(p)) return -1;
+  const int64_t d = p->d, N = p->T * p->Hg * p->Wg, mmax = p->wt * p->wh * p->ww;
+  const int64_t nwt = padded(p->T, p->wt, p->pad) / p->wt, nwh = padded(p->Hg, p->wh, p->pad) / p->wh,
+                nww = padded(p->Wg, p->ww, p->pad) / p->ww;
   const int64_t H = p->H, Hk = kv_heads(p);
   memset(dq, 0, sizeof(double) * (size_t)(p->B * N * H * d));
   memset(dk, 0, sizeof(double) * (size_t)(p->B * N * Hk * d));
@@ -513,7 +547,7 @@ int oracle_joint_attn_bwd(const double* q, const double* k, const double* v, con
   double** dvp = (double**)malloc(sizeof(double*) * (size_t)nmax);
   double* z = (double*)malloc(sizeof(double) * (size_t)nmax);
   double* dpv = (double*)malloc(sizeof(double) * (size_t)nmax);
-  int64_t* tok = (int64_t*)malloc(sizeof(int64_t) * (size_t)m * 3);
+  int64_t* tok = (int64_t*)malloc(sizeof(int64_t) * (size_t)mmax * 3);
   for (int64_t b = 0; b < p->B; ++b)
     for (int64_t h = 0; h < H; ++h) {
       const int64_t hk = kv_head(p, h);
@@ -524,15 +558,7 @@ int oracle_joint_attn_bwd(const double* q, const double* k, const double* v, con
       /* image queries: their window, then the text keys */
       for (int64_t wi = 0; wi < nwt * nwh * nww; ++wi) {
         const int64_t it = wi / (nwh * nww), iy = (wi / nww) % nwh, ix = wi % nww;
-        int64_t j = 0;
-        for (int64_t lt = 0; lt < p->wt; ++lt)
-          for (int64_t ly = 0; ly < p->wh; ++ly)
-            for (int64_t lx = 0; lx < p->ww; ++lx) {
-              tok[3 * j] = floor_mod(it * p->wt + p->st + lt, p->T);
-              tok[3 * j + 1] = floor_mod(iy * p->wh + p->sh + ly, p->Hg);
-              tok[3 * j + 2] = floor_mod(ix * p->ww + p->sw + lx, p->Wg);
-              ++j;
-            }
+        const int64_t m = window_members(p, it, iy, ix, tok);
         /* window members in key slots N - m .. N - 1, so the text keys follow */
         for (int64_t c2 = 0; c2 < m; ++c2) {
           const int64_t o = kv_index(p, b, tok[3 * c2], tok[3 * c2 + 1], tok[3 * c2 + 2], hk);

@@ -19,10 +19,13 @@ import math
 import numpy as np
 
 
-def window_ids(G: int, w: int, s: int) -> np.ndarray:
-    """Window index of every coordinate 0..G-1 on one axis."""
+def window_ids(G: int, w: int, s: int, pad: bool = False) -> np.ndarray:
+    """Window index of every coordinate 0..G-1 on one axis.  With ``pad`` the
+    axis is first padded to the next multiple of w (padding holds no token) and
+    the shift rolls the padded axis."""
     x = np.arange(G)
-    return ((x - s) % G) // w
+    Gp = -(-G // w) * w if pad else G
+    return ((x - s) % Gp) // w
 
 
 def _pool(x: np.ndarray, pool) -> np.ndarray:
@@ -33,16 +36,16 @@ def _pool(x: np.ndarray, pool) -> np.ndarray:
 
 
 def brute_window_attn(q, k, v, window, shift=(0, 0, 0), pool=(0, 0, 0), scale=None,
-                      want_lse=False):
+                      want_lse=False, pad=False):
     q = np.asarray(q, dtype=np.float64)
     k = np.asarray(k, dtype=np.float64)
     v = np.asarray(v, dtype=np.float64)
     B, T, Hg, Wg, H, d = q.shape
     N = T * Hg * Wg
     sc = 1.0 / math.sqrt(d) if scale is None else scale
-    it = window_ids(T, window[0], shift[0])
-    iy = window_ids(Hg, window[1], shift[1])
-    ix = window_ids(Wg, window[2], shift[2])
+    it = window_ids(T, window[0], shift[0], pad)
+    iy = window_ids(Hg, window[1], shift[1], pad)
+    ix = window_ids(Wg, window[2], shift[2], pad)
     wid = np.stack(np.meshgrid(it, iy, ix, indexing="ij"), axis=-1).reshape(N, 3)
     mask = np.all(wid[:, None, :] == wid[None, :, :], axis=-1)  # [N, N]
     qf = q.reshape(B, N, H, d).transpose(0, 2, 1, 3)
@@ -68,7 +71,8 @@ def brute_window_attn(q, k, v, window, shift=(0, 0, 0), pool=(0, 0, 0), scale=No
     return out
 
 
-def brute_joint_attn(q, k, v, qt, kt, vt, window, shift=(0, 0, 0), scale=None, want_lse=False):
+def brute_joint_attn(q, k, v, qt, kt, vt, window, shift=(0, 0, 0), scale=None, want_lse=False,
+                     pad=False):
     """Joint text + image attention as one dense masked softmax over the
     concatenated sequence [N image tokens, L text tokens]: image-image pairs keep
     the same-window mask, every pair that involves a text token is allowed."""
@@ -76,9 +80,9 @@ def brute_joint_attn(q, k, v, qt, kt, vt, window, shift=(0, 0, 0), scale=None, w
     B, T, Hg, Wg, H, d = q.shape
     N, L = T * Hg * Wg, qt.shape[1]
     sc = 1.0 / math.sqrt(d) if scale is None else scale
-    it = window_ids(T, window[0], shift[0])
-    iy = window_ids(Hg, window[1], shift[1])
-    ix = window_ids(Wg, window[2], shift[2])
+    it = window_ids(T, window[0], shift[0], pad)
+    iy = window_ids(Hg, window[1], shift[1], pad)
+    ix = window_ids(Wg, window[2], shift[2], pad)
     wid = np.stack(np.meshgrid(it, iy, ix, indexing="ij"), axis=-1).reshape(N, 3)
     mask = np.ones((N + L, N + L), dtype=bool)
     mask[:N, :N] = np.all(wid[:, None, :] == wid[None, :, :], axis=-1)

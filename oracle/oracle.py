@@ -20,7 +20,8 @@ from . import build as _build
 class _CParams(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int64) for n in
                 ("B", "H", "T", "Hg", "Wg", "d", "wt", "wh", "ww", "st", "sh", "sw",
-                 "pt", "ph", "pw")] + [("scale", ctypes.c_double), ("Hkv", ctypes.c_int64)]
+                 "pt", "ph", "pw")] + [("scale", ctypes.c_double), ("Hkv", ctypes.c_int64),
+                                       ("pad", ctypes.c_int64)]
 
 
 @dataclass
@@ -38,11 +39,12 @@ class OracleParams:
     pool: Tuple[int, int, int] = (0, 0, 0)
     scale: Optional[float] = None
     Hkv: int = 0  # K/V heads (grouped-query attention); 0 = H
+    pad: bool = False  # pad axes the window does not divide; padding is no token
 
     def c(self) -> _CParams:
         sc = self.scale if self.scale is not None else 1.0 / math.sqrt(self.d)
         return _CParams(self.B, self.H, self.T, self.Hg, self.Wg, self.d,
-                        *self.window, *self.shift, *self.pool, sc, self.Hkv)
+                        *self.window, *self.shift, *self.pool, sc, self.Hkv, int(self.pad))
 
     @property
     def kv_heads(self) -> int:

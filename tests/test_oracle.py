@@ -604,3 +604,144 @@ def test_backward_matches_central_differences(oracle_mod):
             args[which][idx] -= 2 * h
             dn = f(*args)
             assert abs((up - dn) / (2 * h) - grad[idx]) < 1e-7
+
+
+# ---------------------------------------------------------------------------
+# Grids the window does not divide (pad = True).  The pages are silent here; the
+# reading pinned below: each axis padded at its far end to the next multiple of
+# the window, the shift rolls the padded axis, padding is neither query nor key.
+# ---------------------------------------------------------------------------
+PADDED = [  # shape, window, pool
+    ((1, 1, 5, 7, 2, 8), (1, 2, 3), (0, 0, 0)),
+    ((1, 3, 5, 4, 1, 4), (2, 4, 3), (0, 0, 0)),
+    ((2, 1, 3, 3, 1, 4), (1, 4, 4), (0, 0, 0)),   # window larger than the grid
+    ((1, 1, 6, 10, 1, 8), (1, 4, 4), (1, 2, 5)),  # pooled cells divide the real grid
+]
+
+
+def _Ppad(shape, window, shift=(0, 0, 0), pool=(0, 0, 0), scale=None):
+    prm = _P(shape, window, shift, pool, scale)
+    prm.pad = True
+    return prm
+
+
+@pytest.mark.parametrize("shape,window,pool", PADDED)
+def test_padded_matches_brute_force_all_shifts(oracle_mod, shape, window, pool):
+    """Dense same-window mask from window ids on the padded axes, every shift."""
+    r = _rng(301)
+    q, k, v = (r.standard_normal(shape) for _ in range(3))
+    shifts = list(itertools.product(*[range(-w, w + 1) for w in window]))
+    if len(shifts) > 40:
+        idx = _rng(302).choice(len(shifts), 40, replace=False)
+        shifts = [shifts[i] for i in idx]
+    for s in shifts:
+        got, lse = oracle_mod.window_attn(q, k, v, _Ppad(shape, window, s, pool), want_lse=True)
+        want, want_lse = oracle_mod.brute_window_attn(q, k, v, window, s, pool, want_lse=True,
+                                                      pad=True)
+        np.testing.assert_allclose(got, want, rtol=0, atol=1e-12, err_msg=str(s))
+        np.testing.assert_allclose(lse, want_lse, rtol=0, atol=1e-12, err_msg=str(s))
+
+
+@pytest.mark.parametrize("shape,window", [(s, w) for s, w, _ in PADDED[:3]])
+def test_padded_shift_zero_is_blockwise_attention(oracle_mod, shape, window):
+    """Shift 0: the windows are the grid's blocks [j w, min((j + 1) w, G)) on each
+    axis, the last one cut short; attention within each block by torch SDPA on
+    the sliced tensors."""
+    r = _rng(303)
+    q, k, v = (r.standard_normal(shape) for _ in range(3))
+    got = oracle_mod.window_attn(q, k, v, _Ppad(shape, window))
+    B, T, Hg, Wg, H, d = shape
+    want = np.zeros(shape)
+    for t0 in range(0, T, window[0]):
+        for y0 in range(0, Hg, window[1]):
+            for x0 in range(0, Wg, window[2]):
+                sl = (slice(None), slice(t0, t0 + window[0]), slice(y0, y0 + window[1]),
+                      slice(x0, x0 + window[2]))
+                blk = [torch.from_numpy(np.ascontiguousarray(a[sl])) for a in (q, k, v)]
+                n = blk[0].shape[1] * blk[0].shape[2] * blk[0].shape[3]
+                qb, kb, vb = (x.reshape(B, n, H, d).transpose(1, 2) for x in blk)
+                o = torch.nn.functional.scaled_dot_product_attention(qb, kb, vb)
+                want[sl] = o.transpose(1, 2).reshape(blk[0].shape).numpy()
+    np.testing.assert_allclose(got, want, rtol=0, atol=1e-12)
+
+
+def test_padded_equals_divisible_grid_with_masked_holes(oracle_mod):
+    """Embed the grid in its padded (divisible) grid and run the unpadded oracle
+    there: an extra feature puts every padding key's logit 1e4 below the rest,
+    so its weight underflows to 0; real queries then match the padded call."""
+    r = _rng(304)
+    shape, window = (1, 3, 5, 7, 2, 8), (2, 2, 3)
+    B, T, Hg, Wg, H, d = shape
+    Tp, Hp, Wp = (-(-G // w) * w for G, w in zip((T, Hg, Wg), window))
+    q, k, v = (r.standard_normal(shape) for _ in range(3))
+    sc = 1.0 / math.sqrt(d)
+    qe, ke, ve = (np.zeros((B, Tp, Hp, Wp, H, d + 1)) for _ in range(3))
+    qe[:, :T, :Hg, :Wg, :, :d] = q * sc
+    qe[..., d] = 1.0
+    ke[:, :T, :Hg, :Wg, :, :d] = k
+    ke[..., d] = -1e4
+    ke[:, :T, :Hg, :Wg, :, d] = 0.0
+    ve[:, :T, :Hg, :Wg, :, :d] = v
+    for s in [(0, 0, 0), (1, 1, 2), (1, 0, 1), (0, 1, 0)]:
+        got, lse = oracle_mod.window_attn(q, k, v, _Ppad(shape, window, s), want_lse=True)
+        emb, lse_e = oracle_mod.window_attn(qe, ke, ve, _P((B, Tp, Hp, Wp, H, d + 1), window, s,
+                                                          scale=1.0), want_lse=True)
+        np.testing.assert_allclose(got, emb[:, :T, :Hg, :Wg, :, :d], rtol=0, atol=1e-12)
+        real = np.zeros((Tp, Hp, Wp), dtype=bool)
+        real[:T, :Hg, :Wg] = True
+        np.testing.assert_allclose(lse, lse_e[:, :, real.reshape(-1)], rtol=0, atol=1e-12)
+
+
+def test_padded_flag_changes_nothing_when_the_window_divides(oracle_mod):
+    r = _rng(305)
+    shape, window = (1, 2, 8, 6, 2, 4), (2, 4, 3)
+    q, k, v = (r.standard_normal(shape) for _ in range(3))
+    for s in [(0, 0, 0), (1, 2, 1)]:
+        a = oracle_mod.window_attn(q, k, v, _P(shape, window, s, (1, 2, 3)))
+        b = oracle_mod.window_attn(q, k, v, _Ppad(shape, window, s, (1, 2, 3)))
+        assert np.array_equal(a, b)
+
+
+@pytest.mark.parametrize("shape,window,shift,pool,L", [
+    ((1, 1, 5, 7, 2, 8), (1, 2, 3), (0, 1, 2), (0, 0, 0), 0),
+    ((1, 3, 5, 4, 1, 4), (2, 4, 3), (1, 3, 1), (0, 0, 0), 0),
+    ((1, 1, 6, 10, 2, 4), (1, 4, 4), (0, 1, 3), (1, 2, 5), 0),
+    ((1, 1, 5, 7, 2, 4), (1, 2, 3), (0, 1, 2), (0, 0, 0), 3),
+])
+def test_padded_backward_matches_autograd(oracle_mod, shape, window, shift, pool, L):
+    """Padded-grid gradients (window, pooled, joint) == torch autograd (fp64)
+    through SDPA with the padded same-window mask (pooled cell means and text
+    tokens appended as keys every query sees; text queries see every key)."""
+    from oracle import window_ids
+    r = _rng(306)
+    B, T, Hg, Wg, H, d = shape
+    N = T * Hg * Wg
+    q, k, v, g = (r.standard_normal(shape) for _ in range(4))
+    qt, kt, vt, gt = (r.standard_normal((B, L, H, d)) for _ in range(4))
+    prm = _Ppad(shape, window, shift, pool)
+    if L:
+        got = oracle_mod.joint_attn_bwd(q, k, v, qt, kt, vt, g, gt, prm)
+    else:
+        got = oracle_mod.window_attn_bwd(q, k, v, g, prm)
+    ids = [window_ids(G, w, s, pad=True) for G, w, s in zip((T, Hg, Wg), window, shift)]
+    wid = np.stack(np.meshgrid(*ids, indexing="ij"), axis=-1).reshape(-1, 3)
+    ts = [torch.from_numpy(x).requires_grad_() for x in (q, k, v, qt, kt, vt)]
+    flat = lambda x: x.reshape(B, -1, H, d)
+    keys, vals = [flat(ts[1])], [flat(ts[2])]
+    if pool != (0, 0, 0):
+        cell = lambda x: x.reshape(B, T // pool[0], pool[0], Hg // pool[1], pool[1],
+                                   Wg // pool[2], pool[2], H, d).mean(dim=(2, 4, 6))
+        keys.append(flat(cell(ts[1])))
+        vals.append(flat(cell(ts[2])))
+    keys.append(ts[4])
+    vals.append(ts[5])
+    qa = torch.cat([flat(ts[0]), ts[3]], 1).transpose(1, 2)
+    ka = torch.cat(keys, 1).transpose(1, 2)
+    va = torch.cat(vals, 1).transpose(1, 2)
+    nk = ka.shape[2]
+    mask = torch.ones(N + L, nk, dtype=torch.bool)
+    mask[:N, :N] = torch.from_numpy(np.all(wid[:, None, :] == wid[None, :, :], axis=-1))
+    o = torch.nn.functional.scaled_dot_product_attention(qa, ka, va, attn_mask=mask)
+    o.backward(torch.cat([flat(torch.from_numpy(g)), torch.from_numpy(gt)], 1).transpose(1, 2))
+    for gg, t in zip(got, ts):
+        np.testing.assert_allclose(gg, t.grad.numpy(), rtol=0, atol=1e-12)

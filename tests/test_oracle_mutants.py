@@ -17,17 +17,25 @@ from oracle.oracle import use_library
 import test_oracle as pins
 
 MUTANTS = {
-    "shift sign on the column axis": ("floor_mod(x - p->sw, p->Wg)", "floor_mod(x + p->sw, p->Wg)"),
+    "shift sign on the column axis": ("floor_mod(x - p->sw, padded(p->Wg, p->ww, p->pad))",
+                                      "floor_mod(x + p->sw, padded(p->Wg, p->ww, p->pad))"),
     "dropped softmax scale": ("z[j++] = p->scale * s;", "z[j++] = s;"),
     "pooled sum not divided": ("xp[o] = acc * inv;", "xp[o] = acc;"),
     "log-sum-exp without the max": ("*lse_out = mx + log(den);", "*lse_out = log(den);"),
     "window members without the shift": (
-        "const int64_t xx = floor_mod(ix * p->ww + p->sw + lx, p->Wg);",
-        "const int64_t xx = floor_mod(ix * p->ww + lx, p->Wg);"),
+        "const int64_t xx = floor_mod(ix * p->ww + p->sw + lx, Wp);",
+        "const int64_t xx = floor_mod(ix * p->ww + lx, Wp);"),
     "no max subtraction": ("z[i] = exp(z[i] - mx);", "z[i] = exp(z[i]);"),
     "rows and columns swapped for keys": (
-        "const double* kv = k + kv_index(p, b, tt, yy, xx, kv_head(p, h));",
-        "const double* kv = k + kv_index(p, b, tt, xx % p->Hg, yy % p->Wg, kv_head(p, h));"),
+        "const double* kv = k + kv_index(p, b, tok[3 * a], tok[3 * a + 1], tok[3 * a + 2], kv_head(p, h));",
+        "const double* kv = k + kv_index(p, b, tok[3 * a], tok[3 * a + 2] % p->Hg, "
+        "tok[3 * a + 1] % p->Wg, kv_head(p, h));"),
+    "padded axis wrapped at the real grid size": (
+        "const int64_t yy = floor_mod(iy * p->wh + p->sh + ly, Hp);",
+        "const int64_t yy = floor_mod(iy * p->wh + p->sh + ly, p->Hg);"),
+    "query window id on the real grid size": (
+        "const int64_t iy = floor_mod(y - p->sh, padded(p->Hg, p->wh, p->pad)) / p->wh;",
+        "const int64_t iy = floor_mod(y - p->sh, p->Hg) / p->wh;"),
     "pooled cells on the shifted origin": (
         "acc += x[kv_index(p, b, ct * p->pt + i, cy * p->ph + j,\n"
         "                                       cx * p->pw + l, h) + c];",
@@ -75,6 +83,12 @@ def _pins():
     for shape, window, shift, L in pins.JOINT:
         yield pins.test_joint_matches_dense_mask_brute_force, {"shape": shape, "window": window,
                                                               "shift": shift, "L": L}
+    for shape, window, pool in pins.PADDED:
+        yield pins.test_padded_matches_brute_force_all_shifts, {"shape": shape, "window": window,
+                                                                "pool": pool}
+    yield pins.test_padded_backward_matches_autograd, {
+        "shape": (1, 1, 5, 7, 2, 8), "window": (1, 2, 3), "shift": (0, 1, 2), "pool": (0, 0, 0),
+        "L": 0}
 
 
 def _build_mutant(tmp_path, old, new):
