@@ -90,7 +90,18 @@ typedef enum basa_status {
 
 typedef enum basa_dtype { BASA_F32 = 0, BASA_BF16 = 1 } basa_dtype;
 
-/* Test-only flag bits for basa_params.flags. */
+/* Flag bits for basa_params.flags. */
+#define BASA_FLAG_PAD_GRID 0x4u            /* grids that a window size does not divide: each
+                                              axis is padded at its far end to the next
+                                              multiple of the window, the shift rolls the
+                                              padded axis (window of coordinate x:
+                                              floor(((x - s) mod Gp) / w)), and padded
+                                              positions are neither queries nor keys.  The
+                                              pages give no rule for such grids; this is the
+                                              usual shifted-window padding.  Without the flag
+                                              such a grid is BASA_ERR_SHAPE.  Pool cells must
+                                              still divide the grid.  The backward runs on
+                                              CUDA cores for padded grids. */
 #define BASA_FLAG_TEST_WITHHOLD_LOADS 0x1u /* the bf16 kernel's loader issues nothing,
                                               so its first wait runs out (tests the
                                               timeout path); output is not written */
@@ -106,7 +117,7 @@ typedef struct basa_params {
   int32_t pt, ph, pw;  /* pooled cell size per axis; all 0 = no global memory */
   float scale;         /* softmax scale on q.k; 0 selects 1/sqrt(d) */
   int32_t dtype;       /* basa_dtype of q, k, v, out and pooled tensors */
-  uint32_t flags;      /* 0, or BASA_FLAG_* test bits */
+  uint32_t flags;      /* 0, or BASA_FLAG_* bits */
   uint32_t wait_timeout_ms; /* bound on each device wait; 0 selects 2000 ms */
   int32_t Hkv;         /* K/V heads (grouped-query attention); 0 selects H.  H must be a
                           multiple of Hkv; query head h reads K/V head h / (H / Hkv).
@@ -306,8 +317,9 @@ BASA_API basa_status basa_test_exp2(const float* x, float* y, int64_t n, cudaStr
  * *n_windows = windows per (b, h) and *n_tiles = 128-row tiles per window.
  * If rows != NULL it receives [n_windows][n_tiles][128] int32 entries: the
  * flattened grid index (t * Hg + y) * Wg + x of the token that row r of the
- * tile holds in shared memory, or -1 for a padding row.  Only the grid, window
- * and shift fields and d/dtype of p are read; shapes outside the bf16 bounds
+ * tile holds in shared memory, or -1 for a padding row (past the tile's
+ * tokens, or a padded position with BASA_FLAG_PAD_GRID).  Only the grid,
+ * window, shift and flags fields and d/dtype of p are read; shapes outside the bf16 bounds
  * return BASA_ERR_UNSUPPORTED.  rows_capacity is the number of int32 entries
  * rows can hold.
  */

@@ -18,11 +18,12 @@ import torch
 
 from . import _lib
 from ._lib import BasaError, BasaParams, BASA_F32, BASA_BF16  # noqa: F401
+from ._lib import BASA_FLAG_PAD_GRID, BASA_FLAG_BWD_CUDA_CORES  # noqa: F401
 
 __all__ = ["window_attn", "window_attn_gm", "full_attn", "joint_attn", "window_attn_bwd",
            "joint_attn_bwd",
            "pool_kv", "workspace_size", "bwd_workspace_size", "joint_workspace_size", "get_status", "window_tiles", "make_params", "BasaError",
-           "library_path"]
+           "library_path", "BASA_FLAG_PAD_GRID", "BASA_FLAG_BWD_CUDA_CORES"]
 
 library_path = _lib.LIB_PATH
 
@@ -285,12 +286,12 @@ def get_status(stream=None) -> int:
     return int(_lib.load().basa_get_status(ctypes.c_void_p(s.cuda_stream)))
 
 
-def window_tiles(grid, window, shift=(0, 0, 0), d=128):
+def window_tiles(grid, window, shift=(0, 0, 0), d=128, flags=0):
     """Host-only tile plan of the bf16 kernel: int32 array [windows, tiles, 128] of
     flattened token indices per shared-memory row (-1 = padding)."""
     import numpy as np
     T, Hg, Wg = grid
-    prm = make_params((1, T, Hg, Wg, 1, d), BASA_BF16, window, shift)
+    prm = make_params((1, T, Hg, Wg, 1, d), BASA_BF16, window, shift, flags=flags)
     lib = _lib.load()
     nw, nt = ctypes.c_int32(), ctypes.c_int32()
     _lib.check(lib.basa_window_tiles(ctypes.byref(prm), ctypes.byref(nw), ctypes.byref(nt),

@@ -18,6 +18,8 @@ STATUS_NAMES = {
 }
 BASA_F32, BASA_BF16 = 0, 1
 BASA_FLAG_TEST_WITHHOLD_LOADS = 0x1
+BASA_FLAG_BWD_CUDA_CORES = 0x2
+BASA_FLAG_PAD_GRID = 0x4
 
 # Every symbol include/basa.h declares.
 EXPORTS = ("basa_status_string", "basa_version", "basa_workspace_size", "basa_pool_kv",

@@ -50,7 +50,9 @@ basa_status normalise(const basa_params* p, bool full, Dims* d) {
     d->pt = d->ph = d->pw = 0;
   } else {
     if (p->wt <= 0 || p->wh <= 0 || p->ww <= 0) return BASA_ERR_INVALID_ARG;
-    if (p->T % p->wt || p->Hg % p->wh || p->Wg % p->ww) return BASA_ERR_SHAPE;
+    const bool pad = (p->flags & BASA_FLAG_PAD_GRID) != 0;
+    if (!pad && (p->T % p->wt || p->Hg % p->wh || p->Wg % p->ww)) return BASA_ERR_SHAPE;
+    if (p->wt > (1 << 20) || p->wh > (1 << 20) || p->ww > (1 << 20)) return BASA_ERR_UNSUPPORTED;
     d->wt = p->wt; d->wh = p->wh; d->ww = p->ww;
     d->st = floor_mod(p->st, p->wt);
     d->sh = floor_mod(p->sh, p->wh);
@@ -63,7 +65,15 @@ basa_status normalise(const basa_params* p, bool full, Dims* d) {
       d->P = (long long)(p->T / p->pt) * (p->Hg / p->ph) * (p->Wg / p->pw);
     }
   }
-  d->nwt = d->T / d->wt; d->nwh = d->Hg / d->wh; d->nww = d->Wg / d->ww;
+  // windows per (padded) axis: ceil(G / w); the grid itself when w divides G
+  d->nwt = (d->T + d->wt - 1) / d->wt;
+  d->nwh = (d->Hg + d->wh - 1) / d->wh;
+  d->nww = (d->Wg + d->ww - 1) / d->ww;
+  d->Tp = d->nwt * d->wt; d->Hgp = d->nwh * d->wh; d->Wgp = d->nww * d->ww;
+  d->padded = (d->Tp != d->T || d->Hgp != d->Hg || d->Wgp != d->Wg) ? 1 : 0;
+  if ((long long)d->Tp * d->Hgp * d->Wgp > (1LL << 30) ||
+      (long long)d->nwt * d->nwh * d->nww > (1LL << 30))
+    return BASA_ERR_UNSUPPORTED;
   return BASA_OK;
 }
 
@@ -475,13 +485,15 @@ basa_status basa_window_tiles(const basa_params* p, int32_t* n_windows, int32_t*
         const uint32_t e = plan.box[cls][ti][bi];
         const int sid = box_shape(e);
         const int bt = plan.shape_bt[sid], bh = plan.shape_bh[sid], bw = plan.shape_bw[sid];
-        const int gt = (ot + box_lt(e)) % d.T, gh = (oh + box_lh(e)) % d.Hg,
-                  gw = (ow + box_lw(e)) % d.Wg;
+        const int gt = (ot + box_lt(e)) % d.Tp, gh = (oh + box_lh(e)) % d.Hgp,
+                  gw = (ow + box_lw(e)) % d.Wgp;
         int row = box_row8(e) * 8;
         for (int a = 0; a < bt; ++a)
           for (int b = 0; b < bh; ++b)
-            for (int c = 0; c < bw; ++c)
-              r[row++] = (int32_t)(((long long)(gt + a) * d.Hg + (gh + b)) * d.Wg + (gw + c));
+            for (int c = 0; c < bw; ++c, ++row) {
+              if (gt + a >= d.T || gh + b >= d.Hg || gw + c >= d.Wg) continue;  // padded
+              r[row] = (int32_t)(((long long)(gt + a) * d.Hg + (gh + b)) * d.Wg + (gw + c));
+            }
       }
     }
   }

@@ -44,7 +44,8 @@ struct BwdArgs {
   void* dv;
   int B, H, Hkv, T, Hg, Wg;
   int wt, wh, ww, st, sh, sw, nwt, nwh, nww;
-  int m;            // tokens per window
+  int Tp, Hgp, Wgp; // padded extents the windows wrap on (T, Hg, Wg unless padded)
+  int m;            // window positions (tokens plus padding)
   int n_chunks;     // query (or key) chunks per window
   long long N;
   float scale;
@@ -84,13 +85,15 @@ __device__ __forceinline__ void st1(void* base, long long i, float x) {
     reinterpret_cast<float*>(base)[i] = x;
 }
 
-// Flattened grid token of member j of window (jt, jh, jw).
+// Flattened grid token of member j of window (jt, jh, jw), or -1 when the
+// position is padding (past T, Hg or Wg on the padded axes).
 __device__ __forceinline__ long long member(const BwdArgs& a, int jt, int jh, int jw, int j) {
   const int lt = j / (a.wh * a.ww), lh = (j / a.ww) % a.wh, lw = j % a.ww;
   int t = jt * a.wt + a.st + lt, y = jh * a.wh + a.sh + lh, x = jw * a.ww + a.sw + lw;
-  t = t >= a.T ? t - a.T : t;
-  y = y >= a.Hg ? y - a.Hg : y;
-  x = x >= a.Wg ? x - a.Wg : x;
+  t = t >= a.Tp ? t - a.Tp : t;
+  y = y >= a.Hgp ? y - a.Hgp : y;
+  x = x >= a.Wgp ? x - a.Wgp : x;
+  if (t >= a.T || y >= a.Hg || x >= a.Wg) return -1;
   return ((long long)t * a.Hg + y) * a.Wg + x;
 }
 
@@ -152,6 +155,7 @@ __global__ void __launch_bounds__(kBwdThreads) bwd_dq_kernel(BwdArgs a) {
   constexpr int QPC = kBwdThreads / TPQ;
   __shared__ float ks[kChunk][D];
   __shared__ float vs[kChunk][D];
+  __shared__ int kok[kChunk];  // key jj of the chunk is a token (not padding)
   long long u = blockIdx.x;
   const int qc = (int)(u % (TEXTQ ? a.t_chunks : a.n_chunks));
   u /= (TEXTQ ? a.t_chunks : a.n_chunks);
@@ -164,12 +168,13 @@ __global__ void __launch_bounds__(kBwdThreads) bwd_dq_kernel(BwdArgs a) {
   const int jw = win % a.nww, jh = (win / a.nww) % a.nwh, jt = win / (a.nww * a.nwh);
   const int part = threadIdx.x % TPQ;
   const long long lq = (long long)qc * QPC + threadIdx.x / TPQ;
-  const bool valid = lq < (TEXTQ ? (long long)a.P : (long long)a.m);
+  const long long n = lq < (TEXTQ ? (long long)a.P : (long long)a.m)
+                          ? (TEXTQ ? lq : member(a, jt, jh, jw, (int)lq)) : -1;
+  const bool valid = n >= 0;  // padding and rows past the window are no query
   float qr[DPT], gr[DPT], acc[DPT];
   float lse = 0.f, dd = 0.f;
   long long qrow = 0;
   if (valid) {
-    const long long n = TEXTQ ? lq : member(a, jt, jh, jw, (int)lq);
     const long long nrows = TEXTQ ? (long long)a.P : a.N;
     qrow = (((long long)b * nrows + n) * a.H + h) * D + part * DPT;
     for (int c = 0; c < DPT; ++c) {
@@ -192,11 +197,17 @@ __global__ void __launch_bounds__(kBwdThreads) bwd_dq_kernel(BwdArgs a) {
       const int jj = idx / D, c = idx % D;
       const long long j = k0 + jj;
       if (j < nbase) {
-        const long long n = TEXTQ ? j : member(a, jt, jh, jw, (int)j);
-        const long long off = (((long long)b * a.N + n) * a.Hkv + hk) * D + c;
+        const long long kn = TEXTQ ? j : member(a, jt, jh, jw, (int)j);
+        if (c == 0) kok[jj] = kn >= 0;
+        if (kn < 0) {  // padding: no key
+          ks[jj][c] = vs[jj][c] = 0.f;
+          continue;
+        }
+        const long long off = (((long long)b * a.N + kn) * a.Hkv + hk) * D + c;
         ks[jj][c] = ld1<BF16>(a.k, off);
         vs[jj][c] = ld1<BF16>(a.v, off);
       } else {
+        if (c == 0) kok[jj] = 1;
         const long long off = (((long long)b * a.P + (j - nbase)) * a.Hkv + hk) * D + c;
         ks[jj][c] = ld1<BF16>(a.kp, off);
         vs[jj][c] = ld1<BF16>(a.vp, off);
@@ -211,7 +222,7 @@ __global__ void __launch_bounds__(kBwdThreads) bwd_dq_kernel(BwdArgs a) {
       }
       s = lane_sum<TPQ>(s);
       dp = lane_sum<TPQ>(dp);
-      const float pw = expf(s * a.scale - lse);
+      const float pw = kok[jj] ? expf(s * a.scale - lse) : 0.f;
       const float ds = pw * (dp - dd);
       for (int c = 0; c < DPT; ++c) acc[c] = fmaf(ds, ks[jj][part * DPT + c], acc[c]);
     }
@@ -245,14 +256,14 @@ __global__ void __launch_bounds__(kBwdThreads) bwd_dkv_kernel(BwdArgs a) {
   const int jw = win % a.nww, jh = (win / a.nww) % a.nwh, jt = win / (a.nww * a.nwh);
   const int part = threadIdx.x % TPQ;
   const long long lk = (long long)kc * KPC + threadIdx.x / TPQ;
-  const bool valid = lk < (POOL ? a.P : a.m);
+  const long long n_row = (!POOL && lk < a.m) ? member(a, jt, jh, jw, (int)lk) : 0;
+  const bool valid = lk < (POOL ? a.P : a.m) && n_row >= 0;  // padding is no key
   float kr[DPT], vr[DPT], dk[DPT], dv[DPT];
-  long long krow = 0, n_row = 0;
+  long long krow = 0;
   if (valid) {
     if (POOL) {
       krow = (((long long)b * a.P + lk) * a.Hkv + hk) * D + part * DPT;
     } else {
-      n_row = member(a, jt, jh, jw, (int)lk);
       krow = (((long long)b * a.N + n_row) * a.Hkv + hk) * D + part * DPT;
     }
     for (int c = 0; c < DPT; ++c) {
@@ -285,6 +296,14 @@ __global__ void __launch_bounds__(kBwdThreads) bwd_dkv_kernel(BwdArgs a) {
           continue;
         }
         const long long n = POOL ? q0 + ii : member(a, jt, jh, jw, (int)(q0 + ii));
+        if (n < 0) {  // padding: no query (weight exp(s - inf) = 0)
+          qs[ii][c] = gs[ii][c] = 0.f;
+          if (c == 0) {
+            ls[ii] = INFINITY;
+            ds_[ii] = 0.f;
+          }
+          continue;
+        }
         const long long off = (((long long)b * a.N + n) * a.H + h) * D + c;
         qs[ii][c] = ld1<BF16>(a.q, off);
         gs[ii][c] = ld1<BF16>(a.dout, off);
@@ -418,6 +437,9 @@ basa_status launch_bwd_common(const Dims& d, const void* q, const void* k, const
   a.wt = d.wt; a.wh = d.wh; a.ww = d.ww;
   a.st = d.st; a.sh = d.sh; a.sw = d.sw;
   a.nwt = d.nwt; a.nwh = d.nwh; a.nww = d.nww;
+  a.Tp = d.Tp > 0 ? d.Tp : d.T;
+  a.Hgp = d.Hgp > 0 ? d.Hgp : d.Hg;
+  a.Wgp = d.Wgp > 0 ? d.Wgp : d.Wg;
   const long long m = (long long)d.wt * d.wh * d.ww;
   if (m > (1LL << 30)) return BASA_ERR_UNSUPPORTED;
   a.m = (int)m;

@@ -18,7 +18,9 @@ struct Dims {
   int wt, wh, ww;     // window
   int st, sh, sw;     // shift reduced to [0, w)
   int pt, ph, pw;     // pool cell; 0 = none
-  int nwt, nwh, nww;  // windows per axis
+  int nwt, nwh, nww;  // windows per axis (of the padded axes)
+  int Tp, Hgp, Wgp;   // padded extents: nw * w (the grid itself unless it is padded)
+  int padded;         // 1: some axis is padded (BASA_FLAG_PAD_GRID and w does not divide G)
   long long N;        // tokens per (b, h)
   long long P;        // extra (pooled or text) key tokens per (b, h); 0 = none
   long long Nq;       // query tokens per (b, h): N, or the text length for text queries

@@ -33,7 +33,9 @@ struct SimtArgs {
   int Hkv;          // K/V heads; query head h reads K/V head h / (H / Hkv)
   int wt, wh, ww, st, sh, sw;
   int nwt, nwh, nww;
-  int m;            // tokens per window
+  int Tp, Hgp, Wgp; // padded extents the windows wrap on (T, Hg, Wg unless padded);
+                    // members at coordinates past T, Hg or Wg are padding: no token
+  int m;            // window positions (tokens plus padding)
   int P;            // pooled tokens (0 = none)
   int n_qchunks;    // query chunks per window
   long long N;
@@ -54,6 +56,7 @@ __global__ void __launch_bounds__(kThreads) simt_window_kernel(SimtArgs a) {
   constexpr int V4 = D / 4;            // float4 per row
   __shared__ float4 ks[kKeyChunk][V4];
   __shared__ float4 vs[kKeyChunk][V4];
+  __shared__ int kok[kKeyChunk];  // key jj of the chunk is a token (not padding)
 
   long long u = blockIdx.x;
   const int qc = (int)(u % a.n_qchunks);
@@ -69,7 +72,7 @@ __global__ void __launch_bounds__(kThreads) simt_window_kernel(SimtArgs a) {
 
   const int part = threadIdx.x % TPQ;
   const int lq = qc * QPC + threadIdx.x / TPQ;
-  const bool valid = a.qsep ? lq < a.Nq : lq < a.m;
+  bool valid = a.qsep ? lq < a.Nq : lq < a.m;
   long long qrow = 0;
   long long qn = 0;
   float qr[DPT];
@@ -81,12 +84,13 @@ __global__ void __launch_bounds__(kThreads) simt_window_kernel(SimtArgs a) {
     for (int c = 0; c < DPT; ++c) qr[c] = qp[c];
   } else if (valid) {
     const int lt = lq / (a.wh * a.ww), lh = (lq / a.ww) % a.wh, lw = lq % a.ww;
-    const int t = (ot + lt) % a.T, y = (oh + lh) % a.Hg, x = (ow + lw) % a.Wg;
-    qn = ((long long)t * a.Hg + y) * a.Wg + x;
-    qrow = token_row(a, b, t, y, x);
+    const int t = (ot + lt) % a.Tp, y = (oh + lh) % a.Hgp, x = (ow + lw) % a.Wgp;
+    valid = t < a.T && y < a.Hg && x < a.Wg;  // a padded position is no query
+    qn = valid ? ((long long)t * a.Hg + y) * a.Wg + x : 0;
+    qrow = valid ? token_row(a, b, t, y, x) : 0;
     const float* qp = a.q + (qrow * a.H + h) * D + part * DPT;
 #pragma unroll
-    for (int c = 0; c < DPT; ++c) qr[c] = qp[c];
+    for (int c = 0; c < DPT; ++c) qr[c] = valid ? qp[c] : 0.f;
   } else {
 #pragma unroll
     for (int c = 0; c < DPT; ++c) qr[c] = 0.f;
@@ -108,11 +112,19 @@ __global__ void __launch_bounds__(kThreads) simt_window_kernel(SimtArgs a) {
       const float4* vr;
       if (j < a.m) {
         const int lt = j / (a.wh * a.ww), lh = (j / a.ww) % a.wh, lw = j % a.ww;
-        const long long row =
-            token_row(a, b, (ot + lt) % a.T, (oh + lh) % a.Hg, (ow + lw) % a.Wg);
+        const int t = (ot + lt) % a.Tp, y = (oh + lh) % a.Hgp, x = (ow + lw) % a.Wgp;
+        const bool tok = t < a.T && y < a.Hg && x < a.Wg;
+        if (c4 == 0) kok[jj] = tok ? 1 : 0;
+        if (!tok) {  // padding: no key
+          ks[jj][c4] = make_float4(0.f, 0.f, 0.f, 0.f);
+          vs[jj][c4] = make_float4(0.f, 0.f, 0.f, 0.f);
+          continue;
+        }
+        const long long row = token_row(a, b, t, y, x);
         kr = reinterpret_cast<const float4*>(a.k + (row * a.Hkv + hk) * D);
         vr = reinterpret_cast<const float4*>(a.v + (row * a.Hkv + hk) * D);
       } else {
+        if (c4 == 0) kok[jj] = 1;
         const long long prow = (long long)b * a.P + (j - a.m);
         kr = reinterpret_cast<const float4*>(a.kp + (prow * a.Hkv + hk) * D);
         vr = reinterpret_cast<const float4*>(a.vp + (prow * a.Hkv + hk) * D);
@@ -130,17 +142,18 @@ __global__ void __launch_bounds__(kThreads) simt_window_kernel(SimtArgs a) {
 #pragma unroll
       for (int c = 0; c < DPT; ++c) dot = fmaf(qr[c], kr[c], dot);
       if (TPQ == 2) dot += __shfl_xor_sync(0xffffffffu, dot, 1);
-      s[jj] = jj < nk ? dot * a.scale : -INFINITY;
+      s[jj] = (jj < nk && kok[jj]) ? dot * a.scale : -INFINITY;
       cmax = fmaxf(cmax, s[jj]);
     }
     const float mnew = fmaxf(mrun, cmax);
+    if (mnew == -INFINITY) continue;  // every key so far is padding (same for every query)
     const float corr = expf(mrun - mnew);  // 0 on the first chunk
     l *= corr;
 #pragma unroll
     for (int c = 0; c < DPT; ++c) acc[c] *= corr;
 #pragma unroll
     for (int jj = 0; jj < kKeyChunk; ++jj) {
-      if (jj < nk) {
+      if (jj < nk && kok[jj]) {
         const float p = expf(s[jj] - mnew);
         l += p;
         const float* vr = reinterpret_cast<const float*>(&vs[jj][0]) + part * DPT;
@@ -181,6 +194,9 @@ basa_status launch_simt(const Dims& d, const void* q, const void* k, const void*
   a.wt = d.wt; a.wh = d.wh; a.ww = d.ww;
   a.st = d.st; a.sh = d.sh; a.sw = d.sw;
   a.nwt = d.nwt; a.nwh = d.nwh; a.nww = d.nww;
+  a.Tp = d.Tp > 0 ? d.Tp : d.T;
+  a.Hgp = d.Hgp > 0 ? d.Hgp : d.Hg;
+  a.Wgp = d.Wgp > 0 ? d.Wgp : d.Wg;
   const long long m = (long long)d.wt * d.wh * d.ww;
   if (m > (1LL << 30)) return BASA_ERR_UNSUPPORTED;
   a.m = (int)m;

@@ -79,6 +79,8 @@ struct __align__(64) TcParams {
   int B, H, T, Hg, Wg;
   int group;  // query heads per K/V head
   int wt, wh, ww, st, sh, sw, nwt, nwh, nww;
+  int Tp, Hgp, Wgp;  // padded extents the window origins wrap on (T, Hg, Wg unless padded)
+  int padded;        // 1: padded positions exist and are masked
   int n_windows;
   int n_shapes;
   int n_qt;   // query tiles per window (flat: per (b, h))
@@ -126,6 +128,7 @@ enum WaitSite : uint32_t {
 struct Unit {
   int b, h, hk, pair, cls, ot, oh, ow, nq;  // hk: the K/V head of query head h
   int split, j0, nk;                        // key tiles [j0, j0 + nk)
+  int holes;                                // the window holds padded positions
 };
 
 // Window mode walks the heads fastest: concurrently running CTAs then read the
@@ -150,6 +153,7 @@ __device__ __forceinline__ Unit decode_unit(const TcParams& p, uint32_t u) {
     U.b = (int)(r / (uint32_t)p.H);
     U.cls = 0;
     U.ot = U.oh = U.ow = 0;
+    U.holes = 0;
   } else {
     U.h = (int)(u % (uint32_t)p.H);
     uint32_t r = u / (uint32_t)p.H;
@@ -162,6 +166,11 @@ __device__ __forceinline__ Unit decode_unit(const TcParams& p, uint32_t u) {
     U.ot = jt * p.wt + p.st;
     U.oh = jh * p.wh + p.sh;
     U.ow = jw * p.ww + p.sw;
+    // An axis's window [o, o + w) on the padded axis (o < Gp, wrapping at Gp)
+    // meets the padding [G, Gp) exactly when Gp > G and o + w > G.
+    U.holes = p.padded && ((p.Tp > p.T && U.ot + p.wt > p.T) ||
+                           (p.Hgp > p.Hg && U.oh + p.wh > p.Hg) ||
+                           (p.Wgp > p.Wg && U.ow + p.ww > p.Wg));
   }
   const int left = p.n_qt - 2 * U.pair;
   U.nq = left < 2 ? left : 2;
@@ -213,11 +222,12 @@ __device__ __forceinline__ void load_tile(const TcParams& p, const PlanView& pv,
   }
   const CUtensorMap* maps = kind == 0 ? p.qm : kind == 1 ? p.km : p.vm;
   load_window_tile<NH>(pv, maps, &p.fill, WinAt{U.cls, U.ot, U.oh, U.ow, U.b}, tile, head, p.T,
-                       p.Hg, p.Wg, p.N, dst, bar);
+                       p.Tp, p.Hgp, p.Wgp, p.N, dst, bar);
 }
 
 // Stores d-half hf of query tile qt from a 128-row x 64-column staging block
-// (128-byte swizzled) with TMA boxes that mirror the load boxes.
+// (128-byte swizzled) with TMA boxes that mirror the load boxes.  Never used on
+// a padded grid (its calls take the warp-staged stores, which skip padded rows).
 template <int D>
 __device__ __forceinline__ void store_half(const TcParams& p, const PlanView& pv, const Unit& U,
                                            int qt, int hf, uint32_t src) {
@@ -249,7 +259,8 @@ __device__ __forceinline__ void store_half(const TcParams& p, const PlanView& pv
 __device__ __forceinline__ long long row_token(const TcParams& p, const PlanView& pv,
                                                const Unit& U, int qt, int r) {
   if (p.flat) return 128LL * qt + r;
-  return window_row_token(pv, WinAt{U.cls, U.ot, U.oh, U.ow, U.b}, qt, r, p.T, p.Hg, p.Wg);
+  return window_row_token(pv, WinAt{U.cls, U.ot, U.oh, U.ow, U.b}, qt, r, p.Tp, p.Hgp, p.Wgp,
+                          p.T, p.Hg, p.Wg);
 }
 
 // Shared-memory plan: the unit's two 128-row query tiles, one 64-column output
@@ -544,6 +555,17 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attn_kernel(const __grid_const
             for (int e = 0; e < 32; ++e)
               if (cc * 32 + e >= kvalid) s[cc][e] = __float_as_uint(-INFINITY);
         }
+        if (U.holes && j < p.n_wkt) {  // keys at padded positions of this window
+          uint32_t okw[4];
+#pragma unroll
+          for (int cc = 0; cc < 4; ++cc)
+            okw[cc] = __ballot_sync(0xffffffffu, row_token(p, pv, U, j, cc * 32 + lane) >= 0);
+#pragma unroll
+          for (int cc = 0; cc < 4; ++cc)
+#pragma unroll
+            for (int e = 0; e < 32; ++e)
+              if (!((okw[cc] >> e) & 1u)) s[cc][e] = __float_as_uint(-INFINITY);
+        }
         float mx0 = -INFINITY, mx1 = -INFINITY;
 #pragma unroll
         for (int cc = 0; cc < 4; ++cc)
@@ -559,7 +581,9 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attn_kernel(const __grid_const
           m = mtile;
         }
         const uint64_t c2 = f2pack(c, c);
-        const uint64_t nm2 = f2pack(-m, -m);
+        // every key so far masked (a tile of padded positions): P = 0, not NaN
+        const float mneg = m == -INFINITY ? 0.f : -m;
+        const uint64_t nm2 = f2pack(mneg, mneg);
         uint64_t rsa = f2pack(0.f, 0.f), rsb = rsa;
 #pragma unroll
         for (int cc = 0; cc < 4; ++cc) {
@@ -775,6 +799,10 @@ basa_status build_and_launch(TcParams* prm, const Dims& d, bool flat, const void
   prm->wt = d.wt; prm->wh = d.wh; prm->ww = d.ww;
   prm->st = d.st; prm->sh = d.sh; prm->sw = d.sw;
   prm->nwt = d.nwt; prm->nwh = d.nwh; prm->nww = d.nww;
+  prm->Tp = flat ? d.T : d.Tp;
+  prm->Hgp = flat ? d.Hg : d.Hgp;
+  prm->Wgp = flat ? d.Wg : d.Wgp;
+  prm->padded = flat ? 0 : d.padded;
   prm->N = d.N;
   prm->Nq = d.Nq;
   prm->lse = lse;
@@ -865,7 +893,8 @@ basa_status build_and_launch(TcParams* prm, const Dims& d, bool flat, const void
   }
   // Output path: warp-staged stores, except for windows of more than two key
   // tiles, where the TMA store boxes measured faster.
-  prm->warp_stores = (flat || prm->n_wkt <= 2) ? 1 : 0;
+  // A padded grid always takes the warp-staged stores (they skip padded rows).
+  prm->warp_stores = (flat || prm->n_wkt <= 2 || prm->padded) ? 1 : 0;
   // K/V ring depth: windows of at most two key tiles and no extra keys stream
   // each K/V tile once per unit and ran faster with 3 slots in flight than with
   // 4; everything else reuses K/V tiles from L2 and runs faster with 4.

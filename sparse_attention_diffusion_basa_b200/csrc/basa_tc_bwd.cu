@@ -858,7 +858,8 @@ basa_status launch_bwd_tc(const Dims& d, const void* q, const void* k, const voi
                           const void* out, const void* dout, const float* lse, float* dD,
                           void* dq, void* dk, void* dv, const PoolGrads* pg, uint32_t timeout_ms,
                           cudaStream_t stream) {
-  if (d.dtype != BASA_BF16 || (d.d != 64 && d.d != 128) || d.qsep || (d.P && !pg))
+  // padded grids: the CUDA-core kernels (these kernels do not mask padded rows)
+  if (d.dtype != BASA_BF16 || (d.d != 64 && d.d != 128) || d.qsep || (d.P && !pg) || d.padded)
     return BASA_ERR_UNSUPPORTED;
   TilePlan plan;
   basa_status st = build_tile_plan(d, &plan);  // before any launch

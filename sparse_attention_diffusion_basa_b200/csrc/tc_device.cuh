@@ -458,24 +458,29 @@ struct WinAt {
 // Loads tile `tile` of window w for one head: each box of the plan through
 // maps[box shape] (rank 5: [d, heads, Wg, Hg, B*T]; NH head-dim halves of 64),
 // then the rows past the tile's tokens as zeros, read out of bounds through
-// `fill` (8-row boxes).  Signals bar with the transaction bytes.
+// `fill` (8-row boxes).  Signals bar with the transaction bytes.  Tp, Hgp, Wgp
+// are the padded extents the window origins wrap on (the grid's own unless it
+// is padded); rows at padded positions read zeros (rows, columns: out of the
+// map's bounds) or another frame (t: the map merges B and T) and are masked by
+// the caller.
 template <int NH>
 __device__ __forceinline__ void load_window_tile(const PlanView& pv, const CUtensorMap* maps,
                                                  const CUtensorMap* fill, const WinAt& w,
-                                                 int tile, int head, int T, int Hg, int Wg,
-                                                 long long N, uint32_t dst, uint32_t bar) {
+                                                 int tile, int head, int T, int Tp, int Hgp,
+                                                 int Wgp, long long N, uint32_t dst,
+                                                 uint32_t bar) {
   const int b0 = pv.first(w.cls, tile), nb = pv.count(w.cls, tile);
 #pragma unroll 1
   for (int bi = 0; bi < nb; ++bi) {
     const uint32_t e = pv.entries[b0 + bi];
     const int sid = box_shape(e);
-    const int gt = wrap(w.ot + box_lt(e), T);
-    const int gh = wrap(w.oh + box_lh(e), Hg);
-    const int gw = wrap(w.ow + box_lw(e), Wg);
-    if constexpr (kChecked) {  // the box lies inside the grid and inside the 128-row tile
+    const int gt = wrap(w.ot + box_lt(e), Tp);
+    const int gh = wrap(w.oh + box_lh(e), Hgp);
+    const int gw = wrap(w.ow + box_lw(e), Wgp);
+    if constexpr (kChecked) {  // the box lies inside the padded grid and the 128-row tile
       const int bt = pv.bt[sid], bh = pv.bh[sid], bw = pv.bw[sid];
-      if (sid >= kMaxShapes || gt < 0 || gh < 0 || gw < 0 || gt + bt > T || gh + bh > Hg ||
-          gw + bw > Wg || box_row8(e) * 8 + bt * bh * bw > 128) {
+      if (sid >= kMaxShapes || gt < 0 || gh < 0 || gw < 0 || gt + bt > Tp || gh + bh > Hgp ||
+          gw + bw > Wgp || box_row8(e) * 8 + bt * bh * bw > 128) {
         check_failed(kCheckLoadBox);
         continue;
       }
@@ -492,11 +497,20 @@ __device__ __forceinline__ void load_window_tile(const PlanView& pv, const CUten
       tma_load_4d(dst + hf * kHalf + r * 128, fill, bar, hf * 64, 0, (int)N, 0);
   }
 }
+template <int NH>
+__device__ __forceinline__ void load_window_tile(const PlanView& pv, const CUtensorMap* maps,
+                                                 const CUtensorMap* fill, const WinAt& w,
+                                                 int tile, int head, int T, int Hg, int Wg,
+                                                 long long N, uint32_t dst, uint32_t bar) {
+  load_window_tile<NH>(pv, maps, fill, w, tile, head, T, T, Hg, Wg, N, dst, bar);
+}
 
 // Flattened grid index of the token in row r of tile `tile` of window w, or -1
-// for a padding row.
+// for a row past the tile's tokens or at a padded position (a coordinate at or
+// past the grid's extent T, Hg, Wg; origins wrap on the padded Tp, Hgp, Wgp).
 __device__ __forceinline__ long long window_row_token(const PlanView& pv, const WinAt& w,
-                                                      int tile, int r, int T, int Hg, int Wg) {
+                                                      int tile, int r, int Tp, int Hgp, int Wgp,
+                                                      int T, int Hg, int Wg) {
   const int b0 = pv.first(w.cls, tile), nb = pv.count(w.cls, tile);
 #pragma unroll 1
   for (int bi = 0; bi < nb; ++bi) {
@@ -507,13 +521,18 @@ __device__ __forceinline__ long long window_row_token(const PlanView& pv, const 
     if (r >= r0 && r < r0 + bt * bh * bw) {
       const int idx = r - r0;
       const int it = idx / (bh * bw), ih = (idx / bw) % bh, iw = idx % bw;
-      const int gt = wrap(w.ot + box_lt(e), T) + it;
-      const int gh = wrap(w.oh + box_lh(e), Hg) + ih;
-      const int gw = wrap(w.ow + box_lw(e), Wg) + iw;
+      const int gt = wrap(w.ot + box_lt(e), Tp) + it;
+      const int gh = wrap(w.oh + box_lh(e), Hgp) + ih;
+      const int gw = wrap(w.ow + box_lw(e), Wgp) + iw;
+      if (gt >= T || gh >= Hg || gw >= Wg) return -1;
       return ((long long)gt * Hg + gh) * Wg + gw;
     }
   }
   return -1;
+}
+__device__ __forceinline__ long long window_row_token(const PlanView& pv, const WinAt& w,
+                                                      int tile, int r, int T, int Hg, int Wg) {
+  return window_row_token(pv, w, tile, r, T, Hg, Wg, T, Hg, Wg);
 }
 
 // SMs of the current device (the persistent grids launch one CTA per SM).

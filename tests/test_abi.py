@@ -150,6 +150,39 @@ def test_tile_plan_covers_each_shifted_window_once(lib, grid, window, shifts):
         assert seen == set(range(grid[0] * grid[1] * grid[2]))
 
 
+PADDED_PLAN_CASES = [  # grids the window does not divide (BASA_FLAG_PAD_GRID)
+    ((1, 48, 85), (1, 16, 16), [(0, 0, 0), (0, 8, 8), (0, 8, 0)]),
+    ((1, 5, 7), (1, 16, 16), [(0, 0, 0), (0, 8, 8)]),
+    ((13, 18, 32), (7, 9, 16), [(3, 4, 8), (0, 0, 0)]),
+    ((5, 10, 16), (3, 5, 8), [(1, 2, 0)]),
+]
+
+
+@pytest.mark.parametrize("grid,window,shifts", PADDED_PLAN_CASES)
+def test_padded_tile_plan_holds_each_padded_window(lib, grid, window, shifts):
+    """Each window's tiles hold exactly the real tokens that share its window ids
+    on the padded axes (ids from the brute-force module's reading: padding at the
+    far end, the shift rolling the padded axis); every token appears once."""
+    from oracle import window_ids
+    from sparse_attention_diffusion_basa_b200 import window_tiles, BASA_FLAG_PAD_GRID
+    T, Hg, Wg = grid
+    for shift in shifts:
+        rows = window_tiles(grid, window, shift, flags=BASA_FLAG_PAD_GRID)
+        ids = [window_ids(G, w, s, pad=True) for G, w, s in zip(grid, window, shift)]
+        wid = np.stack(np.meshgrid(*ids, indexing="ij"), axis=-1).reshape(-1, 3)
+        groups = {}
+        for n, key in enumerate(map(tuple, wid)):
+            groups.setdefault(key, set()).add(n)
+        assert rows.shape[0] == np.prod([-(-G // w) for G, w in zip(grid, window)])
+        seen = []
+        for w in range(rows.shape[0]):
+            toks = rows[w][rows[w] >= 0].tolist()
+            assert len(set(toks)) == len(toks) > 0
+            assert set(toks) in groups.values(), (shift, w)
+            seen += toks
+        assert sorted(seen) == list(range(T * Hg * Wg))
+
+
 def test_tile_plan_counts(lib):
     from sparse_attention_diffusion_basa_b200 import window_tiles
     assert window_tiles((1, 128, 128), (1, 16, 16), (0, 8, 8)).shape == (64, 2, 128)
