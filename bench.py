@@ -240,23 +240,33 @@ def cpu_baseline(w, shift, q, k, v, budget_s=12.0):
 
 
 def main_backward(args, world, rank, local):
-    """Backward of the workload's window attention: dq, dk, dv for a random dout."""
+    """Backward of the workload's window attention: dq, dk, dv for a random dout
+    (joint workloads: also dqt, dkt, dvt for a random dout_t)."""
     import sparse_attention_diffusion_basa_b200 as basa
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     w = WORKLOADS[args.workload]
-    if w.text:
-        raise SystemExit("the backward takes no text tokens")
     shift = w.shifts[-1]
     q, k, v = workload_inputs(w, len(w.shifts) - 1)
     dq, dk, dv = (x.to(dev) for x in (q, k, v))
     g = torch.randn(dq.shape, generator=torch.Generator().manual_seed(7)).to(dq.dtype).to(dev)
-    out, lse = basa.window_attn(dq, dk, dv, w.window, shift, w.pool, return_lse=True)
-    ws = torch.empty(max(basa.bwd_workspace_size(w.shape(), dq.dtype, w.window, shift, w.pool), 1),
-                     dtype=torch.uint8, device=dev)
     flush = L2Flush(dev)
-    step = lambda: basa.window_attn_bwd(dq, dk, dv, out, g, lse, w.window, shift, w.pool,
-                                        workspace=ws)
+    L = w.text
+    if L:
+        qt, kt, vt = (x.to(dev) for x in text_inputs(w, len(w.shifts) - 1))
+        gt = torch.randn(qt.shape, generator=torch.Generator().manual_seed(8)).to(qt.dtype).to(dev)
+        out, out_t, lse, lse_t = basa.joint_attn(dq, dk, dv, qt, kt, vt, w.window, shift,
+                                                 return_lse=True)
+        need = basa.joint_bwd_workspace_size(w.shape(), dq.dtype, w.window, shift, L)
+        ws = torch.empty(max(need, 1), dtype=torch.uint8, device=dev)
+        step = lambda: basa.joint_attn_bwd(dq, dk, dv, qt, kt, vt, out, out_t, g, gt, lse, lse_t,
+                                           w.window, shift, workspace=ws)
+    else:
+        out, lse = basa.window_attn(dq, dk, dv, w.window, shift, w.pool, return_lse=True)
+        ws = torch.empty(max(basa.bwd_workspace_size(w.shape(), dq.dtype, w.window, shift,
+                                                     w.pool), 1), dtype=torch.uint8, device=dev)
+        step = lambda: basa.window_attn_bwd(dq, dk, dv, out, g, lse, w.window, shift, w.pool,
+                                            workspace=ws)
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
@@ -272,14 +282,15 @@ def main_backward(args, world, rank, local):
     B, T, Hg, Wg, H, d = w.shape()
     Hkv = H
     # five contractions per query and key: S (recomputed), dP, dV, dQ, dK (the
-    # forward has two); keys = the window's m plus the P pooled tokens
-    flops = 10.0 * B * H * w.N * (w.m + w.P) * d
+    # forward has two); keys = the window's m plus the P pooled tokens (joint:
+    # image queries see m + L keys, text queries N + L)
+    flops = 10.0 * B * H * (w.N * (w.m + w.P + L) + L * (w.N + L)) * d
     # q, k, v, out, dout read once; dq, dk, dv written once; per query row the
     # lse read and D = rowsum(dout * out) written and read once (12 B); with
     # pooled memory the pooled K, V (bf16) and their fp32 gradients written and
-    # read once
-    nbytes = 2.0 * B * w.N * d * ((3 * H + 2 * Hkv) + (H + 2 * Hkv)) + 12.0 * B * H * w.N \
-        + 2.0 * B * w.P * Hkv * d * (2 * 2 + 2 * 4)
+    # read once; text tokens count as image tokens do
+    nbytes = 2.0 * B * (w.N + L) * d * ((3 * H + 2 * Hkv) + (H + 2 * Hkv)) \
+        + 12.0 * B * H * (w.N + L) + 2.0 * B * w.P * Hkv * d * (2 * 2 + 2 * 4)
     tflops = flops / (ms * 1e-3) / 1e12
     gbs = nbytes / (ms * 1e-3) / 1e9
     peaks = _peaks()
@@ -293,17 +304,21 @@ def main_backward(args, world, rank, local):
                 "frac": gbs / peaks["hbm_gbs"]}
     roof.update({"peak_source": peaks["source"] + " (MEASURED_PEAKS.json, burst)",
                  "traffic": None, "roofline_ms": 1e3 * max(t_tensor, t_hbm),
-                 "kernel": "whole backward: bwd_prep, tc_bwd_kernel (dQ), tc_bwd_kernel (dK, dV)"
-                           + (", pool_kernel, tc_bwd_kernel (pooled dK, dV)" if w.P else "")})
+                 "kernel": ("whole joint backward on CUDA cores: bwd_prep (image, text rows), "
+                            "bwd_dkv_kernel (text keys), bwd_dq_kernel (image, text queries), "
+                            "bwd_dkv_kernel (window keys)") if L else
+                           ("whole backward: bwd_prep, tc_bwd_kernel (dQ), tc_bwd_kernel (dK, dV)"
+                            + (", pool_kernel, tc_bwd_kernel (pooled dK, dV)" if w.P else ""))})
     line = {"metric": "window-attn backward latency (ms) & TFLOP/s", "value": world * tflops,
             "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": "bf16 (tensor cores, fp32 accumulate)" if w.dtype == "bf16" else w.dtype,
+            "dtype": ("bf16 (CUDA cores, fp32 arithmetic)" if L else
+                      "bf16 (tensor cores, fp32 accumulate)") if w.dtype == "bf16" else w.dtype,
             "data": "synthetic",
-            "config": {"workload": f"{w.name} backward", "N": w.N, "m": w.m, "P": w.P,
+            "config": {"workload": f"{w.name} backward", "N": w.N, "m": w.m, "P": w.P, "L": L,
                        "l2": "evicted before every step (256 MiB write, then 256 MiB read; outside the events)"},
             "roofline": roof,
-            "gpu_launches": (5 if w.P else 3) * args.steps, "clocks": clk}
+            "gpu_launches": (6 if L else 5 if w.P else 3) * args.steps, "clocks": clk}
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:

@@ -22,7 +22,8 @@ from ._lib import BASA_FLAG_PAD_GRID, BASA_FLAG_BWD_CUDA_CORES  # noqa: F401
 
 __all__ = ["window_attn", "window_attn_gm", "full_attn", "joint_attn", "window_attn_bwd",
            "joint_attn_bwd",
-           "pool_kv", "workspace_size", "bwd_workspace_size", "joint_workspace_size", "get_status", "window_tiles", "make_params", "BasaError",
+           "pool_kv", "workspace_size", "bwd_workspace_size", "joint_workspace_size",
+           "joint_bwd_workspace_size", "get_status", "window_tiles", "make_params", "BasaError",
            "library_path", "BASA_FLAG_PAD_GRID", "BASA_FLAG_BWD_CUDA_CORES"]
 
 library_path = _lib.LIB_PATH
@@ -101,6 +102,13 @@ def joint_workspace_size(shape, dtype, window, shift, L, hkv=0) -> int:
     """Bytes of device workspace joint_attn uses to split its text-query pass (0: none)."""
     return int(_lib.load().basa_joint_workspace_size(
         ctypes.byref(make_params(shape, dtype, window, shift, (0, 0, 0), hkv=hkv)), int(L)))
+
+
+def joint_bwd_workspace_size(shape, dtype, window, shift, L, hkv=0, flags=0) -> int:
+    """Bytes of device workspace joint_attn_bwd needs (D of the image and text rows)."""
+    return int(_lib.load().basa_joint_bwd_workspace_size(
+        ctypes.byref(make_params(shape, dtype, window, shift, (0, 0, 0), flags=flags, hkv=hkv)),
+        int(L)))
 
 
 def pool_kv(k: torch.Tensor, v: torch.Tensor, pool, out=None, stream=None):
