@@ -40,7 +40,7 @@ class Workload:
     Wg: int
     H: int
     d: int
-    dtype: str                      # "f32" or "bf16"
+    dtype: str                      # "f32", "bf16" or "e4m3" (bf16 output)
     window: Tuple[int, int, int]    # (wt, wh, ww)
     shifts: Tuple[Tuple[int, int, int], ...]  # one (st, sh, sw) per DiT block
     pool: Tuple[int, int, int] = (0, 0, 0)     # (pt, ph, pw); zeros = no global memory
@@ -92,10 +92,14 @@ WORKLOADS = {
     # tokens (the T5 prompt length FLUX uses); q, k, v ~ N(0, 1) for both streams
     "flux1024_text512": Workload("flux1024_text512", 1, 1, 64, 64, 24, 128, "bf16",
                                  (1, 16, 16), ((0, 8, 8),), text=512),
+    # the flux2048 block with q, k, v stored as fp8 e4m3 (the same draws rounded
+    # to e4m3 instead of bf16; descale factors 1)
+    "flux2048_e4m3": Workload("flux2048_e4m3", 1, 1, 128, 128, 24, 128, "e4m3",
+                              (1, 16, 16), ((0, 8, 8),), head_scale=(0.5, 2.0)),
 }
 
 WORKLOAD_INDEX = {"grid16_f32": 0, "flux1024": 1, "flux2048": 2, "wan_video": 3,
-                  "flux2048_gm4": 4, "flux1024_text512": 5}
+                  "flux2048_gm4": 4, "flux1024_text512": 5, "flux2048_e4m3": 2}
 
 
 def seed_for(workload_index: int, block: int, which: str) -> int:
@@ -104,10 +108,12 @@ def seed_for(workload_index: int, block: int, which: str) -> int:
 
 
 def to_storage(x: np.ndarray, dtype: str) -> torch.Tensor:
-    """Round a float array to the storage dtype (RNE for bf16) as a CPU tensor."""
+    """Round a float array to the storage dtype (RNE for bf16 and e4m3) as a CPU tensor."""
     t = torch.from_numpy(np.ascontiguousarray(x, dtype=np.float32))
     if dtype == "bf16":
         return t.to(torch.bfloat16)
+    if dtype == "e4m3":  # OCP fp8 e4m3 (torch.float8_e4m3fn); |x| here stays far below 448
+        return t.to(torch.float8_e4m3fn)
     if dtype == "f32":
         return t
     raise ValueError(f"unknown dtype {dtype!r}")

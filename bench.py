@@ -100,8 +100,9 @@ def workload_numbers(w, shift):
     N, m, P, L = w.N, w.m, w.P, w.text
     pairs = N * (m + P + L) + L * (N + L)
     flops = 4.0 * B * H * d * pairs
-    esize = 2 if w.dtype == "bf16" else 4
-    bytes_ = 4.0 * B * H * (N + L) * d * esize
+    esize = {"bf16": 2, "e4m3": 1}.get(w.dtype, 4)  # q, k, v elements
+    osize = 2 if w.dtype == "e4m3" else esize        # the output (bf16 for e4m3 inputs)
+    bytes_ = B * H * (N + L) * d * (3.0 * esize + osize)
     theo = (N + L) ** 2 / pairs  # full attention over all tokens / this step
     return flops, bytes_, N, m, P, theo
 
@@ -433,8 +434,9 @@ def main():
     q, k, v = workload_inputs(w, blk)
     qh, kh, vh = (x.pin_memory() for x in (q, k, v))
     dq, dk, dv = (x.to(dev) for x in (q, k, v))
-    out = torch.empty_like(dq)
-    outh = torch.empty_like(qh).pin_memory()
+    odt = torch.bfloat16 if dq.dtype == torch.float8_e4m3fn else dq.dtype  # e4m3 -> bf16 out
+    out = torch.empty(dq.shape, dtype=odt, device=dev)
+    outh = torch.empty(qh.shape, dtype=odt).pin_memory()
     ws_bytes = basa.workspace_size(w.shape(), dq.dtype, w.window, shift, w.pool)
     ws = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=dev)
     flush = L2Flush(dev)

@@ -88,7 +88,13 @@ typedef enum basa_status {
                                  an output index outside its tensor and skipped the access */
 } basa_status;
 
-typedef enum basa_dtype { BASA_F32 = 0, BASA_BF16 = 1 } basa_dtype;
+/* Element types.  BASA_FP8_E4M3: q, k, v as OCP e4m3 bytes (basa_window_attn
+ * and basa_full_attn only, d = 128, no pool cell), each tensor's values scaled
+ * by its descale factor in basa_params; the output is bf16 [B, T, Hg, Wg, H, d]
+ * and lse fp32.  Q K^T runs on e4m3 tensor-core MMAs; V is widened to bf16 in
+ * shared memory (exactly) for the bf16 P.V MMA.  Other entry points return
+ * BASA_ERR_UNSUPPORTED for it. */
+typedef enum basa_dtype { BASA_F32 = 0, BASA_BF16 = 1, BASA_FP8_E4M3 = 2 } basa_dtype;
 
 /* Flag bits for basa_params.flags. */
 #define BASA_FLAG_PAD_GRID 0x4u            /* grids that a window size does not divide: each
@@ -122,6 +128,9 @@ typedef struct basa_params {
   int32_t Hkv;         /* K/V heads (grouped-query attention); 0 selects H.  H must be a
                           multiple of Hkv; query head h reads K/V head h / (H / Hkv).
                           k, v and pooled / text K/V then have Hkv heads, q and out H. */
+  float q_descale, k_descale, v_descale; /* BASA_FP8_E4M3 only: the value of an element is
+                          its e4m3 value times its tensor's factor (0 selects 1); other
+                          dtypes ignore them */
 } basa_params;
 
 /* Human-readable name of a status code (static string). */

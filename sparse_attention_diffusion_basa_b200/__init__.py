@@ -17,7 +17,7 @@ from typing import Optional, Sequence, Tuple
 import torch
 
 from . import _lib
-from ._lib import BasaError, BasaParams, BASA_F32, BASA_BF16  # noqa: F401
+from ._lib import BasaError, BasaParams, BASA_F32, BASA_BF16, BASA_FP8_E4M3  # noqa: F401
 from ._lib import BASA_FLAG_PAD_GRID, BASA_FLAG_BWD_CUDA_CORES  # noqa: F401
 
 __all__ = ["window_attn", "window_attn_gm", "full_attn", "joint_attn", "window_attn_bwd",
@@ -28,7 +28,7 @@ __all__ = ["window_attn", "window_attn_gm", "full_attn", "joint_attn", "window_a
 
 library_path = _lib.LIB_PATH
 
-_DT = {torch.float32: BASA_F32, torch.bfloat16: BASA_BF16}
+_DT = {torch.float32: BASA_F32, torch.bfloat16: BASA_BF16, torch.float8_e4m3fn: BASA_FP8_E4M3}
 
 
 def _triple(x, name) -> Tuple[int, int, int]:
@@ -40,13 +40,21 @@ def _triple(x, name) -> Tuple[int, int, int]:
 
 def make_params(shape: Sequence[int], dtype, window=(1, 1, 1), shift=(0, 0, 0),
                 pool=(0, 0, 0), scale: Optional[float] = None, flags: int = 0,
-                wait_timeout_ms: int = 0, hkv: int = 0) -> BasaParams:
+                wait_timeout_ms: int = 0, hkv: int = 0, descale=(0.0, 0.0, 0.0)) -> BasaParams:
     B, T, Hg, Wg, H, d = (int(s) for s in shape)
     if isinstance(dtype, torch.dtype):
         dtype = _DT[dtype]
     w, s, p = _triple(window, "window"), _triple(shift, "shift"), _triple(pool, "pool")
+    dq, dk, dv = (float(x) for x in descale)
     return BasaParams(B, H, T, Hg, Wg, d, *w, *s, *p, float(scale or 0.0), int(dtype),
-                      int(flags), int(wait_timeout_ms), int(hkv))
+                      int(flags), int(wait_timeout_ms), int(hkv), dq, dk, dv)
+
+
+def _out_like(q):
+    """Output tensor of an attention call: bf16 for e4m3 inputs, else q's dtype."""
+    if q.dtype == torch.float8_e4m3fn:
+        return torch.empty(q.shape, dtype=torch.bfloat16, device=q.device)
+    return torch.empty_like(q)
 
 
 def _kv_heads(q, k, v) -> int:
@@ -139,13 +147,17 @@ def pool_kv(k: torch.Tensor, v: torch.Tensor, pool, out=None, stream=None):
 
 def window_attn(q, k, v, window, shift=(0, 0, 0), pool=(0, 0, 0), scale=None,
                 return_lse=False, out=None, workspace=None, flags=0, wait_timeout_ms=0,
-                stream=None):
-    """Shifted local window attention (plus pooled global memory when pool != 0)."""
+                stream=None, descale=(0.0, 0.0, 0.0)):
+    """Shifted local window attention (plus pooled global memory when pool != 0).
+
+    e4m3 inputs (torch.float8_e4m3fn, d = 128, no pool): each tensor's values
+    times its factor in ``descale`` (q, k, v; 0 = 1); the output is bf16."""
     _check_inputs(q, k, v)
     hkv = _kv_heads(q, k, v)
-    prm = make_params(q.shape, q.dtype, window, shift, pool, scale, flags, wait_timeout_ms, hkv)
+    prm = make_params(q.shape, q.dtype, window, shift, pool, scale, flags, wait_timeout_ms, hkv,
+                      descale)
     lib = _lib.load()
-    out = torch.empty_like(q) if out is None else out
+    out = _out_like(q) if out is None else out
     B, T, Hg, Wg, H, d = q.shape
     lse = torch.empty((B, H, T * Hg * Wg), dtype=torch.float32, device=q.device) if return_lse else None
     need = int(lib.basa_workspace_size(ctypes.byref(prm)))
@@ -175,13 +187,16 @@ def window_attn_gm(q, k, v, kp, vp, window, shift=(0, 0, 0), pool=(1, 1, 1), sca
     return (out, lse) if return_lse else out
 
 
-def full_attn(q, k, v, scale=None, return_lse=False, out=None, flags=0, stream=None):
-    """Full softmax attention over all grid tokens (one window covering the grid)."""
+def full_attn(q, k, v, scale=None, return_lse=False, out=None, flags=0, stream=None,
+              descale=(0.0, 0.0, 0.0)):
+    """Full softmax attention over all grid tokens (one window covering the grid);
+    e4m3 inputs as in window_attn."""
     _check_inputs(q, k, v)
     hkv = _kv_heads(q, k, v)
-    prm = make_params(q.shape, q.dtype, (1, 1, 1), (0, 0, 0), (0, 0, 0), scale, flags, hkv=hkv)
+    prm = make_params(q.shape, q.dtype, (1, 1, 1), (0, 0, 0), (0, 0, 0), scale, flags, hkv=hkv,
+                      descale=descale)
     lib = _lib.load()
-    out = torch.empty_like(q) if out is None else out
+    out = _out_like(q) if out is None else out
     B, T, Hg, Wg, H, d = q.shape
     lse = torch.empty((B, H, T * Hg * Wg), dtype=torch.float32, device=q.device) if return_lse else None
     with torch.cuda.device(q.device):

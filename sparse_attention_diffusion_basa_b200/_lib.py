@@ -16,7 +16,7 @@ STATUS_NAMES = {
     4: "BASA_ERR_ALIGN", 5: "BASA_ERR_WORKSPACE", 6: "BASA_ERR_CUDA", 7: "BASA_ERR_TIMEOUT",
     8: "BASA_ERR_SCRATCH_LIMIT", 9: "BASA_ERR_CHECK",
 }
-BASA_F32, BASA_BF16 = 0, 1
+BASA_F32, BASA_BF16, BASA_FP8_E4M3 = 0, 1, 2
 BASA_FLAG_TEST_WITHHOLD_LOADS = 0x1
 BASA_FLAG_BWD_CUDA_CORES = 0x2
 BASA_FLAG_PAD_GRID = 0x4
@@ -34,7 +34,9 @@ class BasaParams(ctypes.Structure):
                 ("B", "H", "T", "Hg", "Wg", "d", "wt", "wh", "ww", "st", "sh", "sw",
                  "pt", "ph", "pw")] + [
         ("scale", ctypes.c_float), ("dtype", ctypes.c_int32), ("flags", ctypes.c_uint32),
-        ("wait_timeout_ms", ctypes.c_uint32), ("Hkv", ctypes.c_int32)]
+        ("wait_timeout_ms", ctypes.c_uint32), ("Hkv", ctypes.c_int32),
+        ("q_descale", ctypes.c_float), ("k_descale", ctypes.c_float),
+        ("v_descale", ctypes.c_float)]
 
 
 class BasaError(RuntimeError):

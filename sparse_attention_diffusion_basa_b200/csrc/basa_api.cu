@@ -23,23 +23,37 @@ static int floor_mod(long long a, int n) {
   return (int)(r < 0 ? r + n : r);
 }
 
-basa_status normalise(const basa_params* p, bool full, Dims* d) {
+basa_status normalise(const basa_params* p, bool full, Dims* d, bool allow_fp8) {
   if (!p || !d) return BASA_ERR_INVALID_ARG;
   if (p->B < 0 || p->H < 0 || p->T < 0 || p->Hg < 0 || p->Wg < 0 || p->d <= 0)
     return BASA_ERR_INVALID_ARG;
-  if (p->dtype != BASA_F32 && p->dtype != BASA_BF16) return BASA_ERR_INVALID_ARG;
+  if (p->dtype != BASA_F32 && p->dtype != BASA_BF16 && p->dtype != BASA_FP8_E4M3)
+    return BASA_ERR_INVALID_ARG;
+  if (p->dtype == BASA_FP8_E4M3) {
+    if (!allow_fp8 || p->d != 128) return BASA_ERR_UNSUPPORTED;
+    if (p->pt != 0 || p->ph != 0 || p->pw != 0) return BASA_ERR_UNSUPPORTED;
+  }
+  const float dq = p->q_descale, dk = p->k_descale, dv = p->v_descale;
+  if (!(dq >= 0.0f) || !(dk >= 0.0f) || !(dv >= 0.0f) || isinf(dq) || isinf(dk) || isinf(dv))
+    return BASA_ERR_INVALID_ARG;
   if (!(p->scale >= 0.0f) || isinf(p->scale)) return BASA_ERR_INVALID_ARG;
   memset(d, 0, sizeof(*d));
   d->B = p->B; d->H = p->H; d->T = p->T; d->Hg = p->Hg; d->Wg = p->Wg; d->d = p->d;
   if (p->Hkv < 0 || (p->Hkv > 0 && p->H % p->Hkv != 0)) return BASA_ERR_INVALID_ARG;
   d->Hkv = p->Hkv > 0 ? p->Hkv : p->H;
   d->dtype = p->dtype;
+  d->qk_descale = 1.0f;
+  d->v_descale = 1.0f;
+  if (p->dtype == BASA_FP8_E4M3) {
+    d->qk_descale = (dq > 0.0f ? dq : 1.0f) * (dk > 0.0f ? dk : 1.0f);
+    d->v_descale = dv > 0.0f ? dv : 1.0f;
+  }
   d->N = (long long)p->T * p->Hg * p->Wg;
   d->Nq = d->N;
   d->scale = p->scale > 0.0f ? p->scale : 1.0f / sqrtf((float)p->d);
   if (p->dtype == BASA_F32) {
     if (p->d != 32 && p->d != 64 && p->d != 128) return BASA_ERR_UNSUPPORTED;
-  } else {
+  } else if (p->dtype == BASA_BF16) {
     if (p->d != 64 && p->d != 128) return BASA_ERR_UNSUPPORTED;
   }
   if ((long long)p->B * p->H * d->N == 0) return BASA_OK;  // empty: valid no-op
@@ -168,7 +182,8 @@ static EncodeTiledFn encode_fn() {
 }
 
 basa_status encode_map(CUtensorMap* map, const void* base, int rank, const uint64_t* dims,
-                       const uint64_t* strides_bytes, const uint32_t* box) {
+                       const uint64_t* strides_bytes, const uint32_t* box,
+                       CUtensorMapDataType type) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return BASA_ERR_CUDA;
   cuuint64_t gd[5], gs[4];
@@ -179,7 +194,7 @@ basa_status encode_map(CUtensorMap* map, const void* base, int rank, const uint6
     es[i] = 1;
   }
   for (int i = 0; i < rank - 1; ++i) gs[i] = strides_bytes[i];
-  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank, const_cast<void*>(base),
+  CUresult r = fn(map, type, (cuuint32_t)rank, const_cast<void*>(base),
                   gd, gs, bx, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? BASA_OK : BASA_ERR_CUDA;
@@ -220,7 +235,7 @@ int basa_version(void) { return 200; }
 
 size_t basa_workspace_size(const basa_params* p) {
   Dims d;
-  if (normalise(p, false, &d) != BASA_OK || d.P == 0) return 0;
+  if (normalise(p, false, &d, true) != BASA_OK || d.P == 0) return 0;
   return 2 * pooled_bytes(d);
 }
 
@@ -258,7 +273,7 @@ basa_status basa_window_attn(const void* q, const void* k, const void* v, void* 
                              void* workspace, const basa_params* p, cudaStream_t stream) {
   NvtxRange nvtx("basa_window_attn");
   Dims d;
-  basa_status s = normalise(p, false, &d);
+  basa_status s = normalise(p, false, &d, true);
   if (s != BASA_OK) return s;
   if ((long long)d.B * d.H * d.N == 0) return BASA_OK;
   if ((s = check_qkvo(q, k, v, out, lse)) != BASA_OK) return s;
@@ -443,7 +458,7 @@ basa_status basa_full_attn(const void* q, const void* k, const void* v, void* ou
                            const basa_params* p, cudaStream_t stream) {
   NvtxRange nvtx("basa_full_attn");
   Dims d;
-  basa_status s = normalise(p, true, &d);
+  basa_status s = normalise(p, true, &d, true);
   if (s != BASA_OK) return s;
   if ((long long)d.B * d.H * d.N == 0) return BASA_OK;
   if ((s = check_qkvo(q, k, v, out, lse)) != BASA_OK) return s;
@@ -463,9 +478,9 @@ basa_status basa_get_status(cudaStream_t stream) {
 basa_status basa_window_tiles(const basa_params* p, int32_t* n_windows, int32_t* n_tiles,
                               int32_t* rows, int64_t rows_capacity) {
   Dims d;
-  basa_status s = normalise(p, false, &d);
+  basa_status s = normalise(p, false, &d, true);
   if (s != BASA_OK) return s;
-  if (d.dtype != BASA_BF16) return BASA_ERR_UNSUPPORTED;
+  if (d.dtype == BASA_F32) return BASA_ERR_UNSUPPORTED;  // the tensor-core kernel's plan
   if ((long long)d.B * d.H * d.N == 0) return BASA_ERR_INVALID_ARG;
   TilePlan plan;
   if ((s = build_tile_plan(d, &plan)) != BASA_OK) return s;

@@ -27,11 +27,14 @@ struct Dims {
   int qsep;           // 1: queries are separate rows [B, Nq, H, d] (text queries)
   float scale;
   int dtype;
+  float qk_descale;   // e4m3: q_descale * k_descale (1 otherwise), folded into the logit scale
+  float v_descale;    // e4m3: applied to the output (1 otherwise)
 };
 
 // Validates p and fills d.  `full` = one window covering the grid, no shift,
-// no pool (full attention).
-basa_status normalise(const basa_params* p, bool full, Dims* d);
+// no pool (full attention).  allow_fp8: the entry point takes e4m3 inputs
+// (otherwise BASA_FP8_E4M3 is BASA_ERR_UNSUPPORTED).
+basa_status normalise(const basa_params* p, bool full, Dims* d, bool allow_fp8 = false);
 
 // ---------------------------------------------------------------------------
 // Tile plan of the bf16 tensor-core kernel (shifted-window index math).
@@ -185,8 +188,9 @@ basa_status launch_ex2_poly_test(const float* x, float* y, long long n, cudaStre
 basa_status read_and_clear_status(cudaStream_t stream);
 cudaError_t take_bwd_status(cudaStream_t stream, unsigned int* status, unsigned int* where);
 
-// Encodes a tiled TMA map through the driver entry point.
+// Encodes a tiled TMA map (128-byte swizzle) through the driver entry point.
 basa_status encode_map(CUtensorMap* map, const void* base, int rank, const uint64_t* dims,
-                       const uint64_t* strides_bytes, const uint32_t* box);
+                       const uint64_t* strides_bytes, const uint32_t* box,
+                       CUtensorMapDataType type = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16);
 
 }  // namespace basa

@@ -100,7 +100,41 @@ struct __align__(64) TcParams {
   uint32_t units_per_split;
   float* part_o;   // [n_splits, B, H, Nq, d]
   float* part_ml;  // [n_splits, B, H, Nq, 2]: base-2 running max, sum
+  float v_scale;   // e4m3 inputs: the V descale factor, applied in the epilogue
 };
+
+// Two e4m3 values (lower byte first) as a bf16 pair.  Exact: every e4m3 value
+// (3 mantissa bits, exponents 2^-9 .. 2^8) is a bf16 value.
+__device__ __forceinline__ uint32_t e4m3x2_to_bf16x2(uint32_t two) {
+  const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)two, __NV_E4M3);
+  const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&h));
+  return pack_bf16(f.x, f.y);
+}
+
+// Widens one e4m3 V tile (128 rows of D bytes, 128-byte swizzled rows) into the
+// bf16 layout the P.V MMA reads (D / 64 halves of 128 rows x 128 bytes, same
+// swizzle).  One warp; each lane converts 16-byte chunks of 16 values.
+template <int D>
+__device__ __forceinline__ void widen_v_tile(uint32_t src, uint32_t dst, int lane) {
+  static_assert(D == 128, "e4m3 tiles have 128-byte rows");
+#pragma unroll 4
+  for (int it = 0; it < 32; ++it) {
+    const int item = it * 32 + lane;
+    const int r = item >> 3, c = item & 7;
+    const uint4 x = ld_shared_v4(src + r * 128 + ((c ^ (r & 7)) << 4));
+    const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+    uint32_t o[8];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      o[2 * e] = e4m3x2_to_bf16x2(w[e] & 0xffffu);
+      o[2 * e + 1] = e4m3x2_to_bf16x2(w[e] >> 16);
+    }
+    const uint32_t half = dst + (uint32_t)(c >> 2) * kHalf + r * 128;
+    const int c2 = 2 * (c & 3);
+    st_shared_v4(half + ((c2 ^ (r & 7)) << 4), o[0], o[1], o[2], o[3]);
+    st_shared_v4(half + (((c2 + 1) ^ (r & 7)) << 4), o[4], o[5], o[6], o[7]);
+  }
+}
 
 
 // Which exponential pairs go to the polynomial: pair e of every 16 when
@@ -202,10 +236,10 @@ __device__ __forceinline__ int query_valid(const TcParams& p, const PlanView& pv
 
 // kind: 0 = q, 1 = k, 2 = v.  Loads one 128-row tile (all head-dim halves) into
 // shared memory at dst and signals bar with the transaction bytes.
-template <int D>
+template <int D, bool kF8 = false>
 __device__ __forceinline__ void load_tile(const TcParams& p, const PlanView& pv, int kind,
                                           const Unit& U, int tile, uint32_t dst, uint32_t bar) {
-  constexpr int NH = D / 64;
+  constexpr int NH = kF8 ? D / 128 : D / 64;  // 128-byte boxes per row (coordinate 0 for e4m3)
   if (kind != 0 && tile >= p.n_wkt) {  // extra keys: pooled global memory or text tokens
     const CUtensorMap* m = kind == 1 ? &p.kpf : &p.vpf;
 #pragma unroll
@@ -263,22 +297,38 @@ __device__ __forceinline__ long long row_token(const TcParams& p, const PlanView
                           p.T, p.Hg, p.Wg);
 }
 
+// Bit r of word r / 32: row r of key tile j of U's window holds a token (not a
+// padded position, not a row past the tile).  Warp-collective.
+__device__ __forceinline__ uint4 key_token_mask(const TcParams& p, const PlanView& pv, const Unit& U,
+                                             int j, int lane) {
+  uint32_t w[4];
+#pragma unroll
+  for (int cc = 0; cc < 4; ++cc)
+    w[cc] = __ballot_sync(0xffffffffu, row_token(p, pv, U, j, cc * 32 + lane) >= 0);
+  return make_uint4(w[0], w[1], w[2], w[3]);
+}
+
 // Shared-memory plan: the unit's two 128-row query tiles, one 64-column output
 // staging block per query tile, and a ring of K/V tiles.  The probabilities P
 // never touch shared memory: they are written into TMEM over their logits and
 // read from there by the P.V MMA.
-template <int D, int kRing>
+template <int D, int kRing, bool kF8 = false>
 struct Smem {
-  static constexpr int kTile = (D / 64) * kHalf;  // Q/K/V tile bytes
+  // Q/K/V tile bytes: 128 rows of D bf16 (D / 64 swizzled halves), or of D e4m3
+  static constexpr int kTile = kF8 ? (D / 128) * kHalf : (D / 64) * kHalf;
+  static constexpr int kVbf = (D / 64) * kHalf;   // one V tile widened to bf16 (e4m3 only)
   static constexpr int NS = kRing;                // K/V ring slots
   static constexpr int q0 = 0;
   static constexpr int stg0 = 2 * kTile;
   static constexpr int ring0 = stg0 + 2 * kHalf;
-  static constexpr int bars = ring0 + NS * kTile;
-  // barrier indices
+  static constexpr int vbf0 = ring0 + NS * kTile;
+  static constexpr int bars = vbf0 + (kF8 ? 2 * kVbf : 0);
+  // barrier indices (VBFULL, VBEMPTY: the two widened V buffers, e4m3 only)
   static constexpr int QFULL = 0, QEMPTY = 2, SFULL = 4, PFULL = 6, OFULL = 8, STAGED = 10,
                        STGFREE = 12, DRAIN = 14, KVFULL = 15, KVEMPTY = 15 + NS,
-                       NBARS = 15 + 2 * NS;
+                       VBFULL = 15 + 2 * NS, VBEMPTY = 17 + 2 * NS,
+                       NBARS = 15 + 2 * NS + (kF8 ? 4 : 0);
+  static_assert(VBEMPTY == VBFULL + 2, "two widened V buffers");
   static constexpr int misc = bars + NBARS * 8;  // tmem slot, abort flag
   static constexpr int plan = misc + 64;         // compact tile plan (kPlanBytes)
   static constexpr int bytes = plan + kPlanBytes;
@@ -294,9 +344,9 @@ struct Smem {
 // alternate: while softmax 0 exponentiates S_0(j+1), the tensor core runs
 // P_1(j) V_j and S_1(j+1), and the other way round, so the exponentials of one
 // tile overlap the MMAs of the other.
-template <int D, int kRing, bool kSplit>
+template <int D, int kRing, bool kSplit, bool kF8 = false>
 __global__ void __launch_bounds__(kThreads, 1) tc_attn_kernel(const __grid_constant__ TcParams p) {
-  using S = Smem<D, kRing>;
+  using S = Smem<D, kRing, kF8>;
   constexpr int NS = S::NS;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -327,6 +377,12 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attn_kernel(const __grid_const
     for (int s = 0; s < NS; ++s) {
       mbar_init(BAR(S::KVFULL + s), 1);
       mbar_init(BAR(S::KVEMPTY + s), 1);
+    }
+    if constexpr (kF8) {
+      for (int b = 0; b < 2; ++b) {
+        mbar_init(BAR(S::VBFULL + b), 1);
+        mbar_init(BAR(S::VBEMPTY + b), 1);
+      }
     }
     *abort_flag = 0u;
     fence_barrier_init();
@@ -380,8 +436,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attn_kernel(const __grid_const
               break;
             if (lane == 0) {
               mbar_expect_tx(BAR(S::KVFULL + slot), S::kTile);
-              load_tile<D>(p, pv, kind, U, j, sbase + S::ring0 + slot * S::kTile,
-                           BAR(S::KVFULL + slot));
+              load_tile<D, kF8>(p, pv, kind, U, j, sbase + S::ring0 + slot * S::kTile,
+                                BAR(S::KVFULL + slot));
             }
             __syncwarp();
             issued_mask |= 1u << slot;
@@ -412,8 +468,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attn_kernel(const __grid_const
             break;
           if (lane == 0) {
             mbar_expect_tx(BAR(S::QFULL + i), S::kTile);
-            load_tile<D>(p, pv, 0, U, 2 * U.pair + i, sbase + S::q0 + i * S::kTile,
-                         BAR(S::QFULL + i));
+            load_tile<D, kF8>(p, pv, 0, U, 2 * U.pair + i, sbase + S::q0 + i * S::kTile,
+                              BAR(S::QFULL + i));
           }
           __syncwarp();
           q_issued |= 1u << i;
@@ -430,10 +486,10 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attn_kernel(const __grid_const
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     // The whole warp walks the schedule and waits; lane 0 issues MMAs and commits.
-    constexpr uint32_t IDS = idesc_bf16(128, false);
+    constexpr uint32_t IDS = kF8 ? idesc_e4m3(128) : idesc_bf16(128, false);
     constexpr uint32_t IDO = idesc_bf16(D, true);
     uint32_t qf[2] = {0u, 0u}, pfull[2] = {0u, 0u};
-    uint32_t kv = 0;
+    uint32_t kv = 0, vbn = 0;
     bool ok = true;
     auto take_slot = [&](uint32_t& slot) -> bool {
       slot = kv % NS;
@@ -447,20 +503,54 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attn_kernel(const __grid_const
       if (lane == 0) mma_commit(BAR(S::KVEMPTY + slot));
       __syncwarp();
     };
+    // V_j for P.V: its ring slot (bf16), or (e4m3) the widened bf16 copy that
+    // warp 3 makes, whose ring slot warp 3 releases; vref = slot or buffer.
+    auto take_v = [&](uint32_t& vaddr, uint32_t& vref) -> bool {
+      if constexpr (kF8) {
+        ++kv;
+        vref = vbn & 1u;
+        const uint32_t par = (vbn >> 1) & 1u;
+        ++vbn;
+        if (!wait_warp(BAR(S::VBFULL + vref), par, abort_flag, limit, kSiteMmaKvFull)) return false;
+        tc_fence_after();
+        vaddr = sbase + S::vbf0 + vref * S::kVbf;
+        return true;
+      } else {
+        if (!take_slot(vref)) return false;
+        vaddr = sbase + S::ring0 + vref * S::kTile;
+        return true;
+      }
+    };
+    auto release_v = [&](uint32_t vref) {
+      if constexpr (kF8) {
+        if (lane == 0) mma_commit(BAR(S::VBEMPTY + vref));
+        __syncwarp();
+      } else {
+        release(vref);
+      }
+    };
     // S_i = Q_i K^T (lane 0 only)
     auto mma_s = [&](int i, uint32_t kslot) {
       const uint32_t qa = sbase + S::q0 + i * S::kTile;
       const uint32_t ka = sbase + S::ring0 + kslot * S::kTile;
+      if constexpr (kF8) {  // 32 e4m3 (32 bytes) per step along the 128-byte rows
 #pragma unroll
-      for (int k = 0; k < D / 16; ++k) {
-        const uint32_t off = (k / 4) * kHalf + (k % 4) * 32;
-        mma_bf16(tmem + i * 128, sdesc(qa + off, 16, 1024), sdesc(ka + off, 16, 1024), IDS,
-                 k > 0 ? 1u : 0u);
+        for (int k = 0; k < D / 32; ++k) {
+          const uint32_t off = (k / 4) * kHalf + (k % 4) * 32;
+          mma_e4m3(tmem + i * 128, sdesc(qa + off, 16, 1024), sdesc(ka + off, 16, 1024), IDS,
+                   k > 0 ? 1u : 0u);
+        }
+      } else {
+#pragma unroll
+        for (int k = 0; k < D / 16; ++k) {
+          const uint32_t off = (k / 4) * kHalf + (k % 4) * 32;
+          mma_bf16(tmem + i * 128, sdesc(qa + off, 16, 1024), sdesc(ka + off, 16, 1024), IDS,
+                   k > 0 ? 1u : 0u);
+        }
       }
     };
     // O_i (+)= P_i V, P_i from TMEM (8 columns per 16 keys) (lane 0 only)
-    auto mma_pv = [&](int i, uint32_t vslot, bool accumulate) {
-      const uint32_t va = sbase + S::ring0 + vslot * S::kTile;
+    auto mma_pv = [&](int i, uint32_t va, bool accumulate) {
 #pragma unroll
       for (int k = 0; k < 8; ++k)
         mma_bf16_ts(tmem + 256 + i * 128, tmem + i * 128 + k * 8,
@@ -486,8 +576,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attn_kernel(const __grid_const
       release(kslot);
       for (int j = 0; j < kcount(U) && ok; ++j) {
         const bool next = j + 1 < kcount(U);
-        uint32_t vslot;
-        if (!(ok = take_slot(vslot))) break;
+        uint32_t vaddr, vref;
+        if (!(ok = take_v(vaddr, vref))) break;
         if (next && !(ok = take_slot(kslot))) break;
         for (int i = 0; i < U.nq && ok; ++i) {
           // P_i(j) in TMEM and O_i rescaled; for j = 0 this also orders the
@@ -498,7 +588,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attn_kernel(const __grid_const
           ++pfull[i];
           tc_fence_after();
           if (lane == 0) {
-            mma_pv(i, vslot, j > 0);
+            mma_pv(i, vaddr, j > 0);
             if (next) {
               mma_s(i, kslot);
               mma_commit(BAR(S::SFULL + i));
@@ -510,7 +600,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attn_kernel(const __grid_const
           __syncwarp();
         }
         if (!ok) break;
-        release(vslot);
+        release_v(vref);
         if (next) release(kslot);
       }
     }
@@ -518,6 +608,42 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attn_kernel(const __grid_const
     if (lane == 0) mma_commit(BAR(S::DRAIN));
     __syncwarp();
     wait_warp(BAR(S::DRAIN), 0u, abort_flag, limit, kSiteMmaDrain, false);
+  } else if (warp == 3) {
+    // ------------------------------------------------------------ V widening (e4m3)
+    // Walks the K/V ring in the loader's order; each V tile is widened to bf16
+    // into one of two buffers for the P.V MMA (whose operands must both be
+    // bf16), then its ring slot is handed back to the loader.
+    if constexpr (kF8) {
+      if (!withhold) {
+        uint32_t kv = 0, vbn = 0;
+        bool ok = true;
+        for (uint32_t u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
+          const Unit U = decode_unit<kSplit>(p, u);
+          for (int j = kbeg(U); j < kbeg(U) + kcount(U) && ok; ++j) {
+            ++kv;  // K_j
+            const uint32_t slot = kv % NS, par = (kv / NS) & 1u;
+            ++kv;
+            const uint32_t b = vbn & 1u, bpar = (vbn >> 1) & 1u;
+            ++vbn;
+            if (!(ok = wait_warp(BAR(S::KVFULL + slot), par, abort_flag, limit, kSiteMmaKvFull)))
+              break;
+            if (!(ok = wait_warp(BAR(S::VBEMPTY + b), bpar ^ 1u, abort_flag, limit,
+                                 kSiteMmaKvFull)))
+              break;
+            tc_fence_after();
+            widen_v_tile<D>(sbase + S::ring0 + slot * S::kTile, sbase + S::vbf0 + b * S::kVbf,
+                            lane);
+            fence_proxy_async();  // the generic stores, before the tensor core reads them
+            __syncwarp();
+            if (lane == 0) {
+              mbar_arrive(BAR(S::VBFULL + b));
+              mbar_arrive(BAR(S::KVEMPTY + slot));
+            }
+            __syncwarp();
+          }
+        }
+      }
+    }
   } else if (warp >= 4) {
     // ------------------------------------------------------------ softmax + epilogue
     const int i = (warp - 4) / 4;      // query tile slot of the unit
@@ -556,10 +682,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attn_kernel(const __grid_const
               if (cc * 32 + e >= kvalid) s[cc][e] = __float_as_uint(-INFINITY);
         }
         if (U.holes && j < p.n_wkt) {  // keys at padded positions of this window
-          uint32_t okw[4];
-#pragma unroll
-          for (int cc = 0; cc < 4; ++cc)
-            okw[cc] = __ballot_sync(0xffffffffu, row_token(p, pv, U, j, cc * 32 + lane) >= 0);
+          const uint4 ok4 = key_token_mask(p, pv, U, j, lane);
+          const uint32_t okw[4] = {ok4.x, ok4.y, ok4.z, ok4.w};
 #pragma unroll
           for (int cc = 0; cc < 4; ++cc)
 #pragma unroll
@@ -664,7 +788,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attn_kernel(const __grid_const
         tc_fence_before();  // the reads of O_i precede the next unit's first P.V MMA
         continue;
       }
-      const float inv = 1.0f / l;
+      float inv = 1.0f / l;
+      if constexpr (kF8) inv = p.v_scale / l;
       const uint64_t inv2 = f2pack(inv, inv);
       if (p.warp_stores) {
         // Warp-staged stores: each warp converts its 32 rows one 64-column half
@@ -768,16 +893,16 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attn_kernel(const __grid_const
   }
 }
 
-template <int D, int kRing, bool kSplit = false>
+template <int D, int kRing, bool kSplit = false, bool kF8 = false>
 basa_status launch_impl(TcParams* prm, cudaStream_t stream) {
-  const int smem = Smem<D, kRing>::alloc;
-  static_assert(Smem<D, kRing>::alloc <= 232448, "shared memory plan exceeds 227 KB");
-  if (cudaFuncSetAttribute(tc_attn_kernel<D, kRing, kSplit>,
+  const int smem = Smem<D, kRing, kF8>::alloc;
+  static_assert(Smem<D, kRing, kF8>::alloc <= 232448, "shared memory plan exceeds 227 KB");
+  if (cudaFuncSetAttribute(tc_attn_kernel<D, kRing, kSplit, kF8>,
                            cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
     return BASA_ERR_CUDA;
   long long grid = tc_sm_count();
   if (grid > prm->n_units) grid = prm->n_units;
-  tc_attn_kernel<D, kRing, kSplit><<<(unsigned)grid, kThreads, smem, stream>>>(*prm);
+  tc_attn_kernel<D, kRing, kSplit, kF8><<<(unsigned)grid, kThreads, smem, stream>>>(*prm);
   return cudaGetLastError() == cudaSuccess ? BASA_OK : BASA_ERR_CUDA;
 }
 
@@ -811,7 +936,15 @@ basa_status build_and_launch(TcParams* prm, const Dims& d, bool flat, const void
 
   prm->flags = flags;
   prm->timeout_ns = (unsigned long long)(timeout_ms ? timeout_ms : 2000u) * 1000000ull;
-  prm->scale_log2 = d.scale * 1.4426950408889634f;
+  prm->scale_log2 = d.scale * d.qk_descale * 1.4426950408889634f;
+  prm->v_scale = d.v_descale;
+  // e4m3 inputs: one-byte elements, 128-element (128-byte) boxes per row; the
+  // output stays bf16 with 64-element boxes
+  const bool f8 = d.dtype == BASA_FP8_E4M3;
+  const uint64_t es = f8 ? 1 : 2;
+  const uint32_t inner = f8 ? 128 : 64;
+  const CUtensorMapDataType ity =
+      f8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
   prm->flat = flat ? 1 : 0;
   prm->P = kp ? (int)d.P : 0;
   TilePlan plan;
@@ -820,20 +953,23 @@ basa_status build_and_launch(TcParams* prm, const Dims& d, bool flat, const void
   // and output views hold Nq tokens (the text length for text queries)
   {
     const uint64_t dims[4] = {D, Hk, (uint64_t)d.N, (uint64_t)d.B};  // k, v (and the fill)
-    const uint64_t strides[3] = {D * 2, Hk * D * 2, (uint64_t)d.N * Hk * D * 2};
+    const uint64_t strides[3] = {D * es, Hk * D * es, (uint64_t)d.N * Hk * D * es};
     const uint64_t qdims[4] = {D, H, (uint64_t)d.Nq, (uint64_t)d.B};
-    const uint64_t qstrides[3] = {D * 2, H * D * 2, (uint64_t)d.Nq * H * D * 2};
-    const uint32_t box128[4] = {64, 1, 128, 1};
-    const uint32_t box8[4] = {64, 1, 8, 1};
+    const uint64_t qstrides[3] = {D * es, H * D * es, (uint64_t)d.Nq * H * D * es};
+    const uint64_t ostrides[3] = {D * 2, H * D * 2, (uint64_t)d.Nq * H * D * 2};
+    const uint32_t box128[4] = {inner, 1, 128, 1};
+    const uint32_t obox128[4] = {64, 1, 128, 1};
+    const uint32_t box8[4] = {inner, 1, 8, 1};
     if (flat) {
-      if ((st = encode_map(&prm->qf, q, 4, qdims, qstrides, box128)) != BASA_OK) goto done;
-      if ((st = encode_map(&prm->kf, k, 4, dims, strides, box128)) != BASA_OK) goto done;
-      if ((st = encode_map(&prm->vf, v, 4, dims, strides, box128)) != BASA_OK) goto done;
-      if ((st = encode_map(&prm->of, out, 4, qdims, qstrides, box128)) != BASA_OK) goto done;
+      if ((st = encode_map(&prm->qf, q, 4, qdims, qstrides, box128, ity)) != BASA_OK) goto done;
+      if ((st = encode_map(&prm->kf, k, 4, dims, strides, box128, ity)) != BASA_OK) goto done;
+      if ((st = encode_map(&prm->vf, v, 4, dims, strides, box128, ity)) != BASA_OK) goto done;
+      if ((st = encode_map(&prm->of, out, 4, qdims, ostrides, obox128)) != BASA_OK) goto done;
     } else {
-      if ((st = encode_map(&prm->fill, k, 4, dims, strides, box8)) != BASA_OK) goto done;
+      if ((st = encode_map(&prm->fill, k, 4, dims, strides, box8, ity)) != BASA_OK) goto done;
     }
   }
+  if (kp && f8) { st = BASA_ERR_UNSUPPORTED; goto done; }
   if (kp) {  // extra keys (pooled cells or text tokens) [d, Hkv, P, B]
     const uint64_t pdims[4] = {D, Hk, (uint64_t)d.P, (uint64_t)d.B};
     const uint64_t pstr[3] = {D * 2, Hk * D * 2, (uint64_t)d.P * Hk * D * 2};
@@ -869,17 +1005,20 @@ basa_status build_and_launch(TcParams* prm, const Dims& d, bool flat, const void
   } else {
     if ((st = pack_plan_image(plan, &prm->plan)) != BASA_OK) goto done;
     const uint64_t dims[5] = {D, H, (uint64_t)d.Wg, (uint64_t)d.Hg, (uint64_t)d.B * d.T};
-    const uint64_t strides[4] = {D * 2, H * D * 2, (uint64_t)d.Wg * H * D * 2,
-                                 (uint64_t)d.Hg * d.Wg * H * D * 2};
+    const uint64_t strides[4] = {D * es, H * D * es, (uint64_t)d.Wg * H * D * es,
+                                 (uint64_t)d.Hg * d.Wg * H * D * es};
+    const uint64_t ostrides[4] = {D * 2, H * D * 2, (uint64_t)d.Wg * H * D * 2,
+                                  (uint64_t)d.Hg * d.Wg * H * D * 2};
     const uint64_t kdims[5] = {D, Hk, (uint64_t)d.Wg, (uint64_t)d.Hg, (uint64_t)d.B * d.T};
-    const uint64_t kstrides[4] = {D * 2, Hk * D * 2, (uint64_t)d.Wg * Hk * D * 2,
-                                  (uint64_t)d.Hg * d.Wg * Hk * D * 2};
+    const uint64_t kstrides[4] = {D * es, Hk * D * es, (uint64_t)d.Wg * Hk * D * es,
+                                  (uint64_t)d.Hg * d.Wg * Hk * D * es};
     for (int s = 0; s < plan.n_shapes; ++s) {
-      const uint32_t box[5] = {64, 1, plan.shape_bw[s], plan.shape_bh[s], plan.shape_bt[s]};
-      if ((st = encode_map(&prm->qm[s], q, 5, dims, strides, box)) != BASA_OK) goto done;
-      if ((st = encode_map(&prm->km[s], k, 5, kdims, kstrides, box)) != BASA_OK) goto done;
-      if ((st = encode_map(&prm->vm[s], v, 5, kdims, kstrides, box)) != BASA_OK) goto done;
-      if ((st = encode_map(&prm->om[s], out, 5, dims, strides, box)) != BASA_OK) goto done;
+      const uint32_t box[5] = {inner, 1, plan.shape_bw[s], plan.shape_bh[s], plan.shape_bt[s]};
+      const uint32_t obox[5] = {64, 1, plan.shape_bw[s], plan.shape_bh[s], plan.shape_bt[s]};
+      if ((st = encode_map(&prm->qm[s], q, 5, dims, strides, box, ity)) != BASA_OK) goto done;
+      if ((st = encode_map(&prm->km[s], k, 5, kdims, kstrides, box, ity)) != BASA_OK) goto done;
+      if ((st = encode_map(&prm->vm[s], v, 5, kdims, kstrides, box, ity)) != BASA_OK) goto done;
+      if ((st = encode_map(&prm->om[s], out, 5, dims, ostrides, obox)) != BASA_OK) goto done;
     }
     prm->n_shapes = plan.n_shapes;
     prm->n_qt = plan.n_tiles;
@@ -900,7 +1039,10 @@ basa_status build_and_launch(TcParams* prm, const Dims& d, bool flat, const void
   // 4; everything else reuses K/V tiles from L2 and runs faster with 4.
   // Split key range: its own instantiation, so that the window kernels carry
   // none of its code.
-  if (prm->n_splits > 1)
+  if (f8) {  // d = 128, no extra keys, no split (checked by the entry points)
+    if (d.d != 128 || prm->n_splits > 1 || prm->n_pkt) { st = BASA_ERR_UNSUPPORTED; goto done; }
+    st = launch_impl<128, 4, false, true>(prm, stream);
+  } else if (prm->n_splits > 1)
     st = d.d == 64 ? launch_impl<64, 8, true>(prm, stream) : launch_impl<128, 4, true>(prm, stream);
   else if (d.d == 64)
     st = launch_impl<64, 8>(prm, stream);

@@ -745,3 +745,21 @@ def test_padded_backward_matches_autograd(oracle_mod, shape, window, shift, pool
     o.backward(torch.cat([flat(torch.from_numpy(g)), torch.from_numpy(gt)], 1).transpose(1, 2))
     for gg, t in zip(got, ts):
         np.testing.assert_allclose(gg, t.grad.numpy(), rtol=0, atol=1e-12)
+
+
+def test_e4m3_decoding_matches_the_format_definition():
+    """The e4m3 inputs reach the oracle through torch's exact float8_e4m3fn ->
+    float64 conversion; every one of the 256 codes decodes to the value the OCP
+    e4m3 definition gives: sign bit, 4 exponent bits with bias 7, 3 mantissa
+    bits, subnormals m * 2^-9 for exponent 0, no infinities, NaN only for
+    S.1111.111 (so the largest finite magnitude is 448)."""
+    codes = torch.arange(256, dtype=torch.int32).to(torch.uint8)
+    got = codes.view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    for c in range(256):
+        s, e, m = c >> 7, (c >> 3) & 15, c & 7
+        if e == 15 and m == 7:
+            assert math.isnan(got[c])
+            continue
+        mag = m * 2.0 ** -9 if e == 0 else (1 + m / 8) * 2.0 ** (e - 7)
+        assert got[c] == (-mag if s else mag), c
+    assert np.nanmax(np.abs(got)) == 448.0
