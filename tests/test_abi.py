@@ -250,3 +250,43 @@ def test_joint_workspace_needs_bf16_and_text(lib):
     assert lib.basa_joint_workspace_size(ctypes.byref(_p(window=(1, 5, 5))), 64) == 0
     n = lib.basa_joint_workspace_size(ctypes.byref(_p()), 64)
     assert n % 256 == 0
+
+
+def test_fp8_and_padding_validation(lib):
+    """Host-side checks of e4m3 inputs and padded grids, all refused before any
+    launch (fake pointers are never dereferenced)."""
+    from sparse_attention_diffusion_basa_b200 import BASA_FLAG_PAD_GRID
+    f8 = 2
+    call = lambda prm: lib.basa_window_attn(_fake(), _fake(), _fake(), _fake(), None, None,
+                                            ctypes.byref(prm), None)
+    # e4m3: d = 128 only, no pooled memory, no negative or infinite descale
+    assert call(_p(shape=(1, 1, 16, 16, 2, 64), dtype=f8)) == 3
+    assert call(_p(shape=(1, 1, 16, 16, 2, 128), dtype=f8, pool=(1, 2, 2))) == 3
+    prm = _p(shape=(1, 1, 16, 16, 2, 128), dtype=f8)
+    prm.v_descale = -1.0
+    assert call(prm) == 1
+    prm.v_descale = float("inf")
+    assert call(prm) == 1
+    # e4m3 is refused by every entry point other than window and full attention
+    p8 = _p(shape=(1, 1, 16, 16, 2, 128), dtype=f8)
+    assert lib.basa_window_attn_gm(_fake(), _fake(), _fake(), _fake(), _fake(), _fake(), None,
+                                   ctypes.byref(p8), None) == 3
+    assert lib.basa_pool_kv(_fake(), _fake(), _fake(), _fake(), ctypes.byref(p8), None) == 3
+    assert lib.basa_window_attn_bwd(*[_fake()] * 5, None, *[_fake()] * 3, None,
+                                    ctypes.byref(p8), None) == 3
+    assert lib.basa_joint_attn(*[_fake()] * 6, 4, _fake(), _fake(), None, None, None,
+                               ctypes.byref(p8), None) == 3
+    assert lib.basa_joint_bwd_workspace_size(ctypes.byref(p8), 4) == 0
+    # padded grids: without the flag a shape error, with it the sizes follow N
+    shape = (2, 1, 20, 28, 3, 64)
+    assert call(_p(shape=shape, window=(1, 16, 16), shift=(0, 8, 8))) == 2
+    pp = _p(shape=shape, window=(1, 16, 16), shift=(0, 8, 8))
+    pp.flags = BASA_FLAG_PAD_GRID
+    N = 20 * 28
+    align = lambda x: (x + 255) // 256 * 256
+    assert lib.basa_bwd_workspace_size(ctypes.byref(pp)) == align(2 * 3 * N * 4)
+    assert lib.basa_joint_bwd_workspace_size(ctypes.byref(pp), 77) == \
+        align(2 * 3 * N * 4) + align(2 * 3 * 77 * 4)
+    # the pool cell must still divide the grid
+    pp.ph, pp.pw, pp.pt = 3, 4, 1
+    assert call(pp) == 2

@@ -75,3 +75,23 @@ def test_reference_arm_under_torchrun(tmp_path):
     assert line["value"] > 0 and line["unit"] == "TFLOP/s"
     assert line["cpu_baseline"]["kind"] == "oracle"
     assert line["e2e"]["h2d_bytes_per_step"] == 0
+
+
+def test_workload_byte_and_flop_accounting():
+    """The bench's algorithmic figures: q, k, v read and out written once (e4m3
+    inputs at one byte, their bf16 output at two), and 4·B·H·d flops per
+    (query, key) pair that the method computes."""
+    sys.path.insert(0, ROOT)
+    import bench
+    from basa_synth import WORKLOADS
+    w16, w8 = WORKLOADS["flux2048"], WORKLOADS["flux2048_e4m3"]
+    f16, b16, N, m, P, theo = bench.workload_numbers(w16, (0, 8, 8))
+    f8, b8, *_ = bench.workload_numbers(w8, (0, 8, 8))
+    assert b16 == 4 * 24 * 16384 * 128 * 2
+    assert b8 == 24 * 16384 * 128 * (3 * 1 + 2)
+    assert f16 == f8 == 4.0 * 24 * 128 * 16384 * 256
+    assert theo == 16384 / 256
+    fj, bj, N, m, P, theo = bench.workload_numbers(WORKLOADS["flux1024_text512"], (0, 8, 8))
+    L = 512
+    assert fj == 4.0 * 24 * 128 * (4096 * (256 + L) + L * (4096 + L))
+    assert bj == 4 * 24 * (4096 + L) * 128 * 2
