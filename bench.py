@@ -204,11 +204,29 @@ def time_steps(fn, steps, flush, sleep_us=200.0):
     return [a.elapsed_time(b) for a, b in ev]
 
 
+def _head(x, h):
+    """Batch 0, head h of an image [B, T, Hg, Wg, H, d] or text [B, L, H, d] tensor."""
+    return np.ascontiguousarray(x[:1, ..., h:h + 1, :])
+
+
 def run_oracle_sample(w, shift, q, k, v, heads, threads=0):
-    """Oracle on all queries of `heads` heads (batch 0); returns (seconds, flops)."""
+    """Oracle on all queries of `heads` heads (batch 0); returns (seconds, flops).
+    Joint workloads: every image and text query of each sampled head."""
     import oracle
     B, T, Hg, Wg, H, d = w.shape()
     N = w.N
+    if w.text:
+        L = w.text
+        qt, kt, vt = (oracle.as_f64(x) for x in text_inputs(w, len(w.shifts) - 1))
+        qf, kf, vf = oracle.as_f64(q), oracle.as_f64(k), oracle.as_f64(v)
+        prm = oracle.OracleParams(1, T, Hg, Wg, 1, d, w.window, shift)
+        dt = 0.0
+        for h in heads:
+            args = [_head(x, h) for x in (qf, kf, vf, qt, kt, vt)]
+            t0 = time.perf_counter()
+            oracle.joint_attn(*args, prm, threads=threads)
+            dt += time.perf_counter() - t0
+        return dt, 4.0 * len(heads) * (N * (w.m + L) + L * (N + L)) * d
     sel = np.array([[0, n, h] for h in heads for n in range(N)], dtype=np.int64)
     prm = oracle.OracleParams(B, T, Hg, Wg, H, d, w.window, shift, w.pool)
     qf, kf, vf = oracle.as_f64(q), oracle.as_f64(k), oracle.as_f64(v)
@@ -220,6 +238,28 @@ def run_oracle_sample(w, shift, q, k, v, heads, threads=0):
     oracle.window_attn(qf, kf, vf, prm, kp=kp, vp=vp, select=sel, threads=threads)
     dt = time.perf_counter() - t0
     return dt, 4.0 * len(sel) * (w.m + w.P) * d
+
+
+def run_oracle_bwd_sample(w, shift, q, k, v, h):
+    """The oracle's backward (gradients of every input) for batch 0, head h;
+    returns (seconds, flops).  Joint workloads: image and text gradients."""
+    import oracle
+    B, T, Hg, Wg, H, d = w.shape()
+    N, L = w.N, w.text
+    rng = np.random.Generator(np.random.PCG64(7))
+    qf, kf, vf = (_head(oracle.as_f64(x), h) for x in (q, k, v))
+    g = rng.standard_normal(qf.shape)
+    prm = oracle.OracleParams(1, T, Hg, Wg, 1, d, w.window, shift, w.pool)
+    t0 = time.perf_counter()
+    if L:
+        qt, kt, vt = (_head(oracle.as_f64(x), h) for x in text_inputs(w, len(w.shifts) - 1))
+        gt = rng.standard_normal(qt.shape)
+        t0 = time.perf_counter()
+        oracle.joint_attn_bwd(qf, kf, vf, qt, kt, vt, g, gt, prm)
+    else:
+        oracle.window_attn_bwd(qf, kf, vf, g, prm)
+    dt = time.perf_counter() - t0
+    return dt, 10.0 * (N * (w.m + w.P + L) + L * (N + L)) * d
 
 
 def cpu_baseline(w, shift, q, k, v, budget_s=12.0):
@@ -236,8 +276,9 @@ def cpu_baseline(w, shift, q, k, v, budget_s=12.0):
         dti, fli = run_oracle_sample(w, shift, q, k, v, heads)
         dt, fl, reps = dt + dti, fl + fli, reps + 1
     return {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
-            "sample": f"all {w.N} queries of {nheads} of {w.H} heads, batch 0, shift {shift}, "
-                      f"{reps} run(s); {dt:.2f} s fp64 on {cores} host threads"}
+            "sample": f"all {w.N} queries of {nheads} of {w.H} heads, batch 0, shift {shift}"
+                      + (f", with the {w.text} text queries of those heads" if w.text else "")
+                      + f", {reps} run(s); {dt:.2f} s fp64 on {cores} host threads"}
 
 
 def main_backward(args, world, rank, local):
@@ -378,22 +419,32 @@ def main_reference(args, world, rank):
     q, k, v = workload_inputs(w, len(w.shifts) - 1)
     cores = oracle.max_threads()
     flops_step = 0.0
+    if args.backward:  # the backward arm: the oracle's gradients, single-threaded C
+        sample = lambda: run_oracle_bwd_sample(w, shift, q, k, v, 0)
+        metric, cores = "window-attn backward latency (ms) & TFLOP/s", 1
+        what = (f"gradients of every input, head 0 of {w.H}, batch 0, per step"
+                + (f" (with its {w.text} text tokens)" if w.text else ""))
+    else:
+        sample = lambda: run_oracle_sample(w, shift, q, k, v, [0])
+        metric = METRIC
+        what = (f"all {w.N} queries of head 0 of {w.H}, batch 0, per step"
+                + (f", and its {w.text} text queries" if w.text else ""))
     for _ in range(args.warmup):
-        run_oracle_sample(w, shift, q, k, v, [0])
+        sample()
     times = []
     for _ in range(args.steps):
-        dt, fl = run_oracle_sample(w, shift, q, k, v, [0])
+        dt, fl = sample()
         times.append(dt)
         flops_step = fl
     total = sum(times)
     val = flops_step * args.steps / total / 1e12
-    line = {"impl": "reference", "metric": METRIC, "value": val, "unit": "TFLOP/s",
+    line = {"impl": "reference", "metric": metric, "value": val, "unit": "TFLOP/s",
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": 1e3 * total / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": arm_config(w, shift, world),
             "cpu_baseline": {"value": val, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
-                             "sample": f"all {w.N} queries of head 0 of {w.H}, batch 0, per step"},
+                             "sample": what},
             "e2e": {"value": val, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)

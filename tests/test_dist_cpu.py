@@ -95,3 +95,19 @@ def test_workload_byte_and_flop_accounting():
     L = 512
     assert fj == 4.0 * 24 * 128 * (4096 * (256 + L) + L * (4096 + L))
     assert bj == 4 * 24 * (4096 + L) * 128 * 2
+
+
+def test_reference_arm_backward_and_joint(tmp_path):
+    """The reference arm times the oracle's backward under --backward, and the
+    joint forward (image and text queries) for a joint workload."""
+    def run(*extra):
+        r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                            "--steps", "1", "--warmup", "1", *extra],
+                           capture_output=True, text=True, timeout=600, cwd=ROOT)
+        assert r.returncode == 0, r.stderr[-2000:]
+        return json.loads(r.stdout.strip().splitlines()[-1])
+    j = run("--backward", "--workload", "grid16_f32")
+    assert j["impl"] == "reference" and j["metric"].startswith("window-attn backward")
+    assert j["value"] > 0 and j["cpu_baseline"]["cores"] == 1
+    j = run("--workload", "flux1024_text512")
+    assert "text queries" in j["cpu_baseline"]["sample"] and j["value"] > 0
