@@ -346,21 +346,20 @@ def main_backward(args, world, rank, local):
                 "frac": gbs / peaks["hbm_gbs"]}
     roof.update({"peak_source": peaks["source"] + " (MEASURED_PEAKS.json, burst)",
                  "traffic": None, "roofline_ms": 1e3 * max(t_tensor, t_hbm),
-                 "kernel": ("whole joint backward on CUDA cores: bwd_prep (image, text rows), "
-                            "bwd_dkv_kernel (text keys), bwd_dq_kernel (image, text queries), "
-                            "bwd_dkv_kernel (window keys)") if L else
+                 "kernel": ("whole joint backward: bwd_prep (image, text rows), tc_bwd_kernel "
+                            "(text keys' dK, dV; image dQ; text dQ; window dK, dV), "
+                            "text_grad_round_kernel") if L else
                            ("whole backward: bwd_prep, tc_bwd_kernel (dQ), tc_bwd_kernel (dK, dV)"
                             + (", pool_kernel, tc_bwd_kernel (pooled dK, dV)" if w.P else ""))})
     line = {"metric": "window-attn backward latency (ms) & TFLOP/s", "value": world * tflops,
             "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": ("bf16 (CUDA cores, fp32 arithmetic)" if L else
-                      "bf16 (tensor cores, fp32 accumulate)") if w.dtype == "bf16" else w.dtype,
+            "dtype": "bf16 (tensor cores, fp32 accumulate)" if w.dtype == "bf16" else w.dtype,
             "data": "synthetic",
             "config": {"workload": f"{w.name} backward", "N": w.N, "m": w.m, "P": w.P, "L": L,
                        "l2": "evicted before every step (256 MiB write, then 256 MiB read; outside the events)"},
             "roofline": roof,
-            "gpu_launches": (6 if L else 5 if w.P else 3) * args.steps, "clocks": clk}
+            "gpu_launches": (7 if L else 5 if w.P else 3) * args.steps, "clocks": clk}
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:

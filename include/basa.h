@@ -251,8 +251,10 @@ BASA_API size_t basa_bwd_workspace_size(const basa_params* p);
  * (the text keys over every image and text query).  Image tensors
  * [B, T, Hg, Wg, H or Hkv, d], text tensors [B, L, H or Hkv, d]; lse, lse_t from
  * the forward call; workspace: basa_joint_bwd_workspace_size(p, L) bytes,
- * 16-byte aligned.  fp32 arithmetic on CUDA cores for both dtypes, gradients
- * rounded once.  L = 0 is basa_window_attn_bwd.  A pool cell in p gives
+ * 16-byte aligned.  bf16 (d = 64 or 128, grids the window divides): tensor
+ * cores, with P and dS rounded to bf16 as MMA operands and the text keys' sums
+ * in fp32; fp32, or BASA_FLAG_BWD_CUDA_CORES, or shapes outside those bounds:
+ * fp32 arithmetic on CUDA cores.  Gradients rounded once.  L = 0 is basa_window_attn_bwd.  A pool cell in p gives
  * BASA_ERR_UNSUPPORTED.  Launches on `stream` only; nothing is allocated.
  */
 BASA_API size_t basa_joint_bwd_workspace_size(const basa_params* p, int64_t L);
