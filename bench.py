@@ -275,10 +275,18 @@ def cpu_baseline(w, shift, q, k, v, budget_s=12.0):
     while nheads == w.H and dt < budget_s * 0.75 and reps < 16:
         dti, fli = run_oracle_sample(w, shift, q, k, v, heads)
         dt, fl, reps = dt + dti, fl + fli, reps + 1
-    return {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
-            "sample": f"all {w.N} queries of {nheads} of {w.H} heads, batch 0, shift {shift}"
-                      + (f", with the {w.text} text queries of those heads" if w.text else "")
-                      + f", {reps} run(s); {dt:.2f} s fp64 on {cores} host threads"}
+    res = {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+           "sample": f"all {w.N} queries of {nheads} of {w.H} heads, batch 0, shift {shift}"
+                     + (f", with the {w.text} text queries of those heads" if w.text else "")
+                     + f", {reps} run(s); {dt:.2f} s fp64 on {cores} host threads"}
+    # the same oracle on one host thread, on one head, where that takes a few
+    # seconds at most (the small and the FLUX image workloads)
+    if fl1 <= 3e9:
+        dt1t, fl1t = run_oracle_sample(w, shift, q, k, v, [0], threads=1)
+        res["one_thread"] = {"value": fl1t / dt1t / 1e12, "unit": "TFLOP/s", "cores": 1,
+                             "sample": f"all {w.N} queries of head 0, batch 0; {dt1t:.2f} s fp64"
+                                       " on 1 host thread"}
+    return res
 
 
 def main_backward(args, world, rank, local):
@@ -346,21 +354,20 @@ def main_backward(args, world, rank, local):
                 "frac": gbs / peaks["hbm_gbs"]}
     roof.update({"peak_source": peaks["source"] + " (MEASURED_PEAKS.json, burst)",
                  "traffic": None, "roofline_ms": 1e3 * max(t_tensor, t_hbm),
-                 "kernel": ("whole joint backward on CUDA cores: bwd_prep (image, text rows), "
-                            "bwd_dkv_kernel (text keys), bwd_dq_kernel (image, text queries), "
-                            "bwd_dkv_kernel (window keys)") if L else
+                 "kernel": ("whole joint backward: bwd_prep (image, text rows), tc_bwd_kernel "
+                            "(text keys' dK, dV; image dQ; text dQ; window dK, dV), "
+                            "text_grad_round_kernel") if L else
                            ("whole backward: bwd_prep, tc_bwd_kernel (dQ), tc_bwd_kernel (dK, dV)"
                             + (", pool_kernel, tc_bwd_kernel (pooled dK, dV)" if w.P else ""))})
     line = {"metric": "window-attn backward latency (ms) & TFLOP/s", "value": world * tflops,
             "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": ("bf16 (CUDA cores, fp32 arithmetic)" if L else
-                      "bf16 (tensor cores, fp32 accumulate)") if w.dtype == "bf16" else w.dtype,
+            "dtype": "bf16 (tensor cores, fp32 accumulate)" if w.dtype == "bf16" else w.dtype,
             "data": "synthetic",
             "config": {"workload": f"{w.name} backward", "N": w.N, "m": w.m, "P": w.P, "L": L,
                        "l2": "evicted before every step (256 MiB write, then 256 MiB read; outside the events)"},
             "roofline": roof,
-            "gpu_launches": (6 if L else 5 if w.P else 3) * args.steps, "clocks": clk}
+            "gpu_launches": (7 if L else 5 if w.P else 3) * args.steps, "clocks": clk}
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -625,8 +632,8 @@ def main():
     line = {
         "metric": METRIC, "value": tflops, "unit": "TFLOP/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max,
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-        "data": "synthetic",
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": w.dtype, "data": "synthetic",
         "config": arm_config(w, shift, world),
         "latency_ms": ms_max,
         # this rank's spread over the timed steps (the mean is latency_ms)
@@ -648,7 +655,7 @@ def main():
         "gpu_launches": args.steps * (2 if (w.P or L) else 1),
         "clocks": clk,
     }
-    if rank == 0 and world == 1 and not args.no_cpu_baseline and not L:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w, shift, q, k, v)
     if rank == 0:
         print(json.dumps(line), flush=True)

@@ -218,8 +218,9 @@ BASA_API basa_status basa_joint_attn(const void* q, const void* k, const void* v
 BASA_API size_t basa_joint_workspace_size(const basa_params* p, int64_t L);
 
 /*
- * Backward of shifted window attention (no global memory): the gradients dq,
- * dk, dv of basa_window_attn's output for the output gradient dout.  The
+ * Backward of shifted window attention, with or without pooled global memory:
+ * the gradients dq, dk, dv of basa_window_attn's output for the output
+ * gradient dout.  The
  * dense-teacher adaptation on the pages ("BASA: Backend-Agnostic Sparse
  * Attention for Fast High-Resolution Diffusion Transformers", zhichai.net topic
  * 178635722, forum review reply 178634520) trains through this attention.
@@ -251,8 +252,10 @@ BASA_API size_t basa_bwd_workspace_size(const basa_params* p);
  * (the text keys over every image and text query).  Image tensors
  * [B, T, Hg, Wg, H or Hkv, d], text tensors [B, L, H or Hkv, d]; lse, lse_t from
  * the forward call; workspace: basa_joint_bwd_workspace_size(p, L) bytes,
- * 16-byte aligned.  fp32 arithmetic on CUDA cores for both dtypes, gradients
- * rounded once.  L = 0 is basa_window_attn_bwd.  A pool cell in p gives
+ * 16-byte aligned.  bf16 (d = 64 or 128, grids the window divides): tensor
+ * cores, with P and dS rounded to bf16 as MMA operands and the text keys' sums
+ * in fp32; fp32, or BASA_FLAG_BWD_CUDA_CORES, or shapes outside those bounds:
+ * fp32 arithmetic on CUDA cores.  Gradients rounded once.  L = 0 is basa_window_attn_bwd.  A pool cell in p gives
  * BASA_ERR_UNSUPPORTED.  Launches on `stream` only; nothing is allocated.
  */
 BASA_API size_t basa_joint_bwd_workspace_size(const basa_params* p, int64_t L);
@@ -289,12 +292,15 @@ BASA_API basa_status basa_full_attn(const void* q, const void* k, const void* v,
  * the library's device code.
  *  - Every GPU that loads the library's device code holds that array until the
  *    process exits.
- *  - If pooled K and V together need more than 32 MiB (each [B, P, H, d] of
- *    p->dtype, rounded up to 256 bytes), the call returns
- *    BASA_ERR_SCRATCH_LIMIT and enqueues nothing.
+ *  - If pooled K and V together need more than 32 MiB (each [B, P, Hkv, d] of
+ *    p->dtype, Hkv = p->Hkv or H when it is 0, rounded up to 256 bytes), the
+ *    call returns BASA_ERR_SCRATCH_LIMIT and enqueues nothing.
  *  - The first call with a given device current looks up the array's device
- *    address (cudaGetSymbolAddress) and caches it; that first call should be
- *    made before any stream capture begins.
+ *    address (cudaGetSymbolAddress) and caches it together with the id of the
+ *    current CUDA context; that first call should be made before any stream
+ *    capture begins.  A call in a new context on the same device (after
+ *    cudaDeviceReset, for instance) looks the address up again, so it too
+ *    should come before any capture in that context.
  *  - All calls on a device share the array: calls whose work overlaps on the
  *    GPU (e.g. on unordered streams) race on it and must be ordered by the
  *    caller.  Nothing in it needs to start at zero: each call overwrites every

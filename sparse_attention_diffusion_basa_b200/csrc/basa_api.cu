@@ -5,18 +5,9 @@
 
 #include <mutex>
 
-#include <nvtx3/nvToolsExt.h>
-
 #include "basa_internal.h"
 
 namespace basa {
-
-// An NVTX range over one library call, so that profilers show each call's
-// launches under its name (a pointer check when no tool is attached).
-struct NvtxRange {
-  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
-  ~NvtxRange() { nvtxRangePop(); }
-};
 
 static int floor_mod(long long a, int n) {
   long long r = a % n;
@@ -417,11 +408,22 @@ basa_status basa_window_attn_bwd(const void* q, const void* k, const void* v, co
   return launch_bwd(d, q, k, v, out, dout, lse, dD, dq, dk, dv, pgp, stream);
 }
 
+// D of the image rows, D of the text rows, and the text keys' fp32 dK, dV sums.
+static size_t joint_bwd_parts(const Dims& d, int64_t L, size_t* off_dt, size_t* off_kp,
+                              size_t* off_vp) {
+  const size_t dd = align256((size_t)d.B * d.H * d.N * sizeof(float));
+  const size_t dt = align256((size_t)d.B * d.H * (size_t)L * sizeof(float));
+  const size_t kp = align256((size_t)d.B * (size_t)L * d.Hkv * d.d * sizeof(float));
+  if (off_dt) *off_dt = dd;
+  if (off_kp) *off_kp = dd + dt;
+  if (off_vp) *off_vp = dd + dt + kp;
+  return dd + dt + 2 * kp;
+}
+
 size_t basa_joint_bwd_workspace_size(const basa_params* p, int64_t L) {
   Dims d;
   if (L < 0 || L > (1LL << 24) || normalise(p, false, &d) != BASA_OK) return 0;
-  return align256((size_t)d.B * d.H * d.N * sizeof(float)) +
-         align256((size_t)d.B * d.H * (size_t)L * sizeof(float));
+  return joint_bwd_parts(d, L, nullptr, nullptr, nullptr);
 }
 
 basa_status basa_joint_attn_bwd(const void* q, const void* k, const void* v, const void* qt,
@@ -447,10 +449,18 @@ basa_status basa_joint_attn_bwd(const void* q, const void* k, const void* v, con
   if (!lse || !lse_t) return BASA_ERR_INVALID_ARG;
   if (!workspace) return BASA_ERR_WORKSPACE;
   if (misaligned(workspace)) return BASA_ERR_ALIGN;
-  float* dD = static_cast<float*>(workspace);
-  float* dD_t = reinterpret_cast<float*>(static_cast<char*>(workspace) +
-                                         align256((size_t)d.B * d.H * d.N * sizeof(float)));
+  size_t off_dt, off_kp, off_vp;
+  joint_bwd_parts(d, L, &off_dt, &off_kp, &off_vp);
+  char* ws = static_cast<char*>(workspace);
+  float* dD = reinterpret_cast<float*>(ws);
+  float* dD_t = reinterpret_cast<float*>(ws + off_dt);
   const JointGrads jg{qt, kt, vt, out_t, dout_t, lse_t, dD_t, dqt, dkt, dvt, (long long)L};
+  if (d.dtype == BASA_BF16 && !(p->flags & BASA_FLAG_BWD_CUDA_CORES)) {
+    s = launch_bwd_tc_joint(d, q, k, v, out, dout, lse, dD, dq, dk, dv, jg,
+                            reinterpret_cast<float*>(ws + off_kp),
+                            reinterpret_cast<float*>(ws + off_vp), p->wait_timeout_ms, stream);
+    if (s != BASA_ERR_UNSUPPORTED) return s;
+  }
   return launch_bwd_joint(d, q, k, v, out, dout, lse, dD, dq, dk, dv, jg, stream);
 }
 

@@ -5,9 +5,20 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "basa.h"
 
 namespace basa {
+
+// An NVTX range over one library call, so that profilers show each call's
+// launches under its name (a pointer check when no tool is attached).
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
 
 // ---------------------------------------------------------------------------
 // Normalised call description (after validation).
@@ -171,6 +182,15 @@ basa_status launch_bwd_tc(const Dims& d, const void* q, const void* k, const voi
                           const void* out, const void* dout, const float* lse, float* dD,
                           void* dq, void* dk, void* dv, const PoolGrads* pg, uint32_t timeout_ms,
                           cudaStream_t stream);
+
+// bf16 joint text + image backward on the tensor cores: D of the image rows
+// into dD and of the text rows into jg.dD_t, the text keys' fp32 sums in dkp,
+// dvp ([B, L, Hkv, d] each), then every gradient.  BASA_ERR_UNSUPPORTED,
+// before any launch, outside the tensor-core kernels' bounds.
+basa_status launch_bwd_tc_joint(const Dims& d, const void* q, const void* k, const void* v,
+                                const void* out, const void* dout, const float* lse, float* dD,
+                                void* dq, void* dk, void* dv, const JointGrads& jg, float* dkp,
+                                float* dvp, uint32_t timeout_ms, cudaStream_t stream);
 
 // The same launch with its parameter block in static storage (no host heap use);
 // calls are serialised by a lock held until the launch has copied the block.

@@ -35,20 +35,59 @@ constexpr int kMaxDevices = 64;
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
 std::mutex g_setup_mu;
-void* g_scratch_addr[kMaxDevices];  // device address of g_noalloc_scratch, per device
+// Device address of g_noalloc_scratch per device, and the id of the CUDA
+// context it was resolved in: a new context on the device (after
+// cudaDeviceReset, say) loads the module afresh, and the array may then sit
+// at another address.
+void* g_scratch_addr[kMaxDevices];
+unsigned long long g_scratch_ctx[kMaxDevices];
 
-// Device address of the scratch array on the current device; resolved once per
-// device, on the first call made with that device current.
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long*);
+
+// Unique id of the calling thread's current CUDA context (driver entry points,
+// so the library links no driver library), or 0 if it cannot be read.
+unsigned long long current_context_id() {
+  static CtxGetCurrentFn get_current = nullptr;
+  static CtxGetIdFn get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* a = nullptr;
+    void* b = nullptr;
+    cudaDriverEntryPointQueryResult qa, qb;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &a, cudaEnableDefault, &qa) == cudaSuccess &&
+        qa == cudaDriverEntryPointSuccess &&
+        cudaGetDriverEntryPoint("cuCtxGetId", &b, cudaEnableDefault, &qb) == cudaSuccess &&
+        qb == cudaDriverEntryPointSuccess) {
+      get_current = reinterpret_cast<CtxGetCurrentFn>(a);
+      get_id = reinterpret_cast<CtxGetIdFn>(b);
+    }
+  });
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (!get_current || !get_id || get_current(&ctx) != CUDA_SUCCESS || !ctx ||
+      get_id(ctx, &id) != CUDA_SUCCESS)
+    return 0;
+  return id;
+}
+
+// Device address of the scratch array on the current device; resolved on the
+// first call made with that device current, and again whenever the current
+// context is not the one the cached address belongs to.
 basa_status scratch_address(void** out) {
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess) return BASA_ERR_CUDA;
   if (dev < 0 || dev >= kMaxDevices) return BASA_ERR_UNSUPPORTED;
+  const unsigned long long ctx = current_context_id();
   std::lock_guard<std::mutex> lock(g_setup_mu);
-  if (!g_scratch_addr[dev]) {
+  if (!g_scratch_addr[dev] || ctx == 0 || ctx != g_scratch_ctx[dev]) {
+    // the lookup also makes the device's primary context current if the
+    // runtime had not done so yet, so the context id is read after it
     void* ptr = nullptr;
     if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || !ptr)
       return BASA_ERR_CUDA;
     g_scratch_addr[dev] = ptr;
+    g_scratch_ctx[dev] = current_context_id();
   }
   *out = g_scratch_addr[dev];
   return BASA_OK;
@@ -64,6 +103,7 @@ using namespace basa;
 extern "C" basa_status basa_window_attn_noalloc(const void* q, const void* k, const void* v,
                                                 void* out, float* lse, const basa_params* p,
                                                 cudaStream_t stream) {
+  NvtxRange nvtx("basa_window_attn_noalloc");
   Dims d;
   basa_status s = normalise(p, false, &d);
   if (s != BASA_OK) return s;

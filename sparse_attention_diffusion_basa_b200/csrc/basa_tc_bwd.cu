@@ -97,12 +97,26 @@ struct __align__(64) BwdTcParams {
   int pt, ph, pw;
   float inv_count;               // 1 / (pt * ph * pw)
   long long q_elems, kv_elems;   // elements of dq and of dk, dv (checked build)
+  // joint text + image (joint = 1): the L text tokens take the pooled slots
+  // (kpf, vpf over kt, vt; dkp, dvp their fp32 sums; no share to the window
+  // rows), their queries are n_tt more flat query tiles of the pooled and the
+  // window dK, dV modes, and the text dQ mode walks every image key tile
+  // (kf, vf) and then the text key tiles
+  int joint;
+  int n_tt;                      // text tiles (128 rows)
+  long long L;
+  CUtensorMap qtf, gtf;          // qt, dout_t as flat rows: [d, H, L, B]
+  CUtensorMap kf, vf;            // k, v as flat rows: [d, Hkv, N, B]
+  const float* lse_t;            // [B, H, L]
+  const float* dD_t;             // [B, H, L]
+  __nv_bfloat16* dqt;            // [B, L, H, d]
+  long long qt_elems;            // elements of dqt (checked build)
 };
 
 // Kernel modes: the dQ kernel (window key tiles, then the pooled tiles), the
 // window dK, dV kernel, and the pooled dK, dV kernel (a pooled key tile against
 // a range of the grid's query tiles, summed into dkp, dvp).
-constexpr int kModeDq = 0, kModeDkv = 1, kModePooled = 2;
+constexpr int kModeDq = 0, kModeDkv = 1, kModePooled = 2, kModeDqText = 3;
 
 // Shared memory: the unit pair, a two-slot ring of step pairs, 2 KB of output
 // staging per epilogue warp, the per-row lse/D values of each ring slot (the dQ
@@ -141,8 +155,18 @@ struct BwdUnit {
 // head, the pooled tile, the query-tile split, the batch).
 template <int MODE>
 __device__ __forceinline__ BwdUnit decode_bwd_unit(const BwdTcParams& p, uint32_t u) {
-  constexpr bool KV = MODE != kModeDq;
+  constexpr bool KV = MODE == kModeDkv || MODE == kModePooled;
   BwdUnit U;
+  if constexpr (MODE == kModeDqText) {  // (b, h, text tile): heads fastest
+    U.h = (int)(u % (uint32_t)p.H);
+    U.hk = U.h / p.group;
+    const uint32_t r = u / (uint32_t)p.H;
+    U.tile = (int)(r % (uint32_t)p.n_tt);
+    U.w.b = (int)(r / (uint32_t)p.n_tt);
+    U.w.cls = U.w.ot = U.w.oh = U.w.ow = 0;
+    U.q0 = U.nq = 0;
+    return U;
+  }
   if constexpr (MODE == kModePooled) {
     U.hk = (int)(u % (uint32_t)p.Hkv);
     U.h = U.hk * p.group;
@@ -153,7 +177,7 @@ __device__ __forceinline__ BwdUnit decode_bwd_unit(const BwdTcParams& p, uint32_
     U.w.b = (int)(r / (uint32_t)p.n_fsplits);
     U.w.cls = U.w.ot = U.w.oh = U.w.ow = 0;
     U.q0 = sp * p.fqt_per_split;
-    const int left = p.n_fqt - U.q0;
+    const int left = p.n_fqt + (p.joint ? p.n_tt : 0) - U.q0;  // joint: image, then text tiles
     U.nq = left < p.fqt_per_split ? left : p.fqt_per_split;
     return U;
   }
@@ -181,14 +205,22 @@ __device__ __forceinline__ BwdUnit decode_bwd_unit(const BwdTcParams& p, uint32_
   return U;
 }
 
-// Steps of unit U: dQ, the window's key tiles then the pooled tiles; dKV, the
-// group's query heads times the window's query tiles; pooled, the group's query
-// heads times the unit's query tiles.
+// Query tiles per query head of a dK, dV unit: the window's (then, joint, the
+// text tiles); pooled: the unit's range of the flat query tiles.
+template <int MODE>
+__device__ __forceinline__ int bwd_per_head(const BwdTcParams& p, const BwdUnit& U) {
+  if constexpr (MODE == kModePooled) return U.nq;
+  return p.n_tiles + (p.joint ? p.n_tt : 0);
+}
+
+// Steps of unit U: dQ, the window's key tiles then the pooled (text) tiles;
+// text dQ, every image key tile then the text tiles; dKV, the group's query
+// heads times the query tiles per head; pooled, the same over the unit's range.
 template <int MODE>
 __device__ __forceinline__ int bwd_steps(const BwdTcParams& p, const BwdUnit& U) {
   if constexpr (MODE == kModeDq) return p.n_tiles + p.n_pt;
-  if constexpr (MODE == kModeDkv) return p.group * p.n_tiles;
-  return p.group * U.nq;
+  if constexpr (MODE == kModeDqText) return p.n_fqt + p.n_tt;
+  return p.group * bwd_per_head<MODE>(p, U);
 }
 
 // lse * log2(e) and D of the 128 rows of query tile `tile` of head h into
@@ -212,18 +244,22 @@ __device__ __forceinline__ void write_row_values(const BwdTcParams& p, const Pla
   }
 }
 
-// The same for flat query tile i of the grid (rows 128 i .. 128 i + 127).
+// The same for flat query tile i of the grid (rows 128 i .. 128 i + 127), or
+// (text) of the text queries.
 __device__ __forceinline__ void write_row_values_flat(const BwdTcParams& p, int b, int i, int h,
-                                                      float* dst, int lane) {
+                                                      float* dst, int lane, bool text = false) {
+  const long long nrows = text ? p.L : p.N;
+  const float* lse = text ? p.lse_t : p.lse;
+  const float* dD = text ? p.dD_t : p.dD;
 #pragma unroll 1
   for (int k = 0; k < 4; ++k) {
     const int r = lane + 32 * k;
     const long long n = 128LL * i + r;
     float l2 = INFINITY, dd = 0.f;
-    if (n < p.N) {
-      const long long x = ((long long)b * p.H + h) * p.N + n;
-      l2 = p.lse[x] * kLog2e;
-      dd = p.dD[x];
+    if (n < nrows) {
+      const long long x = ((long long)b * p.H + h) * nrows + n;
+      l2 = lse[x] * kLog2e;
+      dd = dD[x];
     }
     dst[r] = l2;
     dst[128 + r] = dd;
@@ -266,7 +302,8 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
     tc_bwd_kernel(const __grid_constant__ BwdTcParams p) {
   using S = BwdSmem<D>;
   constexpr int NH = D / 64;
-  constexpr bool KV = MODE != kModeDq;  // dK, dV accumulators (window or pooled keys)
+  // dK, dV accumulators (window or pooled / text keys); else dQ (image or text queries)
+  constexpr bool KV = MODE == kModeDkv || MODE == kModePooled;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -315,6 +352,8 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
     prefetch_tmap(&p.fill);
     if (p.P) { prefetch_tmap(&p.kpf); prefetch_tmap(&p.vpf); }
     if (MODE == kModePooled) { prefetch_tmap(&p.qf); prefetch_tmap(&p.gf); }
+    if (p.joint) { prefetch_tmap(&p.qtf); prefetch_tmap(&p.gtf); }
+    if (MODE == kModeDqText) { prefetch_tmap(&p.kf); prefetch_tmap(&p.vf); }
   }
 
   if (warp == 0) {
@@ -324,7 +363,7 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
     for (uint32_t u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
       const BwdUnit U = decode_bwd_unit<MODE>(p, u);
       const int n_steps = bwd_steps<MODE>(p, U);
-      const int per_head = MODE == kModePooled ? U.nq : p.n_tiles;
+      const int per_head = bwd_per_head<MODE>(p, U);
       for (int s = 0; s < n_steps && ok; ++s) {
         const uint32_t slot = nb & 1u, par = (nb >> 1) & 1u;
         if (!(ok = wait_warp(BAR(S::BEMPTY + slot), par ^ 1u, abort_flag, limit, kBSiteLoadBEmpty)))
@@ -333,14 +372,36 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
         const uint32_t bar = BAR(S::BFULL + slot);
         const int h = KV ? U.h + s / per_head : U.h;  // dKV: the step's query head
         const int tile = KV ? s % per_head : s;
+        // pooled (joint): flat query tile U.q0 + tile, past the grid's tiles
+        // a text tile; dKV (joint): query tiles past the window's are text tiles
+        const int ftile = U.q0 + tile;
+        const bool text_q = (MODE == kModePooled && ftile >= p.n_fqt) ||
+                            (MODE == kModeDkv && tile >= p.n_tiles);
+        const int ttile = MODE == kModePooled ? ftile - p.n_fqt : tile - p.n_tiles;
         if (lane == 0) {
           mbar_expect_tx(bar, 2 * S::kTile);
-          if (MODE == kModePooled) {  // flat query tile U.q0 + tile of the grid
+          if (text_q) {  // text query tile: Qt, dOt
 #pragma unroll
             for (int hf = 0; hf < NH; ++hf) {
-              tma_load_4d(dst + hf * kHalf, &p.qf, bar, hf * 64, h, (U.q0 + tile) * 128, U.w.b);
-              tma_load_4d(dst + S::kTile + hf * kHalf, &p.gf, bar, hf * 64, h,
-                          (U.q0 + tile) * 128, U.w.b);
+              tma_load_4d(dst + hf * kHalf, &p.qtf, bar, hf * 64, h, ttile * 128, U.w.b);
+              tma_load_4d(dst + S::kTile + hf * kHalf, &p.gtf, bar, hf * 64, h, ttile * 128,
+                          U.w.b);
+            }
+          } else if (MODE == kModePooled) {  // flat query tile U.q0 + tile of the grid
+#pragma unroll
+            for (int hf = 0; hf < NH; ++hf) {
+              tma_load_4d(dst + hf * kHalf, &p.qf, bar, hf * 64, h, ftile * 128, U.w.b);
+              tma_load_4d(dst + S::kTile + hf * kHalf, &p.gf, bar, hf * 64, h, ftile * 128,
+                          U.w.b);
+            }
+          } else if (MODE == kModeDqText) {  // every image key tile, then the text tiles
+            const bool img = tile < p.n_fqt;
+            const int row = (img ? tile : tile - p.n_fqt) * 128;
+#pragma unroll
+            for (int hf = 0; hf < NH; ++hf) {
+              tma_load_4d(dst + hf * kHalf, img ? &p.kf : &p.kpf, bar, hf * 64, U.hk, row, U.w.b);
+              tma_load_4d(dst + S::kTile + hf * kHalf, img ? &p.vf : &p.vpf, bar, hf * 64, U.hk,
+                          row, U.w.b);
             }
           } else if (!KV && tile >= p.n_tiles) {  // dQ: pooled key tile
 #pragma unroll
@@ -357,8 +418,10 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
                                  p.Hg, p.Wg, p.N, dst + S::kTile, bar);
           }
         }
-        if (MODE == kModePooled)
-          write_row_values_flat(p, U.w.b, U.q0 + tile, h, rowv + slot * 256, lane);
+        if (text_q)
+          write_row_values_flat(p, U.w.b, ttile, h, rowv + slot * 256, lane, true);
+        else if (MODE == kModePooled)
+          write_row_values_flat(p, U.w.b, ftile, h, rowv + slot * 256, lane);
         else if (KV)
           write_row_values(p, pv, U.w, tile, h, rowv + slot * 256, lane);
         mbar_arrive(BAR(S::BFULL + slot));
@@ -390,6 +453,14 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
             tma_load_4d(dst + S::kTile + hf * kHalf, &p.vpf, BAR(S::AFULL), hf * 64, U.hk,
                         U.tile * 128, U.w.b);
           }
+        } else if (MODE == kModeDqText) {  // text query tile: Qt, dOt
+#pragma unroll
+          for (int hf = 0; hf < NH; ++hf) {
+            tma_load_4d(dst + hf * kHalf, &p.qtf, BAR(S::AFULL), hf * 64, U.h, U.tile * 128,
+                        U.w.b);
+            tma_load_4d(dst + S::kTile + hf * kHalf, &p.gtf, BAR(S::AFULL), hf * 64, U.h,
+                        U.tile * 128, U.w.b);
+          }
         } else {
           load_window_tile<NH>(pv, KV ? p.km : p.qm, &p.fill, U.w, U.tile, KV ? U.hk : U.h, p.T,
                                p.Hg, p.Wg, p.N, dst, BAR(S::AFULL));
@@ -397,7 +468,8 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
                                p.Hg, p.Wg, p.N, dst + S::kTile, BAR(S::AFULL));
         }
       }
-      if (!KV) write_row_values(p, pv, U.w, U.tile, U.h, rowv, lane);
+      if (MODE == kModeDq) write_row_values(p, pv, U.w, U.tile, U.h, rowv, lane);
+      if (MODE == kModeDqText) write_row_values_flat(p, U.w.b, U.tile, U.h, rowv, lane, true);
       mbar_arrive(BAR(S::AFULL));
       ++na;
     }
@@ -559,6 +631,8 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
       long long tok;
       if (MODE == kModePooled)
         tok = 128LL * U.tile + r < p.P ? 128LL * U.tile + r : -1;
+      else if (MODE == kModeDqText)
+        tok = 128LL * U.tile + r < p.L ? 128LL * U.tile + r : -1;
       else
         tok = r < pv.rows[U.tile] ? window_row_token(pv, U.w, U.tile, r, p.T, p.Hg, p.Wg) : -1;
       for (int s = 0; s < n_steps; ++s) {
@@ -666,7 +740,7 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
         const float mul = hc == 0 ? 1.0f : p.scale;
         const uint64_t m2 = f2pack(mul, mul);
         const float* share = nullptr;
-        if (p.P && tok >= 0) {
+        if (p.P && !p.joint && tok >= 0) {  // pooled cells only: text keys are their own rows
           const long long hw = (long long)p.Hg * p.Wg;
           const long long t = tok / hw, y = (tok / p.Wg) % p.Hg, x = tok % p.Wg;
           const long long cell =
@@ -707,8 +781,10 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
           warp_store_row64(stg, w, roff, base, hf * 64, lane, p.kv_elems);
         }
       } else if (hc < NH) {
-        // warpgroup hc writes columns [64 hc, 64 hc + 64) of dQ (times the scale)
-        const long long roff = tok >= 0 ? (((long long)U.w.b * p.N + tok) * p.H + U.h) * D : -1;
+        // warpgroup hc writes columns [64 hc, 64 hc + 64) of dQ (text: dQt), times the scale
+        constexpr bool TQ = MODE == kModeDqText;
+        const long long nrows = TQ ? p.L : p.N;
+        const long long roff = tok >= 0 ? (((long long)U.w.b * nrows + tok) * p.H + U.h) * D : -1;
         const uint64_t m2 = f2pack(p.scale, p.scale);
         uint32_t o[2][32];
         tmem_ld32(tmem + tl + 256 + hc * 64, o[0]);
@@ -723,7 +799,8 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
                                 __uint_as_float(o[e / 16][(2 * e) % 32 + 1])), m2), o0, o1);
           w[e] = pack_bf16(o0, o1);
         }
-        warp_store_row64(stg, w, roff, p.dq, hc * 64, lane, p.q_elems);
+        warp_store_row64(stg, w, roff, TQ ? p.dqt : p.dq, hc * 64, lane,
+                         TQ ? p.qt_elems : p.q_elems);
       }
       tc_fence_before();  // the reads of the accumulators precede the next unit's MMAs
       nl2 = nl2n;
@@ -773,11 +850,60 @@ basa_status launch_bwd_all(BwdTcParams* prm, const Dims& d, long long per, cudaS
   return launch_bwd_kernel<D, kModeDkv>(prm, (long long)d.B * d.Hkv * per, stream);
 }
 
+// Text keys' gradients from their fp32 sums: dkt = scale * dkp, dvt = dvp,
+// rounded to bf16 once ([B, L, Hkv, d], four elements per thread).
+__global__ void __launch_bounds__(256) text_grad_round_kernel(const float* dkp, const float* dvp,
+                                                              __nv_bfloat16* dkt,
+                                                              __nv_bfloat16* dvt, float scale,
+                                                              long long n4) {
+  const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= n4) return;
+  const float4 a = reinterpret_cast<const float4*>(dkp)[i];
+  const float4 b = reinterpret_cast<const float4*>(dvp)[i];
+  uint2 ka, vb;
+  ka.x = pack_bf16(a.x * scale, a.y * scale);
+  ka.y = pack_bf16(a.z * scale, a.w * scale);
+  vb.x = pack_bf16(b.x, b.y);
+  vb.y = pack_bf16(b.z, b.w);
+  reinterpret_cast<uint2*>(dkt)[i] = ka;
+  reinterpret_cast<uint2*>(dvt)[i] = vb;
+}
+
+// The joint backward's launches: D of the image and text rows, the text keys'
+// dK, dV (over the image and the text queries, summed into dkp, dvp), the
+// image dQ (window then text keys), the text dQ (every key), the window dK, dV
+// (window then text queries), and the rounding of the text keys' gradients.
+template <int D>
+basa_status launch_bwd_joint_all(BwdTcParams* prm, const Dims& d, long long per,
+                                 const JointGrads& jg, float* dkp, float* dvp,
+                                 cudaStream_t stream) {
+  basa_status st;
+  const size_t n = (size_t)d.B * jg.L * d.Hkv * d.d;
+  if (cudaMemsetAsync(dkp, 0, n * sizeof(float), stream) != cudaSuccess ||
+      cudaMemsetAsync(dvp, 0, n * sizeof(float), stream) != cudaSuccess)
+    return BASA_ERR_CUDA;
+  const long long text_key_units = (long long)d.B * d.Hkv * prm->n_pt * prm->n_fsplits;
+  if ((st = launch_bwd_kernel<D, kModePooled>(prm, text_key_units, stream)) != BASA_OK) return st;
+  if ((st = launch_bwd_kernel<D, kModeDq>(prm, (long long)d.B * d.H * per, stream)) != BASA_OK)
+    return st;
+  if ((st = launch_bwd_kernel<D, kModeDqText>(prm, (long long)d.B * d.H * prm->n_tt, stream)) !=
+      BASA_OK)
+    return st;
+  if ((st = launch_bwd_kernel<D, kModeDkv>(prm, (long long)d.B * d.Hkv * per, stream)) != BASA_OK)
+    return st;
+  const long long n4 = (long long)(n / 4);
+  text_grad_round_kernel<<<(unsigned)((n4 + 255) / 256), 256, 0, stream>>>(
+      dkp, dvp, static_cast<__nv_bfloat16*>(jg.dkt), static_cast<__nv_bfloat16*>(jg.dvt),
+      d.scale, n4);
+  return cudaGetLastError() == cudaSuccess ? BASA_OK : BASA_ERR_CUDA;
+}
+
 basa_status build_and_launch_bwd(BwdTcParams* prm, const Dims& d, const TilePlan& plan,
                                  const void* q, const void* k, const void* v, const void* out,
                                  const void* dout, const float* lse, float* dD, void* dq,
                                  void* dk, void* dv, const PoolGrads* pg, uint32_t timeout_ms,
-                                 cudaStream_t stream) {
+                                 cudaStream_t stream, const JointGrads* jg = nullptr,
+                                 float* jdkp = nullptr, float* jdvp = nullptr) {
   basa_status st;
   const uint64_t D = (uint64_t)d.d, H = (uint64_t)d.H, Hk = (uint64_t)d.Hkv;
   if ((st = pack_plan_image(plan, &prm->plan)) != BASA_OK) return st;
@@ -826,6 +952,49 @@ basa_status build_and_launch_bwd(BwdTcParams* prm, const Dims& d, const TilePlan
     prm->pt = d.pt; prm->ph = d.ph; prm->pw = d.pw;
     prm->inv_count = 1.0f / (float)(d.pt * d.ph * d.pw);
   }
+  if (jg) {  // text tokens in the pooled slots, text queries as flat tiles, flat image K, V
+    const uint64_t L = (uint64_t)jg->L;
+    const uint64_t tkdims[4] = {D, Hk, L, (uint64_t)d.B};
+    const uint64_t tkstr[3] = {D * 2, Hk * D * 2, L * Hk * D * 2};
+    const uint64_t tqdims[4] = {D, H, L, (uint64_t)d.B};
+    const uint64_t tqstr[3] = {D * 2, H * D * 2, L * H * D * 2};
+    const uint64_t fqdims[4] = {D, H, (uint64_t)d.N, (uint64_t)d.B};
+    const uint64_t fqstr[3] = {D * 2, H * D * 2, (uint64_t)d.N * H * D * 2};
+    const uint64_t fkdims[4] = {D, Hk, (uint64_t)d.N, (uint64_t)d.B};
+    const uint64_t fkstr[3] = {D * 2, Hk * D * 2, (uint64_t)d.N * Hk * D * 2};
+    const uint32_t box128[4] = {64, 1, 128, 1};
+    if ((st = encode_map(&prm->kpf, jg->kt, 4, tkdims, tkstr, box128)) != BASA_OK) return st;
+    if ((st = encode_map(&prm->vpf, jg->vt, 4, tkdims, tkstr, box128)) != BASA_OK) return st;
+    if ((st = encode_map(&prm->qtf, jg->qt, 4, tqdims, tqstr, box128)) != BASA_OK) return st;
+    if ((st = encode_map(&prm->gtf, jg->dout_t, 4, tqdims, tqstr, box128)) != BASA_OK) return st;
+    if ((st = encode_map(&prm->qf, q, 4, fqdims, fqstr, box128)) != BASA_OK) return st;
+    if ((st = encode_map(&prm->gf, dout, 4, fqdims, fqstr, box128)) != BASA_OK) return st;
+    if ((st = encode_map(&prm->kf, k, 4, fkdims, fkstr, box128)) != BASA_OK) return st;
+    if ((st = encode_map(&prm->vf, v, 4, fkdims, fkstr, box128)) != BASA_OK) return st;
+    prm->joint = 1;
+    prm->L = jg->L;
+    prm->P = jg->L;
+    prm->n_tt = (int)((jg->L + 127) / 128);
+    prm->n_pt = prm->n_tt;
+    prm->n_fqt = (int)((d.N + 127) / 128);
+    prm->dkp = jdkp;
+    prm->dvp = jdvp;
+    prm->lse_t = jg->lse_t;
+    prm->dD_t = jg->dD_t;
+    prm->dqt = static_cast<__nv_bfloat16*>(jg->dqt);
+    prm->qt_elems = (long long)d.B * jg->L * d.H * d.d;
+    // split the image and text query tiles so that the text keys' kernel has
+    // about four units per SM
+    const int nq = prm->n_fqt + prm->n_tt;
+    const long long base = (long long)d.B * d.Hkv * prm->n_pt;
+    long long n = (4LL * tc_sm_count() + base - 1) / base;
+    if (n > nq) n = nq;
+    if (n < 1) n = 1;
+    prm->fqt_per_split = (int)((nq + n - 1) / n);
+    prm->n_fsplits = (nq + prm->fqt_per_split - 1) / prm->fqt_per_split;
+    prm->pt = prm->ph = prm->pw = 1;
+    prm->inv_count = 1.0f;
+  }
   prm->lse = lse;
   prm->dD = dD;
   prm->q_elems = (long long)d.B * d.N * d.H * d.d;
@@ -846,8 +1015,15 @@ basa_status build_and_launch_bwd(BwdTcParams* prm, const Dims& d, const TilePlan
   prm->scale = d.scale;
   prm->scale_log2 = d.scale * kLog2e;
   const long long per = (long long)prm->n_windows * plan.n_tiles;
-  // D = rowsum(dout * out), then the gradient kernels
+  // D = rowsum(dout * out) (joint: also of the text rows), then the gradient kernels
   if ((st = launch_bwd_prep(d, out, dout, dD, stream)) != BASA_OK) return st;
+  if (jg) {
+    Dims dt = d;
+    dt.N = jg->L;
+    if ((st = launch_bwd_prep(dt, jg->out_t, jg->dout_t, jg->dD_t, stream)) != BASA_OK) return st;
+    return d.d == 64 ? launch_bwd_joint_all<64>(prm, d, per, *jg, jdkp, jdvp, stream)
+                     : launch_bwd_joint_all<128>(prm, d, per, *jg, jdkp, jdvp, stream);
+  }
   return d.d == 64 ? launch_bwd_all<64>(prm, d, per, stream)
                    : launch_bwd_all<128>(prm, d, per, stream);
 }
@@ -869,6 +1045,25 @@ basa_status launch_bwd_tc(const Dims& d, const void* q, const void* k, const voi
   memset(prm, 0, sizeof(*prm));
   st = build_and_launch_bwd(prm, d, plan, q, k, v, out, dout, lse, dD, dq, dk, dv, pg, timeout_ms,
                             stream);
+  delete prm;
+  return st;
+}
+
+basa_status launch_bwd_tc_joint(const Dims& d, const void* q, const void* k, const void* v,
+                                const void* out, const void* dout, const float* lse, float* dD,
+                                void* dq, void* dk, void* dv, const JointGrads& jg, float* dkp,
+                                float* dvp, uint32_t timeout_ms, cudaStream_t stream) {
+  if (d.dtype != BASA_BF16 || (d.d != 64 && d.d != 128) || d.qsep || d.P || d.padded ||
+      jg.L <= 0 || !dkp || !dvp)
+    return BASA_ERR_UNSUPPORTED;
+  TilePlan plan;
+  basa_status st = build_tile_plan(d, &plan);  // before any launch
+  if (st != BASA_OK) return st;
+  BwdTcParams* prm = new (std::nothrow) BwdTcParams;
+  if (!prm) return BASA_ERR_INVALID_ARG;
+  memset(prm, 0, sizeof(*prm));
+  st = build_and_launch_bwd(prm, d, plan, q, k, v, out, dout, lse, dD, dq, dk, dv, nullptr,
+                            timeout_ms, stream, &jg, dkp, dvp);
   delete prm;
   return st;
 }

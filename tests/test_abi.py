@@ -286,7 +286,7 @@ def test_fp8_and_padding_validation(lib):
     align = lambda x: (x + 255) // 256 * 256
     assert lib.basa_bwd_workspace_size(ctypes.byref(pp)) == align(2 * 3 * N * 4)
     assert lib.basa_joint_bwd_workspace_size(ctypes.byref(pp), 77) == \
-        align(2 * 3 * N * 4) + align(2 * 3 * 77 * 4)
+        align(2 * 3 * N * 4) + align(2 * 3 * 77 * 4) + 2 * align(2 * 77 * 3 * 64 * 4)
     # the pool cell must still divide the grid
     pp.ph, pp.pw, pp.pt = 3, 4, 1
     assert call(pp) == 2

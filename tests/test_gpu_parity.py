@@ -225,6 +225,60 @@ def test_flux2048_gm4_sampled(basa, block):
     _workload_sampled(basa, "flux2048_gm4", block, nsample=192)
 
 
+# ---------------------------------------------------------------- every element at full size
+
+def _workload_rows(basa, name, block, heads=None, batches=None):
+    """Every output row and lse of the listed heads and batches of a full-size
+    workload (default: all of them) against the oracle, in the launch
+    configuration the benchmark times."""
+    w = WORKLOADS[name]
+    q, k, v = workload_inputs(w, block)
+    shift = w.shifts[block]
+    B, T, Hg, Wg, H, d = w.shape()
+    N = w.N
+    heads = list(range(H)) if heads is None else list(heads)
+    batches = list(range(B)) if batches is None else list(batches)
+    out, lse = basa.window_attn(q.cuda(), k.cuda(), v.cuda(), w.window, shift, w.pool,
+                                return_lse=True)
+    torch.cuda.synchronize()
+    assert basa.get_status() == 0
+    prm = oracle_params(w.shape(), w.window, shift, w.pool)
+    qf, kf, vf = oracle.as_f64(q), oracle.as_f64(k), oracle.as_f64(v)
+    kp = vp = None
+    if w.P:
+        kp, vp = oracle.pool_kv(kf, prm), oracle.pool_kv(vf, prm)
+    hsel = np.asarray(heads, dtype=np.int64)
+    for b in batches:
+        # rows (b, n, h), n outer and h inner: the order of out[b, n, heads]
+        sel = np.stack([np.full(N * len(heads), b, dtype=np.int64),
+                        np.repeat(np.arange(N, dtype=np.int64), len(heads)),
+                        np.tile(hsel, N)], axis=1)
+        ref, ref_lse = oracle.window_attn(qf, kf, vf, prm, kp=kp, vp=vp, want_lse=True,
+                                          select=sel)
+        got = out.reshape(B, N, H, d)[b][:, torch.as_tensor(hsel, device=out.device)]
+        assert_close(got.reshape(-1, d), ref, w.dtype, f"{name} block {block} batch {b}")
+        got_lse = lse[b][torch.as_tensor(hsel, device=lse.device)].t().reshape(-1)
+        lerr = float(np.abs(got_lse.double().cpu().numpy() - ref_lse).max())
+        assert lerr <= 2e-2, f"{name} block {block} batch {b}: lse max-abs {lerr}"
+    assert torch.isfinite(out).all()
+
+
+def test_flux2048_every_element(basa):
+    """The benchmark's workload: all 24 heads, all 16384 queries, and the lse."""
+    _workload_rows(basa, "flux2048", 0)
+
+
+def test_flux2048_gm4_block_every_element(basa):
+    """One whole block of the four-block schedule with 1024 pooled tokens (both
+    batches, every head and query); the last block's shift, as benchmarked."""
+    _workload_rows(basa, "flux2048_gm4", 3)
+
+
+def test_wan_video_two_heads_every_element(basa):
+    """Every query of two of Wan's 40 heads (the first and the last)."""
+    _workload_rows(basa, "wan_video", 0, heads=[0, 39])
+
+
 # ---------------------------------------------------------------- polynomial exp2
 
 def test_polynomial_exp2_against_cuda_exp2(basa):

@@ -98,8 +98,7 @@ def _build_mutant(tmp_path, old, new):
     c = tmp_path / "mutant.c"
     c.write_text(mutated)
     so = tmp_path / "libmutant.so"
-    subprocess.check_call(["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-std=c11",
-                           "-o", str(so), str(c), "-lm"])
+    subprocess.check_call(["gcc", *obuild.FLAGS, "-o", str(so), str(c), "-lm"])
     return str(so)
 
 
