@@ -54,6 +54,8 @@ _CSRC = os.path.join(ROOT, "sparse_attention_diffusion_basa_b200", "csrc")
 # the source files whose device code each profiled kernel is built from
 KERNEL_SOURCES = {
     "tc_attn_kernel": [os.path.join(_CSRC, "basa_tc.cu"), os.path.join(_CSRC, "tc_device.cuh")],
+    "tc_attn_pair_kernel": [os.path.join(_CSRC, "basa_tc2.cu"),
+                            os.path.join(_CSRC, "tc_device.cuh")],
     "pool_kernel": [os.path.join(_CSRC, "basa_pool.cu")],
     "tc_bwd_kernel": [os.path.join(_CSRC, "basa_tc_bwd.cu"), os.path.join(_CSRC, "tc_device.cuh")],
 }
@@ -89,6 +91,17 @@ def _traffic(kernel_key, workload):
         return float(e["dram_bytes_per_launch"])
     except Exception:
         return None
+
+
+def attention_kernel(w):
+    """The library's window-attention kernel for the workload: 256-token 2D
+    windows of whole 64-token row groups (bf16, d = 128, no pooled or text keys)
+    run on CTA pairs, the rest on the one-CTA kernel."""
+    wt, wh, ww = w.window
+    if (w.dtype == "bf16" and w.d == 128 and not w.P and not w.text and wt == 1
+            and wh * ww == 256 and 64 % ww == 0):
+        return "tc_attn_pair_kernel"
+    return "tc_attn_kernel"
 
 
 def workload_numbers(w, shift):
@@ -467,6 +480,8 @@ def main():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--full-steps", type=int, default=5)
+    ap.add_argument("--no-blocks", action="store_true",
+                    help="skip the per-block timings of a multi-block shift schedule")
     ap.add_argument("--backward", action="store_true",
                     help="time the backward (dq, dk, dv) of the workload's window attention")
     args = ap.parse_args()
@@ -602,6 +617,32 @@ def main():
         ms_pool = max_over_ranks(sum(t_pool) / len(t_pool), world)
         ms_attn = max_over_ranks(sum(t_attn) / len(t_attn), world)
 
+    # every block of a multi-block shift schedule (FLUX's alternating (0, 0) /
+    # (8, 8) blocks; the four shifts of the pooled schedule): each block's own
+    # inputs, pooling, attention and pooling + attention, and the schedule's
+    # total (the sum of the blocks' steps)
+    blocks_out = None
+    if len(w.shifts) > 1 and not L and not args.no_blocks:
+        blocks_out = []
+        for bi, bshift in enumerate(w.shifts):
+            bq, bk, bv = (x.to(dev) for x in workload_inputs(w, bi))
+            row = {"block": bi, "shift": list(bshift)}
+            if w.P:
+                bkp, bvp = basa.pool_kv(bk, bv, w.pool)
+                tp = time_steps(lambda: basa.pool_kv(bk, bv, w.pool, out=(bkp, bvp)), args.steps,
+                                flush)
+                ta = time_steps(lambda: basa.window_attn_gm(bq, bk, bv, bkp, bvp, w.window, bshift,
+                                                            w.pool, out=out), args.steps, flush)
+                row["pool_ms"] = max_over_ranks(sum(tp) / len(tp), world)
+                row["attn_ms"] = max_over_ranks(sum(ta) / len(ta), world)
+            ts = time_steps(lambda: basa.window_attn(bq, bk, bv, w.window, bshift, w.pool, out=out,
+                                                     workspace=ws if ws_bytes else None),
+                            args.steps, flush)
+            row["step_ms"] = max_over_ranks(sum(ts) / len(ts), world)
+            blocks_out.append(row)
+            del bq, bk, bv
+        assert basa.get_status() == 0, "device wait timed out during the block timings"
+
     # full attention on the same inputs: the speedup denominator
     t_full = time_steps(step_full, args.full_steps, flush)
     ms_full = max_over_ranks(sum(t_full) / len(t_full), world)
@@ -625,8 +666,9 @@ def main():
         roof = {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "frac": gbs / peaks["hbm_gbs"]}
     roof["peak_source"] = peaks["source"]
-    roof["traffic"] = _traffic("tc_attn_kernel", w.name)
-    roof["kernel"] = "tc_attn_kernel"
+    kname = attention_kernel(w)
+    roof["traffic"] = _traffic(kname, w.name)
+    roof["kernel"] = kname
     roof["kernel_ms"] = ms_attn
 
     line = {
@@ -651,10 +693,13 @@ def main():
                 "h2d_bytes_per_step": sum(h.numel() * h.element_size() for h, _ in host_in),
                 "d2h_bytes_per_step": sum(h.numel() * h.element_size() for h, _ in host_out),
                 "pipeline": "two device buffer sets; copy-in, compute and copy-out streams"},
-        "kernels_ms": {"tc_attn_kernel": ms_attn, "pool_kernel": ms_pool},
+        "kernels_ms": {kname: ms_attn, "pool_kernel": ms_pool},
         "gpu_launches": args.steps * (2 if (w.P or L) else 1),
         "clocks": clk,
     }
+    if blocks_out:
+        line["blocks"] = blocks_out
+        line["all_blocks_ms"] = sum(r["step_ms"] for r in blocks_out)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w, shift, q, k, v)
     if rank == 0:

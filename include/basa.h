@@ -320,14 +320,6 @@ BASA_API basa_status basa_window_attn_noalloc(const void* q, const void* k, cons
 BASA_API basa_status basa_get_status(cudaStream_t stream);
 
 /*
- * Test only: y[i] = 2^x[i] computed by the polynomial exponential that the bf16
- * kernel uses for part of its softmax (x <= 0; device pointers to n floats;
- * enqueued on `stream`).  Lets tests compare it with CUDA's own exp2 and its
- * stated error bound (relative error below 1e-4 for -125 <= x <= 0).
- */
-BASA_API basa_status basa_test_exp2(const float* x, float* y, int64_t n, cudaStream_t stream);
-
-/*
  * Host-only description of the bf16 kernel's window tiling (no GPU needed).
  * *n_windows = windows per (b, h) and *n_tiles = 128-row tiles per window.
  * If rows != NULL it receives [n_windows][n_tiles][128] int32 entries: the

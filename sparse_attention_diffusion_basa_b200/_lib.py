@@ -24,7 +24,7 @@ BASA_FLAG_PAD_GRID = 0x4
 # Every symbol include/basa.h declares.
 EXPORTS = ("basa_status_string", "basa_version", "basa_workspace_size", "basa_pool_kv",
            "basa_window_attn", "basa_window_attn_gm", "basa_full_attn", "basa_get_status",
-           "basa_window_tiles", "basa_window_attn_noalloc", "basa_test_exp2",
+           "basa_window_tiles", "basa_window_attn_noalloc",
            "basa_joint_attn", "basa_window_attn_bwd", "basa_bwd_workspace_size",
            "basa_joint_workspace_size", "basa_joint_attn_bwd", "basa_joint_bwd_workspace_size")
 
@@ -93,8 +93,6 @@ def load():
                                       ctypes.POINTER(ctypes.c_int32),
                                       ctypes.POINTER(ctypes.c_int32), ctypes.c_int64]
     lib.basa_window_tiles.restype = ctypes.c_int
-    lib.basa_test_exp2.argtypes = [vp, vp, ctypes.c_int64, vp]
-    lib.basa_test_exp2.restype = ctypes.c_int
     lib.basa_window_attn_noalloc.argtypes = [vp, vp, vp, vp, vp, P, vp]
     lib.basa_window_attn_noalloc.restype = ctypes.c_int
     _lib = lib

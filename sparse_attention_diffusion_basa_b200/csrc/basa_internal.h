@@ -86,9 +86,11 @@ struct TilePlan {
   uint32_t box[kClasses][kMaxTiles][kMaxBoxes];
 };
 
-// Builds the plan for window (wt, wh, ww) with shifts already reduced to [0, w).
-// Returns BASA_ERR_UNSUPPORTED when the bounds of the bf16 kernel are exceeded.
-basa_status build_tile_plan(const Dims& d, TilePlan* plan);
+// Builds the plan for window (wt, wh, ww) with shifts already reduced to [0, w):
+// tiles of whole window rows of at most max_rows (128, or 64 for the CTA-pair
+// kernel) tokens.  Returns BASA_ERR_UNSUPPORTED when the bounds of the bf16
+// kernel are exceeded.
+basa_status build_tile_plan(const Dims& d, TilePlan* plan, int max_rows = 128);
 
 // Window class (wrap bits) of window (jt, jh, jw).
 __host__ __device__ inline int window_class(int jt, int jh, int jw, int nwt, int nwh, int nww,
@@ -118,9 +120,14 @@ struct SplitK {
 
 // bf16 tcgen05 window / full attention.  flat = full attention over the grid.
 // sk (flat only, nullable): split the key range and combine the partials.
+// after_pool: the kernel just launched on `stream` is the pooling of kp, vp;
+// the attention kernel is then launched as its programmatic dependent, so
+// that its start overlaps the pooling's tail (it waits for the pooling grid
+// before it loads a pooled tile).
 basa_status launch_tc(const Dims& d, bool flat, const void* q, const void* k, const void* v,
                       const void* kp, const void* vp, void* out, float* lse, uint32_t flags,
-                      uint32_t timeout_ms, cudaStream_t stream, const SplitK* sk = nullptr);
+                      uint32_t timeout_ms, cudaStream_t stream, const SplitK* sk = nullptr,
+                      bool after_pool = false);
 
 // Splits that keep a flat launch's grid full when it has fewer than half as
 // many units as SMs (1 = no split); the workspace bytes they need; the
@@ -197,10 +204,22 @@ basa_status launch_bwd_tc_joint(const Dims& d, const void* q, const void* k, con
 basa_status launch_tc_static_params(const Dims& d, bool flat, const void* q, const void* k,
                                     const void* v, const void* kp, const void* vp, void* out,
                                     float* lse, uint32_t flags, uint32_t timeout_ms,
-                                    cudaStream_t stream);
+                                    cudaStream_t stream, bool after_pool = false);
 
-// Test hook: y = the kernels' polynomial 2^x (device pointers, n floats).
-basa_status launch_ex2_poly_test(const float* x, float* y, long long n, cudaStream_t stream);
+// bf16 window attention over CTA pairs (basa_tc2.cu) for 256-token windows:
+// pair_kernel_applies checks the call and builds the 64-row tile plan it
+// needs; launch_tc_pair launches (static_params: the parameter block lives in
+// static storage, for the entry points that allocate nothing).  Building with
+// BASA_TC_PAIR=0 keeps those windows on the one-CTA kernel.
+#ifndef BASA_TC_PAIR
+#define BASA_TC_PAIR 0
+#endif
+constexpr bool kPairWindows = BASA_TC_PAIR != 0;
+bool pair_kernel_applies(const Dims& d, bool extra_keys, TilePlan* plan64);
+basa_status launch_tc_pair(const Dims& d, const TilePlan& plan64, const void* q, const void* k,
+                           const void* v, void* out, float* lse, uint32_t flags,
+                           uint32_t timeout_ms, cudaStream_t stream, bool static_params);
+cudaError_t take_pair_status(cudaStream_t stream, unsigned int* status, unsigned int* where);
 
 // Device status word helpers.  read_and_clear_status (basa_tc.cu) synchronises
 // the stream and reads and clears the status words of every kernel file;

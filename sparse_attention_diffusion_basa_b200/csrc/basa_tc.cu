@@ -137,13 +137,6 @@ __device__ __forceinline__ void widen_v_tile(uint32_t src, uint32_t dst, int lan
 }
 
 
-// Which exponential pairs go to the polynomial: pair e of every 16 when
-// e % kEx2Period == kEx2Period - 1 (period 3: 5 of 16 pairs); 0 = none.
-#ifndef BASA_EX2_PERIOD
-#define BASA_EX2_PERIOD 0
-#endif
-constexpr int kEx2Period = BASA_EX2_PERIOD;
-
 // Rescale O only when a tile's row max exceeds the reference max by more than
 // 2^kLazyRescale; until then the stale reference is kept (P stays <= 2^8).
 constexpr float kLazyRescale = 8.0f;
@@ -425,10 +418,16 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attn_kernel(const __grid_const
     if (!withhold) {
       uint32_t kv = 0;
       uint32_t issued_mask = 0, last_par = 0;
-      bool ok = true;
+      bool ok = true, dep_done = false;
       for (uint32_t u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
         const Unit U = decode_unit<kSplit>(p, u);
         for (int j = kbeg(U); j < kbeg(U) + kcount(U) && ok; ++j) {
+          if (j >= p.n_wkt && !dep_done) {
+            // extra keys may be pooled by the kernel this one was launched as a
+            // dependent of: wait for that grid (returns at once otherwise)
+            grid_dependency_wait();
+            dep_done = true;
+          }
           for (int kind = 1; kind <= 2 && ok; ++kind) {
             const uint32_t slot = kv % NS, par = (kv / NS) & 1u;
             if (!(ok = wait_warp(BAR(S::KVEMPTY + slot), par ^ 1u, abort_flag, limit,
@@ -716,14 +715,9 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attn_kernel(const __grid_const
           for (int e = 0; e < 16; ++e) {
             const uint64_t x2 = f2fma(f2pack(__uint_as_float(s[cc][2 * e]),
                                              __uint_as_float(s[cc][2 * e + 1])), c2, nm2);
-            uint64_t p2;
-            if (kEx2Period > 0 && e % (kEx2Period > 0 ? kEx2Period : 1) == kEx2Period - 1) {
-              p2 = ex2_poly_x2(x2);
-            } else {
-              float a0, a1;
-              f2unpack(x2, a0, a1);
-              p2 = f2pack(ex2(a0), ex2(a1));
-            }
+            float a0, a1;
+            f2unpack(x2, a0, a1);
+            const uint64_t p2 = f2pack(ex2(a0), ex2(a1));
             if (e & 1) rsb = f2add(rsb, p2); else rsa = f2add(rsa, p2);
             float p0, p1;
             f2unpack(p2, p0, p1);
@@ -894,7 +888,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attn_kernel(const __grid_const
 }
 
 template <int D, int kRing, bool kSplit = false, bool kF8 = false>
-basa_status launch_impl(TcParams* prm, cudaStream_t stream) {
+basa_status launch_impl(TcParams* prm, cudaStream_t stream, bool dependent) {
   const int smem = Smem<D, kRing, kF8>::alloc;
   static_assert(Smem<D, kRing, kF8>::alloc <= 232448, "shared memory plan exceeds 227 KB");
   if (cudaFuncSetAttribute(tc_attn_kernel<D, kRing, kSplit, kF8>,
@@ -902,7 +896,20 @@ basa_status launch_impl(TcParams* prm, cudaStream_t stream) {
     return BASA_ERR_CUDA;
   long long grid = tc_sm_count();
   if (grid > prm->n_units) grid = prm->n_units;
-  tc_attn_kernel<D, kRing, kSplit, kF8><<<(unsigned)grid, kThreads, smem, stream>>>(*prm);
+  // dependent: launched as the programmatic dependent of the kernel before it
+  // on the stream (the pooling), so that its start overlaps that kernel's tail
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)grid);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = (size_t)smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = dependent ? 1 : 0;
+  if (cudaLaunchKernelEx(&cfg, tc_attn_kernel<D, kRing, kSplit, kF8>, *prm) != cudaSuccess)
+    return BASA_ERR_CUDA;
   return cudaGetLastError() == cudaSuccess ? BASA_OK : BASA_ERR_CUDA;
 }
 
@@ -914,7 +921,7 @@ namespace {
 basa_status build_and_launch(TcParams* prm, const Dims& d, bool flat, const void* q,
                              const void* k, const void* v, const void* kp, const void* vp,
                              void* out, float* lse, uint32_t flags, uint32_t timeout_ms,
-                             cudaStream_t stream, const SplitK* sk) {
+                             cudaStream_t stream, const SplitK* sk, bool after_pool) {
   basa_status st = BASA_OK;
   const uint64_t D = (uint64_t)d.d;
   const uint64_t H = (uint64_t)d.H;
@@ -947,6 +954,7 @@ basa_status build_and_launch(TcParams* prm, const Dims& d, bool flat, const void
       f8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
   prm->flat = flat ? 1 : 0;
   prm->P = kp ? (int)d.P : 0;
+  bool dep = false;  // launched as the dependent of the pooling kernel
   TilePlan plan;
   if (!flat && (st = build_tile_plan(d, &plan)) != BASA_OK) goto done;  // before any driver call
   // flat [d, H, N, B] views (full attention tiles; the fill source); the query
@@ -1039,17 +1047,20 @@ basa_status build_and_launch(TcParams* prm, const Dims& d, bool flat, const void
   // 4; everything else reuses K/V tiles from L2 and runs faster with 4.
   // Split key range: its own instantiation, so that the window kernels carry
   // none of its code.
+  // launched as the pooling kernel's dependent only when it reads pooled tiles
+  dep = after_pool && prm->n_pkt > 0;
   if (f8) {  // d = 128, no extra keys, no split (checked by the entry points)
     if (d.d != 128 || prm->n_splits > 1 || prm->n_pkt) { st = BASA_ERR_UNSUPPORTED; goto done; }
-    st = launch_impl<128, 4, false, true>(prm, stream);
+    st = launch_impl<128, 4, false, true>(prm, stream, dep);
   } else if (prm->n_splits > 1)
-    st = d.d == 64 ? launch_impl<64, 8, true>(prm, stream) : launch_impl<128, 4, true>(prm, stream);
+    st = d.d == 64 ? launch_impl<64, 8, true>(prm, stream, dep)
+                   : launch_impl<128, 4, true>(prm, stream, dep);
   else if (d.d == 64)
-    st = launch_impl<64, 8>(prm, stream);
+    st = launch_impl<64, 8>(prm, stream, dep);
   else if (!flat && prm->n_wkt + prm->n_pkt <= 2)
-    st = launch_impl<128, 3>(prm, stream);
+    st = launch_impl<128, 3>(prm, stream, dep);
   else
-    st = launch_impl<128, 4>(prm, stream);
+    st = launch_impl<128, 4>(prm, stream, dep);
   if (st == BASA_OK && prm->n_splits > 1) st = launch_split_combine(d, *sk, out, lse, stream);
 done:
   return st;
@@ -1064,12 +1075,14 @@ std::mutex g_static_params_mu;
 
 basa_status launch_tc(const Dims& d, bool flat, const void* q, const void* k, const void* v,
                       const void* kp, const void* vp, void* out, float* lse, uint32_t flags,
-                      uint32_t timeout_ms, cudaStream_t stream, const SplitK* sk) {
+                      uint32_t timeout_ms, cudaStream_t stream, const SplitK* sk,
+                      bool after_pool) {
   TcParams* prm = new (std::nothrow) TcParams;
   if (!prm) return BASA_ERR_INVALID_ARG;
   memset(prm, 0, sizeof(*prm));
   const basa_status st =
-      build_and_launch(prm, d, flat, q, k, v, kp, vp, out, lse, flags, timeout_ms, stream, sk);
+      build_and_launch(prm, d, flat, q, k, v, kp, vp, out, lse, flags, timeout_ms, stream, sk,
+                       after_pool);
   delete prm;
   return st;
 }
@@ -1077,11 +1090,11 @@ basa_status launch_tc(const Dims& d, bool flat, const void* q, const void* k, co
 basa_status launch_tc_static_params(const Dims& d, bool flat, const void* q, const void* k,
                                     const void* v, const void* kp, const void* vp, void* out,
                                     float* lse, uint32_t flags, uint32_t timeout_ms,
-                                    cudaStream_t stream) {
+                                    cudaStream_t stream, bool after_pool) {
   std::lock_guard<std::mutex> lock(g_static_params_mu);
   memset(&g_static_params, 0, sizeof(g_static_params));
   return build_and_launch(&g_static_params, d, flat, q, k, v, kp, vp, out, lse, flags,
-                          timeout_ms, stream, nullptr);
+                          timeout_ms, stream, nullptr, after_pool);
 }
 
 namespace {
@@ -1152,25 +1165,6 @@ basa_status launch_split_combine(const Dims& d, const SplitK& sk, void* out, flo
   else
     split_combine_kernel<128><<<(unsigned)blocks, 256, 0, stream>>>(
         sk.part_o, sk.part_ml, static_cast<__nv_bfloat16*>(out), lse, sk.n, d.H, d.Nq, rows);
-  return cudaGetLastError() == cudaSuccess ? BASA_OK : BASA_ERR_CUDA;
-}
-
-namespace {
-__global__ void ex2_poly_test_kernel(const float* x, float* y, long long n) {
-  const long long i = 2 * ((long long)blockIdx.x * blockDim.x + threadIdx.x);
-  if (i >= n) return;
-  const float x1 = i + 1 < n ? x[i + 1] : 0.0f;
-  float y0, y1;
-  f2unpack(ex2_poly_x2(f2pack(x[i], x1)), y0, y1);
-  y[i] = y0;
-  if (i + 1 < n) y[i + 1] = y1;
-}
-}  // namespace
-
-basa_status launch_ex2_poly_test(const float* x, float* y, long long n, cudaStream_t stream) {
-  if (n <= 0) return BASA_OK;
-  const long long pairs = (n + 1) / 2;
-  ex2_poly_test_kernel<<<(unsigned)((pairs + 255) / 256), 256, 0, stream>>>(x, y, n);
   return cudaGetLastError() == cudaSuccess ? BASA_OK : BASA_ERR_CUDA;
 }
 

@@ -113,6 +113,12 @@ __device__ __forceinline__ void tma_store_4d(const CUtensorMap* map, uint32_t sr
       "r"(src), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
       : "memory");
 }
+// Programmatic dependent launch: waits until the grid this one was launched
+// as a dependent of has completed and its writes are visible (returns at once
+// for a grid launched without that dependency).
+__device__ __forceinline__ void grid_dependency_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
@@ -285,38 +291,6 @@ __device__ __forceinline__ float max3(float a, float b, float c) {
   float d;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
   return d;
-}
-
-// 2^x for a pair of x <= 0, computed on the FMA and integer pipes so that part
-// of the softmax's exponentials bypass the MUFU unit (its throughput limit).
-// Method: round-to-nearest argument reduction x = j + f, |f| <= 1/2, through the
-// float constant 1.5 * 2^23 (after the addition its low mantissa bits hold j;
-// the additive reduction of Cody and Waite), a cubic fit of 2^f on [-1/2, 1/2]
-// minimising the maximum relative error (Remez exchange, fitted for this
-// library: 7.5e-5 worst case in fp32 Horner evaluation), then the scale by 2^j
-// applied by adding j to the exponent field (Schraudolph, "A fast, compact
-// approximation of the exponential function", 1999).  x is clamped at -125 so
-// the exponent field cannot underflow; results there are below 2^-124.
-constexpr float kEx2C0 = 0x1.fff692p-1f;
-constexpr float kEx2C1 = 0x1.62f31ap-1f;
-constexpr float kEx2C2 = 0x1.f0de1ap-3f;
-constexpr float kEx2C3 = 0x1.c3f76p-5f;
-__device__ __forceinline__ uint64_t ex2_poly_x2(uint64_t x2) {
-  float x0, x1;
-  f2unpack(x2, x0, x1);
-  x0 = fmaxf(x0, -125.0f);
-  x1 = fmaxf(x1, -125.0f);
-  const uint64_t t = f2add(f2pack(x0, x1), f2pack(12582912.0f, 12582912.0f));
-  const uint64_t j = f2add(t, f2pack(-12582912.0f, -12582912.0f));
-  const uint64_t f = f2fma(j, f2pack(-1.0f, -1.0f), f2pack(x0, x1));
-  uint64_t q = f2fma(f, f2pack(kEx2C3, kEx2C3), f2pack(kEx2C2, kEx2C2));
-  q = f2fma(q, f, f2pack(kEx2C1, kEx2C1));
-  q = f2fma(q, f, f2pack(kEx2C0, kEx2C0));
-  float q0, q1, t0, t1;
-  f2unpack(q, q0, q1);
-  f2unpack(t, t0, t1);
-  return f2pack(__int_as_float(__float_as_int(q0) + (__float_as_int(t0) << 23)),
-                __int_as_float(__float_as_int(q1) + (__float_as_int(t1) << 23)));
 }
 
 __device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr) {
