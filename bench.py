@@ -54,8 +54,6 @@ _CSRC = os.path.join(ROOT, "sparse_attention_diffusion_basa_b200", "csrc")
 # the source files whose device code each profiled kernel is built from
 KERNEL_SOURCES = {
     "tc_attn_kernel": [os.path.join(_CSRC, "basa_tc.cu"), os.path.join(_CSRC, "tc_device.cuh")],
-    "tc_attn_pair_kernel": [os.path.join(_CSRC, "basa_tc2.cu"),
-                            os.path.join(_CSRC, "tc_device.cuh")],
     "pool_kernel": [os.path.join(_CSRC, "basa_pool.cu")],
     "tc_bwd_kernel": [os.path.join(_CSRC, "basa_tc_bwd.cu"), os.path.join(_CSRC, "tc_device.cuh")],
 }
@@ -91,17 +89,6 @@ def _traffic(kernel_key, workload):
         return float(e["dram_bytes_per_launch"])
     except Exception:
         return None
-
-
-def attention_kernel(w):
-    """The library's window-attention kernel for the workload: 256-token 2D
-    windows of whole 64-token row groups (bf16, d = 128, no pooled or text keys)
-    run on CTA pairs, the rest on the one-CTA kernel."""
-    wt, wh, ww = w.window
-    if (w.dtype == "bf16" and w.d == 128 and not w.P and not w.text and wt == 1
-            and wh * ww == 256 and 64 % ww == 0):
-        return "tc_attn_pair_kernel"
-    return "tc_attn_kernel"
 
 
 def workload_numbers(w, shift):
@@ -666,7 +653,7 @@ def main():
         roof = {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "frac": gbs / peaks["hbm_gbs"]}
     roof["peak_source"] = peaks["source"]
-    kname = attention_kernel(w)
+    kname = "tc_attn_kernel"
     roof["traffic"] = _traffic(kname, w.name)
     roof["kernel"] = kname
     roof["kernel_ms"] = ms_attn

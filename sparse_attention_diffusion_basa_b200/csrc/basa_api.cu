@@ -1,8 +1,6 @@
 // C ABI entry points: validation, shift normalisation, the bf16 window tile plan
 // (shifted-window index math), TMA map encoding and dispatch to the kernels.
 #include <math.h>
-#include <stdio.h>
-#include <stdlib.h>
 #include <string.h>
 
 #include <mutex>
@@ -100,16 +98,15 @@ int split(int l0, int n, int cut, Seg* out) {
 }
 }  // namespace
 
-basa_status build_tile_plan(const Dims& d, TilePlan* plan, int max_rows) {
+basa_status build_tile_plan(const Dims& d, TilePlan* plan) {
   memset(plan, 0, sizeof(*plan));
-  if (max_rows != 64 && max_rows != 128) return BASA_ERR_INVALID_ARG;
-  if (d.ww > max_rows || d.wh > 255 || d.wt > 255) return BASA_ERR_UNSUPPORTED;
-  const int R = max_rows / d.ww;  // window rows per tile, at most
+  if (d.ww > 128 || d.wh > 255 || d.wt > 255) return BASA_ERR_UNSUPPORTED;
+  const int R = 128 / d.ww;  // window rows per tile, at most
   struct LocalTile { int t0, h0, bt, bh; } tiles[kMaxTiles];
   int nt = 0;
   for (int h0 = 0; h0 < d.wh; h0 += R) {
     const int c = d.wh - h0 < R ? d.wh - h0 : R;
-    int g = max_rows / (d.ww * c);
+    int g = 128 / (d.ww * c);
     if (g < 1) g = 1;
     for (int t0 = 0; t0 < d.wt; t0 += g) {
       if (nt >= kMaxTiles) return BASA_ERR_UNSUPPORTED;
@@ -252,12 +249,6 @@ static basa_status attn_common(const Dims& d, const void* q, const void* k, cons
                                bool after_pool = false) {
   if (d.dtype == BASA_F32)
     return launch_simt(d, q, k, v, kp, vp, out, lse, stream);
-  if (kPairWindows && !flat) {  // 256-token windows: the CTA-pair kernel
-    TilePlan plan64;
-    if (pair_kernel_applies(d, kp != nullptr, &plan64))
-      return launch_tc_pair(d, plan64, q, k, v, out, lse, p->flags, p->wait_timeout_ms, stream,
-                            false);
-  }
   return launch_tc(d, flat, q, k, v, kp, vp, out, lse, p->flags, p->wait_timeout_ms, stream,
                    nullptr, after_pool);
 }
@@ -487,17 +478,7 @@ basa_status basa_full_attn(const void* q, const void* k, const void* v, void* ou
 }
 
 basa_status basa_get_status(cudaStream_t stream) {
-  // the status words of the one-CTA kernels and the backward, then the pair kernel's
-  const basa_status s = read_and_clear_status(stream);
-  unsigned int vp = 0, wherep = 0;
-  if (take_pair_status(stream, &vp, &wherep) != cudaSuccess) return BASA_ERR_CUDA;
-  if (vp) {
-    if (getenv("BASA_DEBUG"))
-      fprintf(stderr, "basa: CTA-pair kernel status %u at site %u\n", vp, wherep);
-    if (s == BASA_ERR_CHECK || (vp & 2u)) return BASA_ERR_CHECK;
-    return BASA_ERR_TIMEOUT;
-  }
-  return s;
+  return read_and_clear_status(stream);
 }
 
 basa_status basa_window_tiles(const basa_params* p, int32_t* n_windows, int32_t* n_tiles,

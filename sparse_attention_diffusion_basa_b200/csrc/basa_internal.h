@@ -86,11 +86,9 @@ struct TilePlan {
   uint32_t box[kClasses][kMaxTiles][kMaxBoxes];
 };
 
-// Builds the plan for window (wt, wh, ww) with shifts already reduced to [0, w):
-// tiles of whole window rows of at most max_rows (128, or 64 for the CTA-pair
-// kernel) tokens.  Returns BASA_ERR_UNSUPPORTED when the bounds of the bf16
-// kernel are exceeded.
-basa_status build_tile_plan(const Dims& d, TilePlan* plan, int max_rows = 128);
+// Builds the plan for window (wt, wh, ww) with shifts already reduced to [0, w).
+// Returns BASA_ERR_UNSUPPORTED when the bounds of the bf16 kernel are exceeded.
+basa_status build_tile_plan(const Dims& d, TilePlan* plan);
 
 // Window class (wrap bits) of window (jt, jh, jw).
 __host__ __device__ inline int window_class(int jt, int jh, int jw, int nwt, int nwh, int nww,
@@ -205,21 +203,6 @@ basa_status launch_tc_static_params(const Dims& d, bool flat, const void* q, con
                                     const void* v, const void* kp, const void* vp, void* out,
                                     float* lse, uint32_t flags, uint32_t timeout_ms,
                                     cudaStream_t stream, bool after_pool = false);
-
-// bf16 window attention over CTA pairs (basa_tc2.cu) for 256-token windows:
-// pair_kernel_applies checks the call and builds the 64-row tile plan it
-// needs; launch_tc_pair launches (static_params: the parameter block lives in
-// static storage, for the entry points that allocate nothing).  Building with
-// BASA_TC_PAIR=0 keeps those windows on the one-CTA kernel.
-#ifndef BASA_TC_PAIR
-#define BASA_TC_PAIR 0
-#endif
-constexpr bool kPairWindows = BASA_TC_PAIR != 0;
-bool pair_kernel_applies(const Dims& d, bool extra_keys, TilePlan* plan64);
-basa_status launch_tc_pair(const Dims& d, const TilePlan& plan64, const void* q, const void* k,
-                           const void* v, void* out, float* lse, uint32_t flags,
-                           uint32_t timeout_ms, cudaStream_t stream, bool static_params);
-cudaError_t take_pair_status(cudaStream_t stream, unsigned int* status, unsigned int* where);
 
 // Device status word helpers.  read_and_clear_status (basa_tc.cu) synchronises
 // the stream and reads and clears the status words of every kernel file;

@@ -132,12 +132,6 @@ extern "C" basa_status basa_window_attn_noalloc(const void* q, const void* k, co
     vp = vpw;
   }
   if (d.dtype == BASA_F32) return launch_simt(d, q, k, v, kp, vp, out, lse, stream);
-  if (kPairWindows) {  // 256-token windows without pooled tokens: the CTA-pair kernel
-    TilePlan plan64;
-    if (pair_kernel_applies(d, kp != nullptr, &plan64))
-      return launch_tc_pair(d, plan64, q, k, v, out, lse, p->flags, p->wait_timeout_ms, stream,
-                            true);
-  }
   return launch_tc_static_params(d, false, q, k, v, kp, vp, out, lse, p->flags,
                                  p->wait_timeout_ms, stream, d.P > 0);
 }
