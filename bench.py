@@ -91,6 +91,58 @@ def _traffic(kernel_key, workload):
         return None
 
 
+def sdpa_window_attn(q, k, v, window, shift):
+    """Context comparator (not the library): the backend-agnostic route the
+    BASA page describes, i.e. roll the grid by -shift, reshape it into windows,
+    run torch's scaled_dot_product_attention (its own kernel choice) on every
+    window, reshape back and roll by +shift.  q, k, v: [B, T, Hg, Wg, H, d]."""
+    import torch.nn.functional as F
+    B, T, Hg, Wg, H, d = q.shape
+    wt, wh, ww = window
+    nt, nh, nw = T // wt, Hg // wh, Wg // ww
+    dims = (1, 2, 3)
+
+    def to_windows(x):
+        x = torch.roll(x, tuple(-s for s in shift), dims)
+        x = x.view(B, nt, wt, nh, wh, nw, ww, H, d).permute(0, 1, 3, 5, 7, 2, 4, 6, 8)
+        return x.reshape(B * nt * nh * nw, H, wt * wh * ww, d)
+
+    o = F.scaled_dot_product_attention(to_windows(q), to_windows(k), to_windows(v))
+    o = o.view(B, nt, nh, nw, H, wt, wh, ww, d).permute(0, 1, 5, 2, 6, 3, 7, 4, 8)
+    return torch.roll(o.reshape(B, T, Hg, Wg, H, d), tuple(shift), dims)
+
+
+def sdpa_full_attn(q, k, v):
+    """Context comparator: torch's scaled_dot_product_attention over all tokens."""
+    import torch.nn.functional as F
+    B, T, Hg, Wg, H, d = q.shape
+    f = lambda x: x.reshape(B, T * Hg * Wg, H, d).transpose(1, 2)
+    return F.scaled_dot_product_attention(f(q), f(k), f(v)).transpose(1, 2)
+
+
+def sdpa_comparators(q, k, v, w, shift, steps, flush, world):
+    """Times the two SDPA routes under the first torch attention backend that
+    runs them (cuDNN, flash, memory-efficient, then the unfused math path)."""
+    from torch.nn.attention import SDPBackend, sdpa_kernel
+    for backend in (SDPBackend.CUDNN_ATTENTION, SDPBackend.FLASH_ATTENTION,
+                    SDPBackend.EFFICIENT_ATTENTION, SDPBackend.MATH):
+        try:
+            with sdpa_kernel(backend):
+                sdpa_window_attn(q, k, v, w.window, shift)
+                sdpa_full_attn(q, k, v)
+                torch.cuda.synchronize()
+                t_sw = time_steps(lambda: sdpa_window_attn(q, k, v, w.window, shift), steps, flush)
+                t_sf = time_steps(lambda: sdpa_full_attn(q, k, v), steps, flush)
+        except RuntimeError:
+            continue
+        return {"torch_sdpa_window_roll_reshape_ms": max_over_ranks(sum(t_sw) / len(t_sw), world),
+                "torch_sdpa_full_ms": max_over_ranks(sum(t_sf) / len(t_sf), world),
+                "backend": backend.name,
+                "note": "torch.nn.functional.scaled_dot_product_attention; context only, not "
+                        "part of the library"}
+    return None
+
+
 def workload_numbers(w, shift):
     """Algorithmic flops and bytes of one step, and the full-attention cost ratio.
 
@@ -467,6 +519,8 @@ def main():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--full-steps", type=int, default=5)
+    ap.add_argument("--no-comparators", action="store_true",
+                    help="skip the torch SDPA context timings")
     ap.add_argument("--no-blocks", action="store_true",
                     help="skip the per-block timings of a multi-block shift schedule")
     ap.add_argument("--backward", action="store_true",
@@ -634,6 +688,17 @@ def main():
     t_full = time_steps(step_full, args.full_steps, flush)
     ms_full = max_over_ranks(sum(t_full) / len(t_full), world)
 
+    # context: torch SDPA (opaque library kernels, not this library) on the same
+    # inputs, as full attention and as the roll + reshape + SDPA window route
+    comparators = None
+    if dq.dtype == torch.bfloat16 and not w.P and not L and not args.no_comparators:
+        comparators = sdpa_comparators(dq, dk, dv, w, shift, args.full_steps, flush, world)
+        if comparators:
+            ref = sdpa_window_attn(dq, dk, dv, w.window, shift)
+            basa.window_attn(dq, dk, dv, w.window, shift, w.pool, out=out)
+            comparators["max_abs_diff_vs_window_route"] = float((out.float() - ref.float()).abs().max())
+            del ref
+
     # end to end through the public API with host buffers (inputs larger than L2
     # arrive from the host every step)
     flush()
@@ -675,6 +740,7 @@ def main():
                     "ratio": (ms_full / ms_max) / theo,
                     "full_attn_tflops": 4.0 * w.B * w.H * (N + L) ** 2 * w.d / (ms_full * 1e-3) / 1e12},
         "roofline": roof,
+        **({"comparators": comparators} if comparators else {}),
         "e2e": {"value": world * flops / (e2e * 1e-3) / 1e12, "unit": "TFLOP/s",
                 "ms_per_step": e2e,
                 "h2d_bytes_per_step": sum(h.numel() * h.element_size() for h, _ in host_in),

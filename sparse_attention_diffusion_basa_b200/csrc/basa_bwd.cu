@@ -108,40 +108,65 @@ __device__ __forceinline__ float lane_sum(float x) {
 // D = rowsum(dO * O) for every (b, n, h).  HBM-bound: LPR = d * esize / 16
 // consecutive lanes read one row with 16-byte loads (a warp covers 32 / LPR
 // whole rows, so every load instruction reads contiguous bytes), multiply in
-// fp32 and add across their lanes.
+// fp32 and add across their lanes.  Each warp issues the loads of kPrepGroups
+// such row groups before it uses any, so that enough bytes are in flight, and
+// splits the row index in 32-bit arithmetic when the rows fit.
+constexpr int kPrepGroups = 4;
 template <bool BF16, int D>
 __global__ void __launch_bounds__(kBwdThreads) bwd_prep_kernel(BwdArgs a) {
   constexpr int LPR = D * (BF16 ? 2 : 4) / 16;  // lanes per row
-  constexpr int RPW = 32 / LPR;                 // rows per warp
+  constexpr int RPW = 32 / LPR;                 // rows per warp and group
+  constexpr int U = kPrepGroups;
   const long long rows = (long long)a.B * a.N * a.H;
   const long long warp = ((long long)blockIdx.x * kBwdThreads + threadIdx.x) / 32;
   const int lane = threadIdx.x % 32;
-  const long long r = warp * RPW + lane / LPR;
   const int sub = lane % LPR;
-  float acc = 0.f;
-  if (r < rows) {
-    const uint4 x = __ldcs(reinterpret_cast<const uint4*>(a.dout) + r * LPR + sub);
-    const uint4 y = __ldcs(reinterpret_cast<const uint4*>(a.o) + r * LPR + sub);
-    if (BF16) {
-      const __nv_bfloat162* hx = reinterpret_cast<const __nv_bfloat162*>(&x);
-      const __nv_bfloat162* hy = reinterpret_cast<const __nv_bfloat162*>(&y);
+  uint4 x[U], y[U];
+  long long r[U];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const float2 fx = __bfloat1622float2(hx[i]), fy = __bfloat1622float2(hy[i]);
-        acc = fmaf(fx.x, fy.x, acc);
-        acc = fmaf(fx.y, fy.y, acc);
-      }
-    } else {
-      acc = fmaf(__uint_as_float(x.x), __uint_as_float(y.x), acc);
-      acc = fmaf(__uint_as_float(x.y), __uint_as_float(y.y), acc);
-      acc = fmaf(__uint_as_float(x.z), __uint_as_float(y.z), acc);
-      acc = fmaf(__uint_as_float(x.w), __uint_as_float(y.w), acc);
+  for (int u = 0; u < U; ++u) {
+    r[u] = (warp * U + u) * RPW + lane / LPR;
+    if (r[u] < rows) {
+      x[u] = __ldcs(reinterpret_cast<const uint4*>(a.dout) + r[u] * LPR + sub);
+      y[u] = __ldcs(reinterpret_cast<const uint4*>(a.o) + r[u] * LPR + sub);
     }
   }
-  acc = lane_sum<LPR>(acc);
-  if (r < rows && sub == 0) {
-    const long long h = r % a.H, n = (r / a.H) % a.N, b = r / ((long long)a.H * a.N);
-    a.dD[(b * a.H + h) * a.N + n] = acc;
+  const bool small = rows <= 0xffffffffLL;
+#pragma unroll
+  for (int u = 0; u < U; ++u) {
+    float acc = 0.f;
+    if (r[u] < rows) {
+      if (BF16) {
+        const __nv_bfloat162* hx = reinterpret_cast<const __nv_bfloat162*>(&x[u]);
+        const __nv_bfloat162* hy = reinterpret_cast<const __nv_bfloat162*>(&y[u]);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const float2 fx = __bfloat1622float2(hx[i]), fy = __bfloat1622float2(hy[i]);
+          acc = fmaf(fx.x, fy.x, acc);
+          acc = fmaf(fx.y, fy.y, acc);
+        }
+      } else {
+        acc = fmaf(__uint_as_float(x[u].x), __uint_as_float(y[u].x), acc);
+        acc = fmaf(__uint_as_float(x[u].y), __uint_as_float(y[u].y), acc);
+        acc = fmaf(__uint_as_float(x[u].z), __uint_as_float(y[u].z), acc);
+        acc = fmaf(__uint_as_float(x[u].w), __uint_as_float(y[u].w), acc);
+      }
+    }
+    acc = lane_sum<LPR>(acc);
+    if (r[u] < rows && sub == 0) {
+      long long h, n, b;
+      if (small) {
+        const uint32_t rr = (uint32_t)r[u], t = rr / (uint32_t)a.H;
+        h = rr - t * (uint32_t)a.H;
+        n = t % (uint32_t)a.N;
+        b = t / (uint32_t)a.N;
+      } else {
+        h = r[u] % a.H;
+        n = (r[u] / a.H) % a.N;
+        b = r[u] / ((long long)a.H * a.N);
+      }
+      a.dD[(b * a.H + h) * a.N + n] = acc;
+    }
   }
 }
 
@@ -369,7 +394,8 @@ basa_status launch_bwd_typed(BwdArgs& a, const Dims& d, bool prep_only, cudaStre
   a.n_chunks = (a.m + per - 1) / per;
   const long long dq_blocks = (long long)d.B * d.H * nwin * a.n_chunks;
   const long long dkv_blocks = (long long)d.B * d.Hkv * nwin * a.n_chunks;
-  constexpr int rows_per_block = (kBwdThreads / 32) * (32 / (D * (BF16 ? 2 : 4) / 16));
+  constexpr int rows_per_block =
+      (kBwdThreads / 32) * (32 / (D * (BF16 ? 2 : 4) / 16)) * kPrepGroups;
   const long long prep_blocks = (rows + rows_per_block - 1) / rows_per_block;
   if (prep_blocks > 0x7fffffffLL || dq_blocks > 0x7fffffffLL) return BASA_ERR_UNSUPPORTED;
   bwd_prep_kernel<BF16, D><<<(unsigned)prep_blocks, kBwdThreads, 0, stream>>>(a);

@@ -894,8 +894,7 @@ basa_status launch_impl(TcParams* prm, cudaStream_t stream, bool dependent) {
   if (cudaFuncSetAttribute(tc_attn_kernel<D, kRing, kSplit, kF8>,
                            cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
     return BASA_ERR_CUDA;
-  long long grid = tc_sm_count();
-  if (grid > prm->n_units) grid = prm->n_units;
+  const long long grid = persistent_grid(prm->n_units);
   // dependent: launched as the programmatic dependent of the kernel before it
   // on the stream (the pooling), so that its start overlaps that kernel's tail
   cudaLaunchConfig_t cfg = {};

@@ -826,8 +826,7 @@ basa_status launch_bwd_kernel(BwdTcParams* prm, long long units, cudaStream_t st
                            smem) != cudaSuccess)
     return BASA_ERR_CUDA;
   prm->n_units = (uint32_t)units;
-  long long grid = tc_sm_count();
-  if (grid > units) grid = units;
+  const long long grid = persistent_grid(units);
   tc_bwd_kernel<D, MODE><<<(unsigned)grid, kBwdTcThreads, smem, stream>>>(*prm);
   return cudaGetLastError() == cudaSuccess ? BASA_OK : BASA_ERR_CUDA;
 }

@@ -534,6 +534,17 @@ inline int tc_sm_count() {
   return n > 0 ? n : 1;
 }
 
+// CTAs of a persistent grid over `units` work units: as few as keep the number
+// of units per CTA at its minimum, ceil(units / SMs), so that every CTA walks
+// the same number of units (384 units on 148 SMs: 128 CTAs of 3 units, not 88
+// CTAs of 3 and 60 of 2).
+inline long long persistent_grid(long long units) {
+  const long long sms = tc_sm_count();
+  if (units <= 0) return 1;
+  const long long rounds = (units + sms - 1) / sms;
+  return (units + rounds - 1) / rounds;
+}
+
 // Reads this translation unit's device status word after synchronising the
 // stream; returns the status bits and the first give-up site and clears both.
 inline cudaError_t tc_take_status(cudaStream_t stream, unsigned int* status, unsigned int* where) {
