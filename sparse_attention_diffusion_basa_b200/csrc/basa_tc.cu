@@ -26,11 +26,14 @@
 // keeps the running max and sum in fp32 (base-2 exponentials with the scale
 // folded in), writes the bf16 probabilities P back into TMEM over its logits,
 // and rescales its O row in TMEM when the max grows by more than 2^8.  The
-// epilogue divides by the sum and rounds to bf16; each warp then either stages
-// its 32 rows in shared memory and writes them back with 16-byte stores that
-// cover whole 128-byte row segments, or (windows of more than two key tiles)
-// the warpgroup stages the tile and stores it with TMA boxes that mirror the
-// load boxes.
+// epilogue divides by the sum and rounds to bf16.  Window passes stage the
+// tile in shared memory and store it with TMA boxes that mirror the load
+// boxes: with at most two key tiles per window (3-slot ring) both 64-column
+// halves of both query tiles have their own staging blocks, so the warps move
+// on to the next unit while the stores drain, and only the next unit's
+// epilogue waits for the staging to have been read.  Flat passes, padded grids
+// and windows with extra keys instead have each warp stage its 32 rows and
+// write them back with 16-byte stores that cover whole 128-byte row segments.
 //
 // A flat pass with few units (the text queries of a joint call) can split its
 // key tiles into ranges (template parameter kSplit): each split-unit writes its
@@ -78,6 +81,8 @@ struct __align__(64) TcParams {
   unsigned long long timeout_ns;
   int B, H, T, Hg, Wg;
   int group;  // query heads per K/V head
+  // unit decode divisors: H, n_pairs, n_windows, nww, nwh, group
+  FastDiv fd_h, fd_pairs, fd_windows, fd_nww, fd_nwh, fd_group;
   int wt, wh, ww, st, sh, sw, nwt, nwh, nww;
   int Tp, Hgp, Wgp;  // padded extents the window origins wrap on (T, Hg, Wg unless padded)
   int padded;        // 1: padded positions exist and are masked
@@ -174,21 +179,24 @@ __device__ __forceinline__ Unit decode_unit(const TcParams& p, uint32_t u) {
     U.nk = left < p.kt_per_split ? left : p.kt_per_split;
   }
   if (p.flat) {
-    U.pair = (int)(u % (uint32_t)p.n_pairs);
-    const uint32_t r = u / (uint32_t)p.n_pairs;
-    U.h = (int)(r % (uint32_t)p.H);
-    U.b = (int)(r / (uint32_t)p.H);
+    const uint32_t r = p.fd_pairs.div(u);
+    U.pair = (int)(u - r * (uint32_t)p.n_pairs);
+    U.b = (int)p.fd_h.div(r);
+    U.h = (int)(r - (uint32_t)U.b * (uint32_t)p.H);
     U.cls = 0;
     U.ot = U.oh = U.ow = 0;
     U.holes = 0;
   } else {
-    U.h = (int)(u % (uint32_t)p.H);
-    uint32_t r = u / (uint32_t)p.H;
-    U.pair = (int)(r % (uint32_t)p.n_pairs);
-    r /= (uint32_t)p.n_pairs;
-    const int win = (int)(r % (uint32_t)p.n_windows);
-    U.b = (int)(r / (uint32_t)p.n_windows);
-    const int jw = win % p.nww, jh = (win / p.nww) % p.nwh, jt = win / (p.nww * p.nwh);
+    uint32_t r = p.fd_h.div(u);
+    U.h = (int)(u - r * (uint32_t)p.H);
+    uint32_t r2 = p.fd_pairs.div(r);
+    U.pair = (int)(r - r2 * (uint32_t)p.n_pairs);
+    U.b = (int)p.fd_windows.div(r2);
+    const int win = (int)(r2 - (uint32_t)U.b * (uint32_t)p.n_windows);
+    const uint32_t wr = p.fd_nww.div((uint32_t)win);
+    const int jw = win - (int)wr * p.nww;
+    const int jt = (int)p.fd_nwh.div(wr);
+    const int jh = (int)wr - jt * p.nwh;
     U.cls = window_class(jt, jh, jw, p.nwt, p.nwh, p.nww, p.st, p.sh, p.sw);
     U.ot = jt * p.wt + p.st;
     U.oh = jh * p.wh + p.sh;
@@ -201,7 +209,7 @@ __device__ __forceinline__ Unit decode_unit(const TcParams& p, uint32_t u) {
   }
   const int left = p.n_qt - 2 * U.pair;
   U.nq = left < 2 ? left : 2;
-  U.hk = p.group == 1 ? U.h : U.h / p.group;
+  U.hk = (int)p.fd_group.div((uint32_t)U.h);
   return U;
 }
 
@@ -301,8 +309,9 @@ __device__ __forceinline__ uint4 key_token_mask(const TcParams& p, const PlanVie
   return make_uint4(w[0], w[1], w[2], w[3]);
 }
 
-// Shared-memory plan: the unit's two 128-row query tiles, one 64-column output
-// staging block per query tile, and a ring of K/V tiles.  The probabilities P
+// Shared-memory plan: the unit's two 128-row query tiles, output staging (one
+// 64-column block per query tile, or both halves of both query tiles with the
+// 3-slot ring), and a ring of K/V tiles.  The probabilities P
 // never touch shared memory: they are written into TMEM over their logits and
 // read from there by the P.V MMA.
 template <int D, int kRing, bool kF8 = false>
@@ -311,9 +320,12 @@ struct Smem {
   static constexpr int kTile = kF8 ? (D / 128) * kHalf : (D / 64) * kHalf;
   static constexpr int kVbf = (D / 64) * kHalf;   // one V tile widened to bf16 (e4m3 only)
   static constexpr int NS = kRing;                // K/V ring slots
+  // 3-slot ring (windows of at most two key tiles): room to stage both output
+  // halves of both query tiles, so the TMA stores of a unit need no wait
+  static constexpr bool kFullStg = kRing == 3 && !kF8 && D == 128;
   static constexpr int q0 = 0;
   static constexpr int stg0 = 2 * kTile;
-  static constexpr int ring0 = stg0 + 2 * kHalf;
+  static constexpr int ring0 = stg0 + (kFullStg ? 4 : 2) * kHalf;
   static constexpr int vbf0 = ring0 + NS * kTile;
   static constexpr int bars = vbf0 + (kF8 ? 2 * kVbf : 0);
   // barrier indices (VBFULL, VBEMPTY: the two widened V buffers, e4m3 only)
@@ -555,8 +567,11 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attn_kernel(const __grid_const
         mma_bf16_ts(tmem + 256 + i * 128, tmem + i * 128 + k * 8,
                     sdesc(va + k * 2048, kHalf, 1024), IDO, (accumulate || k > 0) ? 1u : 0u);
     };
+    // A unit's coordinates take a chain of integer divisions to decode: the
+    // next unit's are decoded while this unit's exponentials run.
+    Unit Un = decode_unit<kSplit>(p, blockIdx.x);
     for (uint32_t u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
-      const Unit U = decode_unit<kSplit>(p, u);
+      const Unit U = Un;
       uint32_t kslot;
       if (!(ok = take_slot(kslot))) break;
       for (int i = 0; i < U.nq && ok; ++i) {
@@ -573,6 +588,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attn_kernel(const __grid_const
       }
       if (!ok) break;
       release(kslot);
+      if (u + gridDim.x < p.n_units) Un = decode_unit<kSplit>(p, u + gridDim.x);
       for (int j = 0; j < kcount(U) && ok; ++j) {
         const bool next = j + 1 < kcount(U);
         uint32_t vaddr, vref;
@@ -657,9 +673,15 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attn_kernel(const __grid_const
     bool stg_busy = false;  // a TMA store may still be reading the staging block
     const float c = p.scale_log2;
     bool ok = true;
+    // next unit decoded while this unit's last P.V MMA runs
+    Unit Un = decode_unit<kSplit>(p, blockIdx.x);
     for (uint32_t u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
-      const Unit U = decode_unit<kSplit>(p, u);
-      if (i >= U.nq) continue;
+      const Unit U = Un;
+      const bool more = u + gridDim.x < p.n_units;
+      if (i >= U.nq) {
+        if (more) Un = decode_unit<kSplit>(p, u + gridDim.x);
+        continue;
+      }
       const int qt = 2 * U.pair + i;
       float m = -INFINITY, l = 0.f;
       for (int j = kbeg(U); j < kbeg(U) + kcount(U); ++j) {
@@ -754,7 +776,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attn_kernel(const __grid_const
         mbar_arrive(BAR(S::PFULL + i));
       }
       if (!ok) break;
-      // epilogue: O / l -> bf16 -> staging, one 64-column half at a time -> TMA store
+      if (more) Un = decode_unit<kSplit>(p, u + gridDim.x);
+      // epilogue: O / l -> bf16 -> staging -> stores
       if (!(ok = wait_warp(BAR(S::OFULL + i), ofull & 1u, abort_flag, limit, kSiteSmxPvLast)))
         break;
       ++ofull;
@@ -828,8 +851,53 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attn_kernel(const __grid_const
           __syncwarp();
         }
       }
+      if constexpr (S::kFullStg) {
+        if (!p.warp_stores) {
+          const uint32_t stg2 = sbase + S::stg0 + (uint32_t)i * 2u * kHalf;
+          if (stg_busy) {  // the previous unit's stores have read the staging blocks
+            if (leader) {
+              bulk_wait_read0();
+              mbar_arrive(BAR(S::STGFREE + i));
+            }
+            if (!(ok = wait_warp(BAR(S::STGFREE + i), stgfree & 1u, abort_flag, limit,
+                                 kSiteSmxOFree)))
+              break;
+            ++stgfree;
+          }
 #pragma unroll
-      for (int hf = 0; hf < (p.warp_stores ? 0 : D / 64); ++hf) {
+          for (int hf = 0; hf < 2; ++hf) {
+            uint32_t o[2][32];
+            tmem_ld32(tO + hf * 64, o[0]);
+            tmem_ld32(tO + hf * 64 + 32, o[1]);
+            tmem_wait_ld(o[0]);
+            tmem_wait_ld(o[1]);
+            uint32_t w[32];
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+              float o0, o1;
+              f2unpack(f2mul(f2pack(__uint_as_float(o[e / 16][(2 * e) % 32]),
+                                    __uint_as_float(o[e / 16][(2 * e) % 32 + 1])), inv2), o0, o1);
+              w[e] = pack_bf16(o0, o1);
+            }
+#pragma unroll
+            for (int ch = 0; ch < 8; ++ch)
+              st_shared_v4(stg2 + hf * kHalf + swz(r, ch), w[4 * ch], w[4 * ch + 1],
+                           w[4 * ch + 2], w[4 * ch + 3]);
+          }
+          fence_proxy_async();
+          mbar_arrive(BAR(S::STAGED + i));
+          if (leader &&
+              wait_bounded(BAR(S::STAGED + i), staged & 1u, abort_flag, limit, kSiteSmxOStaged)) {
+            store_half<D>(p, pv, U, qt, 0, stg2);
+            store_half<D>(p, pv, U, qt, 1, stg2 + kHalf);
+            bulk_commit();
+          }
+          ++staged;
+          stg_busy = true;
+        }
+      }
+#pragma unroll
+      for (int hf = 0; hf < ((p.warp_stores || S::kFullStg) ? 0 : D / 64); ++hf) {
         uint32_t o[2][32];
         tmem_ld32(tO + hf * 64, o[0]);
         tmem_ld32(tO + hf * 64 + 32, o[1]);
@@ -894,7 +962,9 @@ basa_status launch_impl(TcParams* prm, cudaStream_t stream, bool dependent) {
   if (cudaFuncSetAttribute(tc_attn_kernel<D, kRing, kSplit, kF8>,
                            cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
     return BASA_ERR_CUDA;
-  const long long grid = persistent_grid(prm->n_units);
+  // balanced rounds for a few units per SM (flux1024: 44.1 against 45.8 us);
+  // one CTA per SM for many (flux2048, 11 units per SM: 116.4 against 118.0 us)
+  const long long grid = persistent_grid(prm->n_units, 4);
   // dependent: launched as the programmatic dependent of the kernel before it
   // on the stream (the pooling), so that its start overlaps that kernel's tail
   cudaLaunchConfig_t cfg = {};
@@ -1037,10 +1107,23 @@ basa_status build_and_launch(TcParams* prm, const Dims& d, bool flat, const void
     if (units > 0x7fffffffLL) { st = BASA_ERR_UNSUPPORTED; goto done; }
     prm->n_units = (uint32_t)units;
   }
-  // Output path: warp-staged stores, except for windows of more than two key
-  // tiles, where the TMA store boxes measured faster.
-  // A padded grid always takes the warp-staged stores (they skip padded rows).
-  prm->warp_stores = (flat || prm->n_wkt <= 2 || prm->padded) ? 1 : 0;
+  prm->fd_h = FastDiv(prm->H);
+  prm->fd_pairs = FastDiv(prm->n_pairs);
+  prm->fd_windows = FastDiv(prm->n_windows);
+  prm->fd_nww = FastDiv(prm->nww);
+  prm->fd_nwh = FastDiv(prm->nwh);
+  prm->fd_group = FastDiv(prm->group);
+  // Output path: TMA store boxes for windows (both halves staged at once when
+  // the window has at most two key tiles and no extra keys: flux2048 117.6 ->
+  // 104.8 us, flux1024 44.2 -> 38.3 us against warp-staged stores); warp-staged
+  // stores for flat passes and for windows of at most two key tiles with extra
+  // keys.  A padded grid always takes the warp-staged stores (they skip padded
+  // rows).
+  {
+    const bool ring3 = !f8 && prm->n_splits <= 1 && d.d == 128 && !flat &&
+                       prm->n_wkt + prm->n_pkt <= 2;
+    prm->warp_stores = (flat || prm->padded) ? 1 : ring3 ? 0 : (prm->n_wkt <= 2 ? 1 : 0);
+  }
   // K/V ring depth: windows of at most two key tiles and no extra keys stream
   // each K/V tile once per unit and ran faster with 3 slots in flight than with
   // 4; everything else reuses K/V tiles from L2 and runs faster with 4.

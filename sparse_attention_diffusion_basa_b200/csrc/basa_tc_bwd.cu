@@ -86,6 +86,9 @@ struct __align__(64) BwdTcParams {
   int H, Hkv, group, T, Hg, Wg;
   int wt, wh, ww, st, sh, sw, nwt, nwh, nww;
   int n_windows, n_tiles, n_shapes;
+  // unit decode divisors (set by the launcher): H, Hkv, n_tiles, n_windows,
+  // nww, nwh, group, n_tt, n_pt, n_fsplits
+  FastDiv fd_h, fd_hkv, fd_tiles, fd_windows, fd_nww, fd_nwh, fd_group, fd_tt, fd_pt, fd_fsplits;
   float scale, scale_log2;
   // pooled global memory (P = 0: none)
   float* dkp;  // [B, P, Hkv, d] fp32: sum over the batch's queries of dS^T Q (no scale)
@@ -158,23 +161,23 @@ __device__ __forceinline__ BwdUnit decode_bwd_unit(const BwdTcParams& p, uint32_
   constexpr bool KV = MODE == kModeDkv || MODE == kModePooled;
   BwdUnit U;
   if constexpr (MODE == kModeDqText) {  // (b, h, text tile): heads fastest
-    U.h = (int)(u % (uint32_t)p.H);
-    U.hk = U.h / p.group;
-    const uint32_t r = u / (uint32_t)p.H;
-    U.tile = (int)(r % (uint32_t)p.n_tt);
-    U.w.b = (int)(r / (uint32_t)p.n_tt);
+    const uint32_t r = p.fd_h.div(u);
+    U.h = (int)(u - r * (uint32_t)p.H);
+    U.hk = (int)p.fd_group.div((uint32_t)U.h);
+    U.w.b = (int)p.fd_tt.div(r);
+    U.tile = (int)(r - (uint32_t)U.w.b * (uint32_t)p.n_tt);
     U.w.cls = U.w.ot = U.w.oh = U.w.ow = 0;
     U.q0 = U.nq = 0;
     return U;
   }
   if constexpr (MODE == kModePooled) {
-    U.hk = (int)(u % (uint32_t)p.Hkv);
+    const uint32_t r = p.fd_hkv.div(u);
+    U.hk = (int)(u - r * (uint32_t)p.Hkv);
     U.h = U.hk * p.group;
-    uint32_t r = u / (uint32_t)p.Hkv;
-    U.tile = (int)(r % (uint32_t)p.n_pt);
-    r /= (uint32_t)p.n_pt;
-    const int sp = (int)(r % (uint32_t)p.n_fsplits);
-    U.w.b = (int)(r / (uint32_t)p.n_fsplits);
+    const uint32_t r2 = p.fd_pt.div(r);
+    U.tile = (int)(r - r2 * (uint32_t)p.n_pt);
+    U.w.b = (int)p.fd_fsplits.div(r2);
+    const int sp = (int)(r2 - (uint32_t)U.w.b * (uint32_t)p.n_fsplits);
     U.w.cls = U.w.ot = U.w.oh = U.w.ow = 0;
     U.q0 = sp * p.fqt_per_split;
     const int left = p.n_fqt + (p.joint ? p.n_tt : 0) - U.q0;  // joint: image, then text tiles
@@ -183,13 +186,16 @@ __device__ __forceinline__ BwdUnit decode_bwd_unit(const BwdTcParams& p, uint32_
   }
   U.q0 = U.nq = 0;
   const uint32_t nh = (uint32_t)(KV ? p.Hkv : p.H);
-  const int head = (int)(u % nh);
-  uint32_t r = u / nh;
-  U.tile = (int)(r % (uint32_t)p.n_tiles);
-  r /= (uint32_t)p.n_tiles;
-  const int win = (int)(r % (uint32_t)p.n_windows);
-  const int b = (int)(r / (uint32_t)p.n_windows);
-  const int jw = win % p.nww, jh = (win / p.nww) % p.nwh, jt = win / (p.nww * p.nwh);
+  const uint32_t r = (KV ? p.fd_hkv : p.fd_h).div(u);
+  const int head = (int)(u - r * nh);
+  const uint32_t r2 = p.fd_tiles.div(r);
+  U.tile = (int)(r - r2 * (uint32_t)p.n_tiles);
+  const int b = (int)p.fd_windows.div(r2);
+  const int win = (int)(r2 - (uint32_t)b * (uint32_t)p.n_windows);
+  const uint32_t wr = p.fd_nww.div((uint32_t)win);
+  const int jw = win - (int)wr * p.nww;
+  const int jt = (int)p.fd_nwh.div(wr);
+  const int jh = (int)wr - jt * p.nwh;
   U.w.cls = window_class(jt, jh, jw, p.nwt, p.nwh, p.nww, p.st, p.sh, p.sw);
   U.w.ot = jt * p.wt + p.st;
   U.w.oh = jh * p.wh + p.sh;
@@ -200,7 +206,7 @@ __device__ __forceinline__ BwdUnit decode_bwd_unit(const BwdTcParams& p, uint32_
     U.h = head * p.group;
   } else {
     U.h = head;
-    U.hk = head / p.group;
+    U.hk = (int)p.fd_group.div((uint32_t)head);
   }
   return U;
 }
@@ -826,6 +832,16 @@ basa_status launch_bwd_kernel(BwdTcParams* prm, long long units, cudaStream_t st
                            smem) != cudaSuccess)
     return BASA_ERR_CUDA;
   prm->n_units = (uint32_t)units;
+  prm->fd_h = FastDiv(prm->H);
+  prm->fd_hkv = FastDiv(prm->Hkv);
+  prm->fd_tiles = FastDiv(prm->n_tiles);
+  prm->fd_windows = FastDiv(prm->n_windows);
+  prm->fd_nww = FastDiv(prm->nww);
+  prm->fd_nwh = FastDiv(prm->nwh);
+  prm->fd_group = FastDiv(prm->group);
+  prm->fd_tt = FastDiv(prm->n_tt);
+  prm->fd_pt = FastDiv(prm->n_pt);
+  prm->fd_fsplits = FastDiv(prm->n_fsplits);
   const long long grid = persistent_grid(units);
   tc_bwd_kernel<D, MODE><<<(unsigned)grid, kBwdTcThreads, smem, stream>>>(*prm);
   return cudaGetLastError() == cudaSuccess ? BASA_OK : BASA_ERR_CUDA;

@@ -23,6 +23,25 @@ __device__ unsigned int g_basa_where;   // site of the first wait that gave up
 
 constexpr int kHalf = 128 * 128;  // bytes of one 64-wide head-dim half of a 128-row tile
 
+// Division by a launch constant d >= 1 without the integer-divide sequence
+// (Granlund and Montgomery, "Division by Invariant Integers using
+// Multiplication", PLDI 1994): with l = ceil(log2 d) and the 33-bit multiplier
+// 2^32 + m = ceil(2^(32 + l) / d), n / d = (umulhi(n, m) + n) >> l for every
+// 32-bit n.  d < 1 is taken as 1.
+struct FastDiv {
+  uint32_t d, m, l;
+  FastDiv() = default;
+  explicit FastDiv(int dv) {
+    d = dv > 1 ? (uint32_t)dv : 1u;
+    l = 0;
+    while ((1ull << l) < d) ++l;
+    m = (uint32_t)(((1ull << 32) * ((1ull << l) - d)) / d + 1);
+  }
+  __device__ __forceinline__ uint32_t div(uint32_t n) const {
+    return (uint32_t)(((uint64_t)__umulhi(n, m) + n) >> l);
+  }
+};
+
 // Checked build (compiled with BASA_CHECKED): the kernels verify every TMA box
 // and every output index against their tensors before the access; a failed
 // check skips the access, sets bit 1 of the device status word and records its
@@ -534,14 +553,17 @@ inline int tc_sm_count() {
   return n > 0 ? n : 1;
 }
 
-// CTAs of a persistent grid over `units` work units: as few as keep the number
-// of units per CTA at its minimum, ceil(units / SMs), so that every CTA walks
-// the same number of units (384 units on 148 SMs: 128 CTAs of 3 units, not 88
-// CTAs of 3 and 60 of 2).
-inline long long persistent_grid(long long units) {
+// CTAs of a persistent grid over `units` work units.  Up to `max_rounds`
+// units per CTA: as few CTAs as keep the number of units per CTA at its
+// minimum, ceil(units / SMs), so that every CTA walks the same number of units
+// (384 units on 148 SMs: 128 CTAs of 3 units, not 88 CTAs of 3 and 60 of 2).
+// Beyond that, one CTA per SM: with many units per CTA the uneven last round
+// costs less than the bandwidth of the SMs a balanced grid leaves idle.
+inline long long persistent_grid(long long units, long long max_rounds = 1LL << 40) {
   const long long sms = tc_sm_count();
   if (units <= 0) return 1;
   const long long rounds = (units + sms - 1) / sms;
+  if (rounds > max_rounds) return units < sms ? units : sms;
   return (units + rounds - 1) / rounds;
 }
 
