@@ -31,9 +31,10 @@
 // boxes: with at most two key tiles per window (3-slot ring) both 64-column
 // halves of both query tiles have their own staging blocks, so the warps move
 // on to the next unit while the stores drain, and only the next unit's
-// epilogue waits for the staging to have been read.  Flat passes, padded grids
-// and windows with extra keys instead have each warp stage its 32 rows and
-// write them back with 16-byte stores that cover whole 128-byte row segments.
+// epilogue waits for the staging to have been read; otherwise one half at a
+// time.  Flat passes and padded grids instead have each warp stage its 32 rows
+// and write them back with 16-byte stores that cover whole 128-byte row
+// segments.
 //
 // A flat pass with few units (the text queries of a joint call) can split its
 // key tiles into ranges (template parameter kSplit): each split-unit writes its
@@ -1114,16 +1115,11 @@ basa_status build_and_launch(TcParams* prm, const Dims& d, bool flat, const void
   prm->fd_nwh = FastDiv(prm->nwh);
   prm->fd_group = FastDiv(prm->group);
   // Output path: TMA store boxes for windows (both halves staged at once when
-  // the window has at most two key tiles and no extra keys: flux2048 117.6 ->
-  // 104.8 us, flux1024 44.2 -> 38.3 us against warp-staged stores); warp-staged
-  // stores for flat passes and for windows of at most two key tiles with extra
-  // keys.  A padded grid always takes the warp-staged stores (they skip padded
-  // rows).
-  {
-    const bool ring3 = !f8 && prm->n_splits <= 1 && d.d == 128 && !flat &&
-                       prm->n_wkt + prm->n_pkt <= 2;
-    prm->warp_stores = (flat || prm->padded) ? 1 : ring3 ? 0 : (prm->n_wkt <= 2 ? 1 : 0);
-  }
+  // the window has at most two key tiles and no extra keys), against the
+  // warp-staged stores: flux2048 117.6 -> 104.8 us, flux1024 44.2 -> 38.3 us,
+  // flux2048_gm4 attention 546 -> 521 us.  Warp-staged stores for flat passes;
+  // a padded grid always takes them too (they skip padded rows).
+  prm->warp_stores = (flat || prm->padded) ? 1 : 0;
   // K/V ring depth: windows of at most two key tiles and no extra keys stream
   // each K/V tile once per unit and ran faster with 3 slots in flight than with
   // 4; everything else reuses K/V tiles from L2 and runs faster with 4.
