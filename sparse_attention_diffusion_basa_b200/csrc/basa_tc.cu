@@ -568,8 +568,9 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attn_kernel(const __grid_const
         mma_bf16_ts(tmem + 256 + i * 128, tmem + i * 128 + k * 8,
                     sdesc(va + k * 2048, kHalf, 1024), IDO, (accumulate || k > 0) ? 1u : 0u);
     };
-    // A unit's coordinates take a chain of integer divisions to decode: the
-    // next unit's are decoded while this unit's exponentials run.
+    // A unit's coordinates take a chain of dependent divisions (by reciprocal
+    // multipliers) to decode: the next unit's are decoded while this unit's
+    // exponentials run.
     Unit Un = decode_unit<kSplit>(p, blockIdx.x);
     for (uint32_t u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
       const Unit U = Un;
